@@ -1,0 +1,129 @@
+"""fp64 CPU oracle of the delta-rule recurrent-memory scan (forward).
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the CPU-baseline
+leg of ``bench.py`` may import this package; the product path (the CUDA library and
+its Python binding) never does, and shares no code with it.
+
+The arithmetic lives in ``dr_oracle.c`` (plain C, fp64, one token at a time, OpenMP
+over independent (batch, head) sequences). This module compiles it with gcc on first
+use and marshals numpy arrays through ctypes. See the C file's header for the
+sources on the pages and for the readings taken where the pages are silent.
+
+Parity status: every function here is pinned by ``tests/test_oracle_pins.py``
+against closed forms, brute-force definitions and invariants the pages fix.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "dr_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+LINEAR, DELTANET, GDN, KDA = 0, 1, 2, 3
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile dr_oracle.c into liboracle.so (gcc -O2 -fopenmp); return the path."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-o", tmp, _SRC, "-lm"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        dp = ctypes.POINTER(ctypes.c_double)
+        lib.oracle_dr_scan.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp] + [ctypes.c_int] * 7
+        lib.oracle_dr_scan.restype = ctypes.c_int
+        lib.oracle_vla_scan.argtypes = [dp] * 6 + [ctypes.c_double] + [dp] * 3 + [ctypes.c_int] * 4
+        lib.oracle_vla_scan.restype = ctypes.c_int
+        lib.oracle_num_threads.argtypes = []
+        lib.oracle_num_threads.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def num_threads() -> int:
+    """OpenMP threads the oracle uses (all host cores unless OMP_NUM_THREADS says otherwise)."""
+    return int(_load().oracle_num_threads())
+
+
+def _f64(x):
+    if x is None:
+        return None
+    return np.ascontiguousarray(x, dtype=np.float64)
+
+
+def _ptr(x):
+    if x is None:
+        return None
+    return x.ctypes.data_as(ctypes.POINTER(ctypes.c_double))
+
+
+def dr_scan(q, k, v, beta=None, gate=None, S0=None, mode=DELTANET, residual_pre_decay=False,
+            want_state=True):
+    """Per-token delta-rule scan in fp64.
+
+    q, k: [B,H,T,dk]; v: [B,H,T,dv]; beta: [B,H,T] (ignored for LINEAR);
+    gate: None (LINEAR, DELTANET), [B,H,T] (GDN) or [B,H,T,dk] (KDA), alpha values;
+    S0: [B,H,dv,dk] or None (zeros). Returns (out [B,H,T,dv], S_final [B,H,dv,dk] or None).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or v.shape[:3] != (B, H, T):
+        raise ValueError("shape mismatch")
+    beta = _f64(beta) if mode != LINEAR else None
+    gate = _f64(gate) if mode in (GDN, KDA) else None
+    if beta is not None and beta.shape != (B, H, T):
+        raise ValueError("beta shape")
+    if gate is not None:
+        want = (B, H, T) if mode == GDN else (B, H, T, dk)
+        if gate.shape != want:
+            raise ValueError("gate shape")
+    S0 = _f64(S0)
+    if S0 is not None and S0.shape != (B, H, dv, dk):
+        raise ValueError("S0 shape")
+    out = np.empty((B, H, T, dv), np.float64)
+    Sf = np.empty((B, H, dv, dk), np.float64) if want_state else None
+    rc = _load().oracle_dr_scan(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(gate), _ptr(S0),
+                                _ptr(out), _ptr(Sf), B, H, T, dk, dv, int(mode),
+                                int(bool(residual_pre_decay)))
+    if rc != 0:
+        raise RuntimeError(f"oracle_dr_scan failed ({rc})")
+    return out, Sf
+
+
+def vla_scan(q, k, v, u, S0=None, A0=None, lambda0=1.0, want_state=True):
+    """Per-token VLA Sherman-Morrison scan in fp64.
+
+    q, k, v, u: [B,H,T,d]; S0, A0: [B,H,d,d] or None (zeros, I/lambda0).
+    Returns (out [B,H,T,d], S_final, A_final) (the last two None unless want_state).
+    """
+    q, k, v, u = _f64(q), _f64(k), _f64(v), _f64(u)
+    B, H, T, d = q.shape
+    for x in (k, v, u):
+        if x.shape != q.shape:
+            raise ValueError("shape mismatch")
+    S0, A0 = _f64(S0), _f64(A0)
+    for x in (S0, A0):
+        if x is not None and x.shape != (B, H, d, d):
+            raise ValueError("state shape")
+    out = np.empty((B, H, T, d), np.float64)
+    Sf = np.empty((B, H, d, d), np.float64) if want_state else None
+    Af = np.empty((B, H, d, d), np.float64) if want_state else None
+    rc = _load().oracle_vla_scan(_ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(S0), _ptr(A0),
+                                 float(lambda0), _ptr(out), _ptr(Sf), _ptr(Af), B, H, T, d)
+    if rc != 0:
+        raise RuntimeError(f"oracle_vla_scan failed ({rc})")
+    return out, Sf, Af

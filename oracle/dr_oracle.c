@@ -1,0 +1,252 @@
+/*
+ * Plain fp64 CPU oracle of the delta-rule recurrent-memory scan (forward).
+ *
+ * TEST INFRASTRUCTURE ONLY. Nothing on the product path may call, link or load
+ * this file: only the tests, the package's smoke check and the benchmark's
+ * CPU-baseline leg use it. It shares no code, header, table or helper with the
+ * CUDA library; the two meet only through seeded inputs.
+ *
+ * What it computes is the per-token definition, written out one token at a time,
+ * in fp64, independently for every (batch, head) sequence. There is no chunking,
+ * blocking, fusion or reordering.
+ *
+ * Sources (the three web pages this subject is drawn from):
+ *  - "Mechanisms, trade-offs and cross-layer routing of linear-attention
+ *    architectures" (aitrends.kr), section "Technical details" (기술 상세) and
+ *    "Understanding the key idea": memory W in R^{d_v x d_phi}, readout y = W phi(q);
+ *    DeltaNet prediction vbar = W_{t-1} kappa, residual r = v - vbar, write
+ *    W <- W + beta r (x) kappa; Gated DeltaNet W <- alpha W + beta r_alpha (x) kappa
+ *    (scalar decay); Kimi Delta Attention decays per key-feature channel.
+ *  - "Variational Linear Attention (VLA)" (gist.science 2605.11196), section 2.1
+ *    (plain accumulation S_t = S_{t-1} + v_t k_t^T), section 2.2 (inverse penalty
+ *    A_t = M_t^{-1} kept by a Sherman-Morrison rank-1 update) and section 2.3
+ *    (steps 1-3: A-update, alpha_hat = A_t k_hat / ||A_t k_hat||,
+ *    S_t = S_{t-1} + (v_t - S_{t-1} k_hat_t) alpha_hat_t^T).
+ *
+ * Readings where the pages are silent or garbled (each is listed in the design notes):
+ *  - Gated variants take the residual against the DECAYED state:
+ *    S' = alpha (.) S_{t-1};  r = v - S' k;  S_t = S' + beta r k^T.
+ *    This is the only reading under which "unit k, beta = 1 => S_t k_t = v_t"
+ *    holds for alpha != 1. The literal reading r = v - S_{t-1} k is kept behind
+ *    the flag `residual_pre_decay` (oracle-only option).
+ *  - KDA's alpha_t in (0,1)^{d_k} scales the COLUMNS of S (key-feature axis).
+ *  - Readout after the write: o_t = S_t q_t. No feature map and no 1/sqrt(d_k)
+ *    scale inside the scan; q and k arrive as the caller prepared them.
+ *  - Plain linear attention ignores beta and gate.
+ *  - VLA: z_t = A_{t-1} u_t (Sherman-Morrison for M_t = M_{t-1} + u_t u_t^T),
+ *    A_0 = I / lambda0, readout o_t = S_t q_hat_t, no beta and no decay.
+ *
+ * Layouts (all row-major, contiguous):
+ *   q, k   [B, H, T, dk]      v, out [B, H, T, dv]      beta [B, H, T]
+ *   gate   GDN: [B, H, T]     KDA: [B, H, T, dk]        (alpha values, not logs)
+ *   S0, S_final [B, H, dv, dk]   (S maps keys to values: S k in R^{dv})
+ *   VLA: q, k, v, u, out [B, H, T, d];  S0, S_final, A0, A_final [B, H, d, d]
+ */
+#include <stdlib.h>
+#include <string.h>
+#include <math.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_LINEAR 0
+#define ORACLE_DELTANET 1
+#define ORACLE_GDN 2
+#define ORACLE_KDA 3
+
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}
+
+/* One (batch, head) sequence of the delta-rule family. S is dv x dk, updated in place. */
+static void dr_sequence(const double* q, const double* k, const double* v,
+                        const double* beta, const double* gate, double* S,
+                        double* out, double* decay, double* pred,
+                        long T, int dk, int dv, int mode, int residual_pre_decay) {
+    for (long t = 0; t < T; ++t) {
+        const double* kt = k + t * dk;
+        const double* qt = q + t * dk;
+        const double* vt = v + t * dv;
+        double* ot = out + t * dv;
+
+        if (mode == ORACLE_LINEAR) {
+            /* S_t = S_{t-1} + v_t k_t^T  (VLA page, section 2.1) */
+            for (int i = 0; i < dv; ++i)
+                for (int j = 0; j < dk; ++j)
+                    S[(long)i * dk + j] += vt[i] * kt[j];
+        } else {
+            /* decay factor per key channel j: 1 (DeltaNet), alpha_t (GDN), alpha_t[j] (KDA) */
+            for (int j = 0; j < dk; ++j) {
+                if (mode == ORACLE_DELTANET) decay[j] = 1.0;
+                else if (mode == ORACLE_GDN) decay[j] = gate[t];
+                else decay[j] = gate[t * dk + j];
+            }
+            /* prediction vbar = S' k, with S' = S (.) decay (or S itself, literal reading) */
+            for (int i = 0; i < dv; ++i) {
+                double acc = 0.0;
+                for (int j = 0; j < dk; ++j) {
+                    double s = S[(long)i * dk + j];
+                    if (!residual_pre_decay) s *= decay[j];
+                    acc += s * kt[j];
+                }
+                pred[i] = acc;
+            }
+            /* S_t = S' + beta_t (v_t - vbar) k_t^T */
+            const double b = beta[t];
+            for (int i = 0; i < dv; ++i) {
+                const double r = vt[i] - pred[i];
+                for (int j = 0; j < dk; ++j) {
+                    long ij = (long)i * dk + j;
+                    S[ij] = decay[j] * S[ij] + b * r * kt[j];
+                }
+            }
+        }
+        /* readout after the write: o_t = S_t q_t */
+        for (int i = 0; i < dv; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < dk; ++j) acc += S[(long)i * dk + j] * qt[j];
+            ot[i] = acc;
+        }
+    }
+}
+
+/*
+ * Delta-rule family scan. beta may be NULL for LINEAR; gate is NULL for LINEAR and
+ * DELTANET, [B,H,T] for GDN, [B,H,T,dk] for KDA. S0 NULL means zeros; S_final NULL
+ * means not written. Returns 0, or -1 on a bad argument.
+ */
+int oracle_dr_scan(const double* q, const double* k, const double* v,
+                   const double* beta, const double* gate, const double* S0,
+                   double* out, double* S_final,
+                   int B, int H, int T, int dk, int dv, int mode, int residual_pre_decay) {
+    if (B < 0 || H < 0 || T < 0 || dk <= 0 || dv <= 0) return -1;
+    if (mode < ORACLE_LINEAR || mode > ORACLE_KDA) return -1;
+    if (!q || !k || !v || !out) return -1;
+    if (mode != ORACLE_LINEAR && !beta) return -1;
+    if ((mode == ORACLE_GDN || mode == ORACLE_KDA) && !gate) return -1;
+    const long BH = (long)B * H;
+    const long state = (long)dv * dk;
+    int failed = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < BH; ++bh) {
+        double* S = (double*)malloc(sizeof(double) * (size_t)state);
+        double* decay = (double*)malloc(sizeof(double) * (size_t)dk);
+        double* pred = (double*)malloc(sizeof(double) * (size_t)dv);
+        if (!S || !decay || !pred) {
+            failed = 1;
+        } else {
+            if (S0) memcpy(S, S0 + bh * state, sizeof(double) * (size_t)state);
+            else memset(S, 0, sizeof(double) * (size_t)state);
+            const double* g = NULL;
+            if (mode == ORACLE_GDN) g = gate + bh * T;
+            if (mode == ORACLE_KDA) g = gate + bh * (long)T * dk;
+            dr_sequence(q + bh * (long)T * dk, k + bh * (long)T * dk, v + bh * (long)T * dv,
+                        beta ? beta + bh * T : NULL, g, S, out + bh * (long)T * dv,
+                        decay, pred, T, dk, dv, mode, residual_pre_decay);
+            if (S_final) memcpy(S_final + bh * state, S, sizeof(double) * (size_t)state);
+        }
+        free(S);
+        free(decay);
+        free(pred);
+    }
+    return failed ? -1 : 0;
+}
+
+/* One VLA sequence. S and A are d x d, updated in place; work holds 3*d doubles. */
+static void vla_sequence(const double* q, const double* k, const double* v, const double* u,
+                         double* S, double* A, double* out, double* work, long T, int d) {
+    double* z = work;          /* z_t = A_{t-1} u_t */
+    double* y = work + d;      /* A_t k_hat_t, then alpha_hat_t */
+    double* r = work + 2 * d;  /* v_t - S_{t-1} k_hat_t */
+    for (long t = 0; t < T; ++t) {
+        const double* ut = u + t * d;
+        const double* kt = k + t * d;
+        const double* vt = v + t * d;
+        const double* qt = q + t * d;
+        double* ot = out + t * d;
+
+        /* step 1: A_t = A_{t-1} - z z^T / (1 + u^T z), z = A_{t-1} u  (section 2.3, Sherman-Morrison) */
+        for (int i = 0; i < d; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < d; ++j) acc += A[(long)i * d + j] * ut[j];
+            z[i] = acc;
+        }
+        double den = 1.0;
+        for (int i = 0; i < d; ++i) den += ut[i] * z[i];
+        for (int i = 0; i < d; ++i)
+            for (int j = 0; j < d; ++j) A[(long)i * d + j] -= z[i] * z[j] / den;
+
+        /* step 2: alpha_hat = A_t k_hat / ||A_t k_hat|| */
+        double nrm2 = 0.0;
+        for (int i = 0; i < d; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < d; ++j) acc += A[(long)i * d + j] * kt[j];
+            y[i] = acc;
+            nrm2 += acc * acc;
+        }
+        const double inv = 1.0 / sqrt(nrm2);
+        for (int i = 0; i < d; ++i) y[i] *= inv;
+
+        /* step 3: S_t = S_{t-1} + (v - S_{t-1} k_hat) alpha_hat^T */
+        for (int i = 0; i < d; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < d; ++j) acc += S[(long)i * d + j] * kt[j];
+            r[i] = vt[i] - acc;
+        }
+        for (int i = 0; i < d; ++i)
+            for (int j = 0; j < d; ++j) S[(long)i * d + j] += r[i] * y[j];
+
+        /* readout o_t = S_t q_hat_t */
+        for (int i = 0; i < d; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < d; ++j) acc += S[(long)i * d + j] * qt[j];
+            ot[i] = acc;
+        }
+    }
+}
+
+/*
+ * VLA Sherman-Morrison scan. S0 NULL = zeros; A0 NULL = I / lambda0.
+ * S_final / A_final NULL = not written. Returns 0, or -1 on a bad argument.
+ */
+int oracle_vla_scan(const double* q, const double* k, const double* v, const double* u,
+                    const double* S0, const double* A0, double lambda0,
+                    double* out, double* S_final, double* A_final,
+                    int B, int H, int T, int d) {
+    if (B < 0 || H < 0 || T < 0 || d <= 0) return -1;
+    if (!q || !k || !v || !u || !out) return -1;
+    if (!A0 && !(lambda0 > 0.0)) return -1;
+    const long BH = (long)B * H;
+    const long dd = (long)d * d;
+    int failed = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < BH; ++bh) {
+        double* S = (double*)malloc(sizeof(double) * (size_t)dd);
+        double* A = (double*)malloc(sizeof(double) * (size_t)dd);
+        double* work = (double*)malloc(sizeof(double) * 3 * (size_t)d);
+        if (!S || !A || !work) {
+            failed = 1;
+        } else {
+            if (S0) memcpy(S, S0 + bh * dd, sizeof(double) * (size_t)dd);
+            else memset(S, 0, sizeof(double) * (size_t)dd);
+            if (A0) {
+                memcpy(A, A0 + bh * dd, sizeof(double) * (size_t)dd);
+            } else {
+                memset(A, 0, sizeof(double) * (size_t)dd);
+                for (int i = 0; i < d; ++i) A[(long)i * d + i] = 1.0 / lambda0;
+            }
+            const long off = bh * (long)T * d;
+            vla_sequence(q + off, k + off, v + off, u + off, S, A, out + off, work, T, d);
+            if (S_final) memcpy(S_final + bh * dd, S, sizeof(double) * (size_t)dd);
+            if (A_final) memcpy(A_final + bh * dd, A, sizeof(double) * (size_t)dd);
+        }
+        free(S);
+        free(A);
+        free(work);
+    }
+    return failed ? -1 : 0;
+}
