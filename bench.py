@@ -1,0 +1,437 @@
+"""Benchmark of the forward delta-rule scan on B200: head-tokens/s and roofline fraction.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one dr_scan_fwd call over the whole workload (all B*H sequences, all T tokens),
+inputs resident in HBM. Under torchrun each rank runs the same workload on its own GPU
+(independent sequences, no collective on the data path: weak scaling); the time is the
+max over ranks and `value` counts the head-tokens all ranks processed.
+Rank 0 prints ONE JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("scan fwd tokens/s per B200 (B·H·T/time) and % of roofline "
+          "(TC FLOP/s or HBM GB/s)")
+UNIT = "tokens/s"
+L2_BYTES = 126 * 1024 * 1024
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=2000)
+    p.add_argument("--warmup", type=int, default=20)
+    p.add_argument("--workload", default="gdn_bf16")
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--e2e-steps", type=int, default=20)
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args(argv)
+
+
+# ---------------------------------------------------------------------------------------
+# workload accounting
+# ---------------------------------------------------------------------------------------
+def algorithmic_bytes(w, with_state_in=None, with_state_out=True) -> int:
+    """Bytes the scan must move once: q, k, v in, out out, beta and gates in, S0 in (when
+    given) and S_final out. Per head-token this is the figure the roofline uses."""
+    from delta_rule_recurrent_chunked_b200 import workloads as wl
+
+    isz = 2 if w.dtype == "bf16" else 4
+    BH, T = w.B * w.H, w.T
+    per_head = T * (2 * w.dk + 2 * w.dv) * isz
+    if w.mode != wl.LINEAR:
+        per_head += T * 4
+    if w.mode == wl.GDN:
+        per_head += T * 4
+    elif w.mode == wl.KDA:
+        per_head += T * w.dk * 4
+    state = w.dv * w.dk * 4
+    if with_state_in if with_state_in is not None else w.s0_std > 0:
+        per_head += state
+    if with_state_out:
+        per_head += state
+    return BH * per_head
+
+
+def algorithmic_flops(w) -> int:
+    """Dense-chunk FLOPs of the chunked form (C = 64), triangular halves counted once."""
+    C = 64
+    per_token = 6 * w.dk * w.dv + C * (3 * w.dk + 2 * w.dv) + C * C // 3
+    return w.B * w.H * w.T * per_token
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------------------
+# clocks during the timed region (NVML reads only; nothing is changed)
+# ---------------------------------------------------------------------------------------
+class ClockSampler:
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index, period_s=0.002):
+        self.period = period_s
+        self.samples = []
+        self.reasons = 0
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.handle = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.handle, pynvml.NVML_CLOCK_SM)
+        except Exception:
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.handle, nv.NVML_CLOCK_SM))
+                self.reasons |= int(nv.nvmlDeviceGetCurrentClocksEventReasons(self.handle))
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def start(self):
+        if self.nv is not None:
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
+
+    def stop(self):
+        if self._thread is not None:
+            self._stop.set()
+            self._thread.join()
+        reasons = [k for k, bit in self.REASONS.items() if self.reasons & bit and k != "gpu_idle"]
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": reasons, "samples": len(self.samples)}
+
+
+# ---------------------------------------------------------------------------------------
+# distributed plumbing
+# ---------------------------------------------------------------------------------------
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def max_over_ranks(value: float, group=None, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+
+    if not dist.is_available() or not dist.is_initialized():
+        return value
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX, group=group)
+    return float(t.item())
+
+
+def barrier(device=None):
+    import torch.distributed as dist
+
+    if dist.is_available() and dist.is_initialized():
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# ---------------------------------------------------------------------------------------
+# CPU baseline: the fp64 oracle on the host cores, on a bounded sample of the workload
+# ---------------------------------------------------------------------------------------
+def oracle_sample(inputs, heads, T):
+    from delta_rule_recurrent_chunked_b200 import workloads as wl
+
+    sub = wl.head_slice(inputs, heads)
+    for key in ("q", "k", "v", "beta", "gate", "u"):
+        if sub.get(key) is not None:
+            sub[key] = np.ascontiguousarray(sub[key][:, :, :T])
+    return sub
+
+
+def run_oracle(sub):
+    import oracle
+    from delta_rule_recurrent_chunked_b200 import workloads as wl
+
+    w = sub["workload"]
+    if isinstance(w, wl.VLAWorkload):
+        oracle.vla_scan(sub["q"], sub["k"], sub["v"], sub["u"], lambda0=w.lambda0)
+    else:
+        oracle.dr_scan(sub["q"], sub["k"], sub["v"], sub["beta"], sub["gate"], sub["S0"], w.mode)
+
+
+def cpu_baseline(inputs, target_s=10.0):
+    """Time the oracle on whole heads (all T tokens), as many as fit ~target_s."""
+    import oracle
+
+    w = inputs["workload"]
+    cores = oracle.num_threads()
+    BH = w.B * w.H
+    probe = oracle_sample(inputs, list(range(min(BH, cores))), min(w.T, 512))
+    t0 = time.perf_counter()
+    run_oracle(probe)
+    dt = max(time.perf_counter() - t0, 1e-6)
+    rate = min(BH, cores) * min(w.T, 512) / dt  # head-tokens/s with all cores busy
+    heads = int(max(1, min(BH, round(rate * target_s / w.T))))
+    heads = max(1, (heads // cores) * cores) if heads >= cores else heads
+    sub = oracle_sample(inputs, list(range(heads)), w.T)
+    t0 = time.perf_counter()
+    run_oracle(sub)
+    dt = time.perf_counter() - t0
+    return {"value": heads * w.T / dt, "unit": UNIT, "cores": cores, "kind": "oracle",
+            "sample": f"{heads} of {BH} heads x all {w.T} tokens (fp64 oracle, {dt:.1f} s)"}
+
+
+# ---------------------------------------------------------------------------------------
+# our arm
+# ---------------------------------------------------------------------------------------
+def make_device_inputs(inputs, device):
+    import torch
+
+    w = inputs["workload"]
+    dev = {}
+    for name in ("q", "k", "v"):
+        raw = inputs[name + "_raw"]
+        t = torch.from_numpy(np.ascontiguousarray(raw).view(np.int16)).view(torch.bfloat16) \
+            if w.dtype == "bf16" else torch.from_numpy(np.ascontiguousarray(raw))
+        dev[name] = t.to(device)
+    for name in ("beta", "gate", "S0"):
+        arr = inputs.get(name)
+        dev[name] = None if arr is None else torch.from_numpy(np.ascontiguousarray(arr)).to(device)
+    return dev
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    import torch.distributed as dist
+
+    import delta_rule_recurrent_chunked_b200 as drs
+    from delta_rule_recurrent_chunked_b200 import workloads as wl
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", device_id=device, timeout=timedelta(seconds=120))
+
+    w = wl.workload(args.workload)
+    if isinstance(w, wl.VLAWorkload):
+        raise SystemExit("bench.py times the delta-rule workloads; VLA is a parity workload")
+    inputs = wl.generate_dr(w, seed=rank)
+    mode = {wl.LINEAR: "linear", wl.DELTANET: "deltanet", wl.GDN: "gdn", wl.KDA: "kda"}[w.mode]
+    nbytes = algorithmic_bytes(w)
+    nsets = max(1, min(4, -(-3 * L2_BYTES // max(nbytes, 1))))  # >= 3x L2 across the rotation
+    sets = [make_device_inputs(inputs, device) for _ in range(nsets)]
+    outs = [torch.empty_like(s["v"]) for s in sets]
+    Sfs = [torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device=device) for _ in sets]
+
+    def step(i):
+        s = sets[i % nsets]
+        drs.scan(s["q"], s["k"], s["v"], s["beta"], s["gate"], s["S0"], mode=mode,
+                 out=outs[i % nsets], S_final=Sfs[i % nsets])
+
+    stream = torch.cuda.current_stream(device)
+    for i in range(max(3, args.warmup)):
+        step(i)
+    torch.cuda.synchronize(device)
+    if drs.poll_error(device) != 0:
+        raise RuntimeError("device status set during warm-up")
+
+    K = args.steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    clocks = ClockSampler(local)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    clocks.start()
+    t_wall = time.perf_counter()
+    for i in range(K):
+        starts[i].record(stream)
+        step(i)
+        ends[i].record(stream)
+    torch.cuda.synchronize(device)
+    t_wall = time.perf_counter() - t_wall
+    barrier(device)
+    clk = clocks.stop()
+    total_ms = starts[0].elapsed_time(ends[-1])
+    per_launch = [starts[i].elapsed_time(ends[i]) for i in range(K)]
+    status = drs.poll_error(device)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed region")
+
+    total_ms_max = max_over_ranks(total_ms, device=device)
+    units = world * w.head_tokens * K
+    value = units / (total_ms_max / 1e3)
+    launch_ms = statistics.mean(per_launch)
+
+    # end to end through the C ABI with host buffers: pinned H2D, scan, D2H of the results
+    e2e = run_e2e(args, w, inputs, mode, device, stream)
+    e2e_ms = max_over_ranks(e2e["ms"], device=device)  # slowest rank
+
+    peaks, peak_src = load_peaks()
+    achieved = nbytes / (launch_ms / 1e3) / 1e9
+    flops = algorithmic_flops(w)
+    tflops = flops / (launch_ms / 1e3) / 1e12
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
+        "warmup": max(3, args.warmup), "ms_per_step": total_ms_max / K,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
+        "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv,
+                   "mode": mode, "chunk": 64, "parallelism": f"replicas{world}" if world > 1 else "1gpu",
+                   "l2": f"rotating {nsets} resident input sets ({nsets * nbytes / 2**20:.0f} MiB) > 126 MiB L2",
+                   "kernel": "chunked" if drs.chunked_applies(mode, w.dtype == "bf16", w.dk, w.dv)
+                   else "sequential"},
+        "clocks": {k: clk[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+        "e2e": {"value": world * w.head_tokens / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
+        "gpu_launches": K,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "peak_source": f"{peak_src} hbm_gbs", "bytes_per_launch": nbytes,
+                     "launch_ms": launch_ms,
+                     "tensor_tflops": tflops,
+                     "tensor_frac": tflops / peaks["bf16_tflops"]},
+        "wall_s": t_wall,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(inputs)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, w, inputs, mode, device, stream):
+    """Same workload through the public API with pinned host buffers: per step copy the
+    inputs host->device, run the scan, copy out and S_final device->host."""
+    import torch
+
+    import delta_rule_recurrent_chunked_b200 as drs
+
+    host = {}
+    for name in ("q", "k", "v"):
+        raw = np.ascontiguousarray(inputs[name + "_raw"])
+        t = torch.from_numpy(raw.view(np.int16)).view(torch.bfloat16) if w.dtype == "bf16" \
+            else torch.from_numpy(raw)
+        host[name] = t.pin_memory()
+    for name in ("beta", "gate", "S0"):
+        a = inputs.get(name)
+        host[name] = None if a is None else torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+    dev = {k: (None if t is None else torch.empty_like(t, device=device)) for k, t in host.items()}
+    out = torch.empty_like(dev["v"])
+    Sf = torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device=device)
+    out_h = torch.empty_like(out, device="cpu").pin_memory()
+    Sf_h = torch.empty_like(Sf, device="cpu").pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
+    d2h = out.numel() * out.element_size() + Sf.numel() * Sf.element_size()
+
+    def step():
+        for k, t in host.items():
+            if t is not None:
+                dev[k].copy_(t, non_blocking=True)
+        drs.scan(dev["q"], dev["k"], dev["v"], dev["beta"], dev["gate"], dev["S0"], mode=mode,
+                 out=out, S_final=Sf)
+        out_h.copy_(out, non_blocking=True)
+        Sf_h.copy_(Sf, non_blocking=True)
+
+    for _ in range(3):
+        step()
+    torch.cuda.synchronize(device)
+    n = max(1, args.e2e_steps)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(n):
+        step()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    return {"ms": a.elapsed_time(b) / n, "h2d": h2d, "d2h": d2h}
+
+
+# ---------------------------------------------------------------------------------------
+# reference arm: the fp64 oracle as it stands, on the host cores
+# ---------------------------------------------------------------------------------------
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    import oracle
+    from delta_rule_recurrent_chunked_b200 import workloads as wl
+
+    w = wl.workload(args.workload)
+    inputs = wl.generate(w, seed=0)
+    cores = oracle.num_threads()
+    BH = w.B * w.H
+    heads = list(range(min(BH, cores)))
+    probe = oracle_sample(inputs, heads, min(w.T, 256))
+    t0 = time.perf_counter()
+    run_oracle(probe)
+    rate = len(heads) * min(w.T, 256) / max(time.perf_counter() - t0, 1e-6)
+    steps_total = args.steps + max(3, args.warmup)
+    budget_s = 120.0
+    T_s = int(max(1, min(w.T, rate * budget_s / steps_total / len(heads))))
+    sub = oracle_sample(inputs, heads, T_s)
+    for _ in range(max(3, args.warmup)):
+        run_oracle(sub)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        run_oracle(sub)
+    dt = time.perf_counter() - t0
+    value = len(heads) * T_s * args.steps / dt
+    sample = f"{len(heads)} of {BH} heads x first {T_s} of {w.T} tokens per step (fp64 oracle)"
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": dt * 1e3 / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": {"workload": w.name},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    world, rank, local = dist_env()
+    if args.impl == "reference":
+        run_reference(args, world, rank)
+    else:
+        run_ours(args, world, rank, local)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,170 @@
+"""B200-native forward recurrent-memory scan of delta-rule linear attention.
+
+Thin Python binding over the C-ABI library ``libdrscan.so`` (declared in
+``include/drscan.h``). This module only marshals arguments: it checks tensor dtypes,
+shapes and devices, passes raw device pointers and the current CUDA stream, and raises
+on a non-zero status. Every step of the scan runs in the library's CUDA kernels; there
+is no CPU fallback, and a missing library is an error.
+
+    out, S_final = scan(q, k, v, beta, gate, S0=None, mode="gdn")
+    out, S_final, A_final = vla_scan(q, k, v, u, S0=None, A0=None, lambda0=1.0)
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(PKG, "libdrscan.so")
+
+DR_LINEAR, DR_DELTANET, DR_GDN, DR_KDA = 0, 1, 2, 3
+DR_IN_BF16 = 0x100
+DR_FORCE_SEQUENTIAL = 0x200
+DR_OK, DR_ERR_INVALID_ARG, DR_ERR_UNSUPPORTED, DR_ERR_CUDA, DR_ERR_TIMEOUT, DR_ERR_DEVICE_BOUNDS = (
+    0, -1, -2, -3, -4, -5)
+MODES = {"linear": DR_LINEAR, "deltanet": DR_DELTANET, "gdn": DR_GDN, "kda": DR_KDA}
+
+# Every function the C ABI exports, with its ctypes signature.
+_VP, _I, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
+SIGNATURES = {
+    "dr_scan_fwd": ([_VP] * 8 + [_I] * 6 + [_VP], _I),
+    "vla_scan_fwd": ([_VP] * 6 + [_F] + [_VP] * 3 + [_I] * 4 + [_VP], _I),
+    "dr_status_string": ([_I], ctypes.c_char_p),
+    "dr_poll_error": ([_VP], _I),
+    "dr_debug_timeout_probe": ([_I, _VP], _I),
+    "dr_version": ([], _I),
+}
+
+_lib = None
+
+
+class DrScanError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: status {status} ({status_string(status)})")
+
+
+def lib():
+    """Load libdrscan.so (built in-tree). Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(
+                f"{LIB_PATH} is missing: build it with "
+                "`python -m delta_rule_recurrent_chunked_b200.build` (nvcc, sm_100a)")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (argtypes, restype) in SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.argtypes = argtypes
+            fn.restype = restype
+        _lib = handle
+    return _lib
+
+
+def status_string(status: int) -> str:
+    return lib().dr_status_string(int(status)).decode()
+
+
+def _stream_handle(device):
+    import torch
+
+    return ctypes.c_void_p(torch.cuda.current_stream(device).cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _check(t, name, shape, dtype, device):
+    if t.device != device:
+        raise ValueError(f"{name} must be on {device}, got {t.device}")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def scan(q, k, v, beta=None, gate=None, S0=None, mode="gdn", want_state=True,
+         force_sequential=False, out=None, S_final=None):
+    """Delta-rule scan on the GPU. q, k: [B,H,T,dk]; v: [B,H,T,dv] (bf16 or fp32, same
+    dtype); beta: [B,H,T] fp32; gate: alpha values, [B,H,T] (gdn) or [B,H,T,dk] (kda) fp32;
+    S0: [B,H,dv,dk] fp32 or None. Returns (out like v, S_final fp32 or None)."""
+    import torch
+
+    variant = MODES[mode] if isinstance(mode, str) else int(mode)
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    if q.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("q/k/v must be bf16 or fp32")
+    _check(q, "q", (B, H, T, dk), q.dtype, dev)
+    _check(k, "k", (B, H, T, dk), q.dtype, dev)
+    _check(v, "v", (B, H, T, dv), q.dtype, dev)
+    if variant != DR_LINEAR:
+        _check(beta, "beta", (B, H, T), torch.float32, dev)
+    else:
+        beta = None
+    if variant == DR_GDN:
+        _check(gate, "gate", (B, H, T), torch.float32, dev)
+    elif variant == DR_KDA:
+        _check(gate, "gate", (B, H, T, dk), torch.float32, dev)
+    else:
+        gate = None
+    if S0 is not None:
+        _check(S0, "S0", (B, H, dv, dk), torch.float32, dev)
+    if out is None:
+        out = torch.empty((B, H, T, dv), dtype=q.dtype, device=dev)
+    _check(out, "out", (B, H, T, dv), q.dtype, dev)
+    if want_state and S_final is None:
+        S_final = torch.empty((B, H, dv, dk), dtype=torch.float32, device=dev)
+    if S_final is not None:
+        _check(S_final, "S_final", (B, H, dv, dk), torch.float32, dev)
+    flags = variant | (DR_IN_BF16 if q.dtype == torch.bfloat16 else 0)
+    if force_sequential:
+        flags |= DR_FORCE_SEQUENTIAL
+    rc = lib().dr_scan_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(gate), _ptr(S0), _ptr(out),
+                           _ptr(S_final), B, H, T, dk, dv, flags, _stream_handle(dev))
+    if rc != DR_OK:
+        raise DrScanError(rc, "dr_scan_fwd")
+    return out, S_final
+
+
+def vla_scan(q, k, v, u, S0=None, A0=None, lambda0=1.0, want_state=True, out=None):
+    """VLA Sherman-Morrison scan on the GPU (fp32). q, k, v, u: [B,H,T,d];
+    S0, A0: [B,H,d,d] or None. Returns (out, S_final, A_final)."""
+    import torch
+
+    B, H, T, d = q.shape
+    dev = q.device
+    for name, t in (("q", q), ("k", k), ("v", v), ("u", u)):
+        _check(t, name, (B, H, T, d), torch.float32, dev)
+    for name, t in (("S0", S0), ("A0", A0)):
+        if t is not None:
+            _check(t, name, (B, H, d, d), torch.float32, dev)
+    if out is None:
+        out = torch.empty((B, H, T, d), dtype=torch.float32, device=dev)
+    _check(out, "out", (B, H, T, d), torch.float32, dev)
+    Sf = torch.empty((B, H, d, d), dtype=torch.float32, device=dev) if want_state else None
+    Af = torch.empty((B, H, d, d), dtype=torch.float32, device=dev) if want_state else None
+    rc = lib().vla_scan_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(S0), _ptr(A0),
+                            float(lambda0), _ptr(out), _ptr(Sf), _ptr(Af), B, H, T, d,
+                            _stream_handle(dev))
+    if rc != DR_OK:
+        raise DrScanError(rc, "vla_scan_fwd")
+    return out, Sf, Af
+
+
+def poll_error(device=None) -> int:
+    """Synchronise the current stream and return/clear the device status word."""
+    import torch
+
+    dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+    return int(lib().dr_poll_error(_stream_handle(dev)))
+
+
+def chunked_applies(mode, dtype_is_bf16: bool, dk: int, dv: int) -> bool:
+    """Whether dr_scan_fwd runs the chunked tensor-core kernel for this request."""
+    variant = MODES[mode] if isinstance(mode, str) else int(mode)
+    return dtype_is_bf16 and dk == 128 and variant in (DR_DELTANET, DR_GDN, DR_KDA)

@@ -1,0 +1,136 @@
+// Per-token delta-rule scan with an fp32 state on CUDA cores.
+//
+// Every row of S evolves independently given (k_t, alpha_t, beta_t): with
+// S' = S_{t-1} diag(a_t), row i of the update is
+//     s_i <- a (.) s_i + beta_t (v_t[i] - (a (.) s_i) . k_t) k_t
+// and o_t[i] = s_i . q_t (readout after the write). One thread owns one row of S in
+// registers, so a token costs ~4*dk FMAs per thread and no cross-thread communication.
+// A CTA is one warp covering 32 consecutive rows (value channels) of one (b,h); tokens
+// are staged through shared memory in tiles and broadcast to the warp.
+#pragma once
+
+#include "common.cuh"
+
+namespace drscan {
+
+constexpr int SEQ_TILE = 16;  // tokens staged per shared-memory tile
+
+template <typename TIn>
+__device__ __forceinline__ float to_f32(TIn x);
+template <>
+__device__ __forceinline__ float to_f32<float>(float x) {
+    return x;
+}
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+    return __bfloat162float(x);
+}
+
+template <typename TIn>
+__device__ __forceinline__ TIn from_f32(float x);
+template <>
+__device__ __forceinline__ float from_f32<float>(float x) {
+    return x;
+}
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
+    return __float2bfloat16_rn(x);
+}
+
+// grid: (B*H, dv/32); block: 32 threads.
+template <typename TIn, int MODE, int DK>
+__global__ void __launch_bounds__(32) dr_sequential_kernel(
+    const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
+    const float* __restrict__ beta, const float* __restrict__ gate, const float* __restrict__ S0,
+    TIn* __restrict__ out, float* __restrict__ S_final, int T, int dv) {
+    __shared__ __align__(16) float sk[SEQ_TILE][DK];
+    __shared__ __align__(16) float sq[SEQ_TILE][DK];
+    __shared__ __align__(16) float sa[MODE == DR_KDA ? SEQ_TILE : 1][MODE == DR_KDA ? DK : 4];
+    __shared__ float sv[SEQ_TILE][32];
+    __shared__ float sb[SEQ_TILE];
+    __shared__ float sg[SEQ_TILE];
+
+    const int lane = threadIdx.x;
+    const long bh = blockIdx.x;
+    const int row = blockIdx.y * 32 + lane;
+
+    const TIn* qh = q + bh * (long)T * DK;
+    const TIn* kh = k + bh * (long)T * DK;
+    const TIn* vh = v + bh * (long)T * dv;
+    TIn* oh = out + bh * (long)T * dv;
+
+    float s[DK];
+    if (S0) {
+        const float* src = S0 + (bh * dv + row) * (long)DK;
+#pragma unroll
+        for (int j = 0; j < DK; j += 4) {
+            float4 x = *reinterpret_cast<const float4*>(src + j);
+            s[j] = x.x;
+            s[j + 1] = x.y;
+            s[j + 2] = x.z;
+            s[j + 3] = x.w;
+        }
+    } else {
+#pragma unroll
+        for (int j = 0; j < DK; ++j) s[j] = 0.f;
+    }
+
+    for (int t0 = 0; t0 < T; t0 += SEQ_TILE) {
+        const int nt = min(SEQ_TILE, T - t0);
+        __syncwarp();
+        for (int e = lane; e < nt * DK; e += 32) {
+            const int tt = e / DK, j = e % DK;
+            sk[tt][j] = to_f32(kh[(long)(t0 + tt) * DK + j]);
+            sq[tt][j] = to_f32(qh[(long)(t0 + tt) * DK + j]);
+            if constexpr (MODE == DR_KDA) sa[tt][j] = gate[(bh * T + t0 + tt) * (long)DK + j];
+        }
+        for (int tt = 0; tt < nt; ++tt) sv[tt][lane] = to_f32(vh[(long)(t0 + tt) * dv + row]);
+        if (lane < nt) {
+            sb[lane] = (MODE == DR_LINEAR) ? 1.f : beta[bh * T + t0 + lane];
+            sg[lane] = (MODE == DR_GDN) ? gate[bh * T + t0 + lane] : 1.f;
+        }
+        __syncwarp();
+
+        for (int tt = 0; tt < nt; ++tt) {
+            const float vi = sv[tt][lane];
+            if constexpr (MODE == DR_LINEAR) {
+#pragma unroll
+                for (int j = 0; j < DK; ++j) s[j] = fmaf(vi, sk[tt][j], s[j]);
+            } else {
+                if constexpr (MODE == DR_GDN) {
+                    const float a = sg[tt];
+#pragma unroll
+                    for (int j = 0; j < DK; ++j) s[j] *= a;
+                } else if constexpr (MODE == DR_KDA) {
+#pragma unroll
+                    for (int j = 0; j < DK; ++j) s[j] *= sa[tt][j];
+                }
+                float p0 = 0.f, p1 = 0.f;
+#pragma unroll
+                for (int j = 0; j < DK; j += 2) {
+                    p0 = fmaf(s[j], sk[tt][j], p0);
+                    p1 = fmaf(s[j + 1], sk[tt][j + 1], p1);
+                }
+                const float w = sb[tt] * (vi - (p0 + p1));
+#pragma unroll
+                for (int j = 0; j < DK; ++j) s[j] = fmaf(w, sk[tt][j], s[j]);
+            }
+            float o0 = 0.f, o1 = 0.f;
+#pragma unroll
+            for (int j = 0; j < DK; j += 2) {
+                o0 = fmaf(s[j], sq[tt][j], o0);
+                o1 = fmaf(s[j + 1], sq[tt][j + 1], o1);
+            }
+            oh[(long)(t0 + tt) * dv + row] = from_f32<TIn>(o0 + o1);
+        }
+    }
+
+    if (S_final) {
+        float* dst = S_final + (bh * dv + row) * (long)DK;
+#pragma unroll
+        for (int j = 0; j < DK; j += 4)
+            *reinterpret_cast<float4*>(dst + j) = make_float4(s[j], s[j + 1], s[j + 2], s[j + 3]);
+    }
+}
+
+}  // namespace drscan

@@ -1,0 +1,204 @@
+// Variational Linear Attention scan, warp-specialised, fp32, one CTA per (b,h).
+//
+// Two thread groups of d threads each:
+//  * the A-group owns A (row i in thread i's registers) and produces the write direction
+//    alpha_hat_t for every token: z = A_{t-1} u and y = A_{t-1} k in one pass over the row,
+//    two group reductions (u.z and k.z), then A_t k = y - z (z.k)/(1 + u.z) (Sherman-Morrison
+//    applied to the vector, so no second dependent mat-vec), a third reduction for the
+//    norm, and the rank-1 update of A's row;
+//  * the S-group owns S (row i in thread i's registers); given alpha_hat_t its rows are
+//    independent: r_i = v_i - s_i.k, s_i += r_i alpha_hat, o_i = s_i.q. No reductions.
+// The groups run one token tile apart: while the A-group produces the directions of tile n
+// into a shared-memory ring, the S-group consumes tile n-1. One __syncthreads per tile.
+#pragma once
+
+#include "common.cuh"
+
+namespace drscan {
+
+constexpr int VLA_TILE = 16;
+
+template <int D>
+struct VlaSmem {
+    float uA[2][VLA_TILE][D];
+    float kA[2][VLA_TILE][D];
+    float kS[2][VLA_TILE][D];
+    float vS[2][VLA_TILE][D];
+    float qS[2][VLA_TILE][D];
+    float ring[2][VLA_TILE][D];
+    float zbuf[D];
+    float red1[2][4];
+    float red2[4];
+};
+
+template <int D>
+__device__ __forceinline__ void vla_group_sum2(float& x, float& y, float (*red)[4], int i) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        x += __shfl_xor_sync(0xffffffffu, x, off);
+        y += __shfl_xor_sync(0xffffffffu, y, off);
+    }
+    if constexpr (D > 32) {
+        if ((i & 31) == 0) {
+            red[0][i >> 5] = x;
+            red[1][i >> 5] = y;
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(D) : "memory");
+        x = 0.f;
+        y = 0.f;
+#pragma unroll
+        for (int w = 0; w < D / 32; ++w) {
+            x += red[0][w];
+            y += red[1][w];
+        }
+    } else {
+        __syncwarp();
+    }
+}
+
+template <int D>
+__device__ __forceinline__ float vla_group_sum1(float x, float* red, int i) {
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+    if constexpr (D > 32) {
+        if ((i & 31) == 0) red[i >> 5] = x;
+        asm volatile("bar.sync 1, %0;" ::"n"(D) : "memory");
+        x = 0.f;
+#pragma unroll
+        for (int w = 0; w < D / 32; ++w) x += red[w];
+    }
+    return x;
+}
+
+template <int D>
+__device__ __forceinline__ void vla_load_tile(float (*dst)[D], const float* src, int nt, int tid) {
+    const float4* s4 = reinterpret_cast<const float4*>(src);
+    float4* d4 = reinterpret_cast<float4*>(&dst[0][0]);
+    for (int e = tid; e < nt * D / 4; e += D) d4[e] = s4[e];
+}
+
+// grid: B*H; block: 2*D threads; dynamic shared memory: sizeof(VlaSmem<D>).
+template <int D>
+__global__ void __launch_bounds__(2 * D) vla_sequential_kernel(
+    const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
+    const float* __restrict__ u, const float* __restrict__ S0, const float* __restrict__ A0,
+    float lambda0, float* __restrict__ out, float* __restrict__ S_final,
+    float* __restrict__ A_final, int T) {
+    extern __shared__ __align__(16) unsigned char vla_smem_raw[];
+    VlaSmem<D>& sm = *reinterpret_cast<VlaSmem<D>*>(vla_smem_raw);
+
+    const int tid = threadIdx.x;
+    const bool is_a = tid < D;
+    const int i = is_a ? tid : tid - D;
+    const long bh = blockIdx.x;
+    const long seq = bh * (long)T * D;
+    const long mat = bh * (long)D * D;
+    const int ntiles = (T + VLA_TILE - 1) / VLA_TILE;
+
+    float m[D];  // row i of A (A-group) or of S (S-group)
+    if (is_a) {
+        if (A0) {
+#pragma unroll
+            for (int j = 0; j < D; ++j) m[j] = A0[mat + (long)i * D + j];
+        } else {
+            const float inv = 1.f / lambda0;
+#pragma unroll
+            for (int j = 0; j < D; ++j) m[j] = (j == i) ? inv : 0.f;
+        }
+        if (ntiles > 0) {
+            const int nt = min(VLA_TILE, T);
+            vla_load_tile<D>(sm.uA[0], u + seq, nt, i);
+            vla_load_tile<D>(sm.kA[0], k + seq, nt, i);
+        }
+    } else {
+        if (S0) {
+#pragma unroll
+            for (int j = 0; j < D; ++j) m[j] = S0[mat + (long)i * D + j];
+        } else {
+#pragma unroll
+            for (int j = 0; j < D; ++j) m[j] = 0.f;
+        }
+    }
+    __syncthreads();
+
+    for (int it = 0; it <= ntiles; ++it) {
+        if (is_a) {
+            if (it + 1 < ntiles) {
+                const int t0 = (it + 1) * VLA_TILE;
+                const int nt = min(VLA_TILE, T - t0);
+                vla_load_tile<D>(sm.uA[(it + 1) & 1], u + seq + (long)t0 * D, nt, i);
+                vla_load_tile<D>(sm.kA[(it + 1) & 1], k + seq + (long)t0 * D, nt, i);
+            }
+            if (it < ntiles) {
+                const int b = it & 1;
+                const int nt = min(VLA_TILE, T - it * VLA_TILE);
+                for (int tt = 0; tt < nt; ++tt) {
+                    const float* uu = sm.uA[b][tt];
+                    const float* kk = sm.kA[b][tt];
+                    float z0 = 0.f, z1 = 0.f, y0 = 0.f, y1 = 0.f;
+#pragma unroll
+                    for (int j = 0; j < D; j += 2) {
+                        z0 = fmaf(m[j], uu[j], z0);
+                        z1 = fmaf(m[j + 1], uu[j + 1], z1);
+                        y0 = fmaf(m[j], kk[j], y0);
+                        y1 = fmaf(m[j + 1], kk[j + 1], y1);
+                    }
+                    const float z = z0 + z1, y = y0 + y1;
+                    sm.zbuf[i] = z;
+                    float uz = uu[i] * z, kz = kk[i] * z;
+                    vla_group_sum2<D>(uz, kz, sm.red1, i);
+                    const float c = 1.f / (1.f + uz);
+#pragma unroll
+                    for (int j = 0; j < D; ++j) m[j] = fmaf(-c * z, sm.zbuf[j], m[j]);
+                    const float yt = fmaf(-c * kz, z, y);  // A_t k = A_{t-1}k - c z (z.k)
+                    const float n2 = vla_group_sum1<D>(yt * yt, sm.red2, i);
+                    sm.ring[b][tt][i] = yt * rsqrtf(n2);
+                    if constexpr (D == 32) __syncwarp();
+                }
+            }
+        } else {
+            if (it < ntiles) {
+                const int t0 = it * VLA_TILE;
+                const int nt = min(VLA_TILE, T - t0);
+                vla_load_tile<D>(sm.kS[it & 1], k + seq + (long)t0 * D, nt, i);
+                vla_load_tile<D>(sm.vS[it & 1], v + seq + (long)t0 * D, nt, i);
+                vla_load_tile<D>(sm.qS[it & 1], q + seq + (long)t0 * D, nt, i);
+            }
+            if (it >= 1) {
+                const int b = (it - 1) & 1;
+                const int t0 = (it - 1) * VLA_TILE;
+                const int nt = min(VLA_TILE, T - t0);
+                for (int tt = 0; tt < nt; ++tt) {
+                    const float* kk = sm.kS[b][tt];
+                    const float* qq = sm.qS[b][tt];
+                    const float* al = sm.ring[b][tt];
+                    float p0 = 0.f, p1 = 0.f;
+#pragma unroll
+                    for (int j = 0; j < D; j += 2) {
+                        p0 = fmaf(m[j], kk[j], p0);
+                        p1 = fmaf(m[j + 1], kk[j + 1], p1);
+                    }
+                    const float r = sm.vS[b][tt][i] - (p0 + p1);
+                    float o0 = 0.f, o1 = 0.f;
+#pragma unroll
+                    for (int j = 0; j < D; j += 2) {
+                        m[j] = fmaf(r, al[j], m[j]);
+                        m[j + 1] = fmaf(r, al[j + 1], m[j + 1]);
+                        o0 = fmaf(m[j], qq[j], o0);
+                        o1 = fmaf(m[j + 1], qq[j + 1], o1);
+                    }
+                    out[seq + (long)(t0 + tt) * D + i] = o0 + o1;
+                }
+            }
+        }
+        __syncthreads();
+    }
+
+    float* dst = is_a ? A_final : S_final;
+    if (dst) {
+#pragma unroll
+        for (int j = 0; j < D; ++j) dst[mat + (long)i * D + j] = m[j];
+    }
+}
+
+}  // namespace drscan

@@ -1,0 +1,122 @@
+"""C-ABI library checks that need no GPU: it loads, exports every symbol the header
+declares, and rejects bad arguments with the documented status codes before touching
+the device (no compute call is made here)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import delta_rule_recurrent_chunked_b200 as drs
+from delta_rule_recurrent_chunked_b200 import build as drbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "drscan.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    drbuild.build_library()
+    return drs.lib()
+
+
+def header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?\w+\s*\*?\s*(\w+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_the_boundary():
+    assert set(header_functions()) == set(drs.SIGNATURES), header_functions()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    out = subprocess.check_output(["nm", "-D", "--defined-only", drs.LIB_PATH]).decode()
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    for name in header_functions():
+        assert name in exported, name
+        assert getattr(lib, name) is not None
+
+
+def test_version_and_status_strings(lib):
+    assert lib.dr_version() >= 100
+    codes = [drs.DR_OK, drs.DR_ERR_INVALID_ARG, drs.DR_ERR_UNSUPPORTED, drs.DR_ERR_CUDA,
+             drs.DR_ERR_TIMEOUT, drs.DR_ERR_DEVICE_BOUNDS]
+    texts = [drs.status_string(c) for c in codes]
+    assert all(t and t != "unknown status" for t in texts)
+    assert len(set(texts)) == len(texts)
+    assert drs.status_string(12345) == "unknown status"
+
+
+A = 0x10000  # a fake, 16-byte aligned address: validation rejects before any dereference
+
+
+def call_dr(lib, q=A, k=A, v=A, beta=A, gate=A, S0=None, out=A, Sf=None, B=1, H=1, T=8, dk=32,
+            dv=32, mode=drs.DR_GDN):
+    P = ctypes.c_void_p
+    return lib.dr_scan_fwd(P(q), P(k), P(v), P(beta), P(gate), P(S0), P(out), P(Sf), B, H, T,
+                           dk, dv, mode, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(q=None), drs.DR_ERR_INVALID_ARG),
+    (dict(out=None), drs.DR_ERR_INVALID_ARG),
+    (dict(beta=None), drs.DR_ERR_INVALID_ARG),
+    (dict(gate=None), drs.DR_ERR_INVALID_ARG),
+    (dict(gate=None, mode=drs.DR_KDA), drs.DR_ERR_INVALID_ARG),
+    (dict(k=A + 4), drs.DR_ERR_INVALID_ARG),
+    (dict(S0=A + 8), drs.DR_ERR_INVALID_ARG),
+    (dict(Sf=A + 2), drs.DR_ERR_INVALID_ARG),
+    (dict(T=-1), drs.DR_ERR_INVALID_ARG),
+    (dict(B=-2), drs.DR_ERR_INVALID_ARG),
+    (dict(dk=0), drs.DR_ERR_INVALID_ARG),
+    (dict(mode=7), drs.DR_ERR_INVALID_ARG),
+    (dict(mode=drs.DR_GDN | 0x800), drs.DR_ERR_INVALID_ARG),
+    (dict(dk=48), drs.DR_ERR_UNSUPPORTED),
+    (dict(dv=256), drs.DR_ERR_UNSUPPORTED),
+    (dict(B=0), drs.DR_OK),                      # empty batch: nothing to launch
+    (dict(H=0, T=0), drs.DR_OK),
+    (dict(q=None, k=None, v=None, out=None, beta=None, gate=None, B=0), drs.DR_OK),
+    (dict(q=A + 4, B=0), drs.DR_ERR_INVALID_ARG),  # misaligned is an error even when unused
+])
+def test_dr_scan_argument_validation(lib, kw, code):
+    assert call_dr(lib, **kw) == code
+
+
+def test_linear_and_deltanet_need_no_gate(lib):
+    # a valid request reaches the launch; with B*H == 0 there is nothing to launch
+    assert call_dr(lib, beta=None, gate=None, mode=drs.DR_LINEAR, B=0) == drs.DR_OK
+    assert call_dr(lib, gate=None, mode=drs.DR_DELTANET, B=0) == drs.DR_OK
+
+
+def call_vla(lib, q=A, k=A, v=A, u=A, S0=None, A0=None, lam=1.0, out=A, B=1, H=1, T=8, d=32):
+    P = ctypes.c_void_p
+    return lib.vla_scan_fwd(P(q), P(k), P(v), P(u), P(S0), P(A0), lam, P(out), None, None, B, H,
+                            T, d, None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(u=None), drs.DR_ERR_INVALID_ARG),
+    (dict(q=A + 4), drs.DR_ERR_INVALID_ARG),
+    (dict(lam=0.0), drs.DR_ERR_INVALID_ARG),
+    (dict(lam=-1.0), drs.DR_ERR_INVALID_ARG),
+    (dict(T=-5), drs.DR_ERR_INVALID_ARG),
+    (dict(d=48), drs.DR_ERR_UNSUPPORTED),
+    (dict(d=256), drs.DR_ERR_UNSUPPORTED),
+    (dict(B=0), drs.DR_OK),
+])
+def test_vla_argument_validation(lib, kw, code):
+    assert call_vla(lib, **kw) == code
+
+
+def test_timeout_probe_rejects_bad_limits(lib):
+    assert lib.dr_debug_timeout_probe(0, None) == drs.DR_ERR_INVALID_ARG
+    assert lib.dr_debug_timeout_probe(10**7, None) == drs.DR_ERR_INVALID_ARG
+
+
+def test_product_path_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(drs, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(drs, "_lib", None)
+    with pytest.raises(RuntimeError, match="missing"):
+        drs.lib()

@@ -1,0 +1,223 @@
+"""GPU parity: the CUDA kernels (through the C ABI) against the fp64 oracle.
+
+Tolerance (max|x - y| / max|y| per tensor, out and S_final):
+  fp32 q/k/v: 1e-4;   bf16 q/k/v with fp32 state: 2e-2 (oracle fed the bf16-rounded inputs).
+Small cases span several 64-token chunks and a ragged tail; the full-size workloads are
+checked on sampled heads (heads are independent sequences), in the launch configuration
+the benchmark times.
+"""
+import numpy as np
+import pytest
+
+import delta_rule_recurrent_chunked_b200 as drs
+from delta_rule_recurrent_chunked_b200 import workloads as wl
+
+from helpers import MODE_NAME, oracle_dr, rel_err, tensor_np, to_device
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+TOL = {"fp32": 1e-4, "bf16": 2e-2}
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    drs.lib()
+    yield
+    assert drs.poll_error() == drs.DR_OK
+
+
+def run_dr(dev, w, force_sequential=False, want_state=True):
+    out, Sf = drs.scan(dev["q"], dev["k"], dev["v"], dev["beta"], dev["gate"], dev["S0"],
+                       mode=MODE_NAME[w.mode], want_state=want_state,
+                       force_sequential=force_sequential)
+    torch.cuda.synchronize()
+    return out, Sf
+
+
+def check_dr(oracle, w, seed=0, force_sequential=False, tol=None):
+    inputs = wl.generate_dr(w, seed)
+    dev = to_device(inputs)
+    out, Sf = run_dr(dev, w, force_sequential)
+    ref_out, ref_S = oracle_dr(oracle, inputs)
+    tol = tol or TOL[w.dtype]
+    e_out, e_S = rel_err(tensor_np(out), ref_out), rel_err(tensor_np(Sf), ref_S)
+    assert e_out <= tol and e_S <= tol, (w, e_out, e_S)
+    return e_out, e_S
+
+
+# --- the parity workload: DeltaNet fp32, B1 H2 T256 d32
+def test_deltanet_fp32_workload(oracle):
+    check_dr(oracle, wl.workload("deltanet_fp32"))
+
+
+# --- every variant, fp32 inputs (per-token kernel), ragged T, all head sizes
+@pytest.mark.parametrize("mode", [wl.LINEAR, wl.DELTANET, wl.GDN, wl.KDA])
+@pytest.mark.parametrize("dk,dv", [(32, 32), (64, 32), (128, 64), (32, 128), (128, 128)])
+@pytest.mark.parametrize("T", [1, 65, 130])
+def test_sequential_fp32_variants(oracle, mode, dk, dv, T):
+    w = wl.DRWorkload("t", 2, 2, T, dk, dv, mode, "fp32", s0_std=0.1, gate_mu=-2.0)
+    check_dr(oracle, w, seed=T + dk + dv)
+
+
+# --- bf16 inputs on the per-token kernel (the fp32-state baseline path)
+@pytest.mark.parametrize("mode", [wl.DELTANET, wl.GDN, wl.KDA])
+def test_sequential_bf16(oracle, mode):
+    w = wl.DRWorkload("t", 1, 3, 200, 128, 128, mode, "bf16", s0_std=0.1)
+    check_dr(oracle, w, seed=3, force_sequential=True)
+
+
+# --- bf16 inputs through the default dispatch (chunked kernel where it applies)
+@pytest.mark.parametrize("mode", [wl.DELTANET, wl.GDN, wl.KDA])
+@pytest.mark.parametrize("T", [1, 63, 64, 65, 127, 200, 517])
+def test_bf16_dispatch_ragged(oracle, mode, T):
+    w = wl.DRWorkload("t", 1, 2, T, 128, 128, mode, "bf16", s0_std=0.1)
+    check_dr(oracle, w, seed=T)
+
+
+@pytest.mark.parametrize("dv", [32, 64])
+@pytest.mark.parametrize("mode", [wl.GDN, wl.KDA])
+def test_bf16_dispatch_narrow_values(oracle, mode, dv):
+    w = wl.DRWorkload("t", 2, 2, 300, 128, dv, mode, "bf16", s0_std=0.1)
+    check_dr(oracle, w, seed=dv)
+
+
+def test_bf16_strong_decay_gates(oracle):
+    # gates near 0.5 per step: summed log-decay over a 64-token chunk reaches about -45
+    w = wl.DRWorkload("t", 1, 2, 256, 128, 128, wl.GDN, "bf16", gate_mu=0.0, gate_sigma=0.5)
+    check_dr(oracle, w, seed=5)
+
+
+# --- full-size workloads, sampled heads
+def _check_sampled(oracle, name, heads, seed=0):
+    w = wl.workload(name)
+    inputs = wl.generate_dr(w, seed)
+    dev = to_device(inputs)
+    out, Sf = run_dr(dev, w)
+    sub = wl.head_slice(inputs, heads)
+    ref_out, ref_S = oracle_dr(oracle, sub)
+    o = tensor_np(out).reshape((w.B * w.H,) + tuple(out.shape[2:]))[heads][None]
+    s = tensor_np(Sf).reshape((w.B * w.H,) + tuple(Sf.shape[2:]))[heads][None]
+    e_out, e_S = rel_err(o, ref_out), rel_err(s, ref_S)
+    assert e_out <= TOL[w.dtype] and e_S <= TOL[w.dtype], (name, e_out, e_S)
+    return e_out, e_S
+
+
+def test_gdn_bf16_workload_sampled(oracle):
+    _check_sampled(oracle, "gdn_bf16", [0, 13, 31])
+
+
+def test_kda_bf16_workload_sampled(oracle):
+    _check_sampled(oracle, "kda_bf16", [0, 77, 127])
+
+
+@pytest.mark.parametrize("T", [4096, 32768])
+def test_gdn_long_workload_sampled(oracle, T):
+    _check_sampled(oracle, f"gdn_long_t{T}", [0, 15])
+
+
+# --- edge cases
+def test_empty_sequence_copies_state():
+    S0 = torch.randn(2, 3, 32, 64, device="cuda")
+    q = torch.empty(2, 3, 0, 64, device="cuda")
+    v = torch.empty(2, 3, 0, 32, device="cuda")
+    beta = torch.empty(2, 3, 0, device="cuda")
+    out, Sf = drs.scan(q, q, v, beta, None, S0, mode="deltanet")
+    torch.cuda.synchronize()
+    assert out.shape == (2, 3, 0, 32) and torch.equal(Sf, S0)
+    _, Sf0 = drs.scan(q, q, v, beta, None, None, mode="deltanet")
+    torch.cuda.synchronize()
+    assert torch.count_nonzero(Sf0) == 0
+
+
+def test_state_optional_and_carry(oracle):
+    w = wl.DRWorkload("t", 1, 2, 256, 128, 128, wl.GDN, "bf16", s0_std=0.1)
+    inputs = wl.generate_dr(w, 9)
+    dev = to_device(inputs)
+    out_nostate, none = run_dr(dev, w, want_state=False)
+    assert none is None
+    out, Sf = run_dr(dev, w)
+    assert torch.equal(out_nostate, out)
+    # resume: two halves with the carried fp32 state equal one pass (up to tolerance)
+    h = 128
+    half = {k: (None if t is None else t) for k, t in dev.items()}
+    a = {k: (t[:, :, :h].contiguous() if t is not None and k != "S0" else t) for k, t in half.items()}
+    o1, S1 = drs.scan(a["q"], a["k"], a["v"], a["beta"], a["gate"], dev["S0"], mode="gdn")
+    b = {k: (t[:, :, h:].contiguous() if t is not None and k != "S0" else t) for k, t in half.items()}
+    o2, S2 = drs.scan(b["q"], b["k"], b["v"], b["beta"], b["gate"], S1, mode="gdn")
+    torch.cuda.synchronize()
+    ref_out, ref_S = oracle_dr(oracle, inputs)
+    assert rel_err(tensor_np(torch.cat([o1, o2], dim=2)), ref_out) <= TOL["bf16"]
+    assert rel_err(tensor_np(S2), ref_S) <= TOL["bf16"]
+
+
+def test_heads_are_independent():
+    w = wl.DRWorkload("t", 1, 4, 130, 128, 128, wl.KDA, "bf16")
+    dev = to_device(wl.generate_dr(w, 4))
+    out, Sf = run_dr(dev, w)
+    p = torch.tensor([2, 0, 3, 1], device="cuda")
+    perm = {k: (None if t is None else t[:, p].contiguous()) for k, t in dev.items()}
+    out_p, Sf_p = run_dr(perm, w)
+    assert torch.equal(out_p, out[:, p]) and torch.equal(Sf_p, Sf[:, p])
+
+
+# --- VLA
+@pytest.mark.parametrize("d", [32, 96])
+def test_vla_workload(oracle, d):
+    w = wl.workload(f"vla_fp32_d{d}")
+    inputs = wl.generate_vla(w, 0)
+    dev = {k: torch.from_numpy(inputs[k]).cuda() for k in ("q", "k", "v", "u")}
+    out, Sf, Af = drs.vla_scan(dev["q"], dev["k"], dev["v"], dev["u"], lambda0=w.lambda0)
+    torch.cuda.synchronize()
+    heads = [0, 9, 31]
+    sub = wl.head_slice(inputs, heads)
+    ref_out, ref_S, ref_A = oracle.vla_scan(sub["q"], sub["k"], sub["v"], sub["u"], lambda0=w.lambda0)
+    o = tensor_np(out).reshape(32, w.T, d)[heads][None]
+    s = tensor_np(Sf).reshape(32, d, d)[heads][None]
+    a = tensor_np(Af).reshape(32, d, d)[heads][None]
+    for got, ref in ((o, ref_out), (s, ref_S), (a, ref_A)):
+        assert rel_err(got, ref) <= 1e-4
+
+
+@pytest.mark.parametrize("d", [32, 64, 96, 128])
+@pytest.mark.parametrize("T", [1, 17, 100])
+def test_vla_small_with_initial_state(oracle, d, T):
+    rng = np.random.default_rng(d + T)
+    B, H = 1, 3
+    unit = lambda x: x / np.linalg.norm(x, axis=-1, keepdims=True)
+    q = unit(rng.standard_normal((B, H, T, d))).astype(np.float32)
+    k = unit(rng.standard_normal((B, H, T, d))).astype(np.float32)
+    v = rng.standard_normal((B, H, T, d)).astype(np.float32)
+    u = (rng.standard_normal((B, H, T, d)) / np.sqrt(d)).astype(np.float32)
+    S0 = (0.1 * rng.standard_normal((B, H, d, d))).astype(np.float32)
+    M = rng.standard_normal((B, H, d, d)) / np.sqrt(d)
+    A0 = np.linalg.inv(np.eye(d) + M @ np.swapaxes(M, -1, -2)).astype(np.float32)
+    c = lambda x: torch.from_numpy(x).cuda()
+    out, Sf, Af = drs.vla_scan(c(q), c(k), c(v), c(u), S0=c(S0), A0=c(A0))
+    torch.cuda.synchronize()
+    ro, rs, ra = oracle.vla_scan(q, k, v, u, S0=S0, A0=A0)
+    assert rel_err(tensor_np(out), ro) <= 1e-4
+    assert rel_err(tensor_np(Sf), rs) <= 1e-4
+    assert rel_err(tensor_np(Af), ra) <= 1e-4
+
+
+def test_vla_empty_sequence_returns_initial_state():
+    d = 32
+    z = torch.empty(1, 2, 0, d, device="cuda")
+    out, Sf, Af = drs.vla_scan(z, z, z, z, lambda0=4.0)
+    torch.cuda.synchronize()
+    eye = torch.eye(d, device="cuda") / 4.0
+    assert torch.count_nonzero(Sf) == 0 and torch.allclose(Af, eye.expand_as(Af))
+
+
+# --- failure path: a bounded wait that runs out latches a status, nothing hangs
+def test_timeout_is_reported_and_cleared():
+    rc = drs.lib().dr_debug_timeout_probe(1000, drs._stream_handle(torch.device("cuda")))
+    assert rc == drs.DR_OK
+    assert drs.poll_error() == drs.DR_ERR_TIMEOUT
+    assert drs.poll_error() == drs.DR_OK
+    # the context is still usable
+    x = torch.ones(4, device="cuda")
+    assert float(x.sum()) == 4.0
