@@ -11,21 +11,32 @@
 //     Y      = V - diag(gamma) K S0^T                           residual vs decayed state
 //     O      = diag(gamma) Q S0^T + (P T) Y
 //     S_C^T  = diag(gamma_C) S0^T + Khat^T Y,  Khat^T = K^T diag(gamma_C/gamma) T
-// (KDA: the decay sits inside the operands, K*gamma, Q*gamma and K/gamma per channel.)
+// (KDA: the decay sits inside the operands, K*gamma, Q*gamma and K/gamma per channel, and
+// Khat^T = diag(gamma_C) (K/gamma)^T T.)
 //
 // Contractions on tcgen05 (bf16 operands in 128-byte-swizzled shared memory, fp32
 // accumulators in tensor memory), one CTA per (b, h, slice of BV value channels):
 //   Gram   D_G  = [K;Q] K^T                M=128 N=64 K=128
-//   H      D_H  = K^T Ttilde               M=128 N=64 K=64   (A operand M/N-major)
-//   PT     D_PT = P T                      M=128 N=64 K=64
+//   PT     D_PT = P T                      M=128 N=64 K=64   (B read M/N-major)
+//   H      D_H  = K^T Ttilde               M=128 N=64 K=64   (A and B read M/N-major)
 //   MMA1   D1   = [K;Q] S0^T               M=128 N=BV K=128
 //   MMA2   D2   = [T;PT] Y                 M=128 N=BV K=64
 //   MMA3   S^T += Khat^T Y                 M=128 N=BV K=64   (fp32 state stays in TMEM)
-// The unit-lower solve runs on CUDA cores in fp32. q/k/v tiles arrive by TMA; rows past
-// T are zero-filled by the copy engine and masked in the gate arithmetic.
+// The unit-lower inverse (I + A)^{-1} is built on the CUDA cores: 16x16 diagonal blocks by
+// substitution in fp32, then the off-diagonal blocks by two levels of block products
+// (X21 = -X22 A21 X11) on tf32 mma.sync, whose 16-row tiles are below tcgen05's minimum M.
 //
-// This version runs the stages of a chunk one after another in a single warpgroup
-// (thread r <-> TMEM lane r); loads for the next chunks are in flight meanwhile.
+// Warp roles (384 threads):
+//   warp 0      TMA producer of K and Q tiles; beta and GDN gate scalars
+//   warp 1      chain MMA issuer (MMA1, MMA2, MMA3)
+//   warp 2      prep MMA issuer (Gram, PT, H)
+//   warp 3      tensor-memory allocation, then the TMA producer of V tiles
+//   warps 4-7   chain warpgroup: residual Y, output rows, carried state (TMEM lane = row)
+//   warps 8-11  prep warpgroup: gates, Gram epilogue, UT inverse, operand staging
+// The prep side runs up to one chunk ahead of the chain; the only serial dependency
+// between chunks is the state (MMA1 -> residual -> MMA3 -> state copy -> MMA1).
+// Every wait is bounded: on a timeout the status word is latched, the CTA-wide abort flag
+// is raised and all roles run to the end without waiting or issuing.
 #pragma once
 
 #include <cuda.h>
@@ -37,33 +48,37 @@ namespace drscan {
 
 constexpr int CK = 64;    // chunk length
 constexpr int CDK = 128;  // key dimension of the chunked kernel
+constexpr int CHUNK_THREADS = 384;
 
 template <int MODE, int BV>
 struct ChunkLayout {
     static constexpr bool kKda = MODE == DR_KDA;
-    static constexpr int NS = kKda ? 1 : 2;  // input stages
-    static constexpr int KQ_B = 32768;       // [K;Q] bf16: 2 panels x 128 rows x 128 B
-    static constexpr int KN_B = kKda ? 16384 : 0;
+    static constexpr bool kGdn = MODE == DR_GDN;
+    static constexpr int NS = 2;                          // K/Q stages
+    static constexpr int NSV = (kKda && BV == 128) ? 1 : 2;  // V stages
+    static constexpr int NP = (kKda && BV == 128) ? 1 : 2;   // prepared-operand slots
+    static constexpr int NKN = kKda ? 1 : 0;
+
+    static constexpr int KQ_B = 32768;  // [K;Q] bf16: 2 panels x 128 rows x 128 B
     static constexpr int V_B = CK * BV * 2;
-    static constexpr int GATE_B = kKda ? CK * CDK * 4 : 0;
+    static constexpr int SY_B = ((BV * 128 + 1023) / 1024) * 1024;
 
     static constexpr int KQ = 0;
-    static constexpr int KN = KQ + NS * KQ_B;        // KDA: K/gamma, 2 panels x 64 rows
-    static constexpr int TP = KN + NS * KN_B;        // [T; PT]: 128 rows x 64 cols
-    static constexpr int KH = TP + 16384;            // Khat^T: 128 rows (dk) x 64 cols (t)
-    static constexpr int PM = KH + 16384;            // P: rows 0-63 (rows 64-127 zero)
-    static constexpr int TT = PM + 16384;            // T^T: 64 rows x 64
-    static constexpr int TTS = TT + 8192;            // (diag(gamma_C/gamma) T)^T
-    static constexpr int SS = TTS + 8192;            // S bf16: 2 panels x BV rows
-    static constexpr int SY = SS + BV * 256;         // Y^T: BV rows x 64 (t)
-    static constexpr int V = SY + ((BV * 128 + 1023) / 1024) * 1024;
-    static constexpr int GATE = V + NS * V_B;        // KDA gate fp32 [64][128] (then g)
-    static constexpr int AM = kKda ? GATE : GATE + NS * GATE_B;  // A fp32 [64][68]
-    static constexpr int AM_B = CK * 68 * 4;
-    static constexpr int GV = kKda ? GATE + GATE_B : AM + AM_B;  // g, gamma / gamma_C
-    static constexpr int BAR = GV + 1024;
-    static constexpr int TOTAL = BAR + 128;
-    static_assert(!kKda || AM_B <= GATE_B, "A aliases the KDA gate buffer");
+    static constexpr int KN = KQ + NS * KQ_B;    // KDA: K/gamma, 2 panels x 64 rows
+    static constexpr int TP = KN + NKN * 16384;  // slot: [T; PT] 128 rows x 64
+    static constexpr int KH = TP + NP * 16384;   // slot: Khat^T 128 rows (dk) x 64 (t)
+    static constexpr int PM = KH + NP * 16384;   // P: rows 0-63, rows 64-127 zero
+    static constexpr int TTS = PM + 16384;       // GDN: diag(gamma_C/gamma) T, 64 rows
+    static constexpr int SS = TTS + (kGdn ? 8192 : 0);  // S bf16: 2 panels x BV rows
+    static constexpr int SY = SS + BV * 256;     // Y^T: BV rows x 64
+    static constexpr int V = SY + SY_B;          // V stages: 64 rows x BV bf16
+    static constexpr int AM = V + NSV * V_B;     // A, then X = (I+A)^{-1}: fp32 [64][68]
+    static constexpr int ZS = AM + CK * 68 * 4;  // block-product scratch: fp32 [32][36]
+    static constexpr int GAM = ZS + 32 * 36 * 4; // slot: gamma[64] + gamma_C (GDN), gamma_C[128] (KDA)
+    static constexpr int BG = GAM + NP * 1024;   // per stage: beta[64], GDN alpha[64]
+    static constexpr int PG = BG + NS * 512;     // prep-private: g[64], 1/gamma[64], gamma_C[128]
+    static constexpr int BAR = PG + 1024;
+    static constexpr int TOTAL = BAR + 256;
     static_assert(TOTAL + 1024 <= 232448, "shared memory budget");
 
     static constexpr int COL_G = 0;   // D_G, then D_PT
@@ -72,7 +87,25 @@ struct ChunkLayout {
     static constexpr int COL_D2 = 128 + BV;
     static constexpr int COL_S = 128 + 2 * BV;
     static constexpr int NCOLS = (128 + 3 * BV) <= 256 ? 256 : 512;
-    static constexpr uint32_t TX_BYTES = KQ_B + V_B + GATE_B;
+};
+
+// mbarrier indices inside the BAR block
+enum ChunkBar {
+    B_KQ_FULL = 0,    // [2]
+    B_KQ_EMPTY = 2,   // [2]
+    B_V_FULL = 4,     // [2]
+    B_V_EMPTY = 6,    // [2]
+    B_GO = 8,         // prep -> prep MMA: Gram operands ready, D_G free
+    B_GRAM = 9,       // Gram done
+    B_TREADY = 10,    // prep -> prep MMA: T staged
+    B_HDONE = 11,     // PT and H done
+    B_PREP = 12,      // [2] slot ready for the chain
+    B_SLOT_EMPTY = 14,  // [2] slot consumed by the chain
+    B_MMA1 = 16,
+    B_YREADY = 17,
+    B_MMA23 = 18,
+    B_STATE = 19,     // bf16 state copy ready for MMA1
+    B_COUNT = 20
 };
 
 // bf16 bits of 8 consecutive columns of a row, stored as one 16-byte swizzled chunk.
@@ -93,440 +126,654 @@ __device__ __forceinline__ float ld_bf16(const uint8_t* base, uint32_t off) {
     return __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + off));
 }
 
+__device__ __forceinline__ uint32_t tf32_bits(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return r;
+}
+
+// D(16x8, fp32) += A(16x8, tf32, row) * B(8x8, tf32, col). Fragments: lane = 4*g + tg;
+// A {(g,tg), (g+8,tg), (g,tg+4), (g+8,tg+4)}, B {(k=tg,n=g), (k=tg+4,n=g)},
+// D {(g,2tg), (g,2tg+1), (g+8,2tg), (g+8,2tg+1)}.
+__device__ __forceinline__ void mma_tf32(float* d, const uint32_t* a, const uint32_t* b) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+        "{%8,%9}, {%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b[0]), "r"(b[1]));
+}
+
+// A fragment of the 16x8 tile at (r0, k0) of a row-major fp32 matrix with row stride ld.
+__device__ __forceinline__ void frag_a(uint32_t* a, const float* m, int ld, int r0, int k0,
+                                       int g, int tg) {
+    a[0] = tf32_bits(m[(r0 + g) * ld + k0 + tg]);
+    a[1] = tf32_bits(m[(r0 + g + 8) * ld + k0 + tg]);
+    a[2] = tf32_bits(m[(r0 + g) * ld + k0 + tg + 4]);
+    a[3] = tf32_bits(m[(r0 + g + 8) * ld + k0 + tg + 4]);
+}
+
+// B fragment of the 8x8 tile at (k0, n0) of a row-major (K rows) fp32 matrix.
+__device__ __forceinline__ void frag_b(uint32_t* b, const float* m, int ld, int k0, int n0, int g,
+                                       int tg) {
+    b[0] = tf32_bits(m[(k0 + tg) * ld + n0 + g]);
+    b[1] = tf32_bits(m[(k0 + tg + 4) * ld + n0 + g]);
+}
+
+// Store -D (16x8 fragment) at (r0, n0) of a row-major fp32 matrix.
+__device__ __forceinline__ void store_neg_frag(float* m, int ld, int r0, int n0, const float* d,
+                                               int g, int tg, float sign) {
+    m[(r0 + g) * ld + n0 + 2 * tg] = sign * d[0];
+    m[(r0 + g) * ld + n0 + 2 * tg + 1] = sign * d[1];
+    m[(r0 + g + 8) * ld + n0 + 2 * tg] = sign * d[2];
+    m[(r0 + g + 8) * ld + n0 + 2 * tg + 1] = sign * d[3];
+}
+
+__device__ __forceinline__ void prep_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+
 template <int MODE, int BV>
-__global__ void __launch_bounds__(128, 1) dr_chunked_kernel(
+__global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
-    const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmGate,
-    const float* __restrict__ beta, const float* __restrict__ gate, const float* __restrict__ S0,
+    const __grid_constant__ CUtensorMap tmV, const float* __restrict__ beta,
+    const float* __restrict__ gate, const float* __restrict__ S0,
     __nv_bfloat16* __restrict__ out, float* __restrict__ S_final, int T, int dv) {
     using L = ChunkLayout<MODE, BV>;
     constexpr bool kGdn = MODE == DR_GDN;
     constexpr bool kKda = MODE == DR_KDA;
-    constexpr int NS = L::NS;
+    constexpr int NS = L::NS, NSV = L::NSV, NP = L::NP;
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                              ~uintptr_t(1023));
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BAR);  // [0,NS): full, NS: mma
-    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::BAR + 64);
-    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + L::BAR + 80);
-    float* sG = reinterpret_cast<float*>(sm + L::GV);        // GDN: g[64]; KDA: gamma_C[128]
-    float* sGam = sG + 64;                                    // GDN: gamma[64], gamma_C at [64]
-    float* sA = reinterpret_cast<float*>(sm + L::AM);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + L::BAR);
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(sm + L::BAR + 8 * B_COUNT);
+    uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(sm + L::BAR + 8 * B_COUNT + 16);
+    auto bar = [&](int i) { return smem_u32(&bars[i]); };
 
     const int tid = threadIdx.x;
     const int warp = tid >> 5;
+    const int lane = tid & 31;
     const long bh = blockIdx.x;
     const int v0 = blockIdx.y * BV;
     const int nchunks = (T + CK - 1) / CK;
-    const uint32_t bar_mma = smem_u32(&bars[NS]);
 
     if (tid == 0) {
-        for (int s = 0; s < NS; ++s) mbar_init(smem_u32(&bars[s]), 1);
-        mbar_init(bar_mma, 1);
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(bar(B_KQ_FULL + s), 2);
+            mbar_init(bar(B_KQ_EMPTY + s), 2);
+            mbar_init(bar(B_V_FULL + s), 1);
+            mbar_init(bar(B_V_EMPTY + s), 64);
+            mbar_init(bar(B_PREP + s), 128);
+            mbar_init(bar(B_SLOT_EMPTY + s), 129);
+        }
+        mbar_init(bar(B_GO), 128);
+        mbar_init(bar(B_GRAM), 1);
+        mbar_init(bar(B_TREADY), 128);
+        mbar_init(bar(B_HDONE), 1);
+        mbar_init(bar(B_MMA1), 1);
+        mbar_init(bar(B_YREADY), 128);
+        mbar_init(bar(B_MMA23), 1);
+        mbar_init(bar(B_STATE), 128);
         *abort_flag = 0;
         mbar_init_fence();
-        tma_prefetch_desc(&tmK);
-        tma_prefetch_desc(&tmQ);
-        tma_prefetch_desc(&tmV);
-        if constexpr (kKda) tma_prefetch_desc(&tmGate);
     }
-    if (warp == 0) tmem_alloc(smem_u32(tmem_holder), L::NCOLS);
-    // P's rows 64-127 are never written: keep them zero.
-    for (int e = tid; e < 8192 / 16; e += 128)
+    if (warp == 3) tmem_alloc(smem_u32(tmem_holder), L::NCOLS);
+    // P's rows 64-127 feed an M=128 MMA whose upper half is discarded: keep them zero.
+    for (int e = tid; e < 8192 / 16; e += CHUNK_THREADS)
         reinterpret_cast<uint4*>(sm + L::PM + 8192)[e] = make_uint4(0, 0, 0, 0);
+    fence_async_smem();
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
-    const uint32_t trow = tmem + lane_base;  // this thread's TMEM lane
 
-    auto issue_loads = [&](int chunk, int s) {
-        const uint32_t full = smem_u32(&bars[s]);
-        mbar_arrive_expect_tx(full, L::TX_BYTES);
-        uint8_t* kq = sm + L::KQ + s * L::KQ_B;
-        const int t0 = chunk * CK;
-        for (int p = 0; p < 2; ++p) {
-            tma_load_3d(smem_u32(kq + p * 16384), &tmK, full, p * 64, t0, (int)bh);
-            tma_load_3d(smem_u32(kq + p * 16384 + 8192), &tmQ, full, p * 64, t0, (int)bh);
+    if (warp == 0) {
+        // ------------------------------------------------------------------ producer
+        if (lane == 0) {
+            tma_prefetch_desc(&tmK);
+            tma_prefetch_desc(&tmQ);
+            tma_prefetch_desc(&tmV);
         }
-        tma_load_3d(smem_u32(sm + L::V + s * L::V_B), &tmV, full, v0, t0, (int)bh);
-        if constexpr (kKda) tma_load_3d(smem_u32(sm + L::GATE), &tmGate, full, 0, t0, (int)bh);
-    };
-
-    if (tid == 0) {
-        for (int c = 0; c < NS && c < nchunks; ++c) issue_loads(c, c);
-    }
-
-    // ---- initial state: S^T row j (lane j = key channel) in TMEM, bf16 copy in smem
-    {
-        float sv[BV];
-        const float* src = S0 ? S0 + (bh * dv + v0) * (long)CDK + tid : nullptr;
-#pragma unroll
-        for (int v = 0; v < BV; ++v) sv[v] = src ? src[(long)v * CDK] : 0.f;
-#pragma unroll
-        for (int v = 0; v < BV; ++v) st_bf16(sm + L::SS, sw128_offset(v, tid, BV), sv[v]);
-#pragma unroll
-        for (int c16 = 0; c16 < BV; c16 += 16) tmem_st16(trow + L::COL_S + c16, sv + c16);
-        tmem_wait_st();
-    }
-    fence_async_smem();
-
-    // per-token scalars of the next chunk, prefetched into registers (threads 0..63)
-    float nb = 0.f, ng = 1.f;
-    if (tid < CK && tid < T) {
-        nb = beta[bh * T + tid];
-        if constexpr (kGdn) ng = gate[bh * T + tid];
-    }
-
-    uint32_t mma_phase = 0;
-    bool ok = true;
-    for (int c = 0; c < nchunks && ok; ++c) {
-        const int s = c % NS;
-        const int t0 = c * CK;
-        const int nvalid = min(CK, T - t0);
-        const float b_t = nb;  // beta of row t = tid (threads < 64)
-        const float a_t = ng;  // alpha of row t (GDN)
-        if (tid < CK) {
-            const int tn = t0 + CK + tid;
-            nb = 0.f;
-            ng = 1.f;
-            if (tn < T) {
-                nb = beta[bh * T + tn];
-                if constexpr (kGdn) ng = gate[bh * T + tn];
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % NS;
+            const int t0 = c * CK;
+            if (c >= NS) mbar_wait(bar(B_KQ_EMPTY + s), (uint32_t)(((c / NS) - 1) & 1), abort_flag);
+            float* bg = reinterpret_cast<float*>(sm + L::BG + s * 512);
+            for (int e = lane; e < CK; e += 32) {
+                const int t = t0 + e;
+                bg[e] = t < T ? beta[bh * T + t] : 0.f;
+                if constexpr (kGdn) bg[64 + e] = t < T ? gate[bh * T + t] : 1.f;
             }
-        }
-        uint8_t* kq = sm + L::KQ + s * L::KQ_B;
-        uint8_t* kn = sm + L::KN + s * L::KN_B;
-        const uint8_t* vt = sm + L::V + s * L::V_B;
-
-        if (!mbar_wait(smem_u32(&bars[s]), (uint32_t)((c / NS) & 1), abort_flag)) {
-            ok = false;
-            break;
-        }
-
-        // ---- gate prefix sums
-        if constexpr (kGdn) {
-            if (tid < CK) {
-                float x = (tid < nvalid) ? logf(a_t) : 0.f;
-#pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const float y = __shfl_up_sync(0xffffffffu, x, off);
-                    if ((tid & 31) >= off) x += y;
+            __syncwarp();
+            if (lane == 0) {
+                if (!*abort_flag) {
+                    uint8_t* kq = sm + L::KQ + s * L::KQ_B;
+                    mbar_arrive_expect_tx(bar(B_KQ_FULL + s), L::KQ_B);
+                    for (int p = 0; p < 2; ++p) {
+                        tma_load_3d(smem_u32(kq + p * 16384), &tmK, bar(B_KQ_FULL + s), p * 64, t0,
+                                    (int)bh);
+                        tma_load_3d(smem_u32(kq + p * 16384 + 8192), &tmQ, bar(B_KQ_FULL + s),
+                                    p * 64, t0, (int)bh);
+                    }
                 }
-                if (tid == 31) sG[200] = x;  // scratch: total of rows 0..31
-                sG[tid] = x;
+                mbar_arrive(bar(B_KQ_FULL + s));
             }
-            __syncthreads();
-            if (tid >= 32 && tid < CK) sG[tid] += sG[200];
-            __syncthreads();
-            if (tid < CK) sGam[tid] = expf(sG[tid]);
-            if (tid == 0) sGam[64] = expf(sG[CK - 1]);
-        } else if constexpr (kKda) {
-            // thread j owns key channel j: running log-decay over the chunk's rows; rewrite
-            // K and Q in place as K*gamma, Q*gamma and store K/gamma.
-            const float* gt = reinterpret_cast<const float*>(sm + L::GATE);
-            float run = 0.f;
-            for (int t = 0; t < CK; ++t) {
-                if (t < nvalid) run += logf(gt[t * CDK + tid]);
-                const float e = expf(run);
-                const float ei = expf(-run);
-                const uint32_t ok_ = sw128_offset(t, tid, 128);
-                const uint32_t oq = sw128_offset(64 + t, tid, 128);
-                const float kv = ld_bf16(kq, ok_);
-                st_bf16(kq, ok_, kv * e);
-                st_bf16(kq, oq, ld_bf16(kq, oq) * e);
-                st_bf16(kn, sw128_offset(t, tid, 64), kv * ei);
+        }
+    } else if (warp == 3) {
+        // ------------------------------------------------------------------ V producer
+        if (lane == 0) {
+            for (int c = 0; c < nchunks; ++c) {
+                const int sv = c % NSV;
+                if (c >= NSV)
+                    mbar_wait(bar(B_V_EMPTY + sv), (uint32_t)(((c / NSV) - 1) & 1), abort_flag);
+                if (!*abort_flag) {
+                    mbar_arrive_expect_tx(bar(B_V_FULL + sv), L::V_B);
+                    tma_load_3d(smem_u32(sm + L::V + sv * L::V_B), &tmV, bar(B_V_FULL + sv), v0,
+                                c * CK, (int)bh);
+                }
             }
-            sG[tid] = expf(run);  // gamma_C per key channel
-            fence_async_smem();
         }
-        __syncthreads();
-
-        // ---- decay the carried state: S^T row j *= gamma_C (before MMA3 accumulates)
-        if constexpr (MODE != DR_DELTANET) {
-            const float gC = kKda ? sG[tid] : sGam[64];
-            float sv[BV];
+    } else if (warp == 1) {
+        // ------------------------------------------------------------------ chain MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t id1 = idesc_bf16(128, BV, 0, 0);
+            for (int c = 0; c < nchunks; ++c) {
+                const int s = c % NS, p = c % NP;
+                uint8_t* kq = sm + L::KQ + s * L::KQ_B;
+                mbar_wait(bar(B_PREP + p), (uint32_t)((c / NP) & 1), abort_flag);
+                mbar_wait(bar(B_STATE), (uint32_t)(c & 1), abort_flag);
+                tc_fence_after();
+                if (!*abort_flag) {
 #pragma unroll
-            for (int c16 = 0; c16 < BV; c16 += 16) tmem_ld16(trow + L::COL_S + c16, sv + c16);
-            tmem_wait_ld();
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const int pn = kk >> 2, ko = (kk & 3) * 32;
+                        tc_mma_bf16(tmem + L::COL_D1,
+                                    smem_desc_sw128(smem_u32(kq + pn * 16384 + ko), 16, 1024),
+                                    smem_desc_sw128(smem_u32(sm + L::SS + pn * (BV * 128) + ko), 16,
+                                                    1024),
+                                    id1, kk > 0);
+                    }
+                    tc_commit(bar(B_MMA1));
+                    tc_commit(bar(B_KQ_EMPTY + s));
+                }
+                mbar_wait(bar(B_YREADY), (uint32_t)(c & 1), abort_flag);
+                tc_fence_after();
+                if (!*abort_flag) {
+                    const uint8_t* tp = sm + L::TP + p * 16384;
+                    const uint8_t* kh = sm + L::KH + p * 16384;
 #pragma unroll
-            for (int v = 0; v < BV; ++v) sv[v] *= gC;
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc_mma_bf16(tmem + L::COL_D2,
+                                    smem_desc_sw128(smem_u32(tp + kk * 32), 16, 1024),
+                                    smem_desc_sw128(smem_u32(sm + L::SY + kk * 32), 16, 1024), id1,
+                                    kk > 0);
 #pragma unroll
-            for (int c16 = 0; c16 < BV; c16 += 16) tmem_st16(trow + L::COL_S + c16, sv + c16);
-            tmem_wait_st();
-        }
-
-        // ---- Gram: D_G = [K;Q] K^T  (KDA: [K*g; Q*g] (K/g)^T)
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        if (tid == 0) {
-            constexpr uint32_t idesc = idesc_bf16(128, 64, 0, 0);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const int p = kk >> 2, ko = (kk & 3) * 32;
-                const uint64_t a = smem_desc_sw128(smem_u32(kq + p * 16384 + ko), 16, 1024);
-                const uint64_t b = kKda ? smem_desc_sw128(smem_u32(kn + p * 8192 + ko), 16, 1024)
-                                        : a;
-                tc_mma_bf16(tmem + L::COL_G, a, b, idesc, kk > 0);
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc_mma_bf16(tmem + L::COL_S,
+                                    smem_desc_sw128(smem_u32(kh + kk * 32), 16, 1024),
+                                    smem_desc_sw128(smem_u32(sm + L::SY + kk * 32), 16, 1024), id1,
+                                    1);
+                    tc_commit(bar(B_MMA23));
+                    tc_commit(bar(B_SLOT_EMPTY + p));
+                }
             }
-            tc_commit(bar_mma);
         }
-        if (!mbar_wait(bar_mma, mma_phase, abort_flag)) {
-            ok = false;
-            break;
+    } else if (warp == 2) {
+        // ------------------------------------------------------------------ prep MMA issuer
+        if (lane == 0) {
+            constexpr uint32_t idg = idesc_bf16(128, 64, 0, 0);
+            constexpr uint32_t idp = idesc_bf16(128, 64, 0, 1);
+            constexpr uint32_t idh = idesc_bf16(128, 64, 1, 1);
+            for (int c = 0; c < nchunks; ++c) {
+                const int s = c % NS, p = c % NP;
+                uint8_t* kq = sm + L::KQ + s * L::KQ_B;
+                uint8_t* kn = sm + L::KN;
+                mbar_wait(bar(B_GO), (uint32_t)(c & 1), abort_flag);
+                tc_fence_after();
+                if (!*abort_flag) {
+#pragma unroll
+                    for (int kk = 0; kk < 8; ++kk) {
+                        const int pn = kk >> 2, ko = (kk & 3) * 32;
+                        const uint64_t a = smem_desc_sw128(smem_u32(kq + pn * 16384 + ko), 16, 1024);
+                        const uint64_t b =
+                            kKda ? smem_desc_sw128(smem_u32(kn + pn * 8192 + ko), 16, 1024) : a;
+                        tc_mma_bf16(tmem + L::COL_G, a, b, idg, kk > 0);
+                    }
+                    tc_commit(bar(B_GRAM));
+                }
+                mbar_wait(bar(B_TREADY), (uint32_t)(c & 1), abort_flag);
+                tc_fence_after();
+                if (!*abort_flag) {
+                    const uint8_t* tp = sm + L::TP + p * 16384;
+                    // PT = P T: B = T read M/N-major from the slot's rows 0-63
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc_mma_bf16(tmem + L::COL_G,
+                                    smem_desc_sw128(smem_u32(sm + L::PM + kk * 32), 16, 1024),
+                                    smem_desc_sw128(smem_u32(tp + kk * 2048), 1024, 1024), idp,
+                                    kk > 0);
+                    // H: A = K^T (KDA: (K/g)^T) M/N-major, B = Ttilde (or T) M/N-major
+                    const uint8_t* bt = kGdn ? sm + L::TTS : tp;
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk) {
+                        const uint64_t a =
+                            kKda ? smem_desc_sw128(smem_u32(kn + kk * 2048), 8192, 1024)
+                                 : smem_desc_sw128(smem_u32(kq + kk * 2048), 16384, 1024);
+                        tc_mma_bf16(tmem + L::COL_H, a,
+                                    smem_desc_sw128(smem_u32(bt + kk * 2048), 1024, 1024), idh,
+                                    kk > 0);
+                    }
+                    tc_commit(bar(B_HDONE));
+                    tc_commit(bar(B_KQ_EMPTY + s));
+                }
+            }
         }
-        mma_phase ^= 1;
-        tc_fence_after();
-
-        // ---- Gram epilogue: A (fp32, rows 0-63) and P (bf16 operand)
+    } else if (warp >= 4 && warp < 8) {
+        // ------------------------------------------------------------------ chain warpgroup
+        const int r = tid - 128;  // TMEM lane: value row t (Y, O) or key channel j (state)
+        const uint32_t trow = tmem + ((uint32_t)(r & ~31) << 16);
         {
-            float gr[64];
-#pragma unroll
-            for (int c16 = 0; c16 < 64; c16 += 16) tmem_ld16(trow + L::COL_G + c16, gr + c16);
-            tmem_wait_ld();
-            const int t = tid & 63;
-            const float gt = kGdn ? sG[t] : 0.f;
-            if (tid < 64) {
-#pragma unroll
-                for (int i = 0; i < 64; ++i) {
-                    float a = 0.f;
-                    if (i < t) a = b_t * gr[i] * (kGdn ? expf(gt - sG[i]) : 1.f);
-                    gr[i] = a;
-                }
-#pragma unroll
-                for (int i = 0; i < 64; i += 4)
-                    *reinterpret_cast<float4*>(sA + t * 68 + i) =
-                        make_float4(gr[i], gr[i + 1], gr[i + 2], gr[i + 3]);
-            } else {
-#pragma unroll
-                for (int i = 0; i < 64; ++i) {
-                    float p = 0.f;
-                    if (i <= t) p = gr[i] * (kGdn ? expf(gt - sG[i]) : 1.f);
-                    gr[i] = p;
-                }
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) st_row_chunk(sm + L::PM, t, ch, gr + ch * 8);
-            }
-        }
-        __syncthreads();
-
-        // ---- UT solve on CUDA cores: column j of X = (I + A)^{-1}; T = X diag(beta)
-        if (tid < 64) {
-            const int j = tid;
-            float x[64];
-#pragma unroll
-            for (int t = 0; t < 64; ++t) {
-                float acc = (t == j) ? 1.f : 0.f;
-#pragma unroll
-                for (int i = 0; i < t; i += 4) {
-                    const float4 a4 = *reinterpret_cast<const float4*>(sA + t * 68 + i);
-                    acc = fmaf(-a4.x, x[i], acc);
-                    if (i + 1 < t) acc = fmaf(-a4.y, x[i + 1], acc);
-                    if (i + 2 < t) acc = fmaf(-a4.z, x[i + 2], acc);
-                    if (i + 3 < t) acc = fmaf(-a4.w, x[i + 3], acc);
-                }
-                x[t] = acc;
-            }
-#pragma unroll
-            for (int t = 0; t < 64; ++t) x[t] *= b_t;  // column j scaled by beta_j
-            // [T; PT] rows 0-63 (row t, column j)
-#pragma unroll
-            for (int t = 0; t < 64; ++t) st_bf16(sm + L::TP, sw128_offset(t, j, 128), x[t]);
-            // T^T row j
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) st_row_chunk(sm + L::TT, j, ch, x + ch * 8);
-            if constexpr (kGdn) {
-                const float gC = sGam[64];
-#pragma unroll
-                for (int t = 0; t < 64; ++t) x[t] *= gC / sGam[t];
-            }
-            if constexpr (!kKda) {
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) st_row_chunk(sm + L::TTS, j, ch, x + ch * 8);
-            }
-        }
-        fence_async_smem();
-        __syncthreads();
-
-        // ---- H: Khat^T = K^T Ttilde (KDA: (K/g)^T T); PT = P T
-        if (tid == 0) {
-            constexpr uint32_t idesc_h = idesc_bf16(128, 64, 1, 0);
-            constexpr uint32_t idesc_p = idesc_bf16(128, 64, 0, 0);
-            const uint8_t* bt = sm + (kKda ? L::TT : L::TTS);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t a = kKda ? smem_desc_sw128(smem_u32(kn + kk * 2048), 8192, 1024)
-                                        : smem_desc_sw128(smem_u32(kq + kk * 2048), 16384, 1024);
-                const uint64_t b = smem_desc_sw128(smem_u32(bt + kk * 32), 16, 1024);
-                tc_mma_bf16(tmem + L::COL_H, a, b, idesc_h, kk > 0);
-            }
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t a = smem_desc_sw128(smem_u32(sm + L::PM + kk * 32), 16, 1024);
-                const uint64_t b = smem_desc_sw128(smem_u32(sm + L::TT + kk * 32), 16, 1024);
-                tc_mma_bf16(tmem + L::COL_G, a, b, idesc_p, kk > 0);
-            }
-            tc_commit(bar_mma);
-        }
-        if (!mbar_wait(bar_mma, mma_phase, abort_flag)) {
-            ok = false;
-            break;
-        }
-        mma_phase ^= 1;
-        tc_fence_after();
-        {
-            float h[64];
-#pragma unroll
-            for (int c16 = 0; c16 < 64; c16 += 16) tmem_ld16(trow + L::COL_H + c16, h + c16);
-            tmem_wait_ld();
-            if constexpr (kKda) {
-                const float gC = sG[tid];
-#pragma unroll
-                for (int i = 0; i < 64; ++i) h[i] *= gC;
-            }
-#pragma unroll
-            for (int ch = 0; ch < 8; ++ch) st_row_chunk(sm + L::KH, tid, ch, h + ch * 8);
-            if (tid < 64) {
-#pragma unroll
-                for (int c16 = 0; c16 < 64; c16 += 16) tmem_ld16(trow + L::COL_G + c16, h + c16);
-                tmem_wait_ld();
-#pragma unroll
-                for (int ch = 0; ch < 8; ++ch) st_row_chunk(sm + L::TP, 64 + tid, ch, h + ch * 8);
-            }
-        }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-
-        // ---- MMA1: D1 = [K;Q] S0^T (KDA: [K*g; Q*g] S0^T)
-        if (tid == 0) {
-            constexpr uint32_t idesc = idesc_bf16(128, BV, 0, 0);
-#pragma unroll
-            for (int kk = 0; kk < 8; ++kk) {
-                const int p = kk >> 2, ko = (kk & 3) * 32;
-                const uint64_t a = smem_desc_sw128(smem_u32(kq + p * 16384 + ko), 16, 1024);
-                const uint64_t b =
-                    smem_desc_sw128(smem_u32(sm + L::SS + p * (BV * 128) + ko), 16, 1024);
-                tc_mma_bf16(tmem + L::COL_D1, a, b, idesc, kk > 0);
-            }
-            tc_commit(bar_mma);
-        }
-        if (!mbar_wait(bar_mma, mma_phase, abort_flag)) {
-            ok = false;
-            break;
-        }
-        mma_phase ^= 1;
-        tc_fence_after();
-
-        // ---- residual Y = V - gamma (K S0^T), stored as the B operand Y^T
-        if (tid < 64) {
-            const int t = tid;
-            const float gt = kGdn ? sGam[t] : 1.f;
-            float xr[BV];
-#pragma unroll
-            for (int c16 = 0; c16 < BV; c16 += 16) tmem_ld16(trow + L::COL_D1 + c16, xr + c16);
-            tmem_wait_ld();
-            const uint4* vrow = reinterpret_cast<const uint4*>(vt + t * BV * 2);
-#pragma unroll
-            for (int c8 = 0; c8 < BV / 8; ++c8) {
-                const uint4 w = vrow[c8];
-                const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&w);
-#pragma unroll
-                for (int e = 0; e < 8; ++e) {
-                    const int v = c8 * 8 + e;
-                    st_bf16(sm + L::SY, sw128_offset(v, t, BV),
-                            __bfloat162float(hv[e]) - gt * xr[v]);
-                }
-            }
-        }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-
-        // ---- MMA2: D2 = [T; PT] Y;  MMA3: S^T += Khat^T Y
-        if (tid == 0) {
-            constexpr uint32_t idesc = idesc_bf16(128, BV, 0, 0);
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t a = smem_desc_sw128(smem_u32(sm + L::TP + kk * 32), 16, 1024);
-                const uint64_t b = smem_desc_sw128(smem_u32(sm + L::SY + kk * 32), 16, 1024);
-                tc_mma_bf16(tmem + L::COL_D2, a, b, idesc, kk > 0);
-            }
-#pragma unroll
-            for (int kk = 0; kk < 4; ++kk) {
-                const uint64_t a = smem_desc_sw128(smem_u32(sm + L::KH + kk * 32), 16, 1024);
-                const uint64_t b = smem_desc_sw128(smem_u32(sm + L::SY + kk * 32), 16, 1024);
-                tc_mma_bf16(tmem + L::COL_S, a, b, idesc, 1);
-            }
-            tc_commit(bar_mma);
-        }
-        if (!mbar_wait(bar_mma, mma_phase, abort_flag)) {
-            ok = false;
-            break;
-        }
-        mma_phase ^= 1;
-        tc_fence_after();
-
-        // ---- output rows: O = gamma (Q S0^T) + PT Y  (warps 2-3 own rows 64-127)
-        if (tid >= 64) {
-            const int t = tid - 64;
-            const float gt = kGdn ? sGam[t] : 1.f;
+            const float* src = S0 ? S0 + (bh * dv + v0) * (long)CDK + r : nullptr;
 #pragma unroll
             for (int c16 = 0; c16 < BV; c16 += 16) {
-                float z[16], d[16];
-                tmem_ld16(trow + L::COL_D1 + c16, z);
-                tmem_ld16(trow + L::COL_D2 + c16, d);
-                tmem_wait_ld();
-                if (t < nvalid) {
-                    uint4 w[2];
-                    uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+                float sv[16];
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        wp[e] = pack_bf16(fmaf(gt, z[2 * e], d[2 * e]),
-                                          fmaf(gt, z[2 * e + 1], d[2 * e + 1]));
-                    uint4* dst = reinterpret_cast<uint4*>(out + (bh * T + t0 + t) * (long)dv + v0 +
-                                                          c16);
-                    dst[0] = w[0];
-                    dst[1] = w[1];
+                for (int v = 0; v < 16; ++v) sv[v] = src ? src[(long)(c16 + v) * CDK] : 0.f;
+#pragma unroll
+                for (int v = 0; v < 16; ++v)
+                    st_bf16(sm + L::SS, sw128_offset(c16 + v, r, BV), sv[v]);
+                tmem_st16(trow + L::COL_S + c16, sv);
+            }
+            tmem_wait_st();
+            fence_async_smem();
+            mbar_arrive(bar(B_STATE));
+        }
+        auto prescale = [&](int c) {  // S^T *= gamma_C of chunk c, before MMA3(c)
+            if constexpr (MODE != DR_DELTANET) {
+                const int p = c % NP;
+                mbar_wait(bar(B_PREP + p), (uint32_t)((c / NP) & 1), abort_flag);
+                const float* gam = reinterpret_cast<const float*>(sm + L::GAM + p * 1024);
+                const float gC = kKda ? gam[r] : gam[64];
+#pragma unroll
+                for (int c16 = 0; c16 < BV; c16 += 16) {
+                    float sv[16];
+                    tmem_ld16(trow + L::COL_S + c16, sv);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int v = 0; v < 16; ++v) sv[v] *= gC;
+                    tmem_st16(trow + L::COL_S + c16, sv);
+                }
+                tmem_wait_st();
+            }
+        };
+        if (nchunks > 0) prescale(0);
+        for (int c = 0; c < nchunks; ++c) {
+            const int p = c % NP, svi = c % NSV;
+            const int t0 = c * CK;
+            const int nvalid = min(CK, T - t0);
+            const float* gam = reinterpret_cast<const float*>(sm + L::GAM + p * 1024);
+            mbar_wait(bar(B_MMA1), (uint32_t)(c & 1), abort_flag);
+            tc_fence_after();
+            if (r < 64) {
+                // residual Y = V - gamma_t (S0 k_t), stored as the B operand Y^T
+                mbar_wait(bar(B_V_FULL + svi), (uint32_t)((c / NSV) & 1), abort_flag);
+                const float gt = kGdn ? gam[r] : 1.f;
+                const uint4* vrow =
+                    reinterpret_cast<const uint4*>(sm + L::V + svi * L::V_B + r * BV * 2);
+#pragma unroll
+                for (int c16 = 0; c16 < BV; c16 += 16) {
+                    float x[16];
+                    tmem_ld16(trow + L::COL_D1 + c16, x);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int h = 0; h < 2; ++h) {
+                        const uint4 w = vrow[c16 / 8 + h];
+                        const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&w);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) {
+                            const int v = c16 + h * 8 + e;
+                            st_bf16(sm + L::SY, sw128_offset(v, r, BV),
+                                    fmaf(-gt, x[h * 8 + e], __bfloat162float(hv[e])));
+                        }
+                    }
+                }
+                mbar_arrive(bar(B_V_EMPTY + svi));
+            }
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar(B_YREADY));
+
+            mbar_wait(bar(B_MMA23), (uint32_t)(c & 1), abort_flag);
+            tc_fence_after();
+            if (r >= 64) {
+                // output rows: O = gamma_t (S0 q_t) + (P T Y)_t
+                const int t = r - 64;
+                const float gt = kGdn ? gam[t] : 1.f;
+#pragma unroll
+                for (int c16 = 0; c16 < BV; c16 += 16) {
+                    float z[16], d[16];
+                    tmem_ld16(trow + L::COL_D1 + c16, z);
+                    tmem_ld16(trow + L::COL_D2 + c16, d);
+                    tmem_wait_ld();
+                    if (t < nvalid) {
+                        uint4 w[2];
+                        uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e)
+                            wp[e] = pack_bf16(fmaf(gt, z[2 * e], d[2 * e]),
+                                              fmaf(gt, z[2 * e + 1], d[2 * e + 1]));
+                        uint4* dst = reinterpret_cast<uint4*>(out + (bh * T + t0 + t) * (long)dv +
+                                                              v0 + c16);
+                        dst[0] = w[0];
+                        dst[1] = w[1];
+                    }
                 }
             }
-        }
-        // ---- carried state: bf16 copy for the next MMA1, fp32 S_final after the last chunk
-        {
-            float sv[BV];
+            // carried state: bf16 copy for the next MMA1; fp32 S_final after the last chunk
+            {
+                float* dst = (c == nchunks - 1 && S_final)
+                                 ? S_final + (bh * dv + v0) * (long)CDK + r
+                                 : nullptr;
 #pragma unroll
-            for (int c16 = 0; c16 < BV; c16 += 16) tmem_ld16(trow + L::COL_S + c16, sv + c16);
-            tmem_wait_ld();
+                for (int c16 = 0; c16 < BV; c16 += 16) {
+                    float sv[16];
+                    tmem_ld16(trow + L::COL_S + c16, sv);
+                    tmem_wait_ld();
 #pragma unroll
-            for (int v = 0; v < BV; ++v) st_bf16(sm + L::SS, sw128_offset(v, tid, BV), sv[v]);
-            if (c == nchunks - 1 && S_final) {
-                float* dst = S_final + (bh * dv + v0) * (long)CDK + tid;
+                    for (int v = 0; v < 16; ++v)
+                        st_bf16(sm + L::SS, sw128_offset(c16 + v, r, BV), sv[v]);
+                    if (dst) {
 #pragma unroll
-                for (int v = 0; v < BV; ++v) dst[(long)v * CDK] = sv[v];
+                        for (int v = 0; v < 16; ++v) dst[(long)(c16 + v) * CDK] = sv[v];
+                    }
+                }
             }
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar(B_STATE));
+            mbar_arrive(bar(B_SLOT_EMPTY + p));
+            if (c + 1 < nchunks) prescale(c + 1);
         }
-        fence_async_smem();
-        tc_fence_before();
-        __syncthreads();
-        tc_fence_after();
-        if (tid == 0 && c + NS < nchunks) issue_loads(c + NS, s);
+    } else if (warp >= 8) {
+        // ------------------------------------------------------------------ prep warpgroup
+        const int r = tid - 256;
+        const uint32_t trow = tmem + ((uint32_t)(r & ~31) << 16);
+        const int wq = r >> 5, g8 = lane >> 2, tg = lane & 3;
+        float* pg = reinterpret_cast<float*>(sm + L::PG);  // g[64] | 1/gamma[64] | gamma_C[128]
+        float* sA = reinterpret_cast<float*>(sm + L::AM);
+        float* sZ = reinterpret_cast<float*>(sm + L::ZS);
+        float gpf[kKda ? CK : 1];  // KDA: next chunk's alpha for channel r, prefetched
+        if constexpr (kKda) {
+#pragma unroll
+            for (int t = 0; t < CK; ++t) gpf[t] = t < T ? gate[(bh * T + t) * (long)CDK + r] : 1.f;
+        }
+        for (int c = 0; c < nchunks; ++c) {
+            const int s = c % NS, p = c % NP;
+            const int t0 = c * CK;
+            const int nvalid = min(CK, T - t0);
+            uint8_t* kq = sm + L::KQ + s * L::KQ_B;
+            const float* bg = reinterpret_cast<const float*>(sm + L::BG + s * 512);
+            mbar_wait(bar(B_KQ_FULL + s), (uint32_t)((c / NS) & 1), abort_flag);
+
+            // ---- 1. gates
+            bool fact = true;  // GDN: exp(g_t - g_i) = gamma_t * (1/gamma_i) is safe
+            if constexpr (kGdn) {
+                float x = 0.f;
+                if (r < 64) {
+                    x = (r < nvalid) ? __logf(bg[64 + r]) : 0.f;
+#pragma unroll
+                    for (int off = 1; off < 32; off <<= 1) {
+                        const float y = __shfl_up_sync(0xffffffffu, x, off);
+                        if (lane >= off) x += y;
+                    }
+                    pg[r] = x;
+                }
+                prep_sync();
+                if (r >= 32 && r < 64) {
+                    x += pg[31];
+                    pg[r] = x;
+                }
+                prep_sync();
+                if (r < 64) pg[64 + r] = __expf(-x);
+                prep_sync();
+                fact = pg[63] > -80.f;
+            } else if constexpr (kKda) {
+                // channel r: running product of alpha; rewrite K and Q in place as K*gamma,
+                // Q*gamma and store K/gamma
+                uint8_t* kn = sm + L::KN;
+                float run = 1.f;
+#pragma unroll
+                for (int t = 0; t < CK; ++t) {
+                    if (t < nvalid) run *= gpf[t];
+                    const float inv = __frcp_rn(run);
+                    const uint32_t ok_ = sw128_offset(t, r, 128);
+                    const uint32_t oq = sw128_offset(64 + t, r, 128);
+                    const float kv = ld_bf16(kq, ok_);
+                    st_bf16(kq, ok_, kv * run);
+                    st_bf16(kq, oq, ld_bf16(kq, oq) * run);
+                    st_bf16(kn, sw128_offset(t, r, 64), kv * inv);
+                }
+                pg[128 + r] = run;  // gamma_C for channel r
+#pragma unroll
+                for (int t = 0; t < CK; ++t) {
+                    const int tn = t0 + CK + t;
+                    gpf[t] = tn < T ? gate[(bh * T + tn) * (long)CDK + r] : 1.f;
+                }
+                fence_async_smem();
+            }
+            tc_fence_before();
+            mbar_arrive(bar(B_GO));
+
+            // ---- 2. Gram epilogue: A (fp32, rows 0-63) and P (bf16, rows 0-63 of PM)
+            mbar_wait(bar(B_GRAM), (uint32_t)(c & 1), abort_flag);
+            tc_fence_after();
+            {
+                const int t = r & 63;
+                float rowf = (r < 64) ? bg[t] : 1.f;  // beta_t on A rows
+                float gt = 0.f;
+                if constexpr (kGdn) {
+                    gt = pg[t];
+                    if (fact) rowf *= __expf(gt);
+                }
+#pragma unroll
+                for (int c16 = 0; c16 < 64; c16 += 16) {
+                    float gr[16];
+                    tmem_ld16(trow + L::COL_G + c16, gr);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int e = 0; e < 16; ++e) {
+                        const int i = c16 + e;
+                        float dec = 1.f;
+                        if constexpr (kGdn)
+                            dec = fact ? pg[64 + i] : __expf(fminf(gt - pg[i], 0.f));
+                        const bool keep = (r < 64) ? (i < t) : (i <= t);
+                        gr[e] = keep ? rowf * gr[e] * dec : 0.f;
+                    }
+                    if (r < 64) {
+#pragma unroll
+                        for (int e = 0; e < 16; e += 4)
+                            *reinterpret_cast<float4*>(sA + t * 68 + c16 + e) =
+                                make_float4(gr[e], gr[e + 1], gr[e + 2], gr[e + 3]);
+                    } else {
+                        st_row_chunk(sm + L::PM, t, c16 / 8, gr);
+                        st_row_chunk(sm + L::PM, t, c16 / 8 + 1, gr + 8);
+                    }
+                }
+            }
+            prep_sync();
+
+            // ---- 3. X = (I + A)^{-1}, in place in sA
+            float xcol[16];
+            if (r < 64) {  // diagonal 16x16 blocks, one column per thread
+                const int b = r >> 4, cc = r & 15;
+#pragma unroll
+                for (int t = 0; t < 16; ++t) xcol[t] = (t == cc) ? 1.f : 0.f;
+#pragma unroll
+                for (int i = 0; i < 16; ++i)
+#pragma unroll
+                    for (int t = i + 1; t < 16; ++t)
+                        xcol[t] = fmaf(-sA[(16 * b + t) * 68 + 16 * b + i], xcol[i], xcol[t]);
+            }
+            prep_sync();
+            if (r < 64) {
+                const int b = r >> 4, cc = r & 15;
+#pragma unroll
+                for (int t = 0; t < 16; ++t) sA[(16 * b + t) * 68 + 16 * b + cc] = xcol[t];
+            }
+            prep_sync();
+            if (wq < 2) {  // X(b+1,b) = -X(b+1,b+1) A(b+1,b) X(b,b) for b = 0, 2
+                const int b0 = 32 * wq, b1 = b0 + 16;
+                float* z = sZ + wq * 16 * 20;
+                float acc[2][4] = {};
+#pragma unroll
+                for (int kk = 0; kk < 16; kk += 8) {
+                    uint32_t a[4], bb[2];
+                    frag_a(a, sA, 68, b1, b0 + kk, g8, tg);
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        frag_b(bb, sA, 68, b0 + kk, b0 + 8 * nt, g8, tg);
+                        mma_tf32(acc[nt], a, bb);
+                    }
+                }
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt) store_neg_frag(z, 20, 0, 8 * nt, acc[nt], g8, tg, 1.f);
+                __syncwarp();
+                float acc2[2][4] = {};
+#pragma unroll
+                for (int kk = 0; kk < 16; kk += 8) {
+                    uint32_t a[4], bb[2];
+                    frag_a(a, sA, 68, b1, b1 + kk, g8, tg);
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        frag_b(bb, z, 20, kk, 8 * nt, g8, tg);
+                        mma_tf32(acc2[nt], a, bb);
+                    }
+                }
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+                    store_neg_frag(sA, 68, b1, b0 + 8 * nt, acc2[nt], g8, tg, -1.f);
+            }
+            prep_sync();
+            {  // X[32:64, 0:32] = -X[32:64, 32:64] A[32:64, 0:32] X[0:32, 0:32]
+                const int m0 = 32 + 16 * (wq >> 1), n0 = 16 * (wq & 1);
+                float acc[2][4] = {};
+#pragma unroll
+                for (int kk = 0; kk < 32; kk += 8) {
+                    uint32_t a[4], bb[2];
+                    frag_a(a, sA, 68, m0, kk, g8, tg);
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        frag_b(bb, sA, 68, kk, n0 + 8 * nt, g8, tg);
+                        mma_tf32(acc[nt], a, bb);
+                    }
+                }
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+                    store_neg_frag(sZ, 36, m0 - 32, n0 + 8 * nt, acc[nt], g8, tg, 1.f);
+                prep_sync();
+                float acc2[2][4] = {};
+#pragma unroll
+                for (int kk = 0; kk < 32; kk += 8) {
+                    uint32_t a[4], bb[2];
+                    frag_a(a, sA, 68, m0, 32 + kk, g8, tg);
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt) {
+                        frag_b(bb, sZ, 36, kk, n0 + 8 * nt, g8, tg);
+                        mma_tf32(acc2[nt], a, bb);
+                    }
+                }
+#pragma unroll
+                for (int nt = 0; nt < 2; ++nt)
+                    store_neg_frag(sA, 68, m0, n0 + 8 * nt, acc2[nt], g8, tg, -1.f);
+            }
+            prep_sync();
+
+            // ---- 4. stage T = X diag(beta) into the slot (and Ttilde for GDN's H)
+            if (c >= NP)
+                mbar_wait(bar(B_SLOT_EMPTY + p), (uint32_t)(((c / NP) - 1) & 1), abort_flag);
+            uint8_t* tp = sm + L::TP + p * 16384;
+            float* gam = reinterpret_cast<float*>(sm + L::GAM + p * 1024);
+            {
+                const int t = r & 63;
+                float scale = 1.f;
+                uint8_t* dst = tp;
+                if (r >= 64) {
+                    if constexpr (kGdn) {
+                        scale = __expf(pg[63] - pg[t]);  // gamma_C / gamma_t
+                        dst = sm + L::TTS;
+                    } else {
+                        dst = nullptr;
+                    }
+                }
+                if (dst) {
+#pragma unroll
+                    for (int ch = 0; ch < 8; ++ch) {
+                        const float4 xa = *reinterpret_cast<const float4*>(sA + t * 68 + ch * 8);
+                        const float4 xb = *reinterpret_cast<const float4*>(sA + t * 68 + ch * 8 + 4);
+                        const float4 ba = *reinterpret_cast<const float4*>(bg + ch * 8);
+                        const float4 bb = *reinterpret_cast<const float4*>(bg + ch * 8 + 4);
+                        const float row[8] = {xa.x * ba.x * scale, xa.y * ba.y * scale,
+                                              xa.z * ba.z * scale, xa.w * ba.w * scale,
+                                              xb.x * bb.x * scale, xb.y * bb.y * scale,
+                                              xb.z * bb.z * scale, xb.w * bb.w * scale};
+                        st_row_chunk(dst, t, ch, row);
+                    }
+                }
+                if constexpr (kGdn) {
+                    if (r < 64) gam[r] = __expf(pg[r]);
+                    if (r == 64) gam[64] = __expf(pg[63]);
+                } else if constexpr (kKda) {
+                    gam[r] = pg[128 + r];
+                }
+            }
+            fence_async_smem();
+            mbar_arrive(bar(B_TREADY));
+
+            // ---- 5. PT rows -> slot rows 64-127; Khat^T -> slot
+            mbar_wait(bar(B_HDONE), (uint32_t)(c & 1), abort_flag);
+            tc_fence_after();
+            {
+                uint8_t* kh = sm + L::KH + p * 16384;
+                const float gC = kKda ? pg[128 + r] : 1.f;
+#pragma unroll
+                for (int c16 = 0; c16 < 64; c16 += 16) {
+                    float h[16];
+                    tmem_ld16(trow + L::COL_H + c16, h);
+                    tmem_wait_ld();
+                    if constexpr (kKda) {
+#pragma unroll
+                        for (int e = 0; e < 16; ++e) h[e] *= gC;
+                    }
+                    st_row_chunk(kh, r, c16 / 8, h);
+                    st_row_chunk(kh, r, c16 / 8 + 1, h + 8);
+                }
+                if (r < 64) {
+#pragma unroll
+                    for (int c16 = 0; c16 < 64; c16 += 16) {
+                        float h[16];
+                        tmem_ld16(trow + L::COL_G + c16, h);
+                        tmem_wait_ld();
+                        st_row_chunk(tp, 64 + r, c16 / 8, h);
+                        st_row_chunk(tp, 64 + r, c16 / 8 + 1, h + 8);
+                    }
+                }
+            }
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar(B_PREP + p));
+        }
     }
 
-    if (!ok && tid == 0) {
-        // give outstanding copies and MMAs a bounded chance to land before TMEM is freed
+    tc_fence_before();
+    __syncthreads();
+    if (*abort_flag && tid == 0) {
+        // give copies and MMAs issued before the abort a bounded chance to land
         const uint64_t t0 = global_timer_ns();
         while (global_timer_ns() - t0 < 50000000ull) {
         }
     }
-    tc_fence_before();
     __syncthreads();
     tc_fence_after();
-    if (warp == 0) tmem_dealloc(tmem, L::NCOLS);
+    if (warp == 3) tmem_dealloc(tmem, L::NCOLS);
 }
 
 // ---------------------------------------------------------------------------------------
@@ -571,14 +818,10 @@ int launch_chunked_bv(const void* q, const void* k, const void* v, const float* 
                       const float* gate, const float* S0, void* out, float* S_final, int BH, int T,
                       int dv, cudaStream_t stream) {
     using L = ChunkLayout<MODE, BV>;
-    CUtensorMap mk, mq, mv, mg;
+    CUtensorMap mk, mq, mv;
     if (!make_map_3d(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, BH, T, CDK, 64, true) ||
         !make_map_3d(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, BH, T, CDK, 64, true) ||
         !make_map_3d(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, BH, T, dv, BV, false))
-        return DR_ERR_CUDA;
-    mg = mk;
-    if (MODE == DR_KDA &&
-        !make_map_3d(&mg, gate, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, BH, T, CDK, CDK, false))
         return DR_ERR_CUDA;
     const int smem = L::TOTAL + 1024;
     auto kern = dr_chunked_kernel<MODE, BV>;
@@ -586,8 +829,8 @@ int launch_chunked_bv(const void* q, const void* k, const void* v, const float* 
         cudaSuccess)
         return DR_ERR_CUDA;
     dim3 grid((unsigned)BH, (unsigned)(dv / BV));
-    kern<<<grid, 128, smem, stream>>>(mk, mq, mv, mg, beta, gate, S0,
-                                      static_cast<__nv_bfloat16*>(out), S_final, T, dv);
+    kern<<<grid, CHUNK_THREADS, smem, stream>>>(mk, mq, mv, beta, gate, S0,
+                                                static_cast<__nv_bfloat16*>(out), S_final, T, dv);
     return cudaGetLastError() == cudaSuccess ? DR_OK : DR_ERR_CUDA;
 }
 
