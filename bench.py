@@ -75,6 +75,44 @@ def algorithmic_flops(w) -> int:
     return w.B * w.H * w.T * per_token
 
 
+def workload_config(w, world: int, nsets: int = 0, nbytes: int = 0) -> dict:
+    """The `config` object of the JSON line (shared by both arms)."""
+    from delta_rule_recurrent_chunked_b200 import workloads as wl
+
+    cfg = {"workload": w.name, "B": w.B, "H": w.H, "T": w.T}
+    if isinstance(w, wl.DRWorkload):
+        cfg.update({"dk": w.dk, "dv": w.dv, "mode": wl.MODE_NAMES[w.mode], "chunk": 64})
+    else:
+        cfg.update({"d": w.d, "mode": "vla"})
+    cfg["parallelism"] = f"replicas{world}" if world > 1 else "1gpu"
+    if nsets:
+        cfg["l2"] = (f"rotating {nsets} resident input sets ({nsets * nbytes / 2**20:.0f} MiB)"
+                     " > 126 MiB L2")
+    return cfg
+
+
+def aggregate_value(world: int, head_tokens: int, steps: int, total_ms_max: float) -> float:
+    """Whole-job head-tokens/s: every rank processes the full workload per step (weak
+    scaling); the time is the slowest rank's."""
+    return world * head_tokens * steps / (total_ms_max / 1e3)
+
+
+# DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch from one ncu capture,
+# keyed by workload and the sha256 prefix of the chunked kernel's source at capture time; a
+# changed source reports null. Summaries with the commands are under profiles/.
+NCU_TRAFFIC = {
+    ("gdn_bf16", "63949d27f35ae68e"): 119961088,
+}
+
+
+def kernel_source_sha() -> str:
+    import hashlib
+
+    path = os.path.join(ROOT, "delta_rule_recurrent_chunked_b200", "csrc", "dr_chunked.cuh")
+    with open(path, "rb") as f:
+        return hashlib.sha256(f.read()).hexdigest()[:16]
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(path):
@@ -293,8 +331,7 @@ def run_ours(args, world, rank, local):
         raise RuntimeError(f"device status {status} after the timed region")
 
     total_ms_max = max_over_ranks(total_ms, device=device)
-    units = world * w.head_tokens * K
-    value = units / (total_ms_max / 1e3)
+    value = aggregate_value(world, w.head_tokens, K, total_ms_max)
     launch_ms = statistics.mean(per_launch)
 
     # end to end through the C ABI with host buffers: pinned H2D, scan, D2H of the results
@@ -310,17 +347,16 @@ def run_ours(args, world, rank, local):
         "warmup": max(3, args.warmup), "ms_per_step": total_ms_max / K,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
         "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "H": w.H, "T": w.T, "dk": w.dk, "dv": w.dv,
-                   "mode": mode, "chunk": 64, "parallelism": f"replicas{world}" if world > 1 else "1gpu",
-                   "l2": f"rotating {nsets} resident input sets ({nsets * nbytes / 2**20:.0f} MiB) > 126 MiB L2",
-                   "kernel": "chunked" if drs.chunked_applies(mode, w.dtype == "bf16", w.dk, w.dv)
-                   else "sequential"},
+        "config": dict(workload_config(w, world, nsets, nbytes),
+                       kernel="chunked" if drs.chunked_applies(mode, w.dtype == "bf16", w.dk, w.dv)
+                       else "sequential"),
         "clocks": {k: clk[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
         "e2e": {"value": world * w.head_tokens / (e2e_ms / 1e3), "unit": UNIT,
                 "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
         "gpu_launches": K,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+                     "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": NCU_TRAFFIC.get((w.name, kernel_source_sha())),
                      "peak_source": f"{peak_src} hbm_gbs", "bytes_per_launch": nbytes,
                      "launch_ms": launch_ms,
                      "tensor_tflops": tflops,
@@ -416,7 +452,7 @@ def run_reference(args, world, rank):
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": max(3, args.warmup), "ms_per_step": dt * 1e3 / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
-        "data": "synthetic", "config": {"workload": w.name},
+        "data": "synthetic", "config": workload_config(w, world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},

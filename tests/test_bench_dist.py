@@ -1,0 +1,64 @@
+"""Host-side logic of the multi-process benchmark on CPU: two gloo ranks agree on the
+slowest rank's time and the whole-job aggregate (weak scaling, no data-path collective)."""
+import os
+import socket
+
+import pytest
+
+torch = pytest.importorskip("torch")
+import torch.distributed as dist  # noqa: E402
+import torch.multiprocessing as mp  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    import sys
+    from datetime import timedelta
+
+    sys.path.insert(0, os.path.dirname(os.path.dirname(os.path.abspath(__file__))))
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    import bench
+
+    assert bench.dist_env() == (world, rank, rank)
+    bench.barrier()
+    slow = bench.max_over_ranks(10.0 + 5.0 * rank)  # rank 1 is the slow one
+    value = bench.aggregate_value(world, head_tokens=1000, steps=4, total_ms_max=slow)
+    out[rank] = (slow, value)
+    bench.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_rank_max_and_aggregate():
+    port = _free_port()
+    manager = mp.get_context("spawn").Manager()
+    out = manager.dict()
+    mp.start_processes(_worker, args=(2, port, out), nprocs=2, join=True, start_method="spawn")
+    assert out[0][0] == out[1][0] == 15.0
+    # 2 ranks x 1000 head-tokens x 4 steps in the slowest rank's 15 ms
+    assert out[0][1] == pytest.approx(2 * 1000 * 4 / 0.015)
+
+
+def test_single_process_is_identity():
+    import bench
+
+    assert bench.max_over_ranks(3.5) == 3.5
+    assert bench.aggregate_value(1, 100, 10, 1000.0) == pytest.approx(1000.0)
+
+
+def test_algorithmic_bytes_match_the_per_token_table():
+    import bench
+    from delta_rule_recurrent_chunked_b200 import workloads as wl
+
+    gdn = wl.workload("gdn_bf16")
+    assert bench.algorithmic_bytes(gdn) == gdn.head_tokens * 1048
+    kda = wl.workload("kda_bf16")
+    assert bench.algorithmic_bytes(kda) == kda.head_tokens * 1556
+    long = wl.workload("gdn_long_t4096")
+    assert bench.algorithmic_bytes(long) == long.head_tokens * 1064
