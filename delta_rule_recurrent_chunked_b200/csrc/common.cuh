@@ -86,6 +86,43 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, volatil
 }
 
 // ---------------------------------------------------------------------------------------
+// thread-block clusters (distributed shared memory)
+// ---------------------------------------------------------------------------------------
+// The same shared-memory offset in CTA `rank` of this cluster, as a shared::cluster address.
+__device__ __forceinline__ uint32_t cluster_map(uint32_t saddr, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+    return r;
+}
+
+// Arrive on an mbarrier in another CTA of the cluster (address from cluster_map).
+__device__ __forceinline__ void mbar_arrive_remote(uint32_t cluster_bar) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_bar)
+                 : "memory");
+}
+
+// Bulk copy of `bytes` (multiple of 16) from this CTA's shared memory into another CTA's,
+// completing `bytes` of transaction count on that CTA's mbarrier. Not a multicast.
+__device__ __forceinline__ void bulk_copy_to_peer(uint32_t cluster_dst, uint32_t local_src,
+                                                  uint32_t bytes, uint32_t cluster_bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.shared::cta.mbarrier::complete_tx::bytes [%0], [%1], %2, "
+        "[%3];" ::"r"(cluster_dst),
+        "r"(local_src), "r"(bytes), "r"(cluster_bar)
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_commit_and_wait_read() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+
+__device__ __forceinline__ void cluster_sync_all() {
+    asm volatile("barrier.cluster.arrive.release.aligned;" ::: "memory");
+    asm volatile("barrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// ---------------------------------------------------------------------------------------
 // async proxy fences and TMA
 // ---------------------------------------------------------------------------------------
 // Makes generic-proxy shared-memory writes visible to the async proxy (tensor core, TMA).

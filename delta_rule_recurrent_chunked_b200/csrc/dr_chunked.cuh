@@ -26,13 +26,13 @@
 // substitution in fp32, then the off-diagonal blocks by two levels of block products
 // (X21 = -X22 A21 X11) on tf32 mma.sync, whose 16-row tiles are below tcgen05's minimum M.
 //
-// Warp roles (384 threads):
+// Warp roles (512 threads):
 //   warp 0      TMA producer of K and Q tiles; beta and GDN gate scalars
 //   warp 1      chain MMA issuer (MMA1, MMA2, MMA3)
 //   warp 2      prep MMA issuer (Gram, PT, H)
 //   warp 3      tensor-memory allocation, then the TMA producer of V tiles
 //   warps 4-7   chain warpgroup: residual Y, output rows, carried state (TMEM lane = row)
-//   warps 8-11  prep warpgroup: gates, Gram epilogue, UT inverse, operand staging
+//   warps 8-15  prep warps (two halves): gates, Gram epilogue, UT inverse, operand staging
 // The prep side runs up to one chunk ahead of the chain; the only serial dependency
 // between chunks is the state (MMA1 -> residual -> MMA3 -> state copy -> MMA1).
 // Every wait is bounded: on a timeout the status word is latched, the CTA-wide abort flag
@@ -48,7 +48,7 @@ namespace drscan {
 
 constexpr int CK = 64;    // chunk length
 constexpr int CDK = 128;  // key dimension of the chunked kernel
-constexpr int CHUNK_THREADS = 384;
+constexpr int CHUNK_THREADS = 512;
 
 template <int MODE, int BV>
 struct ChunkLayout {
@@ -56,37 +56,50 @@ struct ChunkLayout {
     static constexpr bool kGdn = MODE == DR_GDN;
     static constexpr int NS = 2;                          // K/Q stages
     static constexpr int NSV = (kKda && BV == 128) ? 1 : 2;  // V stages
-    static constexpr int NP = (kKda && BV == 128) ? 1 : 2;   // prepared-operand slots
+    static constexpr int NP = (kKda && BV >= 64) ? 1 : 2;    // prepared-operand slots
     static constexpr int NKN = kKda ? 1 : 0;
 
     static constexpr int KQ_B = 32768;  // [K;Q] bf16: 2 panels x 128 rows x 128 B
     static constexpr int V_B = CK * BV * 2;
-    static constexpr int SY_B = ((BV * 128 + 1023) / 1024) * 1024;
+    // The chain MMAs run with N = NB >= 64 so that Y and the bf16 state are stored as
+    // M/N-major B operands in 64-column swizzled groups (whole-row 16-byte stores); columns
+    // BV..NB-1 are zero padding.
+    static constexpr int NB = BV < 64 ? 64 : BV;
+    static constexpr int NG = NB / 64;
+    static constexpr int SY_B = NG * 8192;   // Y: 64 rows (t) x NB, per 64-column group 8 KB
+    static constexpr int SS_B = NG * 16384;  // S: 128 rows (key channel) x NB
+
+    // A prepared-operand slot: [T; PT] (128 rows x 64), Khat^T (128 rows (dk) x 64 (t)),
+    // gamma vector. Contiguous, so that one bulk copy hands it to another CTA of the cluster.
+    static constexpr int SLOT_TP = 0, SLOT_KH = 16384, SLOT_GAM = 32768;
+    static constexpr int SLOT_B = 32768 + 1024;
 
     static constexpr int KQ = 0;
     static constexpr int KN = KQ + NS * KQ_B;    // KDA: K/gamma, 2 panels x 64 rows
-    static constexpr int TP = KN + NKN * 16384;  // slot: [T; PT] 128 rows x 64
-    static constexpr int KH = TP + NP * 16384;   // slot: Khat^T 128 rows (dk) x 64 (t)
-    static constexpr int PM = KH + NP * 16384;   // P: rows 0-63, rows 64-127 zero
+    static constexpr int SLOT = KN + NKN * 16384;
+    static constexpr int PM = SLOT + NP * SLOT_B;  // P: rows 0-63, rows 64-127 zero
     static constexpr int TTS = PM + 16384;       // GDN: diag(gamma_C/gamma) T, 64 rows
-    static constexpr int SS = TTS + (kGdn ? 8192 : 0);  // S bf16: 2 panels x BV rows
-    static constexpr int SY = SS + BV * 256;     // Y^T: BV rows x 64
+    static constexpr int SS = TTS + (kGdn ? 8192 : 0);  // S bf16, M/N-major B operand
+    static constexpr int SY = SS + SS_B;         // Y bf16, M/N-major B operand
     static constexpr int V = SY + SY_B;          // V stages: 64 rows x BV bf16
     static constexpr int AM = V + NSV * V_B;     // A, then X = (I+A)^{-1}: fp32 [64][68]
     static constexpr int ZS = AM + CK * 68 * 4;  // block-product scratch: fp32 [32][36]
-    static constexpr int GAM = ZS + 32 * 36 * 4; // slot: gamma[64] + gamma_C (GDN), gamma_C[128] (KDA)
-    static constexpr int BG = GAM + NP * 1024;   // per stage: beta[64], GDN alpha[64]
-    static constexpr int PG = BG + NS * 512;     // prep-private: g[64], 1/gamma[64], gamma_C[128]
-    static constexpr int BAR = PG + 1024;
+    static constexpr int GAM = ZS + 32 * 36 * 4;
+    // per stage: beta[64]; GDN: g[64], 1/gamma[64], gamma[64] (cumulative log-decay and its
+    // exponentials, computed by the producer warp)
+    static constexpr int BG_B = 1024;
+    static constexpr int BG = GAM;
+    static constexpr int PG = BG + NS * BG_B;    // prep-private: KDA scan exchange, gamma_C[128]
+    static constexpr int BAR = PG + 3072;
     static constexpr int TOTAL = BAR + 256;
     static_assert(TOTAL + 1024 <= 232448, "shared memory budget");
 
     static constexpr int COL_G = 0;   // D_G, then D_PT
     static constexpr int COL_H = 64;  // D_H
     static constexpr int COL_D1 = 128;
-    static constexpr int COL_D2 = 128 + BV;
-    static constexpr int COL_S = 128 + 2 * BV;
-    static constexpr int NCOLS = (128 + 3 * BV) <= 256 ? 256 : 512;
+    static constexpr int COL_D2 = 128 + NB;
+    static constexpr int COL_S = 128 + 2 * NB;
+    static constexpr int NCOLS = (128 + 3 * NB) <= 256 ? 256 : 512;
 };
 
 // mbarrier indices inside the BAR block
@@ -105,7 +118,8 @@ enum ChunkBar {
     B_YREADY = 17,
     B_MMA23 = 18,
     B_STATE = 19,     // bf16 state copy ready for MMA1
-    B_COUNT = 20
+    B_PEER_FREE = 20,  // [2] owner side: the other CTAs of the cluster freed their slot
+    B_COUNT = 22
 };
 
 // bf16 bits of 8 consecutive columns of a row, stored as one 16-byte swizzled chunk.
@@ -168,14 +182,14 @@ __device__ __forceinline__ void store_neg_frag(float* m, int ld, int r0, int n0,
     m[(r0 + g + 8) * ld + n0 + 2 * tg + 1] = sign * d[3];
 }
 
-__device__ __forceinline__ void prep_sync() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+__device__ __forceinline__ void prep_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
 
 template <int MODE, int BV>
 __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
     const __grid_constant__ CUtensorMap tmV, const float* __restrict__ beta,
     const float* __restrict__ gate, const float* __restrict__ S0,
-    __nv_bfloat16* __restrict__ out, float* __restrict__ S_final, int T, int dv) {
+    __nv_bfloat16* __restrict__ out, float* __restrict__ S_final, int T, int dv, int share) {
     using L = ChunkLayout<MODE, BV>;
     constexpr bool kGdn = MODE == DR_GDN;
     constexpr bool kKda = MODE == DR_KDA;
@@ -195,6 +209,12 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
     const long bh = blockIdx.x;
     const int v0 = blockIdx.y * BV;
     const int nchunks = (T + CK - 1) / CK;
+    // With `share`, the CTAs of one head (value slices) form a cluster of NC; chunk c's
+    // prepared operands are computed only by CTA c % NC and copied to the others.
+    const int NC = share ? (int)gridDim.y : 1;
+    const int rank = share ? (int)blockIdx.y : 0;
+    auto owner = [&](int c) { return share ? c % NC : rank; };
+    auto slot = [&](int p) { return sm + L::SLOT + p * L::SLOT_B; };
 
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) {
@@ -202,12 +222,13 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             mbar_init(bar(B_KQ_EMPTY + s), 2);
             mbar_init(bar(B_V_FULL + s), 1);
             mbar_init(bar(B_V_EMPTY + s), 64);
-            mbar_init(bar(B_PREP + s), 128);
-            mbar_init(bar(B_SLOT_EMPTY + s), 129);
+            mbar_init(bar(B_PREP + s), 1);
+            mbar_init(bar(B_SLOT_EMPTY + s), 1);
+            mbar_init(bar(B_PEER_FREE + s), NC > 1 ? NC - 1 : 1);
         }
-        mbar_init(bar(B_GO), 128);
+        mbar_init(bar(B_GO), 256);
         mbar_init(bar(B_GRAM), 1);
-        mbar_init(bar(B_TREADY), 128);
+        mbar_init(bar(B_TREADY), 256);
         mbar_init(bar(B_HDONE), 1);
         mbar_init(bar(B_MMA1), 1);
         mbar_init(bar(B_YREADY), 128);
@@ -217,12 +238,16 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
         mbar_init_fence();
     }
     if (warp == 3) tmem_alloc(smem_u32(tmem_holder), L::NCOLS);
-    // P's rows 64-127 feed an M=128 MMA whose upper half is discarded: keep them zero.
+    // P's rows 64-127 feed an M=128 MMA whose upper half is discarded, and the padding
+    // columns of S and Y are read by the chain MMAs: keep them zero.
     for (int e = tid; e < 8192 / 16; e += CHUNK_THREADS)
         reinterpret_cast<uint4*>(sm + L::PM + 8192)[e] = make_uint4(0, 0, 0, 0);
+    for (int e = tid; e < (L::SS_B + L::SY_B) / 16; e += CHUNK_THREADS)
+        reinterpret_cast<uint4*>(sm + L::SS)[e] = make_uint4(0, 0, 0, 0);
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
+    if (share) cluster_sync_all();  // peers' barriers are initialised before any remote arrive
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
@@ -237,11 +262,31 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             const int s = c % NS;
             const int t0 = c * CK;
             if (c >= NS) mbar_wait(bar(B_KQ_EMPTY + s), (uint32_t)(((c / NS) - 1) & 1), abort_flag);
-            float* bg = reinterpret_cast<float*>(sm + L::BG + s * 512);
+            float* bg = reinterpret_cast<float*>(sm + L::BG + s * L::BG_B);
             for (int e = lane; e < CK; e += 32) {
                 const int t = t0 + e;
                 bg[e] = t < T ? beta[bh * T + t] : 0.f;
-                if constexpr (kGdn) bg[64 + e] = t < T ? gate[bh * T + t] : 1.f;
+            }
+            if constexpr (kGdn) {
+                // g_t = sum of log alpha over the chunk's rows up to t (masked rows add 0)
+                float x0 = t0 + lane < T ? __logf(gate[bh * T + t0 + lane]) : 0.f;
+                float x1 = t0 + 32 + lane < T ? __logf(gate[bh * T + t0 + 32 + lane]) : 0.f;
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const float y0 = __shfl_up_sync(0xffffffffu, x0, off);
+                    const float y1 = __shfl_up_sync(0xffffffffu, x1, off);
+                    if (lane >= off) {
+                        x0 += y0;
+                        x1 += y1;
+                    }
+                }
+                x1 += __shfl_sync(0xffffffffu, x0, 31);
+                bg[64 + lane] = x0;
+                bg[96 + lane] = x1;
+                bg[128 + lane] = __expf(-x0);
+                bg[160 + lane] = __expf(-x1);
+                bg[192 + lane] = __expf(x0);
+                bg[224 + lane] = __expf(x1);
             }
             __syncwarp();
             if (lane == 0) {
@@ -275,10 +320,11 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
     } else if (warp == 1) {
         // ------------------------------------------------------------------ chain MMA issuer
         if (lane == 0) {
-            constexpr uint32_t id1 = idesc_bf16(128, BV, 0, 0);
+            constexpr uint32_t id1 = idesc_bf16(128, L::NB, 0, 1);
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c % NS, p = c % NP;
                 uint8_t* kq = sm + L::KQ + s * L::KQ_B;
+                mbar_wait(bar(B_KQ_FULL + s), (uint32_t)((c / NS) & 1), abort_flag);
                 mbar_wait(bar(B_PREP + p), (uint32_t)((c / NP) & 1), abort_flag);
                 mbar_wait(bar(B_STATE), (uint32_t)(c & 1), abort_flag);
                 tc_fence_after();
@@ -288,8 +334,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                         const int pn = kk >> 2, ko = (kk & 3) * 32;
                         tc_mma_bf16(tmem + L::COL_D1,
                                     smem_desc_sw128(smem_u32(kq + pn * 16384 + ko), 16, 1024),
-                                    smem_desc_sw128(smem_u32(sm + L::SS + pn * (BV * 128) + ko), 16,
-                                                    1024),
+                                    smem_desc_sw128(smem_u32(sm + L::SS + kk * 2048), 16384, 1024),
                                     id1, kk > 0);
                     }
                     tc_commit(bar(B_MMA1));
@@ -298,22 +343,21 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 mbar_wait(bar(B_YREADY), (uint32_t)(c & 1), abort_flag);
                 tc_fence_after();
                 if (!*abort_flag) {
-                    const uint8_t* tp = sm + L::TP + p * 16384;
-                    const uint8_t* kh = sm + L::KH + p * 16384;
+                    const uint8_t* tp = slot(p) + L::SLOT_TP;
+                    const uint8_t* kh = slot(p) + L::SLOT_KH;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         tc_mma_bf16(tmem + L::COL_D2,
                                     smem_desc_sw128(smem_u32(tp + kk * 32), 16, 1024),
-                                    smem_desc_sw128(smem_u32(sm + L::SY + kk * 32), 16, 1024), id1,
-                                    kk > 0);
+                                    smem_desc_sw128(smem_u32(sm + L::SY + kk * 2048), 8192, 1024),
+                                    id1, kk > 0);
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
                         tc_mma_bf16(tmem + L::COL_S,
                                     smem_desc_sw128(smem_u32(kh + kk * 32), 16, 1024),
-                                    smem_desc_sw128(smem_u32(sm + L::SY + kk * 32), 16, 1024), id1,
-                                    1);
+                                    smem_desc_sw128(smem_u32(sm + L::SY + kk * 2048), 8192, 1024),
+                                    id1, 1);
                     tc_commit(bar(B_MMA23));
-                    tc_commit(bar(B_SLOT_EMPTY + p));
                 }
             }
         }
@@ -323,11 +367,19 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             constexpr uint32_t idg = idesc_bf16(128, 64, 0, 0);
             constexpr uint32_t idp = idesc_bf16(128, 64, 0, 1);
             constexpr uint32_t idh = idesc_bf16(128, 64, 1, 1);
+            int jo = 0;  // owned chunks seen so far
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c % NS, p = c % NP;
                 uint8_t* kq = sm + L::KQ + s * L::KQ_B;
                 uint8_t* kn = sm + L::KN;
-                mbar_wait(bar(B_GO), (uint32_t)(c & 1), abort_flag);
+                if (owner(c) != rank) {
+                    // the stage is not read on the prep side: release it once it has landed
+                    mbar_wait(bar(B_KQ_FULL + s), (uint32_t)((c / NS) & 1), abort_flag);
+                    mbar_arrive(bar(B_KQ_EMPTY + s));
+                    continue;
+                }
+                const uint32_t jp = (uint32_t)(jo++ & 1);
+                mbar_wait(bar(B_GO), jp, abort_flag);
                 tc_fence_after();
                 if (!*abort_flag) {
 #pragma unroll
@@ -340,10 +392,10 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     }
                     tc_commit(bar(B_GRAM));
                 }
-                mbar_wait(bar(B_TREADY), (uint32_t)(c & 1), abort_flag);
+                mbar_wait(bar(B_TREADY), jp, abort_flag);
                 tc_fence_after();
                 if (!*abort_flag) {
-                    const uint8_t* tp = sm + L::TP + p * 16384;
+                    const uint8_t* tp = slot(p) + L::SLOT_TP;
                     // PT = P T: B = T read M/N-major from the slot's rows 0-63
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
@@ -374,24 +426,36 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
         {
             const float* src = S0 ? S0 + (bh * dv + v0) * (long)CDK + r : nullptr;
 #pragma unroll
-            for (int c16 = 0; c16 < BV; c16 += 16) {
+            for (int c16 = 0; c16 < L::NB; c16 += 16) {
                 float sv[16];
 #pragma unroll
-                for (int v = 0; v < 16; ++v) sv[v] = src ? src[(long)(c16 + v) * CDK] : 0.f;
-#pragma unroll
                 for (int v = 0; v < 16; ++v)
-                    st_bf16(sm + L::SS, sw128_offset(c16 + v, r, BV), sv[v]);
+                    sv[v] = (src && c16 < BV) ? src[(long)(c16 + v) * CDK] : 0.f;
+                if (c16 < BV) {
+                    uint8_t* grp = sm + L::SS + (c16 >> 6) * 16384;
+                    st_row_chunk(grp, r, (c16 & 63) >> 3, sv);
+                    st_row_chunk(grp, r, ((c16 & 63) >> 3) + 1, sv + 8);
+                }
                 tmem_st16(trow + L::COL_S + c16, sv);
             }
             tmem_wait_st();
             fence_async_smem();
             mbar_arrive(bar(B_STATE));
+            // slots start empty: for the first chunks owned by another CTA, expect the copy
+            if (r == 0 && share) {
+                for (int c = 0; c < NP && c < nchunks; ++c) {
+                    if (owner(c) != rank) {
+                        mbar_arrive_expect_tx(bar(B_PREP + c), L::SLOT_B);
+                        mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + c), owner(c)));
+                    }
+                }
+            }
         }
         auto prescale = [&](int c) {  // S^T *= gamma_C of chunk c, before MMA3(c)
             if constexpr (MODE != DR_DELTANET) {
                 const int p = c % NP;
                 mbar_wait(bar(B_PREP + p), (uint32_t)((c / NP) & 1), abort_flag);
-                const float* gam = reinterpret_cast<const float*>(sm + L::GAM + p * 1024);
+                const float* gam = reinterpret_cast<const float*>(slot(p) + L::SLOT_GAM);
                 const float gC = kKda ? gam[r] : gam[64];
 #pragma unroll
                 for (int c16 = 0; c16 < BV; c16 += 16) {
@@ -410,7 +474,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             const int p = c % NP, svi = c % NSV;
             const int t0 = c * CK;
             const int nvalid = min(CK, T - t0);
-            const float* gam = reinterpret_cast<const float*>(sm + L::GAM + p * 1024);
+            const float* gam = reinterpret_cast<const float*>(slot(p) + L::SLOT_GAM);
             mbar_wait(bar(B_MMA1), (uint32_t)(c & 1), abort_flag);
             tc_fence_after();
             if (r < 64) {
@@ -419,21 +483,24 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 const float gt = kGdn ? gam[r] : 1.f;
                 const uint4* vrow =
                     reinterpret_cast<const uint4*>(sm + L::V + svi * L::V_B + r * BV * 2);
+                constexpr int HW = BV < 64 ? BV : 64;  // columns per pass
 #pragma unroll
-                for (int c16 = 0; c16 < BV; c16 += 16) {
-                    float x[16];
-                    tmem_ld16(trow + L::COL_D1 + c16, x);
+                for (int c0 = 0; c0 < BV; c0 += HW) {
+                    float x[HW];
+                    uint4 vw[HW / 8];
+#pragma unroll
+                    for (int c16 = 0; c16 < HW; c16 += 16) tmem_ld16(trow + L::COL_D1 + c0 + c16, x + c16);
+#pragma unroll
+                    for (int i = 0; i < HW / 8; ++i) vw[i] = vrow[c0 / 8 + i];
                     tmem_wait_ld();
 #pragma unroll
-                    for (int h = 0; h < 2; ++h) {
-                        const uint4 w = vrow[c16 / 8 + h];
-                        const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&w);
+                    for (int i = 0; i < HW / 8; ++i) {
+                        const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&vw[i]);
+                        float y[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) {
-                            const int v = c16 + h * 8 + e;
-                            st_bf16(sm + L::SY, sw128_offset(v, r, BV),
-                                    fmaf(-gt, x[h * 8 + e], __bfloat162float(hv[e])));
-                        }
+                        for (int e = 0; e < 8; ++e) y[e] = fmaf(-gt, x[8 * i + e], __bfloat162float(hv[e]));
+                        const int col = c0 + 8 * i;
+                        st_row_chunk(sm + L::SY + (col >> 6) * 8192, r, (col & 63) >> 3, y);
                     }
                 }
                 mbar_arrive(bar(B_V_EMPTY + svi));
@@ -473,138 +540,202 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 float* dst = (c == nchunks - 1 && S_final)
                                  ? S_final + (bh * dv + v0) * (long)CDK + r
                                  : nullptr;
+                constexpr int HW = BV < 64 ? BV : 64;
 #pragma unroll
-                for (int c16 = 0; c16 < BV; c16 += 16) {
-                    float sv[16];
-                    tmem_ld16(trow + L::COL_S + c16, sv);
+                for (int c0 = 0; c0 < BV; c0 += HW) {
+                    float sv[HW];
+#pragma unroll
+                    for (int c16 = 0; c16 < HW; c16 += 16) tmem_ld16(trow + L::COL_S + c0 + c16, sv + c16);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int v = 0; v < 16; ++v)
-                        st_bf16(sm + L::SS, sw128_offset(c16 + v, r, BV), sv[v]);
+                    for (int i = 0; i < HW / 8; ++i) {
+                        const int col = c0 + 8 * i;
+                        st_row_chunk(sm + L::SS + (col >> 6) * 16384, r, (col & 63) >> 3, sv + 8 * i);
+                    }
                     if (dst) {
 #pragma unroll
-                        for (int v = 0; v < 16; ++v) dst[(long)(c16 + v) * CDK] = sv[v];
+                        for (int v = 0; v < HW; ++v) dst[(long)(c0 + v) * CDK] = sv[v];
                     }
                 }
             }
             fence_async_smem();
             tc_fence_before();
             mbar_arrive(bar(B_STATE));
-            mbar_arrive(bar(B_SLOT_EMPTY + p));
+            // slot p is free once every chain thread is done with it (MMA2/3 completed before
+            // the wait above); hand it to whoever fills it next
+            asm volatile("bar.sync 2, 128;" ::: "memory");
+            if (r == 0 && c + NP < nchunks) {
+                const int nxt = c + NP;
+                if (owner(nxt) == rank) {
+                    mbar_arrive(bar(B_SLOT_EMPTY + p));
+                } else {
+                    mbar_arrive_expect_tx(bar(B_PREP + p), L::SLOT_B);
+                    mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + p), owner(nxt)));
+                }
+            }
             if (c + 1 < nchunks) prescale(c + 1);
         }
     } else if (warp >= 8) {
-        // ------------------------------------------------------------------ prep warpgroup
-        const int r = tid - 256;
-        const uint32_t trow = tmem + ((uint32_t)(r & ~31) << 16);
-        const int wq = r >> 5, g8 = lane >> 2, tg = lane & 3;
-        float* pg = reinterpret_cast<float*>(sm + L::PG);  // g[64] | 1/gamma[64] | gamma_C[128]
+        // ------------------------------------------------------------------ prep warps
+        // u: 0..255. Lane-mapped work uses TMEM lane lq = u % 128 and column half hf = u / 128
+        // (warp 8+i reaches TMEM lanes 32*(i%4) .. +31).
+        const int u = tid - 256;
+        const int lq = u & 127, hf = u >> 7;
+        const uint32_t trow = tmem + ((uint32_t)(lq & ~31) << 16);
+        const int wq = u >> 5, g8 = lane >> 2, tg = lane & 3;
+        // KDA scan exchange: pg[128*q + ch] = product over row quarter q; gamma_C at pg[512 + ch]
+        float* pg = reinterpret_cast<float*>(sm + L::PG);
         float* sA = reinterpret_cast<float*>(sm + L::AM);
         float* sZ = reinterpret_cast<float*>(sm + L::ZS);
-        float gpf[kKda ? CK : 1];  // KDA: next chunk's alpha for channel r, prefetched
+        // KDA: thread u owns key channels 2*(u%64), 2*(u%64)+1 on rows 16*(u/64) .. +15 of a
+        // chunk; the next owned chunk's alpha values are prefetched into registers.
+        const int kc = 2 * (u & 63), kq4 = u >> 6;
+        float2 gpf[kKda ? 16 : 1];
         if constexpr (kKda) {
+            const int c0 = rank;
 #pragma unroll
-            for (int t = 0; t < CK; ++t) gpf[t] = t < T ? gate[(bh * T + t) * (long)CDK + r] : 1.f;
+            for (int i = 0; i < 16; ++i) {
+                const int t = c0 * CK + 16 * kq4 + i;
+                gpf[i] = t < T ? *reinterpret_cast<const float2*>(gate + (bh * T + t) * (long)CDK + kc)
+                               : make_float2(1.f, 1.f);
+            }
         }
-        for (int c = 0; c < nchunks; ++c) {
+        int jo = 0;       // owned chunks processed so far
+        int kq_seen = 0;  // K/Q stage phases waited so far (every chunk, in order)
+        for (int c = rank; c < nchunks; c += NC, ++jo) {
             const int s = c % NS, p = c % NP;
+            const uint32_t jp = (uint32_t)(jo & 1);
             const int t0 = c * CK;
             const int nvalid = min(CK, T - t0);
             uint8_t* kq = sm + L::KQ + s * L::KQ_B;
-            const float* bg = reinterpret_cast<const float*>(sm + L::BG + s * 512);
-            mbar_wait(bar(B_KQ_FULL + s), (uint32_t)((c / NS) & 1), abort_flag);
+            const float* bg = reinterpret_cast<const float*>(sm + L::BG + s * L::BG_B);
+            // A parity wait cannot tell "this phase done" from "the previous phase still
+            // pending", so the stages' phases are walked in order, owned chunk or not.
+            for (; kq_seen <= c; ++kq_seen)
+                mbar_wait(bar(B_KQ_FULL + kq_seen % NS), (uint32_t)((kq_seen / NS) & 1), abort_flag);
 
-            // ---- 1. gates
-            bool fact = true;  // GDN: exp(g_t - g_i) = gamma_t * (1/gamma_i) is safe
+            // ---- 1. gates. GDN: g, 1/gamma, gamma come from the producer; the factored form
+            // gamma_t * (1/gamma_i) of exp(g_t - g_i) is used when it cannot overflow.
+            bool fact = true;
             if constexpr (kGdn) {
-                float x = 0.f;
-                if (r < 64) {
-                    x = (r < nvalid) ? __logf(bg[64 + r]) : 0.f;
-#pragma unroll
-                    for (int off = 1; off < 32; off <<= 1) {
-                        const float y = __shfl_up_sync(0xffffffffu, x, off);
-                        if (lane >= off) x += y;
-                    }
-                    pg[r] = x;
-                }
-                prep_sync();
-                if (r >= 32 && r < 64) {
-                    x += pg[31];
-                    pg[r] = x;
-                }
-                prep_sync();
-                if (r < 64) pg[64 + r] = __expf(-x);
-                prep_sync();
-                fact = pg[63] > -80.f;
+                fact = bg[64 + 63] > -80.f;
             } else if constexpr (kKda) {
-                // channel r: running product of alpha; rewrite K and Q in place as K*gamma,
-                // Q*gamma and store K/gamma
+                // running products of alpha per key channel (four row quarters joined through
+                // shared memory); rewrite K and Q in place as K*gamma, Q*gamma; store K/gamma
                 uint8_t* kn = sm + L::KN;
-                float run = 1.f;
+                float2 part = make_float2(1.f, 1.f);
 #pragma unroll
-                for (int t = 0; t < CK; ++t) {
-                    if (t < nvalid) run *= gpf[t];
-                    const float inv = __frcp_rn(run);
-                    const uint32_t ok_ = sw128_offset(t, r, 128);
-                    const uint32_t oq = sw128_offset(64 + t, r, 128);
-                    const float kv = ld_bf16(kq, ok_);
-                    st_bf16(kq, ok_, kv * run);
-                    st_bf16(kq, oq, ld_bf16(kq, oq) * run);
-                    st_bf16(kn, sw128_offset(t, r, 64), kv * inv);
+                for (int i = 0; i < 16; ++i) {
+                    if (16 * kq4 + i < nvalid) {
+                        part.x *= gpf[i].x;
+                        part.y *= gpf[i].y;
+                    }
                 }
-                pg[128 + r] = run;  // gamma_C for channel r
+                if (kq4 < 3) *reinterpret_cast<float2*>(pg + 128 * kq4 + kc) = part;
+                prep_sync();
+                float2 run = make_float2(1.f, 1.f);
+                for (int q = 0; q < kq4; ++q) {
+                    const float2 pq = *reinterpret_cast<const float2*>(pg + 128 * q + kc);
+                    run.x *= pq.x;
+                    run.y *= pq.y;
+                }
 #pragma unroll
-                for (int t = 0; t < CK; ++t) {
-                    const int tn = t0 + CK + t;
-                    gpf[t] = tn < T ? gate[(bh * T + tn) * (long)CDK + r] : 1.f;
+                for (int i0 = 0; i0 < 16; i0 += 8) {
+                    uint32_t kw[8], qw[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int t = 16 * kq4 + i0 + i;
+                        kw[i] = *reinterpret_cast<const uint32_t*>(kq + sw128_offset(t, kc, 128));
+                        qw[i] = *reinterpret_cast<const uint32_t*>(kq + sw128_offset(64 + t, kc, 128));
+                    }
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) {
+                        const int t = 16 * kq4 + i0 + i;
+                        if (t < nvalid) {
+                            run.x *= gpf[i0 + i].x;
+                            run.y *= gpf[i0 + i].y;
+                        }
+                        const float2 k2 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&kw[i]));
+                        const float2 q2 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&qw[i]));
+                        const float ix = __fdividef(1.f, run.x), iy = __fdividef(1.f, run.y);
+                        *reinterpret_cast<uint32_t*>(kq + sw128_offset(t, kc, 128)) =
+                            pack_bf16(k2.x * run.x, k2.y * run.y);
+                        *reinterpret_cast<uint32_t*>(kq + sw128_offset(64 + t, kc, 128)) =
+                            pack_bf16(q2.x * run.x, q2.y * run.y);
+                        *reinterpret_cast<uint32_t*>(kn + sw128_offset(t, kc, 64)) =
+                            pack_bf16(k2.x * ix, k2.y * iy);
+                    }
+                }
+                if (kq4 == 3) *reinterpret_cast<float2*>(pg + 512 + kc) = run;  // gamma_C
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int tn = t0 + NC * CK + 16 * kq4 + i;
+                    gpf[i] = tn < T ? *reinterpret_cast<const float2*>(gate + (bh * T + tn) * (long)CDK + kc)
+                                    : make_float2(1.f, 1.f);
                 }
                 fence_async_smem();
+                prep_sync();
             }
             tc_fence_before();
             mbar_arrive(bar(B_GO));
 
-            // ---- 2. Gram epilogue: A (fp32, rows 0-63) and P (bf16, rows 0-63 of PM)
-            mbar_wait(bar(B_GRAM), (uint32_t)(c & 1), abort_flag);
+            // ---- 2. Gram epilogue: A (fp32, rows 0-63) and P (bf16, rows 0-63 of PM); each
+            // thread takes one half (32 columns) of one row
+            mbar_wait(bar(B_GRAM), jp, abort_flag);
             tc_fence_after();
             {
-                const int t = r & 63;
-                float rowf = (r < 64) ? bg[t] : 1.f;  // beta_t on A rows
+                const int t = lq & 63;
+                const int c32 = 32 * hf;
+                float rowf = (lq < 64) ? bg[t] : 1.f;  // beta_t on A rows
                 float gt = 0.f;
                 if constexpr (kGdn) {
-                    gt = pg[t];
-                    if (fact) rowf *= __expf(gt);
+                    gt = bg[64 + t];
+                    if (fact) rowf *= bg[192 + t];
                 }
+                float gr[32];
+                tmem_ld16(trow + L::COL_G + c32, gr);
+                tmem_ld16(trow + L::COL_G + c32 + 16, gr + 16);
+                float dec[32];
+                if constexpr (kGdn) {
+                    if (fact) {
 #pragma unroll
-                for (int c16 = 0; c16 < 64; c16 += 16) {
-                    float gr[16];
-                    tmem_ld16(trow + L::COL_G + c16, gr);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int e = 0; e < 16; ++e) {
-                        const int i = c16 + e;
-                        float dec = 1.f;
-                        if constexpr (kGdn)
-                            dec = fact ? pg[64 + i] : __expf(fminf(gt - pg[i], 0.f));
-                        const bool keep = (r < 64) ? (i < t) : (i <= t);
-                        gr[e] = keep ? rowf * gr[e] * dec : 0.f;
-                    }
-                    if (r < 64) {
-#pragma unroll
-                        for (int e = 0; e < 16; e += 4)
-                            *reinterpret_cast<float4*>(sA + t * 68 + c16 + e) =
-                                make_float4(gr[e], gr[e + 1], gr[e + 2], gr[e + 3]);
+                        for (int e = 0; e < 32; e += 4) {
+                            const float4 d4 = *reinterpret_cast<const float4*>(bg + 128 + c32 + e);
+                            dec[e] = d4.x;
+                            dec[e + 1] = d4.y;
+                            dec[e + 2] = d4.z;
+                            dec[e + 3] = d4.w;
+                        }
                     } else {
-                        st_row_chunk(sm + L::PM, t, c16 / 8, gr);
-                        st_row_chunk(sm + L::PM, t, c16 / 8 + 1, gr + 8);
+#pragma unroll
+                        for (int e = 0; e < 32; ++e)
+                            dec[e] = __expf(fminf(gt - bg[64 + c32 + e], 0.f));
                     }
+                }
+                tmem_wait_ld();
+#pragma unroll
+                for (int e = 0; e < 32; ++e) {
+                    const int i = c32 + e;
+                    const bool keep = (lq < 64) ? (i < t) : (i <= t);
+                    const float v = kGdn ? rowf * gr[e] * dec[e] : rowf * gr[e];
+                    gr[e] = keep ? v : 0.f;
+                }
+                if (lq < 64) {
+#pragma unroll
+                    for (int e = 0; e < 32; e += 4)
+                        *reinterpret_cast<float4*>(sA + t * 68 + c32 + e) =
+                            make_float4(gr[e], gr[e + 1], gr[e + 2], gr[e + 3]);
+                } else {
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) st_row_chunk(sm + L::PM, t, c32 / 8 + ch, gr + 8 * ch);
                 }
             }
             prep_sync();
 
             // ---- 3. X = (I + A)^{-1}, in place in sA
             float xcol[16];
-            if (r < 64) {  // diagonal 16x16 blocks, one column per thread
-                const int b = r >> 4, cc = r & 15;
+            if (u < 64) {  // diagonal 16x16 blocks, one column per thread
+                const int b = u >> 4, cc = u & 15;
 #pragma unroll
                 for (int t = 0; t < 16; ++t) xcol[t] = (t == cc) ? 1.f : 0.f;
 #pragma unroll
@@ -614,8 +745,8 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                         xcol[t] = fmaf(-sA[(16 * b + t) * 68 + 16 * b + i], xcol[i], xcol[t]);
             }
             prep_sync();
-            if (r < 64) {
-                const int b = r >> 4, cc = r & 15;
+            if (u < 64) {
+                const int b = u >> 4, cc = u & 15;
 #pragma unroll
                 for (int t = 0; t < 16; ++t) sA[(16 * b + t) * 68 + 16 * b + cc] = xcol[t];
             }
@@ -653,113 +784,120 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     store_neg_frag(sA, 68, b1, b0 + 8 * nt, acc2[nt], g8, tg, -1.f);
             }
             prep_sync();
-            {  // X[32:64, 0:32] = -X[32:64, 32:64] A[32:64, 0:32] X[0:32, 0:32]
-                const int m0 = 32 + 16 * (wq >> 1), n0 = 16 * (wq & 1);
-                float acc[2][4] = {};
+            {  // X[32:64, 0:32] = -X[32:64, 32:64] A[32:64, 0:32] X[0:32, 0:32]; one 16x8 tile
+               // of each product per warp
+                const int m0 = 32 + 16 * (wq >> 2), n0 = 8 * (wq & 3);
+                float acc[4] = {};
 #pragma unroll
                 for (int kk = 0; kk < 32; kk += 8) {
                     uint32_t a[4], bb[2];
                     frag_a(a, sA, 68, m0, kk, g8, tg);
-#pragma unroll
-                    for (int nt = 0; nt < 2; ++nt) {
-                        frag_b(bb, sA, 68, kk, n0 + 8 * nt, g8, tg);
-                        mma_tf32(acc[nt], a, bb);
-                    }
+                    frag_b(bb, sA, 68, kk, n0, g8, tg);
+                    mma_tf32(acc, a, bb);
                 }
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-                    store_neg_frag(sZ, 36, m0 - 32, n0 + 8 * nt, acc[nt], g8, tg, 1.f);
+                store_neg_frag(sZ, 36, m0 - 32, n0, acc, g8, tg, 1.f);
                 prep_sync();
-                float acc2[2][4] = {};
+                float acc2[4] = {};
 #pragma unroll
                 for (int kk = 0; kk < 32; kk += 8) {
                     uint32_t a[4], bb[2];
                     frag_a(a, sA, 68, m0, 32 + kk, g8, tg);
-#pragma unroll
-                    for (int nt = 0; nt < 2; ++nt) {
-                        frag_b(bb, sZ, 36, kk, n0 + 8 * nt, g8, tg);
-                        mma_tf32(acc2[nt], a, bb);
-                    }
+                    frag_b(bb, sZ, 36, kk, n0, g8, tg);
+                    mma_tf32(acc2, a, bb);
                 }
-#pragma unroll
-                for (int nt = 0; nt < 2; ++nt)
-                    store_neg_frag(sA, 68, m0, n0 + 8 * nt, acc2[nt], g8, tg, -1.f);
+                store_neg_frag(sA, 68, m0, n0, acc2, g8, tg, -1.f);
             }
             prep_sync();
 
-            // ---- 4. stage T = X diag(beta) into the slot (and Ttilde for GDN's H)
-            if (c >= NP)
-                mbar_wait(bar(B_SLOT_EMPTY + p), (uint32_t)(((c / NP) - 1) & 1), abort_flag);
-            uint8_t* tp = sm + L::TP + p * 16384;
-            float* gam = reinterpret_cast<float*>(sm + L::GAM + p * 1024);
+            // ---- 4. stage T = X diag(beta) into the slot (and Ttilde for GDN's H): thread u
+            // writes half (u/64 % 2) of row u % 64 of T (u < 128) or of Ttilde (u >= 128)
+            if (c >= NP) {
+                // the previous use of slot p (chunk c - NP) must be finished by this CTA's chain
+                const int fills = share ? jo - (rank < NP ? 1 : 0) : c / NP - 1;
+                mbar_wait(bar(B_SLOT_EMPTY + p), (uint32_t)(fills & 1), abort_flag);
+            }
+            uint8_t* tp = slot(p) + L::SLOT_TP;
+            float* gam = reinterpret_cast<float*>(slot(p) + L::SLOT_GAM);
             {
-                const int t = r & 63;
+                const int t = u & 63, half = (u >> 6) & 1;
                 float scale = 1.f;
                 uint8_t* dst = tp;
-                if (r >= 64) {
+                if (u >= 128) {
                     if constexpr (kGdn) {
-                        scale = __expf(pg[63] - pg[t]);  // gamma_C / gamma_t
+                        scale = __expf(bg[64 + 63] - bg[64 + t]);  // gamma_C / gamma_t
                         dst = sm + L::TTS;
                     } else {
                         dst = nullptr;
                     }
                 }
                 if (dst) {
+                    float row[32];
 #pragma unroll
-                    for (int ch = 0; ch < 8; ++ch) {
-                        const float4 xa = *reinterpret_cast<const float4*>(sA + t * 68 + ch * 8);
-                        const float4 xb = *reinterpret_cast<const float4*>(sA + t * 68 + ch * 8 + 4);
-                        const float4 ba = *reinterpret_cast<const float4*>(bg + ch * 8);
-                        const float4 bb = *reinterpret_cast<const float4*>(bg + ch * 8 + 4);
-                        const float row[8] = {xa.x * ba.x * scale, xa.y * ba.y * scale,
-                                              xa.z * ba.z * scale, xa.w * ba.w * scale,
-                                              xb.x * bb.x * scale, xb.y * bb.y * scale,
-                                              xb.z * bb.z * scale, xb.w * bb.w * scale};
-                        st_row_chunk(dst, t, ch, row);
+                    for (int e = 0; e < 32; e += 4) {
+                        const float4 x4 = *reinterpret_cast<const float4*>(sA + t * 68 + 32 * half + e);
+                        const float4 b4 = *reinterpret_cast<const float4*>(bg + 32 * half + e);
+                        row[e] = x4.x * b4.x * scale;
+                        row[e + 1] = x4.y * b4.y * scale;
+                        row[e + 2] = x4.z * b4.z * scale;
+                        row[e + 3] = x4.w * b4.w * scale;
                     }
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) st_row_chunk(dst, t, 4 * half + ch, row + 8 * ch);
                 }
                 if constexpr (kGdn) {
-                    if (r < 64) gam[r] = __expf(pg[r]);
-                    if (r == 64) gam[64] = __expf(pg[63]);
+                    if (u < 64) gam[u] = bg[192 + u];
+                    if (u == 64) gam[64] = bg[192 + 63];
                 } else if constexpr (kKda) {
-                    gam[r] = pg[128 + r];
+                    if (u < 128) gam[u] = pg[512 + u];
                 }
             }
             fence_async_smem();
             mbar_arrive(bar(B_TREADY));
 
-            // ---- 5. PT rows -> slot rows 64-127; Khat^T -> slot
-            mbar_wait(bar(B_HDONE), (uint32_t)(c & 1), abort_flag);
+            // ---- 5. Khat^T -> slot (row lq, column half hf); PT rows -> slot rows 64-127
+            mbar_wait(bar(B_HDONE), jp, abort_flag);
             tc_fence_after();
             {
-                uint8_t* kh = sm + L::KH + p * 16384;
-                const float gC = kKda ? pg[128 + r] : 1.f;
+                uint8_t* kh = slot(p) + L::SLOT_KH;
+                const int c32 = 32 * hf;
+                float h[32];
+                tmem_ld16(trow + L::COL_H + c32, h);
+                tmem_ld16(trow + L::COL_H + c32 + 16, h + 16);
+                tmem_wait_ld();
+                if constexpr (kKda) {
+                    const float gC = pg[512 + lq];
 #pragma unroll
-                for (int c16 = 0; c16 < 64; c16 += 16) {
-                    float h[16];
-                    tmem_ld16(trow + L::COL_H + c16, h);
-                    tmem_wait_ld();
-                    if constexpr (kKda) {
-#pragma unroll
-                        for (int e = 0; e < 16; ++e) h[e] *= gC;
-                    }
-                    st_row_chunk(kh, r, c16 / 8, h);
-                    st_row_chunk(kh, r, c16 / 8 + 1, h + 8);
+                    for (int e = 0; e < 32; ++e) h[e] *= gC;
                 }
-                if (r < 64) {
 #pragma unroll
-                    for (int c16 = 0; c16 < 64; c16 += 16) {
-                        float h[16];
-                        tmem_ld16(trow + L::COL_G + c16, h);
-                        tmem_wait_ld();
-                        st_row_chunk(tp, 64 + r, c16 / 8, h);
-                        st_row_chunk(tp, 64 + r, c16 / 8 + 1, h + 8);
-                    }
+                for (int ch = 0; ch < 4; ++ch) st_row_chunk(kh, lq, c32 / 8 + ch, h + 8 * ch);
+                if (lq < 64) {
+                    tmem_ld16(trow + L::COL_G + c32, h);
+                    tmem_ld16(trow + L::COL_G + c32 + 16, h + 16);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int ch = 0; ch < 4; ++ch) st_row_chunk(tp, 64 + lq, c32 / 8 + ch, h + 8 * ch);
                 }
             }
             fence_async_smem();
             tc_fence_before();
-            mbar_arrive(bar(B_PREP + p));
+            prep_sync();
+            if (u == 0) {
+                if (share && !*abort_flag) {
+                    // hand the slot to the other CTAs of the cluster once they have freed theirs
+                    mbar_wait(bar(B_PEER_FREE + p), jp, abort_flag);
+                    if (!*abort_flag) {
+                        const uint32_t src = smem_u32(slot(p));
+                        for (int q = 0; q < NC; ++q) {
+                            if (q == rank) continue;
+                            bulk_copy_to_peer(cluster_map(src, q), src, L::SLOT_B,
+                                              cluster_map(bar(B_PREP + p), q));
+                        }
+                        bulk_commit_and_wait_read();
+                    }
+                }
+                mbar_arrive(bar(B_PREP + p));
+            }
         }
     }
 
@@ -772,6 +910,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
         }
     }
     __syncthreads();
+    if (share) cluster_sync_all();  // no CTA leaves while the others may still address it
     tc_fence_after();
     if (warp == 3) tmem_dealloc(tmem, L::NCOLS);
 }
@@ -828,9 +967,26 @@ int launch_chunked_bv(const void* q, const void* k, const void* v, const float* 
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
         cudaSuccess)
         return DR_ERR_CUDA;
-    dim3 grid((unsigned)BH, (unsigned)(dv / BV));
-    kern<<<grid, CHUNK_THREADS, smem, stream>>>(mk, mq, mv, beta, gate, S0,
-                                                static_cast<__nv_bfloat16*>(out), S_final, T, dv);
+    const int nc = dv / BV;
+    // sharing pays off while the owner's prep plus its copies fit in the two-chunk window
+    // the stage and slot rings allow; larger clusters measured slower
+    const int share = (MODE != DR_KDA && nc > 1 && nc <= 4) ? 1 : 0;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)BH, (unsigned)nc);
+    cfg.blockDim = dim3(CHUNK_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = 1;
+    attr[0].val.clusterDim.y = share ? nc : 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = share ? 1 : 0;
+    if (cudaLaunchKernelEx(&cfg, kern, mk, mq, mv, beta, gate, S0,
+                           static_cast<__nv_bfloat16*>(out), S_final, T, dv, share) !=
+        cudaSuccess)
+        return DR_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? DR_OK : DR_ERR_CUDA;
 }
 
