@@ -189,7 +189,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
     const __grid_constant__ CUtensorMap tmV, const float* __restrict__ beta,
     const float* __restrict__ gate, const float* __restrict__ S0,
-    __nv_bfloat16* __restrict__ out, float* __restrict__ S_final, int T, int dv, int share) {
+    __nv_bfloat16* __restrict__ out, float* __restrict__ S_final, int T, int dv, int split) {
     using L = ChunkLayout<MODE, BV>;
     constexpr bool kGdn = MODE == DR_GDN;
     constexpr bool kKda = MODE == DR_KDA;
@@ -207,24 +207,27 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
     const int warp = tid >> 5;
     const int lane = tid & 31;
     const long bh = blockIdx.x;
-    const int v0 = blockIdx.y * BV;
     const int nchunks = (T + CK - 1) / CK;
-    // With `share`, the CTAs of one head (value slices) form a cluster of NC; chunk c's
-    // prepared operands are computed only by CTA c % NC and copied to the others.
-    const int NC = share ? (int)gridDim.y : 1;
-    const int rank = share ? (int)blockIdx.y : 0;
-    auto owner = [&](int c) { return share ? c % NC : rank; };
+    // With `split`, the CTAs of one head form a cluster: rank 0 prepares every chunk's
+    // operands ([T; PT], Khat^T, gamma) and copies them into the shared memory of ranks
+    // 1..NCC, each of which runs the chain for one slice of BV value channels. Without it,
+    // one CTA does both for its slice.
+    const int rank = split ? (int)blockIdx.y : 0;
+    const int NCC = split ? (int)gridDim.y - 1 : 1;  // chain CTAs per head
+    const bool is_prep = !split || rank == 0;
+    const bool is_chain = !split || rank > 0;
+    const int v0 = (split ? rank - 1 : (int)blockIdx.y) * BV;
     auto slot = [&](int p) { return sm + L::SLOT + p * L::SLOT_B; };
 
     if (tid == 0) {
         for (int s = 0; s < 2; ++s) {
             mbar_init(bar(B_KQ_FULL + s), 2);
-            mbar_init(bar(B_KQ_EMPTY + s), 2);
+            mbar_init(bar(B_KQ_EMPTY + s), split ? 1 : 2);
             mbar_init(bar(B_V_FULL + s), 1);
             mbar_init(bar(B_V_EMPTY + s), 64);
             mbar_init(bar(B_PREP + s), 1);
             mbar_init(bar(B_SLOT_EMPTY + s), 1);
-            mbar_init(bar(B_PEER_FREE + s), NC > 1 ? NC - 1 : 1);
+            mbar_init(bar(B_PEER_FREE + s), split ? NCC : 1);
         }
         mbar_init(bar(B_GO), 256);
         mbar_init(bar(B_GRAM), 1);
@@ -247,7 +250,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (share) cluster_sync_all();  // peers' barriers are initialised before any remote arrive
+    if (split) cluster_sync_all();  // peers' barriers are initialised before any remote arrive
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
@@ -304,6 +307,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             }
         }
     } else if (warp == 3) {
+        if (!is_chain) goto done;
         // ------------------------------------------------------------------ V producer
         if (lane == 0) {
             for (int c = 0; c < nchunks; ++c) {
@@ -315,6 +319,26 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     tma_load_3d(smem_u32(sm + L::V + sv * L::V_B), &tmV, bar(B_V_FULL + sv), v0,
                                 c * CK, (int)bh);
                 }
+            }
+        }
+    } else if (warp == 1 && !is_chain) {
+        // ------------------------------------------------------------------ slot distributor
+        // (prep CTA of a split cluster): ships each prepared slot to the chain CTAs once all
+        // of them have freed their copy, then hands the slot back to the prep warps
+        if (lane == 0) {
+            for (int c = 0; c < nchunks; ++c) {
+                const int p = c % NP;
+                const uint32_t ph = (uint32_t)((c / NP) & 1);
+                mbar_wait(bar(B_PREP + p), ph, abort_flag);
+                mbar_wait(bar(B_PEER_FREE + p), ph, abort_flag);
+                if (!*abort_flag) {
+                    const uint32_t src = smem_u32(slot(p));
+                    for (int q = 1; q <= NCC; ++q)
+                        bulk_copy_to_peer(cluster_map(src, q), src, L::SLOT_B,
+                                          cluster_map(bar(B_PREP + p), q));
+                    bulk_commit_and_wait_read();
+                }
+                mbar_arrive(bar(B_SLOT_EMPTY + p));
             }
         }
     } else if (warp == 1) {
@@ -362,23 +386,17 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             }
         }
     } else if (warp == 2) {
+        if (!is_prep) goto done;
         // ------------------------------------------------------------------ prep MMA issuer
         if (lane == 0) {
             constexpr uint32_t idg = idesc_bf16(128, 64, 0, 0);
             constexpr uint32_t idp = idesc_bf16(128, 64, 0, 1);
             constexpr uint32_t idh = idesc_bf16(128, 64, 1, 1);
-            int jo = 0;  // owned chunks seen so far
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c % NS, p = c % NP;
                 uint8_t* kq = sm + L::KQ + s * L::KQ_B;
                 uint8_t* kn = sm + L::KN;
-                if (owner(c) != rank) {
-                    // the stage is not read on the prep side: release it once it has landed
-                    mbar_wait(bar(B_KQ_FULL + s), (uint32_t)((c / NS) & 1), abort_flag);
-                    mbar_arrive(bar(B_KQ_EMPTY + s));
-                    continue;
-                }
-                const uint32_t jp = (uint32_t)(jo++ & 1);
+                const uint32_t jp = (uint32_t)(c & 1);
                 mbar_wait(bar(B_GO), jp, abort_flag);
                 tc_fence_after();
                 if (!*abort_flag) {
@@ -420,6 +438,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             }
         }
     } else if (warp >= 4 && warp < 8) {
+        if (!is_chain) goto done;
         // ------------------------------------------------------------------ chain warpgroup
         const int r = tid - 128;  // TMEM lane: value row t (Y, O) or key channel j (state)
         const uint32_t trow = tmem + ((uint32_t)(r & ~31) << 16);
@@ -441,13 +460,11 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             tmem_wait_st();
             fence_async_smem();
             mbar_arrive(bar(B_STATE));
-            // slots start empty: for the first chunks owned by another CTA, expect the copy
-            if (r == 0 && share) {
+            // slots start empty: expect the prep CTA's copies of the first chunks
+            if (r == 0 && split) {
                 for (int c = 0; c < NP && c < nchunks; ++c) {
-                    if (owner(c) != rank) {
-                        mbar_arrive_expect_tx(bar(B_PREP + c), L::SLOT_B);
-                        mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + c), owner(c)));
-                    }
+                    mbar_arrive_expect_tx(bar(B_PREP + c), L::SLOT_B);
+                    mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + c), 0));
                 }
             }
         }
@@ -565,17 +582,17 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             // the wait above); hand it to whoever fills it next
             asm volatile("bar.sync 2, 128;" ::: "memory");
             if (r == 0 && c + NP < nchunks) {
-                const int nxt = c + NP;
-                if (owner(nxt) == rank) {
+                if (!split) {
                     mbar_arrive(bar(B_SLOT_EMPTY + p));
                 } else {
                     mbar_arrive_expect_tx(bar(B_PREP + p), L::SLOT_B);
-                    mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + p), owner(nxt)));
+                    mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + p), 0));
                 }
             }
             if (c + 1 < nchunks) prescale(c + 1);
         }
     } else if (warp >= 8) {
+        if (!is_prep) goto done;
         // ------------------------------------------------------------------ prep warps
         // u: 0..255. Lane-mapped work uses TMEM lane lq = u % 128 and column half hf = u / 128
         // (warp 8+i reaches TMEM lanes 32*(i%4) .. +31).
@@ -592,19 +609,17 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
         const int kc = 2 * (u & 63), kq4 = u >> 6;
         float2 gpf[kKda ? 16 : 1];
         if constexpr (kKda) {
-            const int c0 = rank;
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-                const int t = c0 * CK + 16 * kq4 + i;
+                const int t = 16 * kq4 + i;
                 gpf[i] = t < T ? *reinterpret_cast<const float2*>(gate + (bh * T + t) * (long)CDK + kc)
                                : make_float2(1.f, 1.f);
             }
         }
-        int jo = 0;       // owned chunks processed so far
         int kq_seen = 0;  // K/Q stage phases waited so far (every chunk, in order)
-        for (int c = rank; c < nchunks; c += NC, ++jo) {
+        for (int c = 0; c < nchunks; ++c) {
             const int s = c % NS, p = c % NP;
-            const uint32_t jp = (uint32_t)(jo & 1);
+            const uint32_t jp = (uint32_t)(c & 1);
             const int t0 = c * CK;
             const int nvalid = min(CK, T - t0);
             uint8_t* kq = sm + L::KQ + s * L::KQ_B;
@@ -669,7 +684,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 if (kq4 == 3) *reinterpret_cast<float2*>(pg + 512 + kc) = run;  // gamma_C
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const int tn = t0 + NC * CK + 16 * kq4 + i;
+                    const int tn = t0 + CK + 16 * kq4 + i;
                     gpf[i] = tn < T ? *reinterpret_cast<const float2*>(gate + (bh * T + tn) * (long)CDK + kc)
                                     : make_float2(1.f, 1.f);
                 }
@@ -812,9 +827,9 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             // ---- 4. stage T = X diag(beta) into the slot (and Ttilde for GDN's H): thread u
             // writes half (u/64 % 2) of row u % 64 of T (u < 128) or of Ttilde (u >= 128)
             if (c >= NP) {
-                // the previous use of slot p (chunk c - NP) must be finished by this CTA's chain
-                const int fills = share ? jo - (rank < NP ? 1 : 0) : c / NP - 1;
-                mbar_wait(bar(B_SLOT_EMPTY + p), (uint32_t)(fills & 1), abort_flag);
+                // the previous use of slot p (chunk c - NP) must be finished: by this CTA's
+                // chain, or (split) by the distributor's copies to the chain CTAs
+                mbar_wait(bar(B_SLOT_EMPTY + p), (uint32_t)(((c / NP) - 1) & 1), abort_flag);
             }
             uint8_t* tp = slot(p) + L::SLOT_TP;
             float* gam = reinterpret_cast<float*>(slot(p) + L::SLOT_GAM);
@@ -882,25 +897,11 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             fence_async_smem();
             tc_fence_before();
             prep_sync();
-            if (u == 0) {
-                if (share && !*abort_flag) {
-                    // hand the slot to the other CTAs of the cluster once they have freed theirs
-                    mbar_wait(bar(B_PEER_FREE + p), jp, abort_flag);
-                    if (!*abort_flag) {
-                        const uint32_t src = smem_u32(slot(p));
-                        for (int q = 0; q < NC; ++q) {
-                            if (q == rank) continue;
-                            bulk_copy_to_peer(cluster_map(src, q), src, L::SLOT_B,
-                                              cluster_map(bar(B_PREP + p), q));
-                        }
-                        bulk_commit_and_wait_read();
-                    }
-                }
-                mbar_arrive(bar(B_PREP + p));
-            }
+            if (u == 0) mbar_arrive(bar(B_PREP + p));
         }
     }
 
+done:
     tc_fence_before();
     __syncthreads();
     if (*abort_flag && tid == 0) {
@@ -910,7 +911,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
         }
     }
     __syncthreads();
-    if (share) cluster_sync_all();  // no CTA leaves while the others may still address it
+    if (split) cluster_sync_all();  // no CTA leaves while the others may still address it
     tc_fence_after();
     if (warp == 3) tmem_dealloc(tmem, L::NCOLS);
 }
@@ -955,7 +956,7 @@ inline bool chunked_supported(int variant, int dk, int dv) {
 template <int MODE, int BV>
 int launch_chunked_bv(const void* q, const void* k, const void* v, const float* beta,
                       const float* gate, const float* S0, void* out, float* S_final, int BH, int T,
-                      int dv, cudaStream_t stream) {
+                      int dv, int split, cudaStream_t stream) {
     using L = ChunkLayout<MODE, BV>;
     CUtensorMap mk, mq, mv;
     if (!make_map_3d(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, BH, T, CDK, 64, true) ||
@@ -967,24 +968,21 @@ int launch_chunked_bv(const void* q, const void* k, const void* v, const float* 
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
         cudaSuccess)
         return DR_ERR_CUDA;
-    const int nc = dv / BV;
-    // sharing pays off while the owner's prep plus its copies fit in the two-chunk window
-    // the stage and slot rings allow; larger clusters measured slower
-    const int share = (MODE != DR_KDA && nc > 1 && nc <= 4) ? 1 : 0;
+    const int ny = dv / BV + (split ? 1 : 0);
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)BH, (unsigned)nc);
+    cfg.gridDim = dim3((unsigned)BH, (unsigned)ny);
     cfg.blockDim = dim3(CHUNK_THREADS);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
     attr[0].val.clusterDim.x = 1;
-    attr[0].val.clusterDim.y = share ? nc : 1;
+    attr[0].val.clusterDim.y = split ? ny : 1;
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = share ? 1 : 0;
+    cfg.numAttrs = split ? 1 : 0;
     if (cudaLaunchKernelEx(&cfg, kern, mk, mq, mv, beta, gate, S0,
-                           static_cast<__nv_bfloat16*>(out), S_final, T, dv, share) !=
+                           static_cast<__nv_bfloat16*>(out), S_final, T, dv, split) !=
         cudaSuccess)
         return DR_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? DR_OK : DR_ERR_CUDA;
@@ -1005,24 +1003,41 @@ inline int pick_bv(int variant, long BH, int dv) {
     return best;
 }
 
+// Split mode (a prep CTA plus dv/BV chain CTAs per head, one cluster per head) for the
+// scalar-gate variants when the heads are too few to fill the GPU otherwise: the slice
+// that gives the most chain CTAs while every cluster (<= 5 CTAs) is resident at once.
+// Returns the slice width, or 0 for the unsplit kernel.
+inline int pick_split_bv(int variant, long BH, int dv) {
+    if (variant == DR_KDA) return 0;
+    const int opts[3] = {16, 32, 64};
+    for (int i = 0; i < 3; ++i) {
+        const int bv = opts[i], ncc = dv / bv;
+        if (bv > dv || ncc < 2 || ncc > 4) continue;
+        if (BH * (ncc + 1) <= 148) return bv;
+    }
+    return 0;
+}
+
 template <int MODE>
 int launch_chunked_mode(const void* q, const void* k, const void* v, const float* beta,
                         const float* gate, const float* S0, void* out, float* S_final, int BH,
                         int T, int dv, cudaStream_t stream) {
-    switch (pick_bv(MODE, BH, dv)) {
+    const int split_bv = pick_split_bv(MODE, BH, dv);
+    const int split = split_bv ? 1 : 0;
+    switch (split ? split_bv : pick_bv(MODE, BH, dv)) {
         case 16:
             return launch_chunked_bv<MODE, 16>(q, k, v, beta, gate, S0, out, S_final, BH, T, dv,
-                                               stream);
+                                               split, stream);
         case 32:
             return launch_chunked_bv<MODE, 32>(q, k, v, beta, gate, S0, out, S_final, BH, T, dv,
-                                               stream);
+                                               split, stream);
         case 64:
             return launch_chunked_bv<MODE, 64>(q, k, v, beta, gate, S0, out, S_final, BH, T, dv,
-                                               stream);
+                                               split, stream);
         case 128:
             if constexpr (MODE == DR_KDA)
                 return launch_chunked_bv<MODE, 128>(q, k, v, beta, gate, S0, out, S_final, BH, T,
-                                                    dv, stream);
+                                                    dv, split, stream);
     }
     return DR_ERR_UNSUPPORTED;
 }
