@@ -77,8 +77,8 @@ struct ChunkLayout {
     static constexpr int KQ = 0;
     static constexpr int KN = KQ + NS * KQ_B;    // KDA: K/gamma, 2 panels x 64 rows
     static constexpr int SLOT = KN + NKN * 16384;
-    static constexpr int PM = SLOT + NP * SLOT_B;  // P: rows 0-63, rows 64-127 zero
-    static constexpr int TTS = PM + 16384;       // GDN: diag(gamma_C/gamma) T, 64 rows
+    static constexpr int PM = SLOT + NP * SLOT_B;  // P: 64 rows (A operand of an M=64 MMA)
+    static constexpr int TTS = PM + 8192;        // GDN: diag(gamma_C/gamma) T, 64 rows
     static constexpr int SS = TTS + (kGdn ? 8192 : 0);  // S bf16, M/N-major B operand
     static constexpr int SY = SS + SS_B;         // Y bf16, M/N-major B operand
     static constexpr int V = SY + SY_B;          // V stages: 64 rows x BV bf16
@@ -241,10 +241,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
         mbar_init_fence();
     }
     if (warp == 3) tmem_alloc(smem_u32(tmem_holder), L::NCOLS);
-    // P's rows 64-127 feed an M=128 MMA whose upper half is discarded, and the padding
-    // columns of S and Y are read by the chain MMAs: keep them zero.
-    for (int e = tid; e < 8192 / 16; e += CHUNK_THREADS)
-        reinterpret_cast<uint4*>(sm + L::PM + 8192)[e] = make_uint4(0, 0, 0, 0);
+    // The padding columns of S and Y are read by the chain MMAs: keep them zero.
     for (int e = tid; e < (L::SS_B + L::SY_B) / 16; e += CHUNK_THREADS)
         reinterpret_cast<uint4*>(sm + L::SS)[e] = make_uint4(0, 0, 0, 0);
     fence_async_smem();
@@ -390,7 +387,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
         // ------------------------------------------------------------------ prep MMA issuer
         if (lane == 0) {
             constexpr uint32_t idg = idesc_bf16(128, 64, 0, 0);
-            constexpr uint32_t idp = idesc_bf16(128, 64, 0, 1);
+            constexpr uint32_t idp = idesc_bf16(64, 64, 0, 1);  // D row m -> lane m%16 + 32*(m/16)
             constexpr uint32_t idh = idesc_bf16(128, 64, 1, 1);
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c % NS, p = c % NP;
@@ -886,12 +883,14 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 }
 #pragma unroll
                 for (int ch = 0; ch < 4; ++ch) st_row_chunk(kh, lq, c32 / 8 + ch, h + 8 * ch);
-                if (lq < 64) {
-                    tmem_ld16(trow + L::COL_G + c32, h);
-                    tmem_ld16(trow + L::COL_G + c32 + 16, h + 16);
-                    tmem_wait_ld();
+                // P T was an M=64 MMA: its row 16*q + l sits in lane l (< 16) of quadrant q
+                tmem_ld16(trow + L::COL_G + c32, h);
+                tmem_ld16(trow + L::COL_G + c32 + 16, h + 16);
+                tmem_wait_ld();
+                if ((lq & 31) < 16) {
+                    const int t = 16 * (lq >> 5) + (lq & 15);
 #pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) st_row_chunk(tp, 64 + lq, c32 / 8 + ch, h + 8 * ch);
+                    for (int ch = 0; ch < 4; ++ch) st_row_chunk(tp, 64 + t, c32 / 8 + ch, h + 8 * ch);
                 }
             }
             fence_async_smem();
