@@ -42,6 +42,8 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
+#include <algorithm>
+
 #include "common.cuh"
 
 namespace drscan {
@@ -82,7 +84,13 @@ struct ChunkLayout {
     static constexpr int SS = TTS + (kGdn ? 8192 : 0);  // S bf16, M/N-major B operand
     static constexpr int SY = SS + SS_B;         // Y bf16, M/N-major B operand
     static constexpr int V = SY + SY_B;          // V stages: 64 rows x BV bf16
-    static constexpr int AM = V + NSV * V_B;     // A, then X = (I+A)^{-1}: fp32 [64][68]
+    // In the prep CTA of a split cluster the chain region (S, Y, V) is unused and holds the
+    // temporaries of a second prep group: P, Ttilde, A/X, block scratch.
+    static constexpr int TMP_B = 8192 + 8192 + CK * 68 * 4 + 32 * 36 * 4;
+    static constexpr int CHAIN_USED = SS_B + SY_B + NSV * V_B;
+    static constexpr int CHAIN_B = (!kKda && CHAIN_USED < TMP_B) ? TMP_B : CHAIN_USED;
+    static constexpr int PM2 = SS, TTS2 = SS + 8192, AM2 = SS + 16384, ZS2 = AM2 + CK * 68 * 4;
+    static constexpr int AM = SS + CHAIN_B;      // A, then X = (I+A)^{-1}: fp32 [64][68]
     static constexpr int ZS = AM + CK * 68 * 4;  // block-product scratch: fp32 [32][36]
     static constexpr int GAM = ZS + 32 * 36 * 4;
     // per stage: beta[64]; GDN: g[64], 1/gamma[64], gamma[64] (cumulative log-decay and its
@@ -93,9 +101,10 @@ struct ChunkLayout {
     static constexpr int BAR = PG + 3072;
     static constexpr int TOTAL = BAR + 256;
     static_assert(TOTAL + 1024 <= 232448, "shared memory budget");
+    static_assert(NS % 2 == 0, "each of two prep groups owns whole K/Q stages");
 
-    static constexpr int COL_G = 0;   // D_G, then D_PT
-    static constexpr int COL_H = 64;  // D_H
+    static constexpr int COL_G = 0;   // D_G, then D_PT (second prep group: +128)
+    static constexpr int COL_H = 64;  // D_H (second prep group: +128)
     static constexpr int COL_D1 = 128;
     static constexpr int COL_D2 = 128 + NB;
     static constexpr int COL_S = 128 + 2 * NB;
@@ -118,8 +127,9 @@ enum ChunkBar {
     B_YREADY = 17,
     B_MMA23 = 18,
     B_STATE = 19,     // bf16 state copy ready for MMA1
-    B_PEER_FREE = 20,  // [2] owner side: the other CTAs of the cluster freed their slot
-    B_COUNT = 22
+    B_PEER_FREE = 20,  // [2] prep CTA: every chain CTA freed its copy of the slot
+    B_GRP1 = 22,       // second prep group's GO, GRAM, TREADY, HDONE (prep CTA of a split)
+    B_COUNT = 26
 };
 
 // bf16 bits of 8 consecutive columns of a row, stored as one 16-byte swizzled chunk.
@@ -182,7 +192,10 @@ __device__ __forceinline__ void store_neg_frag(float* m, int ld, int r0, int n0,
     m[(r0 + g + 8) * ld + n0 + 2 * tg + 1] = sign * d[3];
 }
 
-__device__ __forceinline__ void prep_sync() { asm volatile("bar.sync 1, 256;" ::: "memory"); }
+// Named barrier of one prep group (ids 1 and 3; id 2 belongs to the chain warpgroup).
+__device__ __forceinline__ void group_sync(int gi, int nthreads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(1 + 2 * gi), "r"(nthreads) : "memory");
+}
 
 template <int MODE, int BV>
 __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
@@ -208,15 +221,24 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
     const int lane = tid & 31;
     const long bh = blockIdx.x;
     const int nchunks = (T + CK - 1) / CK;
-    // With `split`, the CTAs of one head form a cluster: rank 0 prepares every chunk's
-    // operands ([T; PT], Khat^T, gamma) and copies them into the shared memory of ranks
-    // 1..NCC, each of which runs the chain for one slice of BV value channels. Without it,
-    // one CTA does both for its slice.
+    // With `split` = n > 0, the CTAs of one head form a cluster: ranks 0..n-1 prepare the
+    // chunks' operands ([T; PT], Khat^T, gamma), NGR consecutive chunks per rank in turn, and
+    // copy them into the shared memory of ranks n.., each of which runs the chain for one
+    // slice of BV value channels. Without it, one CTA does both for its slice.
+    const int NPREP = split ? split : 1;
+    const int NGR = (split && !kKda) ? 2 : 1;  // prep groups per prep CTA (KDA is never split)
+    const int SP = NGR * NPREP;                // chunk stride of one prep group
     const int rank = split ? (int)blockIdx.y : 0;
-    const int NCC = split ? (int)gridDim.y - 1 : 1;  // chain CTAs per head
-    const bool is_prep = !split || rank == 0;
-    const bool is_chain = !split || rank > 0;
-    const int v0 = (split ? rank - 1 : (int)blockIdx.y) * BV;
+    const int NCC = split ? (int)gridDim.y - NPREP : 1;  // chain CTAs per head
+    const bool is_prep = !split || rank < NPREP;
+    const bool is_chain = !split || rank >= NPREP;
+    const int v0 = (split ? rank - NPREP : (int)blockIdx.y) * BV;
+    // The chunks this CTA loads, in order: all of them, or (prep CTA of a split cluster)
+    // chunk_of(m) = base + (m / NGR) * SP + m % NGR; ordinal_of inverts it.
+    const int pG = is_chain ? 1 : NGR, pSP = is_chain ? 1 : SP, pbase = is_chain ? 0 : rank * NGR;
+    auto chunk_of = [&](int m) { return pbase + (m / pG) * pSP + m % pG; };
+    auto ordinal_of = [&](int c) { return ((c - pbase) / pSP) * pG + (c - pbase) % pG; };
+    auto owner_of = [&](int c) { return (c / NGR) % NPREP; };  // prep rank of chunk c
     auto slot = [&](int p) { return sm + L::SLOT + p * L::SLOT_B; };
 
     if (tid == 0) {
@@ -229,10 +251,15 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             mbar_init(bar(B_SLOT_EMPTY + s), 1);
             mbar_init(bar(B_PEER_FREE + s), split ? NCC : 1);
         }
-        mbar_init(bar(B_GO), 256);
+        const uint32_t gthreads = 256 / NGR;  // threads per prep group
+        mbar_init(bar(B_GO), gthreads);
         mbar_init(bar(B_GRAM), 1);
-        mbar_init(bar(B_TREADY), 256);
+        mbar_init(bar(B_TREADY), gthreads);
         mbar_init(bar(B_HDONE), 1);
+        mbar_init(bar(B_GRP1 + 0), gthreads);
+        mbar_init(bar(B_GRP1 + 1), 1);
+        mbar_init(bar(B_GRP1 + 2), gthreads);
+        mbar_init(bar(B_GRP1 + 3), 1);
         mbar_init(bar(B_MMA1), 1);
         mbar_init(bar(B_YREADY), 128);
         mbar_init(bar(B_MMA23), 1);
@@ -258,15 +285,29 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmV);
         }
-        for (int c = 0; c < nchunks; ++c) {
-            const int s = c % NS;
+        for (int m = 0;; ++m) {
+            const int c = chunk_of(m);
+            if (c >= nchunks) break;
+            const int s = m % NS;
             const int t0 = c * CK;
-            if (c >= NS) mbar_wait(bar(B_KQ_EMPTY + s), (uint32_t)(((c / NS) - 1) & 1), abort_flag);
-            float* bg = reinterpret_cast<float*>(sm + L::BG + s * L::BG_B);
-            for (int e = lane; e < CK; e += 32) {
-                const int t = t0 + e;
-                bg[e] = t < T ? beta[bh * T + t] : 0.f;
+            if (m >= NS) mbar_wait(bar(B_KQ_EMPTY + s), (uint32_t)(((m / NS) - 1) & 1), abort_flag);
+            // the tile loads go out first; the per-token scalars are computed while they fly
+            // and the stage completes with the second arrival
+            if (lane == 0 && !*abort_flag) {
+                uint8_t* kq = sm + L::KQ + s * L::KQ_B;
+                mbar_arrive_expect_tx(bar(B_KQ_FULL + s), L::KQ_B);
+                for (int p = 0; p < 2; ++p) {
+                    tma_load_3d(smem_u32(kq + p * 16384), &tmK, bar(B_KQ_FULL + s), p * 64, t0,
+                                (int)bh);
+                    tma_load_3d(smem_u32(kq + p * 16384 + 8192), &tmQ, bar(B_KQ_FULL + s), p * 64,
+                                t0, (int)bh);
+                }
+            } else if (lane == 0) {
+                mbar_arrive(bar(B_KQ_FULL + s));
             }
+            float* bg = reinterpret_cast<float*>(sm + L::BG + s * L::BG_B);
+            const float b0 = t0 + lane < T ? beta[bh * T + t0 + lane] : 0.f;
+            const float b1 = t0 + 32 + lane < T ? beta[bh * T + t0 + 32 + lane] : 0.f;
             if constexpr (kGdn) {
                 // g_t = sum of log alpha over the chunk's rows up to t (masked rows add 0)
                 float x0 = t0 + lane < T ? __logf(gate[bh * T + t0 + lane]) : 0.f;
@@ -288,23 +329,12 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 bg[192 + lane] = __expf(x0);
                 bg[224 + lane] = __expf(x1);
             }
+            bg[lane] = b0;
+            bg[32 + lane] = b1;
             __syncwarp();
-            if (lane == 0) {
-                if (!*abort_flag) {
-                    uint8_t* kq = sm + L::KQ + s * L::KQ_B;
-                    mbar_arrive_expect_tx(bar(B_KQ_FULL + s), L::KQ_B);
-                    for (int p = 0; p < 2; ++p) {
-                        tma_load_3d(smem_u32(kq + p * 16384), &tmK, bar(B_KQ_FULL + s), p * 64, t0,
-                                    (int)bh);
-                        tma_load_3d(smem_u32(kq + p * 16384 + 8192), &tmQ, bar(B_KQ_FULL + s),
-                                    p * 64, t0, (int)bh);
-                    }
-                }
-                mbar_arrive(bar(B_KQ_FULL + s));
-            }
+            if (lane == 0) mbar_arrive(bar(B_KQ_FULL + s));
         }
-    } else if (warp == 3) {
-        if (!is_chain) goto done;
+    } else if (warp == 3 && is_chain) {
         // ------------------------------------------------------------------ V producer
         if (lane == 0) {
             for (int c = 0; c < nchunks; ++c) {
@@ -323,14 +353,16 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
         // (prep CTA of a split cluster): ships each prepared slot to the chain CTAs once all
         // of them have freed their copy, then hands the slot back to the prep warps
         if (lane == 0) {
-            for (int c = 0; c < nchunks; ++c) {
+            for (int m = 0;; ++m) {
+                const int c = chunk_of(m);
+                if (c >= nchunks) break;
                 const int p = c % NP;
-                const uint32_t ph = (uint32_t)((c / NP) & 1);
+                const uint32_t ph = (uint32_t)((m / NP) & 1);
                 mbar_wait(bar(B_PREP + p), ph, abort_flag);
                 mbar_wait(bar(B_PEER_FREE + p), ph, abort_flag);
                 if (!*abort_flag) {
                     const uint32_t src = smem_u32(slot(p));
-                    for (int q = 1; q <= NCC; ++q)
+                    for (int q = NPREP; q < NPREP + NCC; ++q)  // the chain ranks
                         bulk_copy_to_peer(cluster_map(src, q), src, L::SLOT_B,
                                           cluster_map(bar(B_PREP + p), q));
                     bulk_commit_and_wait_read();
@@ -382,19 +414,26 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 }
             }
         }
-    } else if (warp == 2) {
-        if (!is_prep) goto done;
+    } else if (warp == 2 || warp == 3) {
         // ------------------------------------------------------------------ prep MMA issuer
+        // warp 2 serves prep group 0; warp 3 serves group 1 in the prep CTA of a split cluster
+        const int gi = warp - 2;
+        if (!is_prep || gi >= NGR) goto done;
         if (lane == 0) {
             constexpr uint32_t idg = idesc_bf16(128, 64, 0, 0);
             constexpr uint32_t idp = idesc_bf16(64, 64, 0, 1);  // D row m -> lane m%16 + 32*(m/16)
             constexpr uint32_t idh = idesc_bf16(128, 64, 1, 1);
-            for (int c = 0; c < nchunks; ++c) {
-                const int s = c % NS, p = c % NP;
+            const int gb = gi ? B_GRP1 : B_GO;
+            const uint32_t cg = L::COL_G + 128 * gi, chh = L::COL_H + 128 * gi;
+            uint8_t* pm = sm + (gi ? L::PM2 : L::PM);
+            uint8_t* tts = sm + (gi ? L::TTS2 : L::TTS);
+            int k = 0;  // the group's chunk ordinal
+            for (int c = pbase + gi; c < nchunks; c += SP, ++k) {
+                const int s = ordinal_of(c) % NS, p = c % NP;
                 uint8_t* kq = sm + L::KQ + s * L::KQ_B;
                 uint8_t* kn = sm + L::KN;
-                const uint32_t jp = (uint32_t)(c & 1);
-                mbar_wait(bar(B_GO), jp, abort_flag);
+                const uint32_t jp = (uint32_t)(k & 1);
+                mbar_wait(bar(gb + 0), jp, abort_flag);
                 tc_fence_after();
                 if (!*abort_flag) {
 #pragma unroll
@@ -403,33 +442,31 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                         const uint64_t a = smem_desc_sw128(smem_u32(kq + pn * 16384 + ko), 16, 1024);
                         const uint64_t b =
                             kKda ? smem_desc_sw128(smem_u32(kn + pn * 8192 + ko), 16, 1024) : a;
-                        tc_mma_bf16(tmem + L::COL_G, a, b, idg, kk > 0);
+                        tc_mma_bf16(tmem + cg, a, b, idg, kk > 0);
                     }
-                    tc_commit(bar(B_GRAM));
+                    tc_commit(bar(gb + 1));
                 }
-                mbar_wait(bar(B_TREADY), jp, abort_flag);
+                mbar_wait(bar(gb + 2), jp, abort_flag);
                 tc_fence_after();
                 if (!*abort_flag) {
                     const uint8_t* tp = slot(p) + L::SLOT_TP;
                     // PT = P T: B = T read M/N-major from the slot's rows 0-63
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk)
-                        tc_mma_bf16(tmem + L::COL_G,
-                                    smem_desc_sw128(smem_u32(sm + L::PM + kk * 32), 16, 1024),
-                                    smem_desc_sw128(smem_u32(tp + kk * 2048), 1024, 1024), idp,
-                                    kk > 0);
+                        tc_mma_bf16(tmem + cg, smem_desc_sw128(smem_u32(pm + kk * 32), 16, 1024),
+                                    smem_desc_sw128(smem_u32(tp + kk * 2048), 1024, 1024), idp, kk > 0);
                     // H: A = K^T (KDA: (K/g)^T) M/N-major, B = Ttilde (or T) M/N-major
-                    const uint8_t* bt = kGdn ? sm + L::TTS : tp;
+                    const uint8_t* bt = kGdn ? tts : tp;
 #pragma unroll
                     for (int kk = 0; kk < 4; ++kk) {
                         const uint64_t a =
                             kKda ? smem_desc_sw128(smem_u32(kn + kk * 2048), 8192, 1024)
                                  : smem_desc_sw128(smem_u32(kq + kk * 2048), 16384, 1024);
-                        tc_mma_bf16(tmem + L::COL_H, a,
+                        tc_mma_bf16(tmem + chh, a,
                                     smem_desc_sw128(smem_u32(bt + kk * 2048), 1024, 1024), idh,
                                     kk > 0);
                     }
-                    tc_commit(bar(B_HDONE));
+                    tc_commit(bar(gb + 3));
                     tc_commit(bar(B_KQ_EMPTY + s));
                 }
             }
@@ -461,7 +498,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             if (r == 0 && split) {
                 for (int c = 0; c < NP && c < nchunks; ++c) {
                     mbar_arrive_expect_tx(bar(B_PREP + c), L::SLOT_B);
-                    mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + c), 0));
+                    mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + c), owner_of(c)));
                 }
             }
         }
@@ -583,7 +620,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     mbar_arrive(bar(B_SLOT_EMPTY + p));
                 } else {
                     mbar_arrive_expect_tx(bar(B_PREP + p), L::SLOT_B);
-                    mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + p), 0));
+                    mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + p), owner_of(c + NP)));
                 }
             }
             if (c + 1 < nchunks) prescale(c + 1);
@@ -591,16 +628,26 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
     } else if (warp >= 8) {
         if (!is_prep) goto done;
         // ------------------------------------------------------------------ prep warps
-        // u: 0..255. Lane-mapped work uses TMEM lane lq = u % 128 and column half hf = u / 128
-        // (warp 8+i reaches TMEM lanes 32*(i%4) .. +31).
-        const int u = tid - 256;
-        const int lq = u & 127, hf = u >> 7;
-        const uint32_t trow = tmem + ((uint32_t)(lq & ~31) << 16);
-        const int wq = u >> 5, g8 = lane >> 2, tg = lane & 3;
-        // KDA scan exchange: pg[128*q + ch] = product over row quarter q; gamma_C at pg[512 + ch]
+        // Without `split`, warps 8-15 form one prep group. In the prep CTA of a split cluster
+        // they form two groups of four warps (8-11 and 12-15) that take alternate chunks, each
+        // with its own TMEM columns, temporaries, mbarriers and named barrier. Group-local
+        // thread u; lq = the TMEM lane this thread reaches (warp 8+i reaches 32*(i%4) .. +31).
+        const int GT = 256 / NGR;                 // threads per group
+        const int HSTEP = GT / 128;               // column halves a thread steps over
+        const int gi = (tid - 256) / GT;
+        const int u = (tid - 256) - gi * GT;
+        const int lq = (tid - 256) & 127;
+        const int wq = u >> 5, GW = GT >> 5, g8 = lane >> 2, tg = lane & 3;
+        const uint32_t trow = tmem + 128 * gi + ((uint32_t)(lq & ~31) << 16);
+        const int gb = gi ? B_GRP1 : B_GO;
+        uint8_t* pm = sm + (gi ? L::PM2 : L::PM);
+        uint8_t* tts = sm + (gi ? L::TTS2 : L::TTS);
+        float* sA = reinterpret_cast<float*>(sm + (gi ? L::AM2 : L::AM));
+        float* sZ = reinterpret_cast<float*>(sm + (gi ? L::ZS2 : L::ZS));
+        auto gsync = [&]() { group_sync(gi, GT); };
+        // KDA (always one group) scan exchange: pg[128*q + ch] = product over row quarter q;
+        // gamma_C at pg[512 + ch]
         float* pg = reinterpret_cast<float*>(sm + L::PG);
-        float* sA = reinterpret_cast<float*>(sm + L::AM);
-        float* sZ = reinterpret_cast<float*>(sm + L::ZS);
         // KDA: thread u owns key channels 2*(u%64), 2*(u%64)+1 on rows 16*(u/64) .. +15 of a
         // chunk; the next owned chunk's alpha values are prefetched into registers.
         const int kc = 2 * (u & 63), kq4 = u >> 6;
@@ -613,18 +660,18 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                                : make_float2(1.f, 1.f);
             }
         }
-        int kq_seen = 0;  // K/Q stage phases waited so far (every chunk, in order)
-        for (int c = 0; c < nchunks; ++c) {
-            const int s = c % NS, p = c % NP;
-            const uint32_t jp = (uint32_t)(c & 1);
+        int k = 0;  // the group's chunk ordinal
+        for (int c = pbase + gi; c < nchunks; c += SP, ++k) {
+            const int mo = ordinal_of(c);  // position among the chunks this CTA loads
+            const int s = mo % NS, p = c % NP;
+            const uint32_t jp = (uint32_t)(k & 1);
             const int t0 = c * CK;
             const int nvalid = min(CK, T - t0);
             uint8_t* kq = sm + L::KQ + s * L::KQ_B;
             const float* bg = reinterpret_cast<const float*>(sm + L::BG + s * L::BG_B);
-            // A parity wait cannot tell "this phase done" from "the previous phase still
-            // pending", so the stages' phases are walked in order, owned chunk or not.
-            for (; kq_seen <= c; ++kq_seen)
-                mbar_wait(bar(B_KQ_FULL + kq_seen % NS), (uint32_t)((kq_seen / NS) & 1), abort_flag);
+            // NGR divides NS, so a group waits on every phase of the stages it reads, in order
+            // (a parity wait cannot tell a completed phase from the one before it still pending)
+            mbar_wait(bar(B_KQ_FULL + s), (uint32_t)((mo / NS) & 1), abort_flag);
 
             // ---- 1. gates. GDN: g, 1/gamma, gamma come from the producer; the factored form
             // gamma_t * (1/gamma_i) of exp(g_t - g_i) is used when it cannot overflow.
@@ -644,7 +691,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     }
                 }
                 if (kq4 < 3) *reinterpret_cast<float2*>(pg + 128 * kq4 + kc) = part;
-                prep_sync();
+                gsync();
                 float2 run = make_float2(1.f, 1.f);
                 for (int q = 0; q < kq4; ++q) {
                     const float2 pq = *reinterpret_cast<const float2*>(pg + 128 * q + kc);
@@ -681,21 +728,21 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 if (kq4 == 3) *reinterpret_cast<float2*>(pg + 512 + kc) = run;  // gamma_C
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const int tn = t0 + CK + 16 * kq4 + i;
+                    const int tn = (c + SP) * CK + 16 * kq4 + i;
                     gpf[i] = tn < T ? *reinterpret_cast<const float2*>(gate + (bh * T + tn) * (long)CDK + kc)
                                     : make_float2(1.f, 1.f);
                 }
                 fence_async_smem();
-                prep_sync();
+                gsync();
             }
             tc_fence_before();
-            mbar_arrive(bar(B_GO));
+            mbar_arrive(bar(gb + 0));
 
-            // ---- 2. Gram epilogue: A (fp32, rows 0-63) and P (bf16, rows 0-63 of PM); each
-            // thread takes one half (32 columns) of one row
-            mbar_wait(bar(B_GRAM), jp, abort_flag);
+            // ---- 2. Gram epilogue: A (fp32, rows 0-63) and P (bf16, rows 0-63 of pm); a
+            // thread takes one or both 32-column halves of TMEM row lq
+            mbar_wait(bar(gb + 1), jp, abort_flag);
             tc_fence_after();
-            {
+            for (int hf = u >> 7; hf < 2; hf += HSTEP) {
                 const int t = lq & 63;
                 const int c32 = 32 * hf;
                 float rowf = (lq < 64) ? bg[t] : 1.f;  // beta_t on A rows
@@ -739,10 +786,10 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                             make_float4(gr[e], gr[e + 1], gr[e + 2], gr[e + 3]);
                 } else {
 #pragma unroll
-                    for (int ch = 0; ch < 4; ++ch) st_row_chunk(sm + L::PM, t, c32 / 8 + ch, gr + 8 * ch);
+                    for (int ch = 0; ch < 4; ++ch) st_row_chunk(pm, t, c32 / 8 + ch, gr + 8 * ch);
                 }
             }
-            prep_sync();
+            gsync();
 
             // ---- 3. X = (I + A)^{-1}, in place in sA
             float xcol[16];
@@ -756,13 +803,13 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     for (int t = i + 1; t < 16; ++t)
                         xcol[t] = fmaf(-sA[(16 * b + t) * 68 + 16 * b + i], xcol[i], xcol[t]);
             }
-            prep_sync();
+            gsync();
             if (u < 64) {
                 const int b = u >> 4, cc = u & 15;
 #pragma unroll
                 for (int t = 0; t < 16; ++t) sA[(16 * b + t) * 68 + 16 * b + cc] = xcol[t];
             }
-            prep_sync();
+            gsync();
             if (wq < 2) {  // X(b+1,b) = -X(b+1,b+1) A(b+1,b) X(b,b) for b = 0, 2
                 const int b0 = 32 * wq, b1 = b0 + 16;
                 float* z = sZ + wq * 16 * 20;
@@ -795,10 +842,11 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 for (int nt = 0; nt < 2; ++nt)
                     store_neg_frag(sA, 68, b1, b0 + 8 * nt, acc2[nt], g8, tg, -1.f);
             }
-            prep_sync();
-            {  // X[32:64, 0:32] = -X[32:64, 32:64] A[32:64, 0:32] X[0:32, 0:32]; one 16x8 tile
-               // of each product per warp
-                const int m0 = 32 + 16 * (wq >> 2), n0 = 8 * (wq & 3);
+            gsync();
+            // X[32:64, 0:32] = -X[32:64, 32:64] A[32:64, 0:32] X[0:32, 0:32], in eight 16x8
+            // tiles per product, spread over the group's warps
+            for (int tile = wq; tile < 8; tile += GW) {
+                const int m0 = 32 + 16 * (tile >> 2), n0 = 8 * (tile & 3);
                 float acc[4] = {};
 #pragma unroll
                 for (int kk = 0; kk < 32; kk += 8) {
@@ -808,7 +856,10 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     mma_tf32(acc, a, bb);
                 }
                 store_neg_frag(sZ, 36, m0 - 32, n0, acc, g8, tg, 1.f);
-                prep_sync();
+            }
+            gsync();
+            for (int tile = wq; tile < 8; tile += GW) {
+                const int m0 = 32 + 16 * (tile >> 2), n0 = 8 * (tile & 3);
                 float acc2[4] = {};
 #pragma unroll
                 for (int kk = 0; kk < 32; kk += 8) {
@@ -819,25 +870,25 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 }
                 store_neg_frag(sA, 68, m0, n0, acc2, g8, tg, -1.f);
             }
-            prep_sync();
+            gsync();
 
-            // ---- 4. stage T = X diag(beta) into the slot (and Ttilde for GDN's H): thread u
-            // writes half (u/64 % 2) of row u % 64 of T (u < 128) or of Ttilde (u >= 128)
-            if (c >= NP) {
-                // the previous use of slot p (chunk c - NP) must be finished: by this CTA's
-                // chain, or (split) by the distributor's copies to the chain CTAs
-                mbar_wait(bar(B_SLOT_EMPTY + p), (uint32_t)(((c / NP) - 1) & 1), abort_flag);
+            // ---- 4. stage T = X diag(beta) into the slot (and Ttilde for GDN's H): virtual
+            // thread v writes half (v/64 % 2) of row v % 64 of T (v < 128) or of Ttilde
+            if (mo >= NP) {
+                // the previous use of slot p must be finished: by this CTA's chain, or (split)
+                // by the distributor's copies to the chain CTAs
+                mbar_wait(bar(B_SLOT_EMPTY + p), (uint32_t)(((mo / NP) - 1) & 1), abort_flag);
             }
             uint8_t* tp = slot(p) + L::SLOT_TP;
             float* gam = reinterpret_cast<float*>(slot(p) + L::SLOT_GAM);
-            {
-                const int t = u & 63, half = (u >> 6) & 1;
+            for (int v = u; v < 256; v += GT) {
+                const int t = v & 63, half = (v >> 6) & 1;
                 float scale = 1.f;
                 uint8_t* dst = tp;
-                if (u >= 128) {
+                if (v >= 128) {
                     if constexpr (kGdn) {
                         scale = __expf(bg[64 + 63] - bg[64 + t]);  // gamma_C / gamma_t
-                        dst = sm + L::TTS;
+                        dst = tts;
                     } else {
                         dst = nullptr;
                     }
@@ -857,19 +908,19 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     for (int ch = 0; ch < 4; ++ch) st_row_chunk(dst, t, 4 * half + ch, row + 8 * ch);
                 }
                 if constexpr (kGdn) {
-                    if (u < 64) gam[u] = bg[192 + u];
-                    if (u == 64) gam[64] = bg[192 + 63];
+                    if (v < 64) gam[v] = bg[192 + v];
+                    if (v == 64) gam[64] = bg[192 + 63];
                 } else if constexpr (kKda) {
-                    if (u < 128) gam[u] = pg[512 + u];
+                    if (v < 128) gam[v] = pg[512 + v];
                 }
             }
             fence_async_smem();
-            mbar_arrive(bar(B_TREADY));
+            mbar_arrive(bar(gb + 2));
 
-            // ---- 5. Khat^T -> slot (row lq, column half hf); PT rows -> slot rows 64-127
-            mbar_wait(bar(B_HDONE), jp, abort_flag);
+            // ---- 5. Khat^T -> slot (row lq); PT rows -> slot rows 64-127
+            mbar_wait(bar(gb + 3), jp, abort_flag);
             tc_fence_after();
-            {
+            for (int hf = u >> 7; hf < 2; hf += HSTEP) {
                 uint8_t* kh = slot(p) + L::SLOT_KH;
                 const int c32 = 32 * hf;
                 float h[32];
@@ -895,7 +946,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             }
             fence_async_smem();
             tc_fence_before();
-            prep_sync();
+            gsync();
             if (u == 0) mbar_arrive(bar(B_PREP + p));
         }
     }
@@ -967,7 +1018,7 @@ int launch_chunked_bv(const void* q, const void* k, const void* v, const float* 
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
         cudaSuccess)
         return DR_ERR_CUDA;
-    const int ny = dv / BV + (split ? 1 : 0);
+    const int ny = dv / BV + split;  // split = prep CTAs per head (0: unsplit)
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)BH, (unsigned)ny);
     cfg.blockDim = dim3(CHUNK_THREADS);
@@ -1002,28 +1053,49 @@ inline int pick_bv(int variant, long BH, int dv) {
     return best;
 }
 
-// Split mode (a prep CTA plus dv/BV chain CTAs per head, one cluster per head) for the
-// scalar-gate variants when the heads are too few to fill the GPU otherwise: the slice
-// that gives the most chain CTAs while every cluster (<= 5 CTAs) is resident at once.
-// Returns the slice width, or 0 for the unsplit kernel.
-inline int pick_split_bv(int variant, long BH, int dv) {
-    if (variant == DR_KDA) return 0;
-    const int opts[3] = {16, 32, 64};
+// Split mode (a cluster per head of `nprep` prep CTAs and dv/BV chain CTAs) for the
+// scalar-gate variants when the heads are too few to fill the GPU otherwise. The plan
+// minimises an estimate of the per-chunk period, in thousands of cycles measured on B200:
+// the chain step (grows with BV), one prep group's latency shared by 2*nprep groups, and the
+// distributor's copies (grow with the chain CTAs) shared by nprep prep CTAs; ties go to the
+// plan with fewer CTAs. Every cluster (<= 8 CTAs) and the whole grid must be resident at once.
+struct SplitPlan {
+    int bv = 0, nprep = 0;  // nprep == 0: unsplit
+};
+
+inline SplitPlan pick_split(int variant, long BH, int dv) {
+    SplitPlan best;
+    if (variant == DR_KDA) return best;
+    double best_t = 7.7;  // unsplit period with one CTA per (head, slice), grid permitting
+    int best_ctas = 1 << 30;
+    const int bvs[3] = {16, 32, 64};
+    const double chain_k[3] = {2.8, 3.2, 3.8};
     for (int i = 0; i < 3; ++i) {
-        const int bv = opts[i], ncc = dv / bv;
-        if (bv > dv || ncc < 2 || ncc > 4) continue;
-        if (BH * (ncc + 1) <= 148) return bv;
+        const int bv = bvs[i], ncc = dv / bv;
+        if (bv > dv || ncc < 2) continue;
+        for (int np = 1; np <= 4; ++np) {
+            const long ctas = BH * (np + ncc);
+            if (np + ncc > 8 || ctas > 148) continue;
+            const double prep = 12.0 / (2 * np), copy = (2.6 + 0.5 * ncc) / np;
+            const double t = std::max(chain_k[i], std::max(prep, copy));
+            if (t < best_t - 0.05 || (t < best_t + 0.05 && ctas < best_ctas)) {
+                best_t = std::min(t, best_t);
+                best_ctas = (int)ctas;
+                best.bv = bv;
+                best.nprep = np;
+            }
+        }
     }
-    return 0;
+    return best;
 }
 
 template <int MODE>
 int launch_chunked_mode(const void* q, const void* k, const void* v, const float* beta,
                         const float* gate, const float* S0, void* out, float* S_final, int BH,
                         int T, int dv, cudaStream_t stream) {
-    const int split_bv = pick_split_bv(MODE, BH, dv);
-    const int split = split_bv ? 1 : 0;
-    switch (split ? split_bv : pick_bv(MODE, BH, dv)) {
+    const SplitPlan plan = pick_split(MODE, BH, dv);
+    const int split = plan.nprep;
+    switch (split ? plan.bv : pick_bv(MODE, BH, dv)) {
         case 16:
             return launch_chunked_bv<MODE, 16>(q, k, v, beta, gate, S0, out, S_final, BH, T, dv,
                                                split, stream);
