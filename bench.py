@@ -101,7 +101,8 @@ def aggregate_value(world: int, head_tokens: int, steps: int, total_ms_max: floa
 # keyed by workload and the sha256 prefix of the chunked kernel's source at capture time; a
 # changed source reports null. Summaries with the commands are under profiles/.
 NCU_TRAFFIC = {
-    ("gdn_bf16", "63949d27f35ae68e"): 119961088,
+    ("gdn_bf16", "985582a75d01dcf3"): 101797888 + 13434880,
+    ("kda_bf16", "985582a75d01dcf3"): 673565696 + 120207104,
 }
 
 

@@ -42,7 +42,6 @@
 #include <cuda.h>
 #include <cudaTypedefs.h>
 
-#include <algorithm>
 
 #include "common.cuh"
 
@@ -197,12 +196,12 @@ __device__ __forceinline__ void group_sync(int gi, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(1 + 2 * gi), "r"(nthreads) : "memory");
 }
 
-template <int MODE, int BV>
+template <int MODE, int BV, bool SPLIT>
 __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
     const __grid_constant__ CUtensorMap tmV, const float* __restrict__ beta,
     const float* __restrict__ gate, const float* __restrict__ S0,
-    __nv_bfloat16* __restrict__ out, float* __restrict__ S_final, int T, int dv, int split) {
+    __nv_bfloat16* __restrict__ out, float* __restrict__ S_final, int T, int dv, int nprep) {
     using L = ChunkLayout<MODE, BV>;
     constexpr bool kGdn = MODE == DR_GDN;
     constexpr bool kKda = MODE == DR_KDA;
@@ -221,12 +220,14 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
     const int lane = tid & 31;
     const long bh = blockIdx.x;
     const int nchunks = (T + CK - 1) / CK;
-    // With `split` = n > 0, the CTAs of one head form a cluster: ranks 0..n-1 prepare the
-    // chunks' operands ([T; PT], Khat^T, gamma), NGR consecutive chunks per rank in turn, and
-    // copy them into the shared memory of ranks n.., each of which runs the chain for one
-    // slice of BV value channels. Without it, one CTA does both for its slice.
-    const int NPREP = split ? split : 1;
-    const int NGR = (split && !kKda) ? 2 : 1;  // prep groups per prep CTA (KDA is never split)
+    // SPLIT: the CTAs of one head form a cluster; ranks 0..nprep-1 prepare the chunks'
+    // operands ([T; PT], Khat^T, gamma), NGR consecutive chunks per rank in turn, and copy
+    // them into the shared memory of ranks nprep.., each of which runs the chain for one
+    // slice of BV value channels. Otherwise one CTA does both for its slice.
+    static_assert(!(SPLIT && kKda), "KDA is never split");
+    constexpr bool split = SPLIT;
+    const int NPREP = SPLIT ? nprep : 1;
+    constexpr int NGR = SPLIT ? 2 : 1;  // prep groups per prep CTA
     const int SP = NGR * NPREP;                // chunk stride of one prep group
     const int rank = split ? (int)blockIdx.y : 0;
     const int NCC = split ? (int)gridDim.y - NPREP : 1;  // chain CTAs per head
@@ -274,7 +275,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
     fence_async_smem();
     tc_fence_before();
     __syncthreads();
-    if (split) cluster_sync_all();  // peers' barriers are initialised before any remote arrive
+    if constexpr (SPLIT) cluster_sync_all();  // peers' barriers are initialised before any remote arrive
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
@@ -632,12 +633,12 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
         // they form two groups of four warps (8-11 and 12-15) that take alternate chunks, each
         // with its own TMEM columns, temporaries, mbarriers and named barrier. Group-local
         // thread u; lq = the TMEM lane this thread reaches (warp 8+i reaches 32*(i%4) .. +31).
-        const int GT = 256 / NGR;                 // threads per group
-        const int HSTEP = GT / 128;               // column halves a thread steps over
+        constexpr int GT = 256 / NGR;  // threads per group; each loop below runs NGR times
         const int gi = (tid - 256) / GT;
         const int u = (tid - 256) - gi * GT;
         const int lq = (tid - 256) & 127;
-        const int wq = u >> 5, GW = GT >> 5, g8 = lane >> 2, tg = lane & 3;
+        constexpr int GW = GT >> 5;
+        const int wq = u >> 5, g8 = lane >> 2, tg = lane & 3;
         const uint32_t trow = tmem + 128 * gi + ((uint32_t)(lq & ~31) << 16);
         const int gb = gi ? B_GRP1 : B_GO;
         uint8_t* pm = sm + (gi ? L::PM2 : L::PM);
@@ -742,7 +743,9 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             // thread takes one or both 32-column halves of TMEM row lq
             mbar_wait(bar(gb + 1), jp, abort_flag);
             tc_fence_after();
-            for (int hf = u >> 7; hf < 2; hf += HSTEP) {
+#pragma unroll
+            for (int i = 0; i < NGR; ++i) {
+                const int hf = (u >> 7) + i;  // column half
                 const int t = lq & 63;
                 const int c32 = 32 * hf;
                 float rowf = (lq < 64) ? bg[t] : 1.f;  // beta_t on A rows
@@ -845,7 +848,9 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             gsync();
             // X[32:64, 0:32] = -X[32:64, 32:64] A[32:64, 0:32] X[0:32, 0:32], in eight 16x8
             // tiles per product, spread over the group's warps
-            for (int tile = wq; tile < 8; tile += GW) {
+#pragma unroll
+            for (int i = 0; i < NGR; ++i) {
+                const int tile = wq + i * GW;
                 const int m0 = 32 + 16 * (tile >> 2), n0 = 8 * (tile & 3);
                 float acc[4] = {};
 #pragma unroll
@@ -858,7 +863,9 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 store_neg_frag(sZ, 36, m0 - 32, n0, acc, g8, tg, 1.f);
             }
             gsync();
-            for (int tile = wq; tile < 8; tile += GW) {
+#pragma unroll
+            for (int i = 0; i < NGR; ++i) {
+                const int tile = wq + i * GW;
                 const int m0 = 32 + 16 * (tile >> 2), n0 = 8 * (tile & 3);
                 float acc2[4] = {};
 #pragma unroll
@@ -881,7 +888,9 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             }
             uint8_t* tp = slot(p) + L::SLOT_TP;
             float* gam = reinterpret_cast<float*>(slot(p) + L::SLOT_GAM);
-            for (int v = u; v < 256; v += GT) {
+#pragma unroll
+            for (int i = 0; i < NGR; ++i) {
+                const int v = u + i * GT;
                 const int t = v & 63, half = (v >> 6) & 1;
                 float scale = 1.f;
                 uint8_t* dst = tp;
@@ -920,7 +929,9 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             // ---- 5. Khat^T -> slot (row lq); PT rows -> slot rows 64-127
             mbar_wait(bar(gb + 3), jp, abort_flag);
             tc_fence_after();
-            for (int hf = u >> 7; hf < 2; hf += HSTEP) {
+#pragma unroll
+            for (int i = 0; i < NGR; ++i) {
+                const int hf = (u >> 7) + i;  // column half
                 uint8_t* kh = slot(p) + L::SLOT_KH;
                 const int c32 = 32 * hf;
                 float h[32];
@@ -961,7 +972,7 @@ done:
         }
     }
     __syncthreads();
-    if (split) cluster_sync_all();  // no CTA leaves while the others may still address it
+    if constexpr (SPLIT) cluster_sync_all();  // no CTA leaves while the others may still address it
     tc_fence_after();
     if (warp == 3) tmem_dealloc(tmem, L::NCOLS);
 }
@@ -1003,10 +1014,10 @@ inline bool chunked_supported(int variant, int dk, int dv) {
            (variant == DR_DELTANET || variant == DR_GDN || variant == DR_KDA);
 }
 
-template <int MODE, int BV>
+template <int MODE, int BV, bool SPLIT>
 int launch_chunked_bv(const void* q, const void* k, const void* v, const float* beta,
                       const float* gate, const float* S0, void* out, float* S_final, int BH, int T,
-                      int dv, int split, cudaStream_t stream) {
+                      int dv, int nprep, cudaStream_t stream) {
     using L = ChunkLayout<MODE, BV>;
     CUtensorMap mk, mq, mv;
     if (!make_map_3d(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, BH, T, CDK, 64, true) ||
@@ -1014,11 +1025,12 @@ int launch_chunked_bv(const void* q, const void* k, const void* v, const float* 
         !make_map_3d(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, BH, T, dv, BV, false))
         return DR_ERR_CUDA;
     const int smem = L::TOTAL + 1024;
-    auto kern = dr_chunked_kernel<MODE, BV>;
+    auto kern = dr_chunked_kernel<MODE, BV, SPLIT>;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
         cudaSuccess)
         return DR_ERR_CUDA;
-    const int ny = dv / BV + split;  // split = prep CTAs per head (0: unsplit)
+    const int split = SPLIT ? nprep : 0;  // prep CTAs per head
+    const int ny = dv / BV + split;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)BH, (unsigned)ny);
     cfg.blockDim = dim3(CHUNK_THREADS);
@@ -1053,40 +1065,59 @@ inline int pick_bv(int variant, long BH, int dv) {
     return best;
 }
 
+// Clusters of `size` CTAs of the chunked kernel (one CTA per SM) that can be resident at
+// once on the current device; cached per device.
+inline int max_active_clusters(int size) {
+    static int cache[16][9] = {};
+    int dev = 0;
+    if (size < 1 || size > 8 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16)
+        return 0;
+    if (cache[dev][size] == 0) {
+        using L = ChunkLayout<DR_GDN, 64>;
+        auto kern = dr_chunked_kernel<DR_GDN, 64, true>;
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(1, (unsigned)size);
+        cfg.blockDim = dim3(CHUNK_THREADS);
+        cfg.dynamicSmemBytes = L::TOTAL + 1024;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 1;
+        attr[0].val.clusterDim.y = (unsigned)size;
+        attr[0].val.clusterDim.z = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        int n = 0;
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 L::TOTAL + 1024) != cudaSuccess ||
+            cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess)
+            n = -1;
+        cache[dev][size] = n;
+    }
+    return cache[dev][size] > 0 ? cache[dev][size] : 0;
+}
+
 // Split mode (a cluster per head of `nprep` prep CTAs and dv/BV chain CTAs) for the
-// scalar-gate variants when the heads are too few to fill the GPU otherwise. The plan
-// minimises an estimate of the per-chunk period, in thousands of cycles measured on B200:
-// the chain step (grows with BV), one prep group's latency shared by 2*nprep groups, and the
-// distributor's copies (grow with the chain CTAs) shared by nprep prep CTAs; ties go to the
-// plan with fewer CTAs. Every cluster (<= 8 CTAs) and the whole grid must be resident at once.
+// scalar-gate variants when the heads are too few to fill the GPU otherwise. Measured on
+// B200 (GDN, dk = dv = 128, T = 4096): two chain CTAs per head (BV = dv/2) beat four, whose
+// extra slot copies cost more than their shorter chain saves; two prep CTAs beat one and
+// match three or four. Every cluster must be resident at once (clusters of 7-8 CTAs fit 15
+// at a time on B200, which puts 16 heads into two waves) and the grid must fit 148 SMs.
 struct SplitPlan {
     int bv = 0, nprep = 0;  // nprep == 0: unsplit
 };
 
 inline SplitPlan pick_split(int variant, long BH, int dv) {
-    SplitPlan best;
-    if (variant == DR_KDA) return best;
-    double best_t = 7.7;  // unsplit period with one CTA per (head, slice), grid permitting
-    int best_ctas = 1 << 30;
-    const int bvs[3] = {16, 32, 64};
-    const double chain_k[3] = {2.8, 3.2, 3.8};
-    for (int i = 0; i < 3; ++i) {
-        const int bv = bvs[i], ncc = dv / bv;
-        if (bv > dv || ncc < 2) continue;
-        for (int np = 1; np <= 4; ++np) {
-            const long ctas = BH * (np + ncc);
-            if (np + ncc > 8 || ctas > 148) continue;
-            const double prep = 12.0 / (2 * np), copy = (2.6 + 0.5 * ncc) / np;
-            const double t = std::max(chain_k[i], std::max(prep, copy));
-            if (t < best_t - 0.05 || (t < best_t + 0.05 && ctas < best_ctas)) {
-                best_t = std::min(t, best_t);
-                best_ctas = (int)ctas;
-                best.bv = bv;
-                best.nprep = np;
-            }
+    SplitPlan plan;
+    if (variant == DR_KDA || dv < 32) return plan;
+    const int bv = dv / 2, ncc = 2;
+    for (int np = 2; np >= 1; --np) {
+        if (BH * (np + ncc) <= 148 && BH <= max_active_clusters(np + ncc)) {
+            plan.bv = bv;
+            plan.nprep = np;
+            break;
         }
     }
-    return best;
+    return plan;
 }
 
 template <int MODE>
@@ -1094,21 +1125,36 @@ int launch_chunked_mode(const void* q, const void* k, const void* v, const float
                         const float* gate, const float* S0, void* out, float* S_final, int BH,
                         int T, int dv, cudaStream_t stream) {
     const SplitPlan plan = pick_split(MODE, BH, dv);
-    const int split = plan.nprep;
-    switch (split ? plan.bv : pick_bv(MODE, BH, dv)) {
+    if constexpr (MODE != DR_KDA) {
+        if (plan.nprep > 0) {
+            switch (plan.bv) {
+                case 16:
+                    return launch_chunked_bv<MODE, 16, true>(q, k, v, beta, gate, S0, out, S_final,
+                                                             BH, T, dv, plan.nprep, stream);
+                case 32:
+                    return launch_chunked_bv<MODE, 32, true>(q, k, v, beta, gate, S0, out, S_final,
+                                                             BH, T, dv, plan.nprep, stream);
+                case 64:
+                    return launch_chunked_bv<MODE, 64, true>(q, k, v, beta, gate, S0, out, S_final,
+                                                             BH, T, dv, plan.nprep, stream);
+            }
+            return DR_ERR_UNSUPPORTED;
+        }
+    }
+    switch (pick_bv(MODE, BH, dv)) {
         case 16:
-            return launch_chunked_bv<MODE, 16>(q, k, v, beta, gate, S0, out, S_final, BH, T, dv,
-                                               split, stream);
+            return launch_chunked_bv<MODE, 16, false>(q, k, v, beta, gate, S0, out, S_final, BH, T,
+                                                      dv, 0, stream);
         case 32:
-            return launch_chunked_bv<MODE, 32>(q, k, v, beta, gate, S0, out, S_final, BH, T, dv,
-                                               split, stream);
+            return launch_chunked_bv<MODE, 32, false>(q, k, v, beta, gate, S0, out, S_final, BH, T,
+                                                      dv, 0, stream);
         case 64:
-            return launch_chunked_bv<MODE, 64>(q, k, v, beta, gate, S0, out, S_final, BH, T, dv,
-                                               split, stream);
+            return launch_chunked_bv<MODE, 64, false>(q, k, v, beta, gate, S0, out, S_final, BH, T,
+                                                      dv, 0, stream);
         case 128:
             if constexpr (MODE == DR_KDA)
-                return launch_chunked_bv<MODE, 128>(q, k, v, beta, gate, S0, out, S_final, BH, T,
-                                                    dv, split, stream);
+                return launch_chunked_bv<MODE, 128, false>(q, k, v, beta, gate, S0, out, S_final,
+                                                           BH, T, dv, 0, stream);
     }
     return DR_ERR_UNSUPPORTED;
 }
