@@ -51,63 +51,92 @@ constexpr int CK = 64;    // chunk length
 constexpr int CDK = 128;  // key dimension of the chunked kernel
 constexpr int CHUNK_THREADS = 512;
 
-template <int MODE, int BV>
+// Shared-memory layout (byte offsets from a 1024-aligned base) and TMEM columns.
+// Unsplit: one CTA holds the prep and the chain operands side by side.
+// SPLIT: prep CTAs and chain CTAs of a cluster share one layout in which the chain operands
+// (two sub-chains' S and Y, the V stages) overlay the prep temporaries of two prep groups.
+template <int MODE, int BV, bool SPLIT = false>
 struct ChunkLayout {
     static constexpr bool kKda = MODE == DR_KDA;
     static constexpr bool kGdn = MODE == DR_GDN;
+    static_assert(!(SPLIT && kKda), "KDA is never split");
     static constexpr int NS = 2;                          // K/Q stages
     static constexpr int NSV = (kKda && BV == 128) ? 1 : 2;  // V stages
     static constexpr int NP = (kKda && BV >= 64) ? 1 : 2;    // prepared-operand slots
     static constexpr int NKN = kKda ? 1 : 0;
+    // Sub-chains: the value slice is cut into NSUB independent column sets, interleaved so
+    // that one's MMAs run while the other's epilogues execute (split chain CTAs only).
+    static constexpr int NSUB = SPLIT ? 2 : 1;
+    static constexpr int BVS = BV / NSUB;  // value channels per sub-chain
 
     static constexpr int KQ_B = 32768;  // [K;Q] bf16: 2 panels x 128 rows x 128 B
     static constexpr int V_B = CK * BV * 2;
     // The chain MMAs run with N = NB >= 64 so that Y and the bf16 state are stored as
     // M/N-major B operands in 64-column swizzled groups (whole-row 16-byte stores); columns
-    // BV..NB-1 are zero padding.
-    static constexpr int NB = BV < 64 ? 64 : BV;
-    static constexpr int NG = NB / 64;
-    static constexpr int SY_B = NG * 8192;   // Y: 64 rows (t) x NB, per 64-column group 8 KB
-    static constexpr int SS_B = NG * 16384;  // S: 128 rows (key channel) x NB
+    // beyond the real ones are zero padding. Group g of S / Y sits at SS + g*16384 /
+    // SY + g*8192 (a sub-chain uses one group).
+    static constexpr int NB = SPLIT ? 64 : (BV < 64 ? 64 : BV);
+    static constexpr int NG = SPLIT ? NSUB : NB / 64;
+    static constexpr int SY_B = NG * 8192;   // Y: 64 rows (t) x 64 columns per group
+    static constexpr int SS_B = NG * 16384;  // S: 128 rows (key channel) x 64 columns per group
 
     // A prepared-operand slot: [T; PT] (128 rows x 64), Khat^T (128 rows (dk) x 64 (t)),
     // gamma vector. Contiguous, so that one bulk copy hands it to another CTA of the cluster.
     static constexpr int SLOT_TP = 0, SLOT_KH = 16384, SLOT_GAM = 32768;
     static constexpr int SLOT_B = 32768 + 1024;
 
+    // prep temporaries of one group: P (64 rows, A operand of an M=64 MMA), Ttilde (GDN:
+    // diag(gamma_C/gamma) T), A then X = (I+A)^{-1} (fp32 [64][68]), block scratch [32][36]
+    static constexpr int AM_B = CK * 68 * 4, ZS_B = 32 * 36 * 4;
+
     static constexpr int KQ = 0;
     static constexpr int KN = KQ + NS * KQ_B;    // KDA: K/gamma, 2 panels x 64 rows
     static constexpr int SLOT = KN + NKN * 16384;
-    static constexpr int PM = SLOT + NP * SLOT_B;  // P: 64 rows (A operand of an M=64 MMA)
-    static constexpr int TTS = PM + 8192;        // GDN: diag(gamma_C/gamma) T, 64 rows
-    static constexpr int SS = TTS + (kGdn ? 8192 : 0);  // S bf16, M/N-major B operand
-    static constexpr int SY = SS + SS_B;         // Y bf16, M/N-major B operand
-    static constexpr int V = SY + SY_B;          // V stages: 64 rows x BV bf16
-    // In the prep CTA of a split cluster the chain region (S, Y, V) is unused and holds the
-    // temporaries of a second prep group: P, Ttilde, A/X, block scratch.
-    static constexpr int TMP_B = 8192 + 8192 + CK * 68 * 4 + 32 * 36 * 4;
-    static constexpr int CHAIN_USED = SS_B + SY_B + NSV * V_B;
-    static constexpr int CHAIN_B = (!kKda && CHAIN_USED < TMP_B) ? TMP_B : CHAIN_USED;
-    static constexpr int PM2 = SS, TTS2 = SS + 8192, AM2 = SS + 16384, ZS2 = AM2 + CK * 68 * 4;
-    static constexpr int AM = SS + CHAIN_B;      // A, then X = (I+A)^{-1}: fp32 [64][68]
-    static constexpr int ZS = AM + CK * 68 * 4;  // block-product scratch: fp32 [32][36]
-    static constexpr int GAM = ZS + 32 * 36 * 4;
+    static constexpr int X0 = SLOT + NP * SLOT_B;  // 1024-aligned
+    // ---- unsplit
+    static constexpr int U_PM = X0, U_TTS = X0 + 8192;
+    static constexpr int U_SS = U_TTS + (kGdn ? 8192 : 0);
+    static constexpr int U_SY = U_SS + SS_B;
+    static constexpr int U_V = U_SY + SY_B;
+    static constexpr int U_AM = U_V + NSV * V_B;
+    static constexpr int U_END = U_AM + AM_B + ZS_B;
+    // ---- split: prep view and chain view of the same region
+    static constexpr int S_PM = X0, S_TTS = X0 + 8192, S_PM2 = X0 + 16384, S_TTS2 = X0 + 24576;
+    static constexpr int S_AM = X0 + 32768, S_ZS = S_AM + AM_B;
+    static constexpr int S_AM2 = S_ZS + ZS_B, S_ZS2 = S_AM2 + AM_B;
+    static constexpr int S_SS = X0, S_SY = X0 + SS_B, S_V = S_SY + SY_B;
+    static constexpr int S_END_PREP = S_ZS2 + ZS_B, S_END_CHAIN = S_V + NSV * V_B;
+    static constexpr int S_END = S_END_PREP > S_END_CHAIN ? S_END_PREP : S_END_CHAIN;
+
+    static constexpr int PM = SPLIT ? S_PM : U_PM;
+    static constexpr int TTS = SPLIT ? S_TTS : U_TTS;
+    static constexpr int PM2 = S_PM2, TTS2 = S_TTS2, AM2 = S_AM2, ZS2 = S_ZS2;
+    static constexpr int SS = SPLIT ? S_SS : U_SS;  // S bf16, M/N-major B operand
+    static constexpr int SY = SPLIT ? S_SY : U_SY;  // Y bf16, M/N-major B operand
+    static constexpr int V = SPLIT ? S_V : U_V;     // V stages: 64 rows x BV bf16
+    static constexpr int AM = SPLIT ? S_AM : U_AM;
+    static constexpr int ZS = AM + AM_B;
     // per stage: beta[64]; GDN: g[64], 1/gamma[64], gamma[64] (cumulative log-decay and its
     // exponentials, computed by the producer warp)
     static constexpr int BG_B = 1024;
-    static constexpr int BG = GAM;
+    static constexpr int BG = SPLIT ? S_END : U_END;
     static constexpr int PG = BG + NS * BG_B;    // prep-private: KDA scan exchange, gamma_C[128]
     static constexpr int BAR = PG + 3072;
-    static constexpr int TOTAL = BAR + 256;
+    static constexpr int TOTAL = BAR + 512;
     static_assert(TOTAL + 1024 <= 232448, "shared memory budget");
     static_assert(NS % 2 == 0, "each of two prep groups owns whole K/Q stages");
+    static_assert(X0 % 1024 == 0 && SS % 1024 == 0 && SY % 1024 == 0 && PM % 1024 == 0 &&
+                      TTS % 1024 == 0 && PM2 % 1024 == 0 && TTS2 % 1024 == 0,
+                  "swizzled operands need 1024-byte alignment");
 
-    static constexpr int COL_G = 0;   // D_G, then D_PT (second prep group: +128)
-    static constexpr int COL_H = 64;  // D_H (second prep group: +128)
-    static constexpr int COL_D1 = 128;
-    static constexpr int COL_D2 = 128 + NB;
-    static constexpr int COL_S = 128 + 2 * NB;
-    static constexpr int NCOLS = (128 + 3 * NB) <= 256 ? 256 : 512;
+    // TMEM columns. Prep: D_G then D_PT at COL_G, D_H at COL_H (second prep group: +128).
+    // Chain: sub-chain g's D1, D2 and fp32 state at COL_D1/COL_D2/COL_S + 64 g.
+    static constexpr int COL_G = 0;
+    static constexpr int COL_H = 64;
+    static constexpr int COL_D1 = SPLIT ? 0 : 128;
+    static constexpr int COL_D2 = SPLIT ? 128 : 128 + NB;
+    static constexpr int COL_S = SPLIT ? 256 : 128 + 2 * NB;
+    static constexpr int NCOLS = SPLIT ? 512 : ((128 + 3 * NB) <= 256 ? 256 : 512);
 };
 
 // mbarrier indices inside the BAR block
@@ -128,7 +157,8 @@ enum ChunkBar {
     B_STATE = 19,     // bf16 state copy ready for MMA1
     B_PEER_FREE = 20,  // [2] prep CTA: every chain CTA freed its copy of the slot
     B_GRP1 = 22,       // second prep group's GO, GRAM, TREADY, HDONE (prep CTA of a split)
-    B_COUNT = 26
+    B_SUB1 = 26,       // second sub-chain's MMA1, YREADY, MMA23, STATE (chain CTA of a split)
+    B_COUNT = 30
 };
 
 // bf16 bits of 8 consecutive columns of a row, stored as one 16-byte swizzled chunk.
@@ -202,7 +232,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
     const __grid_constant__ CUtensorMap tmV, const float* __restrict__ beta,
     const float* __restrict__ gate, const float* __restrict__ S0,
     __nv_bfloat16* __restrict__ out, float* __restrict__ S_final, int T, int dv, int nprep) {
-    using L = ChunkLayout<MODE, BV>;
+    using L = ChunkLayout<MODE, BV, SPLIT>;
     constexpr bool kGdn = MODE == DR_GDN;
     constexpr bool kKda = MODE == DR_KDA;
     constexpr int NS = L::NS, NSV = L::NSV, NP = L::NP;
@@ -261,10 +291,13 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
         mbar_init(bar(B_GRP1 + 1), 1);
         mbar_init(bar(B_GRP1 + 2), gthreads);
         mbar_init(bar(B_GRP1 + 3), 1);
-        mbar_init(bar(B_MMA1), 1);
-        mbar_init(bar(B_YREADY), 128);
-        mbar_init(bar(B_MMA23), 1);
-        mbar_init(bar(B_STATE), 128);
+        for (int g = 0; g < 2; ++g) {
+            const int o = g ? B_SUB1 - B_MMA1 : 0;
+            mbar_init(bar(B_MMA1 + o), 1);
+            mbar_init(bar(B_YREADY + o), 128);
+            mbar_init(bar(B_MMA23 + o), 1);
+            mbar_init(bar(B_STATE + o), 128);
+        }
         *abort_flag = 0;
         mbar_init_fence();
     }
@@ -373,45 +406,56 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------------ chain MMA issuer
+        // per sub-chain g: MMA1 once its state copy is ready, MMA2/MMA3 once its Y is ready
         if (lane == 0) {
+            constexpr int NSUB = L::NSUB;
             constexpr uint32_t id1 = idesc_bf16(128, L::NB, 0, 1);
+            auto sb = [&](int base, int g) { return bar(base + (g ? B_SUB1 - B_MMA1 : 0)); };
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c % NS, p = c % NP;
                 uint8_t* kq = sm + L::KQ + s * L::KQ_B;
                 mbar_wait(bar(B_KQ_FULL + s), (uint32_t)((c / NS) & 1), abort_flag);
                 mbar_wait(bar(B_PREP + p), (uint32_t)((c / NP) & 1), abort_flag);
-                mbar_wait(bar(B_STATE), (uint32_t)(c & 1), abort_flag);
-                tc_fence_after();
-                if (!*abort_flag) {
 #pragma unroll
-                    for (int kk = 0; kk < 8; ++kk) {
-                        const int pn = kk >> 2, ko = (kk & 3) * 32;
-                        tc_mma_bf16(tmem + L::COL_D1,
-                                    smem_desc_sw128(smem_u32(kq + pn * 16384 + ko), 16, 1024),
-                                    smem_desc_sw128(smem_u32(sm + L::SS + kk * 2048), 16384, 1024),
-                                    id1, kk > 0);
+                for (int g = 0; g < NSUB; ++g) {
+                    mbar_wait(sb(B_STATE, g), (uint32_t)(c & 1), abort_flag);
+                    tc_fence_after();
+                    if (!*abort_flag) {
+                        const uint8_t* ss = sm + L::SS + g * 16384;
+#pragma unroll
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const int pn = kk >> 2, ko = (kk & 3) * 32;
+                            tc_mma_bf16(tmem + L::COL_D1 + 64 * g,
+                                        smem_desc_sw128(smem_u32(kq + pn * 16384 + ko), 16, 1024),
+                                        smem_desc_sw128(smem_u32(ss + kk * 2048), 16384, 1024), id1,
+                                        kk > 0);
+                        }
+                        tc_commit(sb(B_MMA1, g));
                     }
-                    tc_commit(bar(B_MMA1));
-                    tc_commit(bar(B_KQ_EMPTY + s));
                 }
-                mbar_wait(bar(B_YREADY), (uint32_t)(c & 1), abort_flag);
-                tc_fence_after();
-                if (!*abort_flag) {
-                    const uint8_t* tp = slot(p) + L::SLOT_TP;
-                    const uint8_t* kh = slot(p) + L::SLOT_KH;
+                if (!*abort_flag) tc_commit(bar(B_KQ_EMPTY + s));
+                const uint8_t* tp = slot(p) + L::SLOT_TP;
+                const uint8_t* kh = slot(p) + L::SLOT_KH;
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        tc_mma_bf16(tmem + L::COL_D2,
-                                    smem_desc_sw128(smem_u32(tp + kk * 32), 16, 1024),
-                                    smem_desc_sw128(smem_u32(sm + L::SY + kk * 2048), 8192, 1024),
-                                    id1, kk > 0);
+                for (int g = 0; g < NSUB; ++g) {
+                    mbar_wait(sb(B_YREADY, g), (uint32_t)(c & 1), abort_flag);
+                    tc_fence_after();
+                    if (!*abort_flag) {
+                        const uint8_t* sy = sm + L::SY + g * 8192;
 #pragma unroll
-                    for (int kk = 0; kk < 4; ++kk)
-                        tc_mma_bf16(tmem + L::COL_S,
-                                    smem_desc_sw128(smem_u32(kh + kk * 32), 16, 1024),
-                                    smem_desc_sw128(smem_u32(sm + L::SY + kk * 2048), 8192, 1024),
-                                    id1, 1);
-                    tc_commit(bar(B_MMA23));
+                        for (int kk = 0; kk < 4; ++kk)
+                            tc_mma_bf16(tmem + L::COL_D2 + 64 * g,
+                                        smem_desc_sw128(smem_u32(tp + kk * 32), 16, 1024),
+                                        smem_desc_sw128(smem_u32(sy + kk * 2048), 8192, 1024), id1,
+                                        kk > 0);
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            tc_mma_bf16(tmem + L::COL_S + 64 * g,
+                                        smem_desc_sw128(smem_u32(kh + kk * 32), 16, 1024),
+                                        smem_desc_sw128(smem_u32(sy + kk * 2048), 8192, 1024), id1,
+                                        1);
+                        tc_commit(sb(B_MMA23, g));
+                    }
                 }
             }
         }
@@ -470,6 +514,153 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     tc_commit(bar(gb + 3));
                     tc_commit(bar(B_KQ_EMPTY + s));
                 }
+            }
+        }
+    } else if (warp >= 4 && warp < 8 && SPLIT) {
+        if (!is_chain) goto done;
+        // ------------------------------------------------------------------ chain warpgroup,
+        // split chain CTA: two sub-chains of BVS value channels, interleaved. Per chunk: the
+        // slot's gammas into registers and S^T *= gamma_C, both residuals, then both outputs
+        // and carried states. The slot goes back to its prep CTA as soon as MMA2/3 are done.
+        constexpr int NSUB = L::NSUB, BVS = L::BVS;
+        constexpr int LW = BVS < 16 ? 16 : BVS;  // TMEM columns read per sub-chain
+        const int r = tid - 128;  // TMEM lane: value row t (Y, O) or key channel j (state)
+        const uint32_t trow = tmem + ((uint32_t)(r & ~31) << 16);
+        auto sb = [&](int base, int g) { return bar(base + (g ? B_SUB1 - B_MMA1 : 0)); };
+        {
+            // slots start empty: expect the prep CTAs' copies of the first chunks
+            if (r == 0) {
+                for (int c = 0; c < NP && c < nchunks; ++c) {
+                    mbar_arrive_expect_tx(bar(B_PREP + c), L::SLOT_B);
+                    mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + c), owner_of(c)));
+                }
+            }
+            const float* src = S0 ? S0 + (bh * dv + v0) * (long)CDK + r : nullptr;
+#pragma unroll
+            for (int g = 0; g < NSUB; ++g) {
+                float sv[LW];
+#pragma unroll
+                for (int v = 0; v < LW; ++v)
+                    sv[v] = (src && v < BVS) ? src[(long)(g * BVS + v) * CDK] : 0.f;
+#pragma unroll
+                for (int i = 0; i < BVS / 8; ++i) st_row_chunk(sm + L::SS + g * 16384, r, i, sv + 8 * i);
+#pragma unroll
+                for (int c16 = 0; c16 < 64; c16 += 16) {
+                    float w[16];
+#pragma unroll
+                    for (int v = 0; v < 16; ++v) w[v] = c16 + v < LW ? sv[c16 + v] : 0.f;
+                    tmem_st16(trow + L::COL_S + 64 * g + c16, w);
+                }
+            }
+            tmem_wait_st();
+            fence_async_smem();
+#pragma unroll
+            for (int g = 0; g < NSUB; ++g) mbar_arrive(sb(B_STATE, g));
+        }
+        for (int c = 0; c < nchunks; ++c) {
+            const int p = c % NP, svi = c % NSV;
+            const int t0 = c * CK;
+            const int nvalid = min(CK, T - t0);
+            mbar_wait(bar(B_PREP + p), (uint32_t)((c / NP) & 1), abort_flag);
+            float gt = 1.f;  // gamma_t of row r & 63 (residual and output rows)
+            if constexpr (MODE != DR_DELTANET) {
+                const float* gam = reinterpret_cast<const float*>(slot(p) + L::SLOT_GAM);
+                if constexpr (kGdn) gt = gam[r & 63];
+                const float gC = gam[64];
+                // S^T *= gamma_C of this chunk, before its MMA3 (TMEM lane r = key channel r)
+#pragma unroll
+                for (int g = 0; g < NSUB; ++g) {
+                    float w[LW];
+#pragma unroll
+                    for (int c16 = 0; c16 < LW; c16 += 16) tmem_ld16(trow + L::COL_S + 64 * g + c16, w + c16);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int v = 0; v < LW; ++v) w[v] *= gC;
+#pragma unroll
+                    for (int c16 = 0; c16 < LW; c16 += 16) tmem_st16(trow + L::COL_S + 64 * g + c16, w + c16);
+                }
+                tmem_wait_st();
+            }
+            // ---- residuals Y = V - gamma_t (S0 k_t) of both sub-chains
+#pragma unroll
+            for (int g = 0; g < NSUB; ++g) {
+                mbar_wait(sb(B_MMA1, g), (uint32_t)(c & 1), abort_flag);
+                tc_fence_after();
+                if (r < 64) {
+                    if (g == 0) mbar_wait(bar(B_V_FULL + svi), (uint32_t)((c / NSV) & 1), abort_flag);
+                    const uint4* vrow = reinterpret_cast<const uint4*>(sm + L::V + svi * L::V_B +
+                                                                       r * BV * 2) + g * (BVS / 8);
+                    float x[LW];
+                    uint4 vw[BVS / 8];
+#pragma unroll
+                    for (int c16 = 0; c16 < LW; c16 += 16) tmem_ld16(trow + L::COL_D1 + 64 * g + c16, x + c16);
+#pragma unroll
+                    for (int i = 0; i < BVS / 8; ++i) vw[i] = vrow[i];
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < BVS / 8; ++i) {
+                        const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&vw[i]);
+                        float y[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) y[e] = fmaf(-gt, x[8 * i + e], __bfloat162float(hv[e]));
+                        st_row_chunk(sm + L::SY + g * 8192, r, i, y);
+                    }
+                    if (g == NSUB - 1) mbar_arrive(bar(B_V_EMPTY + svi));
+                }
+                fence_async_smem();
+                tc_fence_before();
+                mbar_arrive(sb(B_YREADY, g));
+            }
+            // ---- outputs O = gamma_t (S0 q_t) + (P T Y)_t and carried states
+            const bool last = c == nchunks - 1;
+#pragma unroll
+            for (int g = 0; g < NSUB; ++g) {
+                mbar_wait(sb(B_MMA23, g), (uint32_t)(c & 1), abort_flag);
+                tc_fence_after();
+                if (g == NSUB - 1 && r == 0 && c + NP < nchunks) {
+                    // every MMA reading slot p is complete and every thread read its gammas
+                    // before its residual arrival: the slot can be refilled
+                    mbar_arrive_expect_tx(bar(B_PREP + p), L::SLOT_B);
+                    mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + p), owner_of(c + NP)));
+                }
+                if (r >= 64) {
+                    const int t = r - 64;
+                    float z[LW], d[LW];
+#pragma unroll
+                    for (int c16 = 0; c16 < LW; c16 += 16) {
+                        tmem_ld16(trow + L::COL_D1 + 64 * g + c16, z + c16);
+                        tmem_ld16(trow + L::COL_D2 + 64 * g + c16, d + c16);
+                    }
+                    tmem_wait_ld();
+                    if (t < nvalid) {
+                        uint4* dst = reinterpret_cast<uint4*>(out + (bh * T + t0 + t) * (long)dv + v0 +
+                                                              g * BVS);
+#pragma unroll
+                        for (int i = 0; i < BVS / 8; ++i) {
+                            uint4 w;
+                            uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                wp[e] = pack_bf16(fmaf(gt, z[8 * i + 2 * e], d[8 * i + 2 * e]),
+                                                  fmaf(gt, z[8 * i + 2 * e + 1], d[8 * i + 2 * e + 1]));
+                            dst[i] = w;
+                        }
+                    }
+                }
+                float sv[LW];
+#pragma unroll
+                for (int c16 = 0; c16 < LW; c16 += 16) tmem_ld16(trow + L::COL_S + 64 * g + c16, sv + c16);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < BVS / 8; ++i) st_row_chunk(sm + L::SS + g * 16384, r, i, sv + 8 * i);
+                if (last && S_final) {
+                    float* dst = S_final + (bh * dv + v0 + g * BVS) * (long)CDK + r;
+#pragma unroll
+                    for (int v = 0; v < BVS; ++v) dst[(long)v * CDK] = sv[v];
+                }
+                fence_async_smem();
+                tc_fence_before();
+                mbar_arrive(sb(B_STATE, g));
             }
         }
     } else if (warp >= 4 && warp < 8) {
@@ -1018,7 +1209,7 @@ template <int MODE, int BV, bool SPLIT>
 int launch_chunked_bv(const void* q, const void* k, const void* v, const float* beta,
                       const float* gate, const float* S0, void* out, float* S_final, int BH, int T,
                       int dv, int nprep, cudaStream_t stream) {
-    using L = ChunkLayout<MODE, BV>;
+    using L = ChunkLayout<MODE, BV, SPLIT>;
     CUtensorMap mk, mq, mv;
     if (!make_map_3d(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, BH, T, CDK, 64, true) ||
         !make_map_3d(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, BH, T, CDK, 64, true) ||
@@ -1073,7 +1264,7 @@ inline int max_active_clusters(int size) {
     if (size < 1 || size > 8 || cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 16)
         return 0;
     if (cache[dev][size] == 0) {
-        using L = ChunkLayout<DR_GDN, 64>;
+        using L = ChunkLayout<DR_GDN, 64, true>;
         auto kern = dr_chunked_kernel<DR_GDN, 64, true>;
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(1, (unsigned)size);
