@@ -66,7 +66,7 @@ struct ChunkLayout {
     static constexpr int NKN = kKda ? 1 : 0;
     // Sub-chains: the value slice is cut into NSUB independent column sets, interleaved so
     // that one's MMAs run while the other's epilogues execute (split chain CTAs only).
-    static constexpr int NSUB = SPLIT ? 2 : 1;
+    static constexpr int NSUB = 1;
     static constexpr int BVS = BV / NSUB;  // value channels per sub-chain
 
     static constexpr int KQ_B = 32768;  // [K;Q] bf16: 2 panels x 128 rows x 128 B
@@ -105,7 +105,10 @@ struct ChunkLayout {
     static constexpr int S_AM = X0 + 32768, S_ZS = S_AM + AM_B;
     static constexpr int S_AM2 = S_ZS + ZS_B, S_ZS2 = S_AM2 + AM_B;
     static constexpr int S_SS = X0, S_SY = X0 + SS_B, S_V = S_SY + SY_B;
-    static constexpr int S_END_PREP = S_ZS2 + ZS_B, S_END_CHAIN = S_V + NSV * V_B;
+    // a chain CTA's third prepared-operand slot (its ring is three deep when the cluster has
+    // two or more prep CTAs)
+    static constexpr int SLOT2 = (S_V + NSV * V_B + 1023) / 1024 * 1024;
+    static constexpr int S_END_PREP = S_ZS2 + ZS_B, S_END_CHAIN = SLOT2 + SLOT_B;
     static constexpr int S_END = S_END_PREP > S_END_CHAIN ? S_END_PREP : S_END_CHAIN;
 
     static constexpr int PM = SPLIT ? S_PM : U_PM;
@@ -130,12 +133,14 @@ struct ChunkLayout {
                   "swizzled operands need 1024-byte alignment");
 
     // TMEM columns. Prep: D_G then D_PT at COL_G, D_H at COL_H (second prep group: +128).
-    // Chain: sub-chain g's D1, D2 and fp32 state at COL_D1/COL_D2/COL_S + 64 g.
+    // Chain: sub-chain g's D1, D2 and fp32 state at COL_D1/COL_D2/COL_S + 64 g; split chain
+    // CTAs keep two D1 buffers (chunk parity b at +128 b) so that a chunk's outputs can still
+    // be read while the next chunk's MMA1 runs.
     static constexpr int COL_G = 0;
     static constexpr int COL_H = 64;
     static constexpr int COL_D1 = SPLIT ? 0 : 128;
-    static constexpr int COL_D2 = SPLIT ? 128 : 128 + NB;
-    static constexpr int COL_S = SPLIT ? 256 : 128 + 2 * NB;
+    static constexpr int COL_D2 = SPLIT ? 256 : 128 + NB;
+    static constexpr int COL_S = SPLIT ? 384 : 128 + 2 * NB;
     static constexpr int NCOLS = SPLIT ? 512 : ((128 + 3 * NB) <= 256 ? 256 : 512);
 };
 
@@ -158,7 +163,9 @@ enum ChunkBar {
     B_PEER_FREE = 20,  // [2] prep CTA: every chain CTA freed its copy of the slot
     B_GRP1 = 22,       // second prep group's GO, GRAM, TREADY, HDONE (prep CTA of a split)
     B_SUB1 = 26,       // second sub-chain's MMA1, YREADY, MMA23, STATE (chain CTA of a split)
-    B_COUNT = 30
+    B_ODONE = 30,      // [2] split chain CTA: sub-chain g's output rows are read out of TMEM
+    B_PREP2 = 32,      // split chain CTA: third slot ready
+    B_COUNT = 33
 };
 
 // bf16 bits of 8 consecutive columns of a row, stored as one 16-byte swizzled chunk.
@@ -270,6 +277,17 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
     auto chunk_of = [&](int m) { return pbase + (m / pG) * pSP + m % pG; };
     auto ordinal_of = [&](int c) { return ((c - pbase) / pSP) * pG + (c - pbase) % pG; };
     auto owner_of = [&](int c) { return (c / NGR) % NPREP; };  // prep rank of chunk c
+    // Chain-side slot ring: NP slots, or three in a split cluster with two or more prep CTAs
+    // (then no two of the first three chunks share a prep CTA and prep slot, so the initial
+    // credits complete distinct barrier phases).
+    const int npc = (SPLIT && NPREP >= 2) ? 3 : NP;
+    auto cslot = [&](int i) -> uint8_t* {
+        if constexpr (SPLIT) {
+            if (i == 2) return sm + L::SLOT2;
+        }
+        return sm + L::SLOT + i * L::SLOT_B;
+    };
+    auto cprep = [&](int i) { return bar(i == 2 ? B_PREP2 : B_PREP + i); };
     auto slot = [&](int p) { return sm + L::SLOT + p * L::SLOT_B; };
 
     if (tid == 0) {
@@ -282,6 +300,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             mbar_init(bar(B_SLOT_EMPTY + s), 1);
             mbar_init(bar(B_PEER_FREE + s), split ? NCC : 1);
         }
+        mbar_init(bar(B_PREP2), 1);
         const uint32_t gthreads = 256 / NGR;  // threads per prep group
         mbar_init(bar(B_GO), gthreads);
         mbar_init(bar(B_GRAM), 1);
@@ -291,10 +310,12 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
         mbar_init(bar(B_GRP1 + 1), 1);
         mbar_init(bar(B_GRP1 + 2), gthreads);
         mbar_init(bar(B_GRP1 + 3), 1);
+        mbar_init(bar(B_ODONE + 0), 64);
+        mbar_init(bar(B_ODONE + 1), 64);
         for (int g = 0; g < 2; ++g) {
             const int o = g ? B_SUB1 - B_MMA1 : 0;
             mbar_init(bar(B_MMA1 + o), 1);
-            mbar_init(bar(B_YREADY + o), 128);
+            mbar_init(bar(B_YREADY + o), SPLIT ? 64 : 128);
             mbar_init(bar(B_MMA23 + o), 1);
             mbar_init(bar(B_STATE + o), 128);
         }
@@ -356,6 +377,8 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     }
                 }
                 x1 += __shfl_sync(0xffffffffu, x0, 31);
+                if (SPLIT && is_chain && lane == 31)  // gamma_C ring for the chain warpgroup
+                    reinterpret_cast<float*>(sm + L::PG)[c & 3] = __expf(x1);
                 bg[64 + lane] = x0;
                 bg[96 + lane] = x1;
                 bg[128 + lane] = __expf(-x0);
@@ -395,10 +418,12 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 mbar_wait(bar(B_PREP + p), ph, abort_flag);
                 mbar_wait(bar(B_PEER_FREE + p), ph, abort_flag);
                 if (!*abort_flag) {
+                    // into chain slot c % npc of every chain rank
                     const uint32_t src = smem_u32(slot(p));
+                    const uint32_t dst = smem_u32(cslot(c % npc));
                     for (int q = NPREP; q < NPREP + NCC; ++q)  // the chain ranks
-                        bulk_copy_to_peer(cluster_map(src, q), src, L::SLOT_B,
-                                          cluster_map(bar(B_PREP + p), q));
+                        bulk_copy_to_peer(cluster_map(dst, q), src, L::SLOT_B,
+                                          cluster_map(cprep(c % npc), q));
                     bulk_commit_and_wait_read();
                 }
                 mbar_arrive(bar(B_SLOT_EMPTY + p));
@@ -412,20 +437,21 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             constexpr uint32_t id1 = idesc_bf16(128, L::NB, 0, 1);
             auto sb = [&](int base, int g) { return bar(base + (g ? B_SUB1 - B_MMA1 : 0)); };
             for (int c = 0; c < nchunks; ++c) {
-                const int s = c % NS, p = c % NP;
+                const int s = c % NS;
                 uint8_t* kq = sm + L::KQ + s * L::KQ_B;
                 mbar_wait(bar(B_KQ_FULL + s), (uint32_t)((c / NS) & 1), abort_flag);
-                mbar_wait(bar(B_PREP + p), (uint32_t)((c / NP) & 1), abort_flag);
+                mbar_wait(cprep(c % npc), (uint32_t)((c / npc) & 1), abort_flag);
 #pragma unroll
                 for (int g = 0; g < NSUB; ++g) {
                     mbar_wait(sb(B_STATE, g), (uint32_t)(c & 1), abort_flag);
                     tc_fence_after();
                     if (!*abort_flag) {
                         const uint8_t* ss = sm + L::SS + g * 16384;
+                        const uint32_t d1 = L::COL_D1 + 64 * g + (SPLIT ? 128 * (c & 1) : 0);
 #pragma unroll
                         for (int kk = 0; kk < 8; ++kk) {
                             const int pn = kk >> 2, ko = (kk & 3) * 32;
-                            tc_mma_bf16(tmem + L::COL_D1 + 64 * g,
+                            tc_mma_bf16(tmem + d1,
                                         smem_desc_sw128(smem_u32(kq + pn * 16384 + ko), 16, 1024),
                                         smem_desc_sw128(smem_u32(ss + kk * 2048), 16384, 1024), id1,
                                         kk > 0);
@@ -434,11 +460,14 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     }
                 }
                 if (!*abort_flag) tc_commit(bar(B_KQ_EMPTY + s));
-                const uint8_t* tp = slot(p) + L::SLOT_TP;
-                const uint8_t* kh = slot(p) + L::SLOT_KH;
+                const uint8_t* tp = cslot(c % npc) + L::SLOT_TP;
+                const uint8_t* kh = cslot(c % npc) + L::SLOT_KH;
 #pragma unroll
                 for (int g = 0; g < NSUB; ++g) {
                     mbar_wait(sb(B_YREADY, g), (uint32_t)(c & 1), abort_flag);
+                    // split: the previous chunk's output rows must be out of D2 first
+                    if (SPLIT && c > 0)
+                        mbar_wait(bar(B_ODONE + g), (uint32_t)((c - 1) & 1), abort_flag);
                     tc_fence_after();
                     if (!*abort_flag) {
                         const uint8_t* sy = sm + L::SY + g * 8192;
@@ -519,20 +548,32 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
     } else if (warp >= 4 && warp < 8 && SPLIT) {
         if (!is_chain) goto done;
         // ------------------------------------------------------------------ chain warpgroup,
-        // split chain CTA: two sub-chains of BVS value channels, interleaved. Per chunk: the
-        // slot's gammas into registers and S^T *= gamma_C, both residuals, then both outputs
-        // and carried states. The slot goes back to its prep CTA as soon as MMA2/3 are done.
+        // split chain CTA: two sub-chains of BVS value channels, interleaved. Threads 0-63
+        // (TMEM lanes of the K rows) write the residuals, threads 64-127 (Q rows) the outputs,
+        // all 128 (lane = key channel) the carried state. Per chunk: residuals of both
+        // sub-chains; then each sub-chain's state, already scaled by the next chunk's gamma_C
+        // (from the producer's ring) and handed straight to MMA1; then the outputs, which
+        // overlap the next chunk's residuals.
         constexpr int NSUB = L::NSUB, BVS = L::BVS;
         constexpr int LW = BVS < 16 ? 16 : BVS;  // TMEM columns read per sub-chain
+        constexpr int PW = LW < 32 ? LW : 32;    // columns per epilogue piece (registers)
         const int r = tid - 128;  // TMEM lane: value row t (Y, O) or key channel j (state)
         const uint32_t trow = tmem + ((uint32_t)(r & ~31) << 16);
+        const float* gcr = reinterpret_cast<const float*>(sm + L::PG);  // gamma_C by chunk % 4
         auto sb = [&](int base, int g) { return bar(base + (g ? B_SUB1 - B_MMA1 : 0)); };
         {
             // slots start empty: expect the prep CTAs' copies of the first chunks
             if (r == 0) {
-                for (int c = 0; c < NP && c < nchunks; ++c) {
-                    mbar_arrive_expect_tx(bar(B_PREP + c), L::SLOT_B);
-                    mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + c), owner_of(c)));
+                for (int c = 0; c < npc && c < nchunks; ++c) {
+                    mbar_arrive_expect_tx(cprep(c), L::SLOT_B);
+                    mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + c % NP), owner_of(c)));
+                }
+            }
+            float gC0 = 1.f;
+            if constexpr (kGdn) {
+                if (nchunks > 0) {
+                    mbar_wait(bar(B_KQ_FULL + 0), 0u, abort_flag);
+                    gC0 = gcr[0];
                 }
             }
             const float* src = S0 ? S0 + (bh * dv + v0) * (long)CDK + r : nullptr;
@@ -548,119 +589,144 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 for (int c16 = 0; c16 < 64; c16 += 16) {
                     float w[16];
 #pragma unroll
-                    for (int v = 0; v < 16; ++v) w[v] = c16 + v < LW ? sv[c16 + v] : 0.f;
+                    for (int v = 0; v < 16; ++v) w[v] = c16 + v < LW ? sv[c16 + v] * gC0 : 0.f;
                     tmem_st16(trow + L::COL_S + 64 * g + c16, w);
                 }
             }
             tmem_wait_st();
             fence_async_smem();
+            tc_fence_before();
 #pragma unroll
             for (int g = 0; g < NSUB; ++g) mbar_arrive(sb(B_STATE, g));
         }
         for (int c = 0; c < nchunks; ++c) {
-            const int p = c % NP, svi = c % NSV;
+            const int svi = c % NSV;
             const int t0 = c * CK;
             const int nvalid = min(CK, T - t0);
-            mbar_wait(bar(B_PREP + p), (uint32_t)((c / NP) & 1), abort_flag);
-            float gt = 1.f;  // gamma_t of row r & 63 (residual and output rows)
-            if constexpr (MODE != DR_DELTANET) {
-                const float* gam = reinterpret_cast<const float*>(slot(p) + L::SLOT_GAM);
-                if constexpr (kGdn) gt = gam[r & 63];
-                const float gC = gam[64];
-                // S^T *= gamma_C of this chunk, before its MMA3 (TMEM lane r = key channel r)
-#pragma unroll
-                for (int g = 0; g < NSUB; ++g) {
-                    float w[LW];
-#pragma unroll
-                    for (int c16 = 0; c16 < LW; c16 += 16) tmem_ld16(trow + L::COL_S + 64 * g + c16, w + c16);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int v = 0; v < LW; ++v) w[v] *= gC;
-#pragma unroll
-                    for (int c16 = 0; c16 < LW; c16 += 16) tmem_st16(trow + L::COL_S + 64 * g + c16, w + c16);
+            const uint32_t d1 = L::COL_D1 + 128 * (c & 1);
+            const int pc = c % npc;  // chain slot of chunk c
+            mbar_wait(cprep(pc), (uint32_t)((c / npc) & 1), abort_flag);
+            const float gt = kGdn ? reinterpret_cast<const float*>(cslot(pc) + L::SLOT_GAM)[r & 63] : 1.f;
+            // gamma_C of the next chunk, from the producer's ring (its K/Q stage is loaded by now)
+            const bool last = c == nchunks - 1;
+            float gCn = 1.f;
+            if constexpr (kGdn) {
+                if (!last) {
+                    mbar_wait(bar(B_KQ_FULL + (c + 1) % NS), (uint32_t)(((c + 1) / NS) & 1), abort_flag);
+                    gCn = gcr[(c + 1) & 3];
                 }
-                tmem_wait_st();
             }
             // ---- residuals Y = V - gamma_t (S0 k_t) of both sub-chains
+            if (r < 64) {
 #pragma unroll
-            for (int g = 0; g < NSUB; ++g) {
-                mbar_wait(sb(B_MMA1, g), (uint32_t)(c & 1), abort_flag);
-                tc_fence_after();
-                if (r < 64) {
+                for (int g = 0; g < NSUB; ++g) {
+                    mbar_wait(sb(B_MMA1, g), (uint32_t)(c & 1), abort_flag);
+                    tc_fence_after();
                     if (g == 0) mbar_wait(bar(B_V_FULL + svi), (uint32_t)((c / NSV) & 1), abort_flag);
                     const uint4* vrow = reinterpret_cast<const uint4*>(sm + L::V + svi * L::V_B +
                                                                        r * BV * 2) + g * (BVS / 8);
-                    float x[LW];
-                    uint4 vw[BVS / 8];
 #pragma unroll
-                    for (int c16 = 0; c16 < LW; c16 += 16) tmem_ld16(trow + L::COL_D1 + 64 * g + c16, x + c16);
+                    for (int c0 = 0; c0 < LW; c0 += PW) {
+                        constexpr int NV8 = (PW < BVS ? PW : BVS) / 8;  // real 8-column chunks
+                        float x[PW];
+                        uint4 vw[NV8];
 #pragma unroll
-                    for (int i = 0; i < BVS / 8; ++i) vw[i] = vrow[i];
-                    tmem_wait_ld();
+                        for (int c16 = 0; c16 < PW; c16 += 16) tmem_ld16(trow + d1 + 64 * g + c0 + c16, x + c16);
 #pragma unroll
-                    for (int i = 0; i < BVS / 8; ++i) {
-                        const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&vw[i]);
-                        float y[8];
+                        for (int i = 0; i < NV8; ++i) vw[i] = vrow[c0 / 8 + i];
+                        tmem_wait_ld();
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) y[e] = fmaf(-gt, x[8 * i + e], __bfloat162float(hv[e]));
-                        st_row_chunk(sm + L::SY + g * 8192, r, i, y);
+                        for (int i = 0; i < NV8; ++i) {
+                            const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&vw[i]);
+                            float y[8];
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) y[e] = fmaf(-gt, x[8 * i + e], __bfloat162float(hv[e]));
+                            st_row_chunk(sm + L::SY + g * 8192, r, c0 / 8 + i, y);
+                        }
                     }
                     if (g == NSUB - 1) mbar_arrive(bar(B_V_EMPTY + svi));
+                    fence_async_smem();
+                    tc_fence_before();
+                    mbar_arrive(sb(B_YREADY, g));
                 }
-                fence_async_smem();
-                tc_fence_before();
-                mbar_arrive(sb(B_YREADY, g));
             }
-            // ---- outputs O = gamma_t (S0 q_t) + (P T Y)_t and carried states
-            const bool last = c == nchunks - 1;
+            // ---- carried states: bf16 copy for MMA1 of the next chunk, fp32 S_final after
+            // the last; the fp32 state takes the next chunk's gamma_C before its MMA3
 #pragma unroll
             for (int g = 0; g < NSUB; ++g) {
                 mbar_wait(sb(B_MMA23, g), (uint32_t)(c & 1), abort_flag);
                 tc_fence_after();
-                if (g == NSUB - 1 && r == 0 && c + NP < nchunks) {
-                    // every MMA reading slot p is complete and every thread read its gammas
-                    // before its residual arrival: the slot can be refilled
-                    mbar_arrive_expect_tx(bar(B_PREP + p), L::SLOT_B);
-                    mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + p), owner_of(c + NP)));
-                }
-                if (r >= 64) {
-                    const int t = r - 64;
-                    float z[LW], d[LW];
 #pragma unroll
-                    for (int c16 = 0; c16 < LW; c16 += 16) {
-                        tmem_ld16(trow + L::COL_D1 + 64 * g + c16, z + c16);
-                        tmem_ld16(trow + L::COL_D2 + 64 * g + c16, d + c16);
-                    }
+                for (int c0 = 0; c0 < LW; c0 += PW) {
+                    constexpr int NV8 = (PW < BVS ? PW : BVS) / 8;
+                    float sv[PW];
+#pragma unroll
+                    for (int c16 = 0; c16 < PW; c16 += 16) tmem_ld16(trow + L::COL_S + 64 * g + c0 + c16, sv + c16);
                     tmem_wait_ld();
-                    if (t < nvalid) {
-                        uint4* dst = reinterpret_cast<uint4*>(out + (bh * T + t0 + t) * (long)dv + v0 +
-                                                              g * BVS);
 #pragma unroll
-                        for (int i = 0; i < BVS / 8; ++i) {
-                            uint4 w;
-                            uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+                    for (int i = 0; i < NV8; ++i) st_row_chunk(sm + L::SS + g * 16384, r, c0 / 8 + i, sv + 8 * i);
+                    if (last && S_final) {
+                        float* dst = S_final + (bh * dv + v0 + g * BVS + c0) * (long)CDK + r;
 #pragma unroll
-                            for (int e = 0; e < 4; ++e)
-                                wp[e] = pack_bf16(fmaf(gt, z[8 * i + 2 * e], d[8 * i + 2 * e]),
-                                                  fmaf(gt, z[8 * i + 2 * e + 1], d[8 * i + 2 * e + 1]));
-                            dst[i] = w;
+                        for (int v = 0; v < 8 * NV8; ++v) dst[(long)v * CDK] = sv[v];
+                    }
+                    if constexpr (kGdn) {
+                        if (!last) {
+#pragma unroll
+                            for (int v = 0; v < PW; ++v) sv[v] *= gCn;
+#pragma unroll
+                            for (int c16 = 0; c16 < PW; c16 += 16) tmem_st16(trow + L::COL_S + 64 * g + c0 + c16, sv + c16);
                         }
                     }
                 }
-                float sv[LW];
-#pragma unroll
-                for (int c16 = 0; c16 < LW; c16 += 16) tmem_ld16(trow + L::COL_S + 64 * g + c16, sv + c16);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < BVS / 8; ++i) st_row_chunk(sm + L::SS + g * 16384, r, i, sv + 8 * i);
-                if (last && S_final) {
-                    float* dst = S_final + (bh * dv + v0 + g * BVS) * (long)CDK + r;
-#pragma unroll
-                    for (int v = 0; v < BVS; ++v) dst[(long)v * CDK] = sv[v];
-                }
+                if constexpr (kGdn) tmem_wait_st();
                 fence_async_smem();
                 tc_fence_before();
                 mbar_arrive(sb(B_STATE, g));
+            }
+            if (r == 64 && c + npc < nchunks) {
+                // every thread read the slot's gammas before its state arrival and every MMA
+                // reading the slot is complete: expect chunk c + npc in it and credit the prep
+                // CTA that owns that chunk (an output-side thread, off the residual path)
+                mbar_wait(sb(B_STATE, NSUB - 1), (uint32_t)((c + 1) & 1), abort_flag);
+                mbar_arrive_expect_tx(cprep(pc), L::SLOT_B);
+                mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + (c + npc) % NP), owner_of(c + npc)));
+            }
+            // ---- outputs O = gamma_t (S0 q_t) + (P T Y)_t, overlapping the next residuals
+            if (r >= 64) {
+                const int t = r - 64;
+#pragma unroll
+                for (int g = 0; g < NSUB; ++g) {
+                    uint4* dst = reinterpret_cast<uint4*>(out + (bh * T + t0 + t) * (long)dv + v0 +
+                                                          g * BVS);
+#pragma unroll
+                    for (int c0 = 0; c0 < LW; c0 += PW) {
+                        constexpr int NV8 = (PW < BVS ? PW : BVS) / 8;
+                        float z[PW], dd[PW];
+#pragma unroll
+                        for (int c16 = 0; c16 < PW; c16 += 16) {
+                            tmem_ld16(trow + d1 + 64 * g + c0 + c16, z + c16);
+                            tmem_ld16(trow + L::COL_D2 + 64 * g + c0 + c16, dd + c16);
+                        }
+                        tmem_wait_ld();
+                        if (c0 + PW >= LW) {  // D2 and D1 of this sub-chain fully read
+                            tc_fence_before();
+                            mbar_arrive(bar(B_ODONE + g));
+                        }
+                        if (t < nvalid) {
+#pragma unroll
+                            for (int i = 0; i < NV8; ++i) {
+                                uint4 w;
+                                uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+                                for (int e = 0; e < 4; ++e)
+                                    wp[e] = pack_bf16(fmaf(gt, z[8 * i + 2 * e], dd[8 * i + 2 * e]),
+                                                      fmaf(gt, z[8 * i + 2 * e + 1], dd[8 * i + 2 * e + 1]));
+                                dst[c0 / 8 + i] = w;
+                            }
+                        }
+                    }
+                }
             }
         }
     } else if (warp >= 4 && warp < 8) {
