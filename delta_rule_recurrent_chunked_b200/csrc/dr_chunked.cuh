@@ -66,11 +66,13 @@ struct ChunkLayout {
     static constexpr int NKN = kKda ? 1 : 0;
     // Sub-chains: the value slice is cut into NSUB independent column sets, interleaved so
     // that one's MMAs run while the other's epilogues execute (split chain CTAs only).
-    static constexpr int NSUB = 1;
+    static constexpr int NSUB = 1;  // (the chain code is written for NSUB sub-chains)
     static constexpr int BVS = BV / NSUB;  // value channels per sub-chain
 
     static constexpr int KQ_B = 32768;  // [K;Q] bf16: 2 panels x 128 rows x 128 B
     static constexpr int V_B = CK * BV * 2;
+    // split, BV = 64: V rows are one 128-byte swizzled row each (conflict-free row reads)
+    static constexpr bool V_SWZ = SPLIT && BV == 64;
     // The chain MMAs run with N = NB >= 64 so that Y and the bf16 state are stored as
     // M/N-major B operands in 64-column swizzled groups (whole-row 16-byte stores); columns
     // beyond the real ones are zero padding. Group g of S / Y sits at SS + g*16384 /
@@ -165,7 +167,8 @@ enum ChunkBar {
     B_SUB1 = 26,       // second sub-chain's MMA1, YREADY, MMA23, STATE (chain CTA of a split)
     B_ODONE = 30,      // [2] split chain CTA: sub-chain g's output rows are read out of TMEM
     B_PREP2 = 32,      // split chain CTA: third slot ready
-    B_COUNT = 33
+    B_MMA2 = 33,       // split chain CTA: MMA2 done (MMA3 done is B_MMA23)
+    B_COUNT = 34
 };
 
 // bf16 bits of 8 consecutive columns of a row, stored as one 16-byte swizzled chunk.
@@ -301,6 +304,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             mbar_init(bar(B_PEER_FREE + s), split ? NCC : 1);
         }
         mbar_init(bar(B_PREP2), 1);
+        mbar_init(bar(B_MMA2), 1);
         const uint32_t gthreads = 256 / NGR;  // threads per prep group
         mbar_init(bar(B_GO), gthreads);
         mbar_init(bar(B_GRAM), 1);
@@ -465,25 +469,43 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
 #pragma unroll
                 for (int g = 0; g < NSUB; ++g) {
                     mbar_wait(sb(B_YREADY, g), (uint32_t)(c & 1), abort_flag);
-                    // split: the previous chunk's output rows must be out of D2 first
-                    if (SPLIT && c > 0)
-                        mbar_wait(bar(B_ODONE + g), (uint32_t)((c - 1) & 1), abort_flag);
                     tc_fence_after();
-                    if (!*abort_flag) {
-                        const uint8_t* sy = sm + L::SY + g * 8192;
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            tc_mma_bf16(tmem + L::COL_D2 + 64 * g,
-                                        smem_desc_sw128(smem_u32(tp + kk * 32), 16, 1024),
-                                        smem_desc_sw128(smem_u32(sy + kk * 2048), 8192, 1024), id1,
-                                        kk > 0);
+                    const uint8_t* sy = sm + L::SY + g * 8192;
+                    auto mma3 = [&]() {  // S^T += Khat^T Y
 #pragma unroll
                         for (int kk = 0; kk < 4; ++kk)
                             tc_mma_bf16(tmem + L::COL_S + 64 * g,
                                         smem_desc_sw128(smem_u32(kh + kk * 32), 16, 1024),
                                         smem_desc_sw128(smem_u32(sy + kk * 2048), 8192, 1024), id1,
                                         1);
-                        tc_commit(sb(B_MMA23, g));
+                    };
+                    auto mma2 = [&]() {  // D2 = [T; PT] Y
+#pragma unroll
+                        for (int kk = 0; kk < 4; ++kk)
+                            tc_mma_bf16(tmem + L::COL_D2 + 64 * g,
+                                        smem_desc_sw128(smem_u32(tp + kk * 32), 16, 1024),
+                                        smem_desc_sw128(smem_u32(sy + kk * 2048), 8192, 1024), id1,
+                                        kk > 0);
+                    };
+                    if constexpr (SPLIT) {
+                        // the state update first (it is on the chain's critical path), then the
+                        // output rows once the previous chunk's are out of D2
+                        if (!*abort_flag) {
+                            mma3();
+                            tc_commit(sb(B_MMA23, g));
+                        }
+                        if (c > 0) mbar_wait(bar(B_ODONE + g), (uint32_t)((c - 1) & 1), abort_flag);
+                        tc_fence_after();
+                        if (!*abort_flag) {
+                            mma2();
+                            tc_commit(bar(B_MMA2));
+                        }
+                    } else {
+                        if (!*abort_flag) {
+                            mma2();
+                            mma3();
+                            tc_commit(sb(B_MMA23, g));
+                        }
                     }
                 }
             }
@@ -623,8 +645,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     mbar_wait(sb(B_MMA1, g), (uint32_t)(c & 1), abort_flag);
                     tc_fence_after();
                     if (g == 0) mbar_wait(bar(B_V_FULL + svi), (uint32_t)((c / NSV) & 1), abort_flag);
-                    const uint4* vrow = reinterpret_cast<const uint4*>(sm + L::V + svi * L::V_B +
-                                                                       r * BV * 2) + g * (BVS / 8);
+                    const uint8_t* vst = sm + L::V + svi * L::V_B + r * BV * 2;  // row r of V
 #pragma unroll
                     for (int c0 = 0; c0 < LW; c0 += PW) {
                         constexpr int NV8 = (PW < BVS ? PW : BVS) / 8;  // real 8-column chunks
@@ -633,7 +654,11 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
 #pragma unroll
                         for (int c16 = 0; c16 < PW; c16 += 16) tmem_ld16(trow + d1 + 64 * g + c0 + c16, x + c16);
 #pragma unroll
-                        for (int i = 0; i < NV8; ++i) vw[i] = vrow[c0 / 8 + i];
+                        for (int i = 0; i < NV8; ++i) {
+                            const int j = g * (BVS / 8) + c0 / 8 + i;  // 16-byte chunk of the row
+                            vw[i] = *reinterpret_cast<const uint4*>(
+                                vst + ((L::V_SWZ ? (j ^ (r & 7)) : j) << 4));
+                        }
                         tmem_wait_ld();
 #pragma unroll
                         for (int i = 0; i < NV8; ++i) {
@@ -689,12 +714,15 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 // reading the slot is complete: expect chunk c + npc in it and credit the prep
                 // CTA that owns that chunk (an output-side thread, off the residual path)
                 mbar_wait(sb(B_STATE, NSUB - 1), (uint32_t)((c + 1) & 1), abort_flag);
+                mbar_wait(bar(B_MMA2), (uint32_t)(c & 1), abort_flag);
                 mbar_arrive_expect_tx(cprep(pc), L::SLOT_B);
                 mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + (c + npc) % NP), owner_of(c + npc)));
             }
             // ---- outputs O = gamma_t (S0 q_t) + (P T Y)_t, overlapping the next residuals
             if (r >= 64) {
                 const int t = r - 64;
+                mbar_wait(bar(B_MMA2), (uint32_t)(c & 1), abort_flag);
+                tc_fence_after();
 #pragma unroll
                 for (int g = 0; g < NSUB; ++g) {
                     uint4* dst = reinterpret_cast<uint4*>(out + (bh * T + t0 + t) * (long)dv + v0 +
@@ -1279,7 +1307,7 @@ int launch_chunked_bv(const void* q, const void* k, const void* v, const float* 
     CUtensorMap mk, mq, mv;
     if (!make_map_3d(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, BH, T, CDK, 64, true) ||
         !make_map_3d(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, BH, T, CDK, 64, true) ||
-        !make_map_3d(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, BH, T, dv, BV, false))
+        !make_map_3d(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, BH, T, dv, BV, L::V_SWZ))
         return DR_ERR_CUDA;
     const int smem = L::TOTAL + 1024;
     auto kern = dr_chunked_kernel<MODE, BV, SPLIT>;
