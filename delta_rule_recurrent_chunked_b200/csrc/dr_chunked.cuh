@@ -86,6 +86,9 @@ struct ChunkLayout {
     // gamma vector. Contiguous, so that one bulk copy hands it to another CTA of the cluster.
     static constexpr int SLOT_TP = 0, SLOT_KH = 16384, SLOT_GAM = 32768;
     static constexpr int SLOT_B = 32768 + 1024;
+    // A split cluster copies only what the chain reads: PT rows, Khat^T and the gammas (the
+    // T rows feed the prep CTA's own PT and H; the chain's MMA2 rows 0-63 are never read).
+    static constexpr int COPY_OFF = SLOT_TP + 8192, COPY_B = SLOT_GAM + 512 - COPY_OFF;
 
     // prep temporaries of one group: P (64 rows, A operand of an M=64 MMA), Ttilde (GDN:
     // diag(gamma_C/gamma) T), A then X = (I+A)^{-1} (fp32 [64][68]), block scratch [32][36]
@@ -168,7 +171,8 @@ enum ChunkBar {
     B_ODONE = 30,      // [2] split chain CTA: sub-chain g's output rows are read out of TMEM
     B_PREP2 = 32,      // split chain CTA: third slot ready
     B_MMA2 = 33,       // split chain CTA: MMA2 done (MMA3 done is B_MMA23)
-    B_COUNT = 34
+    B_SFREE = 34,      // [3] split chain CTA: chain slot i read by every thread and every MMA
+    B_COUNT = 37
 };
 
 // bf16 bits of 8 consecutive columns of a row, stored as one 16-byte swizzled chunk.
@@ -305,6 +309,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
         }
         mbar_init(bar(B_PREP2), 1);
         mbar_init(bar(B_MMA2), 1);
+        for (int i = 0; i < 3; ++i) mbar_init(bar(B_SFREE + i), 129);  // 128 chain threads + MMA2
         const uint32_t gthreads = 256 / NGR;  // threads per prep group
         mbar_init(bar(B_GO), gthreads);
         mbar_init(bar(B_GRAM), 1);
@@ -337,14 +342,18 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
     tc_fence_after();
     const uint32_t tmem = *tmem_holder;
 
-    if (warp == 0) {
+    if (warp == 0 || (SPLIT && warp == 4 && !is_chain)) {
         // ------------------------------------------------------------------ producer
+        // (a split prep CTA gives each prep group's K/Q stage its own producer: warp 0 loads
+        // the even positions m, warp 4 the odd ones, so neither waits on the other's group)
+        const int mstep = (SPLIT && !is_chain) ? 2 : 1;
+        const int mfirst = (SPLIT && !is_chain && warp == 4) ? 1 : 0;
         if (lane == 0) {
             tma_prefetch_desc(&tmK);
             tma_prefetch_desc(&tmQ);
             tma_prefetch_desc(&tmV);
         }
-        for (int m = 0;; ++m) {
+        for (int m = mfirst;; m += mstep) {
             const int c = chunk_of(m);
             if (c >= nchunks) break;
             const int s = m % NS;
@@ -381,8 +390,6 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     }
                 }
                 x1 += __shfl_sync(0xffffffffu, x0, 31);
-                if (SPLIT && is_chain && lane == 31)  // gamma_C ring for the chain warpgroup
-                    reinterpret_cast<float*>(sm + L::PG)[c & 3] = __expf(x1);
                 bg[64 + lane] = x0;
                 bg[96 + lane] = x1;
                 bg[128 + lane] = __expf(-x0);
@@ -423,47 +430,55 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 mbar_wait(bar(B_PEER_FREE + p), ph, abort_flag);
                 if (!*abort_flag) {
                     // into chain slot c % npc of every chain rank
-                    const uint32_t src = smem_u32(slot(p));
-                    const uint32_t dst = smem_u32(cslot(c % npc));
+                    const uint32_t src = smem_u32(slot(p)) + L::COPY_OFF;
+                    const uint32_t dst = smem_u32(cslot(c % npc)) + L::COPY_OFF;
                     for (int q = NPREP; q < NPREP + NCC; ++q)  // the chain ranks
-                        bulk_copy_to_peer(cluster_map(dst, q), src, L::SLOT_B,
+                        bulk_copy_to_peer(cluster_map(dst, q), src, L::COPY_B,
                                           cluster_map(cprep(c % npc), q));
                     bulk_commit_and_wait_read();
                 }
                 mbar_arrive(bar(B_SLOT_EMPTY + p));
             }
         }
-    } else if (warp == 1) {
+    } else if (warp == 1 || (SPLIT && warp == 2 && is_chain)) {
         // ------------------------------------------------------------------ chain MMA issuer
-        // per sub-chain g: MMA1 once its state copy is ready, MMA2/MMA3 once its Y is ready
+        // Unsplit: warp 1 issues MMA1, MMA2 and MMA3. Split chain CTA: warp 1 issues MMA1 (it
+        // needs only K/Q and the state copy), warp 2 the state update MMA3 and then MMA2, so
+        // neither issuer's waits delay the other's step of the chain.
         if (lane == 0) {
             constexpr int NSUB = L::NSUB;
             constexpr uint32_t id1 = idesc_bf16(128, L::NB, 0, 1);
+            const bool do_mma1 = warp == 1, do_mma23 = !SPLIT || warp == 2;
             auto sb = [&](int base, int g) { return bar(base + (g ? B_SUB1 - B_MMA1 : 0)); };
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c % NS;
                 uint8_t* kq = sm + L::KQ + s * L::KQ_B;
-                mbar_wait(bar(B_KQ_FULL + s), (uint32_t)((c / NS) & 1), abort_flag);
-                mbar_wait(cprep(c % npc), (uint32_t)((c / npc) & 1), abort_flag);
+                if (do_mma1) {
+                    mbar_wait(bar(B_KQ_FULL + s), (uint32_t)((c / NS) & 1), abort_flag);
+                    if constexpr (!SPLIT)
+                        mbar_wait(cprep(c % npc), (uint32_t)((c / npc) & 1), abort_flag);
 #pragma unroll
-                for (int g = 0; g < NSUB; ++g) {
-                    mbar_wait(sb(B_STATE, g), (uint32_t)(c & 1), abort_flag);
-                    tc_fence_after();
-                    if (!*abort_flag) {
-                        const uint8_t* ss = sm + L::SS + g * 16384;
-                        const uint32_t d1 = L::COL_D1 + 64 * g + (SPLIT ? 128 * (c & 1) : 0);
+                    for (int g = 0; g < NSUB; ++g) {
+                        mbar_wait(sb(B_STATE, g), (uint32_t)(c & 1), abort_flag);
+                        tc_fence_after();
+                        if (!*abort_flag) {
+                            const uint8_t* ss = sm + L::SS + g * 16384;
+                            const uint32_t d1 = L::COL_D1 + 64 * g + (SPLIT ? 128 * (c & 1) : 0);
 #pragma unroll
-                        for (int kk = 0; kk < 8; ++kk) {
-                            const int pn = kk >> 2, ko = (kk & 3) * 32;
-                            tc_mma_bf16(tmem + d1,
-                                        smem_desc_sw128(smem_u32(kq + pn * 16384 + ko), 16, 1024),
-                                        smem_desc_sw128(smem_u32(ss + kk * 2048), 16384, 1024), id1,
-                                        kk > 0);
+                            for (int kk = 0; kk < 8; ++kk) {
+                                const int pn = kk >> 2, ko = (kk & 3) * 32;
+                                tc_mma_bf16(tmem + d1,
+                                            smem_desc_sw128(smem_u32(kq + pn * 16384 + ko), 16, 1024),
+                                            smem_desc_sw128(smem_u32(ss + kk * 2048), 16384, 1024),
+                                            id1, kk > 0);
+                            }
+                            tc_commit(sb(B_MMA1, g));
                         }
-                        tc_commit(sb(B_MMA1, g));
                     }
+                    if (!*abort_flag) tc_commit(bar(B_KQ_EMPTY + s));
                 }
-                if (!*abort_flag) tc_commit(bar(B_KQ_EMPTY + s));
+                if (!do_mma23) continue;
+                if constexpr (SPLIT) mbar_wait(cprep(c % npc), (uint32_t)((c / npc) & 1), abort_flag);
                 const uint8_t* tp = cslot(c % npc) + L::SLOT_TP;
                 const uint8_t* kh = cslot(c % npc) + L::SLOT_KH;
 #pragma unroll
@@ -499,6 +514,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                         if (!*abort_flag) {
                             mma2();
                             tc_commit(bar(B_MMA2));
+                            tc_commit(bar(B_SFREE + c % npc));  // last reader of the slot
                         }
                     } else {
                         if (!*abort_flag) {
@@ -570,33 +586,37 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
     } else if (warp >= 4 && warp < 8 && SPLIT) {
         if (!is_chain) goto done;
         // ------------------------------------------------------------------ chain warpgroup,
-        // split chain CTA: two sub-chains of BVS value channels, interleaved. Threads 0-63
-        // (TMEM lanes of the K rows) write the residuals, threads 64-127 (Q rows) the outputs,
-        // all 128 (lane = key channel) the carried state. Per chunk: residuals of both
-        // sub-chains; then each sub-chain's state, already scaled by the next chunk's gamma_C
-        // (from the producer's ring) and handed straight to MMA1; then the outputs, which
-        // overlap the next chunk's residuals.
+        // split chain CTA. Threads 0-63 (TMEM lanes of the K rows) write the residuals,
+        // threads 64-127 (Q rows) the outputs, all 128 (lane = key channel) the carried state.
+        // Per chunk: the residuals; then the state, already scaled by the next chunk's gamma_C
+        // and handed straight to MMA1; then the outputs, which overlap the next chunk's
+        // residuals. (Written for NSUB interleaved column sets; NSUB is 1.)
         constexpr int NSUB = L::NSUB, BVS = L::BVS;
         constexpr int LW = BVS < 16 ? 16 : BVS;  // TMEM columns read per sub-chain
         constexpr int PW = LW < 32 ? LW : 32;    // columns per epilogue piece (registers)
         const int r = tid - 128;  // TMEM lane: value row t (Y, O) or key channel j (state)
         const uint32_t trow = tmem + ((uint32_t)(r & ~31) << 16);
-        const float* gcr = reinterpret_cast<const float*>(sm + L::PG);  // gamma_C by chunk % 4
         auto sb = [&](int base, int g) { return bar(base + (g ? B_SUB1 - B_MMA1 : 0)); };
+        // gamma_t of row r & 63 for the next chunk: each chunk's slot is waited for, and its
+        // gammas read, one chunk ahead (under the previous chunk's MMA3 latency)
+        float gt_next = 1.f;
         {
             // slots start empty: expect the prep CTAs' copies of the first chunks
             if (r == 0) {
                 for (int c = 0; c < npc && c < nchunks; ++c) {
-                    mbar_arrive_expect_tx(cprep(c), L::SLOT_B);
+                    mbar_arrive_expect_tx(cprep(c), L::COPY_B);
                     mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + c % NP), owner_of(c)));
                 }
             }
             float gC0 = 1.f;
-            if constexpr (kGdn) {
-                if (nchunks > 0) {
-                    mbar_wait(bar(B_KQ_FULL + 0), 0u, abort_flag);
-                    gC0 = gcr[0];
+            if (nchunks > 0) {
+                mbar_wait(cprep(0), 0u, abort_flag);
+                if constexpr (kGdn) {
+                    const float* gam = reinterpret_cast<const float*>(cslot(0) + L::SLOT_GAM);
+                    gt_next = gam[r & 63];
+                    gC0 = gam[64];
                 }
+                mbar_arrive(bar(B_SFREE + 0));  // this thread is done reading slot 0
             }
             const float* src = S0 ? S0 + (bh * dv + v0) * (long)CDK + r : nullptr;
 #pragma unroll
@@ -626,18 +646,8 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             const int t0 = c * CK;
             const int nvalid = min(CK, T - t0);
             const uint32_t d1 = L::COL_D1 + 128 * (c & 1);
-            const int pc = c % npc;  // chain slot of chunk c
-            mbar_wait(cprep(pc), (uint32_t)((c / npc) & 1), abort_flag);
-            const float gt = kGdn ? reinterpret_cast<const float*>(cslot(pc) + L::SLOT_GAM)[r & 63] : 1.f;
-            // gamma_C of the next chunk, from the producer's ring (its K/Q stage is loaded by now)
+            const float gt = gt_next;
             const bool last = c == nchunks - 1;
-            float gCn = 1.f;
-            if constexpr (kGdn) {
-                if (!last) {
-                    mbar_wait(bar(B_KQ_FULL + (c + 1) % NS), (uint32_t)(((c + 1) / NS) & 1), abort_flag);
-                    gCn = gcr[(c + 1) & 3];
-                }
-            }
             // ---- residuals Y = V - gamma_t (S0 k_t) of both sub-chains
             if (r < 64) {
 #pragma unroll
@@ -676,7 +686,19 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 }
             }
             // ---- carried states: bf16 copy for MMA1 of the next chunk, fp32 S_final after
-            // the last; the fp32 state takes the next chunk's gamma_C before its MMA3
+            // the last; the fp32 state takes the next chunk's gamma_C (from its slot, waited
+            // here under the MMA3 latency) before that chunk's MMA3
+            float gCn = 1.f;
+            if (!last) {
+                const int pn = (c + 1) % npc;
+                mbar_wait(cprep(pn), (uint32_t)(((c + 1) / npc) & 1), abort_flag);
+                if constexpr (kGdn) {
+                    const float* gam = reinterpret_cast<const float*>(cslot(pn) + L::SLOT_GAM);
+                    gt_next = gam[r & 63];
+                    gCn = gam[64];
+                }
+                mbar_arrive(bar(B_SFREE + pn));  // this thread is done reading that slot
+            }
 #pragma unroll
             for (int g = 0; g < NSUB; ++g) {
                 mbar_wait(sb(B_MMA23, g), (uint32_t)(c & 1), abort_flag);
@@ -708,15 +730,6 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 fence_async_smem();
                 tc_fence_before();
                 mbar_arrive(sb(B_STATE, g));
-            }
-            if (r == 64 && c + npc < nchunks) {
-                // every thread read the slot's gammas before its state arrival and every MMA
-                // reading the slot is complete: expect chunk c + npc in it and credit the prep
-                // CTA that owns that chunk (an output-side thread, off the residual path)
-                mbar_wait(sb(B_STATE, NSUB - 1), (uint32_t)((c + 1) & 1), abort_flag);
-                mbar_wait(bar(B_MMA2), (uint32_t)(c & 1), abort_flag);
-                mbar_arrive_expect_tx(cprep(pc), L::SLOT_B);
-                mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + (c + npc) % NP), owner_of(c + npc)));
             }
             // ---- outputs O = gamma_t (S0 q_t) + (P T Y)_t, overlapping the next residuals
             if (r >= 64) {
@@ -910,6 +923,19 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 }
             }
             if (c + 1 < nchunks) prescale(c + 1);
+        }
+    } else if (SPLIT && warp == 8 && is_chain) {
+        // ------------------------------------------------------------------ slot releaser
+        // (split chain CTA): once every chain thread and every MMA is done with chain slot
+        // c % npc, expect chunk c + npc in it and credit the prep CTA that owns that chunk.
+        // The slot's next phase needs this release, so the waits here never fall two phases
+        // behind.
+        if (lane == 0) {
+            for (int c = 0; c + npc < nchunks; ++c) {
+                mbar_wait(bar(B_SFREE + c % npc), (uint32_t)((c / npc) & 1), abort_flag);
+                mbar_arrive_expect_tx(cprep(c % npc), L::COPY_B);
+                mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + (c + npc) % NP), owner_of(c + npc)));
+            }
         }
     } else if (warp >= 8) {
         if (!is_prep) goto done;
