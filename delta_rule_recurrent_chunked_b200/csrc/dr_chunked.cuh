@@ -272,18 +272,20 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
     constexpr bool split = SPLIT;
     const int NPREP = SPLIT ? nprep : 1;
     constexpr int NGR = SPLIT ? 2 : 1;  // prep groups per prep CTA
-    const int SP = NGR * NPREP;                // chunk stride of one prep group
     const int rank = split ? (int)blockIdx.y : 0;
     const int NCC = split ? (int)gridDim.y - NPREP : 1;  // chain CTAs per head
     const bool is_prep = !split || rank < NPREP;
     const bool is_chain = !split || rank >= NPREP;
     const int v0 = (split ? rank - NPREP : (int)blockIdx.y) * BV;
-    // The chunks this CTA loads, in order: all of them, or (prep CTA of a split cluster)
-    // chunk_of(m) = base + (m / NGR) * SP + m % NGR; ordinal_of inverts it.
-    const int pG = is_chain ? 1 : NGR, pSP = is_chain ? 1 : SP, pbase = is_chain ? 0 : rank * NGR;
-    auto chunk_of = [&](int m) { return pbase + (m / pG) * pSP + m % pG; };
-    auto ordinal_of = [&](int c) { return ((c - pbase) / pSP) * pG + (c - pbase) % pG; };
-    auto owner_of = [&](int c) { return (c / NGR) % NPREP; };  // prep rank of chunk c
+    // Chunks are dealt to the prep CTAs one at a time, so consecutive chunks are prepared and
+    // copied by different CTAs. The chunks this CTA loads, in order: all of them, or (prep
+    // CTA of a split cluster) chunk_of(m) = rank + m * NPREP; ordinal_of inverts it. A prep
+    // CTA's groups take alternate ordinals and its prepared-operand slots follow the ordinal.
+    const int pSP = is_chain ? 1 : NPREP, pbase = is_chain ? 0 : rank;
+    auto chunk_of = [&](int m) { return pbase + m * pSP; };
+    auto ordinal_of = [&](int c) { return (c - pbase) / pSP; };
+    auto owner_of = [&](int c) { return c % NPREP; };           // prep rank of chunk c
+    auto pslot_of = [&](int c) { return (c / NPREP) % NP; };    // its slot in that prep CTA
     // Chain-side slot ring: NP slots, or three in a split cluster with two or more prep CTAs
     // (then no two of the first three chunks share a prep CTA and prep slot, so the initial
     // credits complete distinct barrier phases).
@@ -424,7 +426,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             for (int m = 0;; ++m) {
                 const int c = chunk_of(m);
                 if (c >= nchunks) break;
-                const int p = c % NP;
+                const int p = m % NP;
                 const uint32_t ph = (uint32_t)((m / NP) & 1);
                 mbar_wait(bar(B_PREP + p), ph, abort_flag);
                 mbar_wait(bar(B_PEER_FREE + p), ph, abort_flag);
@@ -540,8 +542,8 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             uint8_t* pm = sm + (gi ? L::PM2 : L::PM);
             uint8_t* tts = sm + (gi ? L::TTS2 : L::TTS);
             int k = 0;  // the group's chunk ordinal
-            for (int c = pbase + gi; c < nchunks; c += SP, ++k) {
-                const int s = ordinal_of(c) % NS, p = c % NP;
+            for (int c = pbase + gi * pSP; c < nchunks; c += NGR * pSP, ++k) {
+                const int s = ordinal_of(c) % NS, p = ordinal_of(c) % NP;
                 uint8_t* kq = sm + L::KQ + s * L::KQ_B;
                 uint8_t* kn = sm + L::KN;
                 const uint32_t jp = (uint32_t)(k & 1);
@@ -605,7 +607,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             if (r == 0) {
                 for (int c = 0; c < npc && c < nchunks; ++c) {
                     mbar_arrive_expect_tx(cprep(c), L::COPY_B);
-                    mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + c % NP), owner_of(c)));
+                    mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + pslot_of(c)), owner_of(c)));
                 }
             }
             float gC0 = 1.f;
@@ -934,7 +936,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             for (int c = 0; c + npc < nchunks; ++c) {
                 mbar_wait(bar(B_SFREE + c % npc), (uint32_t)((c / npc) & 1), abort_flag);
                 mbar_arrive_expect_tx(cprep(c % npc), L::COPY_B);
-                mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + (c + npc) % NP), owner_of(c + npc)));
+                mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + pslot_of(c + npc)), owner_of(c + npc)));
             }
         }
     } else if (warp >= 8) {
@@ -973,9 +975,9 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             }
         }
         int k = 0;  // the group's chunk ordinal
-        for (int c = pbase + gi; c < nchunks; c += SP, ++k) {
+        for (int c = pbase + gi * pSP; c < nchunks; c += NGR * pSP, ++k) {
             const int mo = ordinal_of(c);  // position among the chunks this CTA loads
-            const int s = mo % NS, p = c % NP;
+            const int s = mo % NS, p = mo % NP;
             const uint32_t jp = (uint32_t)(k & 1);
             const int t0 = c * CK;
             const int nvalid = min(CK, T - t0);
@@ -1040,7 +1042,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 if (kq4 == 3) *reinterpret_cast<float2*>(pg + 512 + kc) = run;  // gamma_C
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    const int tn = (c + SP) * CK + 16 * kq4 + i;
+                    const int tn = (c + NGR * pSP) * CK + 16 * kq4 + i;
                     gpf[i] = tn < T ? *reinterpret_cast<const float2*>(gate + (bh * T + tn) * (long)CDK + kc)
                                     : make_float2(1.f, 1.f);
                 }
