@@ -32,6 +32,7 @@ SIGNATURES = {
     "dr_status_string": ([_I], ctypes.c_char_p),
     "dr_poll_error": ([_VP], _I),
     "dr_debug_timeout_probe": ([_I, _VP], _I),
+    "dr_chunked_plan": ([_I, ctypes.c_longlong, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I)], _I),
     "dr_version": ([], _I),
 }
 
@@ -162,6 +163,20 @@ def poll_error(device=None) -> int:
 
     dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
     return int(lib().dr_poll_error(_stream_handle(dev)))
+
+
+def chunked_plan(mode, BH: int, dk: int, dv: int) -> tuple:
+    """(value channels per chain CTA, prep CTAs per head; 0 = unsplit) that dr_scan_fwd uses
+    for bf16 inputs on the current device, or None when the chunked kernel does not apply."""
+    variant = MODES[mode] if isinstance(mode, str) else int(mode)
+    bv, nprep = ctypes.c_int(0), ctypes.c_int(0)
+    st = lib().dr_chunked_plan(variant | DR_IN_BF16, int(BH), int(dk), int(dv),
+                               ctypes.byref(bv), ctypes.byref(nprep))
+    if st == DR_ERR_UNSUPPORTED:
+        return None
+    if st != DR_OK:
+        raise DrScanError(st, "dr_chunked_plan")
+    return bv.value, nprep.value
 
 
 def chunked_applies(mode, dtype_is_bf16: bool, dk: int, dv: int) -> bool:

@@ -112,6 +112,12 @@ __device__ __forceinline__ void bulk_copy_to_peer(uint32_t cluster_dst, uint32_t
         : "memory");
 }
 
+// Waits until every bulk copy this thread committed has fully completed, destination writes
+// included (not only the source reads).
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 __device__ __forceinline__ void bulk_commit_and_wait_read() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
     asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");

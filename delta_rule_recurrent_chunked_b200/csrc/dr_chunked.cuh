@@ -441,6 +441,9 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 }
                 mbar_arrive(bar(B_SLOT_EMPTY + p));
             }
+            // No copy may still be writing into a chain CTA when the cluster's final barrier
+            // lets it exit (after a timeout its chain no longer waits for every slot).
+            bulk_wait_all();
         }
     } else if (warp == 1 || (SPLIT && warp == 2 && is_chain)) {
         // ------------------------------------------------------------------ chain MMA issuer

@@ -234,6 +234,22 @@ int dr_poll_error(cudaStream_t stream) {
     return status;
 }
 
+int dr_chunked_plan(int mode, long long BH, int dk, int dv, int* bv, int* nprep) {
+    if (!bv || !nprep) return DR_ERR_INVALID_ARG;
+    *bv = 0;
+    *nprep = 0;
+    const int variant = mode & DR_MODE_MASK;
+    if (mode & ~(DR_MODE_MASK | DR_IN_BF16 | DR_FORCE_SEQUENTIAL)) return DR_ERR_INVALID_ARG;
+    if (BH < 1 || BH > INT_MAX) return DR_ERR_INVALID_ARG;
+    if (!(mode & DR_IN_BF16) || (mode & DR_FORCE_SEQUENTIAL) ||
+        !drscan::chunked_supported(variant, dk, dv))
+        return DR_ERR_UNSUPPORTED;
+    const drscan::SplitPlan plan = drscan::pick_split(variant, (long)BH, dv);
+    *nprep = plan.nprep;
+    *bv = plan.nprep ? plan.bv : drscan::pick_bv(variant, (long)BH, dv);
+    return DR_OK;
+}
+
 int dr_debug_timeout_probe(int spin_limit, cudaStream_t stream) {
     if (spin_limit < 1 || spin_limit > 1000000) return DR_ERR_INVALID_ARG;
     timeout_probe_kernel<<<1, 32, 0, stream>>>(spin_limit);

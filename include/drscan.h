@@ -122,6 +122,20 @@ const char* dr_status_string(int status);
 int dr_poll_error(cudaStream_t stream);
 
 /*
+ * The launch shape dr_scan_fwd picks for the chunked tensor-core kernel on the current
+ * device, for `BH` = B*H sequences and the same `mode` word (variant | flags):
+ *   *bv    value channels per chain CTA;
+ *   *nprep prep CTAs per head in a split cluster (a cluster of *nprep prep CTAs and dv/(*bv)
+ *          chain CTAs per head, used when the heads are too few to fill the GPU), or 0 when
+ *          one CTA per (head, value slice) does both sides.
+ * Returns DR_OK; DR_ERR_UNSUPPORTED (both set to 0) when the request would run the
+ * per-token kernel instead (fp32 inputs, DR_FORCE_SEQUENTIAL, dk != 128, dv not in
+ * {32, 64, 128}, or plain linear attention); DR_ERR_INVALID_ARG for null pointers, BH < 1
+ * or unknown mode bits. Launches nothing; queries the device's cluster occupancy once.
+ */
+int dr_chunked_plan(int mode, long long BH, int dk, int dv, int* bv, int* nprep);
+
+/*
  * Test hook for the failure path: launches a one-block kernel on `stream` that waits on
  * a shared-memory barrier nothing ever arrives on, with a spin limit of `spin_limit`
  * polls, then latches DR_ERR_TIMEOUT and returns. Nothing faults or hangs.

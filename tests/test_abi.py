@@ -115,6 +115,25 @@ def test_timeout_probe_rejects_bad_limits(lib):
     assert lib.dr_debug_timeout_probe(10**7, None) == drs.DR_ERR_INVALID_ARG
 
 
+def test_chunked_plan_rejects_before_querying_the_device(lib):
+    bv, npr = ctypes.c_int(-1), ctypes.c_int(-1)
+    call = lambda mode, BH, dk, dv, a=ctypes.byref(bv), b=ctypes.byref(npr): \
+        lib.dr_chunked_plan(mode, BH, dk, dv, a, b)
+    assert call(drs.DR_GDN | drs.DR_IN_BF16, 4, 128, 128, None, None) == drs.DR_ERR_INVALID_ARG
+    assert call(drs.DR_GDN | drs.DR_IN_BF16, 0, 128, 128) == drs.DR_ERR_INVALID_ARG
+    assert call(drs.DR_GDN | 0x4000, 4, 128, 128) == drs.DR_ERR_INVALID_ARG
+    # fp32 inputs, forced sequential, other shapes and plain linear attention use the
+    # per-token kernel: no plan, both outputs zeroed
+    for mode, dk, dv in [(drs.DR_GDN, 128, 128),
+                         (drs.DR_GDN | drs.DR_IN_BF16 | drs.DR_FORCE_SEQUENTIAL, 128, 128),
+                         (drs.DR_GDN | drs.DR_IN_BF16, 64, 128),
+                         (drs.DR_KDA | drs.DR_IN_BF16, 128, 96),
+                         (drs.DR_LINEAR | drs.DR_IN_BF16, 128, 128)]:
+        bv.value, npr.value = -1, -1
+        assert call(mode, 4, dk, dv) == drs.DR_ERR_UNSUPPORTED
+        assert (bv.value, npr.value) == (0, 0)
+
+
 def test_product_path_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(drs, "LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(drs, "_lib", None)

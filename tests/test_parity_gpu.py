@@ -84,6 +84,24 @@ def test_bf16_dispatch_narrow_values(oracle, mode, dv):
     check_dr(oracle, w, seed=dv)
 
 
+# Every branch of the chunked kernel's launch plan: a split cluster with two prep CTAs and a
+# three-deep chain slot ring (few heads), with one prep CTA and a two-deep ring, and one CTA
+# per (head, value slice) once the heads fill the GPU. The plan is read back so that a change
+# of the planner cannot silently drop a branch from the tests.
+@pytest.mark.parametrize("mode", [wl.DELTANET, wl.GDN])
+@pytest.mark.parametrize("BH,dv,split", [(2, 128, 2), (40, 128, 1), (40, 64, 1), (46, 128, None),
+                                         (64, 128, 0), (64, 32, 0)])
+def test_bf16_plan_branches(oracle, mode, BH, dv, split):
+    plan = drs.chunked_plan(mode, BH, 128, dv)
+    assert plan is not None
+    bv, nprep = plan
+    assert dv % bv == 0
+    if split is not None:
+        assert nprep == split, plan
+    w = wl.DRWorkload("t", 1, BH, 300, 128, dv, mode, "bf16", s0_std=0.1)
+    check_dr(oracle, w, seed=BH + dv)
+
+
 def test_bf16_strong_decay_gates(oracle):
     # gates near 0.5 per step: summed log-decay over a 64-token chunk reaches about -45
     w = wl.DRWorkload("t", 1, 2, 256, 128, 128, wl.GDN, "bf16", gate_mu=0.0, gate_sigma=0.5)
