@@ -304,14 +304,14 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             mbar_init(bar(B_KQ_FULL + s), 2);
             mbar_init(bar(B_KQ_EMPTY + s), split ? 1 : 2);
             mbar_init(bar(B_V_FULL + s), 1);
-            mbar_init(bar(B_V_EMPTY + s), 64);
+            mbar_init(bar(B_V_EMPTY + s), SPLIT ? 128 : 64);  // residual threads
             mbar_init(bar(B_PREP + s), 1);
             mbar_init(bar(B_SLOT_EMPTY + s), 1);
             mbar_init(bar(B_PEER_FREE + s), split ? NCC : 1);
         }
         mbar_init(bar(B_PREP2), 1);
         mbar_init(bar(B_MMA2), 1);
-        for (int i = 0; i < 3; ++i) mbar_init(bar(B_SFREE + i), 129);  // 128 chain threads + MMA2
+        for (int i = 0; i < 3; ++i) mbar_init(bar(B_SFREE + i), 257);  // 256 chain threads + MMA2
         const uint32_t gthreads = 256 / NGR;  // threads per prep group
         mbar_init(bar(B_GO), gthreads);
         mbar_init(bar(B_GRAM), 1);
@@ -321,14 +321,14 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
         mbar_init(bar(B_GRP1 + 1), 1);
         mbar_init(bar(B_GRP1 + 2), gthreads);
         mbar_init(bar(B_GRP1 + 3), 1);
-        mbar_init(bar(B_ODONE + 0), 64);
+        mbar_init(bar(B_ODONE + 0), SPLIT ? 128 : 64);
         mbar_init(bar(B_ODONE + 1), 64);
         for (int g = 0; g < 2; ++g) {
             const int o = g ? B_SUB1 - B_MMA1 : 0;
             mbar_init(bar(B_MMA1 + o), 1);
-            mbar_init(bar(B_YREADY + o), SPLIT ? 64 : 128);
+            mbar_init(bar(B_YREADY + o), 128);
             mbar_init(bar(B_MMA23 + o), 1);
-            mbar_init(bar(B_STATE + o), 128);
+            mbar_init(bar(B_STATE + o), SPLIT ? 256 : 128);
         }
         *abort_flag = 0;
         mbar_init_fence();
@@ -588,26 +588,29 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 }
             }
         }
-    } else if (warp >= 4 && warp < 8 && SPLIT) {
-        if (!is_chain) goto done;
-        // ------------------------------------------------------------------ chain warpgroup,
-        // split chain CTA. Threads 0-63 (TMEM lanes of the K rows) write the residuals,
-        // threads 64-127 (Q rows) the outputs, all 128 (lane = key channel) the carried state.
+    } else if (SPLIT && is_chain && warp >= 4 && warp < 12) {
+        // ------------------------------------------------------------------ chain warpgroups
+        // of a split chain CTA. Warps 4-7 and 8-11 reach the same TMEM lanes and share the
+        // value columns: warpgroup h takes HC columns from cb (with 16 channels the second only
+        // keeps the barrier counts). Threads 0-63 of each (TMEM lanes of the K rows) write the
+        // residuals, threads 64-127 (Q rows) the outputs, all (lane = key channel) the state.
         // Per chunk: the residuals; then the state, already scaled by the next chunk's gamma_C
-        // and handed straight to MMA1; then the outputs, which overlap the next chunk's
-        // residuals. (Written for NSUB interleaved column sets; NSUB is 1.)
-        constexpr int NSUB = L::NSUB, BVS = L::BVS;
-        constexpr int LW = BVS < 16 ? 16 : BVS;  // TMEM columns read per sub-chain
-        constexpr int PW = LW < 32 ? LW : 32;    // columns per epilogue piece (registers)
-        const int r = tid - 128;  // TMEM lane: value row t (Y, O) or key channel j (state)
+        // and handed straight to MMA1; then the outputs, which overlap the next residuals.
+        const int h = warp >= 8 ? 1 : 0;
+        constexpr int HC = BV >= 32 ? BV / 2 : BV;  // columns per warpgroup
+        const bool active = BV >= 32 || h == 0;
+        const int cb = h * HC;                     // first column (0, 16 or 32)
+        constexpr int LW = HC < 16 ? 16 : HC;      // TMEM columns read (one piece: <= 32)
+        constexpr int NV8 = HC / 8;                // real 8-column chunks
+        static_assert(!SPLIT || LW <= 32, "one epilogue piece per warpgroup");
+        const int r = tid - (h ? 256 : 128);  // TMEM lane: row t (Y, O) or key channel j (state)
         const uint32_t trow = tmem + ((uint32_t)(r & ~31) << 16);
-        auto sb = [&](int base, int g) { return bar(base + (g ? B_SUB1 - B_MMA1 : 0)); };
         // gamma_t of row r & 63 for the next chunk: each chunk's slot is waited for, and its
         // gammas read, one chunk ahead (under the previous chunk's MMA3 latency)
         float gt_next = 1.f;
         {
             // slots start empty: expect the prep CTAs' copies of the first chunks
-            if (r == 0) {
+            if (h == 0 && r == 0) {
                 for (int c = 0; c < npc && c < nchunks; ++c) {
                     mbar_arrive_expect_tx(cprep(c), L::COPY_B);
                     mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + pslot_of(c)), owner_of(c)));
@@ -623,28 +626,31 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 }
                 mbar_arrive(bar(B_SFREE + 0));  // this thread is done reading slot 0
             }
-            const float* src = S0 ? S0 + (bh * dv + v0) * (long)CDK + r : nullptr;
-#pragma unroll
-            for (int g = 0; g < NSUB; ++g) {
+            if (active) {
+                const float* src = S0 ? S0 + (bh * dv + v0 + cb) * (long)CDK + r : nullptr;
                 float sv[LW];
 #pragma unroll
-                for (int v = 0; v < LW; ++v)
-                    sv[v] = (src && v < BVS) ? src[(long)(g * BVS + v) * CDK] : 0.f;
+                for (int v = 0; v < LW; ++v) sv[v] = (src && v < HC) ? src[(long)v * CDK] : 0.f;
 #pragma unroll
-                for (int i = 0; i < BVS / 8; ++i) st_row_chunk(sm + L::SS + g * 16384, r, i, sv + 8 * i);
+                for (int i = 0; i < NV8; ++i) st_row_chunk(sm + L::SS, r, cb / 8 + i, sv + 8 * i);
 #pragma unroll
-                for (int c16 = 0; c16 < 64; c16 += 16) {
+                for (int c16 = 0; c16 < LW; c16 += 16) {
                     float w[16];
 #pragma unroll
-                    for (int v = 0; v < 16; ++v) w[v] = c16 + v < LW ? sv[c16 + v] * gC0 : 0.f;
-                    tmem_st16(trow + L::COL_S + 64 * g + c16, w);
+                    for (int v = 0; v < 16; ++v) w[v] = sv[c16 + v] * gC0;
+                    tmem_st16(trow + L::COL_S + cb + c16, w);
                 }
+            }
+            if (h == 0) {  // the padding columns of the fp32 state start at zero
+                float w[16];
+#pragma unroll
+                for (int v = 0; v < 16; ++v) w[v] = 0.f;
+                for (int c16 = (BV + 15) / 16 * 16; c16 < 64; c16 += 16) tmem_st16(trow + L::COL_S + c16, w);
             }
             tmem_wait_st();
             fence_async_smem();
             tc_fence_before();
-#pragma unroll
-            for (int g = 0; g < NSUB; ++g) mbar_arrive(sb(B_STATE, g));
+            mbar_arrive(bar(B_STATE));
         }
         for (int c = 0; c < nchunks; ++c) {
             const int svi = c % NSV;
@@ -653,46 +659,41 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             const uint32_t d1 = L::COL_D1 + 128 * (c & 1);
             const float gt = gt_next;
             const bool last = c == nchunks - 1;
-            // ---- residuals Y = V - gamma_t (S0 k_t) of both sub-chains
+            // ---- residuals Y = V - gamma_t (S0 k_t), stored as the B operand Y^T
             if (r < 64) {
-#pragma unroll
-                for (int g = 0; g < NSUB; ++g) {
-                    mbar_wait(sb(B_MMA1, g), (uint32_t)(c & 1), abort_flag);
+                if (active) {
+                    mbar_wait(bar(B_MMA1), (uint32_t)(c & 1), abort_flag);
                     tc_fence_after();
-                    if (g == 0) mbar_wait(bar(B_V_FULL + svi), (uint32_t)((c / NSV) & 1), abort_flag);
+                    mbar_wait(bar(B_V_FULL + svi), (uint32_t)((c / NSV) & 1), abort_flag);
                     const uint8_t* vst = sm + L::V + svi * L::V_B + r * BV * 2;  // row r of V
+                    float x[LW];
+                    uint4 vw[NV8];
 #pragma unroll
-                    for (int c0 = 0; c0 < LW; c0 += PW) {
-                        constexpr int NV8 = (PW < BVS ? PW : BVS) / 8;  // real 8-column chunks
-                        float x[PW];
-                        uint4 vw[NV8];
+                    for (int c16 = 0; c16 < LW; c16 += 16) tmem_ld16(trow + d1 + cb + c16, x + c16);
 #pragma unroll
-                        for (int c16 = 0; c16 < PW; c16 += 16) tmem_ld16(trow + d1 + 64 * g + c0 + c16, x + c16);
-#pragma unroll
-                        for (int i = 0; i < NV8; ++i) {
-                            const int j = g * (BVS / 8) + c0 / 8 + i;  // 16-byte chunk of the row
-                            vw[i] = *reinterpret_cast<const uint4*>(
-                                vst + ((L::V_SWZ ? (j ^ (r & 7)) : j) << 4));
-                        }
-                        tmem_wait_ld();
-#pragma unroll
-                        for (int i = 0; i < NV8; ++i) {
-                            const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&vw[i]);
-                            float y[8];
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) y[e] = fmaf(-gt, x[8 * i + e], __bfloat162float(hv[e]));
-                            st_row_chunk(sm + L::SY + g * 8192, r, c0 / 8 + i, y);
-                        }
+                    for (int i = 0; i < NV8; ++i) {
+                        const int j = cb / 8 + i;  // 16-byte chunk of the row
+                        vw[i] = *reinterpret_cast<const uint4*>(
+                            vst + ((L::V_SWZ ? (j ^ (r & 7)) : j) << 4));
                     }
-                    if (g == NSUB - 1) mbar_arrive(bar(B_V_EMPTY + svi));
-                    fence_async_smem();
-                    tc_fence_before();
-                    mbar_arrive(sb(B_YREADY, g));
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < NV8; ++i) {
+                        const __nv_bfloat16* hv = reinterpret_cast<const __nv_bfloat16*>(&vw[i]);
+                        float y[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) y[e] = fmaf(-gt, x[8 * i + e], __bfloat162float(hv[e]));
+                        st_row_chunk(sm + L::SY, r, cb / 8 + i, y);
+                    }
                 }
+                mbar_arrive(bar(B_V_EMPTY + svi));
+                fence_async_smem();
+                tc_fence_before();
+                mbar_arrive(bar(B_YREADY));
             }
-            // ---- carried states: bf16 copy for MMA1 of the next chunk, fp32 S_final after
-            // the last; the fp32 state takes the next chunk's gamma_C (from its slot, waited
-            // here under the MMA3 latency) before that chunk's MMA3
+            // ---- carried state: bf16 copy for MMA1 of the next chunk, fp32 S_final after the
+            // last; the fp32 state takes the next chunk's gamma_C (from its slot, waited here
+            // under the MMA3 latency) before that chunk's MMA3
             float gCn = 1.f;
             if (!last) {
                 const int pn = (c + 1) % npc;
@@ -704,74 +705,63 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 }
                 mbar_arrive(bar(B_SFREE + pn));  // this thread is done reading that slot
             }
+            mbar_wait(bar(B_MMA23), (uint32_t)(c & 1), abort_flag);
+            tc_fence_after();
+            if (active) {
+                float sv[LW];
 #pragma unroll
-            for (int g = 0; g < NSUB; ++g) {
-                mbar_wait(sb(B_MMA23, g), (uint32_t)(c & 1), abort_flag);
-                tc_fence_after();
+                for (int c16 = 0; c16 < LW; c16 += 16) tmem_ld16(trow + L::COL_S + cb + c16, sv + c16);
+                tmem_wait_ld();
 #pragma unroll
-                for (int c0 = 0; c0 < LW; c0 += PW) {
-                    constexpr int NV8 = (PW < BVS ? PW : BVS) / 8;
-                    float sv[PW];
+                for (int i = 0; i < NV8; ++i) st_row_chunk(sm + L::SS, r, cb / 8 + i, sv + 8 * i);
+                if (last && S_final) {
+                    float* dst = S_final + (bh * dv + v0 + cb) * (long)CDK + r;
 #pragma unroll
-                    for (int c16 = 0; c16 < PW; c16 += 16) tmem_ld16(trow + L::COL_S + 64 * g + c0 + c16, sv + c16);
-                    tmem_wait_ld();
+                    for (int v = 0; v < HC; ++v) dst[(long)v * CDK] = sv[v];
+                }
+                if constexpr (kGdn) {
+                    if (!last) {
 #pragma unroll
-                    for (int i = 0; i < NV8; ++i) st_row_chunk(sm + L::SS + g * 16384, r, c0 / 8 + i, sv + 8 * i);
-                    if (last && S_final) {
-                        float* dst = S_final + (bh * dv + v0 + g * BVS + c0) * (long)CDK + r;
+                        for (int v = 0; v < LW; ++v) sv[v] *= gCn;
 #pragma unroll
-                        for (int v = 0; v < 8 * NV8; ++v) dst[(long)v * CDK] = sv[v];
-                    }
-                    if constexpr (kGdn) {
-                        if (!last) {
-#pragma unroll
-                            for (int v = 0; v < PW; ++v) sv[v] *= gCn;
-#pragma unroll
-                            for (int c16 = 0; c16 < PW; c16 += 16) tmem_st16(trow + L::COL_S + 64 * g + c0 + c16, sv + c16);
-                        }
+                        for (int c16 = 0; c16 < LW; c16 += 16) tmem_st16(trow + L::COL_S + cb + c16, sv + c16);
+                        tmem_wait_st();
                     }
                 }
-                if constexpr (kGdn) tmem_wait_st();
-                fence_async_smem();
-                tc_fence_before();
-                mbar_arrive(sb(B_STATE, g));
             }
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar(B_STATE));
             // ---- outputs O = gamma_t (S0 q_t) + (P T Y)_t, overlapping the next residuals
             if (r >= 64) {
                 const int t = r - 64;
                 mbar_wait(bar(B_MMA2), (uint32_t)(c & 1), abort_flag);
                 tc_fence_after();
+                if (active) {
+                    float z[LW], dd[LW];
 #pragma unroll
-                for (int g = 0; g < NSUB; ++g) {
-                    uint4* dst = reinterpret_cast<uint4*>(out + (bh * T + t0 + t) * (long)dv + v0 +
-                                                          g * BVS);
+                    for (int c16 = 0; c16 < LW; c16 += 16) {
+                        tmem_ld16(trow + d1 + cb + c16, z + c16);
+                        tmem_ld16(trow + L::COL_D2 + cb + c16, dd + c16);
+                    }
+                    tmem_wait_ld();
+                    tc_fence_before();
+                    mbar_arrive(bar(B_ODONE));
+                    if (t < nvalid) {
+                        uint4* dst = reinterpret_cast<uint4*>(out + (bh * T + t0 + t) * (long)dv + v0 + cb);
 #pragma unroll
-                    for (int c0 = 0; c0 < LW; c0 += PW) {
-                        constexpr int NV8 = (PW < BVS ? PW : BVS) / 8;
-                        float z[PW], dd[PW];
+                        for (int i = 0; i < NV8; ++i) {
+                            uint4 w;
+                            uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
 #pragma unroll
-                        for (int c16 = 0; c16 < PW; c16 += 16) {
-                            tmem_ld16(trow + d1 + 64 * g + c0 + c16, z + c16);
-                            tmem_ld16(trow + L::COL_D2 + 64 * g + c0 + c16, dd + c16);
-                        }
-                        tmem_wait_ld();
-                        if (c0 + PW >= LW) {  // D2 and D1 of this sub-chain fully read
-                            tc_fence_before();
-                            mbar_arrive(bar(B_ODONE + g));
-                        }
-                        if (t < nvalid) {
-#pragma unroll
-                            for (int i = 0; i < NV8; ++i) {
-                                uint4 w;
-                                uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
-#pragma unroll
-                                for (int e = 0; e < 4; ++e)
-                                    wp[e] = pack_bf16(fmaf(gt, z[8 * i + 2 * e], dd[8 * i + 2 * e]),
-                                                      fmaf(gt, z[8 * i + 2 * e + 1], dd[8 * i + 2 * e + 1]));
-                                dst[c0 / 8 + i] = w;
-                            }
+                            for (int e = 0; e < 4; ++e)
+                                wp[e] = pack_bf16(fmaf(gt, z[8 * i + 2 * e], dd[8 * i + 2 * e]),
+                                                  fmaf(gt, z[8 * i + 2 * e + 1], dd[8 * i + 2 * e + 1]));
+                            dst[i] = w;
                         }
                     }
+                } else {
+                    mbar_arrive(bar(B_ODONE));
                 }
             }
         }
@@ -929,10 +919,10 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             }
             if (c + 1 < nchunks) prescale(c + 1);
         }
-    } else if (SPLIT && warp == 8 && is_chain) {
+    } else if (SPLIT && warp == 12 && is_chain) {
         // ------------------------------------------------------------------ slot releaser
         // (split chain CTA): once every chain thread and every MMA is done with chain slot
-        // c % npc, expect chunk c + npc in it and credit the prep CTA that owns that chunk.
+        // c % npc (warp 12), expect chunk c + npc in it and credit the prep CTA that owns it.
         // The slot's next phase needs this release, so the waits here never fall two phases
         // behind.
         if (lane == 0) {
@@ -1414,10 +1404,11 @@ inline int max_active_clusters(int size) {
 
 // Split mode (a cluster per head of `nprep` prep CTAs and dv/BV chain CTAs) for the
 // scalar-gate variants when the heads are too few to fill the GPU otherwise. Measured on
-// B200 (GDN, dk = dv = 128, T = 4096): two chain CTAs per head (BV = dv/2) beat four, whose
-// extra slot copies cost more than their shorter chain saves; two prep CTAs beat one and
-// match three or four. Every cluster must be resident at once (clusters of 7-8 CTAs fit 15
-// at a time on B200, which puts 16 heads into two waves) and the grid must fit 148 SMs.
+// B200 (GDN, dk = dv = 128): two chain CTAs per head (BV = dv/2) beat four, whose extra slot
+// copies cost more than their shorter chain saves; more prep CTAs help a little (16 heads,
+// T = 32768: 2 / 3 / 4 prep CTAs 0.839 / 0.824 / 0.815 ms), so the plan takes as many as fit,
+// up to four. Every cluster must be resident at once (clusters of 7-8 CTAs fit 15 at a time
+// on B200, which would put 16 heads into two waves) and the grid must fit 148 SMs.
 struct SplitPlan {
     int bv = 0, nprep = 0;  // nprep == 0: unsplit
 };
@@ -1426,7 +1417,7 @@ inline SplitPlan pick_split(int variant, long BH, int dv) {
     SplitPlan plan;
     if (variant == DR_KDA || dv < 32) return plan;
     const int bv = dv / 2, ncc = 2;
-    for (int np = 2; np >= 1; --np) {
+    for (int np = 4; np >= 1; --np) {
         if (BH * (np + ncc) <= 148 && BH <= max_active_clusters(np + ncc)) {
             plan.bv = bv;
             plan.nprep = np;

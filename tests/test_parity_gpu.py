@@ -84,12 +84,13 @@ def test_bf16_dispatch_narrow_values(oracle, mode, dv):
     check_dr(oracle, w, seed=dv)
 
 
-# Every branch of the chunked kernel's launch plan: a split cluster with two prep CTAs and a
-# three-deep chain slot ring (few heads), with one prep CTA and a two-deep ring, and one CTA
-# per (head, value slice) once the heads fill the GPU. The plan is read back so that a change
-# of the planner cannot silently drop a branch from the tests.
+# Every branch of the chunked kernel's launch plan: split clusters with four, three or two
+# prep CTAs and a three-deep chain slot ring (few heads), with one prep CTA and a two-deep
+# ring, and one CTA per (head, value slice) once the heads fill the GPU. The plan is read back
+# so that a change of the planner cannot silently drop a branch from the tests.
 @pytest.mark.parametrize("mode", [wl.DELTANET, wl.GDN])
-@pytest.mark.parametrize("BH,dv,split", [(2, 128, 2), (40, 128, 1), (40, 64, 1), (46, 128, None),
+@pytest.mark.parametrize("BH,dv,split", [(2, 128, 4), (16, 64, 4), (24, 128, 3), (32, 128, 2),
+                                         (40, 128, 1), (40, 64, 1), (46, 128, None),
                                          (64, 128, 0), (64, 32, 0)])
 def test_bf16_plan_branches(oracle, mode, BH, dv, split):
     plan = drs.chunked_plan(mode, BH, 128, dv)
