@@ -48,9 +48,12 @@ def parse_args(argv=None):
 # ---------------------------------------------------------------------------------------
 def algorithmic_bytes(w, with_state_in=None, with_state_out=True) -> int:
     """Bytes the scan must move once: q, k, v in, out out, beta and gates in, S0 in (when
-    given) and S_final out. Per head-token this is the figure the roofline uses."""
+    given) and S_final out. Per head-token this is the figure the roofline uses. VLA: q, k,
+    v, u in and out out (fp32), S_final and A_final out."""
     from delta_rule_recurrent_chunked_b200 import workloads as wl
 
+    if isinstance(w, wl.VLAWorkload):
+        return w.B * w.H * (w.T * 5 * w.d * 4 + (2 * w.d * w.d * 4 if with_state_out else 0))
     isz = 2 if w.dtype == "bf16" else 4
     BH, T = w.B * w.H, w.T
     per_head = T * (2 * w.dk + 2 * w.dv) * isz
@@ -69,7 +72,13 @@ def algorithmic_bytes(w, with_state_in=None, with_state_out=True) -> int:
 
 
 def algorithmic_flops(w) -> int:
-    """Dense-chunk FLOPs of the chunked form (C = 64), triangular halves counted once."""
+    """Dense-chunk FLOPs of the chunked form (C = 64), triangular halves counted once.
+    VLA: about 12 d^2 per head-token (A u, the rank-1 update of A, A k, the write and the
+    readout of S, each a d x d matrix-vector product or outer-product update)."""
+    from delta_rule_recurrent_chunked_b200 import workloads as wl
+
+    if isinstance(w, wl.VLAWorkload):
+        return w.B * w.H * w.T * 12 * w.d * w.d
     C = 64
     per_token = 6 * w.dk * w.dv + C * (3 * w.dk + 2 * w.dv) + C * C // 3
     return w.B * w.H * w.T * per_token
@@ -292,7 +301,7 @@ def run_ours(args, world, rank, local):
 
     w = wl.workload(args.workload)
     if isinstance(w, wl.VLAWorkload):
-        raise SystemExit("bench.py times the delta-rule workloads; VLA is a parity workload")
+        return run_ours_vla(args, world, rank, local, w, device)
     inputs = wl.generate_dr(w, seed=rank)
     mode = {wl.LINEAR: "linear", wl.DELTANET: "deltanet", wl.GDN: "gdn", wl.KDA: "kda"}[w.mode]
     nbytes = algorithmic_bytes(w)
@@ -366,6 +375,130 @@ def run_ours(args, world, rank, local):
                      "launch_ms": launch_ms,
                      "tensor_tflops": tflops,
                      "tensor_frac": tflops / peaks["bf16_tflops"]},
+        "wall_s": t_wall,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(inputs)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def fp32_alu_peak_tflops(device) -> float:
+    """FP32 FMA peak of the device from its unit counts and clock: SMs x 128 FP32 lanes x
+    2 FLOP x the maximum SM clock (148 x 128 x 2 x 1.965 GHz = 74.4 TFLOP/s on B200)."""
+    import torch
+
+    props = torch.cuda.get_device_properties(device)
+    mhz = None
+    try:
+        import pynvml
+
+        pynvml.nvmlInit()
+        h = pynvml.nvmlDeviceGetHandleByIndex(device.index or 0)
+        mhz = pynvml.nvmlDeviceGetMaxClockInfo(h, pynvml.NVML_CLOCK_SM)
+    except Exception:
+        pass
+    mhz = mhz or 1965
+    return props.multi_processor_count * 128 * 2 * mhz * 1e6 / 1e12
+
+
+def run_ours_vla(args, world, rank, local, w, device):
+    """The VLA Sherman-Morrison scan (fp32, sequential per-token kernel) through vla_scan_fwd;
+    a per-token latency-bound path, reported against the FP32 ALU peak."""
+    import torch
+    import torch.distributed as dist
+
+    import delta_rule_recurrent_chunked_b200 as drs
+    from delta_rule_recurrent_chunked_b200 import workloads as wl
+
+    inputs = wl.generate_vla(w, seed=rank)
+    nbytes = algorithmic_bytes(w)
+    nsets = max(1, min(4, -(-3 * L2_BYTES // max(nbytes, 1))))
+    sets = [{k: torch.from_numpy(np.ascontiguousarray(inputs[k])).to(device)
+             for k in ("q", "k", "v", "u")} for _ in range(nsets)]
+    outs = [torch.empty_like(st["v"]) for st in sets]
+
+    def step(i):
+        st = sets[i % nsets]
+        drs.vla_scan(st["q"], st["k"], st["v"], st["u"], lambda0=w.lambda0, out=outs[i % nsets])
+
+    stream = torch.cuda.current_stream(device)
+    for i in range(max(3, args.warmup)):
+        step(i)
+    torch.cuda.synchronize(device)
+    if drs.poll_error(device) != 0:
+        raise RuntimeError("device status set during warm-up")
+    K = args.steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    clocks = ClockSampler(local)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    clocks.start()
+    t_wall = time.perf_counter()
+    for i in range(K):
+        starts[i].record(stream)
+        step(i)
+        ends[i].record(stream)
+    torch.cuda.synchronize(device)
+    t_wall = time.perf_counter() - t_wall
+    barrier(device)
+    clk = clocks.stop()
+    total_ms = starts[0].elapsed_time(ends[-1])
+    launch_ms = statistics.mean(starts[i].elapsed_time(ends[i]) for i in range(K))
+    if drs.poll_error(device) != 0:
+        raise RuntimeError("device status set in the timed region")
+    total_ms_max = max_over_ranks(total_ms, device=device)
+
+    # end to end: pinned host q/k/v/u in, out/S_final/A_final back, every step
+    host = {k: torch.from_numpy(np.ascontiguousarray(inputs[k])).pin_memory()
+            for k in ("q", "k", "v", "u")}
+    dev = {k: torch.empty_like(t, device=device) for k, t in host.items()}
+    out_h = torch.empty_like(host["v"]).pin_memory()
+    st_h = [torch.empty((w.B, w.H, w.d, w.d), dtype=torch.float32).pin_memory() for _ in range(2)]
+
+    def e2e_step():
+        for k2, t in host.items():
+            dev[k2].copy_(t, non_blocking=True)
+        o, Sf, Af = drs.vla_scan(dev["q"], dev["k"], dev["v"], dev["u"], lambda0=w.lambda0)
+        out_h.copy_(o, non_blocking=True)
+        st_h[0].copy_(Sf, non_blocking=True)
+        st_h[1].copy_(Af, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(device)
+    n = max(1, args.e2e_steps)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(n):
+        e2e_step()
+    b.record(stream)
+    torch.cuda.synchronize(device)
+    e2e_ms = max_over_ranks(a.elapsed_time(b) / n, device=device)
+    h2d = sum(t.numel() * 4 for t in host.values())
+    d2h = out_h.numel() * 4 + 2 * st_h[0].numel() * 4
+
+    flops = algorithmic_flops(w)
+    peak = fp32_alu_peak_tflops(device)
+    achieved = flops / (launch_ms / 1e3) / 1e12
+    line = {
+        "metric": METRIC, "value": aggregate_value(world, w.head_tokens, K, total_ms_max),
+        "unit": UNIT, "n_gpus": world, "steps": K, "warmup": max(3, args.warmup),
+        "ms_per_step": total_ms_max / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": dict(workload_config(w, world, nsets, nbytes), kernel="vla_sequential"),
+        "clocks": {k: clk[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+        "e2e": {"value": world * w.head_tokens / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": K,
+        "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                     "frac": achieved / peak, "traffic": None,
+                     "peak_source": "derived: SMs x 128 FP32 lanes x 2 x max SM clock",
+                     "flops_per_launch": flops, "launch_ms": launch_ms,
+                     "hbm_gbs": nbytes / (launch_ms / 1e3) / 1e9},
         "wall_s": t_wall,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -62,3 +62,15 @@ def test_algorithmic_bytes_match_the_per_token_table():
     assert bench.algorithmic_bytes(kda) == kda.head_tokens * 1556
     long = wl.workload("gdn_long_t4096")
     assert bench.algorithmic_bytes(long) == long.head_tokens * 1064
+
+
+def test_vla_accounting_matches_the_per_token_table():
+    import bench
+    from delta_rule_recurrent_chunked_b200 import workloads as wl
+
+    for d, per_token, flops in ((32, 640, 1.23e4), (96, 1920, 1.11e5)):
+        w = wl.workload(f"vla_fp32_d{d}")
+        # per head-token: q, k, v, u in and out out (fp32); the d x d end states once per head
+        assert bench.algorithmic_bytes(w, with_state_out=False) == w.head_tokens * per_token
+        assert bench.algorithmic_bytes(w) == w.head_tokens * per_token + w.B * w.H * 2 * d * d * 4
+        assert bench.algorithmic_flops(w) / w.head_tokens == pytest.approx(flops, rel=0.01)
