@@ -110,8 +110,8 @@ def aggregate_value(world: int, head_tokens: int, steps: int, total_ms_max: floa
 # keyed by workload and the sha256 prefix of the chunked kernel's source at capture time; a
 # changed source reports null. Summaries with the commands are under profiles/.
 NCU_TRAFFIC = {
-    ("gdn_bf16", "41237345faaa4c8f"): 101818880 + 15062016,
-    ("kda_bf16", "41237345faaa4c8f"): 673439488 + 120269056,
+    ("gdn_bf16", "ccf466c9562f095c"): 101832448 + 13261312,
+    ("kda_bf16", "ccf466c9562f095c"): 673327104 + 120072704,
 }
 
 

@@ -26,15 +26,22 @@
 // substitution in fp32, then the off-diagonal blocks by two levels of block products
 // (X21 = -X22 A21 X11) on tf32 mma.sync, whose 16-row tiles are below tcgen05's minimum M.
 //
-// Warp roles (512 threads):
+// Warp roles (512 threads), one CTA per (head, value slice) doing both sides:
 //   warp 0      TMA producer of K and Q tiles; beta and GDN gate scalars
 //   warp 1      chain MMA issuer (MMA1, MMA2, MMA3)
 //   warp 2      prep MMA issuer (Gram, PT, H)
 //   warp 3      tensor-memory allocation, then the TMA producer of V tiles
 //   warps 4-7   chain warpgroup: residual Y, output rows, carried state (TMEM lane = row)
-//   warps 8-15  prep warps (two halves): gates, Gram epilogue, UT inverse, operand staging
+//   warps 8-15  prep warps: gates, Gram epilogue, UT inverse, operand staging
 // The prep side runs up to one chunk ahead of the chain; the only serial dependency
 // between chunks is the state (MMA1 -> residual -> MMA3 -> state copy -> MMA1).
+// Split clusters (few heads; SPLIT): per head, 1-4 prep CTAs and 2 chain CTAs.
+//   prep CTA:  warps 0 and 4 K/Q producers (one stage each), warp 1 distributor (bulk copies
+//              of each prepared slot into the chain CTAs), warps 2 and 3 prep MMA issuers,
+//              warps 8-11 and 12-15 two prep groups on alternate chunks;
+//   chain CTA: warp 0 K/Q producer, warp 1 MMA1 issuer, warp 2 MMA3/MMA2 issuer, warp 3 V
+//              producer, warps 4-7 and 8-11 two chain warpgroups sharing the value columns,
+//              warp 12 slot releaser.
 // Every wait is bounded: on a timeout the status word is latched, the CTA-wide abort flag
 // is raised and all roles run to the end without waiting or issuing.
 #pragma once
@@ -64,10 +71,6 @@ struct ChunkLayout {
     static constexpr int NSV = (kKda && BV == 128) ? 1 : 2;  // V stages
     static constexpr int NP = (kKda && BV >= 64) ? 1 : 2;    // prepared-operand slots
     static constexpr int NKN = kKda ? 1 : 0;
-    // Sub-chains: the value slice is cut into NSUB independent column sets, interleaved so
-    // that one's MMAs run while the other's epilogues execute (split chain CTAs only).
-    static constexpr int NSUB = 1;  // (the chain code is written for NSUB sub-chains)
-    static constexpr int BVS = BV / NSUB;  // value channels per sub-chain
 
     static constexpr int KQ_B = 32768;  // [K;Q] bf16: 2 panels x 128 rows x 128 B
     static constexpr int V_B = CK * BV * 2;
@@ -76,9 +79,9 @@ struct ChunkLayout {
     // The chain MMAs run with N = NB >= 64 so that Y and the bf16 state are stored as
     // M/N-major B operands in 64-column swizzled groups (whole-row 16-byte stores); columns
     // beyond the real ones are zero padding. Group g of S / Y sits at SS + g*16384 /
-    // SY + g*8192 (a sub-chain uses one group).
-    static constexpr int NB = SPLIT ? 64 : (BV < 64 ? 64 : BV);
-    static constexpr int NG = SPLIT ? NSUB : NB / 64;
+    // SY + g*8192.
+    static constexpr int NB = BV < 64 ? 64 : BV;
+    static constexpr int NG = NB / 64;
     static constexpr int SY_B = NG * 8192;   // Y: 64 rows (t) x 64 columns per group
     static constexpr int SS_B = NG * 16384;  // S: 128 rows (key channel) x 64 columns per group
 
@@ -163,16 +166,15 @@ enum ChunkBar {
     B_SLOT_EMPTY = 14,  // [2] slot consumed by the chain
     B_MMA1 = 16,
     B_YREADY = 17,
-    B_MMA23 = 18,
+    B_MMA23 = 18,     // MMA2 and MMA3 done (split chain CTA: MMA3 done)
     B_STATE = 19,     // bf16 state copy ready for MMA1
     B_PEER_FREE = 20,  // [2] prep CTA: every chain CTA freed its copy of the slot
     B_GRP1 = 22,       // second prep group's GO, GRAM, TREADY, HDONE (prep CTA of a split)
-    B_SUB1 = 26,       // second sub-chain's MMA1, YREADY, MMA23, STATE (chain CTA of a split)
-    B_ODONE = 30,      // [2] split chain CTA: sub-chain g's output rows are read out of TMEM
-    B_PREP2 = 32,      // split chain CTA: third slot ready
-    B_MMA2 = 33,       // split chain CTA: MMA2 done (MMA3 done is B_MMA23)
-    B_SFREE = 34,      // [3] split chain CTA: chain slot i read by every thread and every MMA
-    B_COUNT = 37
+    B_ODONE = 26,      // split chain CTA: the output rows are read out of TMEM
+    B_PREP2 = 27,      // split chain CTA: third slot ready
+    B_MMA2 = 28,       // split chain CTA: MMA2 done
+    B_SFREE = 29,      // [3] split chain CTA: chain slot i read by every thread and every MMA
+    B_COUNT = 32
 };
 
 // bf16 bits of 8 consecutive columns of a row, stored as one 16-byte swizzled chunk.
@@ -321,15 +323,11 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
         mbar_init(bar(B_GRP1 + 1), 1);
         mbar_init(bar(B_GRP1 + 2), gthreads);
         mbar_init(bar(B_GRP1 + 3), 1);
-        mbar_init(bar(B_ODONE + 0), SPLIT ? 128 : 64);
-        mbar_init(bar(B_ODONE + 1), 64);
-        for (int g = 0; g < 2; ++g) {
-            const int o = g ? B_SUB1 - B_MMA1 : 0;
-            mbar_init(bar(B_MMA1 + o), 1);
-            mbar_init(bar(B_YREADY + o), 128);
-            mbar_init(bar(B_MMA23 + o), 1);
-            mbar_init(bar(B_STATE + o), SPLIT ? 256 : 128);
-        }
+        mbar_init(bar(B_ODONE), 128);
+        mbar_init(bar(B_MMA1), 1);
+        mbar_init(bar(B_YREADY), 128);
+        mbar_init(bar(B_MMA23), 1);
+        mbar_init(bar(B_STATE), SPLIT ? 256 : 128);
         *abort_flag = 0;
         mbar_init_fence();
     }
@@ -451,10 +449,8 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
         // needs only K/Q and the state copy), warp 2 the state update MMA3 and then MMA2, so
         // neither issuer's waits delay the other's step of the chain.
         if (lane == 0) {
-            constexpr int NSUB = L::NSUB;
             constexpr uint32_t id1 = idesc_bf16(128, L::NB, 0, 1);
             const bool do_mma1 = warp == 1, do_mma23 = !SPLIT || warp == 2;
-            auto sb = [&](int base, int g) { return bar(base + (g ? B_SUB1 - B_MMA1 : 0)); };
             for (int c = 0; c < nchunks; ++c) {
                 const int s = c % NS;
                 uint8_t* kq = sm + L::KQ + s * L::KQ_B;
@@ -462,71 +458,61 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     mbar_wait(bar(B_KQ_FULL + s), (uint32_t)((c / NS) & 1), abort_flag);
                     if constexpr (!SPLIT)
                         mbar_wait(cprep(c % npc), (uint32_t)((c / npc) & 1), abort_flag);
+                    mbar_wait(bar(B_STATE), (uint32_t)(c & 1), abort_flag);
+                    tc_fence_after();
+                    if (!*abort_flag) {
+                        const uint32_t d1 = L::COL_D1 + (SPLIT ? 128 * (c & 1) : 0);
 #pragma unroll
-                    for (int g = 0; g < NSUB; ++g) {
-                        mbar_wait(sb(B_STATE, g), (uint32_t)(c & 1), abort_flag);
-                        tc_fence_after();
-                        if (!*abort_flag) {
-                            const uint8_t* ss = sm + L::SS + g * 16384;
-                            const uint32_t d1 = L::COL_D1 + 64 * g + (SPLIT ? 128 * (c & 1) : 0);
-#pragma unroll
-                            for (int kk = 0; kk < 8; ++kk) {
-                                const int pn = kk >> 2, ko = (kk & 3) * 32;
-                                tc_mma_bf16(tmem + d1,
-                                            smem_desc_sw128(smem_u32(kq + pn * 16384 + ko), 16, 1024),
-                                            smem_desc_sw128(smem_u32(ss + kk * 2048), 16384, 1024),
-                                            id1, kk > 0);
-                            }
-                            tc_commit(sb(B_MMA1, g));
+                        for (int kk = 0; kk < 8; ++kk) {
+                            const int pn = kk >> 2, ko = (kk & 3) * 32;
+                            tc_mma_bf16(tmem + d1,
+                                        smem_desc_sw128(smem_u32(kq + pn * 16384 + ko), 16, 1024),
+                                        smem_desc_sw128(smem_u32(sm + L::SS + kk * 2048), 16384, 1024),
+                                        id1, kk > 0);
                         }
+                        tc_commit(bar(B_MMA1));
+                        tc_commit(bar(B_KQ_EMPTY + s));
                     }
-                    if (!*abort_flag) tc_commit(bar(B_KQ_EMPTY + s));
                 }
                 if (!do_mma23) continue;
                 if constexpr (SPLIT) mbar_wait(cprep(c % npc), (uint32_t)((c / npc) & 1), abort_flag);
                 const uint8_t* tp = cslot(c % npc) + L::SLOT_TP;
                 const uint8_t* kh = cslot(c % npc) + L::SLOT_KH;
+                mbar_wait(bar(B_YREADY), (uint32_t)(c & 1), abort_flag);
+                tc_fence_after();
+                auto mma3 = [&]() {  // S^T += Khat^T Y
 #pragma unroll
-                for (int g = 0; g < NSUB; ++g) {
-                    mbar_wait(sb(B_YREADY, g), (uint32_t)(c & 1), abort_flag);
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc_mma_bf16(tmem + L::COL_S, smem_desc_sw128(smem_u32(kh + kk * 32), 16, 1024),
+                                    smem_desc_sw128(smem_u32(sm + L::SY + kk * 2048), 8192, 1024), id1,
+                                    1);
+                };
+                auto mma2 = [&]() {  // D2 = [T; PT] Y
+#pragma unroll
+                    for (int kk = 0; kk < 4; ++kk)
+                        tc_mma_bf16(tmem + L::COL_D2, smem_desc_sw128(smem_u32(tp + kk * 32), 16, 1024),
+                                    smem_desc_sw128(smem_u32(sm + L::SY + kk * 2048), 8192, 1024), id1,
+                                    kk > 0);
+                };
+                if constexpr (SPLIT) {
+                    // the state update first (it is on the chain's critical path), then the
+                    // output rows once the previous chunk's are out of D2
+                    if (!*abort_flag) {
+                        mma3();
+                        tc_commit(bar(B_MMA23));
+                    }
+                    if (c > 0) mbar_wait(bar(B_ODONE), (uint32_t)((c - 1) & 1), abort_flag);
                     tc_fence_after();
-                    const uint8_t* sy = sm + L::SY + g * 8192;
-                    auto mma3 = [&]() {  // S^T += Khat^T Y
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            tc_mma_bf16(tmem + L::COL_S + 64 * g,
-                                        smem_desc_sw128(smem_u32(kh + kk * 32), 16, 1024),
-                                        smem_desc_sw128(smem_u32(sy + kk * 2048), 8192, 1024), id1,
-                                        1);
-                    };
-                    auto mma2 = [&]() {  // D2 = [T; PT] Y
-#pragma unroll
-                        for (int kk = 0; kk < 4; ++kk)
-                            tc_mma_bf16(tmem + L::COL_D2 + 64 * g,
-                                        smem_desc_sw128(smem_u32(tp + kk * 32), 16, 1024),
-                                        smem_desc_sw128(smem_u32(sy + kk * 2048), 8192, 1024), id1,
-                                        kk > 0);
-                    };
-                    if constexpr (SPLIT) {
-                        // the state update first (it is on the chain's critical path), then the
-                        // output rows once the previous chunk's are out of D2
-                        if (!*abort_flag) {
-                            mma3();
-                            tc_commit(sb(B_MMA23, g));
-                        }
-                        if (c > 0) mbar_wait(bar(B_ODONE + g), (uint32_t)((c - 1) & 1), abort_flag);
-                        tc_fence_after();
-                        if (!*abort_flag) {
-                            mma2();
-                            tc_commit(bar(B_MMA2));
-                            tc_commit(bar(B_SFREE + c % npc));  // last reader of the slot
-                        }
-                    } else {
-                        if (!*abort_flag) {
-                            mma2();
-                            mma3();
-                            tc_commit(sb(B_MMA23, g));
-                        }
+                    if (!*abort_flag) {
+                        mma2();
+                        tc_commit(bar(B_MMA2));
+                        tc_commit(bar(B_SFREE + c % npc));  // last reader of the slot
+                    }
+                } else {
+                    if (!*abort_flag) {
+                        mma2();
+                        mma3();
+                        tc_commit(bar(B_MMA23));
                     }
                 }
             }
@@ -789,12 +775,6 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             fence_async_smem();
             mbar_arrive(bar(B_STATE));
             // slots start empty: expect the prep CTA's copies of the first chunks
-            if (r == 0 && split) {
-                for (int c = 0; c < NP && c < nchunks; ++c) {
-                    mbar_arrive_expect_tx(bar(B_PREP + c), L::SLOT_B);
-                    mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + c), owner_of(c)));
-                }
-            }
         }
         auto prescale = [&](int c) {  // S^T *= gamma_C of chunk c, before MMA3(c)
             if constexpr (MODE != DR_DELTANET) {
@@ -909,14 +889,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             // slot p is free once every chain thread is done with it (MMA2/3 completed before
             // the wait above); hand it to whoever fills it next
             asm volatile("bar.sync 2, 128;" ::: "memory");
-            if (r == 0 && c + NP < nchunks) {
-                if (!split) {
-                    mbar_arrive(bar(B_SLOT_EMPTY + p));
-                } else {
-                    mbar_arrive_expect_tx(bar(B_PREP + p), L::SLOT_B);
-                    mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + p), owner_of(c + NP)));
-                }
-            }
+            if (r == 0 && c + NP < nchunks) mbar_arrive(bar(B_SLOT_EMPTY + p));
             if (c + 1 < nchunks) prescale(c + 1);
         }
     } else if (SPLIT && warp == 12 && is_chain) {
