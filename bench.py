@@ -452,34 +452,23 @@ def run_ours_vla(args, world, rank, local, w, device):
         raise RuntimeError("device status set in the timed region")
     total_ms_max = max_over_ranks(total_ms, device=device)
 
-    # end to end: pinned host q/k/v/u in, out/S_final/A_final back, every step
+    # end to end: pinned host q/k/v/u in, out/S_final/A_final back, every step (pipelined)
     host = {k: torch.from_numpy(np.ascontiguousarray(inputs[k])).pin_memory()
             for k in ("q", "k", "v", "u")}
-    dev = {k: torch.empty_like(t, device=device) for k, t in host.items()}
-    out_h = torch.empty_like(host["v"]).pin_memory()
-    st_h = [torch.empty((w.B, w.H, w.d, w.d), dtype=torch.float32).pin_memory() for _ in range(2)]
 
-    def e2e_step():
-        for k2, t in host.items():
-            dev[k2].copy_(t, non_blocking=True)
-        o, Sf, Af = drs.vla_scan(dev["q"], dev["k"], dev["v"], dev["u"], lambda0=w.lambda0)
-        out_h.copy_(o, non_blocking=True)
-        st_h[0].copy_(Sf, non_blocking=True)
-        st_h[1].copy_(Af, non_blocking=True)
+    def make_outputs():
+        return [torch.empty(host["v"].shape, dtype=torch.float32, device=device),
+                torch.empty((w.B, w.H, w.d, w.d), dtype=torch.float32, device=device),
+                torch.empty((w.B, w.H, w.d, w.d), dtype=torch.float32, device=device)]
 
-    for _ in range(3):
-        e2e_step()
-    torch.cuda.synchronize(device)
-    n = max(1, args.e2e_steps)
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(n):
-        e2e_step()
-    b.record(stream)
-    torch.cuda.synchronize(device)
-    e2e_ms = max_over_ranks(a.elapsed_time(b) / n, device=device)
-    h2d = sum(t.numel() * 4 for t in host.values())
-    d2h = out_h.numel() * 4 + 2 * st_h[0].numel() * 4
+    def launch(d, o):
+        _, Sf, Af = drs.vla_scan(d["q"], d["k"], d["v"], d["u"], lambda0=w.lambda0, out=o[0])
+        o[1].copy_(Sf)
+        o[2].copy_(Af)
+
+    pipe = CopyPipeline(device, host, make_outputs, launch)
+    e2e_ms = max_over_ranks(pipe.run(max(1, args.e2e_steps)), device=device)
+    h2d, d2h = pipe.h2d, pipe.d2h
 
     flops = algorithmic_flops(w)
     peak = fp32_alu_peak_tflops(device)
@@ -509,9 +498,74 @@ def run_ours_vla(args, world, rank, local, w, device):
         print(json.dumps(line), flush=True)
 
 
+class CopyPipeline:
+    """End-to-end steps through the public API, pipelined over three streams: the host->device
+    copy of step i+1 and the device->host copy of step i-1 overlap the scan of step i (PCIe
+    carries both directions at once). Every step still copies its inputs in and its results
+    out inside the timed region; two buffer sets and events keep the steps apart."""
+
+    def __init__(self, device, host_in, make_outputs, launch):
+        import torch
+
+        self.torch = torch
+        self.host_in = host_in                                  # name -> pinned host tensor
+        self.dev_in = [{k: (None if t is None else torch.empty_like(t, device=device))
+                        for k, t in host_in.items()} for _ in range(2)]
+        self.dev_out = [make_outputs() for _ in range(2)]       # list of device tensors
+        self.host_out = [[torch.empty_like(t, device="cpu").pin_memory() for t in outs]
+                         for outs in self.dev_out]
+        self.launch = launch                                    # (dev_in, dev_out) -> None
+        self.s_in, self.s_run, self.s_out = (torch.cuda.Stream(device) for _ in range(3))
+        self.ev_in = [torch.cuda.Event() for _ in range(2)]
+        self.ev_run = [torch.cuda.Event() for _ in range(2)]
+        self.ev_out = [torch.cuda.Event() for _ in range(2)]
+        self.started = [False, False]
+        self.h2d = sum(t.numel() * t.element_size() for t in host_in.values() if t is not None)
+        self.d2h = sum(t.numel() * t.element_size() for t in self.dev_out[0])
+
+    def step(self):
+        torch = self.torch
+        j = self.i % 2
+        with torch.cuda.stream(self.s_in):
+            if self.started[j]:
+                self.s_in.wait_event(self.ev_run[j])       # the scan of step i-2 read dev_in[j]
+            for k, t in self.host_in.items():
+                if t is not None:
+                    self.dev_in[j][k].copy_(t, non_blocking=True)
+            self.ev_in[j].record(self.s_in)
+        with torch.cuda.stream(self.s_run):
+            self.s_run.wait_event(self.ev_in[j])
+            if self.started[j]:
+                self.s_run.wait_event(self.ev_out[j])      # step i-2's results are copied out
+            self.launch(self.dev_in[j], self.dev_out[j])
+            self.ev_run[j].record(self.s_run)
+        with torch.cuda.stream(self.s_out):
+            self.s_out.wait_event(self.ev_run[j])
+            for h, d in zip(self.host_out[j], self.dev_out[j]):
+                h.copy_(d, non_blocking=True)
+            self.ev_out[j].record(self.s_out)
+        self.started[j] = True
+        self.i += 1
+
+    def run(self, n, warmup=3):
+        torch = self.torch
+        self.i = 0
+        for _ in range(warmup):
+            self.step()
+        torch.cuda.synchronize()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(self.s_in)
+        for _ in range(n):
+            self.step()
+        b.record(self.s_out)  # after the last step's device->host copy, which follows all work
+        b.synchronize()
+        return a.elapsed_time(b) / n
+
+
 def run_e2e(args, w, inputs, mode, device, stream):
     """Same workload through the public API with pinned host buffers: per step copy the
-    inputs host->device, run the scan, copy out and S_final device->host."""
+    inputs host->device, run the scan, copy out and S_final device->host (pipelined)."""
     import torch
 
     import delta_rule_recurrent_chunked_b200 as drs
@@ -525,35 +579,18 @@ def run_e2e(args, w, inputs, mode, device, stream):
     for name in ("beta", "gate", "S0"):
         a = inputs.get(name)
         host[name] = None if a is None else torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
-    dev = {k: (None if t is None else torch.empty_like(t, device=device)) for k, t in host.items()}
-    out = torch.empty_like(dev["v"])
-    Sf = torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device=device)
-    out_h = torch.empty_like(out, device="cpu").pin_memory()
-    Sf_h = torch.empty_like(Sf, device="cpu").pin_memory()
-    h2d = sum(t.numel() * t.element_size() for t in host.values() if t is not None)
-    d2h = out.numel() * out.element_size() + Sf.numel() * Sf.element_size()
 
-    def step():
-        for k, t in host.items():
-            if t is not None:
-                dev[k].copy_(t, non_blocking=True)
-        drs.scan(dev["q"], dev["k"], dev["v"], dev["beta"], dev["gate"], dev["S0"], mode=mode,
-                 out=out, S_final=Sf)
-        out_h.copy_(out, non_blocking=True)
-        Sf_h.copy_(Sf, non_blocking=True)
+    def make_outputs():
+        return [torch.empty(host["v"].shape, dtype=host["v"].dtype, device=device),
+                torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device=device)]
 
-    for _ in range(3):
-        step()
-    torch.cuda.synchronize(device)
-    n = max(1, args.e2e_steps)
-    a = torch.cuda.Event(enable_timing=True)
-    b = torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(n):
-        step()
-    b.record(stream)
-    torch.cuda.synchronize(device)
-    return {"ms": a.elapsed_time(b) / n, "h2d": h2d, "d2h": d2h}
+    def launch(d, o):
+        drs.scan(d["q"], d["k"], d["v"], d["beta"], d["gate"], d["S0"], mode=mode,
+                 out=o[0], S_final=o[1])
+
+    pipe = CopyPipeline(device, host, make_outputs, launch)
+    ms = pipe.run(max(1, args.e2e_steps))
+    return {"ms": ms, "h2d": pipe.h2d, "d2h": pipe.d2h}
 
 
 # ---------------------------------------------------------------------------------------
