@@ -182,6 +182,28 @@ def test_heads_are_independent():
     assert torch.equal(out_p, out[:, p]) and torch.equal(Sf_p, Sf[:, p])
 
 
+# --- streams: the library keeps no per-call scratch, so scans on different streams, running
+# at the same time on different inputs (split and unsplit launch plans), are independent
+def test_concurrent_scans_on_two_streams(oracle):
+    cases = [(wl.DRWorkload("t", 1, 2, 700, 128, 128, wl.GDN, "bf16", s0_std=0.1), 11),
+             (wl.DRWorkload("t", 1, 64, 200, 128, 128, wl.KDA, "bf16", s0_std=0.1), 12)]
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    runs = []
+    for (w, seed), st in zip(cases, streams):
+        inputs = wl.generate_dr(w, seed)
+        dev = to_device(inputs)
+        torch.cuda.synchronize()
+        with torch.cuda.stream(st):
+            out, Sf = drs.scan(dev["q"], dev["k"], dev["v"], dev["beta"], dev["gate"], dev["S0"],
+                               mode=MODE_NAME[w.mode])
+        runs.append((w, inputs, out, Sf))
+    torch.cuda.synchronize()
+    for w, inputs, out, Sf in runs:
+        ref_out, ref_S = oracle_dr(oracle, inputs)
+        e_out, e_S = rel_err(tensor_np(out), ref_out), rel_err(tensor_np(Sf), ref_S)
+        assert e_out <= TOL["bf16"] and e_S <= TOL["bf16"], (w, e_out, e_S)
+
+
 # --- VLA
 @pytest.mark.parametrize("d", [32, 96])
 def test_vla_workload(oracle, d):
