@@ -1,0 +1,118 @@
+"""Write the worked-example fixtures in this folder (``*.json``).
+
+Each fixture is a tiny hand-chosen case whose inputs are dyadic rationals: every
+intermediate value of the recurrence is then exact in fp64, and the inputs are exact
+in bf16, so the same case checks the fp64 oracle bit for bit and the CUDA paths within
+their tolerances. The stored expected values are written here by calling the oracle
+only; ``tests/test_golden.py`` pins them against a derivation by hand (the steps are
+also stored in each fixture) and runs the CUDA paths on the same inputs.
+
+Run from the repository root:  python tests/golden/make_golden.py
+"""
+from __future__ import annotations
+
+import json
+import os
+import sys
+
+import numpy as np
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, os.path.dirname(os.path.dirname(HERE)))
+
+import oracle  # noqa: E402  (test infrastructure: the only import this script makes)
+
+DR_PAGE = ('"Mechanisms, trade-offs and cross-layer routing of linear-attention architectures" '
+           '(aitrends.kr), section "Technical details": delta-rule write with residual '
+           'r = v - W kappa, gated (scalar alpha) and per-key-channel (Kimi) decays')
+VLA_PAGE = ('"Variational Linear Attention (VLA)" (gist.science 2605.11196), sections 2.2-2.3: '
+            'Sherman-Morrison update of A = M^-1, alpha_hat = A k_hat / ||A k_hat||, '
+            'S_t = S_{t-1} + (v - S_{t-1} k_hat) alpha_hat^T')
+
+CASES = {
+    "deltanet_d2_t2": dict(
+        mode=oracle.DELTANET,
+        cite=DR_PAGE + "; DeltaNet (alpha = 1)",
+        q=[[1, 0], [1, 1]], k=[[1, 0], [1, 1]], v=[[2, 0], [0, 2]], beta=[0.5, 0.5],
+        derivation=[
+            "t=1: S0 = 0, r = v1 = (2,0), S1 = 1/2 (2,0)^T (1,0) = [[1,0],[0,0]], o1 = S1 q1 = (1,0)",
+            "t=2: S1 k2 = (1,0), r = (0,2) - (1,0) = (-1,2), "
+            "S2 = S1 + 1/2 (-1,2)^T (1,1) = [[1/2,-1/2],[1,1]], o2 = S2 (1,1) = (0,2)",
+        ]),
+    "gdn_d2_t3": dict(
+        mode=oracle.GDN,
+        cite=DR_PAGE + "; Gated DeltaNet, residual against the decayed state",
+        q=[[1, 0], [1, 1], [1, -1]], k=[[1, 0], [0, 1], [1, 0]], v=[[2, 4], [4, 0], [1, 1]],
+        beta=[0.5, 0.5, 0.5], gate=[0.5, 0.5, 0.25],
+        derivation=[
+            "t=1: S1 = 1/2 (2,4)^T (1,0) = [[1,0],[2,0]], o1 = (1,2)",
+            "t=2: alpha S1 = [[1/2,0],[1,0]], (alpha S1) k2 = (0,0), r = (4,0), "
+            "S2 = [[1/2,2],[1,0]], o2 = S2 (1,1) = (5/2,1)",
+            "t=3: alpha S2 = [[1/8,1/2],[1/4,0]], (alpha S2) k3 = (1/8,1/4), r = (7/8,3/4), "
+            "S3 = [[9/16,1/2],[5/8,0]], o3 = S3 (1,-1) = (1/16,5/8)",
+            "(residual against the undecayed state instead: r3 = (1,1) - S2 k3 = (1/2,0), "
+            "S3 = [[3/8,1/2],[1/4,0]], o3 = (-1/8,1/4))",
+        ]),
+    "kda_d2_t2": dict(
+        mode=oracle.KDA,
+        cite=DR_PAGE + "; Kimi Delta Attention, alpha scales the key-channel columns of S",
+        q=[[1, 1], [0, 1]], k=[[1, 0], [0, 1]], v=[[1, 1], [0, 2]], beta=[0.5, 0.5],
+        gate=[[0.5, 0.25], [1.0, 0.5]], S0=[[1, 2], [3, 4]],
+        derivation=[
+            "t=1: S0 diag(1/2,1/4) = [[1/2,1/2],[3/2,1]], its k1 column (1/2,3/2), r = (1/2,-1/2), "
+            "S1 = [[3/4,1/2],[5/4,1]], o1 = S1 (1,1) = (5/4,9/4)",
+            "t=2: S1 diag(1,1/2) = [[3/4,1/4],[5/4,1/2]], its k2 column (1/4,1/2), r = (-1/4,3/2), "
+            "S2 = [[3/4,1/8],[5/4,5/4]], o2 = S2 (0,1) = (1/8,5/4)",
+        ]),
+    "vla_d3_t2": dict(
+        mode="vla",
+        cite=VLA_PAGE,
+        q=[[1, 1, 1], [0, 1, 1]], k=[[2, 1, 1], [1, 2, 1]], v=[[1, 2, 3], [0, 1, 0]],
+        u=[[1, 1, 1], [0, 0, 0]], lambda0=1.0,
+        derivation=[
+            "t=1: A0 = I, z = A0 u1 = (1,1,1), 1 + u1.z = 4, A1 = I - J/4 (J all ones); "
+            "A1 k1 = (1,0,0), alpha_hat = e1, S1 = (1,2,3)^T e1^T, o1 = S1 q1 = (1,2,3)",
+            "t=2: u2 = 0 leaves A2 = A1; A2 k2 = (0,1,0), alpha_hat = e2, S1 k2 = (1,2,3), "
+            "r = (0,1,0) - (1,2,3) = (-1,-1,-3), S2 = S1 + r e2^T = [[1,-1,0],[2,-1,0],[3,-3,0]], "
+            "o2 = S2 (0,1,1) = (-1,-1,-3)",
+        ]),
+}
+
+
+def _bh(x):
+    """A [T, ...] list as a [1, 1, T, ...] float64 array."""
+    return np.asarray(x, np.float64)[None, None]
+
+
+def build_case(name: str, spec: dict) -> dict:
+    fx = {"case": name, "cite": spec["cite"], "derivation": spec["derivation"],
+          "mode": spec["mode"] if spec["mode"] == "vla" else
+          {oracle.DELTANET: "deltanet", oracle.GDN: "gdn", oracle.KDA: "kda"}[spec["mode"]]}
+    inputs = {key: spec[key] for key in ("q", "k", "v", "beta", "gate", "S0", "u", "lambda0")
+              if key in spec}
+    fx["inputs"] = inputs
+    if spec["mode"] == "vla":
+        out, Sf, Af = oracle.vla_scan(_bh(spec["q"]), _bh(spec["k"]), _bh(spec["v"]),
+                                      _bh(spec["u"]), lambda0=spec["lambda0"])
+        fx["expected"] = {"out": out[0, 0].tolist(), "S_final": Sf[0, 0].tolist(),
+                          "A_final": Af[0, 0].tolist()}
+    else:
+        beta = np.asarray(spec["beta"], np.float64)[None, None]
+        gate = None if "gate" not in spec else _bh(spec["gate"])
+        S0 = None if "S0" not in spec else np.asarray(spec["S0"], np.float64)[None, None]
+        out, Sf = oracle.dr_scan(_bh(spec["q"]), _bh(spec["k"]), _bh(spec["v"]), beta, gate, S0,
+                                 spec["mode"])
+        fx["expected"] = {"out": out[0, 0].tolist(), "S_final": Sf[0, 0].tolist()}
+    return fx
+
+
+def main() -> None:
+    for name, spec in CASES.items():
+        with open(os.path.join(HERE, name + ".json"), "w") as f:
+            json.dump(build_case(name, spec), f, indent=1)
+            f.write("\n")
+        print("wrote", name + ".json")
+
+
+if __name__ == "__main__":
+    main()
