@@ -4,7 +4,7 @@ None of these re-type the oracle's recurrence: each compares it with a closed fo
 a brute-force definition of a different shape (causal attention, an explicit matrix
 inverse, an SVD), an invariant, or a special case that reduces to another routine.
 Each names the passage it follows ("Mechanisms, trade-offs and cross-layer routing of
-linear-attention architectures" = the linear-attention survey page; "Variational
+linear-attention architectures" = the linear-attention overview page; "Variational
 Linear Attention (VLA)" = the VLA page).
 """
 import numpy as np
@@ -38,7 +38,7 @@ def _rel(x, y):
 
 
 # --- plain linear attention: readout after the write, against brute-force causal attention
-# VLA page section 2.1 (S_t = S_{t-1} + v_t k_t^T); survey page "Technical details"
+# VLA page section 2.1 (S_t = S_{t-1} + v_t k_t^T); overview page "Technical details"
 # (y = W phi(q)). o_t = S_t q_t = S0 q_t + sum_{i<=t} (q_t.k_i) v_i  => tril_incl(Q K^T) V.
 def test_linear_matches_causal_attention(oracle):
     rng = np.random.default_rng(1)
@@ -73,7 +73,7 @@ def test_identity_when_alpha_one_beta_zero(oracle, mode):
 
 
 # --- unit k, beta = 1 => S_t k_t = v_t exactly after the write (read with q = k).
-# Survey page "Understanding the key idea": the delta rule writes only the residual of
+# Overview page "Understanding the key idea": the delta rule writes only the residual of
 # the memory's prediction. Holds for alpha != 1 only when the residual is taken against
 # the decayed state, which is the reading the oracle implements.
 @pytest.mark.parametrize("mode", [DELTANET, GDN, KDA])
@@ -108,7 +108,7 @@ def test_kda_uniform_channels_equals_gdn(oracle):
 
 
 # --- decay only (beta = 0): S_T = S0 * prod(alpha) -- scalar (GDN) or per key column (KDA)
-# Survey page "Technical details": KDA forgets partially along the key-feature dimension.
+# Overview page "Technical details": KDA forgets partially along the key-feature dimension.
 @pytest.mark.parametrize("mode", [GDN, KDA])
 def test_decay_only_closed_form(oracle, mode):
     rng = np.random.default_rng(6)
