@@ -90,7 +90,9 @@ def workload_config(w, world: int, nsets: int = 0, nbytes: int = 0) -> dict:
 
     cfg = {"workload": w.name, "B": w.B, "H": w.H, "T": w.T}
     if isinstance(w, wl.DRWorkload):
-        cfg.update({"dk": w.dk, "dv": w.dv, "mode": wl.MODE_NAMES[w.mode], "chunk": 64})
+        cfg.update({"dk": w.dk, "dv": w.dv, "mode": wl.MODE_NAMES[w.mode]})
+        if not w.decode:
+            cfg["chunk"] = 64
     else:
         cfg.update({"d": w.d, "mode": "vla"})
     cfg["parallelism"] = f"replicas{world}" if world > 1 else "1gpu"
@@ -107,18 +109,20 @@ def aggregate_value(world: int, head_tokens: int, steps: int, total_ms_max: floa
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch from one ncu capture,
-# keyed by workload and the sha256 prefix of the chunked kernel's source at capture time; a
-# changed source reports null. Summaries with the commands are under profiles/.
+# keyed by workload and the sha256 prefix of the timed kernel's source (dr_chunked.cuh, or
+# dr_decode.cuh for the decode workload) at capture time; a changed source reports null.
+# Summaries with the commands are under profiles/.
 NCU_TRAFFIC = {
     ("gdn_bf16", "ccf466c9562f095c"): 101832448 + 13261312,
     ("kda_bf16", "ccf466c9562f095c"): 673327104 + 120072704,
+    ("gdn_decode_bf16", "350334b801e0108e"): 271628544 + 210415360,
 }
 
 
-def kernel_source_sha() -> str:
+def kernel_source_sha(name: str = "dr_chunked.cuh") -> str:
     import hashlib
 
-    path = os.path.join(ROOT, "delta_rule_recurrent_chunked_b200", "csrc", "dr_chunked.cuh")
+    path = os.path.join(ROOT, "delta_rule_recurrent_chunked_b200", "csrc", name)
     with open(path, "rb") as f:
         return hashlib.sha256(f.read()).hexdigest()[:16]
 
@@ -307,6 +311,8 @@ def run_ours(args, world, rank, local):
     w = wl.workload(args.workload)
     if isinstance(w, wl.VLAWorkload):
         return run_ours_vla(args, world, rank, local, w, device)
+    if w.decode:
+        return run_ours_decode(args, world, rank, local, w, device)
     inputs = wl.generate_dr(w, seed=rank)
     mode = {wl.LINEAR: "linear", wl.DELTANET: "deltanet", wl.GDN: "gdn", wl.KDA: "kda"}[w.mode]
     nbytes = algorithmic_bytes(w)
@@ -493,6 +499,100 @@ def run_ours_vla(args, world, rank, local, w, device):
                      "peak_source": "derived: SMs x 128 FP32 lanes x 2 x max SM clock",
                      "flops_per_launch": flops, "launch_ms": launch_ms,
                      "hbm_gbs": nbytes / (launch_ms / 1e3) / 1e9},
+        "wall_s": t_wall,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(inputs)
+    if world > 1:
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_ours_decode(args, world, rank, local, w, device):
+    """Streaming decode through dr_decode_step: one token per head per step on an fp32 state
+    that stays resident in HBM and is updated in place (HBM-bound: the state is read and
+    written once per step)."""
+    import torch
+    import torch.distributed as dist
+
+    import delta_rule_recurrent_chunked_b200 as drs
+    from delta_rule_recurrent_chunked_b200 import workloads as wl
+
+    inputs = wl.generate_dr(w, seed=rank)
+    mode = wl.MODE_NAMES[w.mode]
+    nbytes = algorithmic_bytes(w)  # per step: the state in and out plus one token's tensors
+    dev = make_device_inputs(inputs, device)  # [B, H, T=1, ...]: drop the token axis
+    tok = {"q": dev["q"].reshape(w.B, w.H, w.dk), "k": dev["k"].reshape(w.B, w.H, w.dk),
+           "v": dev["v"].reshape(w.B, w.H, w.dv), "beta": dev["beta"].reshape(w.B, w.H),
+           "gate": None if dev["gate"] is None else
+           dev["gate"].reshape((w.B, w.H) + ((w.dk,) if w.mode == wl.KDA else ()))}
+    S = dev["S0"].clone()
+    out = torch.empty_like(tok["v"])
+
+    def step(i):
+        drs.decode_step(tok["q"], tok["k"], tok["v"], tok["beta"], tok["gate"], S, mode=mode,
+                        out=out)
+
+    stream = torch.cuda.current_stream(device)
+    for i in range(max(3, args.warmup)):
+        step(i)
+    torch.cuda.synchronize(device)
+    if drs.poll_error(device) != 0:
+        raise RuntimeError("device status set during warm-up")
+    K = args.steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
+    clocks = ClockSampler(local)
+    barrier(device)
+    torch.cuda.synchronize(device)
+    clocks.start()
+    t_wall = time.perf_counter()
+    for i in range(K):
+        starts[i].record(stream)
+        step(i)
+        ends[i].record(stream)
+    torch.cuda.synchronize(device)
+    t_wall = time.perf_counter() - t_wall
+    barrier(device)
+    clk = clocks.stop()
+    total_ms = starts[0].elapsed_time(ends[-1])
+    launch_ms = statistics.mean(starts[i].elapsed_time(ends[i]) for i in range(K))
+    if drs.poll_error(device) != 0:
+        raise RuntimeError("device status set in the timed region")
+    total_ms_max = max_over_ranks(total_ms, device=device)
+
+    # end to end: each step's token (q, k, v, beta, gate) from pinned host memory and its
+    # output back; the state is the model's and stays resident on the device
+    host = {k: t.cpu().pin_memory() for k, t in tok.items() if t is not None}
+
+    def make_outputs():
+        return [torch.empty_like(out)]
+
+    def launch(d, o):
+        drs.decode_step(d["q"], d["k"], d["v"], d["beta"], d.get("gate"), S, mode=mode, out=o[0])
+
+    pipe = CopyPipeline(device, host, make_outputs, launch)
+    e2e_ms = max_over_ranks(pipe.run(max(1, args.e2e_steps)), device=device)
+
+    peaks, peak_src = load_peaks()
+    achieved = nbytes / (launch_ms / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": aggregate_value(world, w.head_tokens, K, total_ms_max),
+        "unit": UNIT, "n_gpus": world, "steps": K, "warmup": max(3, args.warmup),
+        "ms_per_step": total_ms_max / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
+        "config": dict(workload_config(w, world), kernel="decode",
+                       l2=f"resident state {w.B * w.H * w.dv * w.dk * 4 / 2**20:.0f} MiB > 126 MiB L2"),
+        "clocks": {k: clk[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+        "e2e": {"value": world * w.head_tokens / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": pipe.h2d, "d2h_bytes_per_step": pipe.d2h},
+        "gpu_launches": K,
+        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                     "frac": achieved / peaks["hbm_gbs"],
+                     "traffic": NCU_TRAFFIC.get((w.name, kernel_source_sha("dr_decode.cuh"))),
+                     "peak_source": f"{peak_src} hbm_gbs", "bytes_per_launch": nbytes,
+                     "launch_ms": launch_ms},
         "wall_s": t_wall,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -8,6 +8,7 @@ is no CPU fallback, and a missing library is an error.
 
     out, S_final = scan(q, k, v, beta, gate, S0=None, mode="gdn")
     out, S_final, A_final = vla_scan(q, k, v, u, S0=None, A0=None, lambda0=1.0)
+    out = decode_step(q, k, v, beta, gate, S, mode="gdn")     # S updated in place
 """
 from __future__ import annotations
 
@@ -28,6 +29,7 @@ MODES = {"linear": DR_LINEAR, "deltanet": DR_DELTANET, "gdn": DR_GDN, "kda": DR_
 _VP, _I, _F = ctypes.c_void_p, ctypes.c_int, ctypes.c_float
 SIGNATURES = {
     "dr_scan_fwd": ([_VP] * 8 + [_I] * 6 + [_VP], _I),
+    "dr_decode_step": ([_VP] * 7 + [_I] * 5 + [_VP], _I),
     "vla_scan_fwd": ([_VP] * 6 + [_F] + [_VP] * 3 + [_I] * 4 + [_VP], _I),
     "dr_status_string": ([_I], ctypes.c_char_p),
     "dr_poll_error": ([_VP], _I),
@@ -130,6 +132,46 @@ def scan(q, k, v, beta=None, gate=None, S0=None, mode="gdn", want_state=True,
     if rc != DR_OK:
         raise DrScanError(rc, "dr_scan_fwd")
     return out, S_final
+
+
+def decode_step(q, k, v, beta=None, gate=None, S=None, mode="gdn", out=None):
+    """One token of the delta-rule recurrence on a resident state, on the GPU.
+    q, k: [B,H,dk]; v: [B,H,dv] (bf16 or fp32, same dtype); beta: [B,H] fp32; gate:
+    alpha values, [B,H] (gdn) or [B,H,dk] (kda) fp32; S: [B,H,dv,dk] fp32, updated in
+    place. Returns out [B,H,dv] like v."""
+    import torch
+
+    variant = MODES[mode] if isinstance(mode, str) else int(mode)
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    dev = q.device
+    if q.dtype not in (torch.bfloat16, torch.float32):
+        raise ValueError("q/k/v must be bf16 or fp32")
+    _check(q, "q", (B, H, dk), q.dtype, dev)
+    _check(k, "k", (B, H, dk), q.dtype, dev)
+    _check(v, "v", (B, H, dv), q.dtype, dev)
+    if variant != DR_LINEAR:
+        _check(beta, "beta", (B, H), torch.float32, dev)
+    else:
+        beta = None
+    if variant == DR_GDN:
+        _check(gate, "gate", (B, H), torch.float32, dev)
+    elif variant == DR_KDA:
+        _check(gate, "gate", (B, H, dk), torch.float32, dev)
+    else:
+        gate = None
+    if S is None:
+        raise ValueError("decode_step needs the state S (updated in place)")
+    _check(S, "S", (B, H, dv, dk), torch.float32, dev)
+    if out is None:
+        out = torch.empty((B, H, dv), dtype=q.dtype, device=dev)
+    _check(out, "out", (B, H, dv), q.dtype, dev)
+    flags = variant | (DR_IN_BF16 if q.dtype == torch.bfloat16 else 0)
+    rc = lib().dr_decode_step(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(gate), _ptr(S),
+                              _ptr(out), B, H, dk, dv, flags, _stream_handle(dev))
+    if rc != DR_OK:
+        raise DrScanError(rc, "dr_decode_step")
+    return out
 
 
 def vla_scan(q, k, v, u, S0=None, A0=None, lambda0=1.0, want_state=True, out=None):

@@ -8,6 +8,7 @@
 
 #include "common.cuh"
 #include "dr_chunked.cuh"
+#include "dr_decode.cuh"
 #include "dr_sequential.cuh"
 #include "vla_sequential.cuh"
 
@@ -25,6 +26,51 @@ bool dim_supported(int d) { return d == 32 || d == 64 || d == 128; }
 int launch_status() {
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? DR_OK : DR_ERR_CUDA;
+}
+
+template <typename TIn, int MODE, int DK>
+int launch_decode(const void* q, const void* k, const void* v, const float* beta, const float* gate,
+                  float* S, void* out, long rows, int dv, cudaStream_t stream) {
+    constexpr long per_cta = (long)DEC_ROWS * DEC_WARPS;
+    dr_decode_kernel<TIn, MODE, DK><<<(unsigned)((rows + per_cta - 1) / per_cta), DEC_THREADS, 0,
+                                       stream>>>(
+        static_cast<const TIn*>(q), static_cast<const TIn*>(k), static_cast<const TIn*>(v), beta,
+        gate, S, S, static_cast<TIn*>(out), rows, dv);
+    return launch_status();
+}
+
+template <typename TIn, int MODE>
+int dispatch_decode_dk(const void* q, const void* k, const void* v, const float* beta,
+                       const float* gate, float* S, void* out, long rows, int dk, int dv,
+                       cudaStream_t stream) {
+    switch (dk) {
+        case 32:
+            return launch_decode<TIn, MODE, 32>(q, k, v, beta, gate, S, out, rows, dv, stream);
+        case 64:
+            return launch_decode<TIn, MODE, 64>(q, k, v, beta, gate, S, out, rows, dv, stream);
+        case 128:
+            return launch_decode<TIn, MODE, 128>(q, k, v, beta, gate, S, out, rows, dv, stream);
+    }
+    return DR_ERR_UNSUPPORTED;
+}
+
+template <typename TIn>
+int dispatch_decode(const void* q, const void* k, const void* v, const float* beta,
+                    const float* gate, float* S, void* out, long rows, int dk, int dv, int variant,
+                    cudaStream_t stream) {
+    switch (variant) {
+        case DR_LINEAR:
+            return dispatch_decode_dk<TIn, DR_LINEAR>(q, k, v, beta, gate, S, out, rows, dk, dv,
+                                                      stream);
+        case DR_DELTANET:
+            return dispatch_decode_dk<TIn, DR_DELTANET>(q, k, v, beta, gate, S, out, rows, dk, dv,
+                                                        stream);
+        case DR_GDN:
+            return dispatch_decode_dk<TIn, DR_GDN>(q, k, v, beta, gate, S, out, rows, dk, dv, stream);
+        case DR_KDA:
+            return dispatch_decode_dk<TIn, DR_KDA>(q, k, v, beta, gate, S, out, rows, dk, dv, stream);
+    }
+    return DR_ERR_INVALID_ARG;
 }
 
 template <typename TIn, int MODE, int DK>
@@ -180,6 +226,36 @@ int dr_scan_fwd(const void* q, const void* k, const void* v, const float* beta, 
                                                   dv, variant, stream);
     return dispatch_sequential<float>(q, k, v, beta, gate, S0, out, S_final, BH, T, dk, dv,
                                       variant, stream);
+}
+
+int dr_decode_step(const void* q, const void* k, const void* v, const float* beta,
+                   const float* gate, float* S, void* out, int B, int H, int dk, int dv, int mode,
+                   cudaStream_t stream) {
+    const int variant = mode & DR_MODE_MASK;
+    if (mode & ~(DR_MODE_MASK | DR_IN_BF16)) return DR_ERR_INVALID_ARG;
+    if (variant > DR_KDA) return DR_ERR_INVALID_ARG;
+    if (B < 0 || H < 0 || dk <= 0 || dv <= 0) return DR_ERR_INVALID_ARG;
+    const long BH = (long)B * (long)H;
+    if (BH > INT_MAX) return DR_ERR_INVALID_ARG;
+    if (!ok_opt(q) || !ok_opt(k) || !ok_opt(v) || !ok_opt(out) || !ok_opt(beta) ||
+        !ok_opt(gate) || !ok_opt(S))
+        return DR_ERR_INVALID_ARG;
+    if (BH > 0) {
+        if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(out) || !ok_ptr(S))
+            return DR_ERR_INVALID_ARG;
+        if (variant != DR_LINEAR && !ok_ptr(beta)) return DR_ERR_INVALID_ARG;
+        if ((variant == DR_GDN || variant == DR_KDA) && !ok_ptr(gate)) return DR_ERR_INVALID_ARG;
+    }
+    if (!dim_supported(dk) || !dim_supported(dv)) return DR_ERR_UNSUPPORTED;
+    if (BH == 0) return DR_OK;
+    const long rows = BH * dv;
+    if (rows / ((long)DEC_ROWS * DEC_WARPS) >= INT_MAX) return DR_ERR_UNSUPPORTED;
+    if (variant == DR_LINEAR) beta = nullptr;
+    if (variant == DR_LINEAR || variant == DR_DELTANET) gate = nullptr;
+    if (mode & DR_IN_BF16)
+        return dispatch_decode<__nv_bfloat16>(q, k, v, beta, gate, S, out, rows, dk, dv, variant,
+                                              stream);
+    return dispatch_decode<float>(q, k, v, beta, gate, S, out, rows, dk, dv, variant, stream);
 }
 
 int vla_scan_fwd(const float* q, const float* k, const float* v, const float* u, const float* S0,

@@ -42,6 +42,7 @@ class DRWorkload:
     s0_std: float = 0.0
     gate_mu: float = -4.0
     gate_sigma: float = 1.0
+    decode: bool = False  # T = 1 steps on a state resident in HBM (dr_decode_step)
 
     @property
     def head_tokens(self) -> int:
@@ -70,6 +71,9 @@ WORKLOADS = {
 for _T in (4096, 8192, 16384, 32768):
     WORKLOADS[f"gdn_long_t{_T}"] = DRWorkload(f"gdn_long_t{_T}", 1, 16, _T, 128, 128, GDN, "bf16",
                                               s0_std=0.1)
+# streaming decode: one token per step for 4096 heads whose 256 MiB fp32 state stays in HBM
+WORKLOADS["gdn_decode_bf16"] = DRWorkload("gdn_decode_bf16", 128, 32, 1, 128, 128, GDN, "bf16",
+                                          s0_std=0.1, decode=True)
 for _d in (32, 96):
     WORKLOADS[f"vla_fp32_d{_d}"] = VLAWorkload(f"vla_fp32_d{_d}", 4, 8, 4096, _d)
 

@@ -87,6 +87,30 @@ int dr_scan_fwd(const void* q, const void* k, const void* v, const float* beta,
                 int B, int H, int T, int dk, int dv, int mode, cudaStream_t stream);
 
 /*
+ * dr_decode_step -- one token of the same recurrence for B*H heads whose state S stays
+ * resident (streaming inference): on entry S holds S_{t-1}, on return S_t, and out
+ * receives o_t. Same definitions and readings as dr_scan_fwd with T = 1.
+ *
+ *   q, k     [B,H,dk]    bf16 if (mode & DR_IN_BF16) else fp32
+ *   v        [B,H,dv]    same type as q
+ *   beta     [B,H] fp32; NULL allowed only for DR_LINEAR
+ *   gate     alpha values, fp32: NULL for DR_LINEAR / DR_DELTANET, [B,H] for DR_GDN,
+ *            [B,H,dk] for DR_KDA
+ *   S        [B,H,dv,dk] fp32, read and updated in place
+ *   out      [B,H,dv] same type as v (written); may not alias any other argument
+ *   mode     variant | DR_IN_BF16?
+ *
+ * Supported: dk, dv in {32, 64, 128}; B, H >= 0 (B*H = 0 launches nothing). Every pointer
+ * must be 16-byte aligned and, when B*H > 0, non-NULL except as allowed above. The kernel
+ * streams each head's state from HBM and back once (one warp per four rows of S, fp32
+ * arithmetic on CUDA cores). Returns DR_OK or a negative status; on error nothing is
+ * launched.
+ */
+int dr_decode_step(const void* q, const void* k, const void* v, const float* beta,
+                   const float* gate, float* S, void* out, int B, int H, int dk, int dv, int mode,
+                   cudaStream_t stream);
+
+/*
  * vla_scan_fwd -- Variational Linear Attention scan ("Variational Linear Attention
  * (VLA)", sections 2.2-2.3): per head and token, with A the inverse penalty matrix,
  *

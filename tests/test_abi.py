@@ -90,6 +90,37 @@ def test_linear_and_deltanet_need_no_gate(lib):
     assert call_dr(lib, gate=None, mode=drs.DR_DELTANET, B=0) == drs.DR_OK
 
 
+def call_decode(lib, q=A, k=A, v=A, beta=A, gate=A, S=A, out=A, B=1, H=1, dk=32, dv=32,
+                mode=drs.DR_GDN):
+    P = ctypes.c_void_p
+    return lib.dr_decode_step(P(q), P(k), P(v), P(beta), P(gate), P(S), P(out), B, H, dk, dv, mode,
+                              None)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(S=None), drs.DR_ERR_INVALID_ARG),
+    (dict(q=None), drs.DR_ERR_INVALID_ARG),
+    (dict(out=None), drs.DR_ERR_INVALID_ARG),
+    (dict(beta=None), drs.DR_ERR_INVALID_ARG),
+    (dict(gate=None), drs.DR_ERR_INVALID_ARG),
+    (dict(gate=None, mode=drs.DR_KDA), drs.DR_ERR_INVALID_ARG),
+    (dict(S=A + 8), drs.DR_ERR_INVALID_ARG),
+    (dict(v=A + 2), drs.DR_ERR_INVALID_ARG),
+    (dict(B=-1), drs.DR_ERR_INVALID_ARG),
+    (dict(dv=0), drs.DR_ERR_INVALID_ARG),
+    (dict(mode=7), drs.DR_ERR_INVALID_ARG),
+    (dict(mode=drs.DR_GDN | drs.DR_FORCE_SEQUENTIAL), drs.DR_ERR_INVALID_ARG),  # scan-only flag
+    (dict(dk=48), drs.DR_ERR_UNSUPPORTED),
+    (dict(dv=256), drs.DR_ERR_UNSUPPORTED),
+    (dict(B=0), drs.DR_OK),
+    (dict(q=None, k=None, v=None, beta=None, gate=None, S=None, out=None, H=0), drs.DR_OK),
+    (dict(beta=None, gate=None, mode=drs.DR_LINEAR, B=0), drs.DR_OK),
+    (dict(S=A + 4, B=0), drs.DR_ERR_INVALID_ARG),  # misaligned is an error even when unused
+])
+def test_decode_step_argument_validation(lib, kw, code):
+    assert call_decode(lib, **kw) == code
+
+
 def call_vla(lib, q=A, k=A, v=A, u=A, S0=None, A0=None, lam=1.0, out=A, B=1, H=1, T=8, d=32):
     P = ctypes.c_void_p
     return lib.vla_scan_fwd(P(q), P(k), P(v), P(u), P(S0), P(A0), lam, P(out), None, None, B, H,

@@ -74,3 +74,16 @@ def test_vla_accounting_matches_the_per_token_table():
         assert bench.algorithmic_bytes(w, with_state_out=False) == w.head_tokens * per_token
         assert bench.algorithmic_bytes(w) == w.head_tokens * per_token + w.B * w.H * 2 * d * d * 4
         assert bench.algorithmic_flops(w) / w.head_tokens == pytest.approx(flops, rel=0.01)
+
+
+def test_decode_accounting_is_the_state_round_trip_plus_one_token():
+    import bench
+    from delta_rule_recurrent_chunked_b200 import workloads as wl
+
+    w = wl.workload("gdn_decode_bf16")
+    assert w.decode and w.T == 1
+    # per head and step: the fp32 state read and written (2 * 128 * 128 * 4), q, k, v in and
+    # out out (bf16, 4 * 128 * 2), beta and the scalar gate (fp32)
+    assert bench.algorithmic_bytes(w) == w.B * w.H * (2 * 128 * 128 * 4 + 4 * 128 * 2 + 4 + 4)
+    # the resident state alone is larger than the 126 MiB L2
+    assert w.B * w.H * w.dv * w.dk * 4 > 126 * 2**20

@@ -204,6 +204,75 @@ def test_concurrent_scans_on_two_streams(oracle):
         assert e_out <= TOL["bf16"] and e_S <= TOL["bf16"], (w, e_out, e_S)
 
 
+# --- single-token decode on a resident state
+def decode_inputs(dev, w):
+    """Drop the token axis (T = 1) of an uploaded workload: the decode step's shapes."""
+    B, H = w.B, w.H
+    gate = dev["gate"]
+    if gate is not None:
+        gate = gate.reshape((B, H) + ((w.dk,) if w.mode == wl.KDA else ()))
+    return (dev["q"].reshape(B, H, w.dk), dev["k"].reshape(B, H, w.dk),
+            dev["v"].reshape(B, H, w.dv), dev["beta"].reshape(B, H), gate)
+
+
+@pytest.mark.parametrize("mode", [wl.LINEAR, wl.DELTANET, wl.GDN, wl.KDA])
+@pytest.mark.parametrize("dtype", ["fp32", "bf16"])
+@pytest.mark.parametrize("dk,dv", [(32, 32), (64, 128), (128, 64), (128, 128)])
+def test_decode_step_matches_one_token_of_the_oracle(oracle, mode, dtype, dk, dv):
+    w = wl.DRWorkload("decode", 3, 5, 1, dk, dv, mode, dtype, s0_std=0.1)
+    inputs = wl.generate_dr(w, seed=dk + dv + mode)
+    dev = to_device(inputs)
+    q, k, v, beta, gate = decode_inputs(dev, w)
+    S = dev["S0"].clone()
+    out = drs.decode_step(q, k, v, beta, gate, S, mode=MODE_NAME[mode])
+    torch.cuda.synchronize()
+    ref_out, ref_S = oracle_dr(oracle, inputs)
+    assert rel_err(tensor_np(out), ref_out[:, :, 0]) <= TOL[dtype]
+    assert rel_err(tensor_np(S), ref_S) <= TOL[dtype]
+
+
+@pytest.mark.parametrize("mode", [wl.DELTANET, wl.GDN, wl.KDA])
+def test_decode_steps_replay_the_scan(oracle, mode):
+    T = 9
+    w = wl.DRWorkload("replay", 2, 3, T, 64, 64, mode, "fp32", s0_std=0.1)
+    inputs = wl.generate_dr(w, seed=11 + mode)
+    dev = to_device(inputs)
+    S = dev["S0"].clone()
+    outs = []
+    for t in range(T):
+        gate = None if dev["gate"] is None else dev["gate"][:, :, t].contiguous()
+        outs.append(drs.decode_step(dev["q"][:, :, t].contiguous(), dev["k"][:, :, t].contiguous(),
+                                    dev["v"][:, :, t].contiguous(),
+                                    dev["beta"][:, :, t].contiguous(), gate, S,
+                                    mode=MODE_NAME[mode]))
+    torch.cuda.synchronize()
+    ref_out, ref_S = oracle_dr(oracle, inputs)
+    assert rel_err(tensor_np(torch.stack(outs, dim=2)), ref_out) <= 1e-4
+    assert rel_err(tensor_np(S), ref_S) <= 1e-4
+
+
+def test_gdn_decode_workload_every_head(oracle):
+    # the benchmark's decode workload (4096 heads, 256 MiB state), every head checked
+    w = wl.workload("gdn_decode_bf16")
+    inputs = wl.generate_dr(w, 0)
+    dev = to_device(inputs)
+    q, k, v, beta, gate = decode_inputs(dev, w)
+    S = dev["S0"].clone()
+    out = drs.decode_step(q, k, v, beta, gate, S, mode="gdn")
+    torch.cuda.synchronize()
+    ref_out, ref_S = oracle_dr(oracle, inputs)
+    assert rel_err(tensor_np(out), ref_out[:, :, 0]) <= TOL["bf16"]
+    assert rel_err(tensor_np(S), ref_S) <= TOL["bf16"]
+
+
+def test_decode_step_empty_batch_launches_nothing():
+    z = torch.empty(0, 4, 128, device="cuda")
+    S = torch.empty(0, 4, 128, 128, device="cuda")
+    out = drs.decode_step(z, z, z, torch.empty(0, 4, device="cuda"), None, S, mode="deltanet")
+    torch.cuda.synchronize()
+    assert out.shape == (0, 4, 128)
+
+
 # --- VLA
 @pytest.mark.parametrize("d", [32, 96])
 def test_vla_workload(oracle, d):
