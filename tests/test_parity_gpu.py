@@ -273,6 +273,74 @@ def test_decode_step_empty_batch_launches_nothing():
     assert out.shape == (0, 4, 128)
 
 
+# --- maximum sizes: element offsets beyond 2^31
+def _fill_head(t, h, x):
+    t.view(-1, *t.shape[2:])[h] = torch.from_numpy(np.ascontiguousarray(x)).to(t.dtype).to(t.device)
+
+
+def test_chunked_offsets_beyond_int32(oracle):
+    # 16384 heads x 1088 tokens x 128 channels: 2.28e9 elements per q/k/v/out tensor (about
+    # 20 GB in all), so the last head's data lies past 2^31 elements. Only the first and last
+    # heads carry data; every other head has zero keys, queries and values and must read out
+    # exactly zero.
+    B, H, T, dk, dv = 128, 128, 1088, 128, 128
+    BH = B * H
+    assert BH * T * dk > 2**31
+    q = torch.zeros(B, H, T, dk, dtype=torch.bfloat16, device="cuda")
+    k, v = torch.zeros_like(q), torch.zeros_like(q)
+    beta = torch.full((B, H, T), 0.5, device="cuda")
+    gate = torch.full((B, H, T), 0.97, device="cuda")
+    w = wl.DRWorkload("edge", 1, 2, T, dk, dv, wl.GDN, "bf16")
+    small = wl.generate_dr(w, 5)
+    for j, h in enumerate((0, BH - 1)):
+        for name, t in (("q", q), ("k", k), ("v", v)):
+            _fill_head(t, h, small[name][0, j])
+        _fill_head(beta, h, small["beta"][0, j])
+        _fill_head(gate, h, small["gate"][0, j])
+    out, Sf = drs.scan(q, k, v, beta, gate, None, mode="gdn")
+    torch.cuda.synchronize()
+    ref_out, ref_S = oracle_dr(oracle, small)
+    o = out.view(BH, T, dv)
+    s = Sf.view(BH, dv, dk)
+    for j, h in enumerate((0, BH - 1)):
+        assert rel_err(tensor_np(o[h]), ref_out[0, j]) <= TOL["bf16"]
+        assert rel_err(tensor_np(s[h]), ref_S[0, j]) <= TOL["bf16"]
+    for h in (1, BH // 2, BH - 2):
+        assert torch.count_nonzero(o[h]) == 0 and torch.count_nonzero(s[h]) == 0
+    del q, k, v, out, Sf, o, s
+    torch.cuda.empty_cache()
+
+
+def test_decode_offsets_beyond_int32(oracle):
+    # 139264 heads of 128 x 128 fp32 state: 2.28e9 state elements (9.1 GB) in place
+    B, H, dk, dv = 1088, 128, 128, 128
+    BH = B * H
+    assert BH * dv * dk > 2**31
+    w = wl.DRWorkload("edge", 1, 2, 1, dk, dv, wl.KDA, "fp32", s0_std=0.1)
+    small = wl.generate_dr(w, 6)
+    q = torch.zeros(B, H, dk, device="cuda")
+    k, v = torch.zeros_like(q), torch.zeros(B, H, dv, device="cuda")
+    beta = torch.full((B, H), 0.5, device="cuda")
+    gate = torch.full((B, H, dk), 0.9, device="cuda")
+    S = torch.zeros(B, H, dv, dk, device="cuda")
+    for j, h in enumerate((0, BH - 1)):
+        for name, t in (("q", q), ("k", k), ("v", v), ("beta", beta), ("gate", gate)):
+            _fill_head(t, h, small[name][0, j, 0])
+        _fill_head(S, h, small["S0"][0, j])
+    out = drs.decode_step(q, k, v, beta, gate, S, mode="kda")
+    torch.cuda.synchronize()
+    ref_out, ref_S = oracle_dr(oracle, small)
+    o = out.view(BH, dv)
+    s = S.view(BH, dv, dk)
+    for j, h in enumerate((0, BH - 1)):
+        assert rel_err(tensor_np(o[h]), ref_out[0, j, 0]) <= TOL["fp32"]
+        assert rel_err(tensor_np(s[h]), ref_S[0, j]) <= TOL["fp32"]
+    for h in (1, BH // 2, BH - 2):
+        assert torch.count_nonzero(o[h]) == 0 and torch.count_nonzero(s[h]) == 0
+    del q, k, v, S, out, o, s
+    torch.cuda.empty_cache()
+
+
 # --- VLA
 @pytest.mark.parametrize("d", [32, 96])
 def test_vla_workload(oracle, d):
