@@ -260,12 +260,12 @@ def cpu_baseline(inputs, target_s=10.0):
     heads = int(max(1, min(BH, round(rate * target_s / w.T))))
     heads = max(1, (heads // cores) * cores) if heads >= cores else heads
     # when every head fits well inside the target, repeat whole passes to reach it
-    reps = int(max(1, min(50, round(rate * target_s / (heads * w.T)))))
+    reps = int(max(1, min(100, round(rate * target_s / (heads * w.T)))))
     sub = oracle_sample(inputs, list(range(heads)), w.T)
     t0 = time.perf_counter()
     n = 0
-    # the estimate sets the minimum; whole passes continue until the target time (<= 50)
-    while n < reps or (time.perf_counter() - t0 < target_s and n < 50):
+    # the estimate sets the minimum; whole passes continue until the target time (<= 100)
+    while n < reps or (time.perf_counter() - t0 < target_s and n < 100):
         run_oracle(sub)
         n += 1
     reps = n
