@@ -87,3 +87,19 @@ def test_decode_accounting_is_the_state_round_trip_plus_one_token():
     assert bench.algorithmic_bytes(w) == w.B * w.H * (2 * 128 * 128 * 4 + 4 * 128 * 2 + 4 + 4)
     # the resident state alone is larger than the 126 MiB L2
     assert w.B * w.H * w.dv * w.dk * 4 > 126 * 2**20
+
+
+def test_cpu_baseline_runs_whole_passes_up_to_the_target_time(oracle):
+    import re
+
+    import bench
+    from delta_rule_recurrent_chunked_b200 import workloads as wl
+
+    w = wl.workload("gdn_bf16", B=1, H=2, T=256)
+    r = bench.cpu_baseline(wl.generate_dr(w, 0), target_s=1.0)
+    m = re.search(r"(?:(\d+) passes over )?(\d+) of 2 heads x all 256 tokens .* ([\d.]+) s\)", r["sample"])
+    assert m, r["sample"]
+    passes = int(m.group(1) or 1)
+    # either the target time was reached or the pass cap (100) stopped it
+    assert float(m.group(3)) >= 0.95 or passes == 100
+    assert r["kind"] == "oracle" and r["cores"] >= 1 and r["value"] > 0
