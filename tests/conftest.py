@@ -19,5 +19,11 @@ def pytest_configure(config):
 def oracle():
     import oracle as _oracle
 
+    # tests/test_oracle_mutants.py runs the pins against deliberately broken builds of the
+    # oracle, compiled elsewhere; this variable names such a library
+    mutant = os.environ.get("ORACLE_MUTANT_LIB")
+    if mutant:
+        _oracle._LIB = mutant
+        _oracle._lib = None
     _oracle.build()
     return _oracle

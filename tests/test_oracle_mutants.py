@@ -1,0 +1,66 @@
+"""Planted mistakes in the oracle: each is a plausible slip in its arithmetic, and each must
+make at least one pin fail (the CPU tests of tests/test_oracle_pins.py and
+tests/test_golden.py).
+
+Every mutant is a copy of oracle/dr_oracle.c with one textual change, compiled with gcc into
+a temporary directory. The pins then run in a subprocess whose `oracle` fixture loads that
+library. Nothing here touches the GPU or the product path.
+"""
+import os
+import subprocess
+import sys
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+SRC = os.path.join(ROOT, "oracle", "dr_oracle.c")
+
+RESID = "const double r = vt[i] - pred[i];"
+WRITE = "S[ij] = decay[j] * S[ij] + b * r * kt[j];"
+DECAY = "if (!residual_pre_decay) s *= decay[j];"
+MUTANTS = {
+    "residual_sign": [(RESID, "const double r = vt[i] + pred[i];")],
+    "dropped_prediction": [(RESID, "const double r = vt[i];")],
+    "beta_on_v_not_write": [(RESID, "const double r = b * vt[i] - pred[i];"),
+                            (WRITE, "S[ij] = decay[j] * S[ij] + r * kt[j];")],
+    "kda_decay_on_rows": [(DECAY, "if (!residual_pre_decay) s *= decay[i % dk];"),
+                          (WRITE, "S[ij] = decay[i % dk] * S[ij] + b * r * kt[j];")],
+    "residual_against_undecayed_state": [(DECAY, "if (0) s *= decay[j];")],
+    "readout_of_transposed_state": [
+        ("for (int j = 0; j < dk; ++j) acc += S[(long)i * dk + j] * qt[j];",
+         "for (int j = 0; j < dk; ++j) acc += S[(long)(j % dv) * dk + (i % dk)] * qt[j];")],
+    "sherman_morrison_without_u_z": [("for (int i = 0; i < d; ++i) den += ut[i] * z[i];",
+                                      "for (int i = 0; i < d; ++i) den += 0.0 * ut[i] * z[i];")],
+    "vla_direction_not_normalised": [("const double inv = 1.0 / sqrt(nrm2);",
+                                      "const double inv = 1.0;")],
+    "vla_writes_along_k": [("S[(long)i * d + j] += r[i] * y[j];",
+                            "S[(long)i * d + j] += r[i] * kt[j];")],
+}
+
+
+def run_pins(tmp_path, src: str):
+    """Compile `src` as the oracle library and run the pins against it; returns the run."""
+    csrc = tmp_path / "mutant.c"
+    csrc.write_text(src)
+    lib = tmp_path / "libmutant.so"
+    subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-o", str(lib), str(csrc),
+                           "-lm"])
+    env = dict(os.environ, ORACLE_MUTANT_LIB=str(lib))
+    return subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-p", "no:cacheprovider",
+                           "-m", "not gpu", "tests/test_oracle_pins.py", "tests/test_golden.py"],
+                          cwd=ROOT, env=env, capture_output=True, text=True, timeout=600)
+
+
+def test_unmodified_oracle_passes_the_pins_by_the_same_route(tmp_path):
+    run = run_pins(tmp_path, open(SRC).read())
+    assert run.returncode == 0, run.stdout[-2000:]
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_every_planted_mistake_fails_a_pin(tmp_path, name):
+    src = open(SRC).read()
+    for old, new in MUTANTS[name]:
+        assert src.count(old) == 1, (name, old)  # the mutation still targets real code
+        src = src.replace(old, new)
+    run = run_pins(tmp_path, src)
+    assert run.returncode == 1, (name, run.stdout[-2000:])  # 1 = tests ran and some failed
