@@ -170,3 +170,42 @@ def test_product_path_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(drs, "_lib", None)
     with pytest.raises(RuntimeError, match="missing"):
         drs.lib()
+
+
+C_CALLER = r"""
+#include "drscan.h"
+int main(void) {
+    int bv = 0, np = 0;
+    int (*scan)(const void*, const void*, const void*, const float*, const float*, const float*,
+                void*, float*, int, int, int, int, int, int, cudaStream_t) = dr_scan_fwd;
+    int (*decode)(const void*, const void*, const void*, const float*, const float*, float*,
+                  void*, int, int, int, int, int, cudaStream_t) = dr_decode_step;
+    (void)scan;
+    (void)decode;
+    (void)vla_scan_fwd;
+    (void)dr_poll_error;
+    (void)dr_debug_timeout_probe;
+    /* host-only calls: a request rejected before any device query, status text, version */
+    if (dr_chunked_plan(DR_GDN | DR_IN_BF16, 0, 128, 128, &bv, &np) != DR_ERR_INVALID_ARG) return 1;
+    if (!dr_status_string(DR_ERR_TIMEOUT)[0]) return 2;
+    return dr_version() > 0 ? 0 : 3;
+}
+"""
+
+
+def test_header_serves_a_plain_c_caller(lib, tmp_path):
+    # the boundary is a C ABI: a C99 program compiles against the header without warnings,
+    # links against the library and makes its host-only calls
+    import shutil
+
+    cuda_inc = "/usr/local/cuda/include"
+    if not shutil.which("gcc") or not os.path.exists(os.path.join(cuda_inc, "cuda_runtime.h")):
+        pytest.skip("needs gcc and the CUDA runtime headers")
+    src = tmp_path / "caller.c"
+    src.write_text(C_CALLER)
+    exe = tmp_path / "caller"
+    libdir = os.path.dirname(drs.LIB_PATH)
+    subprocess.check_call(["gcc", "-std=c99", "-Wall", "-Wextra", "-Werror",
+                           "-I", os.path.join(ROOT, "include"), "-I", cuda_inc, str(src),
+                           "-L", libdir, "-ldrscan", f"-Wl,-rpath,{libdir}", "-o", str(exe)])
+    assert subprocess.run([str(exe)]).returncode == 0
