@@ -24,7 +24,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 _SRC = os.path.join(_HERE, "dr_oracle.c")
 _LIB = os.path.join(_HERE, "liboracle.so")
 
-LINEAR, DELTANET, GDN, KDA = 0, 1, 2, 3
+LINEAR, DELTANET, GDN, KDA, GDN2 = 0, 1, 2, 3, 4
 
 _lib = None
 
@@ -45,6 +45,8 @@ def _load():
         dp = ctypes.POINTER(ctypes.c_double)
         lib.oracle_dr_scan.argtypes = [dp, dp, dp, dp, dp, dp, dp, dp] + [ctypes.c_int] * 7
         lib.oracle_dr_scan.restype = ctypes.c_int
+        lib.oracle_dr_scan_ex.argtypes = [dp] * 11 + [ctypes.c_int] * 7
+        lib.oracle_dr_scan_ex.restype = ctypes.c_int
         lib.oracle_vla_scan.argtypes = [dp] * 6 + [ctypes.c_double] + [dp] * 3 + [ctypes.c_int] * 4
         lib.oracle_vla_scan.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
@@ -102,6 +104,50 @@ def dr_scan(q, k, v, beta=None, gate=None, S0=None, mode=DELTANET, residual_pre_
     if rc != 0:
         raise RuntimeError(f"oracle_dr_scan failed ({rc})")
     return out, Sf
+
+
+def dr_scan_ex(q, k, v, beta=None, gate=None, S0=None, mode=DELTANET, erase=None, write=None,
+               residual_pre_decay=False):
+    """Per-token delta-rule scan in fp64, every variant including Gated DeltaNet-2, also
+    returning the per-token write values u_t = beta_t r_t (v_t for plain linear attention).
+
+    As dr_scan, plus: mode GDN2 takes gate [B,H,T] (alpha), erase [B,H,T,dk] (b) and
+    write [B,H,T,dv] (w). Returns (out, S_final, u [B,H,T,dv]).
+    """
+    q, k, v = _f64(q), _f64(k), _f64(v)
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    if k.shape != q.shape or v.shape[:3] != (B, H, T):
+        raise ValueError("shape mismatch")
+    beta = _f64(beta) if mode != LINEAR else None
+    gate = _f64(gate) if mode in (GDN, KDA, GDN2) else None
+    if beta is not None and beta.shape != (B, H, T):
+        raise ValueError("beta shape")
+    if gate is not None:
+        want = (B, H, T, dk) if mode == KDA else (B, H, T)
+        if gate.shape != want:
+            raise ValueError("gate shape")
+    if mode == GDN2:
+        erase, write = _f64(erase), _f64(write)
+        if erase is None or erase.shape != (B, H, T, dk):
+            raise ValueError("erase shape")
+        if write is None or write.shape != (B, H, T, dv):
+            raise ValueError("write shape")
+    else:
+        erase = write = None
+    S0 = _f64(S0)
+    if S0 is not None and S0.shape != (B, H, dv, dk):
+        raise ValueError("S0 shape")
+    out = np.empty((B, H, T, dv), np.float64)
+    Sf = np.empty((B, H, dv, dk), np.float64)
+    u = np.empty((B, H, T, dv), np.float64)
+    rc = _load().oracle_dr_scan_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(gate),
+                                   _ptr(erase), _ptr(write), _ptr(S0), _ptr(out), _ptr(Sf),
+                                   _ptr(u), B, H, T, dk, dv, int(mode),
+                                   int(bool(residual_pre_decay)))
+    if rc != 0:
+        raise RuntimeError(f"oracle_dr_scan_ex failed ({rc})")
+    return out, Sf, u
 
 
 def vla_scan(q, k, v, u, S0=None, A0=None, lambda0=1.0, want_state=True):

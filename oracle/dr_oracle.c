@@ -17,6 +17,10 @@
  *    DeltaNet prediction vbar = W_{t-1} kappa, residual r = v - vbar, write
  *    W <- W + beta r (x) kappa; Gated DeltaNet W <- alpha W + beta r_alpha (x) kappa
  *    (scalar decay); Kimi Delta Attention decays per key-feature channel.
+ *    Gated DeltaNet-2 separates a per-key-channel erase gate b and a per-value-channel
+ *    write gate w: erase direction e = b (.) kappa, write target z = w (.) v, and it
+ *    writes the residual r = z - W~ e. The CLVR passages of the same page route a
+ *    layer's internal write signal (write value or residual) to later layers.
  *  - "Variational Linear Attention (VLA)" (gist.science 2605.11196), section 2.1
  *    (plain accumulation S_t = S_{t-1} + v_t k_t^T), section 2.2 (inverse penalty
  *    A_t = M_t^{-1} kept by a Sherman-Morrison rank-1 update) and section 2.3
@@ -33,12 +37,20 @@
  *  - Readout after the write: o_t = S_t q_t. No feature map and no 1/sqrt(d_k)
  *    scale inside the scan; q and k arrive as the caller prepared them.
  *  - Plain linear attention ignores beta and gate.
+ *  - Gated DeltaNet-2: W~ is the decayed memory alpha_t S_{t-1} (scalar alpha, as in
+ *    Gated DeltaNet), and the residual is written along the erase direction e:
+ *    S_t = W~ + beta r e^T, so that with a unit e and beta = 1, S_t e = z exactly.
+ *    With b = w = 1 it is Gated DeltaNet.
+ *  - The exported write value of a token is u_t = beta_t r_t, the vector the step adds
+ *    to memory along its key (along e for Gated DeltaNet-2); plain linear attention
+ *    writes u_t = v_t.
  *  - VLA: z_t = A_{t-1} u_t (Sherman-Morrison for M_t = M_{t-1} + u_t u_t^T),
  *    A_0 = I / lambda0, readout o_t = S_t q_hat_t, no beta and no decay.
  *
  * Layouts (all row-major, contiguous):
  *   q, k   [B, H, T, dk]      v, out [B, H, T, dv]      beta [B, H, T]
- *   gate   GDN: [B, H, T]     KDA: [B, H, T, dk]        (alpha values, not logs)
+ *   gate   GDN, GDN2: [B, H, T]   KDA: [B, H, T, dk]    (alpha values, not logs)
+ *   erase  GDN2: [B, H, T, dk]   write  GDN2: [B, H, T, dv]   u_out [B, H, T, dv]
  *   S0, S_final [B, H, dv, dk]   (S maps keys to values: S k in R^{dv})
  *   VLA: q, k, v, u, out [B, H, T, d];  S0, S_final, A0, A_final [B, H, d, d]
  */
@@ -53,6 +65,7 @@
 #define ORACLE_DELTANET 1
 #define ORACLE_GDN 2
 #define ORACLE_KDA 3
+#define ORACLE_GDN2 4
 
 int oracle_num_threads(void) {
 #ifdef _OPENMP
@@ -62,27 +75,44 @@ int oracle_num_threads(void) {
 #endif
 }
 
-/* One (batch, head) sequence of the delta-rule family. S is dv x dk, updated in place. */
+/* One (batch, head) sequence of the delta-rule family. S is dv x dk, updated in place.
+ * work holds dk + dv doubles (Gated DeltaNet-2's e and z). */
 static void dr_sequence(const double* q, const double* k, const double* v,
-                        const double* beta, const double* gate, double* S,
-                        double* out, double* decay, double* pred,
+                        const double* beta, const double* gate, const double* erase,
+                        const double* write, double* S, double* out, double* u_out,
+                        double* decay, double* pred, double* work,
                         long T, int dk, int dv, int mode, int residual_pre_decay) {
     for (long t = 0; t < T; ++t) {
         const double* kt = k + t * dk;
         const double* qt = q + t * dk;
         const double* vt = v + t * dv;
         double* ot = out + t * dv;
+        double* ut = u_out ? u_out + t * dv : NULL;
 
         if (mode == ORACLE_LINEAR) {
             /* S_t = S_{t-1} + v_t k_t^T  (VLA page, section 2.1) */
             for (int i = 0; i < dv; ++i)
                 for (int j = 0; j < dk; ++j)
                     S[(long)i * dk + j] += vt[i] * kt[j];
+            if (ut)
+                for (int i = 0; i < dv; ++i) ut[i] = vt[i];
         } else {
-            /* decay factor per key channel j: 1 (DeltaNet), alpha_t (GDN), alpha_t[j] (KDA) */
+            /* Gated DeltaNet-2 reads and writes along e = b (.) k with the target z = w (.) v;
+             * every other variant along k with the target v */
+            const double* kk = kt;
+            const double* vv = vt;
+            if (mode == ORACLE_GDN2) {
+                double* e = work;
+                double* z = work + dk;
+                for (int j = 0; j < dk; ++j) e[j] = erase[t * dk + j] * kt[j];
+                for (int i = 0; i < dv; ++i) z[i] = write[t * dv + i] * vt[i];
+                kk = e;
+                vv = z;
+            }
+            /* decay factor per key channel j: 1 (DeltaNet), alpha_t (GDN, GDN2), alpha_t[j] (KDA) */
             for (int j = 0; j < dk; ++j) {
                 if (mode == ORACLE_DELTANET) decay[j] = 1.0;
-                else if (mode == ORACLE_GDN) decay[j] = gate[t];
+                else if (mode == ORACLE_GDN || mode == ORACLE_GDN2) decay[j] = gate[t];
                 else decay[j] = gate[t * dk + j];
             }
             /* prediction vbar = S' k, with S' = S (.) decay (or S itself, literal reading) */
@@ -91,18 +121,19 @@ static void dr_sequence(const double* q, const double* k, const double* v,
                 for (int j = 0; j < dk; ++j) {
                     double s = S[(long)i * dk + j];
                     if (!residual_pre_decay) s *= decay[j];
-                    acc += s * kt[j];
+                    acc += s * kk[j];
                 }
                 pred[i] = acc;
             }
             /* S_t = S' + beta_t (v_t - vbar) k_t^T */
             const double b = beta[t];
             for (int i = 0; i < dv; ++i) {
-                const double r = vt[i] - pred[i];
+                const double r = vv[i] - pred[i];
                 for (int j = 0; j < dk; ++j) {
                     long ij = (long)i * dk + j;
-                    S[ij] = decay[j] * S[ij] + b * r * kt[j];
+                    S[ij] = decay[j] * S[ij] + b * r * kk[j];
                 }
+                if (ut) ut[i] = b * r;
             }
         }
         /* readout after the write: o_t = S_t q_t */
@@ -115,19 +146,23 @@ static void dr_sequence(const double* q, const double* k, const double* v,
 }
 
 /*
- * Delta-rule family scan. beta may be NULL for LINEAR; gate is NULL for LINEAR and
- * DELTANET, [B,H,T] for GDN, [B,H,T,dk] for KDA. S0 NULL means zeros; S_final NULL
- * means not written. Returns 0, or -1 on a bad argument.
+ * Delta-rule family scan with every option. beta may be NULL for LINEAR; gate is NULL for
+ * LINEAR and DELTANET, [B,H,T] for GDN and GDN2, [B,H,T,dk] for KDA; erase [B,H,T,dk] and
+ * write [B,H,T,dv] are GDN2's gates (NULL otherwise). S0 NULL means zeros; S_final and
+ * u_out (the per-token write values) NULL mean not written. Returns 0, or -1 on a bad
+ * argument.
  */
-int oracle_dr_scan(const double* q, const double* k, const double* v,
-                   const double* beta, const double* gate, const double* S0,
-                   double* out, double* S_final,
-                   int B, int H, int T, int dk, int dv, int mode, int residual_pre_decay) {
+int oracle_dr_scan_ex(const double* q, const double* k, const double* v,
+                      const double* beta, const double* gate, const double* erase,
+                      const double* write, const double* S0,
+                      double* out, double* S_final, double* u_out,
+                      int B, int H, int T, int dk, int dv, int mode, int residual_pre_decay) {
     if (B < 0 || H < 0 || T < 0 || dk <= 0 || dv <= 0) return -1;
-    if (mode < ORACLE_LINEAR || mode > ORACLE_KDA) return -1;
+    if (mode < ORACLE_LINEAR || mode > ORACLE_GDN2) return -1;
     if (!q || !k || !v || !out) return -1;
     if (mode != ORACLE_LINEAR && !beta) return -1;
-    if ((mode == ORACLE_GDN || mode == ORACLE_KDA) && !gate) return -1;
+    if ((mode == ORACLE_GDN || mode == ORACLE_KDA || mode == ORACLE_GDN2) && !gate) return -1;
+    if (mode == ORACLE_GDN2 && (!erase || !write)) return -1;
     const long BH = (long)B * H;
     const long state = (long)dv * dk;
     int failed = 0;
@@ -136,24 +171,40 @@ int oracle_dr_scan(const double* q, const double* k, const double* v,
         double* S = (double*)malloc(sizeof(double) * (size_t)state);
         double* decay = (double*)malloc(sizeof(double) * (size_t)dk);
         double* pred = (double*)malloc(sizeof(double) * (size_t)dv);
-        if (!S || !decay || !pred) {
+        double* work = (double*)malloc(sizeof(double) * (size_t)(dk + dv));
+        if (!S || !decay || !pred || !work) {
             failed = 1;
         } else {
             if (S0) memcpy(S, S0 + bh * state, sizeof(double) * (size_t)state);
             else memset(S, 0, sizeof(double) * (size_t)state);
             const double* g = NULL;
-            if (mode == ORACLE_GDN) g = gate + bh * T;
+            if (mode == ORACLE_GDN || mode == ORACLE_GDN2) g = gate + bh * T;
             if (mode == ORACLE_KDA) g = gate + bh * (long)T * dk;
+            const int gdn2 = mode == ORACLE_GDN2;
             dr_sequence(q + bh * (long)T * dk, k + bh * (long)T * dk, v + bh * (long)T * dv,
-                        beta ? beta + bh * T : NULL, g, S, out + bh * (long)T * dv,
-                        decay, pred, T, dk, dv, mode, residual_pre_decay);
+                        beta ? beta + bh * T : NULL, g,
+                        gdn2 ? erase + bh * (long)T * dk : NULL,
+                        gdn2 ? write + bh * (long)T * dv : NULL, S, out + bh * (long)T * dv,
+                        u_out ? u_out + bh * (long)T * dv : NULL, decay, pred, work, T, dk, dv,
+                        mode, residual_pre_decay);
             if (S_final) memcpy(S_final + bh * state, S, sizeof(double) * (size_t)state);
         }
         free(S);
         free(decay);
         free(pred);
+        free(work);
     }
     return failed ? -1 : 0;
+}
+
+/* The delta-rule family scan without Gated DeltaNet-2 and without write values. */
+int oracle_dr_scan(const double* q, const double* k, const double* v,
+                   const double* beta, const double* gate, const double* S0,
+                   double* out, double* S_final,
+                   int B, int H, int T, int dk, int dv, int mode, int residual_pre_decay) {
+    if (mode == ORACLE_GDN2) return -1;
+    return oracle_dr_scan_ex(q, k, v, beta, gate, NULL, NULL, S0, out, S_final, NULL, B, H, T,
+                             dk, dv, mode, residual_pre_decay);
 }
 
 /* One VLA sequence. S and A are d x d, updated in place; work holds 3*d doubles. */

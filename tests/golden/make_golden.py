@@ -29,6 +29,11 @@ VLA_PAGE = ('"Variational Linear Attention (VLA)" (gist.science 2605.11196), sec
             'Sherman-Morrison update of A = M^-1, alpha_hat = A k_hat / ||A k_hat||, '
             'S_t = S_{t-1} + (v - S_{t-1} k_hat) alpha_hat^T')
 
+GDN2_PAGE = ('"Mechanisms, trade-offs and cross-layer routing of linear-attention architectures" '
+             '(aitrends.kr), sections "Methodology" and "Technical details": Gated DeltaNet-2 '
+             'with per-channel erase b and write w, e = b (.) kappa, z = w (.) v, residual '
+             'r = z - W~ e (W~ the decayed memory), written along e')
+
 CASES = {
     "deltanet_d2_t2": dict(
         mode=oracle.DELTANET,
@@ -64,6 +69,20 @@ CASES = {
             "t=2: S1 diag(1,1/2) = [[3/4,1/4],[5/4,1/2]], its k2 column (1/4,1/2), r = (-1/4,3/2), "
             "S2 = [[3/4,1/8],[5/4,5/4]], o2 = S2 (0,1) = (1/8,5/4)",
         ]),
+    "gdn2_d2_t2": dict(
+        mode=oracle.GDN2,
+        cite=GDN2_PAGE,
+        q=[[1, 0], [1, 1]], k=[[1, 1], [1, 0]], v=[[2, 4], [4, 2]], beta=[0.5, 1.0],
+        gate=[0.5, 0.5], erase=[[1, 0], [1, 1]], write=[[1, 0.5], [0.5, 1]], S0=[[1, 2], [0, 1]],
+        derivation=[
+            "t=1: e = b (.) k = (1,0), z = w (.) v = (2,2), W~ = S0/2 = [[1/2,1],[0,1/2]], "
+            "W~ e = (1/2,0), r = (3/2,2), u = beta r = (3/4,1), S1 = W~ + u e^T = [[5/4,1],[1,1/2]], "
+            "o1 = S1 (1,0) = (5/4,1)",
+            "t=2: e = (1,0), z = (2,2), W~ = S1/2 = [[5/8,1/2],[1/2,1/4]], W~ e = (5/8,1/2), "
+            "r = (11/8,3/2), u = r (beta = 1), S2 = [[2,1/2],[2,1/4]] (S2 e = z), "
+            "o2 = S2 (1,1) = (5/2,9/4)",
+            "(written along k instead of e: S1 = W~ + u k1^T = [[5/4,7/4],[1,3/2]])",
+        ]),
     "vla_d3_t2": dict(
         mode="vla",
         cite=VLA_PAGE,
@@ -87,8 +106,10 @@ def _bh(x):
 def build_case(name: str, spec: dict) -> dict:
     fx = {"case": name, "cite": spec["cite"], "derivation": spec["derivation"],
           "mode": spec["mode"] if spec["mode"] == "vla" else
-          {oracle.DELTANET: "deltanet", oracle.GDN: "gdn", oracle.KDA: "kda"}[spec["mode"]]}
-    inputs = {key: spec[key] for key in ("q", "k", "v", "beta", "gate", "S0", "u", "lambda0")
+          {oracle.DELTANET: "deltanet", oracle.GDN: "gdn", oracle.KDA: "kda",
+           oracle.GDN2: "gdn2"}[spec["mode"]]}
+    inputs = {key: spec[key] for key in ("q", "k", "v", "beta", "gate", "erase", "write", "S0",
+                                         "u", "lambda0")
               if key in spec}
     fx["inputs"] = inputs
     if spec["mode"] == "vla":
@@ -100,9 +121,13 @@ def build_case(name: str, spec: dict) -> dict:
         beta = np.asarray(spec["beta"], np.float64)[None, None]
         gate = None if "gate" not in spec else _bh(spec["gate"])
         S0 = None if "S0" not in spec else np.asarray(spec["S0"], np.float64)[None, None]
-        out, Sf = oracle.dr_scan(_bh(spec["q"]), _bh(spec["k"]), _bh(spec["v"]), beta, gate, S0,
-                                 spec["mode"])
-        fx["expected"] = {"out": out[0, 0].tolist(), "S_final": Sf[0, 0].tolist()}
+        erase = None if "erase" not in spec else _bh(spec["erase"])
+        write = None if "write" not in spec else _bh(spec["write"])
+        out, Sf, u = oracle.dr_scan_ex(_bh(spec["q"]), _bh(spec["k"]), _bh(spec["v"]), beta, gate,
+                                       S0, spec["mode"], erase=erase, write=write)
+        # u: the per-token write values beta_t r_t
+        fx["expected"] = {"out": out[0, 0].tolist(), "S_final": Sf[0, 0].tolist(),
+                          "u": u[0, 0].tolist()}
     return fx
 
 

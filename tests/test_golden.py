@@ -21,21 +21,30 @@ import pytest
 from helpers import rel_err
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
-CASES = ["deltanet_d2_t2", "gdn_d2_t3", "kda_d2_t2", "vla_d3_t2"]
+CASES = ["deltanet_d2_t2", "gdn_d2_t3", "kda_d2_t2", "gdn2_d2_t2", "vla_d3_t2"]
 
 # The same cases worked by hand from the per-token definitions (fractions written out).
 HAND = {
+    # u: the write values beta_t r_t of the derivations' residuals r
     "deltanet_d2_t2": {
         "out": [[1, 0], [0, 2]],
         "S_final": [[1 / 2, -1 / 2], [1, 1]],
+        "u": [[1, 0], [-1 / 2, 1]],
     },
     "gdn_d2_t3": {
         "out": [[1, 2], [5 / 2, 1], [1 / 16, 5 / 8]],
         "S_final": [[9 / 16, 1 / 2], [5 / 8, 0]],
+        "u": [[1, 2], [2, 0], [7 / 16, 3 / 8]],
     },
     "kda_d2_t2": {
         "out": [[5 / 4, 9 / 4], [1 / 8, 5 / 4]],
         "S_final": [[3 / 4, 1 / 8], [5 / 4, 5 / 4]],
+        "u": [[1 / 4, -1 / 4], [-1 / 8, 3 / 4]],
+    },
+    "gdn2_d2_t2": {
+        "out": [[5 / 4, 1], [5 / 2, 9 / 4]],
+        "S_final": [[2, 1 / 2], [2, 1 / 4]],
+        "u": [[3 / 4, 1], [11 / 8, 3 / 2]],
     },
     "vla_d3_t2": {
         "out": [[1, 2, 3], [-1, -1, -3]],
@@ -60,13 +69,17 @@ def run_oracle(oracle, fx, residual_pre_decay=False):
         out, Sf, Af = oracle.vla_scan(bh(x["q"]), bh(x["k"]), bh(x["v"]), bh(x["u"]),
                                       lambda0=x["lambda0"])
         return {"out": out[0, 0], "S_final": Sf[0, 0], "A_final": Af[0, 0]}
-    mode = {"deltanet": oracle.DELTANET, "gdn": oracle.GDN, "kda": oracle.KDA}[fx["mode"]]
+    mode = {"deltanet": oracle.DELTANET, "gdn": oracle.GDN, "kda": oracle.KDA,
+            "gdn2": oracle.GDN2}[fx["mode"]]
     beta = np.asarray(x["beta"], np.float64)[None, None]
     gate = bh(x["gate"]) if "gate" in x else None
     S0 = np.asarray(x["S0"], np.float64)[None, None] if "S0" in x else None
-    out, Sf = oracle.dr_scan(bh(x["q"]), bh(x["k"]), bh(x["v"]), beta, gate, S0, mode,
-                             residual_pre_decay=residual_pre_decay)
-    return {"out": out[0, 0], "S_final": Sf[0, 0]}
+    erase = bh(x["erase"]) if "erase" in x else None
+    write = bh(x["write"]) if "write" in x else None
+    out, Sf, u = oracle.dr_scan_ex(bh(x["q"]), bh(x["k"]), bh(x["v"]), beta, gate, S0, mode,
+                                   erase=erase, write=write,
+                                   residual_pre_decay=residual_pre_decay)
+    return {"out": out[0, 0], "S_final": Sf[0, 0], "u": u[0, 0]}
 
 
 @pytest.mark.parametrize("name", CASES)
@@ -83,6 +96,14 @@ def test_oracle_reproduces_the_fixture_exactly(oracle, name):
     got = run_oracle(oracle, fx)
     for key, want in fx["expected"].items():
         assert np.array_equal(got[key], np.asarray(want)), key
+
+
+def test_gdn2_example_recalls_its_write_target():
+    # the reading's exact-recall property on the worked example: at t = 2, beta = 1 and
+    # e2 = (1,0) is a unit vector, so S2 e2 = z2 = w2 (.) v2 = (2, 2)
+    fx = load("gdn2_d2_t2")
+    S2 = np.asarray(fx["expected"]["S_final"])
+    assert np.array_equal(S2 @ np.array([1.0, 0.0]), [2.0, 2.0])
 
 
 def test_gdn_example_separates_the_two_residual_readings(oracle):

@@ -15,16 +15,26 @@ import pytest
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 SRC = os.path.join(ROOT, "oracle", "dr_oracle.c")
 
-RESID = "const double r = vt[i] - pred[i];"
-WRITE = "S[ij] = decay[j] * S[ij] + b * r * kt[j];"
+RESID = "const double r = vv[i] - pred[i];"
+WRITE = "S[ij] = decay[j] * S[ij] + b * r * kk[j];"
 DECAY = "if (!residual_pre_decay) s *= decay[j];"
+UOUT = "if (ut) ut[i] = b * r;"
 MUTANTS = {
-    "residual_sign": [(RESID, "const double r = vt[i] + pred[i];")],
-    "dropped_prediction": [(RESID, "const double r = vt[i];")],
-    "beta_on_v_not_write": [(RESID, "const double r = b * vt[i] - pred[i];"),
-                            (WRITE, "S[ij] = decay[j] * S[ij] + r * kt[j];")],
+    "residual_sign": [(RESID, "const double r = vv[i] + pred[i];")],
+    "dropped_prediction": [(RESID, "const double r = vv[i];")],
+    "beta_on_v_not_write": [(RESID, "const double r = b * vv[i] - pred[i];"),
+                            (WRITE, "S[ij] = decay[j] * S[ij] + r * kk[j];")],
     "kda_decay_on_rows": [(DECAY, "if (!residual_pre_decay) s *= decay[i % dk];"),
-                          (WRITE, "S[ij] = decay[i % dk] * S[ij] + b * r * kt[j];")],
+                          (WRITE, "S[ij] = decay[i % dk] * S[ij] + b * r * kk[j];")],
+    "gdn2_writes_along_k": [(WRITE, "S[ij] = decay[j] * S[ij] + b * r * kt[j];")],
+    "gdn2_reads_along_k": [("acc += s * kk[j];", "acc += s * kt[j];")],
+    "gdn2_target_ignores_write_gate": [("z[i] = write[t * dv + i] * vt[i];", "z[i] = vt[i];")],
+    "gdn2_erase_ignores_gate": [("e[j] = erase[t * dk + j] * kt[j];", "e[j] = kt[j];")],
+    "gdn2_without_decay": [("else if (mode == ORACLE_GDN || mode == ORACLE_GDN2) decay[j] = gate[t];",
+                            "else if (mode == ORACLE_GDN) decay[j] = gate[t];\n"
+                            "                else if (mode == ORACLE_GDN2) decay[j] = 1.0;")],
+    "write_value_without_beta": [(UOUT, "if (ut) ut[i] = r;")],
+    "write_value_is_the_target": [(UOUT, "if (ut) ut[i] = b * vv[i];")],
     "residual_against_undecayed_state": [(DECAY, "if (0) s *= decay[j];")],
     "readout_of_transposed_state": [
         ("for (int j = 0; j < dk; ++j) acc += S[(long)i * dk + j] * qt[j];",

@@ -317,3 +317,126 @@ def test_vla_bounded_state_soft(oracle):
     _, Slin = oracle.dr_scan(q, k, v, None, None, None, LINEAR)
     assert np.linalg.norm(Sf[0, 0]) < 10 * d
     assert np.linalg.norm(Slin[0, 0]) > 3 * np.linalg.norm(Sf[0, 0])
+
+
+# ====================================================================================
+# Gated DeltaNet-2 and the per-token write values (the routed signal of the cross-layer
+# routing passages). Overview page, sections "Methodology" and "Technical details":
+# Gated DeltaNet-2 separates a per-key-channel erase gate b and a per-value-channel write
+# gate w, with e = b (.) kappa, z = w (.) v and the residual r = z - W~ e; the reading
+# taken: W~ = alpha S_{t-1}, S_t = W~ + beta r e^T. The write value of a token is
+# u_t = beta_t r_t (what the step adds along its key); plain linear attention writes v_t.
+# ====================================================================================
+GDN2 = 4
+
+
+def _rand_gdn2(rng, B, H, T, dk, dv):
+    q, k, v, beta, gate, S0 = _rand_dr(rng, B, H, T, dk, dv, GDN)
+    erase = rng.uniform(0.1, 1.0, (B, H, T, dk))
+    write = rng.uniform(0.1, 1.0, (B, H, T, dv))
+    return q, k, v, beta, gate, S0, erase, write
+
+
+def test_gdn2_with_unit_gates_is_gated_deltanet(oracle):
+    rng = np.random.default_rng(40)
+    q, k, v, beta, gate, S0, _, _ = _rand_gdn2(rng, 2, 2, 33, 6, 5)
+    out, Sf, _ = oracle.dr_scan_ex(q, k, v, beta, gate, S0, GDN2, erase=np.ones_like(k),
+                                   write=np.ones_like(v))
+    ref_out, ref_S = oracle.dr_scan(q, k, v, beta, gate, S0, GDN)
+    assert np.array_equal(out, ref_out) and np.array_equal(Sf, ref_S)
+
+
+def test_gdn2_recalls_the_write_target_along_a_unit_erase_direction(oracle):
+    # beta = 1 and a unit e_t = b_t (.) k_t: after the write, S_t e_t = z_t = w_t (.) v_t
+    # exactly, whatever the decay (read back with q_t = e_t)
+    rng = np.random.default_rng(41)
+    B, H, T, dk, dv = 1, 2, 12, 6, 4
+    q, k, v, beta, gate, S0, erase, write = _rand_gdn2(rng, B, H, T, dk, dv)
+    e = _unit(rng.standard_normal((B, H, T, dk)))
+    k = e / erase  # so that b (.) k = e
+    out, _, _ = oracle.dr_scan_ex(e, k, v, np.ones_like(beta), gate, S0, GDN2, erase=erase,
+                                  write=write)
+    assert _rel(out, write * v) < 1e-12
+    # the same with the write gate ignored would recall v instead
+    assert _rel(write * v, v) > 1e-1
+
+
+def test_gdn2_without_erase_only_decays(oracle):
+    # b = 0: e = 0, nothing is read or written; S_T = (prod alpha) S0 and every write value
+    # is beta_t z_t (the whole target, with nothing predicted)
+    rng = np.random.default_rng(42)
+    q, k, v, beta, gate, S0, _, write = _rand_gdn2(rng, 1, 3, 15, 5, 4)
+    out, Sf, u = oracle.dr_scan_ex(q, k, v, beta, gate, S0, GDN2, erase=np.zeros_like(k),
+                                   write=write)
+    decay = np.prod(gate, axis=-1)[..., None, None]
+    assert _rel(Sf, decay * S0) < 1e-13
+    assert _rel(u, beta[..., None] * write * v) < 1e-13
+
+
+def test_gdn2_key_channels_without_erase_are_never_written(oracle):
+    # the erase gate is per key channel: a channel with b = 0 at every step keeps only its
+    # decayed initial column, whatever the keys and values
+    rng = np.random.default_rng(43)
+    q, k, v, beta, gate, S0, erase, write = _rand_gdn2(rng, 2, 1, 21, 7, 3)
+    off = [1, 4]
+    erase[..., off] = 0.0
+    _, Sf, _ = oracle.dr_scan_ex(q, k, v, beta, gate, S0, GDN2, erase=erase, write=write)
+    decay = np.prod(gate, axis=-1)[..., None, None]
+    assert _rel(Sf[..., off], decay * S0[..., off]) < 1e-13
+    on = [0, 2, 3, 5, 6]
+    assert _rel(Sf[..., on], decay * S0[..., on]) > 1e-2
+
+
+def test_gdn2_zero_write_gate_erases_along_e(oracle):
+    # w = 0, beta = 1, unit e: the write removes what the memory holds along e, S_t e_t = 0
+    rng = np.random.default_rng(44)
+    B, H, T, dk, dv = 1, 1, 9, 5, 3
+    q, k, v, beta, gate, S0, erase, write = _rand_gdn2(rng, B, H, T, dk, dv)
+    e = _unit(rng.standard_normal((B, H, T, dk)))
+    out, _, _ = oracle.dr_scan_ex(e, e / erase, v, np.ones_like(beta), gate, S0, GDN2,
+                                  erase=erase, write=np.zeros_like(write))
+    assert np.max(np.abs(out)) < 1e-13
+
+
+@pytest.mark.parametrize("mode", [LINEAR, DELTANET, GDN, KDA, GDN2])
+def test_write_values_rebuild_the_final_state(oracle, mode):
+    # every step is S_t = S_{t-1} diag(a_t) + u_t key_t^T, so the exported write values and
+    # the decays alone rebuild S_T:  S_T = S0 diag(prod_t a_t) + sum_t u_t key_t^T
+    # diag(prod_{s>t} a_s)   (key = e = b (.) k for Gated DeltaNet-2, k otherwise)
+    rng = np.random.default_rng(45 + mode)
+    B, H, T, dk, dv = 2, 2, 17, 6, 4
+    if mode == GDN2:
+        q, k, v, beta, gate, S0, erase, write = _rand_gdn2(rng, B, H, T, dk, dv)
+    else:
+        q, k, v, beta, gate, S0 = _rand_dr(rng, B, H, T, dk, dv, mode)
+        erase = write = None
+    _, Sf, u = oracle.dr_scan_ex(q, k, v, beta, gate, S0, mode, erase=erase, write=write)
+    if mode in (LINEAR, DELTANET):
+        a = np.ones((B, H, T, dk))
+    elif mode in (GDN, GDN2):
+        a = np.repeat(gate[..., None], dk, axis=-1)
+    else:
+        a = gate
+    key = erase * k if mode == GDN2 else k
+    after = np.ones_like(a)  # prod_{s>t} a_s per key channel
+    for t in range(T - 2, -1, -1):
+        after[:, :, t] = after[:, :, t + 1] * a[:, :, t + 1]
+    total = after[:, :, 0] * a[:, :, 0]
+    rebuilt = S0 * total[:, :, None, :] + np.einsum("bhtv,bhtd->bhvd", u, key * after)
+    assert _rel(Sf, rebuilt) < 1e-12
+    if mode == LINEAR:
+        assert np.array_equal(u, v)
+
+
+@pytest.mark.parametrize("mode", [DELTANET, GDN, KDA, GDN2])
+def test_first_write_value_from_a_zero_state(oracle, mode):
+    # with S0 = 0 the first prediction is zero: u_0 = beta_0 v_0 (beta_0 w_0 (.) v_0 for GDN-2)
+    rng = np.random.default_rng(50 + mode)
+    if mode == GDN2:
+        q, k, v, beta, gate, _, erase, write = _rand_gdn2(rng, 1, 2, 3, 4, 5)
+    else:
+        q, k, v, beta, gate, _ = _rand_dr(rng, 1, 2, 3, 4, 5, mode)
+        erase = write = None
+    _, _, u = oracle.dr_scan_ex(q, k, v, beta, gate, None, mode, erase=erase, write=write)
+    target = write * v if mode == GDN2 else v
+    assert _rel(u[:, :, 0], beta[:, :, 0, None] * target[:, :, 0]) < 1e-15
