@@ -49,6 +49,9 @@ def _load():
         lib.oracle_dr_scan_ex.restype = ctypes.c_int
         lib.oracle_vla_scan.argtypes = [dp] * 6 + [ctypes.c_double] + [dp] * 3 + [ctypes.c_int] * 4
         lib.oracle_vla_scan.restype = ctypes.c_int
+        lib.oracle_vla_scan_ex.argtypes = ([dp] * 7 + [ctypes.c_double] + [dp] * 4
+                                           + [ctypes.c_int] * 5)
+        lib.oracle_vla_scan_ex.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
@@ -173,3 +176,31 @@ def vla_scan(q, k, v, u, S0=None, A0=None, lambda0=1.0, want_state=True):
     if rc != 0:
         raise RuntimeError(f"oracle_vla_scan failed ({rc})")
     return out, Sf, Af
+
+
+def vla_scan_ratio(q, k, v, u, S0=None, A0=None, n0=None, lambda0=1.0):
+    """Per-token VLA scan in fp64 with the ratio readout o_t = S_t q_t / (n_t q_t), where
+    n_t = n_{t-1} + (1 - n_{t-1} k_t) alpha_hat_t^T is the same write applied to a value
+    held at 1. q: [B,H,T,d] the feature-mapped queries; k: the unit-norm feature-mapped keys;
+    n0: [B,H,d] or None (zeros). Returns (out, S_final, A_final, n_final)."""
+    q, k, v, u = _f64(q), _f64(k), _f64(v), _f64(u)
+    B, H, T, d = q.shape
+    for x in (k, v, u):
+        if x.shape != q.shape:
+            raise ValueError("shape mismatch")
+    S0, A0, n0 = _f64(S0), _f64(A0), _f64(n0)
+    for x in (S0, A0):
+        if x is not None and x.shape != (B, H, d, d):
+            raise ValueError("state shape")
+    if n0 is not None and n0.shape != (B, H, d):
+        raise ValueError("n0 shape")
+    out = np.empty((B, H, T, d), np.float64)
+    Sf = np.empty((B, H, d, d), np.float64)
+    Af = np.empty((B, H, d, d), np.float64)
+    nf = np.empty((B, H, d), np.float64)
+    rc = _load().oracle_vla_scan_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(S0), _ptr(A0),
+                                    _ptr(n0), float(lambda0), _ptr(out), _ptr(Sf), _ptr(Af),
+                                    _ptr(nf), B, H, T, d, 1)
+    if rc != 0:
+        raise RuntimeError(f"oracle_vla_scan_ex failed ({rc})")
+    return out, Sf, Af, nf

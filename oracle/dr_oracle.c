@@ -46,6 +46,12 @@
  *    writes u_t = v_t.
  *  - VLA: z_t = A_{t-1} u_t (Sherman-Morrison for M_t = M_{t-1} + u_t u_t^T),
  *    A_0 = I / lambda0, readout o_t = S_t q_hat_t, no beta and no decay.
+ *  - VLA ratio readout (section 2.3: the output is a ratio of recurrences, as in linear
+ *    attention, with an ELU+1 feature map): the denominator recurrence is the same write
+ *    applied to one more value channel held at 1, n_t = n_{t-1} + (1 - n_{t-1} k_hat_t)
+ *    alpha_hat_t^T (n_0 = 0 unless given), and o_t = S_t q_t / (n_t q_t). The feature map
+ *    is the caller's, like every other feature map here: q arrives as phi(q) and k_hat as
+ *    phi(k) / ||phi(k)||.
  *
  * Layouts (all row-major, contiguous):
  *   q, k   [B, H, T, dk]      v, out [B, H, T, dv]      beta [B, H, T]
@@ -207,9 +213,11 @@ int oracle_dr_scan(const double* q, const double* k, const double* v,
                              dk, dv, mode, residual_pre_decay);
 }
 
-/* One VLA sequence. S and A are d x d, updated in place; work holds 3*d doubles. */
+/* One VLA sequence. S and A are d x d, updated in place; work holds 3*d doubles. n (d
+ * doubles) is the ratio readout's denominator state, NULL for the plain readout. */
 static void vla_sequence(const double* q, const double* k, const double* v, const double* u,
-                         double* S, double* A, double* out, double* work, long T, int d) {
+                         double* S, double* A, double* n, double* out, double* work, long T,
+                         int d) {
     double* z = work;          /* z_t = A_{t-1} u_t */
     double* y = work + d;      /* A_t k_hat_t, then alpha_hat_t */
     double* r = work + 2 * d;  /* v_t - S_{t-1} k_hat_t */
@@ -251,24 +259,37 @@ static void vla_sequence(const double* q, const double* k, const double* v, cons
         for (int i = 0; i < d; ++i)
             for (int j = 0; j < d; ++j) S[(long)i * d + j] += r[i] * y[j];
 
-        /* readout o_t = S_t q_hat_t */
+        /* ratio readout: the same write on the value 1, n_t = n + (1 - n k_hat) alpha_hat^T */
+        double nq = 1.0;
+        if (n) {
+            double nk = 0.0;
+            for (int j = 0; j < d; ++j) nk += n[j] * kt[j];
+            for (int j = 0; j < d; ++j) n[j] += (1.0 - nk) * y[j];
+            nq = 0.0;
+            for (int j = 0; j < d; ++j) nq += n[j] * qt[j];
+        }
+
+        /* readout o_t = S_t q_hat_t (divided by n_t q_t for the ratio readout) */
         for (int i = 0; i < d; ++i) {
             double acc = 0.0;
             for (int j = 0; j < d; ++j) acc += S[(long)i * d + j] * qt[j];
-            ot[i] = acc;
+            ot[i] = n ? acc / nq : acc;
         }
     }
 }
 
 /*
- * VLA Sherman-Morrison scan. S0 NULL = zeros; A0 NULL = I / lambda0.
- * S_final / A_final NULL = not written. Returns 0, or -1 on a bad argument.
+ * VLA Sherman-Morrison scan with either readout. S0 NULL = zeros; A0 NULL = I / lambda0;
+ * n0 [B,H,d] NULL = zeros (ratio readout only). S_final / A_final / n_final NULL = not
+ * written. readout 0: o_t = S_t q_t; 1: o_t = S_t q_t / (n_t q_t). Returns 0, or -1 on a
+ * bad argument.
  */
-int oracle_vla_scan(const double* q, const double* k, const double* v, const double* u,
-                    const double* S0, const double* A0, double lambda0,
-                    double* out, double* S_final, double* A_final,
-                    int B, int H, int T, int d) {
+int oracle_vla_scan_ex(const double* q, const double* k, const double* v, const double* u,
+                       const double* S0, const double* A0, const double* n0, double lambda0,
+                       double* out, double* S_final, double* A_final, double* n_final,
+                       int B, int H, int T, int d, int readout) {
     if (B < 0 || H < 0 || T < 0 || d <= 0) return -1;
+    if (readout != 0 && readout != 1) return -1;
     if (!q || !k || !v || !u || !out) return -1;
     if (!A0 && !(lambda0 > 0.0)) return -1;
     const long BH = (long)B * H;
@@ -279,7 +300,8 @@ int oracle_vla_scan(const double* q, const double* k, const double* v, const dou
         double* S = (double*)malloc(sizeof(double) * (size_t)dd);
         double* A = (double*)malloc(sizeof(double) * (size_t)dd);
         double* work = (double*)malloc(sizeof(double) * 3 * (size_t)d);
-        if (!S || !A || !work) {
+        double* n = readout ? (double*)malloc(sizeof(double) * (size_t)d) : NULL;
+        if (!S || !A || !work || (readout && !n)) {
             failed = 1;
         } else {
             if (S0) memcpy(S, S0 + bh * dd, sizeof(double) * (size_t)dd);
@@ -290,14 +312,29 @@ int oracle_vla_scan(const double* q, const double* k, const double* v, const dou
                 memset(A, 0, sizeof(double) * (size_t)dd);
                 for (int i = 0; i < d; ++i) A[(long)i * d + i] = 1.0 / lambda0;
             }
+            if (n) {
+                if (n0) memcpy(n, n0 + bh * d, sizeof(double) * (size_t)d);
+                else memset(n, 0, sizeof(double) * (size_t)d);
+            }
             const long off = bh * (long)T * d;
-            vla_sequence(q + off, k + off, v + off, u + off, S, A, out + off, work, T, d);
+            vla_sequence(q + off, k + off, v + off, u + off, S, A, n, out + off, work, T, d);
             if (S_final) memcpy(S_final + bh * dd, S, sizeof(double) * (size_t)dd);
             if (A_final) memcpy(A_final + bh * dd, A, sizeof(double) * (size_t)dd);
+            if (n && n_final) memcpy(n_final + bh * d, n, sizeof(double) * (size_t)d);
         }
         free(S);
         free(A);
         free(work);
+        free(n);
     }
     return failed ? -1 : 0;
+}
+
+/* VLA scan with the plain readout o_t = S_t q_hat_t (see oracle_vla_scan_ex). */
+int oracle_vla_scan(const double* q, const double* k, const double* v, const double* u,
+                    const double* S0, const double* A0, double lambda0,
+                    double* out, double* S_final, double* A_final,
+                    int B, int H, int T, int d) {
+    return oracle_vla_scan_ex(q, k, v, u, S0, A0, NULL, lambda0, out, S_final, A_final, NULL,
+                              B, H, T, d, 0);
 }

@@ -34,6 +34,10 @@ GDN2_PAGE = ('"Mechanisms, trade-offs and cross-layer routing of linear-attentio
              'with per-channel erase b and write w, e = b (.) kappa, z = w (.) v, residual '
              'r = z - W~ e (W~ the decayed memory), written along e')
 
+VLA_RATIO_PAGE = VLA_PAGE + ('; section 2.3: the output is a ratio of recurrences, as in linear '
+                             'attention; the denominator is the same write on a value held at 1, '
+                             'n_t = n_{t-1} + (1 - n_{t-1} k_hat) alpha_hat^T, o_t = S_t q / (n_t q)')
+
 CASES = {
     "deltanet_d2_t2": dict(
         mode=oracle.DELTANET,
@@ -95,6 +99,18 @@ CASES = {
             "r = (0,1,0) - (1,2,3) = (-1,-1,-3), S2 = S1 + r e2^T = [[1,-1,0],[2,-1,0],[3,-3,0]], "
             "o2 = S2 (0,1,1) = (-1,-1,-3)",
         ]),
+    "vla_ratio_d3_t2": dict(
+        mode="vla_ratio",
+        cite=VLA_RATIO_PAGE,
+        q=[[1, 1, 1], [3, 1, 1]], k=[[2, 1, 1], [2, 4, 2]], v=[[1, 2, 3], [0, 1, 0]],
+        u=[[1, 1, 1], [0, 0, 0]], lambda0=1.0,
+        derivation=[
+            "t=1: as vla_d3_t2, A1 = I - J/4, A1 k1 = (1,0,0), alpha_hat = e1, S1 = (1,2,3)^T e1^T; "
+            "n1 = 0 + (1 - 0) e1 = e1, n1 q1 = 1, o1 = S1 q1 / 1 = (1,2,3)",
+            "t=2: u2 = 0 leaves A2 = A1; A2 k2 = (0,2,0), alpha_hat = e2, S1 k2 = (2,4,6), "
+            "r = (-2,-3,-6), S2 = [[1,-2,0],[2,-3,0],[3,-6,0]]; n1 k2 = 2, n2 = e1 + (1-2) e2 "
+            "= (1,-1,0); S2 q2 = (1,3,3), n2 q2 = 2, o2 = (1/2,3/2,3/2)",
+        ]),
 }
 
 
@@ -105,7 +121,7 @@ def _bh(x):
 
 def build_case(name: str, spec: dict) -> dict:
     fx = {"case": name, "cite": spec["cite"], "derivation": spec["derivation"],
-          "mode": spec["mode"] if spec["mode"] == "vla" else
+          "mode": spec["mode"] if spec["mode"] in ("vla", "vla_ratio") else
           {oracle.DELTANET: "deltanet", oracle.GDN: "gdn", oracle.KDA: "kda",
            oracle.GDN2: "gdn2"}[spec["mode"]]}
     inputs = {key: spec[key] for key in ("q", "k", "v", "beta", "gate", "erase", "write", "S0",
@@ -117,6 +133,11 @@ def build_case(name: str, spec: dict) -> dict:
                                       _bh(spec["u"]), lambda0=spec["lambda0"])
         fx["expected"] = {"out": out[0, 0].tolist(), "S_final": Sf[0, 0].tolist(),
                           "A_final": Af[0, 0].tolist()}
+    elif spec["mode"] == "vla_ratio":
+        out, Sf, Af, nf = oracle.vla_scan_ratio(_bh(spec["q"]), _bh(spec["k"]), _bh(spec["v"]),
+                                                _bh(spec["u"]), lambda0=spec["lambda0"])
+        fx["expected"] = {"out": out[0, 0].tolist(), "S_final": Sf[0, 0].tolist(),
+                          "A_final": Af[0, 0].tolist(), "n_final": nf[0, 0].tolist()}
     else:
         beta = np.asarray(spec["beta"], np.float64)[None, None]
         gate = None if "gate" not in spec else _bh(spec["gate"])

@@ -21,7 +21,8 @@ import pytest
 from helpers import rel_err
 
 GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
-CASES = ["deltanet_d2_t2", "gdn_d2_t3", "kda_d2_t2", "gdn2_d2_t2", "vla_d3_t2"]
+CASES = ["deltanet_d2_t2", "gdn_d2_t3", "kda_d2_t2", "gdn2_d2_t2", "vla_d3_t2",
+         "vla_ratio_d3_t2"]
 
 # The same cases worked by hand from the per-token definitions (fractions written out).
 HAND = {
@@ -51,6 +52,12 @@ HAND = {
         "S_final": [[1, -1, 0], [2, -1, 0], [3, -3, 0]],
         "A_final": [[3 / 4, -1 / 4, -1 / 4], [-1 / 4, 3 / 4, -1 / 4], [-1 / 4, -1 / 4, 3 / 4]],
     },
+    "vla_ratio_d3_t2": {
+        "out": [[1, 2, 3], [1 / 2, 3 / 2, 3 / 2]],
+        "S_final": [[1, -2, 0], [2, -3, 0], [3, -6, 0]],
+        "A_final": [[3 / 4, -1 / 4, -1 / 4], [-1 / 4, 3 / 4, -1 / 4], [-1 / 4, -1 / 4, 3 / 4]],
+        "n_final": [1, -1, 0],
+    },
 }
 
 
@@ -69,6 +76,10 @@ def run_oracle(oracle, fx, residual_pre_decay=False):
         out, Sf, Af = oracle.vla_scan(bh(x["q"]), bh(x["k"]), bh(x["v"]), bh(x["u"]),
                                       lambda0=x["lambda0"])
         return {"out": out[0, 0], "S_final": Sf[0, 0], "A_final": Af[0, 0]}
+    if fx["mode"] == "vla_ratio":
+        out, Sf, Af, nf = oracle.vla_scan_ratio(bh(x["q"]), bh(x["k"]), bh(x["v"]), bh(x["u"]),
+                                                lambda0=x["lambda0"])
+        return {"out": out[0, 0], "S_final": Sf[0, 0], "A_final": Af[0, 0], "n_final": nf[0, 0]}
     mode = {"deltanet": oracle.DELTANET, "gdn": oracle.GDN, "kda": oracle.KDA,
             "gdn2": oracle.GDN2}[fx["mode"]]
     beta = np.asarray(x["beta"], np.float64)[None, None]
@@ -140,7 +151,7 @@ def bf16_tensor(torch, a):
 
 
 @pytest.mark.gpu
-@pytest.mark.parametrize("name", ["deltanet_d2_t2", "gdn_d2_t3", "kda_d2_t2"])
+@pytest.mark.parametrize("name", ["deltanet_d2_t2", "gdn_d2_t3", "kda_d2_t2", "gdn2_d2_t2"])
 @pytest.mark.parametrize("path", ["fp32_sequential", "bf16_chunked"])
 def test_cuda_scan_on_the_worked_examples(cuda, name, path):
     torch, drs = cuda
@@ -157,23 +168,24 @@ def test_cuda_scan_on_the_worked_examples(cuda, name, path):
     else:
         tq, tk, tv = (bf16_tensor(torch, a)[None, None].cuda() for a in (q, k, v))
     beta = torch.tensor(x["beta"], dtype=torch.float32, device="cuda")[None, None]
-    gate = None
-    if fx["mode"] == "gdn":
+    gate = erase = write = None
+    if fx["mode"] in ("gdn", "gdn2"):
         gate = torch.tensor(x["gate"], dtype=torch.float32, device="cuda")[None, None]
     elif fx["mode"] == "kda":
         gate = f32(pad(x["gate"], (T, dk), fill=1.0))
+    if fx["mode"] == "gdn2":
+        erase, write = f32(pad(x["erase"], (T, dk))), f32(pad(x["write"], (T, dv)))
     S0 = f32(pad(x["S0"], (dv, dk))) if "S0" in x else None
-    out, Sf = drs.scan(tq, tk, tv, beta, gate, S0, mode=fx["mode"],
-                       force_sequential=path == "fp32_sequential")
+    out, Sf, u = drs.scan_ex(tq, tk, tv, beta, gate, S0, mode=fx["mode"], erase=erase,
+                             write=write, force_sequential=path == "fp32_sequential")
     torch.cuda.synchronize()
-    out = out.double().cpu().numpy()[0, 0]
-    Sf = Sf.double().cpu().numpy()[0, 0]
+    out, Sf, u = (a.double().cpu().numpy()[0, 0] for a in (out, Sf, u))
     tol = 1e-4 if path == "fp32_sequential" else 2e-2
-    want_out, want_S = np.asarray(fx["expected"]["out"]), np.asarray(fx["expected"]["S_final"])
-    assert rel_err(out[:, :d], want_out) <= tol
-    assert rel_err(Sf[:d, :d], want_S) <= tol
+    for got, key in ((out[:, :d], "out"), (Sf[:d, :d], "S_final"), (u[:, :d], "u")):
+        assert rel_err(got, np.asarray(fx["expected"][key])) <= tol, key
     # zero key and value channels receive nothing from the real ones
     assert not np.any(out[:, d:]) and not np.any(Sf[d:, :]) and not np.any(Sf[:, d:])
+    assert not np.any(u[:, d:])
 
 
 @pytest.mark.gpu

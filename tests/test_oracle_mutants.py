@@ -45,6 +45,12 @@ MUTANTS = {
                                       "const double inv = 1.0;")],
     "vla_writes_along_k": [("S[(long)i * d + j] += r[i] * y[j];",
                             "S[(long)i * d + j] += r[i] * kt[j];")],
+    "vla_ratio_normalizer_along_k": [("for (int j = 0; j < d; ++j) n[j] += (1.0 - nk) * y[j];",
+                                      "for (int j = 0; j < d; ++j) n[j] += (1.0 - nk) * kt[j];")],
+    "vla_ratio_normalizer_accumulates": [
+        ("for (int j = 0; j < d; ++j) n[j] += (1.0 - nk) * y[j];",
+         "for (int j = 0; j < d; ++j) n[j] += y[j];")],
+    "vla_ratio_without_division": [("ot[i] = n ? acc / nq : acc;", "ot[i] = acc;")],
 }
 
 

@@ -440,3 +440,68 @@ def test_first_write_value_from_a_zero_state(oracle, mode):
     _, _, u = oracle.dr_scan_ex(q, k, v, beta, gate, None, mode, erase=erase, write=write)
     target = write * v if mode == GDN2 else v
     assert _rel(u[:, :, 0], beta[:, :, 0, None] * target[:, :, 0]) < 1e-15
+
+
+# ====================================================================================
+# VLA ratio readout. VLA page, section 2.3: the output is computed as a ratio of
+# recurrences, as in standard linear attention, with an ELU+1 feature map. Reading taken:
+# the denominator is the same write applied to one more value channel held at 1,
+# n_t = n_{t-1} + (1 - n_{t-1} k_t) alpha_hat_t^T, and o_t = S_t q_t / (n_t q_t), with q
+# the feature-mapped query and k the unit-norm feature-mapped key (the caller's feature map).
+# ====================================================================================
+def _elu1(x):
+    return np.where(x > 0, x + 1.0, np.exp(x))
+
+
+def test_vla_ratio_with_basis_keys_is_normalised_linear_attention(oracle):
+    # u = 0 keeps A = I / lambda0, so alpha_hat = k; with distinct basis keys every write
+    # lands in a fresh direction: S_t = sum_{s<=t} v_s k_s^T and n_t = sum_{s<=t} k_s^T, and
+    # the ratio readout is causal linear attention normalised by its own weights (brute force)
+    rng = np.random.default_rng(60)
+    B, H, d = 1, 3, 8
+    T = d
+    k = np.zeros((B, H, T, d))
+    for h in range(H):
+        k[0, h, np.arange(T), rng.permutation(d)] = 1.0
+    q = _elu1(rng.standard_normal((B, H, T, d)))
+    v = rng.standard_normal((B, H, T, d))
+    out, _, _, nf = oracle.vla_scan_ratio(q, k, v, np.zeros_like(v), lambda0=2.0)
+    w = np.einsum("bhtd,bhsd->bhts", q, k) * np.tril(np.ones((T, T)))
+    ref = np.einsum("bhts,bhsv->bhtv", w, v) / w.sum(-1, keepdims=True)
+    assert _rel(out, ref) < 1e-13
+    assert _rel(nf, k.sum(2)) < 1e-15
+
+
+def test_vla_ratio_reads_back_a_constant_value(oracle):
+    # when every value is the same vector c (and S0 = c n0^T), S and n follow one recurrence,
+    # S_t = c n_t, so every output is exactly c, whatever u, k and q
+    rng = np.random.default_rng(61)
+    B, H, T, d = 2, 2, 40, 6
+    q = _elu1(rng.standard_normal((B, H, T, d)))
+    k = _unit(_elu1(rng.standard_normal((B, H, T, d))))
+    u = rng.standard_normal((B, H, T, d)) / np.sqrt(d)
+    c = rng.standard_normal((B, H, d))
+    v = np.broadcast_to(c[:, :, None, :], (B, H, T, d)).copy()
+    n0 = np.abs(rng.standard_normal((B, H, d)))
+    S0 = np.einsum("bhi,bhj->bhij", c, n0)
+    out, Sf, _, nf = oracle.vla_scan_ratio(q, k, v, u, S0=S0, n0=n0)
+    assert _rel(out, v) < 1e-10
+    assert _rel(Sf, np.einsum("bhi,bhj->bhij", c, nf)) < 1e-10
+
+
+def test_vla_ratio_numerator_is_the_plain_readout(oracle):
+    # S and A follow the same recurrence under either readout; the ratio output times the
+    # denominator n_t q_t is the plain readout S_t q_t
+    rng = np.random.default_rng(62)
+    B, H, T, d = 1, 2, 30, 5
+    q = _elu1(rng.standard_normal((B, H, T, d)))
+    k = _unit(_elu1(rng.standard_normal((B, H, T, d))))
+    v = rng.standard_normal((B, H, T, d))
+    u = rng.standard_normal((B, H, T, d)) / np.sqrt(d)
+    plain, S1, A1 = oracle.vla_scan(q, k, v, u)
+    ratio, S2, A2, _ = oracle.vla_scan_ratio(q, k, v, u)
+    assert np.array_equal(S1, S2) and np.array_equal(A1, A2)
+    # scaling q by a positive number leaves the ratio unchanged but scales the plain readout
+    ratio3, _, _, _ = oracle.vla_scan_ratio(3.0 * q, k, v, u)
+    assert _rel(ratio3, ratio) < 1e-12
+    assert _rel(plain / ratio, np.broadcast_to((plain / ratio)[..., :1], plain.shape)) < 1e-9
