@@ -52,6 +52,8 @@ def _load():
         lib.oracle_vla_scan_ex.argtypes = ([dp] * 7 + [ctypes.c_double] + [dp] * 4
                                            + [ctypes.c_int] * 5)
         lib.oracle_vla_scan_ex.restype = ctypes.c_int
+        lib.oracle_loglinear_scan.argtypes = [dp] * 5 + [ctypes.c_int] * 6
+        lib.oracle_loglinear_scan.restype = ctypes.c_int
         lib.oracle_num_threads.argtypes = []
         lib.oracle_num_threads.restype = ctypes.c_int
         _lib = lib
@@ -204,3 +206,26 @@ def vla_scan_ratio(q, k, v, u, S0=None, A0=None, n0=None, lambda0=1.0):
     if rc != 0:
         raise RuntimeError(f"oracle_vla_scan_ex failed ({rc})")
     return out, Sf, Af, nf
+
+
+def loglinear_levels(T: int) -> int:
+    """Levels a log-linear scan of T tokens needs: level 0 plus one per bit of T - 1."""
+    return max(1, int(T - 1).bit_length() + 1)
+
+
+def loglinear_scan(q, k, v, lam):
+    """Log-linear attention over a Fenwick hierarchy of linear-attention memories, fp64,
+    one token at a time (binary-counter form). q, k: [B,H,T,dk]; v: [B,H,T,dv];
+    lam: [B,H,T,L] level weights (L >= loglinear_levels(T)). Returns out [B,H,T,dv]."""
+    q, k, v, lam = _f64(q), _f64(k), _f64(v), _f64(lam)
+    B, H, T, dk = q.shape
+    dv = v.shape[-1]
+    L = lam.shape[-1]
+    if k.shape != q.shape or v.shape[:3] != (B, H, T) or lam.shape[:3] != (B, H, T):
+        raise ValueError("shape mismatch")
+    out = np.empty((B, H, T, dv), np.float64)
+    rc = _load().oracle_loglinear_scan(_ptr(q), _ptr(k), _ptr(v), _ptr(lam), _ptr(out), B, H, T,
+                                       dk, dv, L)
+    if rc != 0:
+        raise RuntimeError(f"oracle_loglinear_scan failed ({rc})")
+    return out

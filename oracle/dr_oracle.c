@@ -10,7 +10,8 @@
  * in fp64, independently for every (batch, head) sequence. There is no chunking,
  * blocking, fusion or reordering.
  *
- * Sources (the three web pages this subject is drawn from):
+ * Sources (the three web pages this subject is drawn from; the log-linear scan at the end
+ * of this file follows the third, "Adaptive memory decay for log-linear attention"):
  *  - "Mechanisms, trade-offs and cross-layer routing of linear-attention
  *    architectures" (aitrends.kr), section "Technical details" (기술 상세) and
  *    "Understanding the key idea": memory W in R^{d_v x d_phi}, readout y = W phi(q);
@@ -337,4 +338,89 @@ int oracle_vla_scan(const double* q, const double* k, const double* v, const dou
                     int B, int H, int T, int d) {
     return oracle_vla_scan_ex(q, k, v, u, S0, A0, NULL, lambda0, out, S_final, A_final, NULL,
                               B, H, T, d, 0);
+}
+
+/*
+ * Log-linear attention ("Adaptive memory decay for log-linear attention", problem definition
+ * and method sections): the memory is a Fenwick-tree hierarchy, the state grows as O(log T),
+ * and each output is a weighted sum of memory levels with weights lambda_t^(l).
+ *
+ * Reading taken (plain linear-attention memories, no decay or delta rule inside a level):
+ * at step t (0-based) the prefix [0, t] is split into level 0 = {t} and, for every set bit b
+ * of t, level b + 1 = the 2^b tokens before the block of every lower set bit (the Fenwick
+ * decomposition of the prefix), and
+ *     o_t = lambda_t^(0) (v_t k_t^T) q_t + sum_{b : bit b of t} lambda_t^(b+1) M_b q_t,
+ * M_b = sum of v_s k_s^T over level b+1's tokens. The levels are kept as a binary counter:
+ * after token t, with j = the number of trailing ones of t, M_j = v_t k_t^T + sum_{b<j} M_b
+ * and M_b = 0 for b < j (the blocks of the next step). lambda is [B,H,T,L] with
+ * L >= bits(T-1) + 1 levels (level l at index l).
+ */
+static void loglinear_sequence(const double* q, const double* k, const double* v,
+                               const double* lam, double* M, double* cur, double* out,
+                               long T, int dk, int dv, int L) {
+    const long state = (long)dv * dk;
+    memset(M, 0, sizeof(double) * (size_t)state * (size_t)(L > 1 ? L - 1 : 1));
+    for (long t = 0; t < T; ++t) {
+        const double* kt = k + t * dk;
+        const double* qt = q + t * dk;
+        const double* vt = v + t * dv;
+        const double* lt = lam + t * L;
+        double* ot = out + t * dv;
+        for (int i = 0; i < dv; ++i)
+            for (int j = 0; j < dk; ++j) cur[(long)i * dk + j] = vt[i] * kt[j];
+        for (int i = 0; i < dv; ++i) {
+            double acc = 0.0;
+            for (int j = 0; j < dk; ++j) acc += cur[(long)i * dk + j] * qt[j];
+            acc *= lt[0];
+            for (int b = 0; b + 1 < L; ++b) {
+                if (!((t >> b) & 1)) continue;
+                double lev = 0.0;
+                for (int j = 0; j < dk; ++j) lev += M[b * state + (long)i * dk + j] * qt[j];
+                acc += lt[b + 1] * lev;
+            }
+            ot[i] = acc;
+        }
+        /* advance the binary counter to t + 1 */
+        int jt = 0;
+        while ((t >> jt) & 1) ++jt;
+        if (jt + 1 < L) {
+            double* Mj = M + jt * state;
+            for (long e = 0; e < state; ++e) {
+                double x = cur[e];
+                for (int b = 0; b < jt; ++b) x += M[b * state + e];
+                Mj[e] = x;
+            }
+            for (int b = 0; b < jt; ++b) memset(M + b * state, 0, sizeof(double) * (size_t)state);
+        }
+    }
+}
+
+/*
+ * Log-linear attention scan: q, k [B,H,T,dk], v [B,H,T,dv], lambda [B,H,T,L] (weights of
+ * levels 0..L-1), out [B,H,T,dv]. L must cover every position: T <= 2^(L-1). Returns 0, or
+ * -1 on a bad argument.
+ */
+int oracle_loglinear_scan(const double* q, const double* k, const double* v, const double* lam,
+                          double* out, int B, int H, int T, int dk, int dv, int L) {
+    if (B < 0 || H < 0 || T < 0 || dk <= 0 || dv <= 0 || L < 1 || L > 40) return -1;
+    if (T > 1 && (long)(T - 1) >> (L - 1)) return -1;
+    if (!q || !k || !v || !lam || !out) return -1;
+    const long BH = (long)B * H;
+    const long state = (long)dv * dk;
+    int failed = 0;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (long bh = 0; bh < BH; ++bh) {
+        double* M = (double*)malloc(sizeof(double) * (size_t)state * (size_t)(L > 1 ? L - 1 : 1));
+        double* cur = (double*)malloc(sizeof(double) * (size_t)state);
+        if (!M || !cur) {
+            failed = 1;
+        } else {
+            loglinear_sequence(q + bh * (long)T * dk, k + bh * (long)T * dk,
+                               v + bh * (long)T * dv, lam + bh * (long)T * L,
+                               M, cur, out + bh * (long)T * dv, T, dk, dv, L);
+        }
+        free(M);
+        free(cur);
+    }
+    return failed ? -1 : 0;
 }

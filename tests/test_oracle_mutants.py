@@ -51,6 +51,12 @@ MUTANTS = {
         ("for (int j = 0; j < d; ++j) n[j] += (1.0 - nk) * y[j];",
          "for (int j = 0; j < d; ++j) n[j] += y[j];")],
     "vla_ratio_without_division": [("ot[i] = n ? acc / nq : acc;", "ot[i] = acc;")],
+    "loglinear_merge_drops_lower_levels": [("for (int b = 0; b < jt; ++b) x += M[b * state + e];",
+                                            "for (int b = 0; b < 0; ++b) x += M[b * state + e];")],
+    "loglinear_level_weights_shifted": [("acc += lt[b + 1] * lev;", "acc += lt[b] * lev;")],
+    "loglinear_counter_on_trailing_zeros": [("while ((t >> jt) & 1) ++jt;",
+                                             "while (jt < 30 && !((t >> jt) & 1)) ++jt;")],
+    "loglinear_without_own_token": [("acc *= lt[0];", "acc *= 0.0;")],
 }
 
 

@@ -505,3 +505,94 @@ def test_vla_ratio_numerator_is_the_plain_readout(oracle):
     ratio3, _, _, _ = oracle.vla_scan_ratio(3.0 * q, k, v, u)
     assert _rel(ratio3, ratio) < 1e-12
     assert _rel(plain / ratio, np.broadcast_to((plain / ratio)[..., :1], plain.shape)) < 1e-9
+
+
+# ====================================================================================
+# Log-linear attention over a Fenwick hierarchy ("Adaptive memory decay for log-linear
+# attention", problem definition and method sections): the prefix [0, t] is split into the
+# token itself (level 0) and one block of 2^b earlier tokens per set bit b of t (level b + 1);
+# the output is the lambda_t-weighted sum of the levels' linear-attention readouts. The
+# oracle keeps the levels as a binary counter; these pins compare it with the pair-wise
+# masked form, whose level of (t, s < t) is the bit length of t XOR s.
+# ====================================================================================
+def _loglinear_inputs(rng, B, H, T, dk, dv):
+    q = rng.standard_normal((B, H, T, dk))
+    k = rng.standard_normal((B, H, T, dk))
+    v = rng.standard_normal((B, H, T, dv))
+    L = oracle_levels(T)
+    lam = np.log1p(np.exp(0.54 + 0.5 * rng.standard_normal((B, H, T, L))))  # softplus
+    return q, k, v, lam
+
+
+def oracle_levels(T):
+    return max(1, int(T - 1).bit_length() + 1)
+
+
+@pytest.mark.parametrize("T", [1, 2, 7, 64, 100])
+def test_loglinear_matches_the_masked_pairwise_form(oracle, T):
+    rng = np.random.default_rng(70 + T)
+    B, H, dk, dv = 1, 2, 5, 3
+    q, k, v, lam = _loglinear_inputs(rng, B, H, T, dk, dv)
+    assert oracle.loglinear_levels(T) == lam.shape[-1]
+    out = oracle.loglinear_scan(q, k, v, lam)
+    t = np.arange(T)[:, None]
+    s = np.arange(T)[None, :]
+    level = np.vectorize(lambda a, b: int(a ^ b).bit_length())(t, s)  # 0 on the diagonal
+    weight = np.take_along_axis(lam, np.broadcast_to(level, (B, H, T, T)), axis=-1)
+    weight = weight * (s <= t)
+    ref = np.einsum("bhts,bhsv->bhtv", weight * np.einsum("bhtd,bhsd->bhts", q, k), v)
+    assert _rel(out, ref) < 1e-12
+
+
+def test_loglinear_with_unit_weights_is_linear_attention(oracle):
+    # lambda = 1 on every level: the levels partition the prefix, so the scan is causal
+    # linear attention (and the oracle's plain accumulation from a zero state)
+    rng = np.random.default_rng(75)
+    B, H, T, dk, dv = 2, 2, 45, 4, 6
+    q, k, v, lam = _loglinear_inputs(rng, B, H, T, dk, dv)
+    out = oracle.loglinear_scan(q, k, v, np.ones_like(lam))
+    ref = np.einsum("bhts,bhsv->bhtv", np.einsum("bhtd,bhsd->bhts", q, k) * np.tril(np.ones((T, T))), v)
+    assert _rel(out, ref) < 1e-12
+    lin, _ = oracle.dr_scan(q, k, v, mode=LINEAR)
+    assert _rel(out, lin) < 1e-12
+
+
+@pytest.mark.parametrize("level", [0, 1, 2, 3, 5])
+def test_loglinear_one_level_reads_one_fenwick_block(oracle, level):
+    # weights on one level only: level 0 is the token itself; level b + 1 is the block
+    # [hi 2^(b+1), hi 2^(b+1) + 2^b) with hi = t >> (b+1), present when bit b of t is set
+    rng = np.random.default_rng(80 + level)
+    B, H, T, dk, dv = 1, 1, 50, 3, 2
+    q, k, v, lam = _loglinear_inputs(rng, B, H, T, dk, dv)
+    one = np.zeros_like(lam)
+    one[..., level] = 1.0
+    out = oracle.loglinear_scan(q, k, v, one)
+    ref = np.zeros_like(out)
+    for t in range(T):
+        if level == 0:
+            block = [t]
+        else:
+            b = level - 1
+            if not (t >> b) & 1:
+                continue
+            lo = (t >> (b + 1)) << (b + 1)
+            block = list(range(lo, lo + (1 << b)))
+            assert all(s < t for s in block)
+        for s in block:
+            ref[:, :, t] += (q[:, :, t] * k[:, :, s]).sum(-1)[..., None] * v[:, :, s]
+    assert _rel(out, ref) < 1e-12 if np.any(ref) else np.max(np.abs(out)) == 0.0
+
+
+def test_loglinear_worked_example(oracle):
+    # d = 1, T = 4, lambda_t = (1, 1/2, 1/4) for levels 0, 1, 2:
+    # t=0: {0} -> 1 (q0 k0) v0 = 2
+    # t=1 (01): {1} + level 1 {0} -> (2*1)*2 + 1/2 (2*2)*1 = 6
+    # t=2 (10): {2} + level 2 {0,1} -> (1*1)*4 + 1/4 ((1*2)*1 + (1*1)*2) = 5
+    # t=3 (11): {3} + level 1 {2} + level 2 {0,1} -> (1/2*2)*8 + 1/2 (1/2*1)*4
+    #           + 1/4 ((1/2*2)*1 + (1/2*1)*2) = 9.5
+    q = np.array([1, 2, 1, 0.5])[None, None, :, None]
+    k = np.array([2, 1, 1, 2])[None, None, :, None]
+    v = np.array([1, 2, 4, 8])[None, None, :, None]
+    lam = np.broadcast_to(np.array([1, 0.5, 0.25]), (1, 1, 4, 3))
+    out = oracle.loglinear_scan(q, k, v, lam)
+    assert np.array_equal(out[0, 0, :, 0], [2, 6, 5, 9.5])
