@@ -1,12 +1,16 @@
 """Benchmark of the forward delta-rule scan on B200: head-tokens/s and roofline fraction.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+                    [--no-per-config]
 
 One step = one dr_scan_fwd call over the whole workload (all B*H sequences, all T tokens),
 inputs resident in HBM. Under torchrun each rank runs the same workload on its own GPU
 (independent sequences, no collective on the data path: weak scaling); the time is the
 max over ranks and `value` counts the head-tokens all ranks processed.
-Rank 0 prints ONE JSON line.
+Rank 0 prints ONE JSON line. The headline workload is the largest single-GPU configuration
+(KDA, B8 H16 T4096); on one GPU the line also carries every other configuration (the small
+fp32 DeltaNet case, Gated DeltaNet, the long-context sweep, VLA, Gated DeltaNet-2 and the
+decode step) under "per_config", each with its own roofline, e2e and cpu_baseline.
 """
 from __future__ import annotations
 
@@ -29,6 +33,13 @@ METRIC = ("scan fwd tokens/s per B200 (B·H·T/time) and % of roofline "
 UNIT = "tokens/s"
 L2_BYTES = 126 * 1024 * 1024
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+# the largest single-GPU configuration (524,288 head-tokens, 816 MB of algorithmic traffic)
+DEFAULT_WORKLOAD = "kda_bf16"
+# every configuration, in the order the per_config object lists them
+PER_CONFIG = ["deltanet_fp32", "gdn_bf16", "kda_bf16", "gdn_long_t4096", "gdn_long_t8192",
+              "gdn_long_t16384", "gdn_long_t32768", "vla_fp32_d32", "vla_fp32_d96",
+              "vla_ratio_fp32_d32", "vla_ratio_fp32_d96", "gdn2_bf16", "loglinear_bf16",
+              "gdn_decode_bf16"]
 
 
 def parse_args(argv=None):
@@ -36,10 +47,13 @@ def parse_args(argv=None):
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=2000)
     p.add_argument("--warmup", type=int, default=20)
-    p.add_argument("--workload", default="gdn_bf16")
+    p.add_argument("--workload", default=DEFAULT_WORKLOAD)
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--e2e-steps", type=int, default=20)
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-per-config", action="store_true")
+    p.add_argument("--per-config-steps", type=int, default=0,
+                   help="timed steps per extra configuration (0: --steps)")
     return p.parse_args(argv)
 
 
@@ -54,15 +68,19 @@ def algorithmic_bytes(w, with_state_in=None, with_state_out=True) -> int:
 
     if isinstance(w, wl.VLAWorkload):
         return w.B * w.H * (w.T * 5 * w.d * 4 + (2 * w.d * w.d * 4 if with_state_out else 0))
+    if isinstance(w, wl.LogLinearWorkload):  # q, k, v in and out (bf16), lambda in (fp32)
+        return w.B * w.H * w.T * ((2 * w.dk + 2 * w.dv) * 2 + w.levels * 4)
     isz = 2 if w.dtype == "bf16" else 4
     BH, T = w.B * w.H, w.T
     per_head = T * (2 * w.dk + 2 * w.dv) * isz
     if w.mode != wl.LINEAR:
         per_head += T * 4
-    if w.mode == wl.GDN:
+    if w.mode in (wl.GDN, wl.GDN2):
         per_head += T * 4
     elif w.mode == wl.KDA:
         per_head += T * w.dk * 4
+    if w.mode == wl.GDN2:
+        per_head += T * (w.dk + w.dv) * 4  # erase and write gates
     state = w.dv * w.dk * 4
     if with_state_in if with_state_in is not None else w.s0_std > 0:
         per_head += state
@@ -79,6 +97,14 @@ def algorithmic_flops(w) -> int:
 
     if isinstance(w, wl.VLAWorkload):
         return w.B * w.H * w.T * 12 * w.d * w.d
+    if isinstance(w, wl.LogLinearWorkload):
+        # per chunk of 64: Q K^T and P V halves, the chunk state V^T K, and one readout
+        # Q M_b^T per set bit of the chunk index (on average half the chunk-index bits)
+        C = 64
+        nch = -(-w.T // C)
+        bits = sum(bin(c).count("1") for c in range(nch)) / nch
+        per_token = C * w.dk + C * w.dv + 2 * w.dk * w.dv + bits * 2 * w.dk * w.dv
+        return int(w.B * w.H * w.T * per_token)
     C = 64
     per_token = 6 * w.dk * w.dv + C * (3 * w.dk + 2 * w.dv) + C * C // 3
     return w.B * w.H * w.T * per_token
@@ -93,8 +119,10 @@ def workload_config(w, world: int, nsets: int = 0, nbytes: int = 0) -> dict:
         cfg.update({"dk": w.dk, "dv": w.dv, "mode": wl.MODE_NAMES[w.mode]})
         if not w.decode:
             cfg["chunk"] = 64
+    elif isinstance(w, wl.LogLinearWorkload):
+        cfg.update({"dk": w.dk, "dv": w.dv, "mode": "loglinear", "levels": w.levels, "chunk": 64})
     else:
-        cfg.update({"d": w.d, "mode": "vla"})
+        cfg.update({"d": w.d, "mode": "vla_ratio" if w.ratio else "vla"})
     cfg["parallelism"] = f"replicas{world}" if world > 1 else "1gpu"
     if nsets:
         cfg["l2"] = (f"rotating {nsets} resident input sets ({nsets * nbytes / 2**20:.0f} MiB)"
@@ -227,7 +255,7 @@ def oracle_sample(inputs, heads, T):
     from delta_rule_recurrent_chunked_b200 import workloads as wl
 
     sub = wl.head_slice(inputs, heads)
-    for key in ("q", "k", "v", "beta", "gate", "u"):
+    for key in ("q", "k", "v", "beta", "gate", "u", "erase", "write", "lam"):
         if sub.get(key) is not None:
             sub[key] = np.ascontiguousarray(sub[key][:, :, :T])
     return sub
@@ -238,8 +266,15 @@ def run_oracle(sub):
     from delta_rule_recurrent_chunked_b200 import workloads as wl
 
     w = sub["workload"]
-    if isinstance(w, wl.VLAWorkload):
+    if isinstance(w, wl.VLAWorkload) and w.ratio:
+        oracle.vla_scan_ratio(sub["q"], sub["k"], sub["v"], sub["u"], lambda0=w.lambda0)
+    elif isinstance(w, wl.VLAWorkload):
         oracle.vla_scan(sub["q"], sub["k"], sub["v"], sub["u"], lambda0=w.lambda0)
+    elif isinstance(w, wl.LogLinearWorkload):
+        oracle.loglinear_scan(sub["q"], sub["k"], sub["v"], sub["lam"])
+    elif w.mode == wl.GDN2:
+        oracle.dr_scan_ex(sub["q"], sub["k"], sub["v"], sub["beta"], sub["gate"], sub["S0"],
+                          w.mode, erase=sub["erase"], write=sub["write"])
     else:
         oracle.dr_scan(sub["q"], sub["k"], sub["v"], sub["beta"], sub["gate"], sub["S0"], w.mode)
 
@@ -288,52 +323,35 @@ def make_device_inputs(inputs, device):
         t = torch.from_numpy(np.ascontiguousarray(raw).view(np.int16)).view(torch.bfloat16) \
             if w.dtype == "bf16" else torch.from_numpy(np.ascontiguousarray(raw))
         dev[name] = t.to(device)
-    for name in ("beta", "gate", "S0"):
+    for name in ("beta", "gate", "S0", "erase", "write"):
         arr = inputs.get(name)
         dev[name] = None if arr is None else torch.from_numpy(np.ascontiguousarray(arr)).to(device)
     return dev
 
 
-def run_ours(args, world, rank, local):
+def rotation(nbytes: int):
+    """(input sets to rotate over, whether an L2 flush is needed between timed steps): enough
+    resident copies that a set is evicted before it comes round again (>= 3x the 126 MiB L2
+    across the rotation, at most 4 copies); workloads too small for that flush L2 instead."""
+    nsets = max(1, min(4, -(-3 * L2_BYTES // max(nbytes, 1))))
+    return nsets, nsets * nbytes < 2 * L2_BYTES
+
+
+def l2_note(nsets: int, nbytes: int, flush: bool) -> str:
+    if flush:
+        return ("L2 flushed between timed steps (256 MiB write outside the timed launches); "
+                "value from the summed launch times")
+    return (f"rotating {nsets} resident input sets ({nsets * nbytes / 2**20:.0f} MiB)"
+            " > 126 MiB L2")
+
+
+def timed_loop(step, K, device, stream, local, flush=None):
+    """Time K steps with CUDA events on `stream` (warm-up done by the caller), NVML clocks
+    sampled meanwhile. With `flush` (a callable that writes more than L2), the flush runs
+    between timed steps, outside the events, and the total is the sum of the launch times.
+    Returns (total_ms, per-launch ms list, clocks, wall seconds)."""
     import torch
-    import torch.distributed as dist
 
-    import delta_rule_recurrent_chunked_b200 as drs
-    from delta_rule_recurrent_chunked_b200 import workloads as wl
-
-    device = torch.device("cuda", local)
-    torch.cuda.set_device(device)
-    if world > 1:
-        from datetime import timedelta
-
-        dist.init_process_group("nccl", device_id=device, timeout=timedelta(seconds=120))
-
-    w = wl.workload(args.workload)
-    if isinstance(w, wl.VLAWorkload):
-        return run_ours_vla(args, world, rank, local, w, device)
-    if w.decode:
-        return run_ours_decode(args, world, rank, local, w, device)
-    inputs = wl.generate_dr(w, seed=rank)
-    mode = {wl.LINEAR: "linear", wl.DELTANET: "deltanet", wl.GDN: "gdn", wl.KDA: "kda"}[w.mode]
-    nbytes = algorithmic_bytes(w)
-    nsets = max(1, min(4, -(-3 * L2_BYTES // max(nbytes, 1))))  # >= 3x L2 across the rotation
-    sets = [make_device_inputs(inputs, device) for _ in range(nsets)]
-    outs = [torch.empty_like(s["v"]) for s in sets]
-    Sfs = [torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device=device) for _ in sets]
-
-    def step(i):
-        s = sets[i % nsets]
-        drs.scan(s["q"], s["k"], s["v"], s["beta"], s["gate"], s["S0"], mode=mode,
-                 out=outs[i % nsets], S_final=Sfs[i % nsets])
-
-    stream = torch.cuda.current_stream(device)
-    for i in range(max(3, args.warmup)):
-        step(i)
-    torch.cuda.synchronize(device)
-    if drs.poll_error(device) != 0:
-        raise RuntimeError("device status set during warm-up")
-
-    K = args.steps
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
     clocks = ClockSampler(local)
@@ -342,6 +360,8 @@ def run_ours(args, world, rank, local):
     clocks.start()
     t_wall = time.perf_counter()
     for i in range(K):
+        if flush is not None:
+            flush()
         starts[i].record(stream)
         step(i)
         ends[i].record(stream)
@@ -349,51 +369,20 @@ def run_ours(args, world, rank, local):
     t_wall = time.perf_counter() - t_wall
     barrier(device)
     clk = clocks.stop()
-    total_ms = starts[0].elapsed_time(ends[-1])
     per_launch = [starts[i].elapsed_time(ends[i]) for i in range(K)]
-    status = drs.poll_error(device)
-    if status != 0:
-        raise RuntimeError(f"device status {status} after the timed region")
+    total = sum(per_launch) if flush is not None else starts[0].elapsed_time(ends[-1])
+    return total, per_launch, clk, t_wall
 
-    total_ms_max = max_over_ranks(total_ms, device=device)
-    value = aggregate_value(world, w.head_tokens, K, total_ms_max)
-    launch_ms = statistics.mean(per_launch)
 
-    # end to end through the C ABI with host buffers: pinned H2D, scan, D2H of the results
-    e2e = run_e2e(args, w, inputs, mode, device, stream)
-    e2e_ms = max_over_ranks(e2e["ms"], device=device)  # slowest rank
+def make_flush(device):
+    import torch
 
-    peaks, peak_src = load_peaks()
-    achieved = nbytes / (launch_ms / 1e3) / 1e9
-    flops = algorithmic_flops(w)
-    tflops = flops / (launch_ms / 1e3) / 1e12
-    line = {
-        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K,
-        "warmup": max(3, args.warmup), "ms_per_step": total_ms_max / K,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": w.dtype,
-        "data": "synthetic",
-        "config": dict(workload_config(w, world, nsets, nbytes),
-                       kernel="chunked" if drs.chunked_applies(mode, w.dtype == "bf16", w.dk, w.dv)
-                       else "sequential"),
-        "clocks": {k: clk[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
-        "e2e": {"value": world * w.head_tokens / (e2e_ms / 1e3), "unit": UNIT,
-                "h2d_bytes_per_step": e2e["h2d"], "d2h_bytes_per_step": e2e["d2h"]},
-        "gpu_launches": K,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"],
-                     "traffic": NCU_TRAFFIC.get((w.name, kernel_source_sha())),
-                     "peak_source": f"{peak_src} hbm_gbs", "bytes_per_launch": nbytes,
-                     "launch_ms": launch_ms,
-                     "tensor_tflops": tflops,
-                     "tensor_frac": tflops / peaks["bf16_tflops"]},
-        "wall_s": t_wall,
-    }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(inputs)
-    if world > 1:
-        dist.destroy_process_group()
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+    buf = torch.empty(256 * 2**20 // 4, dtype=torch.float32, device=device)
+
+    def flush():
+        buf.fill_(1.0)
+
+    return flush
 
 
 def fp32_alu_peak_tflops(device) -> float:
@@ -415,25 +404,48 @@ def fp32_alu_peak_tflops(device) -> float:
     return props.multi_processor_count * 128 * 2 * mhz * 1e6 / 1e12
 
 
-def run_ours_vla(args, world, rank, local, w, device):
-    """The VLA Sherman-Morrison scan (fp32, sequential per-token kernel) through vla_scan_fwd;
-    a per-token latency-bound path, reported against the FP32 ALU peak."""
+def base_line(args, w, world, K, total_ms_max, clk, e2e_ms, e2e_h2d, e2e_d2h, config, dtype,
+              t_wall):
+    return {
+        "metric": METRIC, "value": aggregate_value(world, w.head_tokens, K, total_ms_max),
+        "unit": UNIT, "n_gpus": world, "steps": K, "warmup": max(3, args.warmup),
+        "ms_per_step": total_ms_max / K, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": dtype, "data": "synthetic", "config": config,
+        "clocks": {k: clk[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
+        "e2e": {"value": world * w.head_tokens / (e2e_ms / 1e3), "unit": UNIT,
+                "h2d_bytes_per_step": e2e_h2d, "d2h_bytes_per_step": e2e_d2h},
+        "gpu_launches": K,
+        "wall_s": t_wall,
+    }
+
+
+def measure_dr(args, w, world, rank, local, device, K, cpu_target):
+    """The delta-rule scan (dr_scan_fwd; Gated DeltaNet-2 through dr_scan_fwd_ex) on one
+    workload: device-timed steps on resident inputs, e2e through the C ABI with host
+    buffers, the roofline of the launch and the oracle on the host cores."""
     import torch
-    import torch.distributed as dist
 
     import delta_rule_recurrent_chunked_b200 as drs
     from delta_rule_recurrent_chunked_b200 import workloads as wl
 
-    inputs = wl.generate_vla(w, seed=rank)
+    inputs = wl.generate_dr(w, seed=rank)
+    mode = wl.MODE_NAMES[w.mode]
     nbytes = algorithmic_bytes(w)
-    nsets = max(1, min(4, -(-3 * L2_BYTES // max(nbytes, 1))))
-    sets = [{k: torch.from_numpy(np.ascontiguousarray(inputs[k])).to(device)
-             for k in ("q", "k", "v", "u")} for _ in range(nsets)]
+    nsets, needs_flush = rotation(nbytes)
+    flush = make_flush(device) if needs_flush else None
+    sets = [make_device_inputs(inputs, device) for _ in range(nsets)]
     outs = [torch.empty_like(st["v"]) for st in sets]
+    Sfs = [torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device=device) for _ in sets]
 
     def step(i):
         st = sets[i % nsets]
-        drs.vla_scan(st["q"], st["k"], st["v"], st["u"], lambda0=w.lambda0, out=outs[i % nsets])
+        if w.mode == wl.GDN2:
+            drs.scan_ex(st["q"], st["k"], st["v"], st["beta"], st["gate"], st["S0"], mode=mode,
+                        erase=st["erase"], write=st["write"], want_u=False,
+                        out=outs[i % nsets], S_final=Sfs[i % nsets])
+        else:
+            drs.scan(st["q"], st["k"], st["v"], st["beta"], st["gate"], st["S0"], mode=mode,
+                     out=outs[i % nsets], S_final=Sfs[i % nsets])
 
     stream = torch.cuda.current_stream(device)
     for i in range(max(3, args.warmup)):
@@ -441,27 +453,74 @@ def run_ours_vla(args, world, rank, local, w, device):
     torch.cuda.synchronize(device)
     if drs.poll_error(device) != 0:
         raise RuntimeError("device status set during warm-up")
-    K = args.steps
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    clocks = ClockSampler(local)
-    barrier(device)
-    torch.cuda.synchronize(device)
-    clocks.start()
-    t_wall = time.perf_counter()
-    for i in range(K):
-        starts[i].record(stream)
+    total_ms, per_launch, clk, t_wall = timed_loop(step, K, device, stream, local, flush)
+    status = drs.poll_error(device)
+    if status != 0:
+        raise RuntimeError(f"device status {status} after the timed region")
+    total_ms_max = max_over_ranks(total_ms, device=device)
+    launch_ms = statistics.mean(per_launch)
+    del sets, outs, Sfs
+
+    e2e = run_e2e(args, w, inputs, mode, device, stream)
+    e2e_ms = max_over_ranks(e2e["ms"], device=device)
+
+    peaks, peak_src = load_peaks()
+    achieved = nbytes / (launch_ms / 1e3) / 1e9
+    tflops = algorithmic_flops(w) / (launch_ms / 1e3) / 1e12
+    chunked = drs.chunked_applies(mode, w.dtype == "bf16", w.dk, w.dv)
+    config = dict(workload_config(w, world), l2=l2_note(nsets, nbytes, needs_flush),
+                  kernel="chunked" if chunked else "sequential")
+    line = base_line(args, w, world, K, total_ms_max, clk, e2e_ms, e2e["h2d"], e2e["d2h"], config,
+                     w.dtype, t_wall)
+    line["roofline"] = {
+        "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+        "frac": achieved / peaks["hbm_gbs"],
+        "traffic": NCU_TRAFFIC.get((w.name, kernel_source_sha())) if chunked else None,
+        "peak_source": f"{peak_src} hbm_gbs", "bytes_per_launch": nbytes,
+        "launch_ms": launch_ms, "tensor_tflops": tflops,
+        "tensor_frac": tflops / peaks["bf16_tflops"]}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(inputs, cpu_target)
+    return line
+
+
+def measure_vla(args, w, world, rank, local, device, K, cpu_target):
+    """The VLA Sherman-Morrison scan (fp32) through vla_scan_fwd; a per-token latency-bound
+    path, reported against the FP32 ALU peak."""
+    import torch
+
+    import delta_rule_recurrent_chunked_b200 as drs
+    from delta_rule_recurrent_chunked_b200 import workloads as wl
+
+    inputs = wl.generate_vla(w, seed=rank)
+    nbytes = algorithmic_bytes(w)
+    nsets, needs_flush = rotation(nbytes)
+    flush = make_flush(device) if needs_flush else None
+    sets = [{k: torch.from_numpy(np.ascontiguousarray(inputs[k])).to(device)
+             for k in ("q", "k", "v", "u")} for _ in range(nsets)]
+    outs = [torch.empty_like(st["v"]) for st in sets]
+
+    def step(i):
+        st = sets[i % nsets]
+        if w.ratio:
+            drs.vla_scan_ratio(st["q"], st["k"], st["v"], st["u"], lambda0=w.lambda0,
+                               out=outs[i % nsets])
+        else:
+            drs.vla_scan(st["q"], st["k"], st["v"], st["u"], lambda0=w.lambda0,
+                         out=outs[i % nsets])
+
+    stream = torch.cuda.current_stream(device)
+    for i in range(max(3, args.warmup)):
         step(i)
-        ends[i].record(stream)
     torch.cuda.synchronize(device)
-    t_wall = time.perf_counter() - t_wall
-    barrier(device)
-    clk = clocks.stop()
-    total_ms = starts[0].elapsed_time(ends[-1])
-    launch_ms = statistics.mean(starts[i].elapsed_time(ends[i]) for i in range(K))
+    if drs.poll_error(device) != 0:
+        raise RuntimeError("device status set during warm-up")
+    total_ms, per_launch, clk, t_wall = timed_loop(step, K, device, stream, local, flush)
     if drs.poll_error(device) != 0:
         raise RuntimeError("device status set in the timed region")
     total_ms_max = max_over_ranks(total_ms, device=device)
+    launch_ms = statistics.mean(per_launch)
+    del sets, outs
 
     # end to end: pinned host q/k/v/u in, out/S_final/A_final back, every step (pipelined)
     host = {k: torch.from_numpy(np.ascontiguousarray(inputs[k])).pin_memory()
@@ -473,48 +532,40 @@ def run_ours_vla(args, world, rank, local, w, device):
                 torch.empty((w.B, w.H, w.d, w.d), dtype=torch.float32, device=device)]
 
     def launch(d, o):
-        _, Sf, Af = drs.vla_scan(d["q"], d["k"], d["v"], d["u"], lambda0=w.lambda0, out=o[0])
+        if w.ratio:
+            _, Sf, Af, _ = drs.vla_scan_ratio(d["q"], d["k"], d["v"], d["u"], lambda0=w.lambda0,
+                                              out=o[0])
+        else:
+            _, Sf, Af = drs.vla_scan(d["q"], d["k"], d["v"], d["u"], lambda0=w.lambda0, out=o[0])
         o[1].copy_(Sf)
         o[2].copy_(Af)
 
     pipe = CopyPipeline(device, host, make_outputs, launch)
     e2e_ms = max_over_ranks(pipe.run(max(1, args.e2e_steps)), device=device)
-    h2d, d2h = pipe.h2d, pipe.d2h
 
     flops = algorithmic_flops(w)
     peak = fp32_alu_peak_tflops(device)
     achieved = flops / (launch_ms / 1e3) / 1e12
-    line = {
-        "metric": METRIC, "value": aggregate_value(world, w.head_tokens, K, total_ms_max),
-        "unit": UNIT, "n_gpus": world, "steps": K, "warmup": max(3, args.warmup),
-        "ms_per_step": total_ms_max / K, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": dict(workload_config(w, world, nsets, nbytes), kernel="vla_sequential"),
-        "clocks": {k: clk[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
-        "e2e": {"value": world * w.head_tokens / (e2e_ms / 1e3), "unit": UNIT,
-                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": K,
-        "roofline": {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                     "frac": achieved / peak, "traffic": None,
-                     "peak_source": "derived: SMs x 128 FP32 lanes x 2 x max SM clock",
-                     "flops_per_launch": flops, "launch_ms": launch_ms,
-                     "hbm_gbs": nbytes / (launch_ms / 1e3) / 1e9},
-        "wall_s": t_wall,
-    }
+    config = dict(workload_config(w, world), l2=l2_note(nsets, nbytes, needs_flush),
+                  kernel="vla_sequential")
+    line = base_line(args, w, world, K, total_ms_max, clk, e2e_ms, pipe.h2d, pipe.d2h, config,
+                     "f32", t_wall)
+    line["roofline"] = {
+        "bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+        "frac": achieved / peak, "traffic": None,
+        "peak_source": "derived: SMs x 128 FP32 lanes x 2 x max SM clock",
+        "flops_per_launch": flops, "launch_ms": launch_ms,
+        "hbm_gbs": nbytes / (launch_ms / 1e3) / 1e9}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(inputs)
-    if world > 1:
-        dist.destroy_process_group()
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+        line["cpu_baseline"] = cpu_baseline(inputs, cpu_target)
+    return line
 
 
-def run_ours_decode(args, world, rank, local, w, device):
+def measure_decode(args, w, world, rank, local, device, K, cpu_target):
     """Streaming decode through dr_decode_step: one token per head per step on an fp32 state
     that stays resident in HBM and is updated in place (HBM-bound: the state is read and
     written once per step)."""
     import torch
-    import torch.distributed as dist
 
     import delta_rule_recurrent_chunked_b200 as drs
     from delta_rule_recurrent_chunked_b200 import workloads as wl
@@ -540,27 +591,11 @@ def run_ours_decode(args, world, rank, local, w, device):
     torch.cuda.synchronize(device)
     if drs.poll_error(device) != 0:
         raise RuntimeError("device status set during warm-up")
-    K = args.steps
-    starts = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    ends = [torch.cuda.Event(enable_timing=True) for _ in range(K)]
-    clocks = ClockSampler(local)
-    barrier(device)
-    torch.cuda.synchronize(device)
-    clocks.start()
-    t_wall = time.perf_counter()
-    for i in range(K):
-        starts[i].record(stream)
-        step(i)
-        ends[i].record(stream)
-    torch.cuda.synchronize(device)
-    t_wall = time.perf_counter() - t_wall
-    barrier(device)
-    clk = clocks.stop()
-    total_ms = starts[0].elapsed_time(ends[-1])
-    launch_ms = statistics.mean(starts[i].elapsed_time(ends[i]) for i in range(K))
+    total_ms, per_launch, clk, t_wall = timed_loop(step, K, device, stream, local)
     if drs.poll_error(device) != 0:
         raise RuntimeError("device status set in the timed region")
     total_ms_max = max_over_ranks(total_ms, device=device)
+    launch_ms = statistics.mean(per_launch)
 
     # end to end: each step's token (q, k, v, beta, gate) from pinned host memory and its
     # output back; the state is the model's and stays resident on the device
@@ -577,26 +612,135 @@ def run_ours_decode(args, world, rank, local, w, device):
 
     peaks, peak_src = load_peaks()
     achieved = nbytes / (launch_ms / 1e3) / 1e9
-    line = {
-        "metric": METRIC, "value": aggregate_value(world, w.head_tokens, K, total_ms_max),
-        "unit": UNIT, "n_gpus": world, "steps": K, "warmup": max(3, args.warmup),
-        "ms_per_step": total_ms_max / K, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": w.dtype, "data": "synthetic",
-        "config": dict(workload_config(w, world), kernel="decode",
-                       l2=f"resident state {w.B * w.H * w.dv * w.dk * 4 / 2**20:.0f} MiB > 126 MiB L2"),
-        "clocks": {k: clk[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
-        "e2e": {"value": world * w.head_tokens / (e2e_ms / 1e3), "unit": UNIT,
-                "h2d_bytes_per_step": pipe.h2d, "d2h_bytes_per_step": pipe.d2h},
-        "gpu_launches": K,
-        "roofline": {"bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                     "frac": achieved / peaks["hbm_gbs"],
-                     "traffic": NCU_TRAFFIC.get((w.name, kernel_source_sha("dr_decode.cuh"))),
-                     "peak_source": f"{peak_src} hbm_gbs", "bytes_per_launch": nbytes,
-                     "launch_ms": launch_ms},
-        "wall_s": t_wall,
-    }
+    config = dict(workload_config(w, world), kernel="decode",
+                  l2=f"resident state {w.B * w.H * w.dv * w.dk * 4 / 2**20:.0f} MiB > 126 MiB L2")
+    line = base_line(args, w, world, K, total_ms_max, clk, e2e_ms, pipe.h2d, pipe.d2h, config,
+                     w.dtype, t_wall)
+    line["roofline"] = {
+        "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+        "frac": achieved / peaks["hbm_gbs"],
+        "traffic": NCU_TRAFFIC.get((w.name, kernel_source_sha("dr_decode.cuh"))),
+        "peak_source": f"{peak_src} hbm_gbs", "bytes_per_launch": nbytes,
+        "launch_ms": launch_ms}
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(inputs)
+        line["cpu_baseline"] = cpu_baseline(inputs, cpu_target)
+    return line
+
+
+def measure_loglinear(args, w, world, rank, local, device, K, cpu_target):
+    """Log-linear attention (loglinear_scan_fwd) on one workload: resident inputs timed on the
+    device, e2e through the C ABI with host buffers, HBM roofline, oracle on the host."""
+    import torch
+
+    import delta_rule_recurrent_chunked_b200 as drs
+    from delta_rule_recurrent_chunked_b200 import workloads as wl
+
+    inputs = wl.generate_loglinear(w, seed=rank)
+    nbytes = algorithmic_bytes(w)
+    nsets, needs_flush = rotation(nbytes)
+    flush = make_flush(device) if needs_flush else None
+
+    def upload():
+        d = {}
+        for name in ("q", "k", "v"):
+            raw = np.ascontiguousarray(inputs[name + "_raw"])
+            d[name] = torch.from_numpy(raw.view(np.int16)).view(torch.bfloat16).to(device)
+        d["lam"] = torch.from_numpy(np.ascontiguousarray(inputs["lam"])).to(device)
+        return d
+
+    sets = [upload() for _ in range(nsets)]
+    outs = [torch.empty_like(st["v"]) for st in sets]
+
+    def step(i):
+        st = sets[i % nsets]
+        drs.loglinear_scan(st["q"], st["k"], st["v"], st["lam"], out=outs[i % nsets])
+
+    stream = torch.cuda.current_stream(device)
+    for i in range(max(3, args.warmup)):
+        step(i)
+    torch.cuda.synchronize(device)
+    if drs.poll_error(device) != 0:
+        raise RuntimeError("device status set during warm-up")
+    total_ms, per_launch, clk, t_wall = timed_loop(step, K, device, stream, local, flush)
+    if drs.poll_error(device) != 0:
+        raise RuntimeError("device status set in the timed region")
+    total_ms_max = max_over_ranks(total_ms, device=device)
+    launch_ms = statistics.mean(per_launch)
+    del sets, outs
+
+    host = {}
+    for name in ("q", "k", "v"):
+        raw = np.ascontiguousarray(inputs[name + "_raw"])
+        host[name] = torch.from_numpy(raw.view(np.int16)).view(torch.bfloat16).pin_memory()
+    host["lam"] = torch.from_numpy(np.ascontiguousarray(inputs["lam"])).pin_memory()
+
+    def make_outputs():
+        return [torch.empty(host["v"].shape, dtype=torch.bfloat16, device=device)]
+
+    def launch(d, o):
+        drs.loglinear_scan(d["q"], d["k"], d["v"], d["lam"], out=o[0])
+
+    pipe = CopyPipeline(device, host, make_outputs, launch)
+    e2e_ms = max_over_ranks(pipe.run(max(1, args.e2e_steps)), device=device)
+
+    peaks, peak_src = load_peaks()
+    achieved = nbytes / (launch_ms / 1e3) / 1e9
+    tflops = algorithmic_flops(w) / (launch_ms / 1e3) / 1e12
+    config = dict(workload_config(w, world), l2=l2_note(nsets, nbytes, needs_flush),
+                  kernel="loglinear")
+    line = base_line(args, w, world, K, total_ms_max, clk, e2e_ms, pipe.h2d, pipe.d2h, config,
+                     "bf16", t_wall)
+    line["roofline"] = {
+        "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+        "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+        "peak_source": f"{peak_src} hbm_gbs", "bytes_per_launch": nbytes,
+        "launch_ms": launch_ms, "tensor_tflops": tflops,
+        "tensor_frac": tflops / peaks["bf16_tflops"]}
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(inputs, cpu_target)
+    return line
+
+
+def measure(args, name, world, rank, local, device, K, cpu_target):
+    from delta_rule_recurrent_chunked_b200 import workloads as wl
+
+    w = wl.workload(name)
+    if isinstance(w, wl.LogLinearWorkload):
+        return measure_loglinear(args, w, world, rank, local, device, K, cpu_target)
+    if isinstance(w, wl.VLAWorkload):
+        return measure_vla(args, w, world, rank, local, device, K, cpu_target)
+    if w.decode:
+        return measure_decode(args, w, world, rank, local, device, K, cpu_target)
+    return measure_dr(args, w, world, rank, local, device, K, cpu_target)
+
+
+# keys of a per_config entry (the rest of a line is shared by all configurations)
+PER_CONFIG_KEYS = ("value", "unit", "ms_per_step", "steps", "dtype", "config", "clocks", "e2e",
+                   "gpu_launches", "roofline", "cpu_baseline")
+
+
+def run_ours(args, world, rank, local):
+    import torch
+    import torch.distributed as dist
+
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", device_id=device, timeout=timedelta(seconds=120))
+
+    line = measure(args, args.workload, world, rank, local, device, args.steps, 10.0)
+    if world == 1 and not args.no_per_config:
+        K = args.per_config_steps or min(args.steps, 200)
+        per = {}
+        for name in PER_CONFIG:
+            if name == args.workload:
+                continue
+            sub = measure(args, name, world, rank, local, device, K, 3.0)
+            per[name] = {k: sub[k] for k in PER_CONFIG_KEYS if k in sub}
+            torch.cuda.empty_cache()
+        line["per_config"] = per
     if world > 1:
         dist.destroy_process_group()
     if rank == 0:
@@ -681,7 +825,7 @@ def run_e2e(args, w, inputs, mode, device, stream):
         t = torch.from_numpy(raw.view(np.int16)).view(torch.bfloat16) if w.dtype == "bf16" \
             else torch.from_numpy(raw)
         host[name] = t.pin_memory()
-    for name in ("beta", "gate", "S0"):
+    for name in ("beta", "gate", "S0", "erase", "write"):
         a = inputs.get(name)
         host[name] = None if a is None else torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
 
@@ -690,8 +834,12 @@ def run_e2e(args, w, inputs, mode, device, stream):
                 torch.empty((w.B, w.H, w.dv, w.dk), dtype=torch.float32, device=device)]
 
     def launch(d, o):
-        drs.scan(d["q"], d["k"], d["v"], d["beta"], d["gate"], d["S0"], mode=mode,
-                 out=o[0], S_final=o[1])
+        if d.get("erase") is not None:
+            drs.scan_ex(d["q"], d["k"], d["v"], d["beta"], d["gate"], d["S0"], mode=mode,
+                        erase=d["erase"], write=d["write"], want_u=False, out=o[0], S_final=o[1])
+        else:
+            drs.scan(d["q"], d["k"], d["v"], d["beta"], d["gate"], d["S0"], mode=mode,
+                     out=o[0], S_final=o[1])
 
     pipe = CopyPipeline(device, host, make_outputs, launch)
     ms = pipe.run(max(1, args.e2e_steps))

@@ -1,4 +1,5 @@
-// Chunked delta-rule scan on sm_100a tensor cores (DeltaNet, Gated DeltaNet, KDA).
+// Chunked delta-rule scan on sm_100a tensor cores (DeltaNet, Gated DeltaNet, KDA, Gated
+// DeltaNet-2).
 //
 // The sequence is cut into chunks of C = 64 tokens. Inside a chunk with entering state
 // S0 (dv x dk), g_t the running sum of log-decay (scalar for GDN, per key channel for
@@ -12,7 +13,10 @@
 //     O      = diag(gamma) Q S0^T + (P T) Y
 //     S_C^T  = diag(gamma_C) S0^T + Khat^T Y,  Khat^T = K^T diag(gamma_C/gamma) T
 // (KDA: the decay sits inside the operands, K*gamma, Q*gamma and K/gamma per channel, and
-// Khat^T = diag(gamma_C) (K/gamma)^T T.)
+// Khat^T = diag(gamma_C) (K/gamma)^T T. Gated DeltaNet-2 is Gated DeltaNet run on its erase
+// directions e = b (.) k and write targets z = w (.) v: the prep warps scale the K tile by b
+// and the V producer the V tile by w, in shared memory.) Rows 0-63 of MMA2 below are
+// T Y = U, the chunk's write values u_t = beta_t r_t, stored when the caller asks for them.
 //
 // Contractions on tcgen05 (bf16 operands in 128-byte-swizzled shared memory, fp32
 // accumulators in tensor memory), one CTA per (b, h, slice of BV value channels):
@@ -55,6 +59,9 @@
 namespace drscan {
 
 constexpr int CK = 64;    // chunk length
+// KDA: lowest summed log alpha of one key channel over one chunk that the anchored
+// factorisation represents exactly (its factors stay below exp(85) in fp32 and bf16)
+constexpr float KDA_MIN_LOG_DECAY = -170.f;
 constexpr int CDK = 128;  // key dimension of the chunked kernel
 constexpr int CHUNK_THREADS = 512;
 
@@ -65,8 +72,9 @@ constexpr int CHUNK_THREADS = 512;
 template <int MODE, int BV, bool SPLIT = false>
 struct ChunkLayout {
     static constexpr bool kKda = MODE == DR_KDA;
-    static constexpr bool kGdn = MODE == DR_GDN;
+    static constexpr bool kGdn = MODE == DR_GDN || MODE == DR_GDN2;  // scalar gate
     static_assert(!(SPLIT && kKda), "KDA is never split");
+    static_assert(!(SPLIT && MODE == DR_GDN2), "Gated DeltaNet-2 is never split");
     static constexpr int NS = 2;                          // K/Q stages
     static constexpr int NSV = (kKda && BV == 128) ? 1 : 2;  // V stages
     static constexpr int NP = (kKda && BV >= 64) ? 1 : 2;    // prepared-operand slots
@@ -174,7 +182,8 @@ enum ChunkBar {
     B_PREP2 = 27,      // split chain CTA: third slot ready
     B_MMA2 = 28,       // split chain CTA: MMA2 done
     B_SFREE = 29,      // [3] split chain CTA: chain slot i read by every thread and every MMA
-    B_COUNT = 32
+    B_VSCALED = 32,    // [2] Gated DeltaNet-2: V stage scaled by the write gate
+    B_COUNT = 34
 };
 
 // bf16 bits of 8 consecutive columns of a row, stored as one 16-byte swizzled chunk.
@@ -246,11 +255,14 @@ template <int MODE, int BV, bool SPLIT>
 __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
     const __grid_constant__ CUtensorMap tmV, const float* __restrict__ beta,
-    const float* __restrict__ gate, const float* __restrict__ S0,
-    __nv_bfloat16* __restrict__ out, float* __restrict__ S_final, int T, int dv, int nprep) {
+    const float* __restrict__ gate, const float* __restrict__ erase,
+    const float* __restrict__ write, const float* __restrict__ S0,
+    __nv_bfloat16* __restrict__ out, float* __restrict__ S_final,
+    __nv_bfloat16* __restrict__ u_out, int T, int dv, int nprep) {
     using L = ChunkLayout<MODE, BV, SPLIT>;
-    constexpr bool kGdn = MODE == DR_GDN;
+    constexpr bool kGdn = L::kGdn;  // scalar gate (Gated DeltaNet and Gated DeltaNet-2)
     constexpr bool kKda = MODE == DR_KDA;
+    constexpr bool kGdn2 = MODE == DR_GDN2;
     constexpr int NS = L::NS, NSV = L::NSV, NP = L::NP;
 
     extern __shared__ uint8_t smem_raw[];
@@ -299,6 +311,10 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
         return sm + L::SLOT + i * L::SLOT_B;
     };
     auto cprep = [&](int i) { return bar(i == 2 ? B_PREP2 : B_PREP + i); };
+    // a split cluster copies the PT rows, Khat^T and the gammas of each slot, and the T rows
+    // as well when the chain CTAs export the write values (rows 0-63 of MMA2)
+    const uint32_t copy_off = u_out ? (uint32_t)L::SLOT_TP : (uint32_t)L::COPY_OFF;
+    const uint32_t copy_b = u_out ? (uint32_t)(L::COPY_B + 8192) : (uint32_t)L::COPY_B;
     auto slot = [&](int p) { return sm + L::SLOT + p * L::SLOT_B; };
 
     if (tid == 0) {
@@ -323,7 +339,10 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
         mbar_init(bar(B_GRP1 + 1), 1);
         mbar_init(bar(B_GRP1 + 2), gthreads);
         mbar_init(bar(B_GRP1 + 3), 1);
-        mbar_init(bar(B_ODONE), 128);
+        // output rows read out of D2 (and, when exporting, the write-value rows)
+        mbar_init(bar(B_ODONE), u_out ? 256 : 128);
+        mbar_init(bar(B_VSCALED + 0), 1);
+        mbar_init(bar(B_VSCALED + 1), 1);
         mbar_init(bar(B_MMA1), 1);
         mbar_init(bar(B_YREADY), 128);
         mbar_init(bar(B_MMA23), 1);
@@ -404,9 +423,11 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
         }
     } else if (warp == 3 && is_chain) {
         // ------------------------------------------------------------------ V producer
-        if (lane == 0) {
-            for (int c = 0; c < nchunks; ++c) {
-                const int sv = c % NSV;
+        // (Gated DeltaNet-2: the whole warp then scales the landed tile in place by the write
+        // gate, z = w (.) v, and releases it on B_VSCALED)
+        for (int c = 0; c < nchunks; ++c) {
+            const int sv = c % NSV;
+            if (lane == 0) {
                 if (c >= NSV)
                     mbar_wait(bar(B_V_EMPTY + sv), (uint32_t)(((c / NSV) - 1) & 1), abort_flag);
                 if (!*abort_flag) {
@@ -414,6 +435,23 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     tma_load_3d(smem_u32(sm + L::V + sv * L::V_B), &tmV, bar(B_V_FULL + sv), v0,
                                 c * CK, (int)bh);
                 }
+            }
+            if constexpr (kGdn2) {
+                __syncwarp();
+                mbar_wait(bar(B_V_FULL + sv), (uint32_t)((c / NSV) & 1), abort_flag);
+                static_assert(!L::V_SWZ, "rows of V are plain BV-element rows here");
+                __nv_bfloat162* vt = reinterpret_cast<__nv_bfloat162*>(sm + L::V + sv * L::V_B);
+                constexpr int PAIRS = CK * BV / 2;
+                for (int e = lane; e < PAIRS; e += 32) {
+                    const int row = e / (BV / 2), col = 2 * (e % (BV / 2));
+                    const int t = c * CK + row;
+                    float2 w2 = make_float2(0.f, 0.f);
+                    if (t < T) w2 = *reinterpret_cast<const float2*>(write + (bh * T + t) * (long)dv + v0 + col);
+                    const float2 x = __bfloat1622float2(vt[e]);
+                    vt[e] = __floats2bfloat162_rn(x.x * w2.x, x.y * w2.y);
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar(B_VSCALED + sv));
             }
         }
     } else if (warp == 1 && !is_chain) {
@@ -430,10 +468,10 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 mbar_wait(bar(B_PEER_FREE + p), ph, abort_flag);
                 if (!*abort_flag) {
                     // into chain slot c % npc of every chain rank
-                    const uint32_t src = smem_u32(slot(p)) + L::COPY_OFF;
-                    const uint32_t dst = smem_u32(cslot(c % npc)) + L::COPY_OFF;
+                    const uint32_t src = smem_u32(slot(p)) + copy_off;
+                    const uint32_t dst = smem_u32(cslot(c % npc)) + copy_off;
                     for (int q = NPREP; q < NPREP + NCC; ++q)  // the chain ranks
-                        bulk_copy_to_peer(cluster_map(dst, q), src, L::COPY_B,
+                        bulk_copy_to_peer(cluster_map(dst, q), src, copy_b,
                                           cluster_map(cprep(c % npc), q));
                     bulk_commit_and_wait_read();
                 }
@@ -598,7 +636,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             // slots start empty: expect the prep CTAs' copies of the first chunks
             if (h == 0 && r == 0) {
                 for (int c = 0; c < npc && c < nchunks; ++c) {
-                    mbar_arrive_expect_tx(cprep(c), L::COPY_B);
+                    mbar_arrive_expect_tx(cprep(c), copy_b);
                     mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + pslot_of(c)), owner_of(c)));
                 }
             }
@@ -638,6 +676,32 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             tc_fence_before();
             mbar_arrive(bar(B_STATE));
         }
+        // write values U = T Y of chunk c (rows 0-63 of D2), read by the residual threads once
+        // MMA2 of that chunk is done; D2 is reused only after they (and the output threads)
+        // arrive on B_ODONE
+        auto export_u = [&](int c) {
+            mbar_wait(bar(B_MMA2), (uint32_t)(c & 1), abort_flag);
+            tc_fence_after();
+            if (active) {
+                float d[LW];
+#pragma unroll
+                for (int c16 = 0; c16 < LW; c16 += 16) tmem_ld16(trow + L::COL_D2 + cb + c16, d + c16);
+                tmem_wait_ld();
+                if (c * CK + r < T) {
+                    uint4* dst = reinterpret_cast<uint4*>(u_out + (bh * T + c * CK + r) * (long)dv + v0 + cb);
+#pragma unroll
+                    for (int i = 0; i < NV8; ++i) {
+                        uint4 w;
+                        uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) wp[e] = pack_bf16(d[8 * i + 2 * e], d[8 * i + 2 * e + 1]);
+                        dst[i] = w;
+                    }
+                }
+            }
+            tc_fence_before();
+            mbar_arrive(bar(B_ODONE));
+        };
         for (int c = 0; c < nchunks; ++c) {
             const int svi = c % NSV;
             const int t0 = c * CK;
@@ -645,6 +709,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             const uint32_t d1 = L::COL_D1 + 128 * (c & 1);
             const float gt = gt_next;
             const bool last = c == nchunks - 1;
+            if (u_out && r < 64 && c > 0) export_u(c - 1);
             // ---- residuals Y = V - gamma_t (S0 k_t), stored as the B operand Y^T
             if (r < 64) {
                 if (active) {
@@ -751,23 +816,38 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 }
             }
         }
+        if (u_out && r < 64 && nchunks > 0) export_u(nchunks - 1);
     } else if (warp >= 4 && warp < 8) {
         if (!is_chain) goto done;
         // ------------------------------------------------------------------ chain warpgroup
         const int r = tid - 128;  // TMEM lane: value row t (Y, O) or key channel j (state)
         const uint32_t trow = tmem + ((uint32_t)(r & ~31) << 16);
+        // KDA: the bf16 copy of a chunk's entering state is scaled per key channel (lane r) by
+        // exp(m), m the chunk's anchor, published by the prep warps before they release the
+        // Gram operands of that chunk (phase c of B_GO)
+        auto state_anchor = [&](int c) -> float {
+            if constexpr (kKda) {
+                mbar_wait(bar(B_GO), (uint32_t)(c & 1), abort_flag);
+                return reinterpret_cast<const float*>(sm + L::BG + (c % NS) * L::BG_B)[128 + r];
+            } else {
+                return 1.f;
+            }
+        };
         {
             const float* src = S0 ? S0 + (bh * dv + v0) * (long)CDK + r : nullptr;
+            const float em = state_anchor(0);
 #pragma unroll
             for (int c16 = 0; c16 < L::NB; c16 += 16) {
-                float sv[16];
+                float sv[16], sb[16];
 #pragma unroll
-                for (int v = 0; v < 16; ++v)
+                for (int v = 0; v < 16; ++v) {
                     sv[v] = (src && c16 < BV) ? src[(long)(c16 + v) * CDK] : 0.f;
+                    sb[v] = sv[v] * em;
+                }
                 if (c16 < BV) {
                     uint8_t* grp = sm + L::SS + (c16 >> 6) * 16384;
-                    st_row_chunk(grp, r, (c16 & 63) >> 3, sv);
-                    st_row_chunk(grp, r, ((c16 & 63) >> 3) + 1, sv + 8);
+                    st_row_chunk(grp, r, (c16 & 63) >> 3, sb);
+                    st_row_chunk(grp, r, ((c16 & 63) >> 3) + 1, sb + 8);
                 }
                 tmem_st16(trow + L::COL_S + c16, sv);
             }
@@ -804,7 +884,8 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             tc_fence_after();
             if (r < 64) {
                 // residual Y = V - gamma_t (S0 k_t), stored as the B operand Y^T
-                mbar_wait(bar(B_V_FULL + svi), (uint32_t)((c / NSV) & 1), abort_flag);
+                mbar_wait(bar((kGdn2 ? B_VSCALED : B_V_FULL) + svi), (uint32_t)((c / NSV) & 1),
+                          abort_flag);
                 const float gt = kGdn ? gam[r] : 1.f;
                 const uint4* vrow =
                     reinterpret_cast<const uint4*>(sm + L::V + svi * L::V_B + r * BV * 2);
@@ -836,6 +917,25 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
 
             mbar_wait(bar(B_MMA23), (uint32_t)(c & 1), abort_flag);
             tc_fence_after();
+            if (r < 64 && u_out) {
+                // write values U = T Y (rows 0-63 of D2)
+#pragma unroll
+                for (int c16 = 0; c16 < BV; c16 += 16) {
+                    float d[16];
+                    tmem_ld16(trow + L::COL_D2 + c16, d);
+                    tmem_wait_ld();
+                    if (r < nvalid) {
+                        uint4 w[2];
+                        uint32_t* wp = reinterpret_cast<uint32_t*>(w);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) wp[e] = pack_bf16(d[2 * e], d[2 * e + 1]);
+                        uint4* dst = reinterpret_cast<uint4*>(u_out + (bh * T + t0 + r) * (long)dv +
+                                                              v0 + c16);
+                        dst[0] = w[0];
+                        dst[1] = w[1];
+                    }
+                }
+            }
             if (r >= 64) {
                 // output rows: O = gamma_t (S0 q_t) + (P T Y)_t
                 const int t = r - 64;
@@ -865,6 +965,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 float* dst = (c == nchunks - 1 && S_final)
                                  ? S_final + (bh * dv + v0) * (long)CDK + r
                                  : nullptr;
+                const float em = (kKda && c + 1 < nchunks) ? state_anchor(c + 1) : 1.f;
                 constexpr int HW = BV < 64 ? BV : 64;
 #pragma unroll
                 for (int c0 = 0; c0 < BV; c0 += HW) {
@@ -872,14 +973,18 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
 #pragma unroll
                     for (int c16 = 0; c16 < HW; c16 += 16) tmem_ld16(trow + L::COL_S + c0 + c16, sv + c16);
                     tmem_wait_ld();
+                    if (dst) {
+#pragma unroll
+                        for (int v = 0; v < HW; ++v) dst[(long)(c0 + v) * CDK] = sv[v];
+                    }
+                    if constexpr (kKda) {
+#pragma unroll
+                        for (int v = 0; v < HW; ++v) sv[v] *= em;
+                    }
 #pragma unroll
                     for (int i = 0; i < HW / 8; ++i) {
                         const int col = c0 + 8 * i;
                         st_row_chunk(sm + L::SS + (col >> 6) * 16384, r, (col & 63) >> 3, sv + 8 * i);
-                    }
-                    if (dst) {
-#pragma unroll
-                        for (int v = 0; v < HW; ++v) dst[(long)(c0 + v) * CDK] = sv[v];
                     }
                 }
             }
@@ -901,7 +1006,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
         if (lane == 0) {
             for (int c = 0; c + npc < nchunks; ++c) {
                 mbar_wait(bar(B_SFREE + c % npc), (uint32_t)((c / npc) & 1), abort_flag);
-                mbar_arrive_expect_tx(cprep(c % npc), L::COPY_B);
+                mbar_arrive_expect_tx(cprep(c % npc), copy_b);
                 mbar_arrive_remote(cluster_map(bar(B_PEER_FREE + pslot_of(c + npc)), owner_of(c + npc)));
             }
         }
@@ -925,18 +1030,21 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
         float* sA = reinterpret_cast<float*>(sm + (gi ? L::AM2 : L::AM));
         float* sZ = reinterpret_cast<float*>(sm + (gi ? L::ZS2 : L::ZS));
         auto gsync = [&]() { group_sync(gi, GT); };
-        // KDA (always one group) scan exchange: pg[128*q + ch] = product over row quarter q;
-        // gamma_C at pg[512 + ch]
+        // KDA (always one group) scan exchange: pg[128*q + ch] = summed log alpha over row
+        // quarter q; exp(G - m) at pg[512 + ch], gamma_C = exp(G) at pg[640 + ch]
         float* pg = reinterpret_cast<float*>(sm + L::PG);
         // KDA: thread u owns key channels 2*(u%64), 2*(u%64)+1 on rows 16*(u/64) .. +15 of a
         // chunk; the next owned chunk's alpha values are prefetched into registers.
+        // Gated DeltaNet-2 prefetches its erase gate b the same way and scales K by it.
         const int kc = 2 * (u & 63), kq4 = u >> 6;
-        float2 gpf[kKda ? 16 : 1];
-        if constexpr (kKda) {
+        constexpr bool kChan = kKda || kGdn2;  // per-key-channel values prefetched per chunk
+        const float* chan = kKda ? gate : erase;
+        float2 gpf[kChan ? 16 : 1];
+        if constexpr (kChan) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const int t = 16 * kq4 + i;
-                gpf[i] = t < T ? *reinterpret_cast<const float2*>(gate + (bh * T + t) * (long)CDK + kc)
+                gpf[i] = t < T ? *reinterpret_cast<const float2*>(chan + (bh * T + t) * (long)CDK + kc)
                                : make_float2(1.f, 1.f);
             }
         }
@@ -958,26 +1066,68 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             bool fact = true;
             if constexpr (kGdn) {
                 fact = bg[64 + 63] > -80.f;
+                if constexpr (kGdn2) {
+                    // erase directions e = b (.) k, in place in the stage's K rows
+#pragma unroll
+                    for (int i0 = 0; i0 < 16; i0 += 8) {
+                        uint32_t kw[8];
+#pragma unroll
+                        for (int i = 0; i < 8; ++i)
+                            kw[i] = *reinterpret_cast<const uint32_t*>(kq + sw128_offset(16 * kq4 + i0 + i, kc, 128));
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) {
+                            const float2 k2 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&kw[i]));
+                            *reinterpret_cast<uint32_t*>(kq + sw128_offset(16 * kq4 + i0 + i, kc, 128)) =
+                                pack_bf16(k2.x * gpf[i0 + i].x, k2.y * gpf[i0 + i].y);
+                        }
+                    }
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) {
+                        const int tn = (c + NGR * pSP) * CK + 16 * kq4 + i;
+                        gpf[i] = tn < T ? *reinterpret_cast<const float2*>(erase + (bh * T + tn) * (long)CDK + kc)
+                                        : make_float2(1.f, 1.f);
+                    }
+                    fence_async_smem();
+                    gsync();
+                }
             } else if constexpr (kKda) {
-                // running products of alpha per key channel (four row quarters joined through
-                // shared memory); rewrite K and Q in place as K*gamma, Q*gamma; store K/gamma
+                // Per key channel c, G = summed log alpha over the chunk (four row quarters
+                // joined through shared memory) and the anchor m = G/2. K and Q are rewritten
+                // in place as K*exp(g - m), Q*exp(g - m) and K*exp(m - g) is stored, so every
+                // factor of exp(g_t - g_i) = exp(g_t - m) * exp(m - g_i) stays within
+                // exp(+-|G|/2): exact for G down to KDA_MIN_LOG_DECAY. The chain multiplies its
+                // bf16 state copy by exp(m) per channel, which restores exp(g_t) in MMA1.
                 uint8_t* kn = sm + L::KN;
-                float2 part = make_float2(1.f, 1.f);
+                float2 lp = make_float2(0.f, 0.f);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     if (16 * kq4 + i < nvalid) {
-                        part.x *= gpf[i].x;
-                        part.y *= gpf[i].y;
+                        lp.x += __logf(gpf[i].x);
+                        lp.y += __logf(gpf[i].y);
                     }
                 }
-                if (kq4 < 3) *reinterpret_cast<float2*>(pg + 128 * kq4 + kc) = part;
+                *reinterpret_cast<float2*>(pg + 128 * kq4 + kc) = lp;
                 gsync();
-                float2 run = make_float2(1.f, 1.f);
-                for (int q = 0; q < kq4; ++q) {
+                float2 G = make_float2(0.f, 0.f), Lb = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
                     const float2 pq = *reinterpret_cast<const float2*>(pg + 128 * q + kc);
-                    run.x *= pq.x;
-                    run.y *= pq.y;
+                    if (q < kq4) {
+                        Lb.x += pq.x;
+                        Lb.y += pq.y;
+                    }
+                    G.x += pq.x;
+                    G.y += pq.y;
                 }
+                const float2 m = make_float2(0.5f * G.x, 0.5f * G.y);
+                if (kq4 == 0) {
+                    if (G.x < KDA_MIN_LOG_DECAY || G.y < KDA_MIN_LOG_DECAY)
+                        raise_status(DR_ERR_GATE_RANGE);
+                    // exp(m) for the chain's copy of the entering state of this chunk
+                    float* bgw = reinterpret_cast<float*>(sm + L::BG + s * L::BG_B);
+                    *reinterpret_cast<float2*>(bgw + 128 + kc) = make_float2(__expf(m.x), __expf(m.y));
+                }
+                float2 run = make_float2(__expf(Lb.x - m.x), __expf(Lb.y - m.y));
 #pragma unroll
                 for (int i0 = 0; i0 < 16; i0 += 8) {
                     uint32_t kw[8], qw[8];
@@ -1005,7 +1155,11 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                             pack_bf16(k2.x * ix, k2.y * iy);
                     }
                 }
-                if (kq4 == 3) *reinterpret_cast<float2*>(pg + 512 + kc) = run;  // gamma_C
+                if (kq4 == 3) {
+                    // exp(G - m) scales Khat^T's rows; gamma_C = exp(G) decays the state
+                    *reinterpret_cast<float2*>(pg + 512 + kc) = run;
+                    *reinterpret_cast<float2*>(pg + 640 + kc) = make_float2(__expf(G.x), __expf(G.y));
+                }
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int tn = (c + NGR * pSP) * CK + 16 * kq4 + i;
@@ -1199,7 +1353,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     if (v < 64) gam[v] = bg[192 + v];
                     if (v == 64) gam[64] = bg[192 + 63];
                 } else if constexpr (kKda) {
-                    if (v < 128) gam[v] = pg[512 + v];
+                    if (v < 128) gam[v] = pg[640 + v];
                 }
             }
             fence_async_smem();
@@ -1290,28 +1444,77 @@ inline bool make_map_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt
 
 inline bool chunked_supported(int variant, int dk, int dv) {
     return dk == CDK && (dv == 32 || dv == 64 || dv == 128) &&
-           (variant == DR_DELTANET || variant == DR_GDN || variant == DR_KDA);
+           (variant == DR_DELTANET || variant == DR_GDN || variant == DR_KDA ||
+            variant == DR_GDN2);
+}
+
+// Arguments of one chunked launch (device pointers as dr_scan_fwd_ex receives them).
+struct ChunkArgs {
+    const void *q, *k, *v;
+    const float *beta, *gate, *erase, *write, *S0;
+    void* out;
+    float* S_final;
+    void* u_out;
+    int BH, T, dv;
+};
+
+// The last tensor map encoded for each (thread, slot): a scan called again on the same
+// buffers and shape (the usual case in a loop) reuses it instead of encoding anew.
+struct MapCacheEntry {
+    const void* base = nullptr;
+    long BH = 0;
+    int T = 0, inner = 0, box = 0;
+    bool swz = false;
+    int dev = -1;
+    CUtensorMap map;
+};
+
+inline bool cached_map_3d(int slot, CUtensorMap* m, const void* base, long BH, int T, int inner,
+                          int box_inner, bool swizzle128) {
+    thread_local MapCacheEntry cache[8];
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    MapCacheEntry& e = cache[slot & 7];
+    if (e.base == base && e.BH == BH && e.T == T && e.inner == inner && e.box == box_inner &&
+        e.swz == swizzle128 && e.dev == dev) {
+        *m = e.map;
+        return true;
+    }
+    if (!make_map_3d(&e.map, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, BH, T, inner, box_inner,
+                     swizzle128)) {
+        e.base = nullptr;
+        return false;
+    }
+    e.base = base, e.BH = BH, e.T = T, e.inner = inner, e.box = box_inner, e.swz = swizzle128;
+    e.dev = dev;
+    *m = e.map;
+    return true;
 }
 
 template <int MODE, int BV, bool SPLIT>
-int launch_chunked_bv(const void* q, const void* k, const void* v, const float* beta,
-                      const float* gate, const float* S0, void* out, float* S_final, int BH, int T,
-                      int dv, int nprep, cudaStream_t stream) {
+int launch_chunked_bv(const ChunkArgs& a, int nprep, cudaStream_t stream) {
     using L = ChunkLayout<MODE, BV, SPLIT>;
     CUtensorMap mk, mq, mv;
-    if (!make_map_3d(&mk, k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, BH, T, CDK, 64, true) ||
-        !make_map_3d(&mq, q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, BH, T, CDK, 64, true) ||
-        !make_map_3d(&mv, v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, BH, T, dv, BV, L::V_SWZ))
+    if (!cached_map_3d(0, &mk, a.k, a.BH, a.T, CDK, 64, true) ||
+        !cached_map_3d(1, &mq, a.q, a.BH, a.T, CDK, 64, true) ||
+        !cached_map_3d(2, &mv, a.v, a.BH, a.T, a.dv, BV, L::V_SWZ))
         return DR_ERR_CUDA;
     const int smem = L::TOTAL + 1024;
     auto kern = dr_chunked_kernel<MODE, BV, SPLIT>;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
-        cudaSuccess)
-        return DR_ERR_CUDA;
+    // the shared-memory opt-in is a per-device property of the function: set it once
+    static bool attr_set[16] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DR_ERR_CUDA;
+    if (dev < 0 || dev >= 16 || !attr_set[dev]) {
+        if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+            cudaSuccess)
+            return DR_ERR_CUDA;
+        if (dev >= 0 && dev < 16) attr_set[dev] = true;
+    }
     const int split = SPLIT ? nprep : 0;  // prep CTAs per head
-    const int ny = dv / BV + split;
+    const int ny = a.dv / BV + split;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3((unsigned)BH, (unsigned)ny);
+    cfg.gridDim = dim3((unsigned)a.BH, (unsigned)ny);
     cfg.blockDim = dim3(CHUNK_THREADS);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
@@ -1322,9 +1525,9 @@ int launch_chunked_bv(const void* q, const void* k, const void* v, const float* 
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = split ? 1 : 0;
-    if (cudaLaunchKernelEx(&cfg, kern, mk, mq, mv, beta, gate, S0,
-                           static_cast<__nv_bfloat16*>(out), S_final, T, dv, split) !=
-        cudaSuccess)
+    if (cudaLaunchKernelEx(&cfg, kern, mk, mq, mv, a.beta, a.gate, a.erase, a.write, a.S0,
+                           static_cast<__nv_bfloat16*>(a.out), a.S_final,
+                           static_cast<__nv_bfloat16*>(a.u_out), a.T, a.dv, split) != cudaSuccess)
         return DR_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? DR_OK : DR_ERR_CUDA;
 }
@@ -1388,7 +1591,7 @@ struct SplitPlan {
 
 inline SplitPlan pick_split(int variant, long BH, int dv) {
     SplitPlan plan;
-    if (variant == DR_KDA || dv < 32) return plan;
+    if (variant == DR_KDA || variant == DR_GDN2 || dv < 32) return plan;
     const int bv = dv / 2, ncc = 2;
     for (int np = 4; np >= 1; --np) {
         if (BH * (np + ncc) <= 148 && BH <= max_active_clusters(np + ncc)) {
@@ -1401,58 +1604,44 @@ inline SplitPlan pick_split(int variant, long BH, int dv) {
 }
 
 template <int MODE>
-int launch_chunked_mode(const void* q, const void* k, const void* v, const float* beta,
-                        const float* gate, const float* S0, void* out, float* S_final, int BH,
-                        int T, int dv, cudaStream_t stream) {
-    const SplitPlan plan = pick_split(MODE, BH, dv);
-    if constexpr (MODE != DR_KDA) {
+int launch_chunked_mode(const ChunkArgs& a, cudaStream_t stream) {
+    const SplitPlan plan = pick_split(MODE, a.BH, a.dv);
+    if constexpr (MODE != DR_KDA && MODE != DR_GDN2) {
         if (plan.nprep > 0) {
             switch (plan.bv) {
                 case 16:
-                    return launch_chunked_bv<MODE, 16, true>(q, k, v, beta, gate, S0, out, S_final,
-                                                             BH, T, dv, plan.nprep, stream);
+                    return launch_chunked_bv<MODE, 16, true>(a, plan.nprep, stream);
                 case 32:
-                    return launch_chunked_bv<MODE, 32, true>(q, k, v, beta, gate, S0, out, S_final,
-                                                             BH, T, dv, plan.nprep, stream);
+                    return launch_chunked_bv<MODE, 32, true>(a, plan.nprep, stream);
                 case 64:
-                    return launch_chunked_bv<MODE, 64, true>(q, k, v, beta, gate, S0, out, S_final,
-                                                             BH, T, dv, plan.nprep, stream);
+                    return launch_chunked_bv<MODE, 64, true>(a, plan.nprep, stream);
             }
             return DR_ERR_UNSUPPORTED;
         }
     }
-    switch (pick_bv(MODE, BH, dv)) {
+    switch (pick_bv(MODE, a.BH, a.dv)) {
         case 16:
-            return launch_chunked_bv<MODE, 16, false>(q, k, v, beta, gate, S0, out, S_final, BH, T,
-                                                      dv, 0, stream);
+            return launch_chunked_bv<MODE, 16, false>(a, 0, stream);
         case 32:
-            return launch_chunked_bv<MODE, 32, false>(q, k, v, beta, gate, S0, out, S_final, BH, T,
-                                                      dv, 0, stream);
+            return launch_chunked_bv<MODE, 32, false>(a, 0, stream);
         case 64:
-            return launch_chunked_bv<MODE, 64, false>(q, k, v, beta, gate, S0, out, S_final, BH, T,
-                                                      dv, 0, stream);
+            return launch_chunked_bv<MODE, 64, false>(a, 0, stream);
         case 128:
-            if constexpr (MODE == DR_KDA)
-                return launch_chunked_bv<MODE, 128, false>(q, k, v, beta, gate, S0, out, S_final,
-                                                           BH, T, dv, 0, stream);
+            if constexpr (MODE == DR_KDA) return launch_chunked_bv<MODE, 128, false>(a, 0, stream);
     }
     return DR_ERR_UNSUPPORTED;
 }
 
-inline int launch_chunked(const void* q, const void* k, const void* v, const float* beta,
-                          const float* gate, const float* S0, void* out, float* S_final, int BH,
-                          int T, int dk, int dv, int variant, cudaStream_t stream) {
-    (void)dk;
+inline int launch_chunked(const ChunkArgs& a, int variant, cudaStream_t stream) {
     switch (variant) {
         case DR_DELTANET:
-            return launch_chunked_mode<DR_DELTANET>(q, k, v, beta, gate, S0, out, S_final, BH, T,
-                                                    dv, stream);
+            return launch_chunked_mode<DR_DELTANET>(a, stream);
         case DR_GDN:
-            return launch_chunked_mode<DR_GDN>(q, k, v, beta, gate, S0, out, S_final, BH, T, dv,
-                                               stream);
+            return launch_chunked_mode<DR_GDN>(a, stream);
         case DR_KDA:
-            return launch_chunked_mode<DR_KDA>(q, k, v, beta, gate, S0, out, S_final, BH, T, dv,
-                                               stream);
+            return launch_chunked_mode<DR_KDA>(a, stream);
+        case DR_GDN2:
+            return launch_chunked_mode<DR_GDN2>(a, stream);
     }
     return DR_ERR_UNSUPPORTED;
 }

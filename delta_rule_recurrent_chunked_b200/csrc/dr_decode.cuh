@@ -6,6 +6,8 @@
 //     r  = v - S' k           residual against the decayed state
 //     S  = S' + beta r k^T    (plain linear attention: S = S + v k^T)
 //     o  = S q                readout after the write
+// Gated DeltaNet-2 takes e = b (.) k for k and z = w (.) v for v; u = beta r (the write
+// value) is optionally stored.
 // Rows of S are independent given (q, k, v[i], alpha, beta), so the step streams S once
 // from HBM and back: the bound is HBM bandwidth (2*dv*dk*4 bytes per head per token).
 // A warp owns 4 consecutive rows of one head; lane l holds key channels
@@ -61,8 +63,9 @@ __device__ __forceinline__ void ld_in(const TIn* p, float* x) {
 template <typename TIn, int MODE, int DK>
 __global__ void __launch_bounds__(DEC_THREADS) dr_decode_kernel(
     const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
-    const float* __restrict__ beta, const float* __restrict__ gate, const float* S_in,
-    float* S_out, TIn* __restrict__ out, long rows, int dv) {
+    const float* __restrict__ beta, const float* __restrict__ gate,
+    const float* __restrict__ erase, const float* __restrict__ write, const float* S_in,
+    float* S_out, TIn* __restrict__ out, TIn* __restrict__ u_out, long rows, int dv) {
     constexpr int EPL = DK / 32;
     const int lane = threadIdx.x & 31;
     const long r0 = ((long)blockIdx.x * DEC_WARPS + (threadIdx.x >> 5)) * DEC_ROWS;
@@ -74,10 +77,16 @@ __global__ void __launch_bounds__(DEC_THREADS) dr_decode_kernel(
     float kk[EPL], qq[EPL], a[EPL];
     ld_in<TIn, EPL>(k + bh * DK + c0, kk);
     ld_in<TIn, EPL>(q + bh * DK + c0, qq);
+    if constexpr (MODE == DR_GDN2) {
+        float eb[EPL];
+        ld_f32<EPL>(erase + bh * DK + c0, eb);
+#pragma unroll
+        for (int e = 0; e < EPL; ++e) kk[e] *= eb[e];
+    }
     if constexpr (MODE == DR_KDA) {
         ld_f32<EPL>(gate + bh * DK + c0, a);
     } else {
-        const float g = MODE == DR_GDN ? gate[bh] : 1.f;
+        const float g = (MODE == DR_GDN || MODE == DR_GDN2) ? gate[bh] : 1.f;
 #pragma unroll
         for (int e = 0; e < EPL; ++e) a[e] = g;
     }
@@ -94,6 +103,7 @@ __global__ void __launch_bounds__(DEC_THREADS) dr_decode_kernel(
             for (int e = 0; e < EPL; ++e) s[j][e] = 0.f;
         }
         vi[j] = to_f32<TIn>(v[bh * dv + i0 + j]);
+        if constexpr (MODE == DR_GDN2) vi[j] *= write[bh * dv + i0 + j];
     }
     // prediction (S' k)_i, reduced over the warp for the four rows at once
     float p[DEC_ROWS];
@@ -115,10 +125,11 @@ __global__ void __launch_bounds__(DEC_THREADS) dr_decode_kernel(
             for (int j = 0; j < DEC_ROWS; ++j) p[j] += __shfl_xor_sync(0xffffffffu, p[j], off);
     }
     // write, then the readout (S q)_i
-    float o[DEC_ROWS];
+    float o[DEC_ROWS], u[DEC_ROWS];
 #pragma unroll
     for (int j = 0; j < DEC_ROWS; ++j) {
         const float w = MODE == DR_LINEAR ? vi[j] : b * (vi[j] - p[j]);
+        u[j] = w;
         o[j] = 0.f;
 #pragma unroll
         for (int e = 0; e < EPL; ++e) {
@@ -135,10 +146,14 @@ __global__ void __launch_bounds__(DEC_THREADS) dr_decode_kernel(
         for (int j = 0; j < DEC_ROWS; ++j) st_f32<EPL>(S_out + (r0 + j) * DK + c0, s[j]);
     }
     if (lane < DEC_ROWS) {
-        float oj = o[0];
+        float oj = o[0], uj = u[0];
 #pragma unroll
-        for (int j = 1; j < DEC_ROWS; ++j) oj = lane == j ? o[j] : oj;
+        for (int j = 1; j < DEC_ROWS; ++j) {
+            oj = lane == j ? o[j] : oj;
+            uj = lane == j ? u[j] : uj;
+        }
         out[bh * dv + i0 + lane] = from_f32<TIn>(oj);
+        if (u_out) u_out[bh * dv + i0 + lane] = from_f32<TIn>(uj);
     }
 }
 

@@ -2,9 +2,11 @@
 //
 // Every row of S evolves independently given (k_t, alpha_t, beta_t): with
 // S' = S_{t-1} diag(a_t), row i of the update is
-//     s_i <- a (.) s_i + beta_t (v_t[i] - (a (.) s_i) . k_t) k_t
-// and o_t[i] = s_i . q_t (readout after the write). One thread owns one row of S in
-// registers, so a token costs ~4*dk FMAs per thread and no cross-thread communication.
+//     s_i <- a (.) s_i + u_t[i] k_t,   u_t[i] = beta_t (v_t[i] - (a (.) s_i) . k_t)
+// and o_t[i] = s_i . q_t (readout after the write). Gated DeltaNet-2 runs the same rows
+// with k_t replaced by its erase direction e_t = b_t (.) k_t and v_t by its write target
+// z_t = w_t (.) v_t. The write values u_t are optionally stored. One thread owns one row of
+// S in registers, so a token costs ~4*dk FMAs per thread and no cross-thread communication.
 // A CTA is one warp covering 32 consecutive rows (value channels) of one (b,h); tokens
 // are staged through shared memory in tiles and broadcast to the warp.
 #pragma once
@@ -41,8 +43,11 @@ __device__ __forceinline__ __nv_bfloat16 from_f32<__nv_bfloat16>(float x) {
 template <typename TIn, int MODE, int DK>
 __global__ void __launch_bounds__(32) dr_sequential_kernel(
     const TIn* __restrict__ q, const TIn* __restrict__ k, const TIn* __restrict__ v,
-    const float* __restrict__ beta, const float* __restrict__ gate, const float* __restrict__ S0,
-    TIn* __restrict__ out, float* __restrict__ S_final, int T, int dv) {
+    const float* __restrict__ beta, const float* __restrict__ gate,
+    const float* __restrict__ erase, const float* __restrict__ write,
+    const float* __restrict__ S0, TIn* __restrict__ out, float* __restrict__ S_final,
+    TIn* __restrict__ u_out, int T, int dv) {
+    constexpr bool kScalarGate = MODE == DR_GDN || MODE == DR_GDN2;
     __shared__ __align__(16) float sk[SEQ_TILE][DK];
     __shared__ __align__(16) float sq[SEQ_TILE][DK];
     __shared__ __align__(16) float sa[MODE == DR_KDA ? SEQ_TILE : 1][MODE == DR_KDA ? DK : 4];
@@ -58,6 +63,7 @@ __global__ void __launch_bounds__(32) dr_sequential_kernel(
     const TIn* kh = k + bh * (long)T * DK;
     const TIn* vh = v + bh * (long)T * dv;
     TIn* oh = out + bh * (long)T * dv;
+    TIn* uh = u_out ? u_out + bh * (long)T * dv : nullptr;
 
     float s[DK];
     if (S0) {
@@ -80,14 +86,20 @@ __global__ void __launch_bounds__(32) dr_sequential_kernel(
         __syncwarp();
         for (int e = lane; e < nt * DK; e += 32) {
             const int tt = e / DK, j = e % DK;
+            const long kt = (bh * T + t0 + tt) * (long)DK + j;
             sk[tt][j] = to_f32(kh[(long)(t0 + tt) * DK + j]);
+            if constexpr (MODE == DR_GDN2) sk[tt][j] *= erase[kt];  // e = b (.) k
             sq[tt][j] = to_f32(qh[(long)(t0 + tt) * DK + j]);
-            if constexpr (MODE == DR_KDA) sa[tt][j] = gate[(bh * T + t0 + tt) * (long)DK + j];
+            if constexpr (MODE == DR_KDA) sa[tt][j] = gate[kt];
         }
-        for (int tt = 0; tt < nt; ++tt) sv[tt][lane] = to_f32(vh[(long)(t0 + tt) * dv + row]);
+        for (int tt = 0; tt < nt; ++tt) {
+            float x = to_f32(vh[(long)(t0 + tt) * dv + row]);
+            if constexpr (MODE == DR_GDN2) x *= write[(bh * T + t0 + tt) * (long)dv + row];  // z
+            sv[tt][lane] = x;
+        }
         if (lane < nt) {
             sb[lane] = (MODE == DR_LINEAR) ? 1.f : beta[bh * T + t0 + lane];
-            sg[lane] = (MODE == DR_GDN) ? gate[bh * T + t0 + lane] : 1.f;
+            sg[lane] = kScalarGate ? gate[bh * T + t0 + lane] : 1.f;
         }
         __syncwarp();
 
@@ -96,8 +108,9 @@ __global__ void __launch_bounds__(32) dr_sequential_kernel(
             if constexpr (MODE == DR_LINEAR) {
 #pragma unroll
                 for (int j = 0; j < DK; ++j) s[j] = fmaf(vi, sk[tt][j], s[j]);
+                if (uh) uh[(long)(t0 + tt) * dv + row] = from_f32<TIn>(vi);
             } else {
-                if constexpr (MODE == DR_GDN) {
+                if constexpr (kScalarGate) {
                     const float a = sg[tt];
 #pragma unroll
                     for (int j = 0; j < DK; ++j) s[j] *= a;
@@ -114,6 +127,7 @@ __global__ void __launch_bounds__(32) dr_sequential_kernel(
                 const float w = sb[tt] * (vi - (p0 + p1));
 #pragma unroll
                 for (int j = 0; j < DK; ++j) s[j] = fmaf(w, sk[tt][j], s[j]);
+                if (uh) uh[(long)(t0 + tt) * dv + row] = from_f32<TIn>(w);
             }
             float o0 = 0.f, o1 = 0.f;
 #pragma unroll

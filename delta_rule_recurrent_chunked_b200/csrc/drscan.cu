@@ -10,6 +10,7 @@
 #include "dr_chunked.cuh"
 #include "dr_decode.cuh"
 #include "dr_sequential.cuh"
+#include "loglinear.cuh"
 #include "vla_sequential.cuh"
 
 using namespace drscan;
@@ -28,97 +29,93 @@ int launch_status() {
     return e == cudaSuccess ? DR_OK : DR_ERR_CUDA;
 }
 
+// Arguments of a decode step (device pointers as dr_decode_step_ex receives them).
+struct DecodeArgs {
+    const void *q, *k, *v;
+    const float *beta, *gate, *erase, *write;
+    float* S;
+    void *out, *u_out;
+    long rows;
+    int dv;
+};
+
 template <typename TIn, int MODE, int DK>
-int launch_decode(const void* q, const void* k, const void* v, const float* beta, const float* gate,
-                  float* S, void* out, long rows, int dv, cudaStream_t stream) {
+int launch_decode(const DecodeArgs& a, cudaStream_t stream) {
     constexpr long per_cta = (long)DEC_ROWS * DEC_WARPS;
-    dr_decode_kernel<TIn, MODE, DK><<<(unsigned)((rows + per_cta - 1) / per_cta), DEC_THREADS, 0,
-                                       stream>>>(
-        static_cast<const TIn*>(q), static_cast<const TIn*>(k), static_cast<const TIn*>(v), beta,
-        gate, S, S, static_cast<TIn*>(out), rows, dv);
+    dr_decode_kernel<TIn, MODE, DK><<<(unsigned)((a.rows + per_cta - 1) / per_cta), DEC_THREADS,
+                                       0, stream>>>(
+        static_cast<const TIn*>(a.q), static_cast<const TIn*>(a.k), static_cast<const TIn*>(a.v),
+        a.beta, a.gate, a.erase, a.write, a.S, a.S, static_cast<TIn*>(a.out),
+        static_cast<TIn*>(a.u_out), a.rows, a.dv);
     return launch_status();
 }
 
 template <typename TIn, int MODE>
-int dispatch_decode_dk(const void* q, const void* k, const void* v, const float* beta,
-                       const float* gate, float* S, void* out, long rows, int dk, int dv,
-                       cudaStream_t stream) {
+int dispatch_decode_dk(const DecodeArgs& a, int dk, cudaStream_t stream) {
     switch (dk) {
         case 32:
-            return launch_decode<TIn, MODE, 32>(q, k, v, beta, gate, S, out, rows, dv, stream);
+            return launch_decode<TIn, MODE, 32>(a, stream);
         case 64:
-            return launch_decode<TIn, MODE, 64>(q, k, v, beta, gate, S, out, rows, dv, stream);
+            return launch_decode<TIn, MODE, 64>(a, stream);
         case 128:
-            return launch_decode<TIn, MODE, 128>(q, k, v, beta, gate, S, out, rows, dv, stream);
+            return launch_decode<TIn, MODE, 128>(a, stream);
     }
     return DR_ERR_UNSUPPORTED;
 }
 
 template <typename TIn>
-int dispatch_decode(const void* q, const void* k, const void* v, const float* beta,
-                    const float* gate, float* S, void* out, long rows, int dk, int dv, int variant,
-                    cudaStream_t stream) {
+int dispatch_decode(const DecodeArgs& a, int dk, int variant, cudaStream_t stream) {
     switch (variant) {
         case DR_LINEAR:
-            return dispatch_decode_dk<TIn, DR_LINEAR>(q, k, v, beta, gate, S, out, rows, dk, dv,
-                                                      stream);
+            return dispatch_decode_dk<TIn, DR_LINEAR>(a, dk, stream);
         case DR_DELTANET:
-            return dispatch_decode_dk<TIn, DR_DELTANET>(q, k, v, beta, gate, S, out, rows, dk, dv,
-                                                        stream);
+            return dispatch_decode_dk<TIn, DR_DELTANET>(a, dk, stream);
         case DR_GDN:
-            return dispatch_decode_dk<TIn, DR_GDN>(q, k, v, beta, gate, S, out, rows, dk, dv, stream);
+            return dispatch_decode_dk<TIn, DR_GDN>(a, dk, stream);
         case DR_KDA:
-            return dispatch_decode_dk<TIn, DR_KDA>(q, k, v, beta, gate, S, out, rows, dk, dv, stream);
+            return dispatch_decode_dk<TIn, DR_KDA>(a, dk, stream);
+        case DR_GDN2:
+            return dispatch_decode_dk<TIn, DR_GDN2>(a, dk, stream);
     }
     return DR_ERR_INVALID_ARG;
 }
 
 template <typename TIn, int MODE, int DK>
-int launch_sequential(const void* q, const void* k, const void* v, const float* beta,
-                      const float* gate, const float* S0, void* out, float* S_final, long BH,
-                      int T, int dv, cudaStream_t stream) {
-    dim3 grid((unsigned)BH, (unsigned)(dv / 32));
+int launch_sequential(const ChunkArgs& a, cudaStream_t stream) {
+    dim3 grid((unsigned)a.BH, (unsigned)(a.dv / 32));
     dr_sequential_kernel<TIn, MODE, DK><<<grid, 32, 0, stream>>>(
-        static_cast<const TIn*>(q), static_cast<const TIn*>(k), static_cast<const TIn*>(v), beta,
-        gate, S0, static_cast<TIn*>(out), S_final, T, dv);
+        static_cast<const TIn*>(a.q), static_cast<const TIn*>(a.k), static_cast<const TIn*>(a.v),
+        a.beta, a.gate, a.erase, a.write, a.S0, static_cast<TIn*>(a.out), a.S_final,
+        static_cast<TIn*>(a.u_out), a.T, a.dv);
     return launch_status();
 }
 
 template <typename TIn, int MODE>
-int dispatch_sequential_dk(const void* q, const void* k, const void* v, const float* beta,
-                           const float* gate, const float* S0, void* out, float* S_final, long BH,
-                           int T, int dk, int dv, cudaStream_t stream) {
+int dispatch_sequential_dk(const ChunkArgs& a, int dk, cudaStream_t stream) {
     switch (dk) {
         case 32:
-            return launch_sequential<TIn, MODE, 32>(q, k, v, beta, gate, S0, out, S_final, BH, T,
-                                                    dv, stream);
+            return launch_sequential<TIn, MODE, 32>(a, stream);
         case 64:
-            return launch_sequential<TIn, MODE, 64>(q, k, v, beta, gate, S0, out, S_final, BH, T,
-                                                    dv, stream);
+            return launch_sequential<TIn, MODE, 64>(a, stream);
         case 128:
-            return launch_sequential<TIn, MODE, 128>(q, k, v, beta, gate, S0, out, S_final, BH, T,
-                                                     dv, stream);
+            return launch_sequential<TIn, MODE, 128>(a, stream);
     }
     return DR_ERR_UNSUPPORTED;
 }
 
 template <typename TIn>
-int dispatch_sequential(const void* q, const void* k, const void* v, const float* beta,
-                        const float* gate, const float* S0, void* out, float* S_final, long BH,
-                        int T, int dk, int dv, int variant, cudaStream_t stream) {
+int dispatch_sequential(const ChunkArgs& a, int dk, int variant, cudaStream_t stream) {
     switch (variant) {
         case DR_LINEAR:
-            return dispatch_sequential_dk<TIn, DR_LINEAR>(q, k, v, beta, gate, S0, out, S_final,
-                                                          BH, T, dk, dv, stream);
+            return dispatch_sequential_dk<TIn, DR_LINEAR>(a, dk, stream);
         case DR_DELTANET:
-            return dispatch_sequential_dk<TIn, DR_DELTANET>(q, k, v, beta, gate, S0, out, S_final,
-                                                            BH, T, dk, dv, stream);
+            return dispatch_sequential_dk<TIn, DR_DELTANET>(a, dk, stream);
         case DR_GDN:
-            return dispatch_sequential_dk<TIn, DR_GDN>(q, k, v, beta, gate, S0, out, S_final, BH,
-                                                       T, dk, dv, stream);
+            return dispatch_sequential_dk<TIn, DR_GDN>(a, dk, stream);
         case DR_KDA:
-            return dispatch_sequential_dk<TIn, DR_KDA>(q, k, v, beta, gate, S0, out, S_final, BH,
-                                                       T, dk, dv, stream);
+            return dispatch_sequential_dk<TIn, DR_KDA>(a, dk, stream);
+        case DR_GDN2:
+            return dispatch_sequential_dk<TIn, DR_GDN2>(a, dk, stream);
     }
     return DR_ERR_INVALID_ARG;
 }
@@ -140,17 +137,30 @@ __global__ void scaled_identity_kernel(float* A, int d, long count, float diag) 
     }
 }
 
-template <int D>
+template <int D, bool RATIO>
 int launch_vla(const float* q, const float* k, const float* v, const float* u, const float* S0,
-               const float* A0, float lambda0, float* out, float* S_final, float* A_final,
-               long BH, int T, cudaStream_t stream) {
+               const float* A0, const float* n0, float lambda0, float* out, float* S_final,
+               float* A_final, float* n_final, long BH, int T, cudaStream_t stream) {
     const int smem = (int)sizeof(VlaSmem<D>);
-    if (cudaFuncSetAttribute(vla_sequential_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             smem) != cudaSuccess)
+    auto kern = vla_sequential_kernel<D, RATIO>;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
         return DR_ERR_CUDA;
-    vla_sequential_kernel<D><<<(unsigned)BH, 2 * D, smem, stream>>>(
-        q, k, v, u, S0, A0, lambda0, out, S_final, A_final, T);
+    kern<<<(unsigned)BH, 2 * D, smem, stream>>>(q, k, v, u, S0, A0, n0, lambda0, out, S_final,
+                                                A_final, n_final, T);
     return launch_status();
+}
+
+template <int D>
+int launch_vla_readout(bool ratio, const float* q, const float* k, const float* v,
+                       const float* u, const float* S0, const float* A0, const float* n0,
+                       float lambda0, float* out, float* S_final, float* A_final, float* n_final,
+                       long BH, int T, cudaStream_t stream) {
+    if (ratio)
+        return launch_vla<D, true>(q, k, v, u, S0, A0, n0, lambda0, out, S_final, A_final,
+                                   n_final, BH, T, stream);
+    return launch_vla<D, false>(q, k, v, u, S0, A0, nullptr, lambda0, out, S_final, A_final,
+                                nullptr, BH, T, stream);
 }
 
 __global__ void timeout_probe_kernel(int spin_limit) {
@@ -188,79 +198,107 @@ const char* dr_status_string(int status) {
             return "device: a bounded barrier wait ran out; outputs are invalid";
         case DR_ERR_DEVICE_BOUNDS:
             return "device: an index check failed; outputs are invalid";
+        case DR_ERR_GATE_RANGE:
+            return "device: a KDA gate's summed log-decay over one chunk is below the chunked "
+                   "kernel's range; outputs are invalid (rerun with DR_FORCE_SEQUENTIAL)";
     }
     return "unknown status";
 }
 
-int dr_scan_fwd(const void* q, const void* k, const void* v, const float* beta, const float* gate,
-                const float* S0, void* out, float* S_final, int B, int H, int T, int dk, int dv,
-                int mode, cudaStream_t stream) {
+int dr_scan_fwd_ex(const void* q, const void* k, const void* v, const float* beta,
+                   const float* gate, const float* erase, const float* write, const float* S0,
+                   void* out, float* S_final, void* u_out, int B, int H, int T, int dk, int dv,
+                   int mode, cudaStream_t stream) {
     const int variant = mode & DR_MODE_MASK;
     if (mode & ~(DR_MODE_MASK | DR_IN_BF16 | DR_FORCE_SEQUENTIAL)) return DR_ERR_INVALID_ARG;
-    if (variant > DR_KDA) return DR_ERR_INVALID_ARG;
+    if (variant > DR_GDN2) return DR_ERR_INVALID_ARG;
     if (B < 0 || H < 0 || T < 0 || dk <= 0 || dv <= 0) return DR_ERR_INVALID_ARG;
     const long BH = (long)B * (long)H;
     if (BH > INT_MAX) return DR_ERR_INVALID_ARG;
+    const bool gated = variant == DR_GDN || variant == DR_KDA || variant == DR_GDN2;
     // per-token tensors are read only when there are tokens (empty tensors may be NULL)
     const bool tokens = BH > 0 && T > 0;
     if (tokens && (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(out)))
         return DR_ERR_INVALID_ARG;
     if (tokens && variant != DR_LINEAR && !ok_ptr(beta)) return DR_ERR_INVALID_ARG;
-    if (tokens && (variant == DR_GDN || variant == DR_KDA) && !ok_ptr(gate))
+    if (tokens && gated && !ok_ptr(gate)) return DR_ERR_INVALID_ARG;
+    if (tokens && variant == DR_GDN2 && (!ok_ptr(erase) || !ok_ptr(write)))
         return DR_ERR_INVALID_ARG;
     if (!ok_opt(q) || !ok_opt(k) || !ok_opt(v) || !ok_opt(out) || !ok_opt(beta) ||
-        !ok_opt(gate) || !ok_opt(S0) || !ok_opt(S_final))
+        !ok_opt(gate) || !ok_opt(erase) || !ok_opt(write) || !ok_opt(S0) ||
+        !ok_opt(S_final) || !ok_opt(u_out))
         return DR_ERR_INVALID_ARG;
     if (!dim_supported(dk) || !dim_supported(dv)) return DR_ERR_UNSUPPORTED;
     if (BH == 0) return DR_OK;
     if (T == 0) return copy_state(S_final, S0, (size_t)BH * dv * dk, stream);
 
     const bool bf16 = (mode & DR_IN_BF16) != 0;
-    if (variant == DR_LINEAR) beta = nullptr;
-    if (variant == DR_LINEAR || variant == DR_DELTANET) gate = nullptr;
+    ChunkArgs a{q, k, v, variant == DR_LINEAR ? nullptr : beta, gated ? gate : nullptr,
+                variant == DR_GDN2 ? erase : nullptr, variant == DR_GDN2 ? write : nullptr,
+                S0, out, S_final, u_out, (int)BH, T, dv};
     if (bf16 && !(mode & DR_FORCE_SEQUENTIAL) && chunked_supported(variant, dk, dv))
-        return launch_chunked(q, k, v, beta, gate, S0, out, S_final, (int)BH, T, dk, dv, variant,
-                              stream);
-    if (bf16)
-        return dispatch_sequential<__nv_bfloat16>(q, k, v, beta, gate, S0, out, S_final, BH, T, dk,
-                                                  dv, variant, stream);
-    return dispatch_sequential<float>(q, k, v, beta, gate, S0, out, S_final, BH, T, dk, dv,
-                                      variant, stream);
+        return launch_chunked(a, variant, stream);
+    if (bf16) return dispatch_sequential<__nv_bfloat16>(a, dk, variant, stream);
+    return dispatch_sequential<float>(a, dk, variant, stream);
 }
 
-int dr_decode_step(const void* q, const void* k, const void* v, const float* beta,
-                   const float* gate, float* S, void* out, int B, int H, int dk, int dv, int mode,
-                   cudaStream_t stream) {
+int dr_scan_fwd(const void* q, const void* k, const void* v, const float* beta, const float* gate,
+                const float* S0, void* out, float* S_final, int B, int H, int T, int dk, int dv,
+                int mode, cudaStream_t stream) {
+    // Gated DeltaNet-2 needs its erase and write gates: only dr_scan_fwd_ex takes them
+    if ((mode & DR_MODE_MASK) == DR_GDN2) return DR_ERR_INVALID_ARG;
+    return dr_scan_fwd_ex(q, k, v, beta, gate, nullptr, nullptr, S0, out, S_final, nullptr, B, H,
+                          T, dk, dv, mode, stream);
+}
+
+int dr_decode_step_ex(const void* q, const void* k, const void* v, const float* beta,
+                      const float* gate, const float* erase, const float* write, float* S,
+                      void* out, void* u_out, int B, int H, int dk, int dv, int mode,
+                      cudaStream_t stream) {
     const int variant = mode & DR_MODE_MASK;
     if (mode & ~(DR_MODE_MASK | DR_IN_BF16)) return DR_ERR_INVALID_ARG;
-    if (variant > DR_KDA) return DR_ERR_INVALID_ARG;
+    if (variant > DR_GDN2) return DR_ERR_INVALID_ARG;
     if (B < 0 || H < 0 || dk <= 0 || dv <= 0) return DR_ERR_INVALID_ARG;
     const long BH = (long)B * (long)H;
     if (BH > INT_MAX) return DR_ERR_INVALID_ARG;
+    const bool gated = variant == DR_GDN || variant == DR_KDA || variant == DR_GDN2;
     if (!ok_opt(q) || !ok_opt(k) || !ok_opt(v) || !ok_opt(out) || !ok_opt(beta) ||
-        !ok_opt(gate) || !ok_opt(S))
+        !ok_opt(gate) || !ok_opt(erase) || !ok_opt(write) || !ok_opt(S) || !ok_opt(u_out))
         return DR_ERR_INVALID_ARG;
     if (BH > 0) {
         if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(out) || !ok_ptr(S))
             return DR_ERR_INVALID_ARG;
         if (variant != DR_LINEAR && !ok_ptr(beta)) return DR_ERR_INVALID_ARG;
-        if ((variant == DR_GDN || variant == DR_KDA) && !ok_ptr(gate)) return DR_ERR_INVALID_ARG;
+        if (gated && !ok_ptr(gate)) return DR_ERR_INVALID_ARG;
+        if (variant == DR_GDN2 && (!ok_ptr(erase) || !ok_ptr(write))) return DR_ERR_INVALID_ARG;
     }
     if (!dim_supported(dk) || !dim_supported(dv)) return DR_ERR_UNSUPPORTED;
     if (BH == 0) return DR_OK;
     const long rows = BH * dv;
     if (rows / ((long)DEC_ROWS * DEC_WARPS) >= INT_MAX) return DR_ERR_UNSUPPORTED;
-    if (variant == DR_LINEAR) beta = nullptr;
-    if (variant == DR_LINEAR || variant == DR_DELTANET) gate = nullptr;
-    if (mode & DR_IN_BF16)
-        return dispatch_decode<__nv_bfloat16>(q, k, v, beta, gate, S, out, rows, dk, dv, variant,
-                                              stream);
-    return dispatch_decode<float>(q, k, v, beta, gate, S, out, rows, dk, dv, variant, stream);
+    DecodeArgs a{q, k, v, variant == DR_LINEAR ? nullptr : beta, gated ? gate : nullptr,
+                 variant == DR_GDN2 ? erase : nullptr, variant == DR_GDN2 ? write : nullptr, S,
+                 out, u_out, rows, dv};
+    if (mode & DR_IN_BF16) return dispatch_decode<__nv_bfloat16>(a, dk, variant, stream);
+    return dispatch_decode<float>(a, dk, variant, stream);
 }
 
-int vla_scan_fwd(const float* q, const float* k, const float* v, const float* u, const float* S0,
-                 const float* A0, float lambda0, float* out, float* S_final, float* A_final, int B,
-                 int H, int T, int d, cudaStream_t stream) {
+int dr_decode_step(const void* q, const void* k, const void* v, const float* beta,
+                   const float* gate, float* S, void* out, int B, int H, int dk, int dv, int mode,
+                   cudaStream_t stream) {
+    if ((mode & DR_MODE_MASK) == DR_GDN2) return DR_ERR_INVALID_ARG;
+    return dr_decode_step_ex(q, k, v, beta, gate, nullptr, nullptr, S, out, nullptr, B, H, dk, dv,
+                             mode, stream);
+}
+
+int vla_scan_fwd_ex(const float* q, const float* k, const float* v, const float* u,
+                    const float* S0, const float* A0, const float* n0, float lambda0, float* out,
+                    float* S_final, float* A_final, float* n_final, int B, int H, int T, int d,
+                    int flags, cudaStream_t stream) {
+    if (flags & ~VLA_RATIO_READOUT) return DR_ERR_INVALID_ARG;
+    const bool ratio = (flags & VLA_RATIO_READOUT) != 0;
+    if (!ratio && (n0 || n_final)) return DR_ERR_INVALID_ARG;
+    if (!ok_opt(n0) || !ok_opt(n_final)) return DR_ERR_INVALID_ARG;
     if (B < 0 || H < 0 || T < 0 || d <= 0) return DR_ERR_INVALID_ARG;
     const long BH = (long)B * (long)H;
     if (BH > INT_MAX) return DR_ERR_INVALID_ARG;
@@ -276,6 +314,7 @@ int vla_scan_fwd(const float* q, const float* k, const float* v, const float* u,
     if (T == 0) {
         const size_t n = (size_t)BH * d * d;
         int rc = copy_state(S_final, S0, n, stream);
+        if (rc == DR_OK && ratio) rc = copy_state(n_final, n0, (size_t)BH * d, stream);
         if (rc != DR_OK || !A_final) return rc;
         if (A0) return copy_state(A_final, A0, n, stream);
         scaled_identity_kernel<<<(unsigned)((n + 255) / 256), 256, 0, stream>>>(A_final, d, (long)n,
@@ -284,19 +323,62 @@ int vla_scan_fwd(const float* q, const float* k, const float* v, const float* u,
     }
     switch (d) {
         case 32:
-            return launch_vla<32>(q, k, v, u, S0, A0, lambda0, out, S_final, A_final, BH, T,
-                                  stream);
+            return launch_vla_readout<32>(ratio, q, k, v, u, S0, A0, n0, lambda0, out, S_final,
+                                          A_final, n_final, BH, T, stream);
         case 64:
-            return launch_vla<64>(q, k, v, u, S0, A0, lambda0, out, S_final, A_final, BH, T,
-                                  stream);
+            return launch_vla_readout<64>(ratio, q, k, v, u, S0, A0, n0, lambda0, out, S_final,
+                                          A_final, n_final, BH, T, stream);
         case 96:
-            return launch_vla<96>(q, k, v, u, S0, A0, lambda0, out, S_final, A_final, BH, T,
-                                  stream);
+            return launch_vla_readout<96>(ratio, q, k, v, u, S0, A0, n0, lambda0, out, S_final,
+                                          A_final, n_final, BH, T, stream);
         case 128:
-            return launch_vla<128>(q, k, v, u, S0, A0, lambda0, out, S_final, A_final, BH, T,
-                                   stream);
+            return launch_vla_readout<128>(ratio, q, k, v, u, S0, A0, n0, lambda0, out, S_final,
+                                           A_final, n_final, BH, T, stream);
     }
     return DR_ERR_UNSUPPORTED;
+}
+
+int vla_scan_fwd(const float* q, const float* k, const float* v, const float* u, const float* S0,
+                 const float* A0, float lambda0, float* out, float* S_final, float* A_final, int B,
+                 int H, int T, int d, cudaStream_t stream) {
+    return vla_scan_fwd_ex(q, k, v, u, S0, A0, nullptr, lambda0, out, S_final, A_final, nullptr,
+                           B, H, T, d, 0, stream);
+}
+
+int loglinear_scan_fwd(const void* q, const void* k, const void* v, const float* lambda,
+                       void* out, int B, int H, int T, int dk, int dv, int L, int mode,
+                       cudaStream_t stream) {
+    if (mode & ~DR_IN_BF16) return DR_ERR_INVALID_ARG;
+    if (B < 0 || H < 0 || T < 0 || dk <= 0 || dv <= 0 || L < 1) return DR_ERR_INVALID_ARG;
+    const long BH = (long)B * (long)H;
+    if (BH > INT_MAX) return DR_ERR_INVALID_ARG;
+    // every position needs its level: level 0 plus one per bit of T - 1
+    int need = 1;
+    while (need < 31 && ((long)(T > 0 ? T - 1 : 0) >> (need - 1)) > 0) ++need;
+    if (L < need) return DR_ERR_INVALID_ARG;
+    const bool tokens = BH > 0 && T > 0;
+    if (tokens && (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(lambda) || !ok_ptr(out)))
+        return DR_ERR_INVALID_ARG;
+    if (!ok_opt(q) || !ok_opt(k) || !ok_opt(v) || !ok_opt(lambda) || !ok_opt(out))
+        return DR_ERR_INVALID_ARG;
+    if (!(mode & DR_IN_BF16) || dk != LL_DK || (dv != 32 && dv != 64 && dv != 128) ||
+        L > LL_LMAX || (long)T > (long)LL_C << LL_LEVELS)
+        return DR_ERR_UNSUPPORTED;
+    if (!tokens) return DR_OK;
+    const int smem = (int)sizeof(LoglinearSmem);
+    static bool attr_set[16] = {};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return DR_ERR_CUDA;
+    if (dev < 0 || dev >= 16 || !attr_set[dev]) {
+        if (cudaFuncSetAttribute(loglinear_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 smem) != cudaSuccess)
+            return DR_ERR_CUDA;
+        if (dev >= 0 && dev < 16) attr_set[dev] = true;
+    }
+    loglinear_kernel<<<dim3((unsigned)BH, (unsigned)(dv / LL_BV)), LL_THREADS, smem, stream>>>(
+        static_cast<const __nv_bfloat16*>(q), static_cast<const __nv_bfloat16*>(k),
+        static_cast<const __nv_bfloat16*>(v), lambda, static_cast<__nv_bfloat16*>(out), T, dv, L);
+    return launch_status();
 }
 
 int dr_poll_error(cudaStream_t stream) {
@@ -311,6 +393,7 @@ int dr_poll_error(cudaStream_t stream) {
 }
 
 int dr_chunked_plan(int mode, long long BH, int dk, int dv, int* bv, int* nprep) {
+    if ((mode & DR_MODE_MASK) > DR_GDN2) return DR_ERR_INVALID_ARG;
     if (!bv || !nprep) return DR_ERR_INVALID_ARG;
     *bv = 0;
     *nprep = 0;

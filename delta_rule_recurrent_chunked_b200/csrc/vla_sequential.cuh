@@ -3,13 +3,21 @@
 // Two thread groups of d threads each:
 //  * the A-group owns A (row i in thread i's registers) and produces the write direction
 //    alpha_hat_t for every token: z = A_{t-1} u and y = A_{t-1} k in one pass over the row,
-//    two group reductions (u.z and k.z), then A_t k = y - z (z.k)/(1 + u.z) (Sherman-Morrison
-//    applied to the vector, so no second dependent mat-vec), a third reduction for the
-//    norm, and the rank-1 update of A's row;
+//    then ONE group reduction of u.z, k.z, y.y, y.z and z.z. With c = 1/(1 + u.z) and
+//    w = c (k.z), A_t k = y - w z (Sherman-Morrison applied to the vector, so no second
+//    dependent mat-vec) and ||A_t k||^2 = y.y - 2 w y.z + w^2 z.z, so the norm needs no
+//    reduction of its own; then the rank-1 update of A's row;
 //  * the S-group owns S (row i in thread i's registers); given alpha_hat_t its rows are
 //    independent: r_i = v_i - s_i.k, s_i += r_i alpha_hat, o_i = s_i.q. No reductions.
 // The groups run one token tile apart: while the A-group produces the directions of tile n
 // into a shared-memory ring, the S-group consumes tile n-1. One __syncthreads per tile.
+//
+// Ratio readout (RATIO): o_t = S_t q_t / (n_t q_t) with n_t = n_{t-1} + (1 - n_{t-1} k_t)
+// alpha_hat_t^T, the same write applied to a value held at 1. The A-group keeps n (element i
+// in thread i) and computes the denominator without another serial reduction: n.k, n.q,
+// y.q and z.q join the first reduction, and with c = 1/(1 + u.z),
+//     alpha_hat.q = (y.q - c (k.z)(z.q)) / ||A_t k||,   n_t q = n.q + (1 - n.k) alpha_hat.q.
+// The denominator rides in the ring next to alpha_hat; the S-group divides its readout.
 #pragma once
 
 #include "common.cuh"
@@ -22,52 +30,41 @@ template <int D>
 struct VlaSmem {
     float uA[2][VLA_TILE][D];
     float kA[2][VLA_TILE][D];
+    float qA[2][VLA_TILE][D];  // ratio readout: the A-group's copy of q
     float kS[2][VLA_TILE][D];
     float vS[2][VLA_TILE][D];
     float qS[2][VLA_TILE][D];
     float ring[2][VLA_TILE][D];
-    float zbuf[D];
-    float red1[2][4];
-    float red2[4];
+    float den[2][VLA_TILE];    // ratio readout: n_t q_t
+    // alternate tokens use alternate buffers: a token's writes never meet a slower thread's
+    // reads of the previous token (one group barrier per token separates them)
+    float zbuf[2][D];
+    float red1[2][9][4];
 };
 
-template <int D>
-__device__ __forceinline__ void vla_group_sum2(float& x, float& y, float (*red)[4], int i) {
+// Sums N values over the D threads of a group (warp shuffles, then one named barrier to
+// join the warps when D > 32); every thread gets the N totals.
+template <int D, int N>
+__device__ __forceinline__ void vla_group_sum(float* x, float (*red)[4], int i) {
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-        x += __shfl_xor_sync(0xffffffffu, x, off);
-        y += __shfl_xor_sync(0xffffffffu, y, off);
-    }
+    for (int off = 16; off > 0; off >>= 1)
+#pragma unroll
+        for (int e = 0; e < N; ++e) x[e] += __shfl_xor_sync(0xffffffffu, x[e], off);
     if constexpr (D > 32) {
         if ((i & 31) == 0) {
-            red[0][i >> 5] = x;
-            red[1][i >> 5] = y;
+#pragma unroll
+            for (int e = 0; e < N; ++e) red[e][i >> 5] = x[e];
         }
         asm volatile("bar.sync 1, %0;" ::"n"(D) : "memory");
-        x = 0.f;
-        y = 0.f;
 #pragma unroll
-        for (int w = 0; w < D / 32; ++w) {
-            x += red[0][w];
-            y += red[1][w];
+        for (int e = 0; e < N; ++e) {
+            x[e] = 0.f;
+#pragma unroll
+            for (int w = 0; w < D / 32; ++w) x[e] += red[e][w];
         }
     } else {
         __syncwarp();
     }
-}
-
-template <int D>
-__device__ __forceinline__ float vla_group_sum1(float x, float* red, int i) {
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
-    if constexpr (D > 32) {
-        if ((i & 31) == 0) red[i >> 5] = x;
-        asm volatile("bar.sync 1, %0;" ::"n"(D) : "memory");
-        x = 0.f;
-#pragma unroll
-        for (int w = 0; w < D / 32; ++w) x += red[w];
-    }
-    return x;
 }
 
 template <int D>
@@ -78,12 +75,13 @@ __device__ __forceinline__ void vla_load_tile(float (*dst)[D], const float* src,
 }
 
 // grid: B*H; block: 2*D threads; dynamic shared memory: sizeof(VlaSmem<D>).
-template <int D>
+template <int D, bool RATIO>
 __global__ void __launch_bounds__(2 * D) vla_sequential_kernel(
     const float* __restrict__ q, const float* __restrict__ k, const float* __restrict__ v,
     const float* __restrict__ u, const float* __restrict__ S0, const float* __restrict__ A0,
-    float lambda0, float* __restrict__ out, float* __restrict__ S_final,
-    float* __restrict__ A_final, int T) {
+    const float* __restrict__ n0, float lambda0, float* __restrict__ out,
+    float* __restrict__ S_final, float* __restrict__ A_final, float* __restrict__ n_final,
+    int T) {
     extern __shared__ __align__(16) unsigned char vla_smem_raw[];
     VlaSmem<D>& sm = *reinterpret_cast<VlaSmem<D>*>(vla_smem_raw);
 
@@ -96,7 +94,9 @@ __global__ void __launch_bounds__(2 * D) vla_sequential_kernel(
     const int ntiles = (T + VLA_TILE - 1) / VLA_TILE;
 
     float m[D];  // row i of A (A-group) or of S (S-group)
+    float nrm = 0.f;  // ratio readout: element i of n (A-group)
     if (is_a) {
+        if constexpr (RATIO) nrm = n0 ? n0[bh * D + i] : 0.f;
         if (A0) {
 #pragma unroll
             for (int j = 0; j < D; ++j) m[j] = A0[mat + (long)i * D + j];
@@ -109,6 +109,7 @@ __global__ void __launch_bounds__(2 * D) vla_sequential_kernel(
             const int nt = min(VLA_TILE, T);
             vla_load_tile<D>(sm.uA[0], u + seq, nt, i);
             vla_load_tile<D>(sm.kA[0], k + seq, nt, i);
+            if constexpr (RATIO) vla_load_tile<D>(sm.qA[0], q + seq, nt, i);
         }
     } else {
         if (S0) {
@@ -128,11 +129,14 @@ __global__ void __launch_bounds__(2 * D) vla_sequential_kernel(
                 const int nt = min(VLA_TILE, T - t0);
                 vla_load_tile<D>(sm.uA[(it + 1) & 1], u + seq + (long)t0 * D, nt, i);
                 vla_load_tile<D>(sm.kA[(it + 1) & 1], k + seq + (long)t0 * D, nt, i);
+                if constexpr (RATIO)
+                    vla_load_tile<D>(sm.qA[(it + 1) & 1], q + seq + (long)t0 * D, nt, i);
             }
             if (it < ntiles) {
                 const int b = it & 1;
                 const int nt = min(VLA_TILE, T - it * VLA_TILE);
                 for (int tt = 0; tt < nt; ++tt) {
+                    const int par = tt & 1;  // VLA_TILE is even: parity of the token index
                     const float* uu = sm.uA[b][tt];
                     const float* kk = sm.kA[b][tt];
                     float z0 = 0.f, z1 = 0.f, y0 = 0.f, y1 = 0.f;
@@ -144,16 +148,38 @@ __global__ void __launch_bounds__(2 * D) vla_sequential_kernel(
                         y1 = fmaf(m[j + 1], kk[j + 1], y1);
                     }
                     const float z = z0 + z1, y = y0 + y1;
-                    sm.zbuf[i] = z;
-                    float uz = uu[i] * z, kz = kk[i] * z;
-                    vla_group_sum2<D>(uz, kz, sm.red1, i);
-                    const float c = 1.f / (1.f + uz);
+                    sm.zbuf[par][i] = z;
+                    // u.z, k.z, y.y, y.z, z.z (and for the ratio readout n.k, n.q, y.q, z.q)
+                    constexpr int NR = RATIO ? 9 : 5;
+                    float r1[NR];
+                    r1[0] = uu[i] * z;
+                    r1[1] = kk[i] * z;
+                    r1[2] = y * y;
+                    r1[3] = y * z;
+                    r1[4] = z * z;
+                    if constexpr (RATIO) {
+                        const float qi = sm.qA[b][tt][i];
+                        r1[5] = nrm * kk[i];
+                        r1[6] = nrm * qi;
+                        r1[7] = y * qi;
+                        r1[8] = z * qi;
+                    }
+                    vla_group_sum<D, NR>(r1, sm.red1[par], i);
+                    const float c = 1.f / (1.f + r1[0]);
+                    const float w = c * r1[1];
+                    const float* zb = sm.zbuf[par];
 #pragma unroll
-                    for (int j = 0; j < D; ++j) m[j] = fmaf(-c * z, sm.zbuf[j], m[j]);
-                    const float yt = fmaf(-c * kz, z, y);  // A_t k = A_{t-1}k - c z (z.k)
-                    const float n2 = vla_group_sum1<D>(yt * yt, sm.red2, i);
-                    sm.ring[b][tt][i] = yt * rsqrtf(n2);
-                    if constexpr (D == 32) __syncwarp();
+                    for (int j = 0; j < D; ++j) m[j] = fmaf(-c * z, zb[j], m[j]);
+                    const float yt = fmaf(-w, z, y);  // A_t k = A_{t-1}k - c z (z.k)
+                    const float n2 = fmaf(w * w, r1[4], fmaf(-2.f * w, r1[3], r1[2]));
+                    const float inv = rsqrtf(n2);
+                    sm.ring[b][tt][i] = yt * inv;
+                    if constexpr (RATIO) {
+                        const float g = 1.f - r1[5];                    // 1 - n.k
+                        const float aq = fmaf(-w, r1[8], r1[7]) * inv;  // alpha_hat.q
+                        nrm = fmaf(g, yt * inv, nrm);
+                        if (i == 0) sm.den[b][tt] = fmaf(g, aq, r1[6]);  // n_t q_t
+                    }
                 }
             }
         } else {
@@ -187,7 +213,10 @@ __global__ void __launch_bounds__(2 * D) vla_sequential_kernel(
                         o0 = fmaf(m[j], qq[j], o0);
                         o1 = fmaf(m[j + 1], qq[j + 1], o1);
                     }
-                    out[seq + (long)(t0 + tt) * D + i] = o0 + o1;
+                    if constexpr (RATIO)
+                        out[seq + (long)(t0 + tt) * D + i] = (o0 + o1) / sm.den[b][tt];
+                    else
+                        out[seq + (long)(t0 + tt) * D + i] = o0 + o1;
                 }
             }
         }
@@ -198,6 +227,9 @@ __global__ void __launch_bounds__(2 * D) vla_sequential_kernel(
     if (dst) {
 #pragma unroll
         for (int j = 0; j < D; ++j) dst[mat + (long)i * D + j] = m[j];
+    }
+    if constexpr (RATIO) {
+        if (is_a && n_final) n_final[bh * D + i] = nrm;
     }
 }
 

@@ -22,6 +22,17 @@
  * and plain linear attention S_t = S_{t-1} + v_t k_t^T ("Variational Linear Attention
  * (VLA)", section 2.1). The kernels apply no feature map and no 1/sqrt(dk) scale: q and
  * k arrive as the caller prepared them (normally L2-normalised per token).
+ *
+ * Gated DeltaNet-2 (same page, sections "Methodology" and "Technical details": a
+ * per-key-channel erase gate b and a per-value-channel write gate w, erase direction
+ * e = b (.) kappa, write target z = w (.) v, residual r = z - W~ e) runs the recurrence
+ * above with a_t = alpha_t (scalar) and k_t, v_t replaced by e_t, z_t: W~ = alpha_t S_{t-1}
+ * is the decayed memory and the residual is written along e_t.
+ *
+ * The write value of a token is u_t = beta_t r_t, the vector the step adds to memory along
+ * its key (S_t = S' + u_t k_t^T; u_t = v_t for plain linear attention). It is the internal
+ * signal the page's cross-layer routing (CLER / CLVR) passages carry to later layers;
+ * dr_scan_fwd_ex and dr_decode_step_ex can return it per token.
  */
 #ifndef DRSCAN_H
 #define DRSCAN_H
@@ -37,7 +48,9 @@ enum {
     DR_LINEAR = 0,   /* S_t = S_{t-1} + v_t k_t^T; beta and gate ignored (may be NULL) */
     DR_DELTANET = 1, /* a_t = 1 */
     DR_GDN = 2,      /* a_t = alpha_t, one scalar per (b,h,t) */
-    DR_KDA = 3       /* a_t = alpha_t[0..dk), one value per key channel */
+    DR_KDA = 3,      /* a_t = alpha_t[0..dk), one value per key channel */
+    DR_GDN2 = 4      /* Gated DeltaNet-2: a_t = alpha_t, k -> b (.) k, v -> w (.) v; only
+                        through dr_scan_fwd_ex / dr_decode_step_ex, which take b and w */
 };
 #define DR_MODE_MASK 0xFF
 /* q, k, v and out are bf16 (else fp32). beta, gate, S0 and S_final are always fp32. */
@@ -53,7 +66,9 @@ enum {
     DR_ERR_UNSUPPORTED = -2, /* a valid request outside the compiled shapes */
     DR_ERR_CUDA = -3,        /* a CUDA runtime/driver call failed (launch, attributes) */
     DR_ERR_TIMEOUT = -4,     /* device: a bounded wait on a barrier ran out; outputs invalid */
-    DR_ERR_DEVICE_BOUNDS = -5 /* device: an index check failed; outputs invalid */
+    DR_ERR_DEVICE_BOUNDS = -5, /* device: an index check failed; outputs invalid */
+    DR_ERR_GATE_RANGE = -6   /* device: a KDA gate decayed past the chunked kernel's range
+                                (see dr_scan_fwd); outputs invalid */
 };
 
 /*
@@ -76,15 +91,38 @@ enum {
  * tcgen05 tensor cores, bf16 operands, fp32 state in tensor memory); everything else
  * runs the per-token kernel with an fp32 state. out may not alias an input.
  *
- * KDA on the chunked kernel factors exp(g_t - g_i) as exp(g_t) * exp(-g_i) inside a
- * chunk (g = running sum of log alpha): the summed log-decay of any key channel over
- * one 64-token chunk must stay above -80, else results are inexact (no error is raised).
+ * KDA on the chunked kernel factors the in-chunk decay exp(g_t - g_i) (g = running sum
+ * of log alpha per key channel) as exp(g_t - m) * exp(m - g_i) with the anchor m = G/2,
+ * G the channel's summed log alpha over the 64-token chunk. This is exact for G >= -170
+ * (alpha about 0.07 per token, every token, every channel); a chunk with any channel
+ * below that latches DR_ERR_GATE_RANGE, which dr_poll_error() reports (the outputs of
+ * that call are then invalid: rerun it with DR_FORCE_SEQUENTIAL, which has no such limit).
  *
  * Returns DR_OK or a negative status; on error nothing is launched.
  */
 int dr_scan_fwd(const void* q, const void* k, const void* v, const float* beta,
                 const float* gate, const float* S0, void* out, float* S_final,
                 int B, int H, int T, int dk, int dv, int mode, cudaStream_t stream);
+
+/*
+ * dr_scan_fwd_ex -- dr_scan_fwd with Gated DeltaNet-2 and the per-token write values.
+ * Same arguments, rules and return values as dr_scan_fwd, plus:
+ *
+ *   erase    [B,H,T,dk] fp32, the erase gate b of DR_GDN2 (NULL for every other variant)
+ *   write    [B,H,T,dv] fp32, the write gate w of DR_GDN2 (NULL for every other variant)
+ *   u_out    [B,H,T,dv] same type as v, or NULL: receives u_t = beta_t r_t for every token
+ *            (v_t for DR_LINEAR). May not alias any other argument.
+ *
+ * DR_GDN2 takes gate [B,H,T] (alpha) like DR_GDN. With bf16 inputs and dk = 128 it runs
+ * the chunked kernel, which scales the k and v tiles by b and w in shared memory before
+ * they enter the tensor-core contractions; it always uses one CTA per (head, value slice).
+ * Asking for u_out adds one [B,H,T,dv] store (and, in a split launch, 8 KB more of each
+ * chunk's operands copied between the CTAs of a cluster).
+ */
+int dr_scan_fwd_ex(const void* q, const void* k, const void* v, const float* beta,
+                   const float* gate, const float* erase, const float* write, const float* S0,
+                   void* out, float* S_final, void* u_out,
+                   int B, int H, int T, int dk, int dv, int mode, cudaStream_t stream);
 
 /*
  * dr_decode_step -- one token of the same recurrence for B*H heads whose state S stays
@@ -111,6 +149,17 @@ int dr_decode_step(const void* q, const void* k, const void* v, const float* bet
                    cudaStream_t stream);
 
 /*
+ * dr_decode_step_ex -- dr_decode_step with Gated DeltaNet-2 and the write value:
+ *   erase [B,H,dk] and write [B,H,dv] fp32, DR_GDN2's gates (NULL otherwise);
+ *   u_out [B,H,dv] same type as v, or NULL: receives this token's u = beta r.
+ * Same rules and return values as dr_decode_step.
+ */
+int dr_decode_step_ex(const void* q, const void* k, const void* v, const float* beta,
+                      const float* gate, const float* erase, const float* write, float* S,
+                      void* out, void* u_out, int B, int H, int dk, int dv, int mode,
+                      cudaStream_t stream);
+
+/*
  * vla_scan_fwd -- Variational Linear Attention scan ("Variational Linear Attention
  * (VLA)", sections 2.2-2.3): per head and token, with A the inverse penalty matrix,
  *
@@ -134,13 +183,66 @@ int vla_scan_fwd(const float* q, const float* k, const float* v, const float* u,
                  float* out, float* S_final, float* A_final,
                  int B, int H, int T, int d, cudaStream_t stream);
 
+/* vla_scan_fwd_ex flag: the ratio readout (see below). */
+#define VLA_RATIO_READOUT 0x1
+
+/*
+ * vla_scan_fwd_ex -- vla_scan_fwd with the ratio readout of "Variational Linear Attention
+ * (VLA)", section 2.3 (the output is a ratio of recurrences, as in standard linear
+ * attention, with an ELU+1 feature map). With flags = VLA_RATIO_READOUT the scan also keeps
+ * the denominator state n (a row of d values: the same write applied to one more value
+ * channel held at 1),
+ *
+ *     n_t = n_{t-1} + (1 - n_{t-1} k_t) alpha_hat_t^T,     o_t = S_t q_t / (n_t q_t),
+ *
+ * and S, A follow vla_scan_fwd exactly. The feature map is the caller's: q holds phi(q)
+ * (ELU+1 of the raw query) and k the unit-norm phi(k) / ||phi(k)||.
+ *
+ *   n0       [B,H,d] fp32 initial denominator state, or NULL for zeros (ratio readout only)
+ *   n_final  [B,H,d] fp32 final denominator state, or NULL to skip (ratio readout only)
+ *   flags    0 (o_t = S_t q_t, exactly vla_scan_fwd) or VLA_RATIO_READOUT
+ *
+ * Other arguments, rules and return values as vla_scan_fwd; n0 / n_final with flags = 0
+ * return DR_ERR_INVALID_ARG. The denominator is not guarded: where n_t q_t is zero the output
+ * is not finite.
+ */
+int vla_scan_fwd_ex(const float* q, const float* k, const float* v, const float* u,
+                    const float* S0, const float* A0, const float* n0, float lambda0,
+                    float* out, float* S_final, float* A_final, float* n_final,
+                    int B, int H, int T, int d, int flags, cudaStream_t stream);
+
+/*
+ * loglinear_scan_fwd -- log-linear attention over a Fenwick hierarchy of linear-attention
+ * memories ("Adaptive memory decay for log-linear attention", problem definition and method
+ * sections: the memory is a Fenwick-tree hierarchy whose state grows as O(log T), and every
+ * output is a weighted sum of memory levels with weights lambda_t^(l)). At step t the
+ * prefix [0, t] splits into level 0 = {t} and, per set bit b of t, level b + 1 = a block of
+ * 2^b earlier tokens (the Fenwick split of the prefix); with M_l the sum of v_s k_s^T over
+ * level l's tokens,
+ *
+ *     o_t = sum_l lambda_t^(l) M_l q_t.
+ *
+ *   q, k     [B,H,T,dk] bf16 (mode = DR_IN_BF16)
+ *   v, out   [B,H,T,dv] bf16
+ *   lambda   [B,H,T,L] fp32 level weights (produced by the caller, e.g. the page's
+ *            softplus MLP); L >= 1 + bit length of T - 1, L <= 16
+ *
+ * Supported: dk = 128, dv in {32, 64, 128}, T <= 32768. Starts from empty memories (no
+ * state in or out). Every non-NULL pointer 16-byte aligned; with B*H*T == 0 nothing is read.
+ * Returns DR_OK or a negative status; on error nothing is launched.
+ */
+int loglinear_scan_fwd(const void* q, const void* k, const void* v, const float* lambda,
+                       void* out, int B, int H, int T, int dk, int dv, int L, int mode,
+                       cudaStream_t stream);
+
 /* Static, human-readable text for a status code (never NULL). */
 const char* dr_status_string(int status);
 
 /*
  * Synchronises `stream`, then returns and clears the status word that kernels on the
- * current device latch when a bounded wait runs out or an index check fails
- * (DR_OK, DR_ERR_TIMEOUT, DR_ERR_DEVICE_BOUNDS), or DR_ERR_CUDA if the synchronisation
+ * current device latch when a bounded wait runs out, an index check fails or a gate is out
+ * of the chunked kernel's range (DR_OK, DR_ERR_TIMEOUT, DR_ERR_DEVICE_BOUNDS,
+ * DR_ERR_GATE_RANGE), or DR_ERR_CUDA if the synchronisation
  * itself failed. The word is a static device variable: the library allocates nothing.
  */
 int dr_poll_error(cudaStream_t stream);

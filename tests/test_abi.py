@@ -42,7 +42,7 @@ def test_library_exports_every_declared_symbol(lib):
 def test_version_and_status_strings(lib):
     assert lib.dr_version() >= 100
     codes = [drs.DR_OK, drs.DR_ERR_INVALID_ARG, drs.DR_ERR_UNSUPPORTED, drs.DR_ERR_CUDA,
-             drs.DR_ERR_TIMEOUT, drs.DR_ERR_DEVICE_BOUNDS]
+             drs.DR_ERR_TIMEOUT, drs.DR_ERR_DEVICE_BOUNDS, drs.DR_ERR_GATE_RANGE]
     texts = [drs.status_string(c) for c in codes]
     assert all(t and t != "unknown status" for t in texts)
     assert len(set(texts)) == len(texts)

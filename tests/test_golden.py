@@ -204,3 +204,20 @@ def test_cuda_vla_on_the_worked_example(cuda):
     assert not np.any(out[:, d:]) and not np.any(Sf[d:, :]) and not np.any(Sf[:, d:])
     eye = np.eye(D)
     assert np.allclose(Af[d:, d:], eye[d:, d:]) and not np.any(Af[:d, d:]) and not np.any(Af[d:, :d])
+
+
+@pytest.mark.gpu
+def test_cuda_vla_ratio_on_the_worked_example(cuda):
+    torch, drs = cuda
+    fx = load("vla_ratio_d3_t2")
+    x = fx["inputs"]
+    T, d = np.asarray(x["q"]).shape
+    D = 32
+    t = lambda a: torch.from_numpy(np.ascontiguousarray(pad(a, (T, D)), np.float32))[None, None].cuda()
+    got = drs.vla_scan_ratio(t(x["q"]), t(x["k"]), t(x["v"]), t(x["u"]), lambda0=x["lambda0"])
+    torch.cuda.synchronize()
+    out, Sf, Af, nf = (a.double().cpu().numpy()[0, 0] for a in got)
+    for g, key in ((out[:, :d], "out"), (Sf[:d, :d], "S_final"), (Af[:d, :d], "A_final"),
+                   (nf[:d], "n_final")):
+        assert rel_err(g, np.asarray(fx["expected"][key])) <= 1e-4, key
+    assert not np.any(nf[d:]) and not np.any(out[:, d:])

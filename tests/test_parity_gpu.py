@@ -12,7 +12,7 @@ import pytest
 import delta_rule_recurrent_chunked_b200 as drs
 from delta_rule_recurrent_chunked_b200 import workloads as wl
 
-from helpers import MODE_NAME, oracle_dr, rel_err, tensor_np, to_device
+from helpers import MODE_NAME, oracle_dr, rel_err, row_rel_err, tensor_np, to_device
 
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
@@ -48,9 +48,17 @@ def check_dr(oracle, w, seed=0, force_sequential=False, tol=None):
     return e_out, e_S
 
 
-# --- the parity workload: DeltaNet fp32, B1 H2 T256 d32
+# --- the parity workload: DeltaNet fp32, B1 H2 T256 d32. Besides the tensor-wide metric,
+# every row (one token's output, one row of the state) must meet 1e-4 relative to its own
+# magnitude.
 def test_deltanet_fp32_workload(oracle):
-    check_dr(oracle, wl.workload("deltanet_fp32"))
+    w = wl.workload("deltanet_fp32")
+    inputs = wl.generate_dr(w, 0)
+    out, Sf = run_dr(to_device(inputs), w)
+    ref_out, ref_S = oracle_dr(oracle, inputs)
+    for got, ref in ((tensor_np(out), ref_out), (tensor_np(Sf), ref_S)):
+        assert rel_err(got, ref) <= TOL["fp32"]
+        assert row_rel_err(got, ref) <= TOL["fp32"], row_rel_err(got, ref)
 
 
 # --- every variant, fp32 inputs (per-token kernel), ragged T, all head sizes
@@ -109,9 +117,62 @@ def test_bf16_strong_decay_gates(oracle):
     check_dr(oracle, w, seed=5)
 
 
+def _check_with_gates(oracle, w, seed, gate_fn):
+    """Parity on a generated workload whose gate array is replaced by gate_fn(inputs) (both
+    sides consume the same replaced array)."""
+    inputs = wl.generate_dr(w, seed)
+    inputs["gate"] = np.ascontiguousarray(gate_fn(inputs), dtype=np.float32)
+    dev = to_device(inputs)
+    out, Sf = run_dr(dev, w)
+    ref_out, ref_S = oracle_dr(oracle, inputs)
+    e_out, e_S = rel_err(tensor_np(out), ref_out), rel_err(tensor_np(Sf), ref_S)
+    assert np.isfinite(e_out) and np.isfinite(e_S), (w, e_out, e_S)
+    assert e_out <= TOL[w.dtype] and e_S <= TOL[w.dtype], (w, e_out, e_S)
+    assert drs.poll_error() == drs.DR_OK
+
+
+# GDN with alpha about 0.12 per step (x ~ N(2, 1)): a chunk's summed log-decay is about -140,
+# far past the point where the factored form exp(g_t) * exp(-g_i) would overflow, so every
+# chunk takes the direct exp(g_t - g_i) branch. Split (2 heads) and unsplit (64 heads) plans,
+# ragged T.
+@pytest.mark.parametrize("BH", [2, 64])
+@pytest.mark.parametrize("T", [200, 300])
+def test_gdn_bf16_very_strong_decay(oracle, BH, T):
+    w = wl.DRWorkload("t", 1, BH, T, 128, 128, wl.GDN, "bf16", s0_std=0.1, gate_mu=2.0)
+    _check_with_gates(oracle, w, 20 + BH + T, lambda inp: inp["gate"])
+
+
+# GDN whose chunks alternate between weak gates (factored branch) and very strong ones
+# (direct branch) inside one sequence.
+@pytest.mark.parametrize("BH", [2, 64])
+def test_gdn_bf16_mixed_decay_chunks(oracle, BH):
+    w = wl.DRWorkload("t", 1, BH, 450, 128, 128, wl.GDN, "bf16", s0_std=0.1)
+
+    def gates(inp):
+        rng = np.random.default_rng(BH)
+        strong = np.exp(-np.logaddexp(0.0, 2.0 + rng.standard_normal(inp["gate"].shape)))
+        g = inp["gate"].astype(np.float64).copy()
+        chunk = (np.arange(w.T) // 64) % 2 == 1
+        g[..., chunk] = strong[..., chunk]
+        return g
+
+    _check_with_gates(oracle, w, 31 + BH, gates)
+
+
+# KDA with strong per-channel gates: x ~ N(0, 1) (alpha about 0.5), x ~ N(1.4, 0.5) (alpha
+# about 0.2: a channel's summed log-decay over one chunk about -100, below fp32's exp range)
+# and x ~ N(2, 1) (alpha about 0.12, about -140 per chunk), unsplit launches, ragged T.
+@pytest.mark.parametrize("mu,sigma", [(0.0, 1.0), (1.4, 0.5), (2.0, 1.0)])
+@pytest.mark.parametrize("BH", [2, 48])
+def test_kda_bf16_strong_decay(oracle, mu, sigma, BH):
+    w = wl.DRWorkload("t", 1, BH, 300, 128, 128, wl.KDA, "bf16", s0_std=0.1, gate_mu=mu,
+                      gate_sigma=sigma)
+    _check_with_gates(oracle, w, 7 + BH, lambda inp: inp["gate"])
+
+
 # --- full-size workloads, sampled heads
 def _check_sampled(oracle, name, heads, seed=0):
-    w = wl.workload(name)
+    w = wl.workload(name) if isinstance(name, str) else name
     inputs = wl.generate_dr(w, seed)
     dev = to_device(inputs)
     out, Sf = run_dr(dev, w)
@@ -132,9 +193,27 @@ def test_kda_bf16_workload_sampled(oracle):
     _check_sampled(oracle, "kda_bf16", [0, 77, 127])
 
 
-@pytest.mark.parametrize("T", [4096, 32768])
+@pytest.mark.parametrize("T", [4096, 8192, 16384, 32768])
 def test_gdn_long_workload_sampled(oracle, T):
     _check_sampled(oracle, f"gdn_long_t{T}", [0, 15])
+
+
+# DeltaNet has no decay, so the rounding of every chunk's bf16 operands stays in the state:
+# the long-context shapes (16 heads, split clusters) on the chunked kernel, sampled heads.
+@pytest.mark.parametrize("T", [4096, 32768])
+def test_deltanet_bf16_long_sampled(oracle, T):
+    w = wl.DRWorkload(f"deltanet_long_t{T}", 1, 16, T, 128, 128, wl.DELTANET, "bf16",
+                      s0_std=0.1)
+    assert drs.chunked_plan("deltanet", 16, 128, 128)[1] > 0  # a split launch
+    _check_sampled(oracle, w, [0, 15])
+
+
+# the same with one CTA per (head, value slice): 64 heads
+def test_deltanet_bf16_long_unsplit_sampled(oracle):
+    w = wl.DRWorkload("deltanet_long_unsplit", 1, 64, 8192, 128, 128, wl.DELTANET, "bf16",
+                      s0_std=0.1)
+    assert drs.chunked_plan("deltanet", 64, 128, 128)[1] == 0
+    _check_sampled(oracle, w, [0, 63])
 
 
 # --- edge cases
@@ -357,6 +436,7 @@ def test_vla_workload(oracle, d):
     a = tensor_np(Af).reshape(32, d, d)[heads][None]
     for got, ref in ((o, ref_out), (s, ref_S), (a, ref_A)):
         assert rel_err(got, ref) <= 1e-4
+        assert row_rel_err(got, ref) <= 1e-4, row_rel_err(got, ref)
 
 
 @pytest.mark.parametrize("d", [32, 64, 96, 128])
