@@ -344,7 +344,9 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
         mbar_init(bar(B_VSCALED + 0), 1);
         mbar_init(bar(B_VSCALED + 1), 1);
         mbar_init(bar(B_MMA1), 1);
-        mbar_init(bar(B_YREADY), 128);
+        // split chain CTA: the residual threads arrive after writing Y, the others once the
+        // state they rescaled in tensor memory for the next MMA3 is stored
+        mbar_init(bar(B_YREADY), SPLIT ? 256 : 128);
         mbar_init(bar(B_MMA23), 1);
         mbar_init(bar(B_STATE), SPLIT ? 256 : 128);
         *abort_flag = 0;
@@ -675,6 +677,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             fence_async_smem();
             tc_fence_before();
             mbar_arrive(bar(B_STATE));
+            if (r >= 64) mbar_arrive(bar(B_YREADY));  // the first MMA3 may use the state
         }
         // write values U = T Y of chunk c (rows 0-63 of D2), read by the residual threads once
         // MMA2 of that chunk is done; D2 is reused only after they (and the output threads)
@@ -758,13 +761,20 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             }
             mbar_wait(bar(B_MMA23), (uint32_t)(c & 1), abort_flag);
             tc_fence_after();
+            // the bf16 copy goes to MMA1 first; the fp32 state is rescaled for the next MMA3
+            // after that hand-off (MMA3 waits for it through B_YREADY)
+            float sv[LW];
             if (active) {
-                float sv[LW];
 #pragma unroll
                 for (int c16 = 0; c16 < LW; c16 += 16) tmem_ld16(trow + L::COL_S + cb + c16, sv + c16);
                 tmem_wait_ld();
 #pragma unroll
                 for (int i = 0; i < NV8; ++i) st_row_chunk(sm + L::SS, r, cb / 8 + i, sv + 8 * i);
+            }
+            fence_async_smem();
+            tc_fence_before();
+            mbar_arrive(bar(B_STATE));
+            if (active) {
                 if (last && S_final) {
                     float* dst = S_final + (bh * dv + v0 + cb) * (long)CDK + r;
 #pragma unroll
@@ -780,9 +790,10 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     }
                 }
             }
-            fence_async_smem();
-            tc_fence_before();
-            mbar_arrive(bar(B_STATE));
+            if (r >= 64 && !last) {
+                tc_fence_before();
+                mbar_arrive(bar(B_YREADY));  // for the next chunk's MMA3
+            }
             // ---- outputs O = gamma_t (S0 q_t) + (P T Y)_t, overlapping the next residuals
             if (r >= 64) {
                 const int t = r - 64;
@@ -1098,12 +1109,24 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 // exp(+-|G|/2): exact for G down to KDA_MIN_LOG_DECAY. The chain multiplies its
                 // bf16 state copy by exp(m) per channel, which restores exp(g_t) in MMA1.
                 uint8_t* kn = sm + L::KN;
-                float2 lp = make_float2(0.f, 0.f);
+                // summed log alpha of this thread's 16 rows: the log of their product, or,
+                // where that product would underflow, the sum of the rows' logs
+                float2 part = make_float2(1.f, 1.f);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     if (16 * kq4 + i < nvalid) {
-                        lp.x += __logf(gpf[i].x);
-                        lp.y += __logf(gpf[i].y);
+                        part.x *= gpf[i].x;
+                        part.y *= gpf[i].y;
+                    }
+                }
+                float2 lp = make_float2(__logf(part.x), __logf(part.y));
+                if (part.x < 1e-30f || part.y < 1e-30f) {
+                    lp = make_float2(0.f, 0.f);
+                    for (int i = 0; i < 16; ++i) {
+                        if (16 * kq4 + i < nvalid) {
+                            lp.x += __logf(gpf[i].x);
+                            lp.y += __logf(gpf[i].y);
+                        }
                     }
                 }
                 *reinterpret_cast<float2*>(pg + 128 * kq4 + kc) = lp;

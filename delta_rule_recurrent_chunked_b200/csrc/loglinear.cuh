@@ -16,7 +16,9 @@
 // query rows each for the outputs and 32 key channels each for the chunk state; every
 // contraction is a bf16 m16n8k16 warp MMA with fp32 accumulation (the tiles are 16-64 rows,
 // the level bookkeeping sits between them). The block states stay in shared memory in fp32
-// (dk x BV per level, for up to LL_LEVELS chunk levels: T <= 64 * 2^LL_LEVELS).
+// (dk x BV per level, for up to LL_LEVELS chunk levels: T <= 64 * 2^LL_LEVELS). The next
+// chunk's tiles are loaded into registers while the current chunk computes (the level
+// states leave no room for a second shared-memory stage) and stored once it is done.
 #pragma once
 
 #include "common.cuh"
@@ -63,6 +65,70 @@ __device__ __forceinline__ void ll_ldsm_x4_t(uint32_t* r, const void* p) {
 
 __device__ __forceinline__ int ll_bitlen(int x) { return 32 - __clz(x); }
 
+// One chunk's tiles in registers, spread over the CTA's threads (rows past T as zeros, their
+// lambdas as zero): loaded from HBM early, stored to shared memory when the tiles are free.
+struct LoglinearStage {
+    static constexpr int NQK = LL_C * (LL_DK / 8) / LL_THREADS;  // 16-byte pieces per thread
+    static constexpr int NV = LL_C * (LL_BV / 8) / LL_THREADS;
+    static constexpr int NL = LL_C * LL_LMAX / LL_THREADS;
+    uint4 qv[NQK], kv[NQK], vv[NV];
+    float lv[NL];
+
+    __device__ __forceinline__ void load(const __nv_bfloat16* __restrict__ q,
+                                         const __nv_bfloat16* __restrict__ k,
+                                         const __nv_bfloat16* __restrict__ v,
+                                         const float* __restrict__ lam, long bh, int T, int dv,
+                                         int v0, int L, int t0, int tid) {
+#pragma unroll
+        for (int i = 0; i < NQK; ++i) {
+            const int e = tid + i * LL_THREADS;
+            const int r = e / (LL_DK / 8), c8 = (e % (LL_DK / 8)) * 8;
+            qv[i] = kv[i] = make_uint4(0, 0, 0, 0);
+            if (t0 + r < T) {
+                qv[i] = *reinterpret_cast<const uint4*>(q + (bh * T + t0 + r) * (long)LL_DK + c8);
+                kv[i] = *reinterpret_cast<const uint4*>(k + (bh * T + t0 + r) * (long)LL_DK + c8);
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < NV; ++i) {
+            const int e = tid + i * LL_THREADS;
+            const int r = e / (LL_BV / 8), c8 = (e % (LL_BV / 8)) * 8;
+            vv[i] = make_uint4(0, 0, 0, 0);
+            if (t0 + r < T) vv[i] = *reinterpret_cast<const uint4*>(v + (bh * T + t0 + r) * (long)dv + v0 + c8);
+        }
+#pragma unroll
+        for (int i = 0; i < NL; ++i) {
+            const int e = tid + i * LL_THREADS;
+            const int r = e / LL_LMAX, l = e % LL_LMAX;
+            lv[i] = (t0 + r < T && l < L) ? lam[(bh * T + t0 + r) * (long)L + l] : 0.f;
+        }
+    }
+
+    __device__ __forceinline__ void store(LoglinearSmem& sm) const;
+};
+
+__device__ __forceinline__ void LoglinearStage::store(LoglinearSmem& sm) const {
+    const int tid = threadIdx.x;
+#pragma unroll
+    for (int i = 0; i < NQK; ++i) {
+        const int e = tid + i * LL_THREADS;
+        const int r = e / (LL_DK / 8), c8 = (e % (LL_DK / 8)) * 8;
+        *reinterpret_cast<uint4*>(&sm.q[r][c8]) = qv[i];
+        *reinterpret_cast<uint4*>(&sm.k[r][c8]) = kv[i];
+    }
+#pragma unroll
+    for (int i = 0; i < NV; ++i) {
+        const int e = tid + i * LL_THREADS;
+        const int r = e / (LL_BV / 8), c8 = (e % (LL_BV / 8)) * 8;
+        *reinterpret_cast<uint4*>(&sm.v[r][c8]) = vv[i];
+    }
+#pragma unroll
+    for (int i = 0; i < NL; ++i) {
+        const int e = tid + i * LL_THREADS;
+        sm.lam[e / LL_LMAX][e % LL_LMAX] = lv[i];
+    }
+}
+
 // grid: (B*H, dv / LL_BV); block: LL_THREADS; dynamic shared memory: sizeof(LoglinearSmem).
 __global__ void __launch_bounds__(LL_THREADS) loglinear_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
@@ -77,32 +143,15 @@ __global__ void __launch_bounds__(LL_THREADS) loglinear_kernel(
     const int nchunks = (T + LL_C - 1) / LL_C;
 
     for (int e = tid; e < LL_LEVELS * LL_DK * LL_MS; e += LL_THREADS) (&sm.m[0][0][0])[e] = 0.f;
+    LoglinearStage stage;
+    if (nchunks > 0) stage.load(q, k, v, lam, bh, T, dv, v0, L, 0, tid);
 
     for (int c = 0; c < nchunks; ++c) {
         const int t0 = c * LL_C;
         __syncthreads();  // the previous chunk is done with every tile
-        // ---- tiles of the chunk (rows past T read as zeros, their lambdas as zero)
-        for (int e = tid; e < LL_C * (LL_DK / 8); e += LL_THREADS) {
-            const int r = e / (LL_DK / 8), c8 = (e % (LL_DK / 8)) * 8;
-            uint4 qv = make_uint4(0, 0, 0, 0), kv = qv;
-            if (t0 + r < T) {
-                qv = *reinterpret_cast<const uint4*>(q + (bh * T + t0 + r) * (long)LL_DK + c8);
-                kv = *reinterpret_cast<const uint4*>(k + (bh * T + t0 + r) * (long)LL_DK + c8);
-            }
-            *reinterpret_cast<uint4*>(&sm.q[r][c8]) = qv;
-            *reinterpret_cast<uint4*>(&sm.k[r][c8]) = kv;
-        }
-        for (int e = tid; e < LL_C * (LL_BV / 8); e += LL_THREADS) {
-            const int r = e / (LL_BV / 8), c8 = (e % (LL_BV / 8)) * 8;
-            uint4 vv = make_uint4(0, 0, 0, 0);
-            if (t0 + r < T) vv = *reinterpret_cast<const uint4*>(v + (bh * T + t0 + r) * (long)dv + v0 + c8);
-            *reinterpret_cast<uint4*>(&sm.v[r][c8]) = vv;
-        }
-        for (int e = tid; e < LL_C * LL_LMAX; e += LL_THREADS) {
-            const int r = e / LL_LMAX, l = e % LL_LMAX;
-            sm.lam[r][l] = (t0 + r < T && l < L) ? lam[(bh * T + t0 + r) * (long)L + l] : 0.f;
-        }
+        stage.store(sm);
         __syncthreads();
+        if (c + 1 < nchunks) stage.load(q, k, v, lam, bh, T, dv, v0, L, t0 + LL_C, tid);
 
         // ---- outputs of rows 16*warp .. +15
         const int r0 = 16 * warp;

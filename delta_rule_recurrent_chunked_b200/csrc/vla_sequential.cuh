@@ -8,7 +8,10 @@
 //    dependent mat-vec) and ||A_t k||^2 = y.y - 2 w y.z + w^2 z.z, so the norm needs no
 //    reduction of its own; then the rank-1 update of A's row;
 //  * the S-group owns S (row i in thread i's registers); given alpha_hat_t its rows are
-//    independent: r_i = v_i - s_i.k, s_i += r_i alpha_hat, o_i = s_i.q. No reductions.
+//    independent: r_i = v_i - s_i.k, s_i += r_i alpha_hat, and the readout after the write
+//    o_i = s_i.q + r_i (alpha_hat.q), with s_i the row before the write: the two dot products
+//    of a token run side by side. alpha_hat.q comes from the A-group (y.q and z.q join its
+//    reduction: alpha_hat.q = (y.q - w z.q) / ||A_t k||). No reductions in the S-group.
 // The groups run one token tile apart: while the A-group produces the directions of tile n
 // into a shared-memory ring, the S-group consumes tile n-1. One __syncthreads per tile.
 //
@@ -30,16 +33,17 @@ template <int D>
 struct VlaSmem {
     float uA[2][VLA_TILE][D];
     float kA[2][VLA_TILE][D];
-    float qA[2][VLA_TILE][D];  // ratio readout: the A-group's copy of q
+    float qA[2][VLA_TILE][D];  // the A-group's copy of q
     float kS[2][VLA_TILE][D];
     float vS[2][VLA_TILE][D];
     float qS[2][VLA_TILE][D];
     float ring[2][VLA_TILE][D];
+    float aq[2][VLA_TILE];     // alpha_hat_t . q_t
     float den[2][VLA_TILE];    // ratio readout: n_t q_t
     // alternate tokens use alternate buffers: a token's writes never meet a slower thread's
     // reads of the previous token (one group barrier per token separates them)
     float zbuf[2][D];
-    float red1[2][9][4];
+    float red1[2][9][4];  // a token's partial sums, one slot per value and warp
 };
 
 // Sums N values over the D threads of a group (warp shuffles, then one named barrier to
@@ -109,7 +113,7 @@ __global__ void __launch_bounds__(2 * D) vla_sequential_kernel(
             const int nt = min(VLA_TILE, T);
             vla_load_tile<D>(sm.uA[0], u + seq, nt, i);
             vla_load_tile<D>(sm.kA[0], k + seq, nt, i);
-            if constexpr (RATIO) vla_load_tile<D>(sm.qA[0], q + seq, nt, i);
+            vla_load_tile<D>(sm.qA[0], q + seq, nt, i);
         }
     } else {
         if (S0) {
@@ -129,8 +133,7 @@ __global__ void __launch_bounds__(2 * D) vla_sequential_kernel(
                 const int nt = min(VLA_TILE, T - t0);
                 vla_load_tile<D>(sm.uA[(it + 1) & 1], u + seq + (long)t0 * D, nt, i);
                 vla_load_tile<D>(sm.kA[(it + 1) & 1], k + seq + (long)t0 * D, nt, i);
-                if constexpr (RATIO)
-                    vla_load_tile<D>(sm.qA[(it + 1) & 1], q + seq + (long)t0 * D, nt, i);
+                vla_load_tile<D>(sm.qA[(it + 1) & 1], q + seq + (long)t0 * D, nt, i);
             }
             if (it < ntiles) {
                 const int b = it & 1;
@@ -139,30 +142,33 @@ __global__ void __launch_bounds__(2 * D) vla_sequential_kernel(
                     const int par = tt & 1;  // VLA_TILE is even: parity of the token index
                     const float* uu = sm.uA[b][tt];
                     const float* kk = sm.kA[b][tt];
-                    float z0 = 0.f, z1 = 0.f, y0 = 0.f, y1 = 0.f;
+                    // four partial sums per product: dependent FMA chains of D/4
+                    float z4[4] = {0.f, 0.f, 0.f, 0.f}, y4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int j = 0; j < D; j += 2) {
-                        z0 = fmaf(m[j], uu[j], z0);
-                        z1 = fmaf(m[j + 1], uu[j + 1], z1);
-                        y0 = fmaf(m[j], kk[j], y0);
-                        y1 = fmaf(m[j + 1], kk[j + 1], y1);
+                    for (int j = 0; j < D; j += 4) {
+#pragma unroll
+                        for (int e = 0; e < 4; ++e) {
+                            z4[e] = fmaf(m[j + e], uu[j + e], z4[e]);
+                            y4[e] = fmaf(m[j + e], kk[j + e], y4[e]);
+                        }
                     }
-                    const float z = z0 + z1, y = y0 + y1;
+                    const float z = (z4[0] + z4[1]) + (z4[2] + z4[3]);
+                    const float y = (y4[0] + y4[1]) + (y4[2] + y4[3]);
                     sm.zbuf[par][i] = z;
-                    // u.z, k.z, y.y, y.z, z.z (and for the ratio readout n.k, n.q, y.q, z.q)
-                    constexpr int NR = RATIO ? 9 : 5;
+                    // u.z, k.z, y.y, y.z, z.z, y.q, z.q (and for the ratio readout n.k, n.q)
+                    constexpr int NR = RATIO ? 9 : 7;
                     float r1[NR];
+                    const float qi = sm.qA[b][tt][i];
                     r1[0] = uu[i] * z;
                     r1[1] = kk[i] * z;
                     r1[2] = y * y;
                     r1[3] = y * z;
                     r1[4] = z * z;
+                    r1[5] = y * qi;
+                    r1[6] = z * qi;
                     if constexpr (RATIO) {
-                        const float qi = sm.qA[b][tt][i];
-                        r1[5] = nrm * kk[i];
-                        r1[6] = nrm * qi;
-                        r1[7] = y * qi;
-                        r1[8] = z * qi;
+                        r1[7] = nrm * kk[i];
+                        r1[8] = nrm * qi;
                     }
                     vla_group_sum<D, NR>(r1, sm.red1[par], i);
                     const float c = 1.f / (1.f + r1[0]);
@@ -174,11 +180,12 @@ __global__ void __launch_bounds__(2 * D) vla_sequential_kernel(
                     const float n2 = fmaf(w * w, r1[4], fmaf(-2.f * w, r1[3], r1[2]));
                     const float inv = rsqrtf(n2);
                     sm.ring[b][tt][i] = yt * inv;
+                    const float aq = fmaf(-w, r1[6], r1[5]) * inv;  // alpha_hat.q
+                    if (i == 0) sm.aq[b][tt] = aq;
                     if constexpr (RATIO) {
-                        const float g = 1.f - r1[5];                    // 1 - n.k
-                        const float aq = fmaf(-w, r1[8], r1[7]) * inv;  // alpha_hat.q
+                        const float g = 1.f - r1[7];  // 1 - n.k
                         nrm = fmaf(g, yt * inv, nrm);
-                        if (i == 0) sm.den[b][tt] = fmaf(g, aq, r1[6]);  // n_t q_t
+                        if (i == 0) sm.den[b][tt] = fmaf(g, aq, r1[8]);  // n_t q_t
                     }
                 }
             }
@@ -198,25 +205,25 @@ __global__ void __launch_bounds__(2 * D) vla_sequential_kernel(
                     const float* kk = sm.kS[b][tt];
                     const float* qq = sm.qS[b][tt];
                     const float* al = sm.ring[b][tt];
-                    float p0 = 0.f, p1 = 0.f;
+                    // s.k and s.q of the row before the write, side by side
+                    float p4[4] = {0.f, 0.f, 0.f, 0.f}, o4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-                    for (int j = 0; j < D; j += 2) {
-                        p0 = fmaf(m[j], kk[j], p0);
-                        p1 = fmaf(m[j + 1], kk[j + 1], p1);
-                    }
-                    const float r = sm.vS[b][tt][i] - (p0 + p1);
-                    float o0 = 0.f, o1 = 0.f;
+                    for (int j = 0; j < D; j += 4) {
 #pragma unroll
-                    for (int j = 0; j < D; j += 2) {
-                        m[j] = fmaf(r, al[j], m[j]);
-                        m[j + 1] = fmaf(r, al[j + 1], m[j + 1]);
-                        o0 = fmaf(m[j], qq[j], o0);
-                        o1 = fmaf(m[j + 1], qq[j + 1], o1);
+                        for (int e = 0; e < 4; ++e) {
+                            p4[e] = fmaf(m[j + e], kk[j + e], p4[e]);
+                            o4[e] = fmaf(m[j + e], qq[j + e], o4[e]);
+                        }
                     }
+                    const float o0 = (o4[0] + o4[1]) + (o4[2] + o4[3]), o1 = 0.f;
+                    const float r = sm.vS[b][tt][i] - ((p4[0] + p4[1]) + (p4[2] + p4[3]));
+#pragma unroll
+                    for (int j = 0; j < D; ++j) m[j] = fmaf(r, al[j], m[j]);
+                    const float o = fmaf(r, sm.aq[b][tt], o0 + o1);  // s_t.q after the write
                     if constexpr (RATIO)
-                        out[seq + (long)(t0 + tt) * D + i] = (o0 + o1) / sm.den[b][tt];
+                        out[seq + (long)(t0 + tt) * D + i] = o / sm.den[b][tt];
                     else
-                        out[seq + (long)(t0 + tt) * D + i] = o0 + o1;
+                        out[seq + (long)(t0 + tt) * D + i] = o;
                 }
             }
         }

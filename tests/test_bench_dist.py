@@ -103,3 +103,19 @@ def test_cpu_baseline_runs_whole_passes_up_to_the_target_time(oracle):
     # either the target time was reached or the pass cap (100) stopped it
     assert float(m.group(3)) >= 0.95 or passes == 100
     assert r["kind"] == "oracle" and r["cores"] >= 1 and r["value"] > 0
+
+
+def test_every_per_config_workload_is_accounted():
+    # the benchmark's configuration list names real workloads, each with positive algorithmic
+    # bytes and FLOPs, and the headline is one of them
+    import bench
+    from delta_rule_recurrent_chunked_b200 import workloads as wl
+
+    assert bench.DEFAULT_WORKLOAD in bench.PER_CONFIG
+    for name in bench.PER_CONFIG:
+        w = wl.workload(name)
+        assert bench.algorithmic_bytes(w) > 0 and bench.algorithmic_flops(w) > 0, name
+        nsets, flush = bench.rotation(bench.algorithmic_bytes(w))
+        assert 1 <= nsets <= 4
+        cfg = bench.workload_config(w, 1)
+        assert cfg["workload"] == name and cfg["B"] * cfg["H"] * cfg["T"] == w.head_tokens
