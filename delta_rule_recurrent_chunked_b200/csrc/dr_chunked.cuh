@@ -82,8 +82,9 @@ struct ChunkLayout {
 
     static constexpr int KQ_B = 32768;  // [K;Q] bf16: 2 panels x 128 rows x 128 B
     static constexpr int V_B = CK * BV * 2;
-    // split, BV = 64: V rows are one 128-byte swizzled row each (conflict-free row reads)
-    static constexpr bool V_SWZ = SPLIT && BV == 64;
+    // BV >= 64: the V tile is stored as 128-byte-swizzled panels of 64 channels (8 KB each),
+    // so that the residual threads, each reading its own row, hit distinct banks
+    static constexpr bool V_SWZ = BV >= 64;
     // The chain MMAs run with N = NB >= 64 so that Y and the bf16 state are stored as
     // M/N-major B operands in 64-column swizzled groups (whole-row 16-byte stores); columns
     // beyond the real ones are zero padding. Group g of S / Y sits at SS + g*16384 /
@@ -434,18 +435,29 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     mbar_wait(bar(B_V_EMPTY + sv), (uint32_t)(((c / NSV) - 1) & 1), abort_flag);
                 if (!*abort_flag) {
                     mbar_arrive_expect_tx(bar(B_V_FULL + sv), L::V_B);
-                    tma_load_3d(smem_u32(sm + L::V + sv * L::V_B), &tmV, bar(B_V_FULL + sv), v0,
-                                c * CK, (int)bh);
+                    constexpr int VB = L::V_SWZ ? 64 : BV;  // channels per TMA box
+#pragma unroll
+                    for (int pn = 0; pn < BV / VB; ++pn)
+                        tma_load_3d(smem_u32(sm + L::V + sv * L::V_B + pn * CK * VB * 2), &tmV,
+                                    bar(B_V_FULL + sv), v0 + pn * VB, c * CK, (int)bh);
                 }
             }
             if constexpr (kGdn2) {
                 __syncwarp();
                 mbar_wait(bar(B_V_FULL + sv), (uint32_t)((c / NSV) & 1), abort_flag);
-                static_assert(!L::V_SWZ, "rows of V are plain BV-element rows here");
                 __nv_bfloat162* vt = reinterpret_cast<__nv_bfloat162*>(sm + L::V + sv * L::V_B);
                 constexpr int PAIRS = CK * BV / 2;
                 for (int e = lane; e < PAIRS; e += 32) {
-                    const int row = e / (BV / 2), col = 2 * (e % (BV / 2));
+                    // the stored pair e at (row, col): plain rows, or swizzled 64-channel panels
+                    int row, col;
+                    if constexpr (L::V_SWZ) {
+                        const int pn = e / (CK * 32), w = e % (CK * 32);  // 32 pairs per row
+                        row = w >> 5;
+                        col = 64 * pn + ((((w >> 2) & 7) ^ (row & 7)) << 3) + 2 * (w & 3);
+                    } else {
+                        row = e / (BV / 2);
+                        col = 2 * (e % (BV / 2));
+                    }
                     const int t = c * CK + row;
                     float2 w2 = make_float2(0.f, 0.f);
                     if (t < T) w2 = *reinterpret_cast<const float2*>(write + (bh * T + t) * (long)dv + v0 + col);
@@ -873,14 +885,17 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 mbar_wait(bar(B_PREP + p), (uint32_t)((c / NP) & 1), abort_flag);
                 const float* gam = reinterpret_cast<const float*>(slot(p) + L::SLOT_GAM);
                 const float gC = kKda ? gam[r] : gam[64];
+                constexpr int PW = BV < 32 ? BV : 32;  // columns per tensor-memory round trip
 #pragma unroll
-                for (int c16 = 0; c16 < BV; c16 += 16) {
-                    float sv[16];
-                    tmem_ld16(trow + L::COL_S + c16, sv);
+                for (int c0 = 0; c0 < BV; c0 += PW) {
+                    float sv[PW];
+#pragma unroll
+                    for (int c16 = 0; c16 < PW; c16 += 16) tmem_ld16(trow + L::COL_S + c0 + c16, sv + c16);
                     tmem_wait_ld();
 #pragma unroll
-                    for (int v = 0; v < 16; ++v) sv[v] *= gC;
-                    tmem_st16(trow + L::COL_S + c16, sv);
+                    for (int v = 0; v < PW; ++v) sv[v] *= gC;
+#pragma unroll
+                    for (int c16 = 0; c16 < PW; c16 += 16) tmem_st16(trow + L::COL_S + c0 + c16, sv + c16);
                 }
                 tmem_wait_st();
             }
@@ -898,8 +913,15 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 mbar_wait(bar((kGdn2 ? B_VSCALED : B_V_FULL) + svi), (uint32_t)((c / NSV) & 1),
                           abort_flag);
                 const float gt = kGdn ? gam[r] : 1.f;
-                const uint4* vrow =
-                    reinterpret_cast<const uint4*>(sm + L::V + svi * L::V_B + r * BV * 2);
+                // row r of V: 16-byte piece jj (channels 8jj .. 8jj+7)
+                const uint8_t* vtile = sm + L::V + svi * L::V_B;
+                auto vpiece = [&](int jj) -> uint4 {
+                    if constexpr (L::V_SWZ)
+                        return *reinterpret_cast<const uint4*>(
+                            vtile + (jj >> 3) * (CK * 128) + r * 128 + (((jj & 7) ^ (r & 7)) << 4));
+                    else
+                        return *reinterpret_cast<const uint4*>(vtile + r * BV * 2 + jj * 16);
+                };
                 constexpr int HW = BV < 64 ? BV : 64;  // columns per pass
 #pragma unroll
                 for (int c0 = 0; c0 < BV; c0 += HW) {
@@ -908,7 +930,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
 #pragma unroll
                     for (int c16 = 0; c16 < HW; c16 += 16) tmem_ld16(trow + L::COL_D1 + c0 + c16, x + c16);
 #pragma unroll
-                    for (int i = 0; i < HW / 8; ++i) vw[i] = vrow[c0 / 8 + i];
+                    for (int i = 0; i < HW / 8; ++i) vw[i] = vpiece(c0 / 8 + i);
                     tmem_wait_ld();
 #pragma unroll
                     for (int i = 0; i < HW / 8; ++i) {
@@ -951,23 +973,29 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 // output rows: O = gamma_t (S0 q_t) + (P T Y)_t
                 const int t = r - 64;
                 const float gt = kGdn ? gam[t] : 1.f;
+                constexpr int PW = BV < 32 ? BV : 32;  // columns per tensor-memory round trip
 #pragma unroll
-                for (int c16 = 0; c16 < BV; c16 += 16) {
-                    float z[16], d[16];
-                    tmem_ld16(trow + L::COL_D1 + c16, z);
-                    tmem_ld16(trow + L::COL_D2 + c16, d);
+                for (int c0 = 0; c0 < BV; c0 += PW) {
+                    float z[PW], d[PW];
+#pragma unroll
+                    for (int c16 = 0; c16 < PW; c16 += 16) {
+                        tmem_ld16(trow + L::COL_D1 + c0 + c16, z + c16);
+                        tmem_ld16(trow + L::COL_D2 + c0 + c16, d + c16);
+                    }
                     tmem_wait_ld();
                     if (t < nvalid) {
-                        uint4 w[2];
-                        uint32_t* wp = reinterpret_cast<uint32_t*>(w);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e)
-                            wp[e] = pack_bf16(fmaf(gt, z[2 * e], d[2 * e]),
-                                              fmaf(gt, z[2 * e + 1], d[2 * e + 1]));
                         uint4* dst = reinterpret_cast<uint4*>(out + (bh * T + t0 + t) * (long)dv +
-                                                              v0 + c16);
-                        dst[0] = w[0];
-                        dst[1] = w[1];
+                                                              v0 + c0);
+#pragma unroll
+                        for (int i = 0; i < PW / 8; ++i) {
+                            uint4 w;
+                            uint32_t* wp = reinterpret_cast<uint32_t*>(&w);
+#pragma unroll
+                            for (int e = 0; e < 4; ++e)
+                                wp[e] = pack_bf16(fmaf(gt, z[8 * i + 2 * e], d[8 * i + 2 * e]),
+                                                  fmaf(gt, z[8 * i + 2 * e + 1], d[8 * i + 2 * e + 1]));
+                            dst[i] = w;
+                        }
                     }
                 }
             }
@@ -1092,12 +1120,6 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                                 pack_bf16(k2.x * gpf[i0 + i].x, k2.y * gpf[i0 + i].y);
                         }
                     }
-#pragma unroll
-                    for (int i = 0; i < 16; ++i) {
-                        const int tn = (c + NGR * pSP) * CK + 16 * kq4 + i;
-                        gpf[i] = tn < T ? *reinterpret_cast<const float2*>(erase + (bh * T + tn) * (long)CDK + kc)
-                                        : make_float2(1.f, 1.f);
-                    }
                     fence_async_smem();
                     gsync();
                 }
@@ -1183,17 +1205,22 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     *reinterpret_cast<float2*>(pg + 512 + kc) = run;
                     *reinterpret_cast<float2*>(pg + 640 + kc) = make_float2(__expf(G.x), __expf(G.y));
                 }
-#pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                    const int tn = (c + NGR * pSP) * CK + 16 * kq4 + i;
-                    gpf[i] = tn < T ? *reinterpret_cast<const float2*>(gate + (bh * T + tn) * (long)CDK + kc)
-                                    : make_float2(1.f, 1.f);
-                }
                 fence_async_smem();
                 gsync();
             }
             tc_fence_before();
             mbar_arrive(bar(gb + 0));
+            if constexpr (kChan) {
+                // the next owned chunk's per-channel values (KDA's gates, Gated DeltaNet-2's
+                // erase gate), issued after this stage's proxy fence so that the fence does
+                // not wait for them; they land under the rest of this chunk's prep
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                    const int tn = (c + NGR * pSP) * CK + 16 * kq4 + i;
+                    gpf[i] = tn < T ? *reinterpret_cast<const float2*>(chan + (bh * T + tn) * (long)CDK + kc)
+                                    : make_float2(1.f, 1.f);
+                }
+            }
 
             // ---- 2. Gram epilogue: A (fp32, rows 0-63) and P (bf16, rows 0-63 of pm); a
             // thread takes one or both 32-column halves of TMEM row lq
@@ -1520,7 +1547,7 @@ int launch_chunked_bv(const ChunkArgs& a, int nprep, cudaStream_t stream) {
     CUtensorMap mk, mq, mv;
     if (!cached_map_3d(0, &mk, a.k, a.BH, a.T, CDK, 64, true) ||
         !cached_map_3d(1, &mq, a.q, a.BH, a.T, CDK, 64, true) ||
-        !cached_map_3d(2, &mv, a.v, a.BH, a.T, a.dv, BV, L::V_SWZ))
+        !cached_map_3d(2, &mv, a.v, a.BH, a.T, a.dv, L::V_SWZ ? 64 : BV, L::V_SWZ))
         return DR_ERR_CUDA;
     const int smem = L::TOTAL + 1024;
     auto kern = dr_chunked_kernel<MODE, BV, SPLIT>;

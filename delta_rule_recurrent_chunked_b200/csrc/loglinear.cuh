@@ -12,10 +12,11 @@
 // The block states M_b are a binary counter over chunks: after chunk c, with j = the number of
 // trailing ones of c, M_j = V_c^T K_c + sum_{b<j} M_b and M_b = 0 for b < j.
 //
-// One CTA per (b, h, slice of BV value channels) walks the chunks in order. Four warps own 16
-// query rows each for the outputs and 32 key channels each for the chunk state; every
-// contraction is a bf16 m16n8k16 warp MMA with fp32 accumulation (the tiles are 16-64 rows,
-// the level bookkeeping sits between them). The block states stay in shared memory in fp32
+// One CTA per (b, h, slice of BV value channels) walks the chunks in order. Eight warps: four
+// own 16 query rows each for the in-chunk part, four the same rows for the block-state
+// readouts and then 32 key channels each for the chunk state; every contraction is a bf16
+// m16n8k16 warp MMA with fp32 accumulation (the tiles are 16-64 rows, the level bookkeeping
+// sits between them). The block states stay in shared memory in fp32
 // (dk x BV per level, for up to LL_LEVELS chunk levels: T <= 64 * 2^LL_LEVELS). The next
 // chunk's tiles are loaded into registers while the current chunk computes (the level
 // states leave no room for a second shared-memory stage) and stored once it is done.
@@ -30,7 +31,7 @@ constexpr int LL_DK = 128;       // key dimension
 constexpr int LL_BV = 32;        // value channels per CTA
 constexpr int LL_LEVELS = 9;     // chunk levels kept (T <= 32768)
 constexpr int LL_LMAX = 16;      // lambda levels per token read (7 in-chunk + LL_LEVELS)
-constexpr int LL_THREADS = 128;
+constexpr int LL_THREADS = 256;
 constexpr int LL_QS = LL_DK + 8;   // bf16 row stride of the Q and K tiles (conflict-free ldmatrix)
 constexpr int LL_VS = LL_BV + 8;   // bf16 row stride of the V tile
 constexpr int LL_MS = LL_BV + 4;   // fp32 row stride of a block state
@@ -41,6 +42,7 @@ struct LoglinearSmem {
     __nv_bfloat16 v[LL_C][LL_VS];
     float lam[LL_C][LL_LMAX];
     float m[LL_LEVELS][LL_DK][LL_MS];  // block states M_b^T: key channel rows, value columns
+    float o[LL_C][LL_BV + 2];          // the block-state part of the chunk's outputs
 };
 
 __device__ __forceinline__ void ll_mma(float* d, const uint32_t* a, const uint32_t* b) {
@@ -130,6 +132,9 @@ __device__ __forceinline__ void LoglinearStage::store(LoglinearSmem& sm) const {
 }
 
 // grid: (B*H, dv / LL_BV); block: LL_THREADS; dynamic shared memory: sizeof(LoglinearSmem).
+// Warps 0-3 take the in-chunk part of the outputs (query rows 16w .. 16w+15); warps 4-7 the
+// readouts of the block states for the same rows, then the chunk state (key channels
+// 32(w-4) .. +31) and the merge. The two halves meet in shared memory before the store.
 __global__ void __launch_bounds__(LL_THREADS) loglinear_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
     const __nv_bfloat16* __restrict__ v, const float* __restrict__ lam,
@@ -138,9 +143,13 @@ __global__ void __launch_bounds__(LL_THREADS) loglinear_kernel(
     LoglinearSmem& sm = *reinterpret_cast<LoglinearSmem*>(ll_smem_raw);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, tg = lane & 3;
+    const bool intra = warp < 4;
+    const int wq = warp & 3;  // row block (both halves) / key-channel block (state)
     const long bh = blockIdx.x;
     const int v0 = blockIdx.y * LL_BV;
     const int nchunks = (T + LL_C - 1) / LL_C;
+    const int r0 = 16 * wq;
+    const int ta = r0 + g, tb = r0 + g + 8;  // this thread's two rows (in-chunk positions)
 
     for (int e = tid; e < LL_LEVELS * LL_DK * LL_MS; e += LL_THREADS) (&sm.m[0][0][0])[e] = 0.f;
     LoglinearStage stage;
@@ -153,13 +162,10 @@ __global__ void __launch_bounds__(LL_THREADS) loglinear_kernel(
         __syncthreads();
         if (c + 1 < nchunks) stage.load(q, k, v, lam, bh, T, dv, v0, L, t0 + LL_C, tid);
 
-        // ---- outputs of rows 16*warp .. +15
-        const int r0 = 16 * warp;
-        const int ta = r0 + g, tb = r0 + g + 8;  // this thread's two rows (in-chunk positions)
         float o[LL_BV / 8][4];
 #pragma unroll
         for (int n = 0; n < LL_BV / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
-        {
+        if (intra) {
             // P = Q K^T over the chunk's 64 keys, weighted by lambda of the pair's level
             float p[LL_C / 8][4];
 #pragma unroll
@@ -188,7 +194,7 @@ __global__ void __launch_bounds__(LL_THREADS) loglinear_kernel(
                     p[n][e] = (s <= t) ? p[n][e] * sm.lam[t][ll_bitlen(t ^ s)] : 0.f;
                 }
             }
-            // O += P V (P from the accumulators as bf16 A fragments)
+            // O = P V (P from the accumulators as bf16 A fragments)
 #pragma unroll
             for (int kk = 0; kk < LL_C / 16; ++kk) {
                 uint32_t a[4];
@@ -205,51 +211,64 @@ __global__ void __launch_bounds__(LL_THREADS) loglinear_kernel(
                     ll_mma(o[2 * n2 + 1], a, b1);
                 }
             }
-        }
-        // earlier chunks: one readout per set bit b of c, weighted by lambda^(7+b)
-        for (int b = 0; b < LL_LEVELS; ++b) {
-            if (!((c >> b) & 1)) continue;
-            float z[LL_BV / 8][4];
+        } else {
+            // earlier chunks: one readout per set bit b of c, weighted by lambda^(7+b)
+            for (int b = 0; b < LL_LEVELS; ++b) {
+                if (!((c >> b) & 1)) continue;
+                float z[LL_BV / 8][4];
 #pragma unroll
-            for (int n = 0; n < LL_BV / 8; ++n) z[n][0] = z[n][1] = z[n][2] = z[n][3] = 0.f;
-            const float(*mb)[LL_MS] = sm.m[b];
+                for (int n = 0; n < LL_BV / 8; ++n) z[n][0] = z[n][1] = z[n][2] = z[n][3] = 0.f;
+                const float(*mb)[LL_MS] = sm.m[b];
 #pragma unroll 4
-            for (int kk = 0; kk < LL_DK / 16; ++kk) {
-                uint32_t a[4];
-                ll_ldsm_x4(a, &sm.q[r0 + (lane & 15)][kk * 16 + (lane >> 4) * 8]);
+                for (int kk = 0; kk < LL_DK / 16; ++kk) {
+                    uint32_t a[4];
+                    ll_ldsm_x4(a, &sm.q[r0 + (lane & 15)][kk * 16 + (lane >> 4) * 8]);
+#pragma unroll
+                    for (int n = 0; n < LL_BV / 8; ++n) {
+                        // B (k = key channel, n = value channel) from the fp32 state, as bf16
+                        const int kc = kk * 16 + 2 * tg, vc = 8 * n + g;
+                        uint32_t bb[2];
+                        bb[0] = pack_bf16(mb[kc][vc], mb[kc + 1][vc]);
+                        bb[1] = pack_bf16(mb[kc + 8][vc], mb[kc + 9][vc]);
+                        ll_mma(z[n], a, bb);
+                    }
+                }
+                const float la = sm.lam[ta][7 + b], lb = sm.lam[tb][7 + b];
 #pragma unroll
                 for (int n = 0; n < LL_BV / 8; ++n) {
-                    // B (k = key channel, n = value channel) from the fp32 state, as bf16
-                    const int kc = kk * 16 + 2 * tg, vc = 8 * n + g;
-                    uint32_t bb[2];
-                    bb[0] = pack_bf16(mb[kc][vc], mb[kc + 1][vc]);
-                    bb[1] = pack_bf16(mb[kc + 8][vc], mb[kc + 9][vc]);
-                    ll_mma(z[n], a, bb);
+                    o[n][0] = fmaf(la, z[n][0], o[n][0]);
+                    o[n][1] = fmaf(la, z[n][1], o[n][1]);
+                    o[n][2] = fmaf(lb, z[n][2], o[n][2]);
+                    o[n][3] = fmaf(lb, z[n][3], o[n][3]);
                 }
             }
-            const float la = sm.lam[ta][7 + b], lb = sm.lam[tb][7 + b];
+            // hand the block-state part of the outputs to the in-chunk warps
 #pragma unroll
             for (int n = 0; n < LL_BV / 8; ++n) {
-                o[n][0] = fmaf(la, z[n][0], o[n][0]);
-                o[n][1] = fmaf(la, z[n][1], o[n][1]);
-                o[n][2] = fmaf(lb, z[n][2], o[n][2]);
-                o[n][3] = fmaf(lb, z[n][3], o[n][3]);
+                const int col = 8 * n + 2 * tg;
+                *reinterpret_cast<float2*>(&sm.o[ta][col]) = make_float2(o[n][0], o[n][1]);
+                *reinterpret_cast<float2*>(&sm.o[tb][col]) = make_float2(o[n][2], o[n][3]);
             }
         }
+        __syncthreads();  // the block-state readouts are done (and their outputs are in sm.o)
+        if (intra) {
 #pragma unroll
-        for (int n = 0; n < LL_BV / 8; ++n) {
-            const int col = v0 + 8 * n + 2 * tg;
-            if (t0 + ta < T)
-                *reinterpret_cast<uint32_t*>(out + (bh * T + t0 + ta) * (long)dv + col) =
-                    pack_bf16(o[n][0], o[n][1]);
-            if (t0 + tb < T)
-                *reinterpret_cast<uint32_t*>(out + (bh * T + t0 + tb) * (long)dv + col) =
-                    pack_bf16(o[n][2], o[n][3]);
+            for (int n = 0; n < LL_BV / 8; ++n) {
+                const int col = 8 * n + 2 * tg;
+                const float2 xa = *reinterpret_cast<const float2*>(&sm.o[ta][col]);
+                const float2 xb = *reinterpret_cast<const float2*>(&sm.o[tb][col]);
+                if (t0 + ta < T)
+                    *reinterpret_cast<uint32_t*>(out + (bh * T + t0 + ta) * (long)dv + v0 + col) =
+                        pack_bf16(o[n][0] + xa.x, o[n][1] + xa.y);
+                if (t0 + tb < T)
+                    *reinterpret_cast<uint32_t*>(out + (bh * T + t0 + tb) * (long)dv + v0 + col) =
+                        pack_bf16(o[n][2] + xb.x, o[n][3] + xb.y);
+            }
+            continue;
         }
-        if (c + 1 == nchunks) break;
-        __syncthreads();  // every readout of the block states is done before they change
+        if (c + 1 == nchunks) continue;
 
-        // ---- this chunk's state V^T K, transposed: rows = key channels 32*warp .. +31
+        // ---- this chunk's state V^T K, transposed: rows = key channels 32*wq .. +31
         float s[2][LL_BV / 8][4];
 #pragma unroll
         for (int mt = 0; mt < 2; ++mt)
@@ -261,7 +280,7 @@ __global__ void __launch_bounds__(LL_THREADS) loglinear_kernel(
             for (int mt = 0; mt < 2; ++mt) {
                 // A (m = key channel, k = token) = K^T: transposed 8x8 loads of the K tile
                 uint32_t a[4];
-                const int kc0 = 32 * warp + 16 * mt;
+                const int kc0 = 32 * wq + 16 * mt;
                 ll_ldsm_x4_t(a, &sm.k[kk * 16 + (lane & 7) + ((lane >> 4) << 3)]
                                      [kc0 + ((lane >> 3) & 1) * 8]);
 #pragma unroll
@@ -274,7 +293,9 @@ __global__ void __launch_bounds__(LL_THREADS) loglinear_kernel(
                 }
             }
         }
-        // ---- binary counter: M_j = this chunk + sum_{b<j} M_b, M_b = 0 for b < j
+        // ---- binary counter: M_j = this chunk + sum_{b<j} M_b, M_b = 0 for b < j. Each
+        // thread touches only its own (key channel, value channel) positions, and every
+        // readout of the block states finished before the barrier above.
         int j = 0;
         while ((c >> j) & 1) ++j;
         if (j < LL_LEVELS) {
@@ -284,7 +305,7 @@ __global__ void __launch_bounds__(LL_THREADS) loglinear_kernel(
                 for (int n = 0; n < LL_BV / 8; ++n) {
 #pragma unroll
                     for (int e = 0; e < 4; ++e) {
-                        const int kc = 32 * warp + 16 * mt + g + ((e & 2) ? 8 : 0);
+                        const int kc = 32 * wq + 16 * mt + g + ((e & 2) ? 8 : 0);
                         const int vc = 8 * n + 2 * tg + (e & 1);
                         float x = s[mt][n][e];
                         for (int b = 0; b < j; ++b) {

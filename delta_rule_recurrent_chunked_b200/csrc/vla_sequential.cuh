@@ -71,11 +71,21 @@ __device__ __forceinline__ void vla_group_sum(float* x, float (*red)[4], int i) 
     }
 }
 
+// Starts the copy of nt token rows of one operand into a tile buffer: 16-byte asynchronous
+// copies (cp.async), so the issuing thread does not wait for HBM; vla_tiles_landed() waits
+// for this thread's copies before the tile barrier that publishes them.
 template <int D>
 __device__ __forceinline__ void vla_load_tile(float (*dst)[D], const float* src, int nt, int tid) {
-    const float4* s4 = reinterpret_cast<const float4*>(src);
-    float4* d4 = reinterpret_cast<float4*>(&dst[0][0]);
-    for (int e = tid; e < nt * D / 4; e += D) d4[e] = s4[e];
+    const char* s = reinterpret_cast<const char*>(src);
+    const uint32_t d = smem_u32(&dst[0][0]);
+    for (int e = tid; e < nt * D / 4; e += D)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(d + 16u * e),
+                     "l"(s + 16l * e)
+                     : "memory");
+}
+
+__device__ __forceinline__ void vla_tiles_landed() {
+    asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
 }
 
 // grid: B*H; block: 2*D threads; dynamic shared memory: sizeof(VlaSmem<D>).
@@ -114,6 +124,7 @@ __global__ void __launch_bounds__(2 * D) vla_sequential_kernel(
             vla_load_tile<D>(sm.uA[0], u + seq, nt, i);
             vla_load_tile<D>(sm.kA[0], k + seq, nt, i);
             vla_load_tile<D>(sm.qA[0], q + seq, nt, i);
+            vla_tiles_landed();
         }
     } else {
         if (S0) {
@@ -227,6 +238,7 @@ __global__ void __launch_bounds__(2 * D) vla_sequential_kernel(
                 }
             }
         }
+        vla_tiles_landed();  // the next tile's copies are in shared memory before the barrier
         __syncthreads();
     }
 
