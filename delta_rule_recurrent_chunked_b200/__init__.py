@@ -25,6 +25,7 @@ DR_FORCE_SEQUENTIAL = 0x200
 DR_OK, DR_ERR_INVALID_ARG, DR_ERR_UNSUPPORTED, DR_ERR_CUDA, DR_ERR_TIMEOUT, DR_ERR_DEVICE_BOUNDS = (
     0, -1, -2, -3, -4, -5)
 DR_ERR_GATE_RANGE = -6
+DR_ERR_NOT_SPD = -7
 MODES = {"linear": DR_LINEAR, "deltanet": DR_DELTANET, "gdn": DR_GDN, "kda": DR_KDA,
          "gdn2": DR_GDN2}
 
@@ -287,9 +288,11 @@ def decode_step(q, k, v, beta=None, gate=None, S=None, mode="gdn", out=None):
     return out
 
 
-def vla_scan(q, k, v, u, S0=None, A0=None, lambda0=1.0, want_state=True, out=None):
+def vla_scan(q, k, v, u, S0=None, A0=None, lambda0=1.0, want_state=True, out=None,
+             sequential=False):
     """VLA Sherman-Morrison scan on the GPU (fp32). q, k, v, u: [B,H,T,d];
-    S0, A0: [B,H,d,d] or None. Returns (out, S_final, A_final)."""
+    S0, A0: [B,H,d,d] or None. Returns (out, S_final, A_final). The chunked pair of
+    kernels runs by default; sequential=True selects the per-token kernel."""
     import torch
 
     B, H, T, d = q.shape
@@ -304,22 +307,25 @@ def vla_scan(q, k, v, u, S0=None, A0=None, lambda0=1.0, want_state=True, out=Non
     _check(out, "out", (B, H, T, d), torch.float32, dev)
     Sf = torch.empty((B, H, d, d), dtype=torch.float32, device=dev) if want_state else None
     Af = torch.empty((B, H, d, d), dtype=torch.float32, device=dev) if want_state else None
-    rc = lib().vla_scan_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(S0), _ptr(A0),
-                            float(lambda0), _ptr(out), _ptr(Sf), _ptr(Af), B, H, T, d,
-                            _stream_handle(dev))
+    flags = VLA_SEQUENTIAL if sequential else 0
+    rc = lib().vla_scan_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(S0), _ptr(A0), None,
+                               float(lambda0), _ptr(out), _ptr(Sf), _ptr(Af), None, B, H, T,
+                               d, flags, _stream_handle(dev))
     if rc != DR_OK:
-        raise DrScanError(rc, "vla_scan_fwd")
+        raise DrScanError(rc, "vla_scan_fwd_ex")
     return out, Sf, Af
 
 
 VLA_RATIO_READOUT = 0x1
+VLA_SEQUENTIAL = 0x2
 
 
 def vla_scan_ratio(q, k, v, u, S0=None, A0=None, n0=None, lambda0=1.0, want_state=True,
-                   out=None):
+                   out=None, sequential=False):
     """VLA scan with the ratio readout o_t = S_t q_t / (n_t q_t) (fp32), through
     vla_scan_fwd_ex. q: [B,H,T,d] feature-mapped queries (phi(q)); k: unit-norm
-    feature-mapped keys; n0: [B,H,d] or None. Returns (out, S_final, A_final, n_final)."""
+    feature-mapped keys; n0: [B,H,d] or None. Returns (out, S_final, A_final, n_final).
+    sequential=True selects the per-token kernel instead of the chunked pair."""
     import torch
 
     B, H, T, d = q.shape
@@ -339,7 +345,8 @@ def vla_scan_ratio(q, k, v, u, S0=None, A0=None, n0=None, lambda0=1.0, want_stat
     nf = torch.empty((B, H, d), dtype=torch.float32, device=dev) if want_state else None
     rc = lib().vla_scan_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(S0), _ptr(A0), _ptr(n0),
                                float(lambda0), _ptr(out), _ptr(Sf), _ptr(Af), _ptr(nf), B, H, T,
-                               d, VLA_RATIO_READOUT, _stream_handle(dev))
+                               d, VLA_RATIO_READOUT | (VLA_SEQUENTIAL if sequential else 0),
+                               _stream_handle(dev))
     if rc != DR_OK:
         raise DrScanError(rc, "vla_scan_fwd_ex")
     return out, Sf, Af, nf

@@ -5,12 +5,14 @@
 #include <climits>
 #include <cstdint>
 #include <cstdio>
+#include <mutex>
 
 #include "common.cuh"
 #include "dr_chunked.cuh"
 #include "dr_decode.cuh"
 #include "dr_sequential.cuh"
 #include "loglinear.cuh"
+#include "vla_chunked.cuh"
 #include "vla_sequential.cuh"
 
 using namespace drscan;
@@ -151,16 +153,82 @@ int launch_vla(const float* q, const float* k, const float* v, const float* u, c
     return launch_status();
 }
 
+// Stream-ordered scratch from a memory pool of this library's own, one per device, that
+// keeps its memory between calls (release threshold at the maximum), so that a call after
+// the first one does not go to the driver for memory.
+int scratch_alloc(void** p, size_t bytes, cudaStream_t stream) {
+    constexpr int kMaxDev = 64;
+    static std::mutex mu;
+    static cudaMemPool_t pools[kMaxDev] = {};
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return DR_ERR_CUDA;
+    cudaMemPool_t pool;
+    {
+        std::lock_guard<std::mutex> lock(mu);
+        if (!pools[dev]) {
+            cudaMemPoolProps props = {};
+            props.allocType = cudaMemAllocationTypePinned;
+            props.handleTypes = cudaMemHandleTypeNone;
+            props.location.type = cudaMemLocationTypeDevice;
+            props.location.id = dev;
+            cudaMemPool_t created;
+            if (cudaMemPoolCreate(&created, &props) != cudaSuccess) return DR_ERR_CUDA;
+            uint64_t keep = UINT64_MAX;
+            cudaMemPoolSetAttribute(created, cudaMemPoolAttrReleaseThreshold, &keep);
+            pools[dev] = created;
+        }
+        pool = pools[dev];
+    }
+    return cudaMallocFromPoolAsync(p, bytes, pool, stream) == cudaSuccess ? DR_OK : DR_ERR_CUDA;
+}
+
+// The chunked pair: the A-phase writes alpha_hat into scratch, the S-phase reads it.
+template <int D, bool RATIO>
+int launch_vla_chunked(const float* q, const float* k, const float* v, const float* u,
+                       const float* S0, const float* A0, const float* n0, float lambda0,
+                       float* out, float* S_final, float* A_final, float* n_final, long BH,
+                       int T, cudaStream_t stream) {
+    const int smem_a = (int)sizeof(VcASmem<D>);
+    const int smem_s = (int)sizeof(VcSSmem<D>);
+    auto ka = vla_aphase_kernel<D>;
+    auto ks = vla_sphase_kernel<D, RATIO>;
+    if (cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_a) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_s) !=
+            cudaSuccess)
+        return DR_ERR_CUDA;
+    void* scratch = nullptr;
+    int rc = scratch_alloc(&scratch, (size_t)BH * T * D * sizeof(float), stream);
+    if (rc != DR_OK) return rc;
+    float* alpha = static_cast<float*>(scratch);
+    ka<<<(unsigned)BH, VC_THREADS, smem_a, stream>>>(k, u, A0, lambda0, A_final, alpha, T);
+    rc = launch_status();
+    if (rc == DR_OK) {
+        ks<<<dim3((unsigned)BH, D / VC_RS), VC_THREADS, smem_s, stream>>>(
+            q, k, v, alpha, S0, n0, out, S_final, n_final, T);
+        rc = launch_status();
+    }
+    if (cudaFreeAsync(scratch, stream) != cudaSuccess && rc == DR_OK) rc = DR_ERR_CUDA;
+    return rc;
+}
+
 template <int D>
-int launch_vla_readout(bool ratio, const float* q, const float* k, const float* v,
-                       const float* u, const float* S0, const float* A0, const float* n0,
-                       float lambda0, float* out, float* S_final, float* A_final, float* n_final,
-                       long BH, int T, cudaStream_t stream) {
+int launch_vla_readout(bool ratio, bool sequential, const float* q, const float* k,
+                       const float* v, const float* u, const float* S0, const float* A0,
+                       const float* n0, float lambda0, float* out, float* S_final,
+                       float* A_final, float* n_final, long BH, int T, cudaStream_t stream) {
+    if (sequential) {
+        if (ratio)
+            return launch_vla<D, true>(q, k, v, u, S0, A0, n0, lambda0, out, S_final, A_final,
+                                       n_final, BH, T, stream);
+        return launch_vla<D, false>(q, k, v, u, S0, A0, nullptr, lambda0, out, S_final,
+                                    A_final, nullptr, BH, T, stream);
+    }
     if (ratio)
-        return launch_vla<D, true>(q, k, v, u, S0, A0, n0, lambda0, out, S_final, A_final,
-                                   n_final, BH, T, stream);
-    return launch_vla<D, false>(q, k, v, u, S0, A0, nullptr, lambda0, out, S_final, A_final,
-                                nullptr, BH, T, stream);
+        return launch_vla_chunked<D, true>(q, k, v, u, S0, A0, n0, lambda0, out, S_final,
+                                           A_final, n_final, BH, T, stream);
+    return launch_vla_chunked<D, false>(q, k, v, u, S0, A0, nullptr, lambda0, out, S_final,
+                                        A_final, nullptr, BH, T, stream);
 }
 
 __global__ void timeout_probe_kernel(int spin_limit) {
@@ -201,6 +269,9 @@ const char* dr_status_string(int status) {
         case DR_ERR_GATE_RANGE:
             return "device: a KDA gate's summed log-decay over one chunk is below the chunked "
                    "kernel's range; outputs are invalid (rerun with DR_FORCE_SEQUENTIAL)";
+        case DR_ERR_NOT_SPD:
+            return "device: VLA's inverse penalty A is not positive definite (a non-positive "
+                   "pivot in I + U A U^T); outputs are invalid";
     }
     return "unknown status";
 }
@@ -295,8 +366,9 @@ int vla_scan_fwd_ex(const float* q, const float* k, const float* v, const float*
                     const float* S0, const float* A0, const float* n0, float lambda0, float* out,
                     float* S_final, float* A_final, float* n_final, int B, int H, int T, int d,
                     int flags, cudaStream_t stream) {
-    if (flags & ~VLA_RATIO_READOUT) return DR_ERR_INVALID_ARG;
+    if (flags & ~(VLA_RATIO_READOUT | VLA_SEQUENTIAL)) return DR_ERR_INVALID_ARG;
     const bool ratio = (flags & VLA_RATIO_READOUT) != 0;
+    const bool sequential = (flags & VLA_SEQUENTIAL) != 0;
     if (!ratio && (n0 || n_final)) return DR_ERR_INVALID_ARG;
     if (!ok_opt(n0) || !ok_opt(n_final)) return DR_ERR_INVALID_ARG;
     if (B < 0 || H < 0 || T < 0 || d <= 0) return DR_ERR_INVALID_ARG;
@@ -323,17 +395,17 @@ int vla_scan_fwd_ex(const float* q, const float* k, const float* v, const float*
     }
     switch (d) {
         case 32:
-            return launch_vla_readout<32>(ratio, q, k, v, u, S0, A0, n0, lambda0, out, S_final,
-                                          A_final, n_final, BH, T, stream);
+            return launch_vla_readout<32>(ratio, sequential, q, k, v, u, S0, A0, n0, lambda0,
+                                          out, S_final, A_final, n_final, BH, T, stream);
         case 64:
-            return launch_vla_readout<64>(ratio, q, k, v, u, S0, A0, n0, lambda0, out, S_final,
-                                          A_final, n_final, BH, T, stream);
+            return launch_vla_readout<64>(ratio, sequential, q, k, v, u, S0, A0, n0, lambda0,
+                                          out, S_final, A_final, n_final, BH, T, stream);
         case 96:
-            return launch_vla_readout<96>(ratio, q, k, v, u, S0, A0, n0, lambda0, out, S_final,
-                                          A_final, n_final, BH, T, stream);
+            return launch_vla_readout<96>(ratio, sequential, q, k, v, u, S0, A0, n0, lambda0,
+                                          out, S_final, A_final, n_final, BH, T, stream);
         case 128:
-            return launch_vla_readout<128>(ratio, q, k, v, u, S0, A0, n0, lambda0, out, S_final,
-                                           A_final, n_final, BH, T, stream);
+            return launch_vla_readout<128>(ratio, sequential, q, k, v, u, S0, A0, n0, lambda0,
+                                           out, S_final, A_final, n_final, BH, T, stream);
     }
     return DR_ERR_UNSUPPORTED;
 }

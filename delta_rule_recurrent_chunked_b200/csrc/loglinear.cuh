@@ -34,14 +34,14 @@ constexpr int LL_LMAX = 16;      // lambda levels per token read (7 in-chunk + L
 constexpr int LL_THREADS = 256;
 constexpr int LL_QS = LL_DK + 8;   // bf16 row stride of the Q and K tiles (conflict-free ldmatrix)
 constexpr int LL_VS = LL_BV + 8;   // bf16 row stride of the V tile
-constexpr int LL_MS = LL_BV + 4;   // fp32 row stride of a block state
+constexpr int LL_MS = LL_DK + 8;   // fp32 row stride of a block state (rows = value channels)
 
 struct LoglinearSmem {
     __nv_bfloat16 q[LL_C][LL_QS];
     __nv_bfloat16 k[LL_C][LL_QS];
     __nv_bfloat16 v[LL_C][LL_VS];
     float lam[LL_C][LL_LMAX];
-    float m[LL_LEVELS][LL_DK][LL_MS];  // block states M_b^T: key channel rows, value columns
+    float m[LL_LEVELS][LL_BV][LL_MS];  // block states M_b: value channel rows, key columns
     float o[LL_C][LL_BV + 2];          // the block-state part of the chunk's outputs
 };
 
@@ -67,6 +67,22 @@ __device__ __forceinline__ void ll_ldsm_x4_t(uint32_t* r, const void* p) {
 
 __device__ __forceinline__ int ll_bitlen(int x) { return 32 - __clz(x); }
 
+// Read-only global loads issued exactly where they stand (volatile asm keeps their place among
+// the kernel's barriers), so that the next chunk's prefetch overlaps the current chunk's work.
+__device__ __forceinline__ uint4 ll_ld_pinned_u4(const void* p) {
+    uint4 r;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+__device__ __forceinline__ float ll_ld_pinned_f(const float* p) {
+    float r;
+    asm volatile("ld.global.nc.f32 %0, [%1];" : "=f"(r) : "l"(p));
+    return r;
+}
+
 // One chunk's tiles in registers, spread over the CTA's threads (rows past T as zeros, their
 // lambdas as zero): loaded from HBM early, stored to shared memory when the tiles are free.
 struct LoglinearStage {
@@ -87,8 +103,8 @@ struct LoglinearStage {
             const int r = e / (LL_DK / 8), c8 = (e % (LL_DK / 8)) * 8;
             qv[i] = kv[i] = make_uint4(0, 0, 0, 0);
             if (t0 + r < T) {
-                qv[i] = *reinterpret_cast<const uint4*>(q + (bh * T + t0 + r) * (long)LL_DK + c8);
-                kv[i] = *reinterpret_cast<const uint4*>(k + (bh * T + t0 + r) * (long)LL_DK + c8);
+                qv[i] = ll_ld_pinned_u4(q + (bh * T + t0 + r) * (long)LL_DK + c8);
+                kv[i] = ll_ld_pinned_u4(k + (bh * T + t0 + r) * (long)LL_DK + c8);
             }
         }
 #pragma unroll
@@ -96,13 +112,13 @@ struct LoglinearStage {
             const int e = tid + i * LL_THREADS;
             const int r = e / (LL_BV / 8), c8 = (e % (LL_BV / 8)) * 8;
             vv[i] = make_uint4(0, 0, 0, 0);
-            if (t0 + r < T) vv[i] = *reinterpret_cast<const uint4*>(v + (bh * T + t0 + r) * (long)dv + v0 + c8);
+            if (t0 + r < T) vv[i] = ll_ld_pinned_u4(v + (bh * T + t0 + r) * (long)dv + v0 + c8);
         }
 #pragma unroll
         for (int i = 0; i < NL; ++i) {
             const int e = tid + i * LL_THREADS;
             const int r = e / LL_LMAX, l = e % LL_LMAX;
-            lv[i] = (t0 + r < T && l < L) ? lam[(bh * T + t0 + r) * (long)L + l] : 0.f;
+            lv[i] = (t0 + r < T && l < L) ? ll_ld_pinned_f(lam + (bh * T + t0 + r) * (long)L + l) : 0.f;
         }
     }
 
@@ -151,7 +167,7 @@ __global__ void __launch_bounds__(LL_THREADS) loglinear_kernel(
     const int r0 = 16 * wq;
     const int ta = r0 + g, tb = r0 + g + 8;  // this thread's two rows (in-chunk positions)
 
-    for (int e = tid; e < LL_LEVELS * LL_DK * LL_MS; e += LL_THREADS) (&sm.m[0][0][0])[e] = 0.f;
+    for (int e = tid; e < LL_LEVELS * LL_BV * LL_MS; e += LL_THREADS) (&sm.m[0][0][0])[e] = 0.f;
     LoglinearStage stage;
     if (nchunks > 0) stage.load(q, k, v, lam, bh, T, dv, v0, L, 0, tid);
 
@@ -225,11 +241,14 @@ __global__ void __launch_bounds__(LL_THREADS) loglinear_kernel(
                     ll_ldsm_x4(a, &sm.q[r0 + (lane & 15)][kk * 16 + (lane >> 4) * 8]);
 #pragma unroll
                     for (int n = 0; n < LL_BV / 8; ++n) {
-                        // B (k = key channel, n = value channel) from the fp32 state, as bf16
+                        // B (k = key channel, n = value channel) from the fp32 state, as bf16:
+                        // two adjacent key channels of one value row per 8-byte load
                         const int kc = kk * 16 + 2 * tg, vc = 8 * n + g;
+                        const float2 lo = *reinterpret_cast<const float2*>(&mb[vc][kc]);
+                        const float2 hi = *reinterpret_cast<const float2*>(&mb[vc][kc + 8]);
                         uint32_t bb[2];
-                        bb[0] = pack_bf16(mb[kc][vc], mb[kc + 1][vc]);
-                        bb[1] = pack_bf16(mb[kc + 8][vc], mb[kc + 9][vc]);
+                        bb[0] = pack_bf16(lo.x, lo.y);
+                        bb[1] = pack_bf16(hi.x, hi.y);
                         ll_mma(z[n], a, bb);
                     }
                 }
@@ -309,10 +328,10 @@ __global__ void __launch_bounds__(LL_THREADS) loglinear_kernel(
                         const int vc = 8 * n + 2 * tg + (e & 1);
                         float x = s[mt][n][e];
                         for (int b = 0; b < j; ++b) {
-                            x += sm.m[b][kc][vc];
-                            sm.m[b][kc][vc] = 0.f;
+                            x += sm.m[b][vc][kc];
+                            sm.m[b][vc][kc] = 0.f;
                         }
-                        sm.m[j][kc][vc] = x;
+                        sm.m[j][vc][kc] = x;
                     }
                 }
             }

@@ -153,15 +153,21 @@ __global__ void __launch_bounds__(2 * D) vla_sequential_kernel(
                     const int par = tt & 1;  // VLA_TILE is even: parity of the token index
                     const float* uu = sm.uA[b][tt];
                     const float* kk = sm.kA[b][tt];
-                    // four partial sums per product: dependent FMA chains of D/4
+                    // four partial sums per product (dependent FMA chains of D/4); the shared
+                    // operands are read four at a time
                     float z4[4] = {0.f, 0.f, 0.f, 0.f}, y4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int j = 0; j < D; j += 4) {
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            z4[e] = fmaf(m[j + e], uu[j + e], z4[e]);
-                            y4[e] = fmaf(m[j + e], kk[j + e], y4[e]);
-                        }
+                        const float4 u4 = *reinterpret_cast<const float4*>(uu + j);
+                        const float4 k4 = *reinterpret_cast<const float4*>(kk + j);
+                        z4[0] = fmaf(m[j], u4.x, z4[0]);
+                        z4[1] = fmaf(m[j + 1], u4.y, z4[1]);
+                        z4[2] = fmaf(m[j + 2], u4.z, z4[2]);
+                        z4[3] = fmaf(m[j + 3], u4.w, z4[3]);
+                        y4[0] = fmaf(m[j], k4.x, y4[0]);
+                        y4[1] = fmaf(m[j + 1], k4.y, y4[1]);
+                        y4[2] = fmaf(m[j + 2], k4.z, y4[2]);
+                        y4[3] = fmaf(m[j + 3], k4.w, y4[3]);
                     }
                     const float z = (z4[0] + z4[1]) + (z4[2] + z4[3]);
                     const float y = (y4[0] + y4[1]) + (y4[2] + y4[3]);
@@ -185,8 +191,15 @@ __global__ void __launch_bounds__(2 * D) vla_sequential_kernel(
                     const float c = 1.f / (1.f + r1[0]);
                     const float w = c * r1[1];
                     const float* zb = sm.zbuf[par];
+                    const float cz = -c * z;
 #pragma unroll
-                    for (int j = 0; j < D; ++j) m[j] = fmaf(-c * z, zb[j], m[j]);
+                    for (int j = 0; j < D; j += 4) {
+                        const float4 z4v = *reinterpret_cast<const float4*>(zb + j);
+                        m[j] = fmaf(cz, z4v.x, m[j]);
+                        m[j + 1] = fmaf(cz, z4v.y, m[j + 1]);
+                        m[j + 2] = fmaf(cz, z4v.z, m[j + 2]);
+                        m[j + 3] = fmaf(cz, z4v.w, m[j + 3]);
+                    }
                     const float yt = fmaf(-w, z, y);  // A_t k = A_{t-1}k - c z (z.k)
                     const float n2 = fmaf(w * w, r1[4], fmaf(-2.f * w, r1[3], r1[2]));
                     const float inv = rsqrtf(n2);
@@ -220,16 +233,27 @@ __global__ void __launch_bounds__(2 * D) vla_sequential_kernel(
                     float p4[4] = {0.f, 0.f, 0.f, 0.f}, o4[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
                     for (int j = 0; j < D; j += 4) {
-#pragma unroll
-                        for (int e = 0; e < 4; ++e) {
-                            p4[e] = fmaf(m[j + e], kk[j + e], p4[e]);
-                            o4[e] = fmaf(m[j + e], qq[j + e], o4[e]);
-                        }
+                        const float4 k4 = *reinterpret_cast<const float4*>(kk + j);
+                        const float4 q4 = *reinterpret_cast<const float4*>(qq + j);
+                        p4[0] = fmaf(m[j], k4.x, p4[0]);
+                        p4[1] = fmaf(m[j + 1], k4.y, p4[1]);
+                        p4[2] = fmaf(m[j + 2], k4.z, p4[2]);
+                        p4[3] = fmaf(m[j + 3], k4.w, p4[3]);
+                        o4[0] = fmaf(m[j], q4.x, o4[0]);
+                        o4[1] = fmaf(m[j + 1], q4.y, o4[1]);
+                        o4[2] = fmaf(m[j + 2], q4.z, o4[2]);
+                        o4[3] = fmaf(m[j + 3], q4.w, o4[3]);
                     }
                     const float o0 = (o4[0] + o4[1]) + (o4[2] + o4[3]), o1 = 0.f;
                     const float r = sm.vS[b][tt][i] - ((p4[0] + p4[1]) + (p4[2] + p4[3]));
 #pragma unroll
-                    for (int j = 0; j < D; ++j) m[j] = fmaf(r, al[j], m[j]);
+                    for (int j = 0; j < D; j += 4) {
+                        const float4 a4 = *reinterpret_cast<const float4*>(al + j);
+                        m[j] = fmaf(r, a4.x, m[j]);
+                        m[j + 1] = fmaf(r, a4.y, m[j + 1]);
+                        m[j + 2] = fmaf(r, a4.z, m[j + 2]);
+                        m[j + 3] = fmaf(r, a4.w, m[j + 3]);
+                    }
                     const float o = fmaf(r, sm.aq[b][tt], o0 + o1);  // s_t.q after the write
                     if constexpr (RATIO)
                         out[seq + (long)(t0 + tt) * D + i] = o / sm.den[b][tt];

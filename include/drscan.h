@@ -67,8 +67,11 @@ enum {
     DR_ERR_CUDA = -3,        /* a CUDA runtime/driver call failed (launch, attributes) */
     DR_ERR_TIMEOUT = -4,     /* device: a bounded wait on a barrier ran out; outputs invalid */
     DR_ERR_DEVICE_BOUNDS = -5, /* device: an index check failed; outputs invalid */
-    DR_ERR_GATE_RANGE = -6   /* device: a KDA gate decayed past the chunked kernel's range
+    DR_ERR_GATE_RANGE = -6,  /* device: a KDA gate decayed past the chunked kernel's range
                                 (see dr_scan_fwd); outputs invalid */
+    DR_ERR_NOT_SPD = -7      /* device: the chunked VLA scan met a non-positive pivot in
+                                I + U A U^T, i.e. A was not positive definite (an A0 that is
+                                not an inverse penalty); outputs invalid */
 };
 
 /*
@@ -175,7 +178,16 @@ int dr_decode_step_ex(const void* q, const void* k, const void* v, const float* 
  *   S_final, A_final  [B,H,d,d] fp32, or NULL to skip
  *
  * Supported: d in {32, 64, 96, 128}; T >= 0. Non-NULL pointers 16-byte aligned; when
- * B*H*T == 0, q, k, v, u and out are not read and may be NULL.
+ * B*H*T == 0, q, k, v, u and out are not read and may be NULL. A0, when given, must be
+ * symmetric positive definite (it is the inverse of a penalty matrix).
+ *
+ * The scan runs chunked, 64 tokens at a time, in two kernels. The first turns the chunk's
+ * Sherman-Morrison steps into one Woodbury update (a 64 x 64 Cholesky factorisation of
+ * I + U A U^T) and writes every alpha_hat_t; the second applies the write and readout in
+ * the WY form of a delta rule whose read key is k_t and write key alpha_hat_t. Between them
+ * alpha_hat lives in B*H*T*d*4 bytes of scratch, taken stream-ordered from a memory pool of
+ * the library's own (kept between calls) and released in stream order after the second
+ * kernel. Where A stops being positive definite the device latches DR_ERR_NOT_SPD.
  * Returns DR_OK or a negative status; on error nothing is launched.
  */
 int vla_scan_fwd(const float* q, const float* k, const float* v, const float* u,
@@ -185,6 +197,10 @@ int vla_scan_fwd(const float* q, const float* k, const float* v, const float* u,
 
 /* vla_scan_fwd_ex flag: the ratio readout (see below). */
 #define VLA_RATIO_READOUT 0x1
+/* vla_scan_fwd_ex flag: the per-token kernel (one CTA per head, the Sherman-Morrison steps
+ * one token at a time) instead of the chunked pair. Same results up to rounding, no
+ * scratch memory; slower. For testing and as a baseline. */
+#define VLA_SEQUENTIAL 0x2
 
 /*
  * vla_scan_fwd_ex -- vla_scan_fwd with the ratio readout of "Variational Linear Attention
@@ -200,7 +216,8 @@ int vla_scan_fwd(const float* q, const float* k, const float* v, const float* u,
  *
  *   n0       [B,H,d] fp32 initial denominator state, or NULL for zeros (ratio readout only)
  *   n_final  [B,H,d] fp32 final denominator state, or NULL to skip (ratio readout only)
- *   flags    0 (o_t = S_t q_t, exactly vla_scan_fwd) or VLA_RATIO_READOUT
+ *   flags    0 (o_t = S_t q_t, exactly vla_scan_fwd) or VLA_RATIO_READOUT, optionally
+ *            with VLA_SEQUENTIAL
  *
  * Other arguments, rules and return values as vla_scan_fwd; n0 / n_final with flags = 0
  * return DR_ERR_INVALID_ARG. The denominator is not guarded: where n_t q_t is zero the output

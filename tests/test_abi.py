@@ -42,7 +42,8 @@ def test_library_exports_every_declared_symbol(lib):
 def test_version_and_status_strings(lib):
     assert lib.dr_version() >= 100
     codes = [drs.DR_OK, drs.DR_ERR_INVALID_ARG, drs.DR_ERR_UNSUPPORTED, drs.DR_ERR_CUDA,
-             drs.DR_ERR_TIMEOUT, drs.DR_ERR_DEVICE_BOUNDS, drs.DR_ERR_GATE_RANGE]
+             drs.DR_ERR_TIMEOUT, drs.DR_ERR_DEVICE_BOUNDS, drs.DR_ERR_GATE_RANGE,
+             drs.DR_ERR_NOT_SPD]
     texts = [drs.status_string(c) for c in codes]
     assert all(t and t != "unknown status" for t in texts)
     assert len(set(texts)) == len(texts)
@@ -139,6 +140,21 @@ def call_vla(lib, q=A, k=A, v=A, u=A, S0=None, A0=None, lam=1.0, out=A, B=1, H=1
 ])
 def test_vla_argument_validation(lib, kw, code):
     assert call_vla(lib, **kw) == code
+
+
+def call_vla_ex(lib, flags, B=1, n0=None):
+    P = ctypes.c_void_p
+    return lib.vla_scan_fwd_ex(P(A), P(A), P(A), P(A), None, None, P(n0), 1.0, P(A), None, None,
+                               None, B, 1, 8, 32, flags, None)
+
+
+def test_vla_ex_flags(lib):
+    assert call_vla_ex(lib, 0x4) == drs.DR_ERR_INVALID_ARG
+    assert call_vla_ex(lib, drs.VLA_SEQUENTIAL | 0x8) == drs.DR_ERR_INVALID_ARG
+    assert call_vla_ex(lib, drs.VLA_SEQUENTIAL, n0=A) == drs.DR_ERR_INVALID_ARG  # n0: ratio only
+    for flags in (0, drs.VLA_SEQUENTIAL, drs.VLA_RATIO_READOUT,
+                  drs.VLA_RATIO_READOUT | drs.VLA_SEQUENTIAL):
+        assert call_vla_ex(lib, flags, B=0) == drs.DR_OK
 
 
 def test_timeout_probe_rejects_bad_limits(lib):

@@ -420,13 +420,15 @@ def test_decode_offsets_beyond_int32(oracle):
     torch.cuda.empty_cache()
 
 
-# --- VLA
+# --- VLA: the chunked pair (default) and the per-token kernel (sequential=True)
+@pytest.mark.parametrize("sequential", [False, True])
 @pytest.mark.parametrize("d", [32, 96])
-def test_vla_workload(oracle, d):
+def test_vla_workload(oracle, d, sequential):
     w = wl.workload(f"vla_fp32_d{d}")
     inputs = wl.generate_vla(w, 0)
     dev = {k: torch.from_numpy(inputs[k]).cuda() for k in ("q", "k", "v", "u")}
-    out, Sf, Af = drs.vla_scan(dev["q"], dev["k"], dev["v"], dev["u"], lambda0=w.lambda0)
+    out, Sf, Af = drs.vla_scan(dev["q"], dev["k"], dev["v"], dev["u"], lambda0=w.lambda0,
+                               sequential=sequential)
     torch.cuda.synchronize()
     heads = [0, 9, 31]
     sub = wl.head_slice(inputs, heads)
@@ -439,9 +441,10 @@ def test_vla_workload(oracle, d):
         assert row_rel_err(got, ref) <= 1e-4, row_rel_err(got, ref)
 
 
+@pytest.mark.parametrize("sequential", [False, True])
 @pytest.mark.parametrize("d", [32, 64, 96, 128])
-@pytest.mark.parametrize("T", [1, 17, 100])
-def test_vla_small_with_initial_state(oracle, d, T):
+@pytest.mark.parametrize("T", [1, 17, 64, 65, 100, 129])
+def test_vla_small_with_initial_state(oracle, d, T, sequential):
     rng = np.random.default_rng(d + T)
     B, H = 1, 3
     unit = lambda x: x / np.linalg.norm(x, axis=-1, keepdims=True)
@@ -453,8 +456,9 @@ def test_vla_small_with_initial_state(oracle, d, T):
     M = rng.standard_normal((B, H, d, d)) / np.sqrt(d)
     A0 = np.linalg.inv(np.eye(d) + M @ np.swapaxes(M, -1, -2)).astype(np.float32)
     c = lambda x: torch.from_numpy(x).cuda()
-    out, Sf, Af = drs.vla_scan(c(q), c(k), c(v), c(u), S0=c(S0), A0=c(A0))
+    out, Sf, Af = drs.vla_scan(c(q), c(k), c(v), c(u), S0=c(S0), A0=c(A0), sequential=sequential)
     torch.cuda.synchronize()
+    assert drs.poll_error() == drs.DR_OK
     ro, rs, ra = oracle.vla_scan(q, k, v, u, S0=S0, A0=A0)
     assert rel_err(tensor_np(out), ro) <= 1e-4
     assert rel_err(tensor_np(Sf), rs) <= 1e-4
@@ -468,6 +472,43 @@ def test_vla_empty_sequence_returns_initial_state():
     torch.cuda.synchronize()
     eye = torch.eye(d, device="cuda") / 4.0
     assert torch.count_nonzero(Sf) == 0 and torch.allclose(Af, eye.expand_as(Af))
+
+
+@pytest.mark.parametrize("d", [32, 128])
+def test_vla_chunked_long_sequence_with_state(oracle, d):
+    # 1000 tokens: 15 full chunks and a ragged one, entering S0 and A0 (a positive definite
+    # inverse penalty), every head against the oracle
+    rng = np.random.default_rng(40 + d)
+    B, H, T = 2, 2, 1000
+    unit = lambda x: x / np.linalg.norm(x, axis=-1, keepdims=True)
+    q = unit(rng.standard_normal((B, H, T, d))).astype(np.float32)
+    k = unit(rng.standard_normal((B, H, T, d))).astype(np.float32)
+    v = rng.standard_normal((B, H, T, d)).astype(np.float32)
+    u = (rng.standard_normal((B, H, T, d)) / np.sqrt(d)).astype(np.float32)
+    S0 = (0.1 * rng.standard_normal((B, H, d, d))).astype(np.float32)
+    M = rng.standard_normal((B, H, d, d)) / np.sqrt(d)
+    A0 = np.linalg.inv(np.eye(d) + M @ np.swapaxes(M, -1, -2)).astype(np.float32)
+    c = lambda x: torch.from_numpy(x).cuda()
+    out, Sf, Af = drs.vla_scan(c(q), c(k), c(v), c(u), S0=c(S0), A0=c(A0))
+    torch.cuda.synchronize()
+    assert drs.poll_error() == drs.DR_OK
+    ro, rs, ra = oracle.vla_scan(q, k, v, u, S0=S0, A0=A0)
+    for got, ref in ((out, ro), (Sf, rs), (Af, ra)):
+        assert rel_err(tensor_np(got), ref) <= 1e-4
+        assert row_rel_err(tensor_np(got), ref) <= 1e-4
+
+
+def test_vla_chunked_non_positive_definite_a0_is_reported():
+    # A0 = -10 I is no inverse penalty: I + U A0 U^T has a negative pivot, which the chunked
+    # kernel reports instead of returning numbers
+    d, T = 32, 64
+    rng = np.random.default_rng(5)
+    x = torch.from_numpy((rng.standard_normal((1, 1, T, d)) / np.sqrt(d)).astype(np.float32)).cuda()
+    A0 = -10.0 * torch.eye(d, device="cuda").expand(1, 1, d, d).contiguous()
+    drs.vla_scan(x, x, x, x, A0=A0)
+    torch.cuda.synchronize()
+    assert drs.poll_error() == drs.DR_ERR_NOT_SPD
+    assert drs.poll_error() == drs.DR_OK
 
 
 # --- failure path: a bounded wait that runs out latches a status, nothing hangs
