@@ -26,6 +26,8 @@ DR_OK, DR_ERR_INVALID_ARG, DR_ERR_UNSUPPORTED, DR_ERR_CUDA, DR_ERR_TIMEOUT, DR_E
     0, -1, -2, -3, -4, -5)
 DR_ERR_GATE_RANGE = -6
 DR_ERR_NOT_SPD = -7
+DR_ERR_SCRATCH_LIMIT = -8
+VLA_NOALLOC_MAX_FLOATS = 16777216
 MODES = {"linear": DR_LINEAR, "deltanet": DR_DELTANET, "gdn": DR_GDN, "kda": DR_KDA,
          "gdn2": DR_GDN2}
 
@@ -38,6 +40,7 @@ SIGNATURES = {
     "dr_decode_step_ex": ([_VP] * 10 + [_I] * 5 + [_VP], _I),
     "vla_scan_fwd": ([_VP] * 6 + [_F] + [_VP] * 3 + [_I] * 4 + [_VP], _I),
     "vla_scan_fwd_ex": ([_VP] * 7 + [_F] + [_VP] * 4 + [_I] * 5 + [_VP], _I),
+    "vla_scan_fwd_noalloc": ([_VP] * 7 + [_F] + [_VP] * 4 + [_I] * 5 + [_VP], _I),
     "loglinear_scan_fwd": ([_VP] * 5 + [_I] * 7 + [_VP], _I),
     "dr_status_string": ([_I], ctypes.c_char_p),
     "dr_poll_error": ([_VP], _I),

@@ -246,6 +246,68 @@ __global__ void timeout_probe_kernel(int spin_limit) {
     }
 }
 
+// ---- scratch of the no-allocation VLA entry point
+
+// Write directions of vla_scan_fwd_noalloc: a fixed array instead of pool memory. Every GPU
+// that loads the library holds it until the process exits. Host code only ever passes its
+// device address, looked up per device below (the array's name is a host-side stand-in).
+static __device__ __align__(256) float g_vla_noalloc_scratch[VLA_NOALLOC_MAX_FLOATS];
+
+// Device address of g_vla_noalloc_scratch on the current device, looked up once per device
+// (the first call on a device, with that device current).
+int noalloc_scratch(float** out) {
+    constexpr int kMaxDev = 64;
+    static std::mutex mu;
+    static float* addr[kMaxDev] = {};
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDev) return DR_ERR_CUDA;
+    std::lock_guard<std::mutex> lock(mu);
+    if (!addr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_vla_noalloc_scratch) != cudaSuccess || !p)
+            return DR_ERR_CUDA;
+        addr[dev] = static_cast<float*>(p);
+    }
+    *out = addr[dev];
+    return DR_OK;
+}
+
+// The chunked pair with the directions in the fixed array (nothing allocated or freed).
+template <int D, bool RATIO>
+int launch_vla_noalloc(const float* q, const float* k, const float* v, const float* u,
+                       const float* S0, const float* A0, const float* n0, float lambda0,
+                       float* out, float* S_final, float* A_final, float* n_final, long BH,
+                       int T, float* alpha, cudaStream_t stream) {
+    const int smem_a = (int)sizeof(VcASmem<D>);
+    const int smem_s = (int)sizeof(VcSSmem<D>);
+    auto ka = vla_aphase_kernel<D>;
+    auto ks = vla_sphase_kernel<D, RATIO>;
+    if (cudaFuncSetAttribute(ka, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_a) !=
+            cudaSuccess ||
+        cudaFuncSetAttribute(ks, cudaFuncAttributeMaxDynamicSharedMemorySize, smem_s) !=
+            cudaSuccess)
+        return DR_ERR_CUDA;
+    ka<<<(unsigned)BH, VC_THREADS, smem_a, stream>>>(k, u, A0, lambda0, A_final, alpha, T);
+    int rc = launch_status();
+    if (rc != DR_OK) return rc;
+    ks<<<dim3((unsigned)BH, D / VC_RS), VC_THREADS, smem_s, stream>>>(q, k, v, alpha, S0, n0, out,
+                                                                    S_final, n_final, T);
+    return launch_status();
+}
+
+template <int D>
+int launch_vla_noalloc_readout(bool ratio, const float* q, const float* k, const float* v,
+                               const float* u, const float* S0, const float* A0,
+                               const float* n0, float lambda0, float* out, float* S_final,
+                               float* A_final, float* n_final, long BH, int T, float* alpha,
+                               cudaStream_t stream) {
+    if (ratio)
+        return launch_vla_noalloc<D, true>(q, k, v, u, S0, A0, n0, lambda0, out, S_final,
+                                           A_final, n_final, BH, T, alpha, stream);
+    return launch_vla_noalloc<D, false>(q, k, v, u, S0, A0, nullptr, lambda0, out, S_final,
+                                        A_final, nullptr, BH, T, alpha, stream);
+}
+
 }  // namespace
 
 extern "C" {
@@ -272,6 +334,9 @@ const char* dr_status_string(int status) {
         case DR_ERR_NOT_SPD:
             return "device: VLA's inverse penalty A is not positive definite (a non-positive "
                    "pivot in I + U A U^T); outputs are invalid";
+        case DR_ERR_SCRATCH_LIMIT:
+            return "request too large for vla_scan_fwd_noalloc's fixed scratch array "
+                   "(B*H*T*d > VLA_NOALLOC_MAX_FLOATS); use vla_scan_fwd_ex";
     }
     return "unknown status";
 }
@@ -415,6 +480,51 @@ int vla_scan_fwd(const float* q, const float* k, const float* v, const float* u,
                  int H, int T, int d, cudaStream_t stream) {
     return vla_scan_fwd_ex(q, k, v, u, S0, A0, nullptr, lambda0, out, S_final, A_final, nullptr,
                            B, H, T, d, 0, stream);
+}
+
+int vla_scan_fwd_noalloc(const float* q, const float* k, const float* v, const float* u,
+                         const float* S0, const float* A0, const float* n0, float lambda0,
+                         float* out, float* S_final, float* A_final, float* n_final, int B,
+                         int H, int T, int d, int flags, cudaStream_t stream) {
+    if (flags & ~VLA_RATIO_READOUT) return DR_ERR_INVALID_ARG;
+    const bool ratio = (flags & VLA_RATIO_READOUT) != 0;
+    if (!ratio && (n0 || n_final)) return DR_ERR_INVALID_ARG;
+    if (!ok_opt(n0) || !ok_opt(n_final)) return DR_ERR_INVALID_ARG;
+    if (B < 0 || H < 0 || T < 0 || d <= 0) return DR_ERR_INVALID_ARG;
+    const long BH = (long)B * (long)H;
+    if (BH > INT_MAX) return DR_ERR_INVALID_ARG;
+    const bool tokens = BH > 0 && T > 0;
+    if (tokens && (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(u) || !ok_ptr(out)))
+        return DR_ERR_INVALID_ARG;
+    if (!ok_opt(q) || !ok_opt(k) || !ok_opt(v) || !ok_opt(u) || !ok_opt(out) || !ok_opt(S0) ||
+        !ok_opt(A0) || !ok_opt(S_final) || !ok_opt(A_final))
+        return DR_ERR_INVALID_ARG;
+    if (!A0 && !(lambda0 > 0.f)) return DR_ERR_INVALID_ARG;
+    if (d != 32 && d != 64 && d != 96 && d != 128) return DR_ERR_UNSUPPORTED;
+    if ((double)BH * (double)T * (double)d > (double)VLA_NOALLOC_MAX_FLOATS)
+        return DR_ERR_SCRATCH_LIMIT;
+    if (!tokens)  // no scan to run: the state copies of vla_scan_fwd_ex, which allocate nothing
+        return vla_scan_fwd_ex(q, k, v, u, S0, A0, n0, lambda0, out, S_final, A_final, n_final,
+                               B, H, T, d, flags, stream);
+    float* alpha = nullptr;
+    const int rc = noalloc_scratch(&alpha);
+    if (rc != DR_OK) return rc;
+    switch (d) {
+        case 32:
+            return launch_vla_noalloc_readout<32>(ratio, q, k, v, u, S0, A0, n0, lambda0, out,
+                                                  S_final, A_final, n_final, BH, T, alpha, stream);
+        case 64:
+            return launch_vla_noalloc_readout<64>(ratio, q, k, v, u, S0, A0, n0, lambda0, out,
+                                                  S_final, A_final, n_final, BH, T, alpha, stream);
+        case 96:
+            return launch_vla_noalloc_readout<96>(ratio, q, k, v, u, S0, A0, n0, lambda0, out,
+                                                  S_final, A_final, n_final, BH, T, alpha, stream);
+        case 128:
+            return launch_vla_noalloc_readout<128>(ratio, q, k, v, u, S0, A0, n0, lambda0, out,
+                                                   S_final, A_final, n_final, BH, T, alpha,
+                                                   stream);
+    }
+    return DR_ERR_UNSUPPORTED;
 }
 
 int loglinear_scan_fwd(const void* q, const void* k, const void* v, const float* lambda,

@@ -69,9 +69,11 @@ enum {
     DR_ERR_DEVICE_BOUNDS = -5, /* device: an index check failed; outputs invalid */
     DR_ERR_GATE_RANGE = -6,  /* device: a KDA gate decayed past the chunked kernel's range
                                 (see dr_scan_fwd); outputs invalid */
-    DR_ERR_NOT_SPD = -7      /* device: the chunked VLA scan met a non-positive pivot in
+    DR_ERR_NOT_SPD = -7,     /* device: the chunked VLA scan met a non-positive pivot in
                                 I + U A U^T, i.e. A was not positive definite (an A0 that is
                                 not an inverse penalty); outputs invalid */
+    DR_ERR_SCRATCH_LIMIT = -8 /* vla_scan_fwd_noalloc: B*H*T*d is above
+                                 VLA_NOALLOC_MAX_FLOATS, the size of its fixed scratch array */
 };
 
 /*
@@ -227,6 +229,38 @@ int vla_scan_fwd_ex(const float* q, const float* k, const float* v, const float*
                     const float* S0, const float* A0, const float* n0, float lambda0,
                     float* out, float* S_final, float* A_final, float* n_final,
                     int B, int H, int T, int d, int flags, cudaStream_t stream);
+
+/* Largest B*H*T*d that vla_scan_fwd_noalloc accepts: its scratch array holds this many
+ * floats (64 MiB). */
+#define VLA_NOALLOC_MAX_FLOATS 16777216
+
+/*
+ * vla_scan_fwd_noalloc -- vla_scan_fwd_ex (chunked pair only) without any memory allocation.
+ * The pages have no counterpart: this entry point exists for callers that must not allocate
+ * device memory, such as a serving engine that reserves all device memory up front for its
+ * own allocator and forbids later allocations, or code that runs where a driver allocation
+ * may block or synchronise (a latency-bound step, an allocator's own callback). The chunked
+ * VLA scan needs B*H*T*d floats of scratch for the write directions between its two
+ * kernels; vla_scan_fwd_ex takes them from a memory pool, this entry point from a fixed
+ * array compiled into the library, which every GPU that loads the library holds
+ * (VLA_NOALLOC_MAX_FLOATS floats, 64 MiB) until the process exits.
+ *
+ * Arguments, layout and results are those of vla_scan_fwd_ex; flags is 0 or
+ * VLA_RATIO_READOUT (VLA_SEQUENTIAL returns DR_ERR_INVALID_ARG: the per-token kernel needs no
+ * scratch). B*H*T*d above VLA_NOALLOC_MAX_FLOATS returns DR_ERR_SCRATCH_LIMIT before
+ * anything is launched. The call makes no cudaMalloc, cudaFree or pool allocation.
+ *
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress,
+ * once per device, with that device current); make that first call before any stream
+ * capture. Every call on a device shares the one array, and the array keeps the last call's
+ * contents (every element a call reads is written by that call first). Calls that overlap on
+ * the GPU (different streams, or different host threads) race on the array: serialise them.
+ * Returns DR_OK or a negative status; on error nothing is launched.
+ */
+int vla_scan_fwd_noalloc(const float* q, const float* k, const float* v, const float* u,
+                         const float* S0, const float* A0, const float* n0, float lambda0,
+                         float* out, float* S_final, float* A_final, float* n_final,
+                         int B, int H, int T, int d, int flags, cudaStream_t stream);
 
 /*
  * loglinear_scan_fwd -- log-linear attention over a Fenwick hierarchy of linear-attention
