@@ -1077,6 +1077,17 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
         // Gated DeltaNet-2 prefetches its erase gate b the same way and scales K by it.
         const int kc = 2 * (u & 63), kq4 = u >> 6;
         constexpr bool kChan = kKda || kGdn2;  // per-key-channel values prefetched per chunk
+        // Byte offsets of (row 16*kq4 + i, channels kc, kc+1) in the 128-byte-swizzled K/Q
+        // stage (128 rows per panel) and K/gamma tile (64 rows per panel): the swizzle of row
+        // i depends on i & 7 only, so row i's offset is a per-thread base plus the 16-byte
+        // chunk position xsw(i & 7) plus a constant, and no swizzle arithmetic is left per
+        // access in the loops below.
+        const uint32_t kq_row0 = (uint32_t)(kc >> 6) * 128u * 128u + (uint32_t)(16 * kq4) * 128u +
+                                 (uint32_t)(kc & 7) * 2u;
+        const uint32_t kn_row0 = (uint32_t)(kc >> 6) * 64u * 128u + (uint32_t)(16 * kq4) * 128u +
+                                 (uint32_t)(kc & 7) * 2u;
+        const uint32_t kc_chunk = (uint32_t)((kc & 63) >> 3);
+        auto xsw = [&](int i) -> uint32_t { return ((kc_chunk ^ (uint32_t)(i & 7)) << 4); };
         const float* chan = kKda ? gate : erase;
         float2 gpf[kChan ? 16 : 1];
         if constexpr (kChan) {
@@ -1107,16 +1118,17 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 fact = bg[64 + 63] > -80.f;
                 if constexpr (kGdn2) {
                     // erase directions e = b (.) k, in place in the stage's K rows
+                    uint8_t* kr = kq + kq_row0;
 #pragma unroll
                     for (int i0 = 0; i0 < 16; i0 += 8) {
                         uint32_t kw[8];
 #pragma unroll
                         for (int i = 0; i < 8; ++i)
-                            kw[i] = *reinterpret_cast<const uint32_t*>(kq + sw128_offset(16 * kq4 + i0 + i, kc, 128));
+                            kw[i] = *reinterpret_cast<const uint32_t*>(kr + xsw(i) + (i0 + i) * 128);
 #pragma unroll
                         for (int i = 0; i < 8; ++i) {
                             const float2 k2 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&kw[i]));
-                            *reinterpret_cast<uint32_t*>(kq + sw128_offset(16 * kq4 + i0 + i, kc, 128)) =
+                            *reinterpret_cast<uint32_t*>(kr + xsw(i) + (i0 + i) * 128) =
                                 pack_bf16(k2.x * gpf[i0 + i].x, k2.y * gpf[i0 + i].y);
                         }
                     }
@@ -1133,22 +1145,25 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 uint8_t* kn = sm + L::KN;
                 // summed log alpha of this thread's 16 rows: the log of their product, or,
                 // where that product would underflow, the sum of the rows' logs
+                // rows past the end of a ragged chunk count as alpha = 1 (so that every loop
+                // below runs without a per-row test)
+                if (nvalid < CK) {
+#pragma unroll
+                    for (int i = 0; i < 16; ++i)
+                        if (16 * kq4 + i >= nvalid) gpf[i] = make_float2(1.f, 1.f);
+                }
                 float2 part = make_float2(1.f, 1.f);
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
-                    if (16 * kq4 + i < nvalid) {
-                        part.x *= gpf[i].x;
-                        part.y *= gpf[i].y;
-                    }
+                    part.x *= gpf[i].x;
+                    part.y *= gpf[i].y;
                 }
                 float2 lp = make_float2(__logf(part.x), __logf(part.y));
                 if (part.x < 1e-30f || part.y < 1e-30f) {
                     lp = make_float2(0.f, 0.f);
                     for (int i = 0; i < 16; ++i) {
-                        if (16 * kq4 + i < nvalid) {
-                            lp.x += __logf(gpf[i].x);
-                            lp.y += __logf(gpf[i].y);
-                        }
+                        lp.x += __logf(gpf[i].x);
+                        lp.y += __logf(gpf[i].y);
                     }
                 }
                 *reinterpret_cast<float2*>(pg + 128 * kq4 + kc) = lp;
@@ -1173,30 +1188,28 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     *reinterpret_cast<float2*>(bgw + 128 + kc) = make_float2(__expf(m.x), __expf(m.y));
                 }
                 float2 run = make_float2(__expf(Lb.x - m.x), __expf(Lb.y - m.y));
+                uint8_t* kr = kq + kq_row0;  // K row 16*kq4 (Q rows sit 64 rows further on)
+                uint8_t* nr = kn + kn_row0;
 #pragma unroll
                 for (int i0 = 0; i0 < 16; i0 += 8) {
                     uint32_t kw[8], qw[8];
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        const int t = 16 * kq4 + i0 + i;
-                        kw[i] = *reinterpret_cast<const uint32_t*>(kq + sw128_offset(t, kc, 128));
-                        qw[i] = *reinterpret_cast<const uint32_t*>(kq + sw128_offset(64 + t, kc, 128));
+                        kw[i] = *reinterpret_cast<const uint32_t*>(kr + xsw(i) + (i0 + i) * 128);
+                        qw[i] = *reinterpret_cast<const uint32_t*>(kr + xsw(i) + (64 + i0 + i) * 128);
                     }
 #pragma unroll
                     for (int i = 0; i < 8; ++i) {
-                        const int t = 16 * kq4 + i0 + i;
-                        if (t < nvalid) {
-                            run.x *= gpf[i0 + i].x;
-                            run.y *= gpf[i0 + i].y;
-                        }
+                        run.x *= gpf[i0 + i].x;
+                        run.y *= gpf[i0 + i].y;
                         const float2 k2 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&kw[i]));
                         const float2 q2 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&qw[i]));
                         const float ix = __fdividef(1.f, run.x), iy = __fdividef(1.f, run.y);
-                        *reinterpret_cast<uint32_t*>(kq + sw128_offset(t, kc, 128)) =
+                        *reinterpret_cast<uint32_t*>(kr + xsw(i) + (i0 + i) * 128) =
                             pack_bf16(k2.x * run.x, k2.y * run.y);
-                        *reinterpret_cast<uint32_t*>(kq + sw128_offset(64 + t, kc, 128)) =
+                        *reinterpret_cast<uint32_t*>(kr + xsw(i) + (64 + i0 + i) * 128) =
                             pack_bf16(q2.x * run.x, q2.y * run.y);
-                        *reinterpret_cast<uint32_t*>(kn + sw128_offset(t, kc, 64)) =
+                        *reinterpret_cast<uint32_t*>(nr + xsw(i) + (i0 + i) * 128) =
                             pack_bf16(k2.x * ix, k2.y * iy);
                     }
                 }
