@@ -139,13 +139,15 @@ def aggregate_value(world: int, head_tokens: int, steps: int, total_ms_max: floa
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch from one ncu capture,
-# keyed by workload and the sha256 prefix of the timed kernel's source (dr_chunked.cuh, or
-# dr_decode.cuh for the decode workload) at capture time; a changed source reports null.
-# Summaries with the commands are under profiles/.
+# keyed by workload and the sha256 prefix of the timed kernel's source (dr_chunked.cuh,
+# dr_decode.cuh for the decode workload, loglinear.cuh for log-linear attention) at capture
+# time; a changed source reports null. Summaries with the commands are under profiles/.
 NCU_TRAFFIC = {
-    ("gdn_bf16", "ccf466c9562f095c"): 101832448 + 13261312,
-    ("kda_bf16", "ccf466c9562f095c"): 673327104 + 120072704,
-    ("gdn_decode_bf16", "350334b801e0108e"): 271628544 + 210415360,
+    ("kda_bf16", "c20c5b6c976514f5"): 673301760 + 121483008,
+    ("gdn_bf16", "c20c5b6c976514f5"): 101820160 + 13235712,
+    ("gdn_long_t32768", "c20c5b6c976514f5"): 408017408 + 113290240,
+    ("gdn_decode_bf16", "6c9773f81f64a408"): 271627008 + 211260672,
+    ("loglinear_bf16", "9a05bbf81176e812"): 107536384 + 19725312,
 }
 
 
@@ -701,7 +703,8 @@ def measure_loglinear(args, w, world, rank, local, device, K, cpu_target):
                      "bf16", t_wall)
     line["roofline"] = {
         "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-        "frac": achieved / peaks["hbm_gbs"], "traffic": None,
+        "frac": achieved / peaks["hbm_gbs"],
+        "traffic": NCU_TRAFFIC.get((w.name, kernel_source_sha("loglinear.cuh"))),
         "peak_source": f"{peak_src} hbm_gbs", "bytes_per_launch": nbytes,
         "launch_ms": launch_ms, "tensor_tflops": tflops,
         "tensor_frac": tflops / peaks["bf16_tflops"]}
