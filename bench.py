@@ -491,9 +491,9 @@ def measure_dr(args, w, world, rank, local, device, K, cpu_target):
 
 
 def measure_vla(args, w, world, rank, local, device, K, cpu_target):
-    """The VLA Sherman-Morrison scan (fp32) through vla_scan_fwd_ex: the chunked pair (the
-    Woodbury A-phase, then the WY S-phase), two launches per step on CUDA cores, reported
-    against the FP32 ALU peak over the whole step."""
+    """The VLA Sherman-Morrison scan (fp32) through vla_scan_fwd_ex: the chunked scan as one
+    fused cluster kernel per step (the Woodbury A-phase and the WY S-phase at once, on CUDA
+    cores), reported against the FP32 ALU peak over the whole step."""
     import torch
 
     import delta_rule_recurrent_chunked_b200 as drs
@@ -555,10 +555,9 @@ def measure_vla(args, w, world, rank, local, device, K, cpu_target):
     peak = fp32_alu_peak_tflops(device)
     achieved = flops / (launch_ms / 1e3) / 1e12
     config = dict(workload_config(w, world), l2=l2_note(nsets, nbytes, needs_flush),
-                  kernel="vla_aphase + vla_sphase")
+                  kernel="vla_fused")
     line = base_line(args, w, world, K, total_ms_max, clk, e2e_ms, pipe.h2d, pipe.d2h, config,
                      "f32", t_wall)
-    line["gpu_launches"] = 2 * K
     line["roofline"] = {
         "bound": "alu", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
         "frac": achieved / peak, "traffic": None,

@@ -292,10 +292,11 @@ def decode_step(q, k, v, beta=None, gate=None, S=None, mode="gdn", out=None):
 
 
 def vla_scan(q, k, v, u, S0=None, A0=None, lambda0=1.0, want_state=True, out=None,
-             sequential=False):
+             sequential=False, two_kernel=False):
     """VLA Sherman-Morrison scan on the GPU (fp32). q, k, v, u: [B,H,T,d];
-    S0, A0: [B,H,d,d] or None. Returns (out, S_final, A_final). The chunked pair of
-    kernels runs by default; sequential=True selects the per-token kernel."""
+    S0, A0: [B,H,d,d] or None. Returns (out, S_final, A_final). The chunked scan runs as one
+    fused cluster kernel by default; two_kernel=True runs its two phases as separate kernels
+    (with pool scratch), sequential=True the per-token kernel."""
     import torch
 
     B, H, T, d = q.shape
@@ -310,7 +311,7 @@ def vla_scan(q, k, v, u, S0=None, A0=None, lambda0=1.0, want_state=True, out=Non
     _check(out, "out", (B, H, T, d), torch.float32, dev)
     Sf = torch.empty((B, H, d, d), dtype=torch.float32, device=dev) if want_state else None
     Af = torch.empty((B, H, d, d), dtype=torch.float32, device=dev) if want_state else None
-    flags = VLA_SEQUENTIAL if sequential else 0
+    flags = _vla_path_flags(sequential, two_kernel)
     rc = lib().vla_scan_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(S0), _ptr(A0), None,
                                float(lambda0), _ptr(out), _ptr(Sf), _ptr(Af), None, B, H, T,
                                d, flags, _stream_handle(dev))
@@ -321,14 +322,19 @@ def vla_scan(q, k, v, u, S0=None, A0=None, lambda0=1.0, want_state=True, out=Non
 
 VLA_RATIO_READOUT = 0x1
 VLA_SEQUENTIAL = 0x2
+VLA_TWO_KERNEL = 0x4
+
+
+def _vla_path_flags(sequential: bool, two_kernel: bool) -> int:
+    return (VLA_SEQUENTIAL if sequential else 0) | (VLA_TWO_KERNEL if two_kernel else 0)
 
 
 def vla_scan_ratio(q, k, v, u, S0=None, A0=None, n0=None, lambda0=1.0, want_state=True,
-                   out=None, sequential=False):
+                   out=None, sequential=False, two_kernel=False):
     """VLA scan with the ratio readout o_t = S_t q_t / (n_t q_t) (fp32), through
     vla_scan_fwd_ex. q: [B,H,T,d] feature-mapped queries (phi(q)); k: unit-norm
     feature-mapped keys; n0: [B,H,d] or None. Returns (out, S_final, A_final, n_final).
-    sequential=True selects the per-token kernel instead of the chunked pair."""
+    two_kernel / sequential select the other paths, as in vla_scan."""
     import torch
 
     B, H, T, d = q.shape
@@ -348,7 +354,7 @@ def vla_scan_ratio(q, k, v, u, S0=None, A0=None, n0=None, lambda0=1.0, want_stat
     nf = torch.empty((B, H, d), dtype=torch.float32, device=dev) if want_state else None
     rc = lib().vla_scan_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(u), _ptr(S0), _ptr(A0), _ptr(n0),
                                float(lambda0), _ptr(out), _ptr(Sf), _ptr(Af), _ptr(nf), B, H, T,
-                               d, VLA_RATIO_READOUT | (VLA_SEQUENTIAL if sequential else 0),
+                               d, VLA_RATIO_READOUT | _vla_path_flags(sequential, two_kernel),
                                _stream_handle(dev))
     if rc != DR_OK:
         raise DrScanError(rc, "vla_scan_fwd_ex")

@@ -212,11 +212,55 @@ int launch_vla_chunked(const float* q, const float* k, const float* v, const flo
     return rc;
 }
 
+// The fused kernel: one cluster of 1 + D/32 CTAs per head, both phases at once, no scratch.
+// Returns DR_ERR_UNSUPPORTED (nothing launched) when no such cluster fits on the device.
+template <int D, bool RATIO>
+int launch_vla_fused(const float* q, const float* k, const float* v, const float* u,
+                     const float* S0, const float* A0, const float* n0, float lambda0,
+                     float* out, float* S_final, float* A_final, float* n_final, long BH, int T,
+                     cudaStream_t stream) {
+    constexpr int CS = 1 + D / VC_RS;
+    const int smem = vc_fused_smem_bytes<D>();
+    auto kern = vla_fused_kernel<D, RATIO>;
+    if (BH * CS > INT_MAX) return DR_ERR_UNSUPPORTED;
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+        cudaSuccess)
+        return DR_ERR_CUDA;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(BH * CS));
+    cfg.blockDim = dim3(VC_THREADS);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = CS;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    int clusters = 0;
+    if (cudaOccupancyMaxActiveClusters(&clusters, kern, &cfg) != cudaSuccess) return DR_ERR_CUDA;
+    if (clusters < 1) return DR_ERR_UNSUPPORTED;
+    if (cudaLaunchKernelEx(&cfg, kern, q, k, v, u, S0, A0, n0, lambda0, out, S_final, A_final,
+                           n_final, T) != cudaSuccess)
+        return DR_ERR_CUDA;
+    return launch_status();
+}
+
 template <int D>
-int launch_vla_readout(bool ratio, bool sequential, const float* q, const float* k,
-                       const float* v, const float* u, const float* S0, const float* A0,
-                       const float* n0, float lambda0, float* out, float* S_final,
-                       float* A_final, float* n_final, long BH, int T, cudaStream_t stream) {
+int launch_vla_readout(bool ratio, bool sequential, bool two_kernel, const float* q,
+                       const float* k, const float* v, const float* u, const float* S0,
+                       const float* A0, const float* n0, float lambda0, float* out,
+                       float* S_final, float* A_final, float* n_final, long BH, int T,
+                       cudaStream_t stream) {
+    if (!sequential && !two_kernel) {
+        const int rc = ratio ? launch_vla_fused<D, true>(q, k, v, u, S0, A0, n0, lambda0, out,
+                                                         S_final, A_final, n_final, BH, T, stream)
+                             : launch_vla_fused<D, false>(q, k, v, u, S0, A0, nullptr, lambda0,
+                                                          out, S_final, A_final, nullptr, BH, T,
+                                                          stream);
+        if (rc != DR_ERR_UNSUPPORTED) return rc;  // else: the two-kernel pair below
+    }
     if (sequential) {
         if (ratio)
             return launch_vla<D, true>(q, k, v, u, S0, A0, n0, lambda0, out, S_final, A_final,
@@ -431,9 +475,11 @@ int vla_scan_fwd_ex(const float* q, const float* k, const float* v, const float*
                     const float* S0, const float* A0, const float* n0, float lambda0, float* out,
                     float* S_final, float* A_final, float* n_final, int B, int H, int T, int d,
                     int flags, cudaStream_t stream) {
-    if (flags & ~(VLA_RATIO_READOUT | VLA_SEQUENTIAL)) return DR_ERR_INVALID_ARG;
+    if (flags & ~(VLA_RATIO_READOUT | VLA_SEQUENTIAL | VLA_TWO_KERNEL)) return DR_ERR_INVALID_ARG;
     const bool ratio = (flags & VLA_RATIO_READOUT) != 0;
     const bool sequential = (flags & VLA_SEQUENTIAL) != 0;
+    const bool two_kernel = (flags & VLA_TWO_KERNEL) != 0;
+    if (sequential && two_kernel) return DR_ERR_INVALID_ARG;
     if (!ratio && (n0 || n_final)) return DR_ERR_INVALID_ARG;
     if (!ok_opt(n0) || !ok_opt(n_final)) return DR_ERR_INVALID_ARG;
     if (B < 0 || H < 0 || T < 0 || d <= 0) return DR_ERR_INVALID_ARG;
@@ -460,17 +506,17 @@ int vla_scan_fwd_ex(const float* q, const float* k, const float* v, const float*
     }
     switch (d) {
         case 32:
-            return launch_vla_readout<32>(ratio, sequential, q, k, v, u, S0, A0, n0, lambda0,
-                                          out, S_final, A_final, n_final, BH, T, stream);
+            return launch_vla_readout<32>(ratio, sequential, two_kernel, q, k, v, u, S0, A0, n0,
+                                          lambda0, out, S_final, A_final, n_final, BH, T, stream);
         case 64:
-            return launch_vla_readout<64>(ratio, sequential, q, k, v, u, S0, A0, n0, lambda0,
-                                          out, S_final, A_final, n_final, BH, T, stream);
+            return launch_vla_readout<64>(ratio, sequential, two_kernel, q, k, v, u, S0, A0, n0,
+                                          lambda0, out, S_final, A_final, n_final, BH, T, stream);
         case 96:
-            return launch_vla_readout<96>(ratio, sequential, q, k, v, u, S0, A0, n0, lambda0,
-                                          out, S_final, A_final, n_final, BH, T, stream);
+            return launch_vla_readout<96>(ratio, sequential, two_kernel, q, k, v, u, S0, A0, n0,
+                                          lambda0, out, S_final, A_final, n_final, BH, T, stream);
         case 128:
-            return launch_vla_readout<128>(ratio, sequential, q, k, v, u, S0, A0, n0, lambda0,
-                                           out, S_final, A_final, n_final, BH, T, stream);
+            return launch_vla_readout<128>(ratio, sequential, two_kernel, q, k, v, u, S0, A0, n0,
+                                           lambda0, out, S_final, A_final, n_final, BH, T, stream);
     }
     return DR_ERR_UNSUPPORTED;
 }

@@ -101,6 +101,58 @@ __device__ __forceinline__ float vc_comp(const float4& f, int q) {
     return q == 0 ? f.x : (q == 1 ? f.y : (q == 2 ? f.z : f.w));
 }
 
+// ---- cluster hand-off of the write directions (fused kernel)
+// The A-phase CTA (cluster rank 0) writes a chunk's alpha_hat rows into its own K A_c tile
+// (dead by then) and one thread copies the tile into the ring slot of every S-phase CTA
+// (ranks 1 ..) with a bulk copy that completes its bytes on that CTA's `full` barrier of the
+// slot. An S-phase CTA arms that barrier (expected bytes) before it hands the slot back by
+// arriving on the A-phase CTA's `empty` barrier. Every wait is bounded (mbar-style, with the
+// CTA's abort flag); after a timeout a CTA stops sending and receiving and runs its loops to
+// the end, so every thread reaches the cluster barrier that ends the kernel.
+struct VcLink {
+    uint32_t al_base;    // shared::cta address of the S-phase layout's al[0][0][0]
+    uint32_t full_bar;   // shared::cta address of full[0] (full[1] at +8)
+    uint32_t empty_bar;  // shared::cta address of empty[0] (empty[1] at +8)
+    int nranks;          // S-phase CTAs of the cluster
+    volatile int* abort;
+};
+
+__device__ __forceinline__ uint32_t vc_cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+
+// Bytes of one chunk's alpha_hat tile (64 rows of D floats, padded rows of D + 4).
+template <int D>
+constexpr uint32_t vc_tile_bytes() {
+    return (uint32_t)(VC_C * (D + 4) * 4);
+}
+
+// Phase wait with cluster-scope acquire (the data behind the barrier was written by another
+// CTA of the cluster), bounded like mbar_wait.
+__device__ __forceinline__ bool vc_wait_cluster(uint32_t bar, uint32_t parity,
+                                                volatile int* abort) {
+    const uint64_t t0 = global_timer_ns();
+    for (uint32_t it = 0;; ++it) {
+        uint32_t ok;
+        asm volatile(
+            "{\n\t.reg .pred p;\n\t"
+            "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t"
+            "selp.u32 %0, 1, 0, p;\n\t}"
+            : "=r"(ok)
+            : "r"(bar), "r"(parity)
+            : "memory");
+        if (ok) return true;
+        if (*abort) return false;
+        if ((it & 31u) == 31u && global_timer_ns() - t0 > DRSCAN_WAIT_LIMIT_NS) {
+            raise_status(DR_ERR_TIMEOUT);
+            *abort = 1;
+            return false;
+        }
+    }
+}
+
 // ---------------------------------------------------------------------------------------
 // A-phase
 // ---------------------------------------------------------------------------------------
@@ -116,21 +168,22 @@ struct VcASmem {
     float dinv[VC_C];                // 1 / L_tt
 };
 
-// grid: B*H; block: VC_THREADS; dynamic shared memory: sizeof(VcASmem<D>).
-template <int D>
-__global__ void __launch_bounds__(VC_THREADS, 1)
-    vla_aphase_kernel(const float* __restrict__ k, const float* __restrict__ u,
-                      const float* __restrict__ A0, float lambda0, float* __restrict__ A_final,
-                      float* __restrict__ alpha, int T) {
-    extern __shared__ __align__(16) unsigned char vc_smem_raw[];
-    VcASmem<D>& sm = *reinterpret_cast<VcASmem<D>*>(vc_smem_raw);
+// One head's A-phase. PUSH = false: alpha_hat to global memory (row per token); PUSH = true:
+// into the S-phase CTAs of the cluster through `link`.
+template <int D, bool PUSH>
+__device__ __forceinline__ void vc_aphase(unsigned char* smem_raw, long bh,
+                                          const float* __restrict__ k,
+                                          const float* __restrict__ u,
+                                          const float* __restrict__ A0, float lambda0,
+                                          float* __restrict__ A_final, float* __restrict__ alpha,
+                                          int T, const VcLink& link) {
+    VcASmem<D>& sm = *reinterpret_cast<VcASmem<D>*>(smem_raw);
     constexpr int CT = D / 16;  // columns per thread in the 16-column-group tilings
     const int tid = threadIdx.x;
     const int rg = tid >> 4, cg = tid & 15;
-    const long bh = blockIdx.x;
     const float* kh = k + bh * (long)T * D;
     const float* uh = u + bh * (long)T * D;
-    float* ah = alpha + bh * (long)T * D;
+    float* ah = PUSH ? nullptr : alpha + bh * (long)T * D;
     const int nchunks = (T + VC_C - 1) / VC_C;
 
     for (int e = tid; e < D * D; e += VC_THREADS) {
@@ -420,11 +473,40 @@ __global__ void __launch_bounds__(VC_THREADS, 1)
 #pragma unroll
                 for (int off = 8; off > 0; off >>= 1) n2 += __shfl_xor_sync(0xffffffffu, n2, off);
                 const int r = rg + 16 * i;
-                if (r < nv) {
-                    const float inv = rsqrtf(n2);
-                    float* dst = ah + (long)(t0 + r) * D + cg * CT;
+                if constexpr (PUSH) {
+                    // into this thread's own K A_c entries; rows past the end of the sequence
+                    // go out as zeros
+                    const float inv = r < nv ? rsqrtf(n2) : 0.f;
+                    float* dst = &sm.ka[r][cg * CT];
 #pragma unroll
                     for (int j = 0; j < CT; ++j) dst[j] = acc[i][j] * inv;
+                } else {
+                    if (r < nv) {
+                        const float inv = rsqrtf(n2);
+                        float* dst = ah + (long)(t0 + r) * D + cg * CT;
+#pragma unroll
+                        for (int j = 0; j < CT; ++j) dst[j] = acc[i][j] * inv;
+                    }
+                }
+            }
+        }
+        if constexpr (PUSH) {
+            // the tile is complete: copy it to every S-phase CTA once ring slot c % 2 (last
+            // filled for chunk c - 2) has been read by all of them
+            fence_async_smem();
+            __syncthreads();
+            if (tid == 0) {
+                const uint32_t slot = (uint32_t)(c & 1);
+                if (c >= 2)
+                    vc_wait_cluster(link.empty_bar + 8u * slot, (uint32_t)(((c >> 1) + 1) & 1),
+                                    link.abort);
+                if (!*link.abort) {
+                    for (int qr = 1; qr <= link.nranks; ++qr)
+                        bulk_copy_to_peer(
+                            cluster_map(link.al_base + slot * vc_tile_bytes<D>(), (uint32_t)qr),
+                            smem_u32(&sm.ka[0][0]), vc_tile_bytes<D>(),
+                            cluster_map(link.full_bar + 8u * slot, (uint32_t)qr));
+                    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
                 }
             }
         }
@@ -453,8 +535,15 @@ __global__ void __launch_bounds__(VC_THREADS, 1)
                 for (int j = 0; j < CT; ++j) dst[j] -= acc[i][j];
             }
         }
+        if constexpr (PUSH) {
+            // the next chunk's first step rewrites the tile: its copies must have read it
+            if (tid == 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+        }
         vc_wait_copies();
         __syncthreads();
+    }
+    if constexpr (PUSH) {
+        if (tid == 0) bulk_wait_all();  // every copy has landed before the kernel can end
     }
 
     if (A_final) {
@@ -463,6 +552,16 @@ __global__ void __launch_bounds__(VC_THREADS, 1)
             A_final[bh * D * D + e] = sm.A[r][c];
         }
     }
+}
+
+// grid: B*H; block: VC_THREADS; dynamic shared memory: sizeof(VcASmem<D>).
+template <int D>
+__global__ void __launch_bounds__(VC_THREADS, 1)
+    vla_aphase_kernel(const float* __restrict__ k, const float* __restrict__ u,
+                      const float* __restrict__ A0, float lambda0, float* __restrict__ A_final,
+                      float* __restrict__ alpha, int T) {
+    extern __shared__ __align__(16) unsigned char vc_smem_raw[];
+    vc_aphase<D, false>(vc_smem_raw, blockIdx.x, k, u, A0, lambda0, A_final, alpha, T, VcLink{});
 }
 
 // ---------------------------------------------------------------------------------------
@@ -484,22 +583,24 @@ struct VcSSmem {
     float on[VC_C];              // ratio readout: q_t . n_c
 };
 
-// grid: (B*H, D / VC_RS); block: VC_THREADS; dynamic shared memory: sizeof(VcSSmem<D>).
-template <int D, bool RATIO>
-__global__ void __launch_bounds__(VC_THREADS, 1)
-    vla_sphase_kernel(const float* __restrict__ q, const float* __restrict__ k,
-                      const float* __restrict__ v, const float* __restrict__ alpha,
-                      const float* __restrict__ S0, const float* __restrict__ n0,
-                      float* __restrict__ out, float* __restrict__ S_final,
-                      float* __restrict__ n_final, int T) {
-    extern __shared__ __align__(16) unsigned char vc_smem_raw[];
-    VcSSmem<D>& sm = *reinterpret_cast<VcSSmem<D>*>(vc_smem_raw);
+// One head's S-phase for rows row0 .. row0 + 31 of S. PULL = false: alpha_hat from global
+// memory; PULL = true: from this CTA's ring, filled by the cluster's A-phase CTA (`link`).
+template <int D, bool RATIO, bool PULL>
+__device__ __forceinline__ void vc_sphase(unsigned char* smem_raw, long bh, int row0,
+                                          const float* __restrict__ q,
+                                          const float* __restrict__ k,
+                                          const float* __restrict__ v,
+                                          const float* __restrict__ alpha,
+                                          const float* __restrict__ S0,
+                                          const float* __restrict__ n0, float* __restrict__ out,
+                                          float* __restrict__ S_final,
+                                          float* __restrict__ n_final, int T,
+                                          const VcLink& link) {
+    VcSSmem<D>& sm = *reinterpret_cast<VcSSmem<D>*>(smem_raw);
     constexpr int CT = D / 16;
     constexpr int NRC = VC_RS + (RATIO ? 1 : 0);  // columns of R (value rows + n)
     const int tid = threadIdx.x;
     const int rg = tid >> 4, cg = tid & 15;
-    const long bh = blockIdx.x;
-    const int row0 = blockIdx.y * VC_RS;  // first row of S in this CTA
     const long seq = bh * (long)T * D;
     const int nchunks = (T + VC_C - 1) / VC_C;
 
@@ -514,7 +615,7 @@ __global__ void __launch_bounds__(VC_THREADS, 1)
         const int nv = min(VC_C, T);
         vc_load_rows<D>(sm.k, k + seq, nv, tid);
         vc_load_rows<D>(sm.q, q + seq, nv, tid);
-        vc_load_rows<D>(sm.al[0], alpha + seq, nv, tid);
+        if constexpr (!PULL) vc_load_rows<D>(sm.al[0], alpha + seq, nv, tid);
         vc_load_cols<D, VC_RS>(sm.v, v + seq, row0, nv, tid);
     }
     vc_wait_copies();
@@ -525,8 +626,13 @@ __global__ void __launch_bounds__(VC_THREADS, 1)
         const int nv = min(VC_C, T - t0);
         const int nv_next = min(VC_C, T - t0 - VC_C);
         const int b = c & 1;
-        if (nv_next > 0)
-            vc_load_rows<D>(sm.al[b ^ 1], alpha + seq + (long)(t0 + VC_C) * D, nv_next, tid);
+        if constexpr (PULL) {
+            // this chunk's directions: the k-th fill of slot b completes its phase k
+            vc_wait_cluster(link.full_bar + 8u * b, (uint32_t)((c >> 1) & 1), link.abort);
+        } else {
+            if (nv_next > 0)
+                vc_load_rows<D>(sm.al[b ^ 1], alpha + seq + (long)(t0 + VC_C) * D, nv_next, tid);
+        }
 
         // 1. [G; P] = [K; Q] Alpha^T: rows rg + 16 i (i < 4 from K, i >= 4 from Q),
         //    columns cg + 16 j
@@ -753,6 +859,14 @@ __global__ void __launch_bounds__(VC_THREADS, 1)
         }
         vc_wait_copies();
         __syncthreads();
+        if constexpr (PULL) {
+            // slot b is read (steps 1 and 5): arm it for chunk c + 2, then hand it back to the
+            // A-phase CTA
+            if (tid == 0 && !*link.abort) {
+                if (c + 2 < nchunks) mbar_arrive_expect_tx(link.full_bar + 8u * b, vc_tile_bytes<D>());
+                mbar_arrive_remote(cluster_map(link.empty_bar + 8u * b, 0));
+            }
+        }
     }
 
     if (S_final) {
@@ -762,9 +876,88 @@ __global__ void __launch_bounds__(VC_THREADS, 1)
         }
     }
     if constexpr (RATIO) {
-        if (n_final && blockIdx.y == 0)
+        if (n_final && row0 == 0)
             for (int c = tid; c < D; c += VC_THREADS) n_final[bh * D + c] = sm.S[VC_RS][c];
     }
+}
+
+// grid: (B*H, D / VC_RS); block: VC_THREADS; dynamic shared memory: sizeof(VcSSmem<D>).
+template <int D, bool RATIO>
+__global__ void __launch_bounds__(VC_THREADS, 1)
+    vla_sphase_kernel(const float* __restrict__ q, const float* __restrict__ k,
+                      const float* __restrict__ v, const float* __restrict__ alpha,
+                      const float* __restrict__ S0, const float* __restrict__ n0,
+                      float* __restrict__ out, float* __restrict__ S_final,
+                      float* __restrict__ n_final, int T) {
+    extern __shared__ __align__(16) unsigned char vc_smem_raw[];
+    vc_sphase<D, RATIO, false>(vc_smem_raw, blockIdx.x, (int)blockIdx.y * VC_RS, q, k, v, alpha,
+                               S0, n0, out, S_final, n_final, T, VcLink{});
+}
+
+// ---------------------------------------------------------------------------------------
+// Fused: both phases in one cluster per head
+// ---------------------------------------------------------------------------------------
+// Cluster of 1 + D/32 CTAs per (b,h): rank 0 runs the A-phase and hands every chunk's
+// alpha_hat rows to ranks 1 .. D/32 (the S-phase for 32 rows of S each) through their
+// shared-memory rings, so that both phases run at once on different SMs and no scratch
+// memory is needed.
+template <int D>
+constexpr int vc_fused_bar_offset() {
+    constexpr int a = (int)sizeof(VcASmem<D>), b = (int)sizeof(VcSSmem<D>);
+    return ((a > b ? a : b) + 15) / 16 * 16;
+}
+
+template <int D>
+constexpr int vc_fused_smem_bytes() {
+    return vc_fused_bar_offset<D>() + 48;  // full[2], empty[2], abort flag
+}
+
+// grid: B*H*(1 + D/32) with clusters of (1 + D/32, 1, 1); block: VC_THREADS; dynamic shared
+// memory: vc_fused_smem_bytes<D>().
+template <int D, bool RATIO>
+__global__ void __launch_bounds__(VC_THREADS, 1)
+    vla_fused_kernel(const float* __restrict__ q, const float* __restrict__ k,
+                     const float* __restrict__ v, const float* __restrict__ u,
+                     const float* __restrict__ S0, const float* __restrict__ A0,
+                     const float* __restrict__ n0, float lambda0, float* __restrict__ out,
+                     float* __restrict__ S_final, float* __restrict__ A_final,
+                     float* __restrict__ n_final, int T) {
+    extern __shared__ __align__(16) unsigned char vc_smem_raw[];
+    constexpr int NS = D / VC_RS;  // S-phase CTAs per head
+    uint8_t* bars = vc_smem_raw + vc_fused_bar_offset<D>();
+    volatile int* abort_flag = reinterpret_cast<volatile int*>(bars + 32);
+    const uint32_t rank = vc_cluster_rank();
+    const long bh = blockIdx.x / (NS + 1);
+    if (threadIdx.x == 0) {
+        mbar_init(smem_u32(bars), 1);        // full[0]: armed by this CTA, bytes from rank 0
+        mbar_init(smem_u32(bars + 8), 1);    // full[1]
+        mbar_init(smem_u32(bars + 16), NS);  // empty[0]: one arrival per S-phase CTA
+        mbar_init(smem_u32(bars + 24), NS);  // empty[1]
+        *abort_flag = 0;
+        if (rank != 0) {
+            // the slots of the first two chunks, armed before any copy can be issued
+            const int nchunks = (T + VC_C - 1) / VC_C;
+            for (int c = 0; c < 2 && c < nchunks; ++c)
+                mbar_arrive_expect_tx(smem_u32(bars + 8 * c), vc_tile_bytes<D>());
+        }
+        mbar_init_fence();
+    }
+    __syncthreads();
+    cluster_sync_all();  // every barrier of the cluster is initialised before any remote arrival
+
+    VcLink link;
+    link.al_base = smem_u32(&reinterpret_cast<VcSSmem<D>*>(vc_smem_raw)->al[0][0][0]);
+    link.full_bar = smem_u32(bars);
+    link.empty_bar = smem_u32(bars + 16);
+    link.nranks = NS;
+    link.abort = abort_flag;
+    if (rank == 0)
+        vc_aphase<D, true>(vc_smem_raw, bh, k, u, A0, lambda0, A_final, nullptr, T, link);
+    else
+        vc_sphase<D, RATIO, true>(vc_smem_raw, bh, (int)(rank - 1) * VC_RS, q, k, v, nullptr, S0,
+                                  n0, out, S_final, n_final, T, link);
+    // no CTA may leave while another can still write into its shared memory or arrive on it
+    cluster_sync_all();
 }
 
 }  // namespace drscan

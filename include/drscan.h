@@ -183,13 +183,13 @@ int dr_decode_step_ex(const void* q, const void* k, const void* v, const float* 
  * B*H*T == 0, q, k, v, u and out are not read and may be NULL. A0, when given, must be
  * symmetric positive definite (it is the inverse of a penalty matrix).
  *
- * The scan runs chunked, 64 tokens at a time, in two kernels. The first turns the chunk's
- * Sherman-Morrison steps into one Woodbury update (a 64 x 64 Cholesky factorisation of
- * I + U A U^T) and writes every alpha_hat_t; the second applies the write and readout in
- * the WY form of a delta rule whose read key is k_t and write key alpha_hat_t. Between them
- * alpha_hat lives in B*H*T*d*4 bytes of scratch, taken stream-ordered from a memory pool of
- * the library's own (kept between calls) and released in stream order after the second
- * kernel. Where A stops being positive definite the device latches DR_ERR_NOT_SPD.
+ * The scan runs chunked, 64 tokens at a time. An A-phase turns the chunk's Sherman-Morrison
+ * steps into one Woodbury update (a 64 x 64 Cholesky factorisation of I + U A U^T) and
+ * produces every alpha_hat_t; an S-phase applies the write and readout in the WY form of a
+ * delta rule whose read key is k_t and write key alpha_hat_t, 32 rows of S per CTA. By
+ * default both run at once in one kernel, a cluster of 1 + d/32 CTAs per head that passes
+ * alpha_hat through shared memory (no scratch). Where A stops being positive definite the
+ * device latches DR_ERR_NOT_SPD.
  * Returns DR_OK or a negative status; on error nothing is launched.
  */
 int vla_scan_fwd(const float* q, const float* k, const float* v, const float* u,
@@ -200,9 +200,15 @@ int vla_scan_fwd(const float* q, const float* k, const float* v, const float* u,
 /* vla_scan_fwd_ex flag: the ratio readout (see below). */
 #define VLA_RATIO_READOUT 0x1
 /* vla_scan_fwd_ex flag: the per-token kernel (one CTA per head, the Sherman-Morrison steps
- * one token at a time) instead of the chunked pair. Same results up to rounding, no
+ * one token at a time) instead of the chunked scan. Same results up to rounding, no
  * scratch memory; slower. For testing and as a baseline. */
 #define VLA_SEQUENTIAL 0x2
+/* vla_scan_fwd_ex flag: the chunked scan as two kernels, the A-phase for every head first,
+ * then the S-phase, with alpha_hat in B*H*T*d*4 bytes of scratch taken stream-ordered from a
+ * memory pool of the library's own (kept between calls) and released in stream order after
+ * the second kernel. Same results as the fused kernel; slower (the phases do not overlap).
+ * The fused kernel also falls back to this pair where its cluster does not fit. */
+#define VLA_TWO_KERNEL 0x4
 
 /*
  * vla_scan_fwd_ex -- vla_scan_fwd with the ratio readout of "Variational Linear Attention
@@ -219,7 +225,7 @@ int vla_scan_fwd(const float* q, const float* k, const float* v, const float* u,
  *   n0       [B,H,d] fp32 initial denominator state, or NULL for zeros (ratio readout only)
  *   n_final  [B,H,d] fp32 final denominator state, or NULL to skip (ratio readout only)
  *   flags    0 (o_t = S_t q_t, exactly vla_scan_fwd) or VLA_RATIO_READOUT, optionally
- *            with VLA_SEQUENTIAL
+ *            with one of VLA_SEQUENTIAL and VLA_TWO_KERNEL
  *
  * Other arguments, rules and return values as vla_scan_fwd; n0 / n_final with flags = 0
  * return DR_ERR_INVALID_ARG. The denominator is not guarded: where n_t q_t is zero the output
@@ -235,19 +241,20 @@ int vla_scan_fwd_ex(const float* q, const float* k, const float* v, const float*
 #define VLA_NOALLOC_MAX_FLOATS 16777216
 
 /*
- * vla_scan_fwd_noalloc -- vla_scan_fwd_ex (chunked pair only) without any memory allocation.
+ * vla_scan_fwd_noalloc -- vla_scan_fwd_ex with VLA_TWO_KERNEL, without any memory allocation.
  * The pages have no counterpart: this entry point exists for callers that must not allocate
  * device memory, such as a serving engine that reserves all device memory up front for its
  * own allocator and forbids later allocations, or code that runs where a driver allocation
- * may block or synchronise (a latency-bound step, an allocator's own callback). The chunked
- * VLA scan needs B*H*T*d floats of scratch for the write directions between its two
- * kernels; vla_scan_fwd_ex takes them from a memory pool, this entry point from a fixed
- * array compiled into the library, which every GPU that loads the library holds
- * (VLA_NOALLOC_MAX_FLOATS floats, 64 MiB) until the process exits.
+ * may block or synchronise (a latency-bound step, an allocator's own callback). The
+ * two-kernel form of the chunked VLA scan needs B*H*T*d floats of scratch for the write
+ * directions between its kernels; vla_scan_fwd_ex takes them from a memory pool, this entry
+ * point from a fixed array compiled into the library, which every GPU that loads the library
+ * holds (VLA_NOALLOC_MAX_FLOATS floats, 64 MiB) until the process exits. (The default fused
+ * form of vla_scan_fwd_ex needs no scratch either, where its cluster fits on the device.)
  *
  * Arguments, layout and results are those of vla_scan_fwd_ex; flags is 0 or
- * VLA_RATIO_READOUT (VLA_SEQUENTIAL returns DR_ERR_INVALID_ARG: the per-token kernel needs no
- * scratch). B*H*T*d above VLA_NOALLOC_MAX_FLOATS returns DR_ERR_SCRATCH_LIMIT before
+ * VLA_RATIO_READOUT (other flags return DR_ERR_INVALID_ARG: the two-kernel pair is always
+ * the one that runs). B*H*T*d above VLA_NOALLOC_MAX_FLOATS returns DR_ERR_SCRATCH_LIMIT before
  * anything is launched. The call makes no cudaMalloc, cudaFree or pool allocation.
  *
  * The first call on a device looks up the array's device address (cudaGetSymbolAddress,

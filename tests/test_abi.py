@@ -149,11 +149,13 @@ def call_vla_ex(lib, flags, B=1, n0=None):
 
 
 def test_vla_ex_flags(lib):
-    assert call_vla_ex(lib, 0x4) == drs.DR_ERR_INVALID_ARG
-    assert call_vla_ex(lib, drs.VLA_SEQUENTIAL | 0x8) == drs.DR_ERR_INVALID_ARG
+    assert call_vla_ex(lib, 0x8) == drs.DR_ERR_INVALID_ARG
+    assert call_vla_ex(lib, drs.VLA_SEQUENTIAL | 0x10) == drs.DR_ERR_INVALID_ARG
     assert call_vla_ex(lib, drs.VLA_SEQUENTIAL, n0=A) == drs.DR_ERR_INVALID_ARG  # n0: ratio only
-    for flags in (0, drs.VLA_SEQUENTIAL, drs.VLA_RATIO_READOUT,
-                  drs.VLA_RATIO_READOUT | drs.VLA_SEQUENTIAL):
+    assert call_vla_ex(lib, drs.VLA_SEQUENTIAL | drs.VLA_TWO_KERNEL) == drs.DR_ERR_INVALID_ARG
+    for flags in (0, drs.VLA_SEQUENTIAL, drs.VLA_TWO_KERNEL, drs.VLA_RATIO_READOUT,
+                  drs.VLA_RATIO_READOUT | drs.VLA_SEQUENTIAL,
+                  drs.VLA_RATIO_READOUT | drs.VLA_TWO_KERNEL):
         assert call_vla_ex(lib, flags, B=0) == drs.DR_OK
 
 

@@ -14,6 +14,10 @@ from delta_rule_recurrent_chunked_b200 import workloads as wl
 
 from helpers import MODE_NAME, oracle_dr, rel_err, row_rel_err, tensor_np, to_device
 
+# the three VLA paths of vla_scan_fwd_ex: the fused cluster kernel (default), the two-kernel
+# pair, the per-token kernel
+VLA_PATHS = {"fused": {}, "two_kernel": {"two_kernel": True}, "sequential": {"sequential": True}}
+
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
@@ -421,14 +425,14 @@ def test_decode_offsets_beyond_int32(oracle):
 
 
 # --- VLA: the chunked pair (default) and the per-token kernel (sequential=True)
-@pytest.mark.parametrize("sequential", [False, True])
+@pytest.mark.parametrize("path", ["fused", "two_kernel", "sequential"])
 @pytest.mark.parametrize("d", [32, 96])
-def test_vla_workload(oracle, d, sequential):
+def test_vla_workload(oracle, d, path):
     w = wl.workload(f"vla_fp32_d{d}")
     inputs = wl.generate_vla(w, 0)
     dev = {k: torch.from_numpy(inputs[k]).cuda() for k in ("q", "k", "v", "u")}
     out, Sf, Af = drs.vla_scan(dev["q"], dev["k"], dev["v"], dev["u"], lambda0=w.lambda0,
-                               sequential=sequential)
+                               **VLA_PATHS[path])
     torch.cuda.synchronize()
     heads = [0, 9, 31]
     sub = wl.head_slice(inputs, heads)
@@ -441,10 +445,10 @@ def test_vla_workload(oracle, d, sequential):
         assert row_rel_err(got, ref) <= 1e-4, row_rel_err(got, ref)
 
 
-@pytest.mark.parametrize("sequential", [False, True])
+@pytest.mark.parametrize("path", ["fused", "two_kernel", "sequential"])
 @pytest.mark.parametrize("d", [32, 64, 96, 128])
 @pytest.mark.parametrize("T", [1, 17, 64, 65, 100, 129])
-def test_vla_small_with_initial_state(oracle, d, T, sequential):
+def test_vla_small_with_initial_state(oracle, d, T, path):
     rng = np.random.default_rng(d + T)
     B, H = 1, 3
     unit = lambda x: x / np.linalg.norm(x, axis=-1, keepdims=True)
@@ -456,7 +460,7 @@ def test_vla_small_with_initial_state(oracle, d, T, sequential):
     M = rng.standard_normal((B, H, d, d)) / np.sqrt(d)
     A0 = np.linalg.inv(np.eye(d) + M @ np.swapaxes(M, -1, -2)).astype(np.float32)
     c = lambda x: torch.from_numpy(x).cuda()
-    out, Sf, Af = drs.vla_scan(c(q), c(k), c(v), c(u), S0=c(S0), A0=c(A0), sequential=sequential)
+    out, Sf, Af = drs.vla_scan(c(q), c(k), c(v), c(u), S0=c(S0), A0=c(A0), **VLA_PATHS[path])
     torch.cuda.synchronize()
     assert drs.poll_error() == drs.DR_OK
     ro, rs, ra = oracle.vla_scan(q, k, v, u, S0=S0, A0=A0)
@@ -496,6 +500,21 @@ def test_vla_chunked_long_sequence_with_state(oracle, d):
     for got, ref in ((out, ro), (Sf, rs), (Af, ra)):
         assert rel_err(tensor_np(got), ref) <= 1e-4
         assert row_rel_err(tensor_np(got), ref) <= 1e-4
+
+
+@pytest.mark.parametrize("d", [32, 96])
+def test_vla_fused_equals_two_kernel_bitwise(d):
+    # the fused kernel passes alpha_hat through shared memory instead of global memory; the
+    # arithmetic of both phases is the same, so every output must match bit for bit
+    w = wl.workload(f"vla_ratio_fp32_d{d}", T=700)
+    inputs = wl.generate_vla(w, 9)
+    dev = {k: torch.from_numpy(inputs[k]).cuda() for k in ("q", "k", "v", "u")}
+    a = drs.vla_scan_ratio(dev["q"], dev["k"], dev["v"], dev["u"])
+    b = drs.vla_scan_ratio(dev["q"], dev["k"], dev["v"], dev["u"], two_kernel=True)
+    torch.cuda.synchronize()
+    assert drs.poll_error() == drs.DR_OK
+    for x, y in zip(a, b):
+        assert torch.equal(x, y)
 
 
 def test_vla_chunked_non_positive_definite_a0_is_reported():

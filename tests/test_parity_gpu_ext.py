@@ -17,6 +17,10 @@ from delta_rule_recurrent_chunked_b200 import workloads as wl
 
 from helpers import MODE_NAME, oracle_dr_ex, rel_err, tensor_np, to_device
 
+# the three VLA paths of vla_scan_fwd_ex: the fused cluster kernel (default), the two-kernel
+# pair, the per-token kernel
+VLA_PATHS = {"fused": {}, "two_kernel": {"two_kernel": True}, "sequential": {"sequential": True}}
+
 torch = pytest.importorskip("torch")
 pytestmark = pytest.mark.gpu
 
@@ -165,14 +169,14 @@ def test_decode_step_ex(oracle, mode, dtype, dk, dv):
 
 # --- VLA ratio readout ("Variational Linear Attention (VLA)", section 2.3): the normaliser
 # n_t = n_{t-1} + (1 - n_{t-1} k_t) alpha_hat_t^T and o_t = S_t q_t / (n_t q_t), fp32, 1e-4
-@pytest.mark.parametrize("sequential", [False, True])
+@pytest.mark.parametrize("path", ["fused", "two_kernel", "sequential"])
 @pytest.mark.parametrize("d", [32, 96])
-def test_vla_ratio_workload(oracle, d, sequential):
+def test_vla_ratio_workload(oracle, d, path):
     w = wl.workload(f"vla_ratio_fp32_d{d}")
     inputs = wl.generate_vla(w, 0)
     dev = {k: torch.from_numpy(inputs[k]).cuda() for k in ("q", "k", "v", "u")}
     out, Sf, Af, nf = drs.vla_scan_ratio(dev["q"], dev["k"], dev["v"], dev["u"], lambda0=w.lambda0,
-                                         sequential=sequential)
+                                         **VLA_PATHS[path])
     torch.cuda.synchronize()
     heads = [0, 13, 31]
     sub = wl.head_slice(inputs, heads)
@@ -183,10 +187,10 @@ def test_vla_ratio_workload(oracle, d, sequential):
         assert rel_err(g, r) <= 1e-4, rel_err(g, r)
 
 
-@pytest.mark.parametrize("sequential", [False, True])
+@pytest.mark.parametrize("path", ["fused", "two_kernel", "sequential"])
 @pytest.mark.parametrize("d", [32, 64, 96, 128])
 @pytest.mark.parametrize("T", [1, 17, 64, 100, 129])
-def test_vla_ratio_small_with_initial_state(oracle, d, T, sequential):
+def test_vla_ratio_small_with_initial_state(oracle, d, T, path):
     rng = np.random.default_rng(7 * d + T)
     B, H = 1, 3
     elu1 = lambda x: np.where(x > 0, x + 1.0, np.exp(np.minimum(x, 0.0)))
@@ -201,7 +205,7 @@ def test_vla_ratio_small_with_initial_state(oracle, d, T, sequential):
     n0 = (0.5 + rng.uniform(size=(B, H, d)) / d).astype(np.float32)
     c = lambda x: torch.from_numpy(x).cuda()
     got = drs.vla_scan_ratio(c(q), c(k), c(v), c(u), S0=c(S0), A0=c(A0), n0=c(n0),
-                             sequential=sequential)
+                             **VLA_PATHS[path])
     torch.cuda.synchronize()
     ref = oracle.vla_scan_ratio(q, k, v, u, S0=S0, A0=A0, n0=n0)
     for g, r in zip(got, ref):
