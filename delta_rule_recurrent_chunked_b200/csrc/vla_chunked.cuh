@@ -274,9 +274,11 @@ __device__ __forceinline__ void vc_aphase(unsigned char* smem_raw, long bh,
         // U is not read again in this chunk: fetch the next chunk's rows under the factorisation
         if (nv_next > 0) vc_load_rows<D>(sm.u, uh + (long)(t0 + VC_C) * D, nv_next, tid);
 
-        // 3. M = L L^T by 16 x 16 blocks; the block rows of W = L^-1 (U A_c) follow each
-        //    diagonal block (forward substitution), and the trailing rows of M and of U A_c
-        //    take the block's contribution before the next one.
+        // 3. M = L L^T by 16 x 16 blocks. Per block: warp 0 factors the diagonal block (after
+        //    taking the previous block's contribution to it) while the other warps apply the
+        //    previous block's contribution to the rest of the trailing rows of M and of U A_c;
+        //    then the block rows of W = L^-1 (U A_c) (forward substitution, a thread per
+        //    column) and the panel below the block (a thread per row).
 #pragma unroll 1
         for (int jb = 0; jb < 4; ++jb) {
             const int b0 = 16 * jb;
@@ -285,6 +287,22 @@ __device__ __forceinline__ void vc_aphase(unsigned char* smem_raw, long bh,
                 const int l = tid & 15;
                 float r[16];
                 vc_ld<16>(&sm.m[b0 + l][b0], r);
+                if (jb > 0) {
+                    // the previous block's contribution to this diagonal block (the other
+                    // warps take the rest of the trailing matrix meanwhile)
+                    const int p0 = b0 - 16;
+                    float pl[16];
+                    vc_ld<16>(&sm.m[b0 + l][p0], pl);
+#pragma unroll
+                    for (int mm = 0; mm < 16; ++mm) {
+                        float pm[16];
+                        vc_ld<16>(&sm.m[b0 + mm][p0], pm);
+                        float dsum = 0.f;
+#pragma unroll
+                        for (int t = 0; t < 16; ++t) dsum = fmaf(pl[t], pm[t], dsum);
+                        if (mm <= l) r[mm] -= dsum;
+                    }
+                }
                 float my_inv = 0.f;
                 bool bad = false;
 #pragma unroll
@@ -313,6 +331,61 @@ __device__ __forceinline__ void vc_aphase(unsigned char* smem_raw, long bh,
                         if (mm <= l) sm.m[b0 + l][b0 + mm] = r[mm];
                     sm.dinv[b0 + l] = my_inv;
                     if (bad && l == 0) raise_status(DR_ERR_NOT_SPD);
+                }
+            } else if (jb > 0) {
+                const int p0 = b0 - 16;  // the block whose contribution is applied
+                const int n4 = (VC_C - 16 - p0) / 4;  // trailing rows, in groups of four
+                const int nm = n4 * n4;               // 4 x 4 tiles of the trailing block of M
+                const int nu = n4 * (D / 4);          // 4 x 4 tiles of the trailing rows of U A_c
+                for (int e = tid - 32; e < nm + nu; e += VC_THREADS - 32) {
+                    float li[4][16];
+                    float acc[4][4];
+                    if (e < nm) {
+                        const int ti = e / n4, ts = e - ti * n4;
+                        const int i0 = p0 + 16 + 4 * ti, s0 = p0 + 16 + 4 * ts;
+                        if (s0 > i0 + 3) continue;  // strictly above the diagonal: unused
+                        if (ti < 4 && ts < 4) continue;  // the next diagonal block: warp 0's
+#pragma unroll
+                        for (int a = 0; a < 4; ++a) vc_ld<16>(&sm.m[i0 + a][p0], li[a]);
+#pragma unroll
+                        for (int a = 0; a < 4; ++a) vc_ld<4>(&sm.m[i0 + a][s0], acc[a]);
+#pragma unroll
+                        for (int bb = 0; bb < 4; ++bb) {
+                            float ls[16];
+                            vc_ld<16>(&sm.m[s0 + bb][p0], ls);
+#pragma unroll
+                            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                                for (int t = 0; t < 16; ++t)
+                                    acc[a][bb] = fmaf(-li[a][t], ls[t], acc[a][bb]);
+                        }
+#pragma unroll
+                        for (int a = 0; a < 4; ++a)
+                            *reinterpret_cast<float4*>(&sm.m[i0 + a][s0]) =
+                                make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+                    } else {
+                        const int f = e - nm;
+                        const int ti = f / (D / 4), tc = f - ti * (D / 4);
+                        const int i0 = p0 + 16 + 4 * ti, c0 = 4 * tc;
+#pragma unroll
+                        for (int a = 0; a < 4; ++a) vc_ld<16>(&sm.m[i0 + a][p0], li[a]);
+#pragma unroll
+                        for (int a = 0; a < 4; ++a) vc_ld<4>(&sm.ua[i0 + a][c0], acc[a]);
+#pragma unroll
+                        for (int t = 0; t < 16; ++t) {
+                            float w4[4];
+                            vc_ld<4>(&sm.ua[p0 + t][c0], w4);
+#pragma unroll
+                            for (int a = 0; a < 4; ++a)
+#pragma unroll
+                                for (int j = 0; j < 4; ++j)
+                                    acc[a][j] = fmaf(-li[a][t], w4[j], acc[a][j]);
+                        }
+#pragma unroll
+                        for (int a = 0; a < 4; ++a)
+                            *reinterpret_cast<float4*>(&sm.ua[i0 + a][c0]) =
+                                make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+                    }
                 }
             }
             __syncthreads();
@@ -347,61 +420,6 @@ __device__ __forceinline__ void vc_aphase(unsigned char* smem_raw, long bh,
                         make_float4(x[t], x[t + 1], x[t + 2], x[t + 3]);
             }
             __syncthreads();
-            if (jb < 3) {
-                const int n4 = (VC_C - 16 - b0) / 4;  // trailing rows, in groups of four
-                const int nm = n4 * n4;               // 4 x 4 tiles of the trailing block of M
-                const int nu = n4 * (D / 4);          // 4 x 4 tiles of the trailing rows of U A_c
-                for (int e = tid; e < nm + nu; e += VC_THREADS) {
-                    float li[4][16];
-                    float acc[4][4];
-                    if (e < nm) {
-                        const int ti = e / n4, ts = e - ti * n4;
-                        const int i0 = b0 + 16 + 4 * ti, s0 = b0 + 16 + 4 * ts;
-                        if (s0 > i0 + 3) continue;  // strictly above the diagonal: unused
-#pragma unroll
-                        for (int a = 0; a < 4; ++a) vc_ld<16>(&sm.m[i0 + a][b0], li[a]);
-#pragma unroll
-                        for (int a = 0; a < 4; ++a) vc_ld<4>(&sm.m[i0 + a][s0], acc[a]);
-#pragma unroll
-                        for (int bb = 0; bb < 4; ++bb) {
-                            float ls[16];
-                            vc_ld<16>(&sm.m[s0 + bb][b0], ls);
-#pragma unroll
-                            for (int a = 0; a < 4; ++a)
-#pragma unroll
-                                for (int t = 0; t < 16; ++t)
-                                    acc[a][bb] = fmaf(-li[a][t], ls[t], acc[a][bb]);
-                        }
-#pragma unroll
-                        for (int a = 0; a < 4; ++a)
-                            *reinterpret_cast<float4*>(&sm.m[i0 + a][s0]) =
-                                make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
-                    } else {
-                        const int f = e - nm;
-                        const int ti = f / (D / 4), tc = f - ti * (D / 4);
-                        const int i0 = b0 + 16 + 4 * ti, c0 = 4 * tc;
-#pragma unroll
-                        for (int a = 0; a < 4; ++a) vc_ld<16>(&sm.m[i0 + a][b0], li[a]);
-#pragma unroll
-                        for (int a = 0; a < 4; ++a) vc_ld<4>(&sm.ua[i0 + a][c0], acc[a]);
-#pragma unroll
-                        for (int t = 0; t < 16; ++t) {
-                            float w4[4];
-                            vc_ld<4>(&sm.ua[b0 + t][c0], w4);
-#pragma unroll
-                            for (int a = 0; a < 4; ++a)
-#pragma unroll
-                                for (int j = 0; j < 4; ++j)
-                                    acc[a][j] = fmaf(-li[a][t], w4[j], acc[a][j]);
-                        }
-#pragma unroll
-                        for (int a = 0; a < 4; ++a)
-                            *reinterpret_cast<float4*>(&sm.ua[i0 + a][c0]) =
-                                make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
-                    }
-                }
-                __syncthreads();
-            }
         }
 
         // 4. tril(K W^T) (s <= t): rows rg + 16 i, columns cg + 16 j, over L's storage
