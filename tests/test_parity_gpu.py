@@ -502,6 +502,23 @@ def test_vla_chunked_long_sequence_with_state(oracle, d):
         assert row_rel_err(tensor_np(got), ref) <= 1e-4
 
 
+def test_vla_fused_many_clusters_d128(oracle):
+    # 80 heads at d = 128: clusters of 5 CTAs, 400 CTAs in all, more than one wave on the
+    # device; first, middle and last heads against the oracle
+    w = wl.VLAWorkload("vla_many", B=4, H=20, T=150, d=128)
+    inputs = wl.generate_vla(w, 12)
+    dev = {k: torch.from_numpy(inputs[k]).cuda() for k in ("q", "k", "v", "u")}
+    out, Sf, Af = drs.vla_scan(dev["q"], dev["k"], dev["v"], dev["u"])
+    torch.cuda.synchronize()
+    assert drs.poll_error() == drs.DR_OK
+    heads = [0, 41, 79]
+    sub = wl.head_slice(inputs, heads)
+    ref = oracle.vla_scan(sub["q"], sub["k"], sub["v"], sub["u"])
+    got = [tensor_np(t).reshape((80,) + tuple(t.shape[2:]))[heads][None] for t in (out, Sf, Af)]
+    for g, r in zip(got, ref):
+        assert rel_err(g, r) <= 1e-4
+
+
 @pytest.mark.parametrize("d", [32, 96])
 def test_vla_fused_equals_two_kernel_bitwise(d):
     # the fused kernel passes alpha_hat through shared memory instead of global memory; the
