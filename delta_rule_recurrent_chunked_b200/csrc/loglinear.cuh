@@ -13,8 +13,8 @@
 // trailing ones of c, M_j = V_c^T K_c + sum_{b<j} M_b and M_b = 0 for b < j.
 //
 // One CTA per (b, h, slice of BV value channels) walks the chunks in order. Eight warps: four
-// own 16 query rows each for the in-chunk part, four the same rows for the block-state
-// readouts and then 32 key channels each for the chunk state; every contraction is a bf16
+// own 16 query rows each for the in-chunk part and then 32 key channels each for the chunk
+// state and the merge, four the same rows for the block-state readouts; every contraction is a bf16
 // m16n8k16 warp MMA with fp32 accumulation (the tiles are 16-64 rows, the level bookkeeping
 // sits between them). The block states stay in shared memory in fp32
 // (dk x BV per level, for up to LL_LEVELS chunk levels: T <= 64 * 2^LL_LEVELS). The next
@@ -148,9 +148,10 @@ __device__ __forceinline__ void LoglinearStage::store(LoglinearSmem& sm) const {
 }
 
 // grid: (B*H, dv / LL_BV); block: LL_THREADS; dynamic shared memory: sizeof(LoglinearSmem).
-// Warps 0-3 take the in-chunk part of the outputs (query rows 16w .. 16w+15); warps 4-7 the
-// readouts of the block states for the same rows, then the chunk state (key channels
-// 32(w-4) .. +31) and the merge. The two halves meet in shared memory before the store.
+// Warps 0-3 take the in-chunk part of the outputs (query rows 16w .. 16w+15) and the chunk
+// state (key channels 32w .. +31), which they merge into the block states once the readouts
+// are done; warps 4-7 the readouts of the block states for the same rows. The two halves of
+// the outputs meet in shared memory before the store.
 __global__ void __launch_bounds__(LL_THREADS) loglinear_kernel(
     const __nv_bfloat16* __restrict__ q, const __nv_bfloat16* __restrict__ k,
     const __nv_bfloat16* __restrict__ v, const float* __restrict__ lam,
@@ -181,6 +182,7 @@ __global__ void __launch_bounds__(LL_THREADS) loglinear_kernel(
         float o[LL_BV / 8][4];
 #pragma unroll
         for (int n = 0; n < LL_BV / 8; ++n) o[n][0] = o[n][1] = o[n][2] = o[n][3] = 0.f;
+        float s[2][LL_BV / 8][4];  // this chunk's state V^T K (in-chunk warps)
         if (intra) {
             // P = Q K^T over the chunk's 64 keys, weighted by lambda of the pair's level
             float p[LL_C / 8][4];
@@ -225,6 +227,34 @@ __global__ void __launch_bounds__(LL_THREADS) loglinear_kernel(
                     const uint32_t b0[2] = {b[0], b[1]}, b1[2] = {b[2], b[3]};
                     ll_mma(o[2 * n2], a, b0);
                     ll_mma(o[2 * n2 + 1], a, b1);
+                }
+            }
+            // this chunk's state V^T K, transposed (rows = key channels 32*wq .. +31), here so
+            // that it overlaps the other warps' block-state readouts
+            if (c + 1 < nchunks) {
+#pragma unroll
+                for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+                    for (int n = 0; n < LL_BV / 8; ++n)
+                        s[mt][n][0] = s[mt][n][1] = s[mt][n][2] = s[mt][n][3] = 0.f;
+#pragma unroll
+                for (int kk = 0; kk < LL_C / 16; ++kk) {  // over the chunk's tokens
+#pragma unroll
+                    for (int mt = 0; mt < 2; ++mt) {
+                        // A (m = key channel, k = token) = K^T: transposed 8x8 loads of the K tile
+                        uint32_t a[4];
+                        const int kc0 = 32 * wq + 16 * mt;
+                        ll_ldsm_x4_t(a, &sm.k[kk * 16 + (lane & 7) + ((lane >> 4) << 3)]
+                                             [kc0 + ((lane >> 3) & 1) * 8]);
+#pragma unroll
+                        for (int n2 = 0; n2 < LL_BV / 16; ++n2) {
+                            uint32_t b[4];
+                            ll_ldsm_x4_t(b, &sm.v[kk * 16 + (lane & 15)][n2 * 16 + (lane >> 4) * 8]);
+                            const uint32_t b0[2] = {b[0], b[1]}, b1[2] = {b[2], b[3]};
+                            ll_mma(s[mt][2 * n2], a, b0);
+                            ll_mma(s[mt][2 * n2 + 1], a, b1);
+                        }
+                    }
                 }
             }
         } else {
@@ -283,55 +313,29 @@ __global__ void __launch_bounds__(LL_THREADS) loglinear_kernel(
                     *reinterpret_cast<uint32_t*>(out + (bh * T + t0 + tb) * (long)dv + v0 + col) =
                         pack_bf16(o[n][2] + xb.x, o[n][3] + xb.y);
             }
-            continue;
-        }
-        if (c + 1 == nchunks) continue;
-
-        // ---- this chunk's state V^T K, transposed: rows = key channels 32*wq .. +31
-        float s[2][LL_BV / 8][4];
+            // binary counter: M_j = this chunk + sum_{b<j} M_b, M_b = 0 for b < j. Each thread
+            // touches only its own (key channel, value channel) positions, and every readout
+            // of the block states finished before the barrier above.
+            if (c + 1 < nchunks) {
+                int j = 0;
+                while ((c >> j) & 1) ++j;
+                if (j < LL_LEVELS) {
 #pragma unroll
-        for (int mt = 0; mt < 2; ++mt)
+                    for (int mt = 0; mt < 2; ++mt) {
 #pragma unroll
-            for (int n = 0; n < LL_BV / 8; ++n) s[mt][n][0] = s[mt][n][1] = s[mt][n][2] = s[mt][n][3] = 0.f;
+                        for (int n = 0; n < LL_BV / 8; ++n) {
 #pragma unroll
-        for (int kk = 0; kk < LL_C / 16; ++kk) {  // over the chunk's tokens
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
-                // A (m = key channel, k = token) = K^T: transposed 8x8 loads of the K tile
-                uint32_t a[4];
-                const int kc0 = 32 * wq + 16 * mt;
-                ll_ldsm_x4_t(a, &sm.k[kk * 16 + (lane & 7) + ((lane >> 4) << 3)]
-                                     [kc0 + ((lane >> 3) & 1) * 8]);
-#pragma unroll
-                for (int n2 = 0; n2 < LL_BV / 16; ++n2) {
-                    uint32_t b[4];
-                    ll_ldsm_x4_t(b, &sm.v[kk * 16 + (lane & 15)][n2 * 16 + (lane >> 4) * 8]);
-                    const uint32_t b0[2] = {b[0], b[1]}, b1[2] = {b[2], b[3]};
-                    ll_mma(s[mt][2 * n2], a, b0);
-                    ll_mma(s[mt][2 * n2 + 1], a, b1);
-                }
-            }
-        }
-        // ---- binary counter: M_j = this chunk + sum_{b<j} M_b, M_b = 0 for b < j. Each
-        // thread touches only its own (key channel, value channel) positions, and every
-        // readout of the block states finished before the barrier above.
-        int j = 0;
-        while ((c >> j) & 1) ++j;
-        if (j < LL_LEVELS) {
-#pragma unroll
-            for (int mt = 0; mt < 2; ++mt) {
-#pragma unroll
-                for (int n = 0; n < LL_BV / 8; ++n) {
-#pragma unroll
-                    for (int e = 0; e < 4; ++e) {
-                        const int kc = 32 * wq + 16 * mt + g + ((e & 2) ? 8 : 0);
-                        const int vc = 8 * n + 2 * tg + (e & 1);
-                        float x = s[mt][n][e];
-                        for (int b = 0; b < j; ++b) {
-                            x += sm.m[b][vc][kc];
-                            sm.m[b][vc][kc] = 0.f;
+                            for (int e = 0; e < 4; ++e) {
+                                const int kc = 32 * wq + 16 * mt + g + ((e & 2) ? 8 : 0);
+                                const int vc = 8 * n + 2 * tg + (e & 1);
+                                float x = s[mt][n][e];
+                                for (int b = 0; b < j; ++b) {
+                                    x += sm.m[b][vc][kc];
+                                    sm.m[b][vc][kc] = 0.f;
+                                }
+                                sm.m[j][vc][kc] = x;
+                            }
                         }
-                        sm.m[j][vc][kc] = x;
                     }
                 }
             }
