@@ -447,9 +447,9 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 mbar_wait(bar(B_V_FULL + sv), (uint32_t)((c / NSV) & 1), abort_flag);
                 __nv_bfloat162* vt = reinterpret_cast<__nv_bfloat162*>(sm + L::V + sv * L::V_B);
                 constexpr int PAIRS = CK * BV / 2;
-                for (int e = lane; e < PAIRS; e += 32) {
-                    // the stored pair e at (row, col): plain rows, or swizzled 64-channel panels
-                    int row, col;
+                constexpr int VB16 = 16;  // gate loads in flight per lane
+                // the stored pair e at (row, col): plain rows, or swizzled 64-channel panels
+                auto pair_pos = [&](int e, int& row, int& col) {
                     if constexpr (L::V_SWZ) {
                         const int pn = e / (CK * 32), w = e % (CK * 32);  // 32 pairs per row
                         row = w >> 5;
@@ -458,11 +458,28 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                         row = e / (BV / 2);
                         col = 2 * (e % (BV / 2));
                     }
-                    const int t = c * CK + row;
-                    float2 w2 = make_float2(0.f, 0.f);
-                    if (t < T) w2 = *reinterpret_cast<const float2*>(write + (bh * T + t) * (long)dv + v0 + col);
-                    const float2 x = __bfloat1622float2(vt[e]);
-                    vt[e] = __floats2bfloat162_rn(x.x * w2.x, x.y * w2.y);
+                };
+                // the write gates of 16 pairs per lane are loaded together, then applied
+                for (int e0 = lane; e0 < PAIRS; e0 += 32 * VB16) {
+                    float2 w2[VB16];
+#pragma unroll
+                    for (int i = 0; i < VB16; ++i) {
+                        const int e = e0 + 32 * i;
+                        int row = 0, col = 0;
+                        if (e < PAIRS) pair_pos(e, row, col);
+                        const int t = c * CK + row;
+                        w2[i] = (e < PAIRS && t < T)
+                                    ? *reinterpret_cast<const float2*>(write + (bh * T + t) * (long)dv + v0 + col)
+                                    : make_float2(0.f, 0.f);
+                    }
+#pragma unroll
+                    for (int i = 0; i < VB16; ++i) {
+                        const int e = e0 + 32 * i;
+                        if (e < PAIRS) {
+                            const float2 x = __bfloat1622float2(vt[e]);
+                            vt[e] = __floats2bfloat162_rn(x.x * w2[i].x, x.y * w2[i].y);
+                        }
+                    }
                 }
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar(B_VSCALED + sv));
