@@ -8,8 +8,12 @@
 // z_t = w_t (.) v_t. The write values u_t are optionally stored. One thread owns one row of
 // S in registers, so a token costs ~4*dk FMAs per thread and no cross-thread communication.
 // A CTA is one warp covering 32 consecutive rows (value channels) of one (b,h); tokens
-// are staged through shared memory in tiles and broadcast to the warp.
+// are staged through shared memory in tiles and broadcast to the warp. For fp32 inputs
+// without per-channel gates the tiles are double-buffered: the next tile is copied with
+// cp.async while the current one is scanned.
 #pragma once
+
+#include <type_traits>
 
 #include "common.cuh"
 
@@ -48,12 +52,15 @@ __global__ void __launch_bounds__(32) dr_sequential_kernel(
     const float* __restrict__ S0, TIn* __restrict__ out, float* __restrict__ S_final,
     TIn* __restrict__ u_out, int T, int dv) {
     constexpr bool kScalarGate = MODE == DR_GDN || MODE == DR_GDN2;
-    __shared__ __align__(16) float sk[SEQ_TILE][DK];
-    __shared__ __align__(16) float sq[SEQ_TILE][DK];
+    // double-buffered asynchronous tile copies (fp32 inputs, no per-channel gates)
+    constexpr bool kAsync = std::is_same<TIn, float>::value && MODE != DR_KDA && MODE != DR_GDN2;
+    constexpr int NBUF = kAsync ? 2 : 1;
+    __shared__ __align__(16) float skb[NBUF][SEQ_TILE][DK];
+    __shared__ __align__(16) float sqb[NBUF][SEQ_TILE][DK];
     __shared__ __align__(16) float sa[MODE == DR_KDA ? SEQ_TILE : 1][MODE == DR_KDA ? DK : 4];
-    __shared__ float sv[SEQ_TILE][32];
-    __shared__ float sb[SEQ_TILE];
-    __shared__ float sg[SEQ_TILE];
+    __shared__ __align__(16) float svb[NBUF][SEQ_TILE][32];
+    __shared__ __align__(16) float sbb[NBUF][SEQ_TILE];
+    __shared__ __align__(16) float sgb[NBUF][SEQ_TILE];
 
     const int lane = threadIdx.x;
     const long bh = blockIdx.x;
@@ -81,10 +88,61 @@ __global__ void __launch_bounds__(32) dr_sequential_kernel(
         for (int j = 0; j < DK; ++j) s[j] = 0.f;
     }
 
-    for (int t0 = 0; t0 < T; t0 += SEQ_TILE) {
+    // asynchronous copy of the tile starting at token t0c into buffer b: the k and q rows,
+    // this warp's 32 value channels of v, and the per-token beta and gate
+    auto copy_tile = [&](int t0c, int b) {
+        const int ntc = min(SEQ_TILE, T - t0c);
+        for (int e = lane; e < ntc * DK / 4; e += 32) {
+            const int tt = (4 * e) / DK, j = (4 * e) % DK;
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(&skb[b][tt][j])),
+                         "l"(reinterpret_cast<const float*>(kh) + (long)(t0c + tt) * DK + j)
+                         : "memory");
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(&sqb[b][tt][j])),
+                         "l"(reinterpret_cast<const float*>(qh) + (long)(t0c + tt) * DK + j)
+                         : "memory");
+        }
+        for (int e = lane; e < ntc * 8; e += 32) {  // 8 pieces of 16 bytes per token
+            const int tt = e >> 3, j = 4 * (e & 7);
+            asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(&svb[b][tt][j])),
+                         "l"(reinterpret_cast<const float*>(vh) + (long)(t0c + tt) * dv +
+                             blockIdx.y * 32 + j)
+                         : "memory");
+        }
+        if (lane < ntc) {
+            if (MODE != DR_LINEAR)
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(&sbb[b][lane])),
+                             "l"(beta + bh * T + t0c + lane)
+                             : "memory");
+            if (kScalarGate)
+                asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_u32(&sgb[b][lane])),
+                             "l"(gate + bh * T + t0c + lane)
+                             : "memory");
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    if constexpr (kAsync) {
+        if (T > 0) copy_tile(0, 0);
+    }
+
+    for (int t0 = 0, it = 0; t0 < T; t0 += SEQ_TILE, ++it) {
         const int nt = min(SEQ_TILE, T - t0);
+        const int cur = kAsync ? (it & 1) : 0;
+        float(*sk)[DK] = skb[cur];
+        float(*sq)[DK] = sqb[cur];
+        float(*sv)[32] = svb[cur];
+        float* sb = sbb[cur];
+        float* sg = sgb[cur];
         __syncwarp();
-        for (int e = lane; e < nt * DK; e += 32) {
+        if constexpr (kAsync) {
+            // the next tile goes out now; this one's copies are waited for
+            if (t0 + SEQ_TILE < T) {
+                copy_tile(t0 + SEQ_TILE, cur ^ 1);
+                asm volatile("cp.async.wait_group 1;" ::: "memory");
+            } else {
+                asm volatile("cp.async.wait_group 0;" ::: "memory");
+            }
+        }
+        for (int e = lane; e < (kAsync ? 0 : nt * DK); e += 32) {
             const int tt = e / DK, j = e % DK;
             const long kt = (bh * T + t0 + tt) * (long)DK + j;
             sk[tt][j] = to_f32(kh[(long)(t0 + tt) * DK + j]);
@@ -92,14 +150,16 @@ __global__ void __launch_bounds__(32) dr_sequential_kernel(
             sq[tt][j] = to_f32(qh[(long)(t0 + tt) * DK + j]);
             if constexpr (MODE == DR_KDA) sa[tt][j] = gate[kt];
         }
-        for (int tt = 0; tt < nt; ++tt) {
-            float x = to_f32(vh[(long)(t0 + tt) * dv + row]);
-            if constexpr (MODE == DR_GDN2) x *= write[(bh * T + t0 + tt) * (long)dv + row];  // z
-            sv[tt][lane] = x;
+        if constexpr (!kAsync) {
+            for (int tt = 0; tt < nt; ++tt) {
+                float x = to_f32(vh[(long)(t0 + tt) * dv + row]);
+                if constexpr (MODE == DR_GDN2) x *= write[(bh * T + t0 + tt) * (long)dv + row];  // z
+                sv[tt][lane] = x;
+            }
         }
         if (lane < nt) {
-            sb[lane] = (MODE == DR_LINEAR) ? 1.f : beta[bh * T + t0 + lane];
-            sg[lane] = kScalarGate ? gate[bh * T + t0 + lane] : 1.f;
+            if (!kAsync || MODE == DR_LINEAR) sb[lane] = (MODE == DR_LINEAR) ? 1.f : beta[bh * T + t0 + lane];
+            if (!kAsync || !kScalarGate) sg[lane] = kScalarGate ? gate[bh * T + t0 + lane] : 1.f;
         }
         __syncwarp();
 
