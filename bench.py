@@ -143,11 +143,12 @@ def aggregate_value(world: int, head_tokens: int, steps: int, total_ms_max: floa
 # dr_decode.cuh for the decode workload, loglinear.cuh for log-linear attention) at capture
 # time; a changed source reports null. Summaries with the commands are under profiles/.
 NCU_TRAFFIC = {
-    ("kda_bf16", "c20c5b6c976514f5"): 673301760 + 121483008,
-    ("gdn_bf16", "c20c5b6c976514f5"): 101820160 + 13235712,
-    ("gdn_long_t32768", "c20c5b6c976514f5"): 408017408 + 113290240,
+    ("kda_bf16", "abb1b7e75281f50e"): 673300736 + 120170496,
+    ("gdn_bf16", "abb1b7e75281f50e"): 101819392 + 13308672,
+    ("gdn_long_t32768", "abb1b7e75281f50e"): 408011776 + 113220352,
+    ("gdn2_bf16", "abb1b7e75281f50e"): 236016384 + 27737088,
     ("gdn_decode_bf16", "6c9773f81f64a408"): 271627008 + 211260672,
-    ("loglinear_bf16", "9a05bbf81176e812"): 107536384 + 19725312,
+    ("loglinear_bf16", "79c1bdb9297c23dc"): 107535616 + 22006784,
 }
 
 
