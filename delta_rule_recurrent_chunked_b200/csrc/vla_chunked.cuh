@@ -22,6 +22,11 @@
 // same write with its value held at 1: it is one more row of the state in every CTA, and
 // the readout divides by its output n_t q_t.
 //
+// Fused (vla_fused_kernel, one cluster per (b,h)): the A-phase CTA keeps only what the next
+// chunk needs, [U A_c; K A_c], M, its factor and A_{c+1}; it hands W and K A_c to the S-phase
+// CTAs of the cluster, each of which forms Y and the directions itself before its S-phase
+// step. Every CTA of a cluster runs one of the two phases at a time, on its own SM.
+//
 // Everything is fp32 on CUDA cores: the tolerance of fp32 inputs is below what one tf32
 // tensor-core pass keeps.
 #pragma once
@@ -102,17 +107,17 @@ __device__ __forceinline__ float vc_comp(const float4& f, int q) {
 }
 
 // ---- cluster hand-off of the write directions (fused kernel)
-// The A-phase CTA (cluster rank 0) writes a chunk's alpha_hat rows into its own K A_c tile
-// (dead by then) and one thread copies the tile into the ring slot of every S-phase CTA
-// (ranks 1 ..) with a bulk copy that completes its bytes on that CTA's `full` barrier of the
-// slot. An S-phase CTA arms that barrier (expected bytes) before it hands the slot back by
-// arriving on the A-phase CTA's `empty` barrier. Every wait is bounded (mbar-style, with the
+// Once a chunk's Cholesky factor is done, one thread of the A-phase CTA (cluster rank 0)
+// copies its W and K A_c tiles (adjacent in shared memory) into al[0] and al[1] of every
+// S-phase CTA (ranks 1 ..) with one bulk copy that completes its bytes on that CTA's `full`
+// barrier. An S-phase CTA arms that barrier (expected bytes) for the next chunk before it
+// hands the pair back by arriving on the A-phase CTA's `empty` barrier. Every wait is bounded (mbar-style, with the
 // CTA's abort flag); after a timeout a CTA stops sending and receiving and runs its loops to
 // the end, so every thread reaches the cluster barrier that ends the kernel.
 struct VcLink {
     uint32_t al_base;    // shared::cta address of the S-phase layout's al[0][0][0]
-    uint32_t full_bar;   // shared::cta address of full[0] (full[1] at +8)
-    uint32_t empty_bar;  // shared::cta address of empty[0] (empty[1] at +8)
+    uint32_t full_bar;   // shared::cta address of the `full` barrier
+    uint32_t empty_bar;  // shared::cta address of the `empty` barrier
     int nranks;          // S-phase CTAs of the cluster
     volatile int* abort;
 };
@@ -151,6 +156,106 @@ __device__ __forceinline__ bool vc_wait_cluster(uint32_t bar, uint32_t parity,
             return false;
         }
     }
+}
+
+// ---------------------------------------------------------------------------------------
+// Write directions of one chunk
+// ---------------------------------------------------------------------------------------
+// From the chunk's K rows, W = L^-1 (U A_c) and K A_c (shared-memory tiles of row stride
+// D + 4): Y = K A_c - tril(K W^T) W (s <= t) and alpha_hat_t = Y_t / |Y_t|. g is a 64 x 68
+// scratch for tril(K W^T). TO_GLOBAL: rows t < nv go to dst (row per token); otherwise
+// alpha_hat replaces K A_c in place, rows past the end of the sequence set to zero, and the
+// block is synchronised at the end. The A-phase kernel and the S-phase CTAs of the fused
+// kernel run this same code, so both forms give the same bits.
+template <int D, bool TO_GLOBAL>
+__device__ __forceinline__ void vc_alpha_hat(const float (*k)[D + 4], const float (*w)[D + 4],
+                                             float (*ka)[D + 4], float (*g)[VC_C + 4], int nv,
+                                             float* __restrict__ dst, int tid) {
+    constexpr int CT = D / 16;
+    const int rg = tid >> 4, cg = tid & 15;
+    // tril(K W^T): rows rg + 16 i, columns cg + 16 j
+    {
+        float acc[4][4];
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
+#pragma unroll 2
+        for (int kk = 0; kk < D; kk += 4) {
+            float4 a[4], b[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                a[i] = *reinterpret_cast<const float4*>(&k[rg + 16 * i][kk]);
+                b[i] = *reinterpret_cast<const float4*>(&w[cg + 16 * i][kk]);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    acc[i][j] = fmaf(a[i].x, b[j].x, acc[i][j]);
+                    acc[i][j] = fmaf(a[i].y, b[j].y, acc[i][j]);
+                    acc[i][j] = fmaf(a[i].z, b[j].z, acc[i][j]);
+                    acc[i][j] = fmaf(a[i].w, b[j].w, acc[i][j]);
+                }
+        }
+        __syncthreads();  // every thread is done with what g held before it is overwritten
+#pragma unroll
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const int r = rg + 16 * i, s = cg + 16 * j;
+                g[r][s] = s <= r ? acc[i][j] : 0.f;
+            }
+    }
+    __syncthreads();
+    // Y = K A_c - tril(K W^T) W (rows rg + 16 i, columns cg*CT + j), normalised by rows over
+    // the 16 threads of a row group
+    {
+        float acc[4][CT];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) vc_ld<CT>(&ka[rg + 16 * i][cg * CT], acc[i]);
+#pragma unroll 2
+        for (int s = 0; s < VC_C; s += 4) {
+            float4 a[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) a[i] = *reinterpret_cast<const float4*>(&g[rg + 16 * i][s]);
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float b[CT];
+                vc_ld<CT>(&w[s + q][cg * CT], b);
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const float av = vc_comp(a[i], q);
+#pragma unroll
+                    for (int j = 0; j < CT; ++j) acc[i][j] = fmaf(-av, b[j], acc[i][j]);
+                }
+            }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float n2 = 0.f;
+#pragma unroll
+            for (int j = 0; j < CT; ++j) n2 = fmaf(acc[i][j], acc[i][j], n2);
+#pragma unroll
+            for (int off = 8; off > 0; off >>= 1) n2 += __shfl_xor_sync(0xffffffffu, n2, off);
+            const int r = rg + 16 * i;
+            if constexpr (TO_GLOBAL) {
+                if (r < nv) {
+                    const float inv = rsqrtf(n2);
+                    float* o = dst + (long)r * D + cg * CT;
+#pragma unroll
+                    for (int j = 0; j < CT; ++j) o[j] = acc[i][j] * inv;
+                }
+            } else {
+                // each thread rewrites only the K A_c entries it read
+                const float inv = r < nv ? rsqrtf(n2) : 0.f;
+                float* o = &ka[r][cg * CT];
+#pragma unroll
+                for (int j = 0; j < CT; ++j) o[j] = acc[i][j] * inv;
+            }
+        }
+    }
+    if constexpr (!TO_GLOBAL) __syncthreads();
 }
 
 // ---------------------------------------------------------------------------------------
@@ -271,38 +376,50 @@ __device__ __forceinline__ void vc_aphase(unsigned char* smem_raw, long bh,
                 }
         }
         __syncthreads();
-        // U is not read again in this chunk: fetch the next chunk's rows under the factorisation
-        if (nv_next > 0) vc_load_rows<D>(sm.u, uh + (long)(t0 + VC_C) * D, nv_next, tid);
+        // U is not read again in this chunk (nor K when the S-phase CTAs form the write
+        // directions): fetch the next chunk's rows under the factorisation
+        if (nv_next > 0) {
+            vc_load_rows<D>(sm.u, uh + (long)(t0 + VC_C) * D, nv_next, tid);
+            if constexpr (PUSH) vc_load_rows<D>(sm.k, kh + (long)(t0 + VC_C) * D, nv_next, tid);
+        }
 
-        // 3. M = L L^T by 16 x 16 blocks. Per block: warp 0 factors the diagonal block (after
-        //    taking the previous block's contribution to it) while the other warps apply the
-        //    previous block's contribution to the rest of the trailing rows of M and of U A_c;
-        //    then the block rows of W = L^-1 (U A_c) (forward substitution, a thread per
-        //    column) and the panel below the block (a thread per row).
+        // 3. M = L L^T by 16 x 16 blocks. Per block: warp 1 first applies the previous block's
+        //    contribution to this diagonal block and hands it to warp 0 on a named barrier;
+        //    warp 0 factors it while warps 1-7 apply that contribution to the rest of the
+        //    trailing rows of M and of U A_c; then the block rows of W = L^-1 (U A_c) (forward
+        //    substitution, a thread per column) and the panel below the block (a thread per row).
+        // M[i0..i0+3][s0..s0+3] -= P[i0..][.] P[s0..][.]^T, P = M's columns p0..p0+15 (the panel)
+        auto m_tile = [&](int i0, int s0, int p0) {
+            float li[4][16];
+            float acc[4][4];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) vc_ld<16>(&sm.m[i0 + a][p0], li[a]);
+#pragma unroll
+            for (int a = 0; a < 4; ++a) vc_ld<4>(&sm.m[i0 + a][s0], acc[a]);
+#pragma unroll
+            for (int bb = 0; bb < 4; ++bb) {
+                float ls[16];
+                vc_ld<16>(&sm.m[s0 + bb][p0], ls);
+#pragma unroll
+                for (int a = 0; a < 4; ++a)
+#pragma unroll
+                    for (int t = 0; t < 16; ++t) acc[a][bb] = fmaf(-li[a][t], ls[t], acc[a][bb]);
+            }
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+                *reinterpret_cast<float4*>(&sm.m[i0 + a][s0]) =
+                    make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+        };
 #pragma unroll 1
         for (int jb = 0; jb < 4; ++jb) {
             const int b0 = 16 * jb;
             if (tid < 32) {
                 // diagonal block in one warp: lane l (l < 16) holds row b0 + l in registers
                 const int l = tid & 15;
+                // warp 1 has applied the previous block's contribution to this block
+                if (jb > 0) asm volatile("bar.sync 1, 64;" ::: "memory");
                 float r[16];
                 vc_ld<16>(&sm.m[b0 + l][b0], r);
-                if (jb > 0) {
-                    // the previous block's contribution to this diagonal block (the other
-                    // warps take the rest of the trailing matrix meanwhile)
-                    const int p0 = b0 - 16;
-                    float pl[16];
-                    vc_ld<16>(&sm.m[b0 + l][p0], pl);
-#pragma unroll
-                    for (int mm = 0; mm < 16; ++mm) {
-                        float pm[16];
-                        vc_ld<16>(&sm.m[b0 + mm][p0], pm);
-                        float dsum = 0.f;
-#pragma unroll
-                        for (int t = 0; t < 16; ++t) dsum = fmaf(pl[t], pm[t], dsum);
-                        if (mm <= l) r[mm] -= dsum;
-                    }
-                }
                 float my_inv = 0.f;
                 bool bad = false;
 #pragma unroll
@@ -334,36 +451,32 @@ __device__ __forceinline__ void vc_aphase(unsigned char* smem_raw, long bh,
                 }
             } else if (jb > 0) {
                 const int p0 = b0 - 16;  // the block whose contribution is applied
+                if (tid < 64) {
+                    // warp 1: the ten lower 4 x 4 tiles of this diagonal block first (tile q
+                    // is row group ti, column group ts <= ti), then release warp 0
+                    const int q = tid - 32;
+                    if (q < 10) {
+                        const int ti = q < 1 ? 0 : q < 3 ? 1 : q < 6 ? 2 : 3;
+                        const int ts = q - ti * (ti + 1) / 2;
+                        m_tile(b0 + 4 * ti, b0 + 4 * ts, p0);
+                    }
+                    __syncwarp();
+                    __threadfence_block();
+                    asm volatile("bar.arrive 1, 64;" ::: "memory");
+                }
                 const int n4 = (VC_C - 16 - p0) / 4;  // trailing rows, in groups of four
                 const int nm = n4 * n4;               // 4 x 4 tiles of the trailing block of M
                 const int nu = n4 * (D / 4);          // 4 x 4 tiles of the trailing rows of U A_c
                 for (int e = tid - 32; e < nm + nu; e += VC_THREADS - 32) {
-                    float li[4][16];
-                    float acc[4][4];
                     if (e < nm) {
                         const int ti = e / n4, ts = e - ti * n4;
                         const int i0 = p0 + 16 + 4 * ti, s0 = p0 + 16 + 4 * ts;
                         if (s0 > i0 + 3) continue;  // strictly above the diagonal: unused
-                        if (ti < 4 && ts < 4) continue;  // the next diagonal block: warp 0's
-#pragma unroll
-                        for (int a = 0; a < 4; ++a) vc_ld<16>(&sm.m[i0 + a][p0], li[a]);
-#pragma unroll
-                        for (int a = 0; a < 4; ++a) vc_ld<4>(&sm.m[i0 + a][s0], acc[a]);
-#pragma unroll
-                        for (int bb = 0; bb < 4; ++bb) {
-                            float ls[16];
-                            vc_ld<16>(&sm.m[s0 + bb][p0], ls);
-#pragma unroll
-                            for (int a = 0; a < 4; ++a)
-#pragma unroll
-                                for (int t = 0; t < 16; ++t)
-                                    acc[a][bb] = fmaf(-li[a][t], ls[t], acc[a][bb]);
-                        }
-#pragma unroll
-                        for (int a = 0; a < 4; ++a)
-                            *reinterpret_cast<float4*>(&sm.m[i0 + a][s0]) =
-                                make_float4(acc[a][0], acc[a][1], acc[a][2], acc[a][3]);
+                        if (ti < 4 && ts < 4) continue;  // the diagonal block: done above
+                        m_tile(i0, s0, p0);
                     } else {
+                        float li[4][16];
+                        float acc[4][4];
                         const int f = e - nm;
                         const int ti = f / (D / 4), tc = f - ti * (D / 4);
                         const int i0 = p0 + 16 + 4 * ti, c0 = 4 * tc;
@@ -422,111 +535,27 @@ __device__ __forceinline__ void vc_aphase(unsigned char* smem_raw, long bh,
             __syncthreads();
         }
 
-        // 4. tril(K W^T) (s <= t): rows rg + 16 i, columns cg + 16 j, over L's storage
-        {
-            float acc[4][4];
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) acc[i][j] = 0.f;
-#pragma unroll 2
-            for (int kk = 0; kk < D; kk += 4) {
-                float4 a[4], b[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    a[i] = *reinterpret_cast<const float4*>(&sm.k[rg + 16 * i][kk]);
-                    b[i] = *reinterpret_cast<const float4*>(&sm.ua[cg + 16 * i][kk]);
-                }
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-#pragma unroll
-                    for (int j = 0; j < 4; ++j) {
-                        acc[i][j] = fmaf(a[i].x, b[j].x, acc[i][j]);
-                        acc[i][j] = fmaf(a[i].y, b[j].y, acc[i][j]);
-                        acc[i][j] = fmaf(a[i].z, b[j].z, acc[i][j]);
-                        acc[i][j] = fmaf(a[i].w, b[j].w, acc[i][j]);
-                    }
-            }
-            __syncthreads();  // every thread is done with L before it is overwritten
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-#pragma unroll
-                for (int j = 0; j < 4; ++j) {
-                    const int r = rg + 16 * i, s = cg + 16 * j;
-                    sm.m[r][s] = s <= r ? acc[i][j] : 0.f;
-                }
-        }
-        __syncthreads();
-        if (nv_next > 0) vc_load_rows<D>(sm.k, kh + (long)(t0 + VC_C) * D, nv_next, tid);
-
-        // 5. Y = K A_c - tril(K W^T) W (rows rg + 16 i, columns cg*CT + j), normalised by
-        //    rows over the 16 threads of a row group, written out as alpha_hat
-        {
-            float acc[4][CT];
-#pragma unroll
-            for (int i = 0; i < 4; ++i) vc_ld<CT>(&sm.ka[rg + 16 * i][cg * CT], acc[i]);
-#pragma unroll 2
-            for (int s = 0; s < VC_C; s += 4) {
-                float4 a[4];
-#pragma unroll
-                for (int i = 0; i < 4; ++i)
-                    a[i] = *reinterpret_cast<const float4*>(&sm.m[rg + 16 * i][s]);
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    float b[CT];
-                    vc_ld<CT>(&sm.ua[s + q][cg * CT], b);
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) {
-                        const float av = vc_comp(a[i], q);
-#pragma unroll
-                        for (int j = 0; j < CT; ++j) acc[i][j] = fmaf(-av, b[j], acc[i][j]);
-                    }
-                }
-            }
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float n2 = 0.f;
-#pragma unroll
-                for (int j = 0; j < CT; ++j) n2 = fmaf(acc[i][j], acc[i][j], n2);
-#pragma unroll
-                for (int off = 8; off > 0; off >>= 1) n2 += __shfl_xor_sync(0xffffffffu, n2, off);
-                const int r = rg + 16 * i;
-                if constexpr (PUSH) {
-                    // into this thread's own K A_c entries; rows past the end of the sequence
-                    // go out as zeros
-                    const float inv = r < nv ? rsqrtf(n2) : 0.f;
-                    float* dst = &sm.ka[r][cg * CT];
-#pragma unroll
-                    for (int j = 0; j < CT; ++j) dst[j] = acc[i][j] * inv;
-                } else {
-                    if (r < nv) {
-                        const float inv = rsqrtf(n2);
-                        float* dst = ah + (long)(t0 + r) * D + cg * CT;
-#pragma unroll
-                        for (int j = 0; j < CT; ++j) dst[j] = acc[i][j] * inv;
-                    }
-                }
-            }
-        }
         if constexpr (PUSH) {
-            // the tile is complete: copy it to every S-phase CTA once ring slot c % 2 (last
-            // filled for chunk c - 2) has been read by all of them
+            // W (in place of U A_c) and K A_c, adjacent tiles, go to every S-phase CTA, which
+            // forms the chunk's write directions itself: the next chunk's A-phase needs only
+            // W. The CTAs release the slot pair once they are done with the chunk.
             fence_async_smem();
             __syncthreads();
             if (tid == 0) {
-                const uint32_t slot = (uint32_t)(c & 1);
-                if (c >= 2)
-                    vc_wait_cluster(link.empty_bar + 8u * slot, (uint32_t)(((c >> 1) + 1) & 1),
-                                    link.abort);
+                if (c >= 1) vc_wait_cluster(link.empty_bar, (uint32_t)((c - 1) & 1), link.abort);
                 if (!*link.abort) {
                     for (int qr = 1; qr <= link.nranks; ++qr)
-                        bulk_copy_to_peer(
-                            cluster_map(link.al_base + slot * vc_tile_bytes<D>(), (uint32_t)qr),
-                            smem_u32(&sm.ka[0][0]), vc_tile_bytes<D>(),
-                            cluster_map(link.full_bar + 8u * slot, (uint32_t)qr));
+                        bulk_copy_to_peer(cluster_map(link.al_base, (uint32_t)qr),
+                                          smem_u32(&sm.ua[0][0]), 2 * vc_tile_bytes<D>(),
+                                          cluster_map(link.full_bar, (uint32_t)qr));
                     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
                 }
             }
+        } else {
+            // 4-5. the chunk's write directions, written out row per token (L's storage
+            //      takes tril(K W^T))
+            vc_alpha_hat<D, true>(sm.k, sm.ua, sm.ka, sm.m, nv, ah + (long)t0 * D, tid);
+            if (nv_next > 0) vc_load_rows<D>(sm.k, kh + (long)(t0 + VC_C) * D, nv_next, tid);
         }
 
         // 6. A_{c+1} = A_c - W^T W: rows rg*CT + i, columns cg*CT + j
@@ -591,7 +620,8 @@ struct VcSSmem {
     static constexpr int PR = VC_RS + 4;
     float k[VC_C][P];
     float q[VC_C][P];
-    float al[2][VC_C][P];        // alpha_hat rows, double buffered
+    float al[2][VC_C][P];        // alpha_hat rows, double buffered (fused: W, then K A_c and
+                                 // alpha_hat in its place)
     float S[VC_RS + 1][P];       // this CTA's rows of S (+ n for the ratio readout)
     float g[VC_C][VC_C + 4];     // strictly lower part of K Alpha^T
     float p[VC_C][VC_C + 4];     // lower part (diagonal included) of Q Alpha^T
@@ -602,7 +632,8 @@ struct VcSSmem {
 };
 
 // One head's S-phase for rows row0 .. row0 + 31 of S. PULL = false: alpha_hat from global
-// memory; PULL = true: from this CTA's ring, filled by the cluster's A-phase CTA (`link`).
+// memory; PULL = true: W and K A_c of each chunk arrive from the cluster's A-phase CTA
+// (`link`) into al[0] and al[1], and this CTA forms alpha_hat in al[1].
 template <int D, bool RATIO, bool PULL>
 __device__ __forceinline__ void vc_sphase(unsigned char* smem_raw, long bh, int row0,
                                           const float* __restrict__ q,
@@ -645,12 +676,14 @@ __device__ __forceinline__ void vc_sphase(unsigned char* smem_raw, long bh, int 
         const int nv_next = min(VC_C, T - t0 - VC_C);
         const int b = c & 1;
         if constexpr (PULL) {
-            // this chunk's directions: the k-th fill of slot b completes its phase k
-            vc_wait_cluster(link.full_bar + 8u * b, (uint32_t)((c >> 1) & 1), link.abort);
+            // this chunk's W and K A_c: the c-th fill of the slot pair completes phase c
+            vc_wait_cluster(link.full_bar, (uint32_t)(c & 1), link.abort);
+            vc_alpha_hat<D, false>(sm.k, sm.al[0], sm.al[1], sm.p, nv, nullptr, tid);
         } else {
             if (nv_next > 0)
                 vc_load_rows<D>(sm.al[b ^ 1], alpha + seq + (long)(t0 + VC_C) * D, nv_next, tid);
         }
+        float (*alh)[VcSSmem<D>::P] = sm.al[PULL ? 1 : b];  // this chunk's alpha_hat rows
 
         // 1. [G; P] = [K; Q] Alpha^T: rows rg + 16 i (i < 4 from K, i >= 4 from Q),
         //    columns cg + 16 j
@@ -669,7 +702,7 @@ __device__ __forceinline__ void vc_sphase(unsigned char* smem_raw, long bh, int 
                         i < 4 ? &sm.k[rg + 16 * i][kk] : &sm.q[rg + 16 * (i - 4)][kk]);
 #pragma unroll
                 for (int j = 0; j < 4; ++j)
-                    bb[j] = *reinterpret_cast<const float4*>(&sm.al[b][cg + 16 * j][kk]);
+                    bb[j] = *reinterpret_cast<const float4*>(&alh[cg + 16 * j][kk]);
 #pragma unroll
                 for (int i = 0; i < 8; ++i)
 #pragma unroll
@@ -855,14 +888,14 @@ __device__ __forceinline__ void vc_sphase(unsigned char* smem_raw, long bh, int 
             for (int s = 0; s < VC_C; ++s) {
                 const float2 x2 = *reinterpret_cast<const float2*>(&sm.r[s][rg * 2]);
                 float bb[CT];
-                vc_ld<CT>(&sm.al[b][s][cg * CT], bb);
+                vc_ld<CT>(&alh[s][cg * CT], bb);
 #pragma unroll
                 for (int j = 0; j < CT; ++j) {
                     acc[0][j] = fmaf(x2.x, bb[j], acc[0][j]);
                     acc[1][j] = fmaf(x2.y, bb[j], acc[1][j]);
                 }
                 if constexpr (RATIO) {
-                    if (tid < D) accn = fmaf(sm.r[s][VC_RS], sm.al[b][s][tid], accn);
+                    if (tid < D) accn = fmaf(sm.r[s][VC_RS], alh[s][tid], accn);
                 }
             }
 #pragma unroll
@@ -878,11 +911,11 @@ __device__ __forceinline__ void vc_sphase(unsigned char* smem_raw, long bh, int 
         vc_wait_copies();
         __syncthreads();
         if constexpr (PULL) {
-            // slot b is read (steps 1 and 5): arm it for chunk c + 2, then hand it back to the
-            // A-phase CTA
+            // the slot pair is read (alpha_hat by steps 1 and 5): arm it for chunk c + 1, then
+            // hand it back to the A-phase CTA
             if (tid == 0 && !*link.abort) {
-                if (c + 2 < nchunks) mbar_arrive_expect_tx(link.full_bar + 8u * b, vc_tile_bytes<D>());
-                mbar_arrive_remote(cluster_map(link.empty_bar + 8u * b, 0));
+                if (c + 1 < nchunks) mbar_arrive_expect_tx(link.full_bar, 2 * vc_tile_bytes<D>());
+                mbar_arrive_remote(cluster_map(link.empty_bar, 0));
             }
         }
     }
@@ -915,9 +948,10 @@ __global__ void __launch_bounds__(VC_THREADS, 1)
 // ---------------------------------------------------------------------------------------
 // Fused: both phases in one cluster per head
 // ---------------------------------------------------------------------------------------
-// Cluster of 1 + D/32 CTAs per (b,h): rank 0 runs the A-phase and hands every chunk's
-// alpha_hat rows to ranks 1 .. D/32 (the S-phase for 32 rows of S each) through their
-// shared-memory rings, so that both phases run at once on different SMs and no scratch
+// Cluster of 1 + D/32 CTAs per (b,h): rank 0 runs the A-phase and hands every chunk's W and
+// K A_c to ranks 1 .. D/32 (the S-phase for 32 rows of S each, which first form the chunk's
+// alpha_hat rows) through their shared memory, so that both phases run at once on different
+// SMs, the A-phase's serial chain holds only what the next chunk needs, and no scratch
 // memory is needed.
 template <int D>
 constexpr int vc_fused_bar_offset() {
@@ -927,7 +961,7 @@ constexpr int vc_fused_bar_offset() {
 
 template <int D>
 constexpr int vc_fused_smem_bytes() {
-    return vc_fused_bar_offset<D>() + 48;  // full[2], empty[2], abort flag
+    return vc_fused_bar_offset<D>() + 48;  // full (at +0), empty (at +16), abort flag (at +32)
 }
 
 // grid: B*H*(1 + D/32) with clusters of (1 + D/32, 1, 1); block: VC_THREADS; dynamic shared
@@ -947,16 +981,12 @@ __global__ void __launch_bounds__(VC_THREADS, 1)
     const uint32_t rank = vc_cluster_rank();
     const long bh = blockIdx.x / (NS + 1);
     if (threadIdx.x == 0) {
-        mbar_init(smem_u32(bars), 1);        // full[0]: armed by this CTA, bytes from rank 0
-        mbar_init(smem_u32(bars + 8), 1);    // full[1]
-        mbar_init(smem_u32(bars + 16), NS);  // empty[0]: one arrival per S-phase CTA
-        mbar_init(smem_u32(bars + 24), NS);  // empty[1]
+        mbar_init(smem_u32(bars), 1);        // full: armed by this CTA, bytes from rank 0
+        mbar_init(smem_u32(bars + 16), NS);  // empty: one arrival per S-phase CTA
         *abort_flag = 0;
-        if (rank != 0) {
-            // the slots of the first two chunks, armed before any copy can be issued
-            const int nchunks = (T + VC_C - 1) / VC_C;
-            for (int c = 0; c < 2 && c < nchunks; ++c)
-                mbar_arrive_expect_tx(smem_u32(bars + 8 * c), vc_tile_bytes<D>());
+        if (rank != 0 && T > 0) {
+            // the slot pair of the first chunk, armed before any copy can be issued
+            mbar_arrive_expect_tx(smem_u32(bars), 2 * vc_tile_bytes<D>());
         }
         mbar_init_fence();
     }
