@@ -108,16 +108,16 @@ __device__ __forceinline__ float vc_comp(const float4& f, int q) {
 
 // ---- cluster hand-off of the write directions (fused kernel)
 // Once a chunk's Cholesky factor is done, one thread of the A-phase CTA (cluster rank 0)
-// copies its W and K A_c tiles (adjacent in shared memory) into al[0] and al[1] of every
-// S-phase CTA (ranks 1 ..) with one bulk copy that completes its bytes on that CTA's `full`
-// barrier. An S-phase CTA arms that barrier (expected bytes) for the next chunk before it
-// hands the pair back by arriving on the A-phase CTA's `empty` barrier. Every wait is bounded (mbar-style, with the
+// copies its W and K A_c tiles (adjacent in shared memory) into a slot pair of every S-phase
+// CTA (ranks 1 ..) with one bulk copy that completes its bytes on that CTA's `full` barrier
+// of the pair. An S-phase CTA arms that barrier (expected bytes) for the pair's next chunk
+// before it hands the pair back by arriving on the A-phase CTA's `empty` barrier of the pair. Every wait is bounded (mbar-style, with the
 // CTA's abort flag); after a timeout a CTA stops sending and receiving and runs its loops to
 // the end, so every thread reaches the cluster barrier that ends the kernel.
 struct VcLink {
     uint32_t al_base;    // shared::cta address of the S-phase layout's al[0][0][0]
-    uint32_t full_bar;   // shared::cta address of the `full` barrier
-    uint32_t empty_bar;  // shared::cta address of the `empty` barrier
+    uint32_t full_bar;   // shared::cta address of full[0] (full[1] at +8)
+    uint32_t empty_bar;  // shared::cta address of empty[0] (empty[1] at +8)
     int nranks;          // S-phase CTAs of the cluster
     volatile int* abort;
 };
@@ -132,6 +132,14 @@ __device__ __forceinline__ uint32_t vc_cluster_rank() {
 template <int D>
 constexpr uint32_t vc_tile_bytes() {
     return (uint32_t)(VC_C * (D + 4) * 4);
+}
+
+// Slot pairs (W, K A_c) of an S-phase CTA in the fused kernel: two, so that a chunk's copy
+// lands while the previous chunk is worked on, where shared memory has room for them (up to
+// D = 96); one at D = 128.
+template <int D>
+constexpr int vc_nslot() {
+    return D <= 96 ? 2 : 1;
 }
 
 // Phase wait with cluster-scope acquire (the data behind the barrier was written by another
@@ -542,12 +550,18 @@ __device__ __forceinline__ void vc_aphase(unsigned char* smem_raw, long bh,
             fence_async_smem();
             __syncthreads();
             if (tid == 0) {
-                if (c >= 1) vc_wait_cluster(link.empty_bar, (uint32_t)((c - 1) & 1), link.abort);
+                // pair sp last held chunk c - NSL: its release is phase c / NSL - 1 of `empty`
+                constexpr int NSL = vc_nslot<D>();
+                const int sp = c % NSL;
+                if (c >= NSL)
+                    vc_wait_cluster(link.empty_bar + 8u * sp, (uint32_t)((c / NSL - 1) & 1),
+                                    link.abort);
                 if (!*link.abort) {
                     for (int qr = 1; qr <= link.nranks; ++qr)
-                        bulk_copy_to_peer(cluster_map(link.al_base, (uint32_t)qr),
-                                          smem_u32(&sm.ua[0][0]), 2 * vc_tile_bytes<D>(),
-                                          cluster_map(link.full_bar, (uint32_t)qr));
+                        bulk_copy_to_peer(
+                            cluster_map(link.al_base + sp * 2 * vc_tile_bytes<D>(), (uint32_t)qr),
+                            smem_u32(&sm.ua[0][0]), 2 * vc_tile_bytes<D>(),
+                            cluster_map(link.full_bar + 8u * sp, (uint32_t)qr));
                     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
                 }
             }
@@ -620,8 +634,9 @@ struct VcSSmem {
     static constexpr int PR = VC_RS + 4;
     float k[VC_C][P];
     float q[VC_C][P];
-    float al[2][VC_C][P];        // alpha_hat rows, double buffered (fused: W, then K A_c and
-                                 // alpha_hat in its place)
+    // alpha_hat rows, double buffered; fused: slot pair s holds W in al[2s] and K A_c, then
+    // alpha_hat in its place, in al[2s + 1]
+    float al[2 * vc_nslot<D>()][VC_C][P];
     float S[VC_RS + 1][P];       // this CTA's rows of S (+ n for the ratio readout)
     float g[VC_C][VC_C + 4];     // strictly lower part of K Alpha^T
     float p[VC_C][VC_C + 4];     // lower part (diagonal included) of Q Alpha^T
@@ -675,15 +690,17 @@ __device__ __forceinline__ void vc_sphase(unsigned char* smem_raw, long bh, int 
         const int nv = min(VC_C, T - t0);
         const int nv_next = min(VC_C, T - t0 - VC_C);
         const int b = c & 1;
+        constexpr int NSL = vc_nslot<D>();
+        const int sp = c % NSL;  // fused: this chunk's slot pair
         if constexpr (PULL) {
-            // this chunk's W and K A_c: the c-th fill of the slot pair completes phase c
-            vc_wait_cluster(link.full_bar, (uint32_t)(c & 1), link.abort);
-            vc_alpha_hat<D, false>(sm.k, sm.al[0], sm.al[1], sm.p, nv, nullptr, tid);
+            // this chunk's W and K A_c: the k-th fill of pair sp completes its phase k
+            vc_wait_cluster(link.full_bar + 8u * sp, (uint32_t)((c / NSL) & 1), link.abort);
+            vc_alpha_hat<D, false>(sm.k, sm.al[2 * sp], sm.al[2 * sp + 1], sm.p, nv, nullptr, tid);
         } else {
             if (nv_next > 0)
                 vc_load_rows<D>(sm.al[b ^ 1], alpha + seq + (long)(t0 + VC_C) * D, nv_next, tid);
         }
-        float (*alh)[VcSSmem<D>::P] = sm.al[PULL ? 1 : b];  // this chunk's alpha_hat rows
+        float (*alh)[VcSSmem<D>::P] = sm.al[PULL ? 2 * sp + 1 : b];  // this chunk's alpha_hat
 
         // 1. [G; P] = [K; Q] Alpha^T: rows rg + 16 i (i < 4 from K, i >= 4 from Q),
         //    columns cg + 16 j
@@ -911,11 +928,12 @@ __device__ __forceinline__ void vc_sphase(unsigned char* smem_raw, long bh, int 
         vc_wait_copies();
         __syncthreads();
         if constexpr (PULL) {
-            // the slot pair is read (alpha_hat by steps 1 and 5): arm it for chunk c + 1, then
-            // hand it back to the A-phase CTA
+            // pair sp is read (alpha_hat by steps 1 and 5): arm it for chunk c + NSL, then hand
+            // it back to the A-phase CTA
             if (tid == 0 && !*link.abort) {
-                if (c + 1 < nchunks) mbar_arrive_expect_tx(link.full_bar, 2 * vc_tile_bytes<D>());
-                mbar_arrive_remote(cluster_map(link.empty_bar, 0));
+                if (c + NSL < nchunks)
+                    mbar_arrive_expect_tx(link.full_bar + 8u * sp, 2 * vc_tile_bytes<D>());
+                mbar_arrive_remote(cluster_map(link.empty_bar + 8u * sp, 0));
             }
         }
     }
@@ -961,8 +979,11 @@ constexpr int vc_fused_bar_offset() {
 
 template <int D>
 constexpr int vc_fused_smem_bytes() {
-    return vc_fused_bar_offset<D>() + 48;  // full (at +0), empty (at +16), abort flag (at +32)
+    return vc_fused_bar_offset<D>() + 48;  // full[2] (at +0), empty[2] (at +16), abort (at +32)
 }
+static_assert(vc_fused_smem_bytes<32>() <= 232448 && vc_fused_smem_bytes<64>() <= 232448 &&
+                  vc_fused_smem_bytes<96>() <= 232448 && vc_fused_smem_bytes<128>() <= 232448,
+              "shared memory per CTA");
 
 // grid: B*H*(1 + D/32) with clusters of (1 + D/32, 1, 1); block: VC_THREADS; dynamic shared
 // memory: vc_fused_smem_bytes<D>().
@@ -981,12 +1002,16 @@ __global__ void __launch_bounds__(VC_THREADS, 1)
     const uint32_t rank = vc_cluster_rank();
     const long bh = blockIdx.x / (NS + 1);
     if (threadIdx.x == 0) {
-        mbar_init(smem_u32(bars), 1);        // full: armed by this CTA, bytes from rank 0
-        mbar_init(smem_u32(bars + 16), NS);  // empty: one arrival per S-phase CTA
+        mbar_init(smem_u32(bars), 1);        // full[0]: armed by this CTA, bytes from rank 0
+        mbar_init(smem_u32(bars + 8), 1);    // full[1]
+        mbar_init(smem_u32(bars + 16), NS);  // empty[0]: one arrival per S-phase CTA
+        mbar_init(smem_u32(bars + 24), NS);  // empty[1]
         *abort_flag = 0;
-        if (rank != 0 && T > 0) {
-            // the slot pair of the first chunk, armed before any copy can be issued
-            mbar_arrive_expect_tx(smem_u32(bars), 2 * vc_tile_bytes<D>());
+        if (rank != 0) {
+            // the slot pairs of the first chunks, armed before any copy can be issued
+            const int nchunks = (T + VC_C - 1) / VC_C;
+            for (int c = 0; c < vc_nslot<D>() && c < nchunks; ++c)
+                mbar_arrive_expect_tx(smem_u32(bars + 8 * c), 2 * vc_tile_bytes<D>());
         }
         mbar_init_fence();
     }
