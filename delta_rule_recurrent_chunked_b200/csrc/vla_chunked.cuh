@@ -277,7 +277,8 @@ struct VcASmem {
     float k[VC_C][P];
     float ua[VC_C][P];               // U A_c, then W = L^-1 U A_c
     float ka[VC_C][P];               // K A_c
-    float m[VC_C][VC_C + 4];         // I + U A_c U^T, then L (lower), then tril(K W^T)
+    float m[VC_C][VC_C + 4];         // I + U A_c U^T, then L's diagonal blocks, then tril(K W^T)
+    float pt[16][VC_C + 4];          // the panel of L below the current diagonal block, transposed
     float dinv[VC_C];                // 1 / L_tt
 };
 
@@ -396,22 +397,26 @@ __device__ __forceinline__ void vc_aphase(unsigned char* smem_raw, long bh,
         //    warp 0 factors it while warps 1-7 apply that contribution to the rest of the
         //    trailing rows of M and of U A_c; then the block rows of W = L^-1 (U A_c) (forward
         //    substitution, a thread per column) and the panel below the block (a thread per row).
-        // M[i0..i0+3][s0..s0+3] -= P[i0..][.] P[s0..][.]^T, P = M's columns p0..p0+15 (the panel)
-        auto m_tile = [&](int i0, int s0, int p0) {
-            float li[4][16];
+        // M[i0..i0+3][s0..s0+3] -= P[i0..][.] P[s0..][.]^T, P = the panel (rows of L below the
+        // previous diagonal block, held transposed in pt: four rows are one float4 per t)
+        auto m_tile = [&](int i0, int s0) {
+            float li[4][16], ls[4][16];
             float acc[4][4];
 #pragma unroll
-            for (int a = 0; a < 4; ++a) vc_ld<16>(&sm.m[i0 + a][p0], li[a]);
+            for (int t = 0; t < 16; ++t) {
+                const float4 x = *reinterpret_cast<const float4*>(&sm.pt[t][i0]);
+                const float4 y = *reinterpret_cast<const float4*>(&sm.pt[t][s0]);
+                li[0][t] = x.x, li[1][t] = x.y, li[2][t] = x.z, li[3][t] = x.w;
+                ls[0][t] = y.x, ls[1][t] = y.y, ls[2][t] = y.z, ls[3][t] = y.w;
+            }
 #pragma unroll
             for (int a = 0; a < 4; ++a) vc_ld<4>(&sm.m[i0 + a][s0], acc[a]);
 #pragma unroll
             for (int bb = 0; bb < 4; ++bb) {
-                float ls[16];
-                vc_ld<16>(&sm.m[s0 + bb][p0], ls);
 #pragma unroll
                 for (int a = 0; a < 4; ++a)
 #pragma unroll
-                    for (int t = 0; t < 16; ++t) acc[a][bb] = fmaf(-li[a][t], ls[t], acc[a][bb]);
+                    for (int t = 0; t < 16; ++t) acc[a][bb] = fmaf(-li[a][t], ls[bb][t], acc[a][bb]);
             }
 #pragma unroll
             for (int a = 0; a < 4; ++a)
@@ -466,7 +471,7 @@ __device__ __forceinline__ void vc_aphase(unsigned char* smem_raw, long bh,
                     if (q < 10) {
                         const int ti = q < 1 ? 0 : q < 3 ? 1 : q < 6 ? 2 : 3;
                         const int ts = q - ti * (ti + 1) / 2;
-                        m_tile(b0 + 4 * ti, b0 + 4 * ts, p0);
+                        m_tile(b0 + 4 * ti, b0 + 4 * ts);
                     }
                     __syncwarp();
                     __threadfence_block();
@@ -481,7 +486,7 @@ __device__ __forceinline__ void vc_aphase(unsigned char* smem_raw, long bh,
                         const int i0 = p0 + 16 + 4 * ti, s0 = p0 + 16 + 4 * ts;
                         if (s0 > i0 + 3) continue;  // strictly above the diagonal: unused
                         if (ti < 4 && ts < 4) continue;  // the diagonal block: done above
-                        m_tile(i0, s0, p0);
+                        m_tile(i0, s0);
                     } else {
                         float li[4][16];
                         float acc[4][4];
@@ -489,7 +494,10 @@ __device__ __forceinline__ void vc_aphase(unsigned char* smem_raw, long bh,
                         const int ti = f / (D / 4), tc = f - ti * (D / 4);
                         const int i0 = p0 + 16 + 4 * ti, c0 = 4 * tc;
 #pragma unroll
-                        for (int a = 0; a < 4; ++a) vc_ld<16>(&sm.m[i0 + a][p0], li[a]);
+                        for (int t = 0; t < 16; ++t) {
+                            const float4 x = *reinterpret_cast<const float4*>(&sm.pt[t][i0]);
+                            li[0][t] = x.x, li[1][t] = x.y, li[2][t] = x.z, li[3][t] = x.w;
+                        }
 #pragma unroll
                         for (int a = 0; a < 4; ++a) vc_ld<4>(&sm.ua[i0 + a][c0], acc[a]);
 #pragma unroll
@@ -535,10 +543,9 @@ __device__ __forceinline__ void vc_aphase(unsigned char* smem_raw, long bh,
 #pragma unroll
                     for (int s = t + 1; s < 16; ++s) x[s] = fmaf(-x[t], sm.m[b0 + s][b0 + t], x[s]);
                 }
+                // into the transposed panel, which only the next block's updates read
 #pragma unroll
-                for (int t = 0; t < 16; t += 4)
-                    *reinterpret_cast<float4*>(&sm.m[i][b0 + t]) =
-                        make_float4(x[t], x[t + 1], x[t + 2], x[t + 3]);
+                for (int t = 0; t < 16; ++t) sm.pt[t][i] = x[t];
             }
             __syncthreads();
         }
