@@ -412,7 +412,7 @@ def fp32_alu_peak_tflops(device) -> float:
 
 
 def base_line(args, w, world, K, total_ms_max, clk, e2e_ms, e2e_h2d, e2e_d2h, config, dtype,
-              t_wall):
+              t_wall, launches_per_step=1):
     return {
         "metric": METRIC, "value": aggregate_value(world, w.head_tokens, K, total_ms_max),
         "unit": UNIT, "n_gpus": world, "steps": K, "warmup": max(3, args.warmup),
@@ -421,7 +421,7 @@ def base_line(args, w, world, K, total_ms_max, clk, e2e_ms, e2e_h2d, e2e_d2h, co
         "clocks": {k: clk[k] for k in ("sm_mhz", "sm_max_mhz", "reasons")},
         "e2e": {"value": world * w.head_tokens / (e2e_ms / 1e3), "unit": UNIT,
                 "h2d_bytes_per_step": e2e_h2d, "d2h_bytes_per_step": e2e_d2h},
-        "gpu_launches": K,
+        "gpu_launches": K * launches_per_step,
         "wall_s": t_wall,
     }
 
@@ -475,10 +475,14 @@ def measure_dr(args, w, world, rank, local, device, K, cpu_target):
     achieved = nbytes / (launch_ms / 1e3) / 1e9
     tflops = algorithmic_flops(w) / (launch_ms / 1e3) / 1e12
     chunked = drs.chunked_applies(mode, w.dtype == "bf16", w.dk, w.dv)
+    # Gated DeltaNet-2 on the chunked path is two launches per call: the pre-scaling of k and
+    # v by the erase and write gates, then the chunked kernel; the roofline is the call's
+    prescaled = chunked and w.mode == wl.GDN2
     config = dict(workload_config(w, world), l2=l2_note(nsets, nbytes, needs_flush),
-                  kernel="chunked" if chunked else "sequential")
+                  kernel=("prescale+chunked" if prescaled else "chunked") if chunked
+                  else "sequential")
     line = base_line(args, w, world, K, total_ms_max, clk, e2e_ms, e2e["h2d"], e2e["d2h"], config,
-                     w.dtype, t_wall)
+                     w.dtype, t_wall, launches_per_step=2 if prescaled else 1)
     line["roofline"] = {
         "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
         "frac": achieved / peaks["hbm_gbs"],

@@ -14,8 +14,8 @@
 //     S_C^T  = diag(gamma_C) S0^T + Khat^T Y,  Khat^T = K^T diag(gamma_C/gamma) T
 // (KDA: the decay sits inside the operands, K*gamma, Q*gamma and K/gamma per channel, and
 // Khat^T = diag(gamma_C) (K/gamma)^T T. Gated DeltaNet-2 is Gated DeltaNet run on its erase
-// directions e = b (.) k and write targets z = w (.) v: the prep warps scale the K tile by b
-// and the V producer the V tile by w, in shared memory.) Rows 0-63 of MMA2 below are
+// directions e = b (.) k and write targets z = w (.) v, which its entry point forms in
+// scratch before this kernel runs.) Rows 0-63 of MMA2 below are
 // T Y = U, the chunk's write values u_t = beta_t r_t, stored when the caller asks for them.
 //
 // Contractions on tcgen05 (bf16 operands in 128-byte-swizzled shared memory, fp32
@@ -72,9 +72,9 @@ constexpr int CHUNK_THREADS = 512;
 template <int MODE, int BV, bool SPLIT = false>
 struct ChunkLayout {
     static constexpr bool kKda = MODE == DR_KDA;
-    static constexpr bool kGdn = MODE == DR_GDN || MODE == DR_GDN2;  // scalar gate
+    static constexpr bool kGdn = MODE == DR_GDN;  // scalar gate
     static_assert(!(SPLIT && kKda), "KDA is never split");
-    static_assert(!(SPLIT && MODE == DR_GDN2), "Gated DeltaNet-2 is never split");
+    static_assert(MODE != DR_GDN2, "Gated DeltaNet-2 runs as Gated DeltaNet on (q, e, z)");
     static constexpr int NS = 2;                          // K/Q stages
     static constexpr int NSV = (kKda && BV == 128) ? 1 : 2;  // V stages
     static constexpr int NP = (kKda && BV >= 64) ? 1 : 2;    // prepared-operand slots
@@ -183,8 +183,7 @@ enum ChunkBar {
     B_PREP2 = 27,      // split chain CTA: third slot ready
     B_MMA2 = 28,       // split chain CTA: MMA2 done
     B_SFREE = 29,      // [3] split chain CTA: chain slot i read by every thread and every MMA
-    B_VSCALED = 32,    // [2] Gated DeltaNet-2: V stage scaled by the write gate
-    B_COUNT = 34
+    B_COUNT = 32
 };
 
 // bf16 bits of 8 consecutive columns of a row, stored as one 16-byte swizzled chunk.
@@ -256,14 +255,12 @@ template <int MODE, int BV, bool SPLIT>
 __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
     const __grid_constant__ CUtensorMap tmV, const float* __restrict__ beta,
-    const float* __restrict__ gate, const float* __restrict__ erase,
-    const float* __restrict__ write, const float* __restrict__ S0,
+    const float* __restrict__ gate, const float* __restrict__ S0,
     __nv_bfloat16* __restrict__ out, float* __restrict__ S_final,
     __nv_bfloat16* __restrict__ u_out, int T, int dv, int nprep) {
     using L = ChunkLayout<MODE, BV, SPLIT>;
-    constexpr bool kGdn = L::kGdn;  // scalar gate (Gated DeltaNet and Gated DeltaNet-2)
+    constexpr bool kGdn = L::kGdn;  // scalar gate (Gated DeltaNet)
     constexpr bool kKda = MODE == DR_KDA;
-    constexpr bool kGdn2 = MODE == DR_GDN2;
     constexpr int NS = L::NS, NSV = L::NSV, NP = L::NP;
 
     extern __shared__ uint8_t smem_raw[];
@@ -342,8 +339,6 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
         mbar_init(bar(B_GRP1 + 3), 1);
         // output rows read out of D2 (and, when exporting, the write-value rows)
         mbar_init(bar(B_ODONE), u_out ? 256 : 128);
-        mbar_init(bar(B_VSCALED + 0), 1);
-        mbar_init(bar(B_VSCALED + 1), 1);
         mbar_init(bar(B_MMA1), 1);
         // split chain CTA: the residual threads arrive after writing Y, the others once the
         // state they rescaled in tensor memory for the next MMA3 is stored
@@ -426,8 +421,6 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
         }
     } else if (warp == 3 && is_chain) {
         // ------------------------------------------------------------------ V producer
-        // (Gated DeltaNet-2: the whole warp then scales the landed tile in place by the write
-        // gate, z = w (.) v, and releases it on B_VSCALED)
         for (int c = 0; c < nchunks; ++c) {
             const int sv = c % NSV;
             if (lane == 0) {
@@ -441,48 +434,6 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                         tma_load_3d(smem_u32(sm + L::V + sv * L::V_B + pn * CK * VB * 2), &tmV,
                                     bar(B_V_FULL + sv), v0 + pn * VB, c * CK, (int)bh);
                 }
-            }
-            if constexpr (kGdn2) {
-                __syncwarp();
-                mbar_wait(bar(B_V_FULL + sv), (uint32_t)((c / NSV) & 1), abort_flag);
-                __nv_bfloat162* vt = reinterpret_cast<__nv_bfloat162*>(sm + L::V + sv * L::V_B);
-                constexpr int PAIRS = CK * BV / 2;
-                constexpr int VB16 = 16;  // gate loads in flight per lane
-                // the stored pair e at (row, col): plain rows, or swizzled 64-channel panels
-                auto pair_pos = [&](int e, int& row, int& col) {
-                    if constexpr (L::V_SWZ) {
-                        const int pn = e / (CK * 32), w = e % (CK * 32);  // 32 pairs per row
-                        row = w >> 5;
-                        col = 64 * pn + ((((w >> 2) & 7) ^ (row & 7)) << 3) + 2 * (w & 3);
-                    } else {
-                        row = e / (BV / 2);
-                        col = 2 * (e % (BV / 2));
-                    }
-                };
-                // the write gates of 16 pairs per lane are loaded together, then applied
-                for (int e0 = lane; e0 < PAIRS; e0 += 32 * VB16) {
-                    float2 w2[VB16];
-#pragma unroll
-                    for (int i = 0; i < VB16; ++i) {
-                        const int e = e0 + 32 * i;
-                        int row = 0, col = 0;
-                        if (e < PAIRS) pair_pos(e, row, col);
-                        const int t = c * CK + row;
-                        w2[i] = (e < PAIRS && t < T)
-                                    ? *reinterpret_cast<const float2*>(write + (bh * T + t) * (long)dv + v0 + col)
-                                    : make_float2(0.f, 0.f);
-                    }
-#pragma unroll
-                    for (int i = 0; i < VB16; ++i) {
-                        const int e = e0 + 32 * i;
-                        if (e < PAIRS) {
-                            const float2 x = __bfloat1622float2(vt[e]);
-                            vt[e] = __floats2bfloat162_rn(x.x * w2[i].x, x.y * w2[i].y);
-                        }
-                    }
-                }
-                __syncwarp();
-                if (lane == 0) mbar_arrive(bar(B_VSCALED + sv));
             }
         }
     } else if (warp == 1 && !is_chain) {
@@ -927,7 +878,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             tc_fence_after();
             if (r < 64) {
                 // residual Y = V - gamma_t (S0 k_t), stored as the B operand Y^T
-                mbar_wait(bar((kGdn2 ? B_VSCALED : B_V_FULL) + svi), (uint32_t)((c / NSV) & 1),
+                mbar_wait(bar(B_V_FULL + svi), (uint32_t)((c / NSV) & 1),
                           abort_flag);
                 const float gt = kGdn ? gam[r] : 1.f;
                 // row r of V: 16-byte piece jj (channels 8jj .. 8jj+7)
@@ -1091,9 +1042,8 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
         float* pg = reinterpret_cast<float*>(sm + L::PG);
         // KDA: thread u owns key channels 2*(u%64), 2*(u%64)+1 on rows 16*(u/64) .. +15 of a
         // chunk; the next owned chunk's alpha values are prefetched into registers.
-        // Gated DeltaNet-2 prefetches its erase gate b the same way and scales K by it.
         const int kc = 2 * (u & 63), kq4 = u >> 6;
-        constexpr bool kChan = kKda || kGdn2;  // per-key-channel values prefetched per chunk
+        constexpr bool kChan = kKda;  // per-key-channel values prefetched per chunk
         // Byte offsets of (row 16*kq4 + i, channels kc, kc+1) in the 128-byte-swizzled K/Q
         // stage (128 rows per panel) and K/gamma tile (64 rows per panel): the swizzle of row
         // i depends on i & 7 only, so row i's offset is a per-thread base plus the 16-byte
@@ -1105,7 +1055,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                                  (uint32_t)(kc & 7) * 2u;
         const uint32_t kc_chunk = (uint32_t)((kc & 63) >> 3);
         auto xsw = [&](int i) -> uint32_t { return ((kc_chunk ^ (uint32_t)(i & 7)) << 4); };
-        const float* chan = kKda ? gate : erase;
+        const float* chan = gate;
         float2 gpf[kChan ? 16 : 1];
         if constexpr (kChan) {
 #pragma unroll
@@ -1133,25 +1083,6 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             bool fact = true;
             if constexpr (kGdn) {
                 fact = bg[64 + 63] > -80.f;
-                if constexpr (kGdn2) {
-                    // erase directions e = b (.) k, in place in the stage's K rows
-                    uint8_t* kr = kq + kq_row0;
-#pragma unroll
-                    for (int i0 = 0; i0 < 16; i0 += 8) {
-                        uint32_t kw[8];
-#pragma unroll
-                        for (int i = 0; i < 8; ++i)
-                            kw[i] = *reinterpret_cast<const uint32_t*>(kr + xsw(i) + (i0 + i) * 128);
-#pragma unroll
-                        for (int i = 0; i < 8; ++i) {
-                            const float2 k2 = __bfloat1622float2(*reinterpret_cast<__nv_bfloat162*>(&kw[i]));
-                            *reinterpret_cast<uint32_t*>(kr + xsw(i) + (i0 + i) * 128) =
-                                pack_bf16(k2.x * gpf[i0 + i].x, k2.y * gpf[i0 + i].y);
-                        }
-                    }
-                    fence_async_smem();
-                    gsync();
-                }
             } else if constexpr (kKda) {
                 // Per key channel c, G = summed log alpha over the chunk (four row quarters
                 // joined through shared memory) and the anchor m = G/2. K and Q are rewritten
@@ -1241,9 +1172,9 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             tc_fence_before();
             mbar_arrive(bar(gb + 0));
             if constexpr (kChan) {
-                // the next owned chunk's per-channel values (KDA's gates, Gated DeltaNet-2's
-                // erase gate), issued after this stage's proxy fence so that the fence does
-                // not wait for them; they land under the rest of this chunk's prep
+                // the next owned chunk's per-channel gates, issued after this stage's proxy
+                // fence so that the fence does not wait for them; they land under the rest of
+                // this chunk's prep
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int tn = (c + NGR * pSP) * CK + 16 * kq4 + i;
@@ -1522,13 +1453,15 @@ inline bool make_map_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt
     return r == CUDA_SUCCESS;
 }
 
+// Shapes and variants the chunked path takes (Gated DeltaNet-2 through its pre-scaled inputs).
 inline bool chunked_supported(int variant, int dk, int dv) {
     return dk == CDK && (dv == 32 || dv == 64 || dv == 128) &&
            (variant == DR_DELTANET || variant == DR_GDN || variant == DR_KDA ||
             variant == DR_GDN2);
 }
 
-// Arguments of one chunked launch (device pointers as dr_scan_fwd_ex receives them).
+// Arguments of one chunked launch (device pointers as dr_scan_fwd_ex receives them; erase
+// and write are read only by the Gated DeltaNet-2 pre-scaling).
 struct ChunkArgs {
     const void *q, *k, *v;
     const float *beta, *gate, *erase, *write, *S0;
@@ -1605,7 +1538,7 @@ int launch_chunked_bv(const ChunkArgs& a, int nprep, cudaStream_t stream) {
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = split ? 1 : 0;
-    if (cudaLaunchKernelEx(&cfg, kern, mk, mq, mv, a.beta, a.gate, a.erase, a.write, a.S0,
+    if (cudaLaunchKernelEx(&cfg, kern, mk, mq, mv, a.beta, a.gate, a.S0,
                            static_cast<__nv_bfloat16*>(a.out), a.S_final,
                            static_cast<__nv_bfloat16*>(a.u_out), a.T, a.dv, split) != cudaSuccess)
         return DR_ERR_CUDA;
@@ -1671,7 +1604,7 @@ struct SplitPlan {
 
 inline SplitPlan pick_split(int variant, long BH, int dv) {
     SplitPlan plan;
-    if (variant == DR_KDA || variant == DR_GDN2 || dv < 32) return plan;
+    if (variant == DR_KDA || dv < 32) return plan;
     const int bv = dv / 2, ncc = 2;
     for (int np = 4; np >= 1; --np) {
         if (BH * (np + ncc) <= 148 && BH <= max_active_clusters(np + ncc)) {
@@ -1686,7 +1619,7 @@ inline SplitPlan pick_split(int variant, long BH, int dv) {
 template <int MODE>
 int launch_chunked_mode(const ChunkArgs& a, cudaStream_t stream) {
     const SplitPlan plan = pick_split(MODE, a.BH, a.dv);
-    if constexpr (MODE != DR_KDA && MODE != DR_GDN2) {
+    if constexpr (MODE != DR_KDA) {
         if (plan.nprep > 0) {
             switch (plan.bv) {
                 case 16:
@@ -1720,8 +1653,6 @@ inline int launch_chunked(const ChunkArgs& a, int variant, cudaStream_t stream) 
             return launch_chunked_mode<DR_GDN>(a, stream);
         case DR_KDA:
             return launch_chunked_mode<DR_KDA>(a, stream);
-        case DR_GDN2:
-            return launch_chunked_mode<DR_GDN2>(a, stream);
     }
     return DR_ERR_UNSUPPORTED;
 }

@@ -131,6 +131,34 @@ int copy_state(float* dst, const float* src, size_t count, cudaStream_t stream) 
     return e == cudaSuccess ? DR_OK : DR_ERR_CUDA;
 }
 
+// Gated DeltaNet-2's erase directions e = b (.) k and write targets z = w (.) v in bf16 (each
+// product in fp32, rounded to nearest even), for the chunked path, which then runs Gated
+// DeltaNet on (q, e, z). A thread per 8 consecutive elements: the k part, then the v part.
+__global__ void gdn2_prescale_kernel(const __nv_bfloat16* __restrict__ k,
+                                     const float* __restrict__ b,
+                                     const __nv_bfloat16* __restrict__ v,
+                                     const float* __restrict__ w, __nv_bfloat16* __restrict__ e,
+                                     __nv_bfloat16* __restrict__ z, long nk8, long nv8) {
+    const long u = blockIdx.x * (long)blockDim.x + threadIdx.x;
+    if (u >= nk8 + nv8) return;
+    const bool kpart = u < nk8;
+    const long o = 8 * (kpart ? u : u - nk8);
+    const __nv_bfloat16* x = kpart ? k : v;
+    const float* g = kpart ? b : w;
+    const uint4 xr = *reinterpret_cast<const uint4*>(x + o);
+    const float4 g0 = *reinterpret_cast<const float4*>(g + o);
+    const float4 g1 = *reinterpret_cast<const float4*>(g + o + 4);
+    const __nv_bfloat162* xp = reinterpret_cast<const __nv_bfloat162*>(&xr);
+    const float2 a0 = __bfloat1622float2(xp[0]), a1 = __bfloat1622float2(xp[1]);
+    const float2 a2 = __bfloat1622float2(xp[2]), a3 = __bfloat1622float2(xp[3]);
+    uint4 y;
+    y.x = pack_bf16(a0.x * g0.x, a0.y * g0.y);
+    y.y = pack_bf16(a1.x * g0.z, a1.y * g0.w);
+    y.z = pack_bf16(a2.x * g1.x, a2.y * g1.y);
+    y.w = pack_bf16(a3.x * g1.z, a3.y * g1.w);
+    *reinterpret_cast<uint4*>((kpart ? e : z) + o) = y;
+}
+
 __global__ void scaled_identity_kernel(float* A, int d, long count, float diag) {
     long e = blockIdx.x * (long)blockDim.x + threadIdx.x;
     if (e < count) {
@@ -180,6 +208,30 @@ int scratch_alloc(void** p, size_t bytes, cudaStream_t stream) {
         pool = pools[dev];
     }
     return cudaMallocFromPoolAsync(p, bytes, pool, stream) == cudaSuccess ? DR_OK : DR_ERR_CUDA;
+}
+
+// Gated DeltaNet-2 on the chunked path: e and z into stream-ordered scratch, then the Gated
+// DeltaNet kernel (and its plan) on (q, e, z).
+int launch_gdn2_chunked(ChunkArgs a, int dk, cudaStream_t stream) {
+    const long nk = (long)a.BH * a.T * dk, nv = (long)a.BH * a.T * a.dv;
+    void* scratch = nullptr;
+    int rc = scratch_alloc(&scratch, (size_t)(nk + nv) * sizeof(__nv_bfloat16), stream);
+    if (rc != DR_OK) return rc;
+    __nv_bfloat16* e = static_cast<__nv_bfloat16*>(scratch);
+    __nv_bfloat16* z = e + nk;
+    const long units = (nk + nv) / 8;
+    gdn2_prescale_kernel<<<(unsigned)((units + 255) / 256), 256, 0, stream>>>(
+        static_cast<const __nv_bfloat16*>(a.k), a.erase, static_cast<const __nv_bfloat16*>(a.v),
+        a.write, e, z, nk / 8, nv / 8);
+    rc = launch_status();
+    if (rc == DR_OK) {
+        a.k = e;
+        a.v = z;
+        a.erase = a.write = nullptr;
+        rc = launch_chunked(a, DR_GDN, stream);
+    }
+    if (cudaFreeAsync(scratch, stream) != cudaSuccess && rc == DR_OK) rc = DR_ERR_CUDA;
+    return rc;
 }
 
 // The chunked pair: the A-phase writes alpha_hat into scratch, the S-phase reads it.
@@ -417,7 +469,8 @@ int dr_scan_fwd_ex(const void* q, const void* k, const void* v, const float* bet
                 variant == DR_GDN2 ? erase : nullptr, variant == DR_GDN2 ? write : nullptr,
                 S0, out, S_final, u_out, (int)BH, T, dv};
     if (bf16 && !(mode & DR_FORCE_SEQUENTIAL) && chunked_supported(variant, dk, dv))
-        return launch_chunked(a, variant, stream);
+        return variant == DR_GDN2 ? launch_gdn2_chunked(a, dk, stream)
+                                  : launch_chunked(a, variant, stream);
     if (bf16) return dispatch_sequential<__nv_bfloat16>(a, dk, variant, stream);
     return dispatch_sequential<float>(a, dk, variant, stream);
 }

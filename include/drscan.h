@@ -119,8 +119,12 @@ int dr_scan_fwd(const void* q, const void* k, const void* v, const float* beta,
  *            (v_t for DR_LINEAR). May not alias any other argument.
  *
  * DR_GDN2 takes gate [B,H,T] (alpha) like DR_GDN. With bf16 inputs and dk = 128 it runs
- * the chunked kernel, which scales the k and v tiles by b and w in shared memory before
- * they enter the tensor-core contractions; it always uses one CTA per (head, value slice).
+ * as two kernels on `stream`: the first writes e = b (.) k and z = w (.) v in bf16 (each
+ * product in fp32, rounded to nearest even) into B*H*T*(dk+dv)*2 bytes of scratch taken
+ * stream-ordered from a memory pool of the library's own (kept between calls, released in
+ * stream order after the call's last kernel); the second is the chunked Gated DeltaNet
+ * kernel, with its plan, on (q, e, z). DR_ERR_CUDA if the scratch cannot be had. Other
+ * inputs of DR_GDN2 take the per-token kernel, which applies b and w itself.
  * Asking for u_out adds one [B,H,T,dv] store (and, in a split launch, 8 KB more of each
  * chunk's operands copied between the CTAs of a cluster).
  */
@@ -307,7 +311,8 @@ int dr_poll_error(cudaStream_t stream);
 
 /*
  * The launch shape dr_scan_fwd picks for the chunked tensor-core kernel on the current
- * device, for `BH` = B*H sequences and the same `mode` word (variant | flags):
+ * device, for `BH` = B*H sequences and the same `mode` word (variant | flags; DR_GDN2 gets
+ * DR_GDN's plan, the kernel its chunked path runs on the pre-scaled inputs):
  *   *bv    value channels per chain CTA;
  *   *nprep prep CTAs per head in a split cluster (a cluster of *nprep prep CTAs and dv/(*bv)
  *          chain CTAs per head, used when the heads are too few to fill the GPU), or 0 when
