@@ -139,25 +139,31 @@ def aggregate_value(world: int, head_tokens: int, steps: int, total_ms_max: floa
 
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch from one ncu capture,
-# keyed by workload and the sha256 prefix of the timed kernel's source (dr_chunked.cuh,
-# dr_decode.cuh for the decode workload, loglinear.cuh for log-linear attention) at capture
-# time; a changed source reports null. Summaries with the commands are under profiles/.
+# keyed by workload and the sha256 prefix of the timed kernel's source (dr_chunked.cuh;
+# dr_chunked.cuh and drscan.cu for Gated DeltaNet-2's two kernels; dr_decode.cuh for the
+# decode workload; loglinear.cuh for log-linear attention) at capture time; a changed source
+# reports null. Summaries with the commands are under profiles/.
 NCU_TRAFFIC = {
-    ("kda_bf16", "abb1b7e75281f50e"): 673300736 + 120170496,
-    ("gdn_bf16", "abb1b7e75281f50e"): 101819392 + 13308672,
-    ("gdn_long_t32768", "abb1b7e75281f50e"): 408011776 + 113220352,
-    ("gdn2_bf16", "abb1b7e75281f50e"): 236016384 + 27737088,
+    ("kda_bf16", "a75847421d95ddbc"): 673533184 + 119739904,
+    ("gdn_bf16", "a75847421d95ddbc"): 101868288 + 12880128,
+    ("gdn_long_t32768", "a75847421d95ddbc"): 408205824 + 112992256,
+    # Gated DeltaNet-2: the pre-scaling kernel and the chunked kernel of one call
+    ("gdn2_bf16", "d285f93d654df439"): 201335552 + 45257216 + 101834240 + 12926464,
     ("gdn_decode_bf16", "6c9773f81f64a408"): 271627008 + 211260672,
     ("loglinear_bf16", "79c1bdb9297c23dc"): 107535616 + 22006784,
 }
 
 
-def kernel_source_sha(name: str = "dr_chunked.cuh") -> str:
+def kernel_source_sha(*names: str) -> str:
+    """sha256 prefix of the timed kernels' sources (dr_chunked.cuh by default; several files
+    are hashed in the order given)."""
     import hashlib
 
-    path = os.path.join(ROOT, "delta_rule_recurrent_chunked_b200", "csrc", name)
-    with open(path, "rb") as f:
-        return hashlib.sha256(f.read()).hexdigest()[:16]
+    h = hashlib.sha256()
+    for name in names or ("dr_chunked.cuh",):
+        with open(os.path.join(ROOT, "delta_rule_recurrent_chunked_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
 
 
 def load_peaks():
@@ -486,7 +492,9 @@ def measure_dr(args, w, world, rank, local, device, K, cpu_target):
     line["roofline"] = {
         "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
         "frac": achieved / peaks["hbm_gbs"],
-        "traffic": NCU_TRAFFIC.get((w.name, kernel_source_sha())) if chunked else None,
+        "traffic": (NCU_TRAFFIC.get((w.name, kernel_source_sha("dr_chunked.cuh", "drscan.cu")))
+                    if prescaled else NCU_TRAFFIC.get((w.name, kernel_source_sha()))
+                    if chunked else None),
         "peak_source": f"{peak_src} hbm_gbs", "bytes_per_launch": nbytes,
         "launch_ms": launch_ms, "tensor_tflops": tflops,
         "tensor_frac": tflops / peaks["bf16_tflops"]}
