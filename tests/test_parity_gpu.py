@@ -478,7 +478,7 @@ def test_vla_empty_sequence_returns_initial_state():
     assert torch.count_nonzero(Sf) == 0 and torch.allclose(Af, eye.expand_as(Af))
 
 
-@pytest.mark.parametrize("d", [32, 128])
+@pytest.mark.parametrize("d", [32, 96, 128])
 def test_vla_chunked_long_sequence_with_state(oracle, d):
     # 1000 tokens: 15 full chunks and a ragged one, entering S0 and A0 (a positive definite
     # inverse penalty), every head against the oracle
@@ -519,11 +519,12 @@ def test_vla_fused_many_clusters_d128(oracle):
         assert rel_err(g, r) <= 1e-4
 
 
-@pytest.mark.parametrize("d", [32, 96])
+@pytest.mark.parametrize("d", [32, 64, 96, 128])
 def test_vla_fused_equals_two_kernel_bitwise(d):
-    # the fused kernel passes alpha_hat through shared memory instead of global memory; the
-    # arithmetic of both phases is the same, so every output must match bit for bit
-    w = wl.workload(f"vla_ratio_fp32_d{d}", T=700)
+    # the fused kernel hands W and K A_c to the S-phase CTAs, which form alpha_hat with the
+    # same code the two-kernel form's A-phase runs (two slot pairs up to d = 96, one at 128);
+    # the arithmetic is the same, so every output must match bit for bit
+    w = wl.VLAWorkload(f"vla_ratio_d{d}", B=2, H=4, T=700, d=d, ratio=True)
     inputs = wl.generate_vla(w, 9)
     dev = {k: torch.from_numpy(inputs[k]).cuda() for k in ("q", "k", "v", "u")}
     a = drs.vla_scan_ratio(dev["q"], dev["k"], dev["v"], dev["u"])
