@@ -191,8 +191,9 @@ int dr_decode_step_ex(const void* q, const void* k, const void* v, const float* 
  * steps into one Woodbury update (a 64 x 64 Cholesky factorisation of I + U A U^T) and
  * produces every alpha_hat_t; an S-phase applies the write and readout in the WY form of a
  * delta rule whose read key is k_t and write key alpha_hat_t, 32 rows of S per CTA. By
- * default both run at once in one kernel, a cluster of 1 + d/32 CTAs per head that passes
- * alpha_hat through shared memory (no scratch). Where A stops being positive definite the
+ * default both run at once in one kernel, a cluster of 1 + d/32 CTAs per head whose A-phase
+ * CTA passes each chunk's W = L^-1 U A and K A through shared memory to the S-phase CTAs,
+ * which form alpha_hat themselves (no scratch). Where A stops being positive definite the
  * device latches DR_ERR_NOT_SPD.
  * Returns DR_OK or a negative status; on error nothing is launched.
  */
