@@ -466,7 +466,9 @@ def measure_dr(args, w, world, rank, local, device, K, cpu_target):
     torch.cuda.synchronize(device)
     if drs.poll_error(device) != 0:
         raise RuntimeError("device status set during warm-up")
+    seg0 = drs.segment_counters(device)
     total_ms, per_launch, clk, t_wall = timed_loop(step, K, device, stream, local, flush)
+    seg1 = drs.segment_counters(device)
     status = drs.poll_error(device)
     if status != 0:
         raise RuntimeError(f"device status {status} after the timed region")
@@ -484,11 +486,21 @@ def measure_dr(args, w, world, rank, local, device, K, cpu_target):
     # Gated DeltaNet-2 on the chunked path is two launches per call: the pre-scaling of k and
     # v by the erase and write gates, then the chunked kernel; the roofline is the call's
     prescaled = chunked and w.mode == wl.GDN2
+    # the segmented scan (few heads, long sequences) is four launches of this library per
+    # call: the zero-start pass over all segments, the window rerun, the hand-off check and
+    # the chained kernel's conditional launch (which returns at once when the checks pass)
+    nseg = drs.chunked_plan_ex(mode, w.B * w.H, w.T, w.dk, w.dv)[2] if chunked else 1
+    kname = "chunked" if nseg == 1 else f"segmented chunked ({nseg} segments per head)"
     config = dict(workload_config(w, world), l2=l2_note(nsets, nbytes, needs_flush),
-                  kernel=("prescale+chunked" if prescaled else "chunked") if chunked
+                  kernel=("prescale+" + kname if prescaled else kname) if chunked
                   else "sequential")
+    if nseg > 1:
+        # timed calls that took the segmented scan, and how many of them a failed hand-off
+        # check sent back to the chained kernel
+        config["segmented"] = {"calls": seg1[0] - seg0[0], "chained_reruns": seg1[1] - seg0[1]}
     line = base_line(args, w, world, K, total_ms_max, clk, e2e_ms, e2e["h2d"], e2e["d2h"], config,
-                     w.dtype, t_wall, launches_per_step=2 if prescaled else 1)
+                     w.dtype, t_wall,
+                     launches_per_step=(1 if prescaled else 0) + (4 if nseg > 1 else 1))
     line["roofline"] = {
         "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
         "frac": achieved / peaks["hbm_gbs"],

@@ -22,6 +22,7 @@ LIB_PATH = os.path.join(PKG, "libdrscan.so")
 DR_LINEAR, DR_DELTANET, DR_GDN, DR_KDA, DR_GDN2 = 0, 1, 2, 3, 4
 DR_IN_BF16 = 0x100
 DR_FORCE_SEQUENTIAL = 0x200
+DR_CHAINED = 0x400
 DR_OK, DR_ERR_INVALID_ARG, DR_ERR_UNSUPPORTED, DR_ERR_CUDA, DR_ERR_TIMEOUT, DR_ERR_DEVICE_BOUNDS = (
     0, -1, -2, -3, -4, -5)
 DR_ERR_GATE_RANGE = -6
@@ -46,6 +47,9 @@ SIGNATURES = {
     "dr_poll_error": ([_VP], _I),
     "dr_debug_timeout_probe": ([_I, _VP], _I),
     "dr_chunked_plan": ([_I, ctypes.c_longlong, _I, _I, ctypes.POINTER(_I), ctypes.POINTER(_I)], _I),
+    "dr_chunked_plan_ex": ([_I, ctypes.c_longlong, _I, _I, _I, ctypes.POINTER(_I),
+                            ctypes.POINTER(_I), ctypes.POINTER(_I)], _I),
+    "dr_segment_counters": ([ctypes.POINTER(ctypes.c_ulonglong)] * 2, _I),
     "dr_version": ([], _I),
 }
 
@@ -101,10 +105,11 @@ def _check(t, name, shape, dtype, device):
 
 
 def scan(q, k, v, beta=None, gate=None, S0=None, mode="gdn", want_state=True,
-         force_sequential=False, out=None, S_final=None):
+         force_sequential=False, out=None, S_final=None, chained=False):
     """Delta-rule scan on the GPU. q, k: [B,H,T,dk]; v: [B,H,T,dv] (bf16 or fp32, same
     dtype); beta: [B,H,T] fp32; gate: alpha values, [B,H,T] (gdn) or [B,H,T,dk] (kda) fp32;
-    S0: [B,H,dv,dk] fp32 or None. Returns (out like v, S_final fp32 or None)."""
+    S0: [B,H,dv,dk] fp32 or None. chained=True keeps Gated DeltaNet off the segmented scan
+    (DR_CHAINED). Returns (out like v, S_final fp32 or None)."""
     import torch
 
     variant = MODES[mode] if isinstance(mode, str) else int(mode)
@@ -138,6 +143,8 @@ def scan(q, k, v, beta=None, gate=None, S0=None, mode="gdn", want_state=True,
     flags = variant | (DR_IN_BF16 if q.dtype == torch.bfloat16 else 0)
     if force_sequential:
         flags |= DR_FORCE_SEQUENTIAL
+    if chained:
+        flags |= DR_CHAINED
     rc = lib().dr_scan_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(gate), _ptr(S0), _ptr(out),
                            _ptr(S_final), B, H, T, dk, dv, flags, _stream_handle(dev))
     if rc != DR_OK:
@@ -147,7 +154,7 @@ def scan(q, k, v, beta=None, gate=None, S0=None, mode="gdn", want_state=True,
 
 def scan_ex(q, k, v, beta=None, gate=None, S0=None, mode="gdn", erase=None, write=None,
             want_state=True, want_u=True, force_sequential=False, out=None, S_final=None,
-            u_out=None):
+            u_out=None, chained=False):
     """scan() with Gated DeltaNet-2 and the per-token write values, through dr_scan_fwd_ex.
     mode "gdn2" takes gate [B,H,T] (alpha), erase [B,H,T,dk] (b) and write [B,H,T,dv] (w),
     fp32. Returns (out, S_final or None, u or None): u [B,H,T,dv] like v holds the write
@@ -194,6 +201,8 @@ def scan_ex(q, k, v, beta=None, gate=None, S0=None, mode="gdn", erase=None, writ
     flags = variant | (DR_IN_BF16 if q.dtype == torch.bfloat16 else 0)
     if force_sequential:
         flags |= DR_FORCE_SEQUENTIAL
+    if chained:
+        flags |= DR_CHAINED
     rc = lib().dr_scan_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(beta), _ptr(gate), _ptr(erase),
                               _ptr(write), _ptr(S0), _ptr(out), _ptr(S_final), _ptr(u_out),
                               B, H, T, dk, dv, flags, _stream_handle(dev))
@@ -410,6 +419,36 @@ def chunked_plan(mode, BH: int, dk: int, dv: int) -> tuple:
     if st != DR_OK:
         raise DrScanError(st, "dr_chunked_plan")
     return bv.value, nprep.value
+
+
+def chunked_plan_ex(mode, BH: int, T: int, dk: int, dv: int, chained=False) -> tuple:
+    """(value channels per chain CTA, prep CTAs per head, segments per head) for bf16 inputs
+    of length T on the current device, or None when the chunked kernel does not apply. With
+    more than one segment the first two describe the launches over B*H*segments sequences."""
+    variant = MODES[mode] if isinstance(mode, str) else int(mode)
+    bv, nprep, nseg = ctypes.c_int(0), ctypes.c_int(0), ctypes.c_int(0)
+    flags = variant | DR_IN_BF16 | (DR_CHAINED if chained else 0)
+    st = lib().dr_chunked_plan_ex(flags, int(BH), int(T), int(dk), int(dv), ctypes.byref(bv),
+                                  ctypes.byref(nprep), ctypes.byref(nseg))
+    if st == DR_ERR_UNSUPPORTED:
+        return None
+    if st != DR_OK:
+        raise DrScanError(st, "dr_chunked_plan_ex")
+    return bv.value, nprep.value, nseg.value
+
+
+def segment_counters(device=None) -> tuple:
+    """(segmented scans, chained reruns after a failed hand-off check) on the device since
+    the library was loaded; waits for the device's work first."""
+    import torch
+
+    dev = device if device is not None else torch.device("cuda", torch.cuda.current_device())
+    with torch.cuda.device(dev):
+        scans, reruns = ctypes.c_ulonglong(0), ctypes.c_ulonglong(0)
+        st = lib().dr_segment_counters(ctypes.byref(scans), ctypes.byref(reruns))
+    if st != DR_OK:
+        raise DrScanError(st, "dr_segment_counters")
+    return scans.value, reruns.value
 
 
 def chunked_applies(mode, dtype_is_bf16: bool, dk: int, dv: int) -> bool:

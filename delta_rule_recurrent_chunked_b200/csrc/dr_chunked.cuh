@@ -251,13 +251,37 @@ __device__ __forceinline__ void group_sync(int gi, int nthreads) {
     asm volatile("bar.sync %0, %1;" ::"r"(1 + 2 * gi), "r"(nthreads) : "memory");
 }
 
+// Per-launch options of the segmented scan (all off in a plain launch):
+//   Ts         tokens from one sequence's start to the next in beta, gate, out and u_out (the
+//              K/Q/V tensor maps carry the same stride); T for a plain launch
+//   S_ckpt     when set, the state after the first ckpt_chunks chunks of each sequence is
+//              written there too ([seq, dv, dk] fp32, like S_final)
+//   expand     when set, a token whose step could grow a state difference (beta_t |k_t|^2 > 2,
+//              or a gate above 1) ORs 1 into *expand
+//   run_if     when set, the launch does nothing unless *run_if != 0 (every CTA returns first)
+struct ChunkSeg {
+    long Ts;
+    float* S_ckpt;
+    int ckpt_chunks;
+    int* expand;
+    const int* run_if;
+};
+
+// Per-device counts of segmented scans and of the chained reruns their checks asked for.
+__device__ unsigned long long g_seg_scans = 0, g_seg_reruns = 0;
+
 template <int MODE, int BV, bool SPLIT>
 __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
     const __grid_constant__ CUtensorMap tmV, const float* __restrict__ beta,
     const float* __restrict__ gate, const float* __restrict__ S0,
     __nv_bfloat16* __restrict__ out, float* __restrict__ S_final,
-    __nv_bfloat16* __restrict__ u_out, int T, int dv, int nprep) {
+    __nv_bfloat16* __restrict__ u_out, int T, int dv, int nprep, const ChunkSeg seg) {
+    // a conditional launch whose condition is off: every CTA leaves before any barrier
+    if (seg.run_if && *seg.run_if == 0) return;
+    if (seg.run_if && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
+        atomicAdd(&g_seg_reruns, 1ull);
+    const long Ts = seg.Ts;
     using L = ChunkLayout<MODE, BV, SPLIT>;
     constexpr bool kGdn = L::kGdn;  // scalar gate (Gated DeltaNet)
     constexpr bool kKda = MODE == DR_KDA;
@@ -391,12 +415,15 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 mbar_arrive(bar(B_KQ_FULL + s));
             }
             float* bg = reinterpret_cast<float*>(sm + L::BG + s * L::BG_B);
-            const float b0 = t0 + lane < T ? beta[bh * T + t0 + lane] : 0.f;
-            const float b1 = t0 + 32 + lane < T ? beta[bh * T + t0 + 32 + lane] : 0.f;
+            const float b0 = t0 + lane < T ? beta[bh * Ts + t0 + lane] : 0.f;
+            const float b1 = t0 + 32 + lane < T ? beta[bh * Ts + t0 + 32 + lane] : 0.f;
             if constexpr (kGdn) {
                 // g_t = sum of log alpha over the chunk's rows up to t (masked rows add 0)
-                float x0 = t0 + lane < T ? __logf(gate[bh * T + t0 + lane]) : 0.f;
-                float x1 = t0 + 32 + lane < T ? __logf(gate[bh * T + t0 + 32 + lane]) : 0.f;
+                const float a0 = t0 + lane < T ? gate[bh * Ts + t0 + lane] : 1.f;
+                const float a1 = t0 + 32 + lane < T ? gate[bh * Ts + t0 + 32 + lane] : 1.f;
+                if (seg.expand && (a0 > 1.f || a1 > 1.f)) atomicOr(seg.expand, 1);
+                float x0 = t0 + lane < T ? __logf(a0) : 0.f;
+                float x1 = t0 + 32 + lane < T ? __logf(a1) : 0.f;
 #pragma unroll
                 for (int off = 1; off < 32; off <<= 1) {
                     const float y0 = __shfl_up_sync(0xffffffffu, x0, off);
@@ -671,7 +698,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 for (int c16 = 0; c16 < LW; c16 += 16) tmem_ld16(trow + L::COL_D2 + cb + c16, d + c16);
                 tmem_wait_ld();
                 if (c * CK + r < T) {
-                    uint4* dst = reinterpret_cast<uint4*>(u_out + (bh * T + c * CK + r) * (long)dv + v0 + cb);
+                    uint4* dst = reinterpret_cast<uint4*>(u_out + (bh * Ts + c * CK + r) * (long)dv + v0 + cb);
 #pragma unroll
                     for (int i = 0; i < NV8; ++i) {
                         uint4 w;
@@ -760,6 +787,11 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
 #pragma unroll
                     for (int v = 0; v < HC; ++v) dst[(long)v * CDK] = sv[v];
                 }
+                if (seg.S_ckpt && c + 1 == seg.ckpt_chunks) {
+                    float* dst = seg.S_ckpt + (bh * dv + v0 + cb) * (long)CDK + r;
+#pragma unroll
+                    for (int v = 0; v < HC; ++v) dst[(long)v * CDK] = sv[v];
+                }
                 if constexpr (kGdn) {
                     if (!last) {
 #pragma unroll
@@ -790,7 +822,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     tc_fence_before();
                     mbar_arrive(bar(B_ODONE));
                     if (t < nvalid) {
-                        uint4* dst = reinterpret_cast<uint4*>(out + (bh * T + t0 + t) * (long)dv + v0 + cb);
+                        uint4* dst = reinterpret_cast<uint4*>(out + (bh * Ts + t0 + t) * (long)dv + v0 + cb);
 #pragma unroll
                         for (int i = 0; i < NV8; ++i) {
                             uint4 w;
@@ -930,7 +962,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                         uint32_t* wp = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
                         for (int e = 0; e < 8; ++e) wp[e] = pack_bf16(d[2 * e], d[2 * e + 1]);
-                        uint4* dst = reinterpret_cast<uint4*>(u_out + (bh * T + t0 + r) * (long)dv +
+                        uint4* dst = reinterpret_cast<uint4*>(u_out + (bh * Ts + t0 + r) * (long)dv +
                                                               v0 + c16);
                         dst[0] = w[0];
                         dst[1] = w[1];
@@ -952,7 +984,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     }
                     tmem_wait_ld();
                     if (t < nvalid) {
-                        uint4* dst = reinterpret_cast<uint4*>(out + (bh * T + t0 + t) * (long)dv +
+                        uint4* dst = reinterpret_cast<uint4*>(out + (bh * Ts + t0 + t) * (long)dv +
                                                               v0 + c0);
 #pragma unroll
                         for (int i = 0; i < PW / 8; ++i) {
@@ -972,6 +1004,9 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 float* dst = (c == nchunks - 1 && S_final)
                                  ? S_final + (bh * dv + v0) * (long)CDK + r
                                  : nullptr;
+                float* dck = (seg.S_ckpt && c + 1 == seg.ckpt_chunks)
+                                 ? seg.S_ckpt + (bh * dv + v0) * (long)CDK + r
+                                 : nullptr;
                 const float em = (kKda && c + 1 < nchunks) ? state_anchor(c + 1) : 1.f;
                 constexpr int HW = BV < 64 ? BV : 64;
 #pragma unroll
@@ -983,6 +1018,10 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     if (dst) {
 #pragma unroll
                         for (int v = 0; v < HW; ++v) dst[(long)(c0 + v) * CDK] = sv[v];
+                    }
+                    if (dck) {
+#pragma unroll
+                        for (int v = 0; v < HW; ++v) dck[(long)(c0 + v) * CDK] = sv[v];
                     }
                     if constexpr (kKda) {
 #pragma unroll
@@ -1061,7 +1100,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
                 const int t = 16 * kq4 + i;
-                gpf[i] = t < T ? *reinterpret_cast<const float2*>(chan + (bh * T + t) * (long)CDK + kc)
+                gpf[i] = t < T ? *reinterpret_cast<const float2*>(chan + (bh * Ts + t) * (long)CDK + kc)
                                : make_float2(1.f, 1.f);
             }
         }
@@ -1178,7 +1217,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
 #pragma unroll
                 for (int i = 0; i < 16; ++i) {
                     const int tn = (c + NGR * pSP) * CK + 16 * kq4 + i;
-                    gpf[i] = tn < T ? *reinterpret_cast<const float2*>(chan + (bh * T + tn) * (long)CDK + kc)
+                    gpf[i] = tn < T ? *reinterpret_cast<const float2*>(chan + (bh * Ts + tn) * (long)CDK + kc)
                                     : make_float2(1.f, 1.f);
                 }
             }
@@ -1219,6 +1258,14 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     }
                 }
                 tmem_wait_ld();
+                if (seg.expand && lq < 64 && (t >> 5) == hf) {
+                    // the step's transition diag(a)(I - beta k k^T) is non-expansive while
+                    // beta |k|^2 <= 2 (|k|^2 is the Gram's diagonal)
+                    float kk = 0.f;
+#pragma unroll
+                    for (int e = 0; e < 32; ++e) kk = (c32 + e == t) ? gr[e] : kk;
+                    if (bg[t] * kk > 2.f) atomicOr(seg.expand, 1);
+                }
 #pragma unroll
                 for (int e = 0; e < 32; ++e) {
                     const int i = c32 + e;
@@ -1437,13 +1484,14 @@ inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
     return fn;
 }
 
-// 3D map over a [BH, T, inner] row-major tensor, box {box_inner, 64 rows, 1}.
+// 3D map over BH sequences of T rows of `inner` elements, row-major, Ts rows from one
+// sequence's start to the next (Ts = T: a [BH, T, inner] tensor); box {box_inner, 64 rows, 1}.
 inline bool make_map_3d(CUtensorMap* m, const void* base, CUtensorMapDataType dt, int esize,
-                        long BH, int T, int inner, int box_inner, bool swizzle128) {
+                        long BH, int T, long Ts, int inner, int box_inner, bool swizzle128) {
     auto enc = tensor_map_encoder();
     if (!enc) return false;
     cuuint64_t dims[3] = {(cuuint64_t)inner, (cuuint64_t)T, (cuuint64_t)BH};
-    cuuint64_t strides[2] = {(cuuint64_t)inner * esize, (cuuint64_t)inner * esize * T};
+    cuuint64_t strides[2] = {(cuuint64_t)inner * esize, (cuuint64_t)inner * esize * Ts};
     cuuint32_t box[3] = {(cuuint32_t)box_inner, (cuuint32_t)CK, 1};
     cuuint32_t estr[3] = {1, 1, 1};
     CUresult r = enc(m, dt, 3, const_cast<void*>(base), dims, strides, box, estr,
@@ -1475,42 +1523,50 @@ struct ChunkArgs {
 // buffers and shape (the usual case in a loop) reuses it instead of encoding anew.
 struct MapCacheEntry {
     const void* base = nullptr;
-    long BH = 0;
+    long BH = 0, Ts = 0;
     int T = 0, inner = 0, box = 0;
     bool swz = false;
     int dev = -1;
     CUtensorMap map;
 };
 
-inline bool cached_map_3d(int slot, CUtensorMap* m, const void* base, long BH, int T, int inner,
-                          int box_inner, bool swizzle128) {
-    thread_local MapCacheEntry cache[8];
+inline bool cached_map_3d(int slot, CUtensorMap* m, const void* base, long BH, int T, long Ts,
+                          int inner, int box_inner, bool swizzle128) {
+    thread_local MapCacheEntry cache[16];
     int dev = -1;
     if (cudaGetDevice(&dev) != cudaSuccess) return false;
-    MapCacheEntry& e = cache[slot & 7];
-    if (e.base == base && e.BH == BH && e.T == T && e.inner == inner && e.box == box_inner &&
-        e.swz == swizzle128 && e.dev == dev) {
+    MapCacheEntry& e = cache[slot & 15];
+    if (e.base == base && e.BH == BH && e.T == T && e.Ts == Ts && e.inner == inner &&
+        e.box == box_inner && e.swz == swizzle128 && e.dev == dev) {
         *m = e.map;
         return true;
     }
-    if (!make_map_3d(&e.map, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, BH, T, inner, box_inner,
-                     swizzle128)) {
+    if (!make_map_3d(&e.map, base, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, BH, T, Ts, inner,
+                     box_inner, swizzle128)) {
         e.base = nullptr;
         return false;
     }
-    e.base = base, e.BH = BH, e.T = T, e.inner = inner, e.box = box_inner, e.swz = swizzle128;
+    e.base = base, e.BH = BH, e.T = T, e.Ts = Ts, e.inner = inner, e.box = box_inner;
+    e.swz = swizzle128;
     e.dev = dev;
     *m = e.map;
     return true;
 }
 
+// A plain launch: sequences back to back, no checkpoint, no checks, unconditional.
+inline ChunkSeg plain_seg(const ChunkArgs& a) { return ChunkSeg{(long)a.T, nullptr, 0, nullptr, nullptr}; }
+
+// `maps` picks the set of cached tensor-map slots (0, 1, 2: the launches of one segmented
+// scan keep their own maps).
 template <int MODE, int BV, bool SPLIT>
-int launch_chunked_bv(const ChunkArgs& a, int nprep, cudaStream_t stream) {
+int launch_chunked_bv(const ChunkArgs& a, int nprep, const ChunkSeg& sg, int maps,
+                      cudaStream_t stream) {
     using L = ChunkLayout<MODE, BV, SPLIT>;
     CUtensorMap mk, mq, mv;
-    if (!cached_map_3d(0, &mk, a.k, a.BH, a.T, CDK, 64, true) ||
-        !cached_map_3d(1, &mq, a.q, a.BH, a.T, CDK, 64, true) ||
-        !cached_map_3d(2, &mv, a.v, a.BH, a.T, a.dv, L::V_SWZ ? 64 : BV, L::V_SWZ))
+    const int m0 = 4 * maps;
+    if (!cached_map_3d(m0, &mk, a.k, a.BH, a.T, sg.Ts, CDK, 64, true) ||
+        !cached_map_3d(m0 + 1, &mq, a.q, a.BH, a.T, sg.Ts, CDK, 64, true) ||
+        !cached_map_3d(m0 + 2, &mv, a.v, a.BH, a.T, sg.Ts, a.dv, L::V_SWZ ? 64 : BV, L::V_SWZ))
         return DR_ERR_CUDA;
     const int smem = L::TOTAL + 1024;
     auto kern = dr_chunked_kernel<MODE, BV, SPLIT>;
@@ -1540,7 +1596,7 @@ int launch_chunked_bv(const ChunkArgs& a, int nprep, cudaStream_t stream) {
     cfg.numAttrs = split ? 1 : 0;
     if (cudaLaunchKernelEx(&cfg, kern, mk, mq, mv, a.beta, a.gate, a.S0,
                            static_cast<__nv_bfloat16*>(a.out), a.S_final,
-                           static_cast<__nv_bfloat16*>(a.u_out), a.T, a.dv, split) != cudaSuccess)
+                           static_cast<__nv_bfloat16*>(a.u_out), a.T, a.dv, split, sg) != cudaSuccess)
         return DR_ERR_CUDA;
     return cudaGetLastError() == cudaSuccess ? DR_OK : DR_ERR_CUDA;
 }
@@ -1616,33 +1672,170 @@ inline SplitPlan pick_split(int variant, long BH, int dv) {
     return plan;
 }
 
+// One launch with a given plan (nprep == 0: unsplit, value slice from pick_bv).
 template <int MODE>
-int launch_chunked_mode(const ChunkArgs& a, cudaStream_t stream) {
-    const SplitPlan plan = pick_split(MODE, a.BH, a.dv);
+int launch_chunked_plan(const ChunkArgs& a, const SplitPlan& plan, const ChunkSeg& sg, int maps,
+                        cudaStream_t stream) {
     if constexpr (MODE != DR_KDA) {
         if (plan.nprep > 0) {
             switch (plan.bv) {
                 case 16:
-                    return launch_chunked_bv<MODE, 16, true>(a, plan.nprep, stream);
+                    return launch_chunked_bv<MODE, 16, true>(a, plan.nprep, sg, maps, stream);
                 case 32:
-                    return launch_chunked_bv<MODE, 32, true>(a, plan.nprep, stream);
+                    return launch_chunked_bv<MODE, 32, true>(a, plan.nprep, sg, maps, stream);
                 case 64:
-                    return launch_chunked_bv<MODE, 64, true>(a, plan.nprep, stream);
+                    return launch_chunked_bv<MODE, 64, true>(a, plan.nprep, sg, maps, stream);
             }
             return DR_ERR_UNSUPPORTED;
         }
     }
     switch (pick_bv(MODE, a.BH, a.dv)) {
         case 16:
-            return launch_chunked_bv<MODE, 16, false>(a, 0, stream);
+            return launch_chunked_bv<MODE, 16, false>(a, 0, sg, maps, stream);
         case 32:
-            return launch_chunked_bv<MODE, 32, false>(a, 0, stream);
+            return launch_chunked_bv<MODE, 32, false>(a, 0, sg, maps, stream);
         case 64:
-            return launch_chunked_bv<MODE, 64, false>(a, 0, stream);
+            return launch_chunked_bv<MODE, 64, false>(a, 0, sg, maps, stream);
         case 128:
-            if constexpr (MODE == DR_KDA) return launch_chunked_bv<MODE, 128, false>(a, 0, stream);
+            if constexpr (MODE == DR_KDA)
+                return launch_chunked_bv<MODE, 128, false>(a, 0, sg, maps, stream);
     }
     return DR_ERR_UNSUPPORTED;
+}
+
+template <int MODE>
+int launch_chunked_mode(const ChunkArgs& a, cudaStream_t stream) {
+    return launch_chunked_plan<MODE>(a, pick_split(MODE, a.BH, a.dv), plain_seg(a), 0, stream);
+}
+
+// ---------------------------------------------------------------------------------------
+// Segmented scan (Gated DeltaNet, few heads, long sequences)
+//
+// With few heads the chained kernel leaves SMs idle and runs one chain of T/64 dependent
+// chunks per head. The segmented form cuts each head into G equal segments and runs them as
+// independent sequences:
+//   1. every segment from a zero state (segment 0 from S0): outputs, end states E, and the
+//      state Z after the first SEG_WINDOW chunks;
+//   2. the first SEG_WINDOW chunks of every segment again, from its true entering state
+//      (S0, or E of the segment before): exact outputs there, and the state X at the window's
+//      end;
+//   3. a check per segment: with the entering state known, X is the true state at the end of
+//      the window; the outputs after the window, computed from Z, are kept only if every
+//      value row of X - Z is at most SEG_EPS times the largest row norm of X. While every
+//      step's transition diag(a)(I - beta k k^T) is non-expansive (gate <= 1 and
+//      beta |k|^2 <= 2, checked by the kernel on every token), that difference never grows
+//      afterwards, so every later output and the end state move by at most that much.
+//      SEG_EPS = 2^-7 sits above the kernel's own rounding: its bf16 copy of the state
+//      rounds two nearly equal states apart by up to one bf16 step (2^-8 of an element), so
+//      two runs whose states agree to far below that still differ by up to about 2^-8 of the
+//      row norm (measured on B200: 0.3e-3 to 2.1e-3 under the Gated DeltaNet workload's
+//      gates; 2.8e-2 and more once the gate's log-mean is -6 or weaker, too little decay);
+//   4. when any check fails, a conditional launch of the chained kernel recomputes everything
+//      (it returns at once when the checks passed): the result is always the chained one to
+//      within SEG_EPS of the state's scale.
+// A gate strictly below 1 makes the difference decay by gamma_C per chunk, so with the
+// decays these models use the window's eight chunks shrink it far below the threshold (to
+// about 4e-8 of the row norm in fp64 for gates exp(-softplus(x)), x ~ N(-4, 1)).
+// ---------------------------------------------------------------------------------------
+constexpr int SEG_WINDOW = 8;        // chunks rerun from the true entering state
+constexpr int SEG_MIN_CHUNKS = 32;   // shortest segment (four windows)
+constexpr float SEG_EPS = 1.0f / 128.f;
+
+struct SegPlan {
+    int nseg = 1;     // segments per head (1: the chained kernel alone)
+    SplitPlan split;  // plan of the segment launches (BH * nseg sequences)
+};
+
+// Segments only pay where the chain is long: measured on B200 (Gated DeltaNet, dk = dv =
+// 128), a chained chunk step takes about 3.1 K cycles, a step of the segment launches (two
+// prep CTAs per cluster) about 3.65 K, and the window rerun, the checks and the conditional
+// launch add about 90 K cycles (46 us) whatever the length. In units of a chained step:
+//   chained   nch
+//   segmented 1.18 * nch / G + 29
+// The plan takes the G with the lowest estimate among those that keep every segment at
+// least SEG_MIN_CHUNKS long and let all B*H*G segments run at once as clusters of at least
+// two prep and two chain CTAs, and segments only when that estimate is below 0.9 * nch.
+inline SegPlan pick_segments(int variant, long BH, int T, int dv) {
+    SegPlan sp;
+    if (variant != DR_GDN || dv < 32 || T % CK != 0) return sp;
+    const int nch = T / CK;
+    double best = 0.9 * nch;
+    for (int G = 2; G <= nch / SEG_MIN_CHUNKS; ++G) {
+        if (nch % G) continue;
+        const long n = BH * G;
+        if (n * 4 > 148 || n > max_active_clusters(4)) break;
+        const SplitPlan p = pick_split(variant, n, dv);
+        if (p.nprep < 2) continue;
+        const double est = 1.18 * nch / G + 29.0;
+        if (est < best) {
+            best = est;
+            sp.nseg = G;
+            sp.split = p;
+        }
+    }
+    return sp;
+}
+
+// Step 3 of the segmented scan, one block per sequence s = head * G + segment. X, Z and E are
+// [BH * G, dv, CDK] fp32. The last segment's E is the head's final state (a failed check's
+// rerun overwrites it). Any failed check ORs 2 into *flag. A warp takes dv/16 value rows and
+// issues all their loads before it reduces.
+constexpr int SEG_CHECK_THREADS = 512;
+__global__ void __launch_bounds__(SEG_CHECK_THREADS) seg_handoff_check_kernel(
+    const float* __restrict__ X, const float* __restrict__ Z, const float* __restrict__ E,
+    float* __restrict__ S_final, int* __restrict__ flag, int G, int dv, float eps) {
+    constexpr int NW = SEG_CHECK_THREADS / 32, RMAX = CDK / NW;  // rows per warp, dv <= 128
+    const long s = blockIdx.x;
+    const int g = (int)(s % G);
+    const long head = s / G;
+    const long n = (long)dv * CDK;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    if (s == 0 && tid == 0) atomicAdd(&g_seg_scans, 1ull);
+    if (g == G - 1 && S_final) {
+        const float4* src = reinterpret_cast<const float4*>(E + s * n);
+        float4* dst = reinterpret_cast<float4*>(S_final + head * n);
+        for (long e = tid; e < n / 4; e += SEG_CHECK_THREADS) dst[e] = src[e];
+    }
+    if (g == 0) return;
+    __shared__ float red[2][NW];
+    float4 x[RMAX], z[RMAX];
+#pragma unroll
+    for (int i = 0; i < RMAX; ++i) {
+        const int row = warp + NW * i;
+        if (row < dv) {
+            x[i] = reinterpret_cast<const float4*>(X + s * n + (long)row * CDK)[lane];
+            z[i] = reinterpret_cast<const float4*>(Z + s * n + (long)row * CDK)[lane];
+        }
+    }
+    float dmax = 0.f, xmax = 0.f;
+#pragma unroll
+    for (int i = 0; i < RMAX; ++i) {
+        if (warp + NW * i >= dv) break;
+        float d2 = (x[i].x - z[i].x) * (x[i].x - z[i].x) + (x[i].y - z[i].y) * (x[i].y - z[i].y) +
+                   (x[i].z - z[i].z) * (x[i].z - z[i].z) + (x[i].w - z[i].w) * (x[i].w - z[i].w);
+        float x2 = x[i].x * x[i].x + x[i].y * x[i].y + x[i].z * x[i].z + x[i].w * x[i].w;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) {
+            d2 += __shfl_xor_sync(0xffffffffu, d2, off);
+            x2 += __shfl_xor_sync(0xffffffffu, x2, off);
+        }
+        // a NaN anywhere makes the comparison below fail
+        dmax = (d2 > dmax || d2 != d2) ? d2 : dmax;
+        xmax = fmaxf(xmax, x2);
+    }
+    if (lane == 0) {
+        red[0][warp] = dmax;
+        red[1][warp] = xmax;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        float d = 0.f, xm = 0.f;
+        for (int w = 0; w < NW; ++w) {
+            d = (red[0][w] > d || red[0][w] != red[0][w]) ? red[0][w] : d;
+            xm = fmaxf(xm, red[1][w]);
+        }
+        if (!(d <= eps * eps * xm)) atomicOr(flag, 2);
+    }
 }
 
 inline int launch_chunked(const ChunkArgs& a, int variant, cudaStream_t stream) {

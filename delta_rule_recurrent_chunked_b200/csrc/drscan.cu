@@ -210,9 +210,81 @@ int scratch_alloc(void** p, size_t bytes, cudaStream_t stream) {
     return cudaMallocFromPoolAsync(p, bytes, pool, stream) == cudaSuccess ? DR_OK : DR_ERR_CUDA;
 }
 
+// The segmented scan of Gated DeltaNet (steps in dr_chunked.cuh): scratch for four sets of
+// per-segment states and the check word, stream-ordered from the library's pool.
+int launch_gdn_segmented(const ChunkArgs& a, const SegPlan& sp, cudaStream_t stream) {
+    const int G = sp.nseg;
+    const long nseq = (long)a.BH * G;
+    const int Tseg = a.T / G;
+    const size_t sb = (size_t)a.dv * CDK * sizeof(float);  // one state
+    void* scratch = nullptr;
+    int rc = scratch_alloc(&scratch, 4 * nseq * sb + 256, stream);
+    if (rc != DR_OK) return rc;
+    float* E = static_cast<float*>(scratch);  // end state of each segment (zero start)
+    float* Z = E + nseq * (sb / 4);           // state after the window (zero start)
+    float* X = Z + nseq * (sb / 4);           // state after the window (true start)
+    float* Sin = X + nseq * (sb / 4);         // entering states
+    int* flag = reinterpret_cast<int*>(Sin + nseq * (sb / 4));
+    const size_t pitch = (size_t)G * sb;
+    auto ok = [](cudaError_t e) { return e == cudaSuccess ? DR_OK : DR_ERR_CUDA; };
+    rc = ok(cudaMemsetAsync(flag, 0, sizeof(int), stream));
+    // 1. every segment from zero, segment 0 from S0
+    ChunkArgs p1 = a;
+    p1.BH = (int)nseq;
+    p1.T = Tseg;
+    p1.S_final = E;
+    if (a.S0) {
+        if (rc == DR_OK) rc = ok(cudaMemsetAsync(Sin, 0, nseq * sb, stream));
+        if (rc == DR_OK)
+            rc = ok(cudaMemcpy2DAsync(Sin, pitch, a.S0, sb, sb, (size_t)a.BH,
+                                      cudaMemcpyDeviceToDevice, stream));
+        p1.S0 = Sin;
+    }
+    if (rc == DR_OK)
+        rc = launch_chunked_plan<DR_GDN>(p1, sp.split, ChunkSeg{Tseg, Z, SEG_WINDOW, flag, nullptr},
+                                         1, stream);
+    // 2. the window of every segment from its true entering state
+    if (rc == DR_OK) rc = ok(cudaMemcpyAsync(Sin + sb / 4, E, (nseq - 1) * sb,
+                                             cudaMemcpyDeviceToDevice, stream));
+    if (rc == DR_OK)
+        rc = a.S0 ? ok(cudaMemcpy2DAsync(Sin, pitch, a.S0, sb, sb, (size_t)a.BH,
+                                         cudaMemcpyDeviceToDevice, stream))
+                  : ok(cudaMemset2DAsync(Sin, pitch, 0, sb, (size_t)a.BH, stream));
+    ChunkArgs p2 = a;
+    p2.BH = (int)nseq;
+    p2.T = SEG_WINDOW * CK;
+    p2.S0 = Sin;
+    p2.S_final = X;
+    if (rc == DR_OK)
+        rc = launch_chunked_plan<DR_GDN>(p2, sp.split, ChunkSeg{Tseg, nullptr, 0, flag, nullptr},
+                                         2, stream);
+    // 3. the hand-off checks (and the final states)
+    if (rc == DR_OK) {
+        seg_handoff_check_kernel<<<(unsigned)nseq, SEG_CHECK_THREADS, 0, stream>>>(X, Z, E, a.S_final, flag, G,
+                                                                     a.dv, SEG_EPS);
+        rc = launch_status();
+    }
+    // 4. the chained scan, run only if a check failed
+    if (rc == DR_OK)
+        rc = launch_chunked_plan<DR_GDN>(a, pick_split(DR_GDN, a.BH, a.dv),
+                                         ChunkSeg{(long)a.T, nullptr, 0, nullptr, flag}, 3, stream);
+    if (cudaFreeAsync(scratch, stream) != cudaSuccess && rc == DR_OK) rc = DR_ERR_CUDA;
+    return rc;
+}
+
+// The chunked path: the segmented scan where its plan applies (Gated DeltaNet, few heads,
+// long sequences; not with DR_CHAINED), else one launch of the chained kernel.
+int launch_chunked_auto(const ChunkArgs& a, int variant, bool chained, cudaStream_t stream) {
+    if (!chained && variant == DR_GDN) {
+        const SegPlan sp = pick_segments(DR_GDN, a.BH, a.T, a.dv);
+        if (sp.nseg > 1) return launch_gdn_segmented(a, sp, stream);
+    }
+    return launch_chunked(a, variant, stream);
+}
+
 // Gated DeltaNet-2 on the chunked path: e and z into stream-ordered scratch, then the Gated
 // DeltaNet kernel (and its plan) on (q, e, z).
-int launch_gdn2_chunked(ChunkArgs a, int dk, cudaStream_t stream) {
+int launch_gdn2_chunked(ChunkArgs a, int dk, bool chained, cudaStream_t stream) {
     const long nk = (long)a.BH * a.T * dk, nv = (long)a.BH * a.T * a.dv;
     void* scratch = nullptr;
     int rc = scratch_alloc(&scratch, (size_t)(nk + nv) * sizeof(__nv_bfloat16), stream);
@@ -228,7 +300,7 @@ int launch_gdn2_chunked(ChunkArgs a, int dk, cudaStream_t stream) {
         a.k = e;
         a.v = z;
         a.erase = a.write = nullptr;
-        rc = launch_chunked(a, DR_GDN, stream);
+        rc = launch_chunked_auto(a, DR_GDN, chained, stream);
     }
     if (cudaFreeAsync(scratch, stream) != cudaSuccess && rc == DR_OK) rc = DR_ERR_CUDA;
     return rc;
@@ -442,7 +514,8 @@ int dr_scan_fwd_ex(const void* q, const void* k, const void* v, const float* bet
                    void* out, float* S_final, void* u_out, int B, int H, int T, int dk, int dv,
                    int mode, cudaStream_t stream) {
     const int variant = mode & DR_MODE_MASK;
-    if (mode & ~(DR_MODE_MASK | DR_IN_BF16 | DR_FORCE_SEQUENTIAL)) return DR_ERR_INVALID_ARG;
+    if (mode & ~(DR_MODE_MASK | DR_IN_BF16 | DR_FORCE_SEQUENTIAL | DR_CHAINED))
+        return DR_ERR_INVALID_ARG;
     if (variant > DR_GDN2) return DR_ERR_INVALID_ARG;
     if (B < 0 || H < 0 || T < 0 || dk <= 0 || dv <= 0) return DR_ERR_INVALID_ARG;
     const long BH = (long)B * (long)H;
@@ -469,8 +542,9 @@ int dr_scan_fwd_ex(const void* q, const void* k, const void* v, const float* bet
                 variant == DR_GDN2 ? erase : nullptr, variant == DR_GDN2 ? write : nullptr,
                 S0, out, S_final, u_out, (int)BH, T, dv};
     if (bf16 && !(mode & DR_FORCE_SEQUENTIAL) && chunked_supported(variant, dk, dv))
-        return variant == DR_GDN2 ? launch_gdn2_chunked(a, dk, stream)
-                                  : launch_chunked(a, variant, stream);
+        return variant == DR_GDN2
+                   ? launch_gdn2_chunked(a, dk, (mode & DR_CHAINED) != 0, stream)
+                   : launch_chunked_auto(a, variant, (mode & DR_CHAINED) != 0, stream);
     if (bf16) return dispatch_sequential<__nv_bfloat16>(a, dk, variant, stream);
     return dispatch_sequential<float>(a, dk, variant, stream);
 }
@@ -673,13 +747,40 @@ int dr_poll_error(cudaStream_t stream) {
     return status;
 }
 
+int dr_segment_counters(unsigned long long* scans, unsigned long long* reruns) {
+    if (!scans || !reruns) return DR_ERR_INVALID_ARG;
+    if (cudaDeviceSynchronize() != cudaSuccess ||
+        cudaMemcpyFromSymbol(scans, drscan::g_seg_scans, sizeof(*scans)) != cudaSuccess ||
+        cudaMemcpyFromSymbol(reruns, drscan::g_seg_reruns, sizeof(*reruns)) != cudaSuccess)
+        return DR_ERR_CUDA;
+    return DR_OK;
+}
+
+int dr_chunked_plan_ex(int mode, long long BH, int T, int dk, int dv, int* bv, int* nprep,
+                       int* nseg) {
+    if (!nseg || T < 0) return DR_ERR_INVALID_ARG;
+    *nseg = 1;
+    int rc = dr_chunked_plan(mode, BH, dk, dv, bv, nprep);
+    if (rc != DR_OK || (mode & DR_CHAINED)) return rc;
+    const int variant = mode & DR_MODE_MASK;
+    const drscan::SegPlan sp = drscan::pick_segments(
+        variant == DR_GDN2 ? DR_GDN : variant, (long)BH, T, dv);
+    if (sp.nseg > 1) {
+        *nseg = sp.nseg;
+        *bv = sp.split.bv;
+        *nprep = sp.split.nprep;
+    }
+    return DR_OK;
+}
+
 int dr_chunked_plan(int mode, long long BH, int dk, int dv, int* bv, int* nprep) {
     if ((mode & DR_MODE_MASK) > DR_GDN2) return DR_ERR_INVALID_ARG;
     if (!bv || !nprep) return DR_ERR_INVALID_ARG;
     *bv = 0;
     *nprep = 0;
     const int variant = mode & DR_MODE_MASK;
-    if (mode & ~(DR_MODE_MASK | DR_IN_BF16 | DR_FORCE_SEQUENTIAL)) return DR_ERR_INVALID_ARG;
+    if (mode & ~(DR_MODE_MASK | DR_IN_BF16 | DR_FORCE_SEQUENTIAL | DR_CHAINED))
+        return DR_ERR_INVALID_ARG;
     if (BH < 1 || BH > INT_MAX) return DR_ERR_INVALID_ARG;
     if (!(mode & DR_IN_BF16) || (mode & DR_FORCE_SEQUENTIAL) ||
         !drscan::chunked_supported(variant, dk, dv))

@@ -58,6 +58,9 @@ enum {
 /* Use the per-token kernel (fp32 state, CUDA cores) even where the chunked tensor-core
  * kernel applies. Same results up to rounding; slower. For testing and as a baseline. */
 #define DR_FORCE_SEQUENTIAL 0x200
+/* Keep Gated DeltaNet on the chained chunked kernel (one pass, one dependent chain of chunks
+ * per head) where dr_scan_fwd would take the segmented scan (see dr_scan_fwd). */
+#define DR_CHAINED 0x400
 
 /* status codes */
 enum {
@@ -87,7 +90,7 @@ enum {
  *   S0       [B,H,dv,dk] fp32 initial state, or NULL for zeros
  *   out      [B,H,T,dv] same type as v (written)
  *   S_final  [B,H,dv,dk] fp32 final state, or NULL to skip (written)
- *   mode     variant | DR_IN_BF16? | DR_FORCE_SEQUENTIAL?
+ *   mode     variant | DR_IN_BF16? | DR_FORCE_SEQUENTIAL? | DR_CHAINED?
  *
  * Supported: dk, dv in {32, 64, 128}; B, H >= 0 (B*H < 2^31); T >= 0 (T = 0 copies S0
  * into S_final). Every non-NULL pointer must be 16-byte aligned; when B*H*T == 0 the
@@ -102,6 +105,27 @@ enum {
  * (alpha about 0.07 per token, every token, every channel); a chunk with any channel
  * below that latches DR_ERR_GATE_RANGE, which dr_poll_error() reports (the outputs of
  * that call are then invalid: rerun it with DR_FORCE_SEQUENTIAL, which has no such limit).
+ *
+ * Segmented scan (Gated DeltaNet, bf16, dk = 128, T a multiple of 64, heads too few to
+ * fill the GPU; see dr_chunked_plan_ex). A sequence's state carries over from chunk to chunk,
+ * so the chained kernel runs T/64 dependent chunk steps per head ("Mechanisms, trade-offs and
+ * cross-layer routing of linear-attention architectures", Technical details: the state is
+ * decayed by alpha and corrected by the delta rule at every token). With few heads the call
+ * instead cuts each head into G equal segments and runs them at once: every segment from a
+ * zero state (the first from S0); then the first 8 chunks of every segment again from its
+ * true entering state (S0, or the end state of the segment before it); then, per segment, a
+ * check that the state at the end of those 8 chunks agrees with the zero-start one within
+ * 2^-7 of its largest value-row norm (row-wise 2-norm). A step whose transition
+ * diag(alpha)(I - beta k k^T) could grow a difference (alpha > 1 or beta |k|^2 > 2, both
+ * checked on every token) also fails the check. When every check passes, the later outputs
+ * and S_final stand: they differ from the chained scan's by at most that bound (times |q|),
+ * the size of the kernel's own rounding: its bf16 copy of the state already sets two runs
+ * from nearly equal states up to about 2^-8 of the row norm apart. When any check fails,
+ * the chained kernel reruns the
+ * whole call on the device (no host round trip), so the result is the chained one; a gate
+ * close to 1 everywhere makes the check fail and the call then costs about twice the
+ * chained kernel. The segmented scan takes 4 * B*H*G * dv*dk*4 bytes of scratch from the
+ * library's stream-ordered pool (DR_ERR_CUDA if it cannot be had). DR_CHAINED turns it off.
  *
  * Returns DR_OK or a negative status; on error nothing is launched.
  */
@@ -324,6 +348,24 @@ int dr_poll_error(cudaStream_t stream);
  * or unknown mode bits. Launches nothing; queries the device's cluster occupancy once.
  */
 int dr_chunked_plan(int mode, long long BH, int dk, int dv, int* bv, int* nprep);
+
+/*
+ * dr_chunked_plan with the sequence length: also reports, in *nseg, how many segments per
+ * head the segmented scan of dr_scan_fwd cuts each sequence into (1: the chained kernel
+ * alone; then *bv and *nprep are dr_chunked_plan's). With *nseg > 1, *bv and *nprep are
+ * the plan of the segment launches, which run B*H*(*nseg) sequences of T/(*nseg) tokens.
+ * Same return values as dr_chunked_plan; T < 0 is DR_ERR_INVALID_ARG.
+ */
+int dr_chunked_plan_ex(int mode, long long BH, int T, int dk, int dv, int* bv, int* nprep,
+                       int* nseg);
+
+/*
+ * How often the segmented scan ran on the current device since the library was loaded
+ * (*scans) and how many of those calls failed a hand-off check and were recomputed by the
+ * chained kernel (*reruns). Waits for the device to finish its work first. Returns DR_OK,
+ * DR_ERR_INVALID_ARG for null pointers, DR_ERR_CUDA if the device cannot be read.
+ */
+int dr_segment_counters(unsigned long long* scans, unsigned long long* reruns);
 
 /*
  * Test hook for the failure path: launches a one-block kernel on `stream` that waits on

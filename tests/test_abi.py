@@ -183,6 +183,30 @@ def test_chunked_plan_rejects_before_querying_the_device(lib):
         assert (bv.value, npr.value) == (0, 0)
 
 
+def test_chunked_plan_ex_rejects_before_querying_the_device(lib):
+    bv, npr, ns = ctypes.c_int(-1), ctypes.c_int(-1), ctypes.c_int(-1)
+    call = lambda mode, BH, T, dk, dv, c=ctypes.byref(ns): lib.dr_chunked_plan_ex(
+        mode, BH, T, dk, dv, ctypes.byref(bv), ctypes.byref(npr), c)
+    assert call(drs.DR_GDN | drs.DR_IN_BF16, 4, 4096, 128, 128, None) == drs.DR_ERR_INVALID_ARG
+    assert call(drs.DR_GDN | drs.DR_IN_BF16, 4, -1, 128, 128) == drs.DR_ERR_INVALID_ARG
+    assert call(drs.DR_GDN | drs.DR_IN_BF16, 0, 4096, 128, 128) == drs.DR_ERR_INVALID_ARG
+    assert call(drs.DR_GDN | drs.DR_IN_BF16 | 0x4000, 4, 4096, 128, 128) == drs.DR_ERR_INVALID_ARG
+    # the per-token kernel's requests: no plan, one segment
+    ns.value = -1
+    assert call(drs.DR_GDN | drs.DR_IN_BF16 | drs.DR_CHAINED | drs.DR_FORCE_SEQUENTIAL, 4, 4096,
+                128, 128) == drs.DR_ERR_UNSUPPORTED
+    assert (bv.value, npr.value, ns.value) == (0, 0, 1)
+
+
+def test_scan_accepts_the_chained_flag_and_rejects_unknown_bits(lib):
+    # B*H = 0: validated, nothing launched
+    P = ctypes.c_void_p
+    for mode, code in [(drs.DR_GDN | drs.DR_IN_BF16 | drs.DR_CHAINED, drs.DR_OK),
+                       (drs.DR_GDN | drs.DR_IN_BF16 | 0x800, drs.DR_ERR_INVALID_ARG)]:
+        assert lib.dr_scan_fwd(None, None, None, None, None, None, None, None, 0, 4, 64, 128,
+                               128, mode, None) == code
+
+
 def test_product_path_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(drs, "LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(drs, "_lib", None)
