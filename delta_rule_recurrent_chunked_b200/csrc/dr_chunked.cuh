@@ -259,12 +259,18 @@ __device__ __forceinline__ void group_sync(int gi, int nthreads) {
 //   expand     when set, a token whose step could grow a state difference (beta_t |k_t|^2 > 2,
 //              or a gate above 1) ORs 1 into *expand
 //   run_if     when set, the launch does nothing unless *run_if != 0 (every CTA returns first)
+//   G, ext     G > 1: sequence bh is segment bh % G of head bh / G (T tokens each, Ts = T);
+//              every segment but the last runs on for ext more tokens (a multiple of 64) into
+//              the next one, whose outputs there it writes, and every segment but the first
+//              writes no output for its own first ext tokens; S0 is [heads, dv, dk] and enters
+//              segment 0 only (the others start from zero)
 struct ChunkSeg {
     long Ts;
     float* S_ckpt;
     int ckpt_chunks;
     int* expand;
     const int* run_if;
+    int G, ext;
 };
 
 // Per-device counts of segmented scans and of the chained reruns their checks asked for.
@@ -276,12 +282,18 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
     const __grid_constant__ CUtensorMap tmV, const float* __restrict__ beta,
     const float* __restrict__ gate, const float* __restrict__ S0,
     __nv_bfloat16* __restrict__ out, float* __restrict__ S_final,
-    __nv_bfloat16* __restrict__ u_out, int T, int dv, int nprep, const ChunkSeg seg) {
+    __nv_bfloat16* __restrict__ u_out, int T_seq, int dv, int nprep, const ChunkSeg seg) {
     // a conditional launch whose condition is off: every CTA leaves before any barrier
     if (seg.run_if && *seg.run_if == 0) return;
     if (seg.run_if && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
         atomicAdd(&g_seg_reruns, 1ull);
     const long Ts = seg.Ts;
+    const int gseg = seg.G > 1 ? (int)(blockIdx.x % seg.G) : 0;
+    const int T = T_seq + ((seg.G > 1 && gseg < seg.G - 1) ? seg.ext : 0);  // tokens this CTA runs
+    const int cskip = (seg.G > 1 && gseg > 0) ? seg.ext / CK : 0;  // chunks whose outputs it leaves
+    const float* S0q = !S0          ? nullptr
+                       : seg.G > 1 ? (gseg == 0 ? S0 + (long)(blockIdx.x / seg.G) * dv * CDK : nullptr)
+                                   : S0 + (long)blockIdx.x * dv * CDK;
     using L = ChunkLayout<MODE, BV, SPLIT>;
     constexpr bool kGdn = L::kGdn;  // scalar gate (Gated DeltaNet)
     constexpr bool kKda = MODE == DR_KDA;
@@ -660,7 +672,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 mbar_arrive(bar(B_SFREE + 0));  // this thread is done reading slot 0
             }
             if (active) {
-                const float* src = S0 ? S0 + (bh * dv + v0 + cb) * (long)CDK + r : nullptr;
+                const float* src = S0q ? S0q + (v0 + cb) * (long)CDK + r : nullptr;
                 float sv[LW];
 #pragma unroll
                 for (int v = 0; v < LW; ++v) sv[v] = (src && v < HC) ? src[(long)v * CDK] : 0.f;
@@ -697,7 +709,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
 #pragma unroll
                 for (int c16 = 0; c16 < LW; c16 += 16) tmem_ld16(trow + L::COL_D2 + cb + c16, d + c16);
                 tmem_wait_ld();
-                if (c * CK + r < T) {
+                if (c * CK + r < T && c >= cskip) {
                     uint4* dst = reinterpret_cast<uint4*>(u_out + (bh * Ts + c * CK + r) * (long)dv + v0 + cb);
 #pragma unroll
                     for (int i = 0; i < NV8; ++i) {
@@ -821,7 +833,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     tmem_wait_ld();
                     tc_fence_before();
                     mbar_arrive(bar(B_ODONE));
-                    if (t < nvalid) {
+                    if (t < nvalid && c >= cskip) {
                         uint4* dst = reinterpret_cast<uint4*>(out + (bh * Ts + t0 + t) * (long)dv + v0 + cb);
 #pragma unroll
                         for (int i = 0; i < NV8; ++i) {
@@ -857,7 +869,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
             }
         };
         {
-            const float* src = S0 ? S0 + (bh * dv + v0) * (long)CDK + r : nullptr;
+            const float* src = S0q ? S0q + (long)v0 * CDK + r : nullptr;
             const float em = state_anchor(0);
 #pragma unroll
             for (int c16 = 0; c16 < L::NB; c16 += 16) {
@@ -957,7 +969,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     float d[16];
                     tmem_ld16(trow + L::COL_D2 + c16, d);
                     tmem_wait_ld();
-                    if (r < nvalid) {
+                    if (r < nvalid && c >= cskip) {
                         uint4 w[2];
                         uint32_t* wp = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
@@ -983,7 +995,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                         tmem_ld16(trow + L::COL_D2 + c0 + c16, d + c16);
                     }
                     tmem_wait_ld();
-                    if (t < nvalid) {
+                    if (t < nvalid && c >= cskip) {
                         uint4* dst = reinterpret_cast<uint4*>(out + (bh * Ts + t0 + t) * (long)dv +
                                                               v0 + c0);
 #pragma unroll
@@ -1554,7 +1566,9 @@ inline bool cached_map_3d(int slot, CUtensorMap* m, const void* base, long BH, i
 }
 
 // A plain launch: sequences back to back, no checkpoint, no checks, unconditional.
-inline ChunkSeg plain_seg(const ChunkArgs& a) { return ChunkSeg{(long)a.T, nullptr, 0, nullptr, nullptr}; }
+inline ChunkSeg plain_seg(const ChunkArgs& a) {
+    return ChunkSeg{(long)a.T, nullptr, 0, nullptr, nullptr, 0, 0};
+}
 
 // `maps` picks the set of cached tensor-map slots (0, 1, 2: the launches of one segmented
 // scan keep their own maps).
@@ -1564,9 +1578,10 @@ int launch_chunked_bv(const ChunkArgs& a, int nprep, const ChunkSeg& sg, int map
     using L = ChunkLayout<MODE, BV, SPLIT>;
     CUtensorMap mk, mq, mv;
     const int m0 = 4 * maps;
-    if (!cached_map_3d(m0, &mk, a.k, a.BH, a.T, sg.Ts, CDK, 64, true) ||
-        !cached_map_3d(m0 + 1, &mq, a.q, a.BH, a.T, sg.Ts, CDK, 64, true) ||
-        !cached_map_3d(m0 + 2, &mv, a.v, a.BH, a.T, sg.Ts, a.dv, L::V_SWZ ? 64 : BV, L::V_SWZ))
+    const int rows = a.T + (sg.G > 1 ? sg.ext : 0);  // tokens one sequence may read
+    if (!cached_map_3d(m0, &mk, a.k, a.BH, rows, sg.Ts, CDK, 64, true) ||
+        !cached_map_3d(m0 + 1, &mq, a.q, a.BH, rows, sg.Ts, CDK, 64, true) ||
+        !cached_map_3d(m0 + 2, &mv, a.v, a.BH, rows, sg.Ts, a.dv, L::V_SWZ ? 64 : BV, L::V_SWZ))
         return DR_ERR_CUDA;
     const int smem = L::TOTAL + 1024;
     auto kern = dr_chunked_kernel<MODE, BV, SPLIT>;
@@ -1712,46 +1727,48 @@ int launch_chunked_mode(const ChunkArgs& a, cudaStream_t stream) {
 // Segmented scan (Gated DeltaNet, few heads, long sequences)
 //
 // With few heads the chained kernel leaves SMs idle and runs one chain of T/64 dependent
-// chunks per head. The segmented form cuts each head into G equal segments and runs them as
-// independent sequences:
-//   1. every segment from a zero state (segment 0 from S0): outputs, end states E, and the
-//      state Z after the first SEG_WINDOW chunks;
-//   2. the first SEG_WINDOW chunks of every segment again, from its true entering state
-//      (S0, or E of the segment before): exact outputs there, and the state X at the window's
-//      end;
-//   3. a check per segment: with the entering state known, X is the true state at the end of
-//      the window; the outputs after the window, computed from Z, are kept only if every
-//      value row of X - Z is at most SEG_EPS times the largest row norm of X. While every
-//      step's transition diag(a)(I - beta k k^T) is non-expansive (gate <= 1 and
-//      beta |k|^2 <= 2, checked by the kernel on every token), that difference never grows
-//      afterwards, so every later output and the end state move by at most that much.
-//      SEG_EPS = 2^-7 sits above the kernel's own rounding: its bf16 copy of the state
-//      rounds two nearly equal states apart by up to one bf16 step (2^-8 of an element), so
-//      two runs whose states agree to far below that still differ by up to about 2^-8 of the
-//      row norm (measured on B200: 0.3e-3 to 2.1e-3 under the Gated DeltaNet workload's
-//      gates; 2.8e-2 and more once the gate's log-mean is -6 or weaker, too little decay);
-//   4. when any check fails, a conditional launch of the chained kernel recomputes everything
+// chunks per head. The segmented form cuts each head into G equal segments and runs them in
+// one launch as independent sequences:
+//   1. segment g starts from a zero state (segment 0 from S0) and writes its outputs, except
+//      for its first SEG_WINDOW chunks when g > 0; it records its state Z after those chunks.
+//      Every segment but the last then runs SEG_WINDOW chunks on into the next segment,
+//      carrying its state, and writes the outputs there: the next segment's window is thus
+//      computed from the state that segment g reached, and X, the state at the end, is that
+//      same point once more, reached through the segments before;
+//   2. a check per boundary: the outputs of segment g after its window, computed from Z_g,
+//      are kept only if every value row of X_{g-1} - Z_g is at most SEG_EPS times the
+//      largest row norm of X_{g-1}. While every step's transition diag(a)(I - beta k k^T) is
+//      non-expansive (gate <= 1 and beta |k|^2 <= 2, checked by the kernel on every token),
+//      that difference never grows afterwards, so every later output and the end state move
+//      by at most that much. By induction over the segments, X_{g-1} is itself the chained
+//      state to within the same bound. SEG_EPS = 2^-7 sits above the kernel's own rounding:
+//      its bf16 copy of the state rounds two nearly equal states apart by up to one bf16
+//      step (2^-8 of an element), so two runs whose states agree to far below that still
+//      differ by up to about 2^-8 of the row norm (measured on B200: 0.3e-3 to 2.1e-3 under
+//      the Gated DeltaNet workload's gates; 2.8e-2 and more once the gate's log-mean is -6 or
+//      weaker, too little decay);
+//   3. when any check fails, a conditional launch of the chained kernel recomputes everything
 //      (it returns at once when the checks passed): the result is always the chained one to
 //      within SEG_EPS of the state's scale.
 // A gate strictly below 1 makes the difference decay by gamma_C per chunk, so with the
 // decays these models use the window's eight chunks shrink it far below the threshold (to
 // about 4e-8 of the row norm in fp64 for gates exp(-softplus(x)), x ~ N(-4, 1)).
 // ---------------------------------------------------------------------------------------
-constexpr int SEG_WINDOW = 8;        // chunks rerun from the true entering state
+constexpr int SEG_WINDOW = 8;        // chunks of overlap between consecutive segments
 constexpr int SEG_MIN_CHUNKS = 32;   // shortest segment (four windows)
 constexpr float SEG_EPS = 1.0f / 128.f;
 
 struct SegPlan {
     int nseg = 1;     // segments per head (1: the chained kernel alone)
-    SplitPlan split;  // plan of the segment launches (BH * nseg sequences)
+    SplitPlan split;  // plan of the segment launch (BH * nseg sequences)
 };
 
-// Segments only pay where the chain is long: measured on B200 (Gated DeltaNet, dk = dv =
-// 128), a chained chunk step takes about 3.1 K cycles, a step of the segment launches (two
-// prep CTAs per cluster) about 3.65 K, and the window rerun, the checks and the conditional
-// launch add about 90 K cycles (46 us) whatever the length. In units of a chained step:
+// Segments pay where the chain is long: measured on B200 (Gated DeltaNet, dk = dv = 128), a
+// chained chunk step takes about 3.1 K cycles and a step of the segment launch (two prep
+// CTAs per cluster) about 3.65 K; the check and the conditional launch add about 8 us. In
+// units of a chained step:
 //   chained   nch
-//   segmented 1.18 * nch / G + 29
+//   segmented 1.18 * (nch / G + SEG_WINDOW) + 5
 // The plan takes the G with the lowest estimate among those that keep every segment at
 // least SEG_MIN_CHUNKS long and let all B*H*G segments run at once as clusters of at least
 // two prep and two chain CTAs, and segments only when that estimate is below 0.9 * nch.
@@ -1766,7 +1783,7 @@ inline SegPlan pick_segments(int variant, long BH, int T, int dv) {
         if (n * 4 > 148 || n > max_active_clusters(4)) break;
         const SplitPlan p = pick_split(variant, n, dv);
         if (p.nprep < 2) continue;
-        const double est = 1.18 * nch / G + 29.0;
+        const double est = 1.18 * (nch / G + SEG_WINDOW) + 5.0;
         if (est < best) {
             best = est;
             sp.nseg = G;
@@ -1776,14 +1793,16 @@ inline SegPlan pick_segments(int variant, long BH, int T, int dv) {
     return sp;
 }
 
-// Step 3 of the segmented scan, one block per sequence s = head * G + segment. X, Z and E are
-// [BH * G, dv, CDK] fp32. The last segment's E is the head's final state (a failed check's
-// rerun overwrites it). Any failed check ORs 2 into *flag. A warp takes dv/16 value rows and
-// issues all their loads before it reduces.
+// Step 2 of the segmented scan, one block per sequence s = head * G + segment. X and Z are
+// [BH * G, dv, CDK] fp32: X[s] is where segment s's run ended (the state after the window of
+// segment s + 1, or the head's final state for the last segment), Z[s] the zero-start state
+// after segment s's own window. The last segment's X is the head's final state (a failed
+// check's rerun overwrites it). Any failed check ORs 2 into *flag. A warp takes dv/16 value
+// rows and issues all their loads before it reduces.
 constexpr int SEG_CHECK_THREADS = 512;
 __global__ void __launch_bounds__(SEG_CHECK_THREADS) seg_handoff_check_kernel(
-    const float* __restrict__ X, const float* __restrict__ Z, const float* __restrict__ E,
-    float* __restrict__ S_final, int* __restrict__ flag, int G, int dv, float eps) {
+    const float* __restrict__ X, const float* __restrict__ Z, float* __restrict__ S_final,
+    int* __restrict__ flag, int G, int dv, float eps) {
     constexpr int NW = SEG_CHECK_THREADS / 32, RMAX = CDK / NW;  // rows per warp, dv <= 128
     const long s = blockIdx.x;
     const int g = (int)(s % G);
@@ -1792,19 +1811,21 @@ __global__ void __launch_bounds__(SEG_CHECK_THREADS) seg_handoff_check_kernel(
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     if (s == 0 && tid == 0) atomicAdd(&g_seg_scans, 1ull);
     if (g == G - 1 && S_final) {
-        const float4* src = reinterpret_cast<const float4*>(E + s * n);
+        const float4* src = reinterpret_cast<const float4*>(X + s * n);
         float4* dst = reinterpret_cast<float4*>(S_final + head * n);
         for (long e = tid; e < n / 4; e += SEG_CHECK_THREADS) dst[e] = src[e];
     }
     if (g == 0) return;
+    const float* xs = X + (s - 1) * n;  // the true state after segment s's window
+    const float* zs = Z + s * n;
     __shared__ float red[2][NW];
     float4 x[RMAX], z[RMAX];
 #pragma unroll
     for (int i = 0; i < RMAX; ++i) {
         const int row = warp + NW * i;
         if (row < dv) {
-            x[i] = reinterpret_cast<const float4*>(X + s * n + (long)row * CDK)[lane];
-            z[i] = reinterpret_cast<const float4*>(Z + s * n + (long)row * CDK)[lane];
+            x[i] = reinterpret_cast<const float4*>(xs + (long)row * CDK)[lane];
+            z[i] = reinterpret_cast<const float4*>(zs + (long)row * CDK)[lane];
         }
     }
     float dmax = 0.f, xmax = 0.f;

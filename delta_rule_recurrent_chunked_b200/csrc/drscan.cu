@@ -210,64 +210,39 @@ int scratch_alloc(void** p, size_t bytes, cudaStream_t stream) {
     return cudaMallocFromPoolAsync(p, bytes, pool, stream) == cudaSuccess ? DR_OK : DR_ERR_CUDA;
 }
 
-// The segmented scan of Gated DeltaNet (steps in dr_chunked.cuh): scratch for four sets of
+// The segmented scan of Gated DeltaNet (steps in dr_chunked.cuh): scratch for two sets of
 // per-segment states and the check word, stream-ordered from the library's pool.
 int launch_gdn_segmented(const ChunkArgs& a, const SegPlan& sp, cudaStream_t stream) {
     const int G = sp.nseg;
     const long nseq = (long)a.BH * G;
-    const int Tseg = a.T / G;
-    const size_t sb = (size_t)a.dv * CDK * sizeof(float);  // one state
+    const size_t sn = (size_t)a.dv * CDK;  // floats per state
     void* scratch = nullptr;
-    int rc = scratch_alloc(&scratch, 4 * nseq * sb + 256, stream);
+    int rc = scratch_alloc(&scratch, 2 * nseq * sn * sizeof(float) + 256, stream);
     if (rc != DR_OK) return rc;
-    float* E = static_cast<float*>(scratch);  // end state of each segment (zero start)
-    float* Z = E + nseq * (sb / 4);           // state after the window (zero start)
-    float* X = Z + nseq * (sb / 4);           // state after the window (true start)
-    float* Sin = X + nseq * (sb / 4);         // entering states
-    int* flag = reinterpret_cast<int*>(Sin + nseq * (sb / 4));
-    const size_t pitch = (size_t)G * sb;
-    auto ok = [](cudaError_t e) { return e == cudaSuccess ? DR_OK : DR_ERR_CUDA; };
-    rc = ok(cudaMemsetAsync(flag, 0, sizeof(int), stream));
-    // 1. every segment from zero, segment 0 from S0
-    ChunkArgs p1 = a;
-    p1.BH = (int)nseq;
-    p1.T = Tseg;
-    p1.S_final = E;
-    if (a.S0) {
-        if (rc == DR_OK) rc = ok(cudaMemsetAsync(Sin, 0, nseq * sb, stream));
-        if (rc == DR_OK)
-            rc = ok(cudaMemcpy2DAsync(Sin, pitch, a.S0, sb, sb, (size_t)a.BH,
-                                      cudaMemcpyDeviceToDevice, stream));
-        p1.S0 = Sin;
-    }
+    float* X = static_cast<float*>(scratch);  // end state of each segment's run
+    float* Z = X + nseq * sn;                 // zero-start state after the window
+    int* flag = reinterpret_cast<int*>(Z + nseq * sn);
+    rc = cudaMemsetAsync(flag, 0, sizeof(int), stream) == cudaSuccess ? DR_OK : DR_ERR_CUDA;
+    // 1. all segments at once, each but the last running on through the next one's window
+    ChunkArgs p = a;
+    p.BH = (int)nseq;
+    p.T = a.T / G;
+    p.S_final = X;
     if (rc == DR_OK)
-        rc = launch_chunked_plan<DR_GDN>(p1, sp.split, ChunkSeg{Tseg, Z, SEG_WINDOW, flag, nullptr},
-                                         1, stream);
-    // 2. the window of every segment from its true entering state
-    if (rc == DR_OK) rc = ok(cudaMemcpyAsync(Sin + sb / 4, E, (nseq - 1) * sb,
-                                             cudaMemcpyDeviceToDevice, stream));
-    if (rc == DR_OK)
-        rc = a.S0 ? ok(cudaMemcpy2DAsync(Sin, pitch, a.S0, sb, sb, (size_t)a.BH,
-                                         cudaMemcpyDeviceToDevice, stream))
-                  : ok(cudaMemset2DAsync(Sin, pitch, 0, sb, (size_t)a.BH, stream));
-    ChunkArgs p2 = a;
-    p2.BH = (int)nseq;
-    p2.T = SEG_WINDOW * CK;
-    p2.S0 = Sin;
-    p2.S_final = X;
-    if (rc == DR_OK)
-        rc = launch_chunked_plan<DR_GDN>(p2, sp.split, ChunkSeg{Tseg, nullptr, 0, flag, nullptr},
-                                         2, stream);
-    // 3. the hand-off checks (and the final states)
+        rc = launch_chunked_plan<DR_GDN>(
+            p, sp.split, ChunkSeg{(long)p.T, Z, SEG_WINDOW, flag, nullptr, G, SEG_WINDOW * CK}, 1,
+            stream);
+    // 2. the hand-off checks (and the final states)
     if (rc == DR_OK) {
-        seg_handoff_check_kernel<<<(unsigned)nseq, SEG_CHECK_THREADS, 0, stream>>>(X, Z, E, a.S_final, flag, G,
-                                                                     a.dv, SEG_EPS);
+        seg_handoff_check_kernel<<<(unsigned)nseq, SEG_CHECK_THREADS, 0, stream>>>(
+            X, Z, a.S_final, flag, G, a.dv, SEG_EPS);
         rc = launch_status();
     }
-    // 4. the chained scan, run only if a check failed
+    // 3. the chained scan, run only if a check failed
     if (rc == DR_OK)
-        rc = launch_chunked_plan<DR_GDN>(a, pick_split(DR_GDN, a.BH, a.dv),
-                                         ChunkSeg{(long)a.T, nullptr, 0, nullptr, flag}, 3, stream);
+        rc = launch_chunked_plan<DR_GDN>(
+            a, pick_split(DR_GDN, a.BH, a.dv),
+            ChunkSeg{(long)a.T, nullptr, 0, nullptr, flag, 0, 0}, 2, stream);
     if (cudaFreeAsync(scratch, stream) != cudaSuccess && rc == DR_OK) rc = DR_ERR_CUDA;
     return rc;
 }

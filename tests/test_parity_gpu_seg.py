@@ -1,9 +1,10 @@
 """GPU parity of the segmented Gated DeltaNet scan (few heads, long sequences).
 
-dr_scan_fwd cuts each head into segments that run at once from zero states, reruns the first
-eight chunks of every segment from its true entering state, and keeps the zero-start outputs
-after that window only where a device-side check shows the two states agree (and no token's
-step could grow a difference); otherwise the chained kernel reruns the call. These tests pin
+dr_scan_fwd cuts each head into segments that run at once from zero states; every segment
+but the last runs eight chunks on into the next one, carrying its state, and writes the
+outputs there. The zero-start outputs after that window are kept only where a device-side
+check shows the two states at the window's end agree (and no token's step could grow a
+difference); otherwise the chained kernel reruns the call. These tests pin
 both outcomes against the fp64 oracle at the bf16 tolerance (2e-2, max|x - y| / max|y|), and
 pin the fallback against the chained kernel bit for bit.
 """
@@ -42,16 +43,15 @@ def _scan(dev, mode, chained=False, want_u=False):
 def test_plan_segments_only_gated_deltanet_with_few_heads():
     plan = drs.chunked_plan_ex
     assert plan("gdn", 16, 8192, 128, 128) == (64, 2, 2)
+    assert plan("gdn", 16, 4096, 128, 128)[2] == 2
     assert plan("gdn", 16, 32768, 128, 128)[2] == 2
     assert plan("gdn", 2, 32768, 128, 128)[2] == 16
     assert plan("gdn", 1, 8192, 128, 128)[2] == 4
     assert plan("gdn2", 16, 8192, 128, 128)[2] == 2
-    # the chained plan is kept when asked for, when the heads already fill the GPU, where the
-    # chain is too short for the segments' fixed cost to pay (64 chunks), for a T that is not
-    # a multiple of 64 or too short to cut, and for the other variants
+    # the chained plan is kept when asked for, when the heads already fill the GPU, for a T
+    # that is not a multiple of 64 or too short to cut in two, and for the other variants
     assert plan("gdn", 16, 8192, 128, 128, chained=True) == drs.chunked_plan("gdn", 16, 128, 128) + (1,)
     assert plan("gdn", 32, 32768, 128, 128)[2] == 1
-    assert plan("gdn", 16, 4096, 128, 128)[2] == 1
     assert plan("gdn", 16, 4096 + 64, 128, 128)[2] == 1
     assert plan("gdn", 2, 4095, 128, 128)[2] == 1
     assert plan("gdn", 2, 4096 - 64, 128, 128)[2] == 1
@@ -60,7 +60,7 @@ def test_plan_segments_only_gated_deltanet_with_few_heads():
 
 
 @pytest.mark.parametrize("B,H,T,s0", [(1, 2, 8192, True), (1, 2, 16384, False), (2, 3, 8192, True),
-                                      (1, 1, 16384, True)])
+                                      (1, 1, 16384, True), (1, 16, 4096, True)])
 def test_segmented_gdn_matches_oracle(oracle, B, H, T, s0):
     w = wl.DRWorkload("gdn_seg", B, H, T, 128, 128, wl.GDN, "bf16", s0_std=0.1 if s0 else 0.0)
     assert drs.chunked_plan_ex("gdn", B * H, T, 128, 128)[2] > 1
