@@ -486,9 +486,9 @@ def measure_dr(args, w, world, rank, local, device, K, cpu_target):
     # Gated DeltaNet-2 on the chunked path is two launches per call: the pre-scaling of k and
     # v by the erase and write gates, then the chunked kernel; the roofline is the call's
     prescaled = chunked and w.mode == wl.GDN2
-    # the segmented scan (few heads, long sequences) is four launches of this library per
-    # call: the zero-start pass over all segments, the window rerun, the hand-off check and
-    # the chained kernel's conditional launch (which returns at once when the checks pass)
+    # the segmented scan (few heads, long sequences) is three launches of this library per
+    # call: all segments at once, the hand-off check and the chained kernel's conditional
+    # launch (which returns at once when the checks pass)
     nseg = drs.chunked_plan_ex(mode, w.B * w.H, w.T, w.dk, w.dv)[2] if chunked else 1
     kname = "chunked" if nseg == 1 else f"segmented chunked ({nseg} segments per head)"
     config = dict(workload_config(w, world), l2=l2_note(nsets, nbytes, needs_flush),
@@ -500,12 +500,13 @@ def measure_dr(args, w, world, rank, local, device, K, cpu_target):
         config["segmented"] = {"calls": seg1[0] - seg0[0], "chained_reruns": seg1[1] - seg0[1]}
     line = base_line(args, w, world, K, total_ms_max, clk, e2e_ms, e2e["h2d"], e2e["d2h"], config,
                      w.dtype, t_wall,
-                     launches_per_step=(1 if prescaled else 0) + (4 if nseg > 1 else 1))
+                     launches_per_step=(1 if prescaled else 0) + (3 if nseg > 1 else 1))
     line["roofline"] = {
         "bound": "hbm", "achieved": achieved, "peak": peaks["hbm_gbs"], "unit": "GB/s",
         "frac": achieved / peaks["hbm_gbs"],
+        # a call of several launches (pre-scaling, segments) is keyed by both sources
         "traffic": (NCU_TRAFFIC.get((w.name, kernel_source_sha("dr_chunked.cuh", "drscan.cu")))
-                    if prescaled else NCU_TRAFFIC.get((w.name, kernel_source_sha()))
+                    if prescaled or nseg > 1 else NCU_TRAFFIC.get((w.name, kernel_source_sha()))
                     if chunked else None),
         "peak_source": f"{peak_src} hbm_gbs", "bytes_per_launch": nbytes,
         "launch_ms": launch_ms, "tensor_tflops": tflops,
