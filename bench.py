@@ -140,15 +140,18 @@ def aggregate_value(world: int, head_tokens: int, steps: int, total_ms_max: floa
 
 # DRAM traffic (dram__bytes_read.sum + dram__bytes_write.sum) per launch from one ncu capture,
 # keyed by workload and the sha256 prefix of the timed kernel's source (dr_chunked.cuh;
-# dr_chunked.cuh and drscan.cu for Gated DeltaNet-2's two kernels; dr_decode.cuh for the
-# decode workload; loglinear.cuh for log-linear attention) at capture time; a changed source
-# reports null. Summaries with the commands are under profiles/.
+# dr_chunked.cuh and drscan.cu for Gated DeltaNet-2's two kernels and for the segmented
+# scan's three launches, summed per call; dr_decode.cuh for the decode workload;
+# loglinear.cuh for log-linear attention) at capture time; a changed source reports null.
+# Summaries with the commands are under profiles/.
 NCU_TRAFFIC = {
-    ("kda_bf16", "a75847421d95ddbc"): 673533184 + 119739904,
-    ("gdn_bf16", "a75847421d95ddbc"): 101868288 + 12880128,
-    ("gdn_long_t32768", "a75847421d95ddbc"): 408205824 + 112992256,
+    ("kda_bf16", "f911c9419ba63bc2"): 673315328 + 119190272,
+    ("gdn_bf16", "f911c9419ba63bc2"): 101823744 + 12931584,
     # Gated DeltaNet-2: the pre-scaling kernel and the chunked kernel of one call
-    ("gdn2_bf16", "d285f93d654df439"): 201335552 + 45257216 + 101834240 + 12926464,
+    ("gdn2_bf16", "736a00be23dba115"): 201334272 + 44804864 + 101836032 + 9884416,
+    # the segmented scan: the segment launch, the hand-off check, the conditional launch
+    ("gdn_long_t32768", "736a00be23dba115"): 414370560 + 115732480 + 3169280 + 67840,
+    ("gdn_long_t8192", "736a00be23dba115"): 109014016 + 14511616 + 3169024 + 68096,
     ("gdn_decode_bf16", "6c9773f81f64a408"): 271627008 + 211260672,
     ("loglinear_bf16", "79c1bdb9297c23dc"): 107535616 + 22006784,
 }

@@ -111,21 +111,23 @@ enum {
  * so the chained kernel runs T/64 dependent chunk steps per head ("Mechanisms, trade-offs and
  * cross-layer routing of linear-attention architectures", Technical details: the state is
  * decayed by alpha and corrected by the delta rule at every token). With few heads the call
- * instead cuts each head into G equal segments and runs them at once: every segment from a
- * zero state (the first from S0); then the first 8 chunks of every segment again from its
- * true entering state (S0, or the end state of the segment before it); then, per segment, a
- * check that the state at the end of those 8 chunks agrees with the zero-start one within
- * 2^-7 of its largest value-row norm (row-wise 2-norm). A step whose transition
- * diag(alpha)(I - beta k k^T) could grow a difference (alpha > 1 or beta |k|^2 > 2, both
- * checked on every token) also fails the check. When every check passes, the later outputs
- * and S_final stand: they differ from the chained scan's by at most that bound (times |q|),
- * the size of the kernel's own rounding: its bf16 copy of the state already sets two runs
- * from nearly equal states up to about 2^-8 of the row norm apart. When any check fails,
- * the chained kernel reruns the
- * whole call on the device (no host round trip), so the result is the chained one; a gate
- * close to 1 everywhere makes the check fail and the call then costs about twice the
- * chained kernel. The segmented scan takes 4 * B*H*G * dv*dk*4 bytes of scratch from the
- * library's stream-ordered pool (DR_ERR_CUDA if it cannot be had). DR_CHAINED turns it off.
+ * instead cuts each head into G equal segments and runs them at once, in one launch: every
+ * segment from a zero state (the first from S0); every segment but the last runs 8 chunks on
+ * into the next one, carrying its state, and writes the outputs there, while the next one
+ * writes none for those chunks. A check per boundary then compares the carried state at the
+ * end of those 8 chunks with the next segment's zero-start state there: they must agree
+ * within 2^-7 of the carried state's largest value-row norm (row-wise 2-norm). A step whose
+ * transition diag(alpha)(I - beta k k^T) could grow a difference (alpha > 1 or
+ * beta |k|^2 > 2, both checked on every token) also fails the check. When every check
+ * passes, the outputs and S_final stand: they differ from the chained scan's by at most that
+ * bound (times |q|), the size of the kernel's own rounding: its bf16 copy of the state
+ * already sets two runs from nearly equal states up to about 2^-8 of the row norm apart.
+ * When any check fails, the chained kernel reruns the whole call on the device (no host
+ * round trip), so the result is the chained one; a gate close to 1 everywhere makes the
+ * check fail and the call then costs up to about twice the chained kernel. The segmented
+ * scan takes 2 * B*H*G * dv*dk*4 bytes of scratch from the library's stream-ordered pool
+ * (DR_ERR_CUDA if it cannot be had). DR_CHAINED turns it off; dr_segment_counters counts its
+ * calls and reruns.
  *
  * Returns DR_OK or a negative status; on error nothing is launched.
  */
