@@ -276,7 +276,10 @@ struct ChunkSeg {
 // Per-device counts of segmented scans and of the chained reruns their checks asked for.
 __device__ unsigned long long g_seg_scans = 0, g_seg_reruns = 0;
 
-template <int MODE, int BV, bool SPLIT>
+// SEG: the segment launch of the segmented scan (Gated DeltaNet, split clusters), the only
+// instances that read seg.G, seg.ext, seg.S_ckpt and seg.expand; the others compile without
+// that code.
+template <int MODE, int BV, bool SPLIT, bool SEG = false>
 __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
     const __grid_constant__ CUtensorMap tmV, const float* __restrict__ beta,
@@ -287,13 +290,15 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
     if (seg.run_if && *seg.run_if == 0) return;
     if (seg.run_if && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
         atomicAdd(&g_seg_reruns, 1ull);
+    static_assert(!SEG || (SPLIT && MODE == DR_GDN), "segments run on split Gated DeltaNet");
     const long Ts = seg.Ts;
-    const int gseg = seg.G > 1 ? (int)(blockIdx.x % seg.G) : 0;
-    const int T = T_seq + ((seg.G > 1 && gseg < seg.G - 1) ? seg.ext : 0);  // tokens this CTA runs
-    const int cskip = (seg.G > 1 && gseg > 0) ? seg.ext / CK : 0;  // chunks whose outputs it leaves
-    const float* S0q = !S0          ? nullptr
-                       : seg.G > 1 ? (gseg == 0 ? S0 + (long)(blockIdx.x / seg.G) * dv * CDK : nullptr)
-                                   : S0 + (long)blockIdx.x * dv * CDK;
+    const int gseg = SEG ? (int)(blockIdx.x % seg.G) : 0;
+    // tokens this CTA runs, and the chunks whose outputs it leaves to the segment before
+    const int T = SEG ? T_seq + (gseg < seg.G - 1 ? seg.ext : 0) : T_seq;
+    const int cskip = SEG ? (gseg > 0 ? seg.ext / CK : 0) : 0;
+    const float* S0q = !S0   ? nullptr
+                       : SEG ? (gseg == 0 ? S0 + (long)(blockIdx.x / seg.G) * dv * CDK : nullptr)
+                             : S0 + (long)blockIdx.x * dv * CDK;
     using L = ChunkLayout<MODE, BV, SPLIT>;
     constexpr bool kGdn = L::kGdn;  // scalar gate (Gated DeltaNet)
     constexpr bool kKda = MODE == DR_KDA;
@@ -433,7 +438,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 // g_t = sum of log alpha over the chunk's rows up to t (masked rows add 0)
                 const float a0 = t0 + lane < T ? gate[bh * Ts + t0 + lane] : 1.f;
                 const float a1 = t0 + 32 + lane < T ? gate[bh * Ts + t0 + 32 + lane] : 1.f;
-                if (seg.expand && (a0 > 1.f || a1 > 1.f)) atomicOr(seg.expand, 1);
+                if (SEG && (a0 > 1.f || a1 > 1.f)) atomicOr(seg.expand, 1);
                 float x0 = t0 + lane < T ? __logf(a0) : 0.f;
                 float x1 = t0 + 32 + lane < T ? __logf(a1) : 0.f;
 #pragma unroll
@@ -709,7 +714,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
 #pragma unroll
                 for (int c16 = 0; c16 < LW; c16 += 16) tmem_ld16(trow + L::COL_D2 + cb + c16, d + c16);
                 tmem_wait_ld();
-                if (c * CK + r < T && c >= cskip) {
+                if (c * CK + r < T && (!SEG || c >= cskip)) {
                     uint4* dst = reinterpret_cast<uint4*>(u_out + (bh * Ts + c * CK + r) * (long)dv + v0 + cb);
 #pragma unroll
                     for (int i = 0; i < NV8; ++i) {
@@ -799,7 +804,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
 #pragma unroll
                     for (int v = 0; v < HC; ++v) dst[(long)v * CDK] = sv[v];
                 }
-                if (seg.S_ckpt && c + 1 == seg.ckpt_chunks) {
+                if (SEG && c + 1 == seg.ckpt_chunks) {
                     float* dst = seg.S_ckpt + (bh * dv + v0 + cb) * (long)CDK + r;
 #pragma unroll
                     for (int v = 0; v < HC; ++v) dst[(long)v * CDK] = sv[v];
@@ -833,7 +838,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     tmem_wait_ld();
                     tc_fence_before();
                     mbar_arrive(bar(B_ODONE));
-                    if (t < nvalid && c >= cskip) {
+                    if (t < nvalid && (!SEG || c >= cskip)) {
                         uint4* dst = reinterpret_cast<uint4*>(out + (bh * Ts + t0 + t) * (long)dv + v0 + cb);
 #pragma unroll
                         for (int i = 0; i < NV8; ++i) {
@@ -969,7 +974,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     float d[16];
                     tmem_ld16(trow + L::COL_D2 + c16, d);
                     tmem_wait_ld();
-                    if (r < nvalid && c >= cskip) {
+                    if (r < nvalid) {
                         uint4 w[2];
                         uint32_t* wp = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
@@ -995,7 +1000,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                         tmem_ld16(trow + L::COL_D2 + c0 + c16, d + c16);
                     }
                     tmem_wait_ld();
-                    if (t < nvalid && c >= cskip) {
+                    if (t < nvalid) {
                         uint4* dst = reinterpret_cast<uint4*>(out + (bh * Ts + t0 + t) * (long)dv +
                                                               v0 + c0);
 #pragma unroll
@@ -1016,9 +1021,6 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 float* dst = (c == nchunks - 1 && S_final)
                                  ? S_final + (bh * dv + v0) * (long)CDK + r
                                  : nullptr;
-                float* dck = (seg.S_ckpt && c + 1 == seg.ckpt_chunks)
-                                 ? seg.S_ckpt + (bh * dv + v0) * (long)CDK + r
-                                 : nullptr;
                 const float em = (kKda && c + 1 < nchunks) ? state_anchor(c + 1) : 1.f;
                 constexpr int HW = BV < 64 ? BV : 64;
 #pragma unroll
@@ -1030,10 +1032,6 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     if (dst) {
 #pragma unroll
                         for (int v = 0; v < HW; ++v) dst[(long)(c0 + v) * CDK] = sv[v];
-                    }
-                    if (dck) {
-#pragma unroll
-                        for (int v = 0; v < HW; ++v) dck[(long)(c0 + v) * CDK] = sv[v];
                     }
                     if constexpr (kKda) {
 #pragma unroll
@@ -1270,7 +1268,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     }
                 }
                 tmem_wait_ld();
-                if (seg.expand && lq < 64 && (t >> 5) == hf) {
+                if (SEG && lq < 64 && (t >> 5) == hf) {
                     // the step's transition diag(a)(I - beta k k^T) is non-expansive while
                     // beta |k|^2 <= 2 (|k|^2 is the Gram's diagonal)
                     float kk = 0.f;
@@ -1572,7 +1570,7 @@ inline ChunkSeg plain_seg(const ChunkArgs& a) {
 
 // `maps` picks the set of cached tensor-map slots (0, 1, 2: the launches of one segmented
 // scan keep their own maps).
-template <int MODE, int BV, bool SPLIT>
+template <int MODE, int BV, bool SPLIT, bool SEG = false>
 int launch_chunked_bv(const ChunkArgs& a, int nprep, const ChunkSeg& sg, int maps,
                       cudaStream_t stream) {
     using L = ChunkLayout<MODE, BV, SPLIT>;
@@ -1584,7 +1582,7 @@ int launch_chunked_bv(const ChunkArgs& a, int nprep, const ChunkSeg& sg, int map
         !cached_map_3d(m0 + 2, &mv, a.v, a.BH, rows, sg.Ts, a.dv, L::V_SWZ ? 64 : BV, L::V_SWZ))
         return DR_ERR_CUDA;
     const int smem = L::TOTAL + 1024;
-    auto kern = dr_chunked_kernel<MODE, BV, SPLIT>;
+    auto kern = dr_chunked_kernel<MODE, BV, SPLIT, SEG>;
     // the shared-memory opt-in is a per-device property of the function: set it once
     static bool attr_set[16] = {};
     int dev = 0;
@@ -1687,35 +1685,41 @@ inline SplitPlan pick_split(int variant, long BH, int dv) {
     return plan;
 }
 
-// One launch with a given plan (nprep == 0: unsplit, value slice from pick_bv).
-template <int MODE>
+// One launch with a given plan (nprep == 0: unsplit, value slice from pick_bv). SEG: the
+// segment launch of the segmented scan (split Gated DeltaNet only).
+template <int MODE, bool SEG = false>
 int launch_chunked_plan(const ChunkArgs& a, const SplitPlan& plan, const ChunkSeg& sg, int maps,
                         cudaStream_t stream) {
+    static_assert(!SEG || MODE == DR_GDN, "segments run on Gated DeltaNet");
     if constexpr (MODE != DR_KDA) {
         if (plan.nprep > 0) {
             switch (plan.bv) {
                 case 16:
-                    return launch_chunked_bv<MODE, 16, true>(a, plan.nprep, sg, maps, stream);
+                    return launch_chunked_bv<MODE, 16, true, SEG>(a, plan.nprep, sg, maps, stream);
                 case 32:
-                    return launch_chunked_bv<MODE, 32, true>(a, plan.nprep, sg, maps, stream);
+                    return launch_chunked_bv<MODE, 32, true, SEG>(a, plan.nprep, sg, maps, stream);
                 case 64:
-                    return launch_chunked_bv<MODE, 64, true>(a, plan.nprep, sg, maps, stream);
+                    return launch_chunked_bv<MODE, 64, true, SEG>(a, plan.nprep, sg, maps, stream);
             }
             return DR_ERR_UNSUPPORTED;
         }
     }
-    switch (pick_bv(MODE, a.BH, a.dv)) {
-        case 16:
-            return launch_chunked_bv<MODE, 16, false>(a, 0, sg, maps, stream);
-        case 32:
-            return launch_chunked_bv<MODE, 32, false>(a, 0, sg, maps, stream);
-        case 64:
-            return launch_chunked_bv<MODE, 64, false>(a, 0, sg, maps, stream);
-        case 128:
-            if constexpr (MODE == DR_KDA)
-                return launch_chunked_bv<MODE, 128, false>(a, 0, sg, maps, stream);
+    if constexpr (SEG) {
+        return DR_ERR_UNSUPPORTED;
+    } else {
+        switch (pick_bv(MODE, a.BH, a.dv)) {
+            case 16:
+                return launch_chunked_bv<MODE, 16, false>(a, 0, sg, maps, stream);
+            case 32:
+                return launch_chunked_bv<MODE, 32, false>(a, 0, sg, maps, stream);
+            case 64:
+                return launch_chunked_bv<MODE, 64, false>(a, 0, sg, maps, stream);
+            case 128:
+                if constexpr (MODE == DR_KDA)
+                    return launch_chunked_bv<MODE, 128, false>(a, 0, sg, maps, stream);
+        }
+        return DR_ERR_UNSUPPORTED;
     }
-    return DR_ERR_UNSUPPORTED;
 }
 
 template <int MODE>

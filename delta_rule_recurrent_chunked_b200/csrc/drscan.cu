@@ -229,7 +229,7 @@ int launch_gdn_segmented(const ChunkArgs& a, const SegPlan& sp, cudaStream_t str
     p.T = a.T / G;
     p.S_final = X;
     if (rc == DR_OK)
-        rc = launch_chunked_plan<DR_GDN>(
+        rc = launch_chunked_plan<DR_GDN, true>(
             p, sp.split, ChunkSeg{(long)p.T, Z, SEG_WINDOW, flag, nullptr, G, SEG_WINDOW * CK}, 1,
             stream);
     // 2. the hand-off checks (and the final states)

@@ -146,3 +146,38 @@ def test_segmented_calls_in_a_row_agree():
     _scan(dev, "gdn", chained=True)
     b = _scan(dev, "gdn")
     assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+# without S_final the check kernel has no final state to copy; the outputs are unchanged
+def test_segmented_without_final_state(oracle):
+    w = wl.DRWorkload("gdn_seg_nostate", 1, 2, 8192, 128, 128, wl.GDN, "bf16", s0_std=0.1)
+    inputs = wl.generate_dr(w, seed=9)
+    dev = to_device(inputs)
+    out, Sf, _ = drs.scan_ex(dev["q"], dev["k"], dev["v"], dev["beta"], dev["gate"], dev["S0"],
+                             mode="gdn", want_state=False, want_u=False)
+    torch.cuda.synchronize()
+    assert Sf is None and drs.poll_error() == drs.DR_OK
+    ref_out, _ = oracle_dr(oracle, inputs)
+    assert rel_err(tensor_np(out), ref_out) <= TOL
+    out2, _, _ = _scan(dev, "gdn")
+    assert torch.equal(out, out2)
+
+
+# two segmented calls in flight on two streams take scratch of their own
+def test_segmented_calls_on_two_streams(oracle):
+    ws = [wl.DRWorkload(f"gdn_seg_s{i}", 1, 2, 8192, 128, 128, wl.GDN, "bf16", s0_std=0.1)
+          for i in range(2)]
+    inputs = [wl.generate_dr(w, seed=20 + i) for i, w in enumerate(ws)]
+    devs = [to_device(x) for x in inputs]
+    streams = [torch.cuda.Stream() for _ in devs]
+    torch.cuda.synchronize()
+    results = []
+    for dev, st in zip(devs, streams):
+        with torch.cuda.stream(st):
+            results.append(drs.scan(dev["q"], dev["k"], dev["v"], dev["beta"], dev["gate"],
+                                    dev["S0"], mode="gdn"))
+    torch.cuda.synchronize()
+    assert drs.poll_error() == drs.DR_OK
+    for x, (out, Sf) in zip(inputs, results):
+        ref_out, ref_S = oracle_dr(oracle, x)
+        assert rel_err(tensor_np(out), ref_out) <= TOL and rel_err(tensor_np(Sf), ref_S) <= TOL
