@@ -181,3 +181,21 @@ def test_segmented_calls_on_two_streams(oracle):
     for x, (out, Sf) in zip(inputs, results):
         ref_out, ref_S = oracle_dr(oracle, x)
         assert rel_err(tensor_np(out), ref_out) <= TOL and rel_err(tensor_np(Sf), ref_S) <= TOL
+
+
+# narrower value heads run the segment launch on the split instances with 32 and 16 value
+# channels per chain CTA
+@pytest.mark.parametrize("dv", [32, 64])
+def test_segmented_gdn_narrow_values(oracle, dv):
+    w = wl.DRWorkload("gdn_seg_dv", 1, 4, 8192, 128, dv, wl.GDN, "bf16", s0_std=0.1)
+    plan = drs.chunked_plan_ex("gdn", 4, 8192, 128, dv)
+    assert plan[0] == dv // 2 and plan[2] > 1, plan
+    inputs = wl.generate_dr(w, seed=10 + dv)
+    dev = to_device(inputs)
+    before = drs.segment_counters()
+    out, Sf, _ = _scan(dev, "gdn")
+    after = drs.segment_counters()
+    assert (after[0] - before[0], after[1] - before[1]) == (1, 0)
+    ref_out, ref_S = oracle_dr(oracle, inputs)
+    e_out, e_S = rel_err(tensor_np(out), ref_out), rel_err(tensor_np(Sf), ref_S)
+    assert e_out <= TOL and e_S <= TOL, (dv, e_out, e_S)
