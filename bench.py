@@ -52,6 +52,8 @@ def parse_args(argv=None):
     p.add_argument("--e2e-steps", type=int, default=20)
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--no-per-config", action="store_true")
+    p.add_argument("--chained", action="store_true",
+                   help="time the chained chunked kernel where the segmented scan would run")
     p.add_argument("--no-e2e", action="store_true",
                    help="skip the end-to-end leg (profiling runs: only the timed launches)")
     p.add_argument("--per-config-steps", type=int, default=0,
@@ -463,7 +465,7 @@ def measure_dr(args, w, world, rank, local, device, K, cpu_target):
                         out=outs[i % nsets], S_final=Sfs[i % nsets])
         else:
             drs.scan(st["q"], st["k"], st["v"], st["beta"], st["gate"], st["S0"], mode=mode,
-                     out=outs[i % nsets], S_final=Sfs[i % nsets])
+                     out=outs[i % nsets], S_final=Sfs[i % nsets], chained=args.chained)
 
     stream = torch.cuda.current_stream(device)
     for i in range(max(3, args.warmup)):
@@ -494,7 +496,8 @@ def measure_dr(args, w, world, rank, local, device, K, cpu_target):
     # the segmented scan (few heads, long sequences) is three launches of this library per
     # call: all segments at once, the hand-off check and the chained kernel's conditional
     # launch (which returns at once when the checks pass)
-    nseg = drs.chunked_plan_ex(mode, w.B * w.H, w.T, w.dk, w.dv)[2] if chunked else 1
+    nseg = (drs.chunked_plan_ex(mode, w.B * w.H, w.T, w.dk, w.dv, chained=args.chained)[2]
+            if chunked else 1)
     kname = "chunked" if nseg == 1 else f"segmented chunked ({nseg} segments per head)"
     config = dict(workload_config(w, world), l2=l2_note(nsets, nbytes, needs_flush),
                   kernel=("prescale+" + kname if prescaled else kname) if chunked
@@ -885,7 +888,7 @@ def run_e2e(args, w, inputs, mode, device, stream):
                         erase=d["erase"], write=d["write"], want_u=False, out=o[0], S_final=o[1])
         else:
             drs.scan(d["q"], d["k"], d["v"], d["beta"], d["gate"], d["S0"], mode=mode,
-                     out=o[0], S_final=o[1])
+                     out=o[0], S_final=o[1], chained=args.chained)
 
     pipe = CopyPipeline(device, host, make_outputs, launch)
     ms = pipe.run(max(1, args.e2e_steps))

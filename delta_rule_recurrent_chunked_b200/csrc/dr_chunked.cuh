@@ -276,9 +276,9 @@ struct ChunkSeg {
 // Per-device counts of segmented scans and of the chained reruns their checks asked for.
 __device__ unsigned long long g_seg_scans = 0, g_seg_reruns = 0;
 
-// SEG: the segment launch of the segmented scan (Gated DeltaNet, split clusters), the only
-// instances that read seg.G, seg.ext, seg.S_ckpt and seg.expand; the others compile without
-// that code.
+// SEG: the segment launch of the segmented scan (Gated DeltaNet on split clusters, KDA on
+// one CTA per sequence), the only instances that read seg.G, seg.ext, seg.S_ckpt and
+// seg.expand; the others compile without that code.
 template <int MODE, int BV, bool SPLIT, bool SEG = false>
 __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
     const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
@@ -290,7 +290,8 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
     if (seg.run_if && *seg.run_if == 0) return;
     if (seg.run_if && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
         atomicAdd(&g_seg_reruns, 1ull);
-    static_assert(!SEG || (SPLIT && MODE == DR_GDN), "segments run on split Gated DeltaNet");
+    static_assert(!SEG || (SPLIT && MODE == DR_GDN) || (!SPLIT && MODE == DR_KDA),
+                  "segments run on split Gated DeltaNet and on unsplit KDA");
     const long Ts = seg.Ts;
     const int gseg = SEG ? (int)(blockIdx.x % seg.G) : 0;
     // tokens this CTA runs, and the chunks whose outputs it leaves to the segment before
@@ -974,7 +975,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     float d[16];
                     tmem_ld16(trow + L::COL_D2 + c16, d);
                     tmem_wait_ld();
-                    if (r < nvalid) {
+                    if (r < nvalid && (!SEG || c >= cskip)) {
                         uint4 w[2];
                         uint32_t* wp = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
@@ -1000,7 +1001,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                         tmem_ld16(trow + L::COL_D2 + c0 + c16, d + c16);
                     }
                     tmem_wait_ld();
-                    if (t < nvalid) {
+                    if (t < nvalid && (!SEG || c >= cskip)) {
                         uint4* dst = reinterpret_cast<uint4*>(out + (bh * Ts + t0 + t) * (long)dv +
                                                               v0 + c0);
 #pragma unroll
@@ -1021,6 +1022,9 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 float* dst = (c == nchunks - 1 && S_final)
                                  ? S_final + (bh * dv + v0) * (long)CDK + r
                                  : nullptr;
+                float* dck = (SEG && c + 1 == seg.ckpt_chunks)
+                                 ? seg.S_ckpt + (bh * dv + v0) * (long)CDK + r
+                                 : nullptr;
                 const float em = (kKda && c + 1 < nchunks) ? state_anchor(c + 1) : 1.f;
                 constexpr int HW = BV < 64 ? BV : 64;
 #pragma unroll
@@ -1032,6 +1036,10 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     if (dst) {
 #pragma unroll
                         for (int v = 0; v < HW; ++v) dst[(long)(c0 + v) * CDK] = sv[v];
+                    }
+                    if (SEG && dck) {
+#pragma unroll
+                        for (int v = 0; v < HW; ++v) dck[(long)(c0 + v) * CDK] = sv[v];
                     }
                     if constexpr (kKda) {
 #pragma unroll
@@ -1148,6 +1156,13 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
 #pragma unroll
                     for (int i = 0; i < 16; ++i)
                         if (16 * kq4 + i >= nvalid) gpf[i] = make_float2(1.f, 1.f);
+                }
+                if constexpr (SEG) {
+                    // a gate above 1 could grow a state difference
+                    bool up = false;
+#pragma unroll
+                    for (int i = 0; i < 16; ++i) up |= gpf[i].x > 1.f || gpf[i].y > 1.f;
+                    if (up) atomicOr(seg.expand, 1);
                 }
                 float2 part = make_float2(1.f, 1.f);
 #pragma unroll
@@ -1685,12 +1700,12 @@ inline SplitPlan pick_split(int variant, long BH, int dv) {
     return plan;
 }
 
-// One launch with a given plan (nprep == 0: unsplit, value slice from pick_bv). SEG: the
-// segment launch of the segmented scan (split Gated DeltaNet only).
+// One launch with a given plan (nprep == 0: unsplit, value slice plan.bv, or pick_bv's when
+// 0). SEG: the segment launch of the segmented scan (split Gated DeltaNet, unsplit KDA).
 template <int MODE, bool SEG = false>
 int launch_chunked_plan(const ChunkArgs& a, const SplitPlan& plan, const ChunkSeg& sg, int maps,
                         cudaStream_t stream) {
-    static_assert(!SEG || MODE == DR_GDN, "segments run on Gated DeltaNet");
+    static_assert(!SEG || MODE == DR_GDN || MODE == DR_KDA, "segments: GDN and KDA");
     if constexpr (MODE != DR_KDA) {
         if (plan.nprep > 0) {
             switch (plan.bv) {
@@ -1704,19 +1719,20 @@ int launch_chunked_plan(const ChunkArgs& a, const SplitPlan& plan, const ChunkSe
             return DR_ERR_UNSUPPORTED;
         }
     }
-    if constexpr (SEG) {
+    if constexpr (SEG && MODE != DR_KDA) {
         return DR_ERR_UNSUPPORTED;
     } else {
-        switch (pick_bv(MODE, a.BH, a.dv)) {
+        switch (plan.bv ? plan.bv : pick_bv(MODE, a.BH, a.dv)) {
             case 16:
-                return launch_chunked_bv<MODE, 16, false>(a, 0, sg, maps, stream);
+                if constexpr (!SEG) return launch_chunked_bv<MODE, 16, false>(a, 0, sg, maps, stream);
+                break;
             case 32:
-                return launch_chunked_bv<MODE, 32, false>(a, 0, sg, maps, stream);
+                return launch_chunked_bv<MODE, 32, false, SEG>(a, 0, sg, maps, stream);
             case 64:
-                return launch_chunked_bv<MODE, 64, false>(a, 0, sg, maps, stream);
+                return launch_chunked_bv<MODE, 64, false, SEG>(a, 0, sg, maps, stream);
             case 128:
                 if constexpr (MODE == DR_KDA)
-                    return launch_chunked_bv<MODE, 128, false>(a, 0, sg, maps, stream);
+                    return launch_chunked_bv<MODE, 128, false, SEG>(a, 0, sg, maps, stream);
         }
         return DR_ERR_UNSUPPORTED;
     }
@@ -1776,8 +1792,32 @@ struct SegPlan {
 // The plan takes the G with the lowest estimate among those that keep every segment at
 // least SEG_MIN_CHUNKS long and let all B*H*G segments run at once as clusters of at least
 // two prep and two chain CTAs, and segments only when that estimate is below 0.9 * nch.
+//
+// KDA runs unsplit, one CTA per (head, value slice), and its prep, about 13.9 K cycles per
+// chunk on B200, sets the pace whatever the slice width: with few heads the chained plan
+// splits the values into narrow slices whose CTAs each repeat the whole prep. The segment
+// launch gives every sequence one CTA with all dv value channels instead, so in units of a
+// chunk step (chained nch) the segmented scan takes nch / G + SEG_WINDOW + 2, for the G that
+// keeps B*H*G CTAs within one per SM.
 inline SegPlan pick_segments(int variant, long BH, int T, int dv) {
     SegPlan sp;
+    if (variant == DR_KDA) {
+        if (T % CK != 0) return sp;
+        const int nch = T / CK;
+        double best = 0.9 * nch;
+        for (int G = 2; G <= nch / SEG_MIN_CHUNKS; ++G) {
+            if (nch % G) continue;
+            if (BH * G > 148) break;
+            const double est = nch / G + SEG_WINDOW + 2.0;
+            if (est < best) {
+                best = est;
+                sp.nseg = G;
+                sp.split.bv = dv;
+                sp.split.nprep = 0;
+            }
+        }
+        return sp;
+    }
     if (variant != DR_GDN || dv < 32 || T % CK != 0) return sp;
     const int nch = T / CK;
     double best = 0.9 * nch;

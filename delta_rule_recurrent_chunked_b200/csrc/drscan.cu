@@ -210,9 +210,10 @@ int scratch_alloc(void** p, size_t bytes, cudaStream_t stream) {
     return cudaMallocFromPoolAsync(p, bytes, pool, stream) == cudaSuccess ? DR_OK : DR_ERR_CUDA;
 }
 
-// The segmented scan of Gated DeltaNet (steps in dr_chunked.cuh): scratch for two sets of
-// per-segment states and the check word, stream-ordered from the library's pool.
-int launch_gdn_segmented(const ChunkArgs& a, const SegPlan& sp, cudaStream_t stream) {
+// The segmented scan (steps in dr_chunked.cuh) of Gated DeltaNet or KDA: scratch for two sets
+// of per-segment states and the check word, stream-ordered from the library's pool.
+template <int MODE>
+int launch_segmented(const ChunkArgs& a, const SegPlan& sp, cudaStream_t stream) {
     const int G = sp.nseg;
     const long nseq = (long)a.BH * G;
     const size_t sn = (size_t)a.dv * CDK;  // floats per state
@@ -229,7 +230,7 @@ int launch_gdn_segmented(const ChunkArgs& a, const SegPlan& sp, cudaStream_t str
     p.T = a.T / G;
     p.S_final = X;
     if (rc == DR_OK)
-        rc = launch_chunked_plan<DR_GDN, true>(
+        rc = launch_chunked_plan<MODE, true>(
             p, sp.split, ChunkSeg{(long)p.T, Z, SEG_WINDOW, flag, nullptr, G, SEG_WINDOW * CK}, 1,
             stream);
     // 2. the hand-off checks (and the final states)
@@ -240,19 +241,21 @@ int launch_gdn_segmented(const ChunkArgs& a, const SegPlan& sp, cudaStream_t str
     }
     // 3. the chained scan, run only if a check failed
     if (rc == DR_OK)
-        rc = launch_chunked_plan<DR_GDN>(
-            a, pick_split(DR_GDN, a.BH, a.dv),
-            ChunkSeg{(long)a.T, nullptr, 0, nullptr, flag, 0, 0}, 2, stream);
+        rc = launch_chunked_plan<MODE>(a, pick_split(MODE, a.BH, a.dv),
+                                       ChunkSeg{(long)a.T, nullptr, 0, nullptr, flag, 0, 0}, 2,
+                                       stream);
     if (cudaFreeAsync(scratch, stream) != cudaSuccess && rc == DR_OK) rc = DR_ERR_CUDA;
     return rc;
 }
 
-// The chunked path: the segmented scan where its plan applies (Gated DeltaNet, few heads,
-// long sequences; not with DR_CHAINED), else one launch of the chained kernel.
+// The chunked path: the segmented scan where its plan applies (Gated DeltaNet and KDA, few
+// heads, long sequences; not with DR_CHAINED), else one launch of the chained kernel.
 int launch_chunked_auto(const ChunkArgs& a, int variant, bool chained, cudaStream_t stream) {
-    if (!chained && variant == DR_GDN) {
-        const SegPlan sp = pick_segments(DR_GDN, a.BH, a.T, a.dv);
-        if (sp.nseg > 1) return launch_gdn_segmented(a, sp, stream);
+    if (!chained && (variant == DR_GDN || variant == DR_KDA)) {
+        const SegPlan sp = pick_segments(variant, a.BH, a.T, a.dv);
+        if (sp.nseg > 1)
+            return variant == DR_KDA ? launch_segmented<DR_KDA>(a, sp, stream)
+                                     : launch_segmented<DR_GDN>(a, sp, stream);
     }
     return launch_chunked(a, variant, stream);
 }

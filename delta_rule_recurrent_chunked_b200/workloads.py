@@ -99,6 +99,10 @@ WORKLOADS = {
 for _T in (4096, 8192, 16384, 32768):
     WORKLOADS[f"gdn_long_t{_T}"] = DRWorkload(f"gdn_long_t{_T}", 1, 16, _T, 128, 128, GDN, "bf16",
                                               s0_std=0.1)
+# long-context KDA with few heads (not one of the timed configurations; the segmented scan's
+# KDA case)
+WORKLOADS["kda_long_t32768"] = DRWorkload("kda_long_t32768", 1, 16, 32768, 128, 128, KDA, "bf16",
+                                          s0_std=0.1)
 WORKLOADS["gdn2_bf16"] = DRWorkload("gdn2_bf16", 4, 8, 4096, 128, 128, GDN2, "bf16")
 WORKLOADS["loglinear_bf16"] = LogLinearWorkload("loglinear_bf16", 4, 8, 4096, 128, 128)
 # streaming decode: one token per step for 4096 heads whose 256 MiB fp32 state stays in HBM

@@ -58,8 +58,8 @@ enum {
 /* Use the per-token kernel (fp32 state, CUDA cores) even where the chunked tensor-core
  * kernel applies. Same results up to rounding; slower. For testing and as a baseline. */
 #define DR_FORCE_SEQUENTIAL 0x200
-/* Keep Gated DeltaNet on the chained chunked kernel (one pass, one dependent chain of chunks
- * per head) where dr_scan_fwd would take the segmented scan (see dr_scan_fwd). */
+/* Keep Gated DeltaNet and KDA on the chained chunked kernel (one pass, one dependent chain of
+ * chunks per head) where dr_scan_fwd would take the segmented scan (see dr_scan_fwd). */
 #define DR_CHAINED 0x400
 
 /* status codes */
@@ -106,8 +106,8 @@ enum {
  * below that latches DR_ERR_GATE_RANGE, which dr_poll_error() reports (the outputs of
  * that call are then invalid: rerun it with DR_FORCE_SEQUENTIAL, which has no such limit).
  *
- * Segmented scan (Gated DeltaNet, bf16, dk = 128, T a multiple of 64, heads too few to
- * fill the GPU; see dr_chunked_plan_ex). A sequence's state carries over from chunk to chunk,
+ * Segmented scan (Gated DeltaNet and KDA, bf16, dk = 128, T a multiple of 64, heads too few
+ * to fill the GPU; see dr_chunked_plan_ex). A sequence's state carries over from chunk to chunk,
  * so the chained kernel runs T/64 dependent chunk steps per head ("Mechanisms, trade-offs and
  * cross-layer routing of linear-attention architectures", Technical details: the state is
  * decayed by alpha and corrected by the delta rule at every token). With few heads the call

@@ -1,4 +1,4 @@
-"""GPU parity of the segmented Gated DeltaNet scan (few heads, long sequences).
+"""GPU parity of the segmented scan of Gated DeltaNet and KDA (few heads, long sequences).
 
 dr_scan_fwd cuts each head into segments that run at once from zero states; every segment
 but the last runs eight chunks on into the next one, carrying its state, and writes the
@@ -56,7 +56,11 @@ def test_plan_segments_only_gated_deltanet_with_few_heads():
     assert plan("gdn", 2, 4095, 128, 128)[2] == 1
     assert plan("gdn", 2, 4096 - 64, 128, 128)[2] == 1
     assert plan("deltanet", 2, 32768, 128, 128)[2] == 1
-    assert plan("kda", 2, 32768, 128, 128)[2] == 1
+    # KDA: one CTA per segment with every value channel
+    assert plan("kda", 16, 32768, 128, 128) == (128, 0, 8)
+    assert plan("kda", 2, 32768, 128, 128) == (128, 0, 16)
+    assert plan("kda", 4, 8192, 128, 64) == (64, 0, 4)
+    assert plan("kda", 128, 4096, 128, 128)[2] == 1
 
 
 @pytest.mark.parametrize("B,H,T,s0", [(1, 2, 8192, True), (1, 2, 16384, False), (2, 3, 8192, True),
@@ -199,3 +203,61 @@ def test_segmented_gdn_narrow_values(oracle, dv):
     ref_out, ref_S = oracle_dr(oracle, inputs)
     e_out, e_S = rel_err(tensor_np(out), ref_out), rel_err(tensor_np(Sf), ref_S)
     assert e_out <= TOL and e_S <= TOL, (dv, e_out, e_S)
+
+
+# KDA: the segment launch is the unsplit kernel with every value channel in one CTA
+@pytest.mark.parametrize("H,T,dv,s0", [(2, 8192, 128, True), (4, 8192, 64, False),
+                                       (1, 16384, 128, True)])
+def test_segmented_kda_matches_oracle(oracle, H, T, dv, s0):
+    w = wl.DRWorkload("kda_seg", 1, H, T, 128, dv, wl.KDA, "bf16", s0_std=0.1 if s0 else 0.0)
+    assert drs.chunked_plan_ex("kda", H, T, 128, dv)[2] > 1
+    inputs = wl.generate_dr(w, seed=30 + H)
+    dev = to_device(inputs)
+    before = drs.segment_counters()
+    out, Sf, _ = _scan(dev, "kda")
+    after = drs.segment_counters()
+    assert (after[0] - before[0], after[1] - before[1]) == (1, 0)
+    ref_out, ref_S = oracle_dr(oracle, inputs)
+    e_out, e_S = rel_err(tensor_np(out), ref_out), rel_err(tensor_np(Sf), ref_S)
+    assert e_out <= TOL and e_S <= TOL, (e_out, e_S)
+    out_c, Sf_c, _ = _scan(dev, "kda", chained=True)
+    assert rel_err(tensor_np(out), tensor_np(out_c)) <= 1e-2
+    assert rel_err(tensor_np(Sf), tensor_np(Sf_c)) <= 1e-2
+
+
+def _kda_fallback_equals_chained(oracle, inputs):
+    dev = to_device(inputs)
+    before = drs.segment_counters()
+    out, Sf, _ = _scan(dev, "kda")
+    after = drs.segment_counters()
+    assert (after[0] - before[0], after[1] - before[1]) == (1, 1)
+    out_c, Sf_c, _ = _scan(dev, "kda", chained=True)
+    assert torch.equal(out, out_c) and torch.equal(Sf, Sf_c)
+    ref_out, ref_S = oracle_dr(oracle, inputs)
+    e_out, e_S = rel_err(tensor_np(out), ref_out), rel_err(tensor_np(Sf), ref_S)
+    assert e_out <= TOL and e_S <= TOL, (e_out, e_S)
+
+
+# per-channel gates all but 1: too little decay over the window, the chained kernel reruns
+def test_kda_weak_decay_falls_back_to_the_chained_scan(oracle):
+    w = wl.DRWorkload("kda_weak", 1, 2, 8192, 128, 128, wl.KDA, "bf16", s0_std=0.1,
+                      gate_mu=-12.0)
+    _kda_fallback_equals_chained(oracle, wl.generate_dr(w, seed=40))
+
+
+# one channel of one token's gate above 1
+def test_kda_gate_above_one_falls_back_to_the_chained_scan(oracle):
+    w = wl.DRWorkload("kda_gt1", 1, 2, 8192, 128, 128, wl.KDA, "bf16", s0_std=0.1)
+    inputs = wl.generate_dr(w, seed=41)
+    inputs["gate"][0, 1, 5000, 17] = 1.2
+    _kda_fallback_equals_chained(oracle, inputs)
+
+
+# one token whose step can grow a difference (beta |k|^2 = 3.6 > 2)
+def test_kda_expanding_step_falls_back_to_the_chained_scan(oracle):
+    w = wl.DRWorkload("kda_expand", 1, 2, 8192, 128, 128, wl.KDA, "bf16", s0_std=0.1)
+    inputs = wl.generate_dr(w, seed=42)
+    inputs["k"][0, 0, 6000] *= 2.0  # bf16 values: exact
+    inputs["k_raw"] = wl.bf16_bits(inputs["k"])
+    inputs["beta"][0, 0, 6000] = 0.9
+    _kda_fallback_equals_chained(oracle, inputs)
