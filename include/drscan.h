@@ -117,7 +117,7 @@ enum {
  * writes none for those chunks. A check per boundary then compares the carried state at the
  * end of those 8 chunks with the next segment's zero-start state there: they must agree
  * within 2^-7 of the carried state's largest value-row norm (row-wise 2-norm). A step whose
- * transition diag(alpha)(I - beta k k^T) could grow a difference (alpha > 1 or
+ * transition diag(alpha)(I - beta k k^T) could grow a difference (any alpha > 1 or
  * beta |k|^2 > 2, both checked on every token) also fails the check. When every check
  * passes, the outputs and S_final stand: they differ from the chained scan's by at most that
  * bound (times |q|), the size of the kernel's own rounding: its bf16 copy of the state
