@@ -297,6 +297,9 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
     // tokens this CTA runs, and the chunks whose outputs it leaves to the segment before
     const int T = SEG ? T_seq + (gseg < seg.G - 1 ? seg.ext : 0) : T_seq;
     const int cskip = SEG ? (gseg > 0 ? seg.ext / CK : 0) : 0;
+    // the one-CTA chain path below is compiled into split instances too (unused there): it
+    // carries the segment code only in the unsplit segment instances
+    constexpr bool kSegU = SEG && !SPLIT;
     const float* S0q = !S0   ? nullptr
                        : SEG ? (gseg == 0 ? S0 + (long)(blockIdx.x / seg.G) * dv * CDK : nullptr)
                              : S0 + (long)blockIdx.x * dv * CDK;
@@ -975,7 +978,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                     float d[16];
                     tmem_ld16(trow + L::COL_D2 + c16, d);
                     tmem_wait_ld();
-                    if (r < nvalid && (!SEG || c >= cskip)) {
+                    if (r < nvalid && (!kSegU || c >= cskip)) {
                         uint4 w[2];
                         uint32_t* wp = reinterpret_cast<uint32_t*>(w);
 #pragma unroll
@@ -1001,7 +1004,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                         tmem_ld16(trow + L::COL_D2 + c0 + c16, d + c16);
                     }
                     tmem_wait_ld();
-                    if (t < nvalid && (!SEG || c >= cskip)) {
+                    if (t < nvalid && (!kSegU || c >= cskip)) {
                         uint4* dst = reinterpret_cast<uint4*>(out + (bh * Ts + t0 + t) * (long)dv +
                                                               v0 + c0);
 #pragma unroll
@@ -1022,7 +1025,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
                 float* dst = (c == nchunks - 1 && S_final)
                                  ? S_final + (bh * dv + v0) * (long)CDK + r
                                  : nullptr;
-                float* dck = (SEG && c + 1 == seg.ckpt_chunks)
+                float* dck = (kSegU && c + 1 == seg.ckpt_chunks)
                                  ? seg.S_ckpt + (bh * dv + v0) * (long)CDK + r
                                  : nullptr;
                 const float em = (kKda && c + 1 < nchunks) ? state_anchor(c + 1) : 1.f;
@@ -1037,7 +1040,7 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
 #pragma unroll
                         for (int v = 0; v < HW; ++v) dst[(long)(c0 + v) * CDK] = sv[v];
                     }
-                    if (SEG && dck) {
+                    if (kSegU && dck) {
 #pragma unroll
                         for (int v = 0; v < HW; ++v) dck[(long)(c0 + v) * CDK] = sv[v];
                     }
