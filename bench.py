@@ -147,15 +147,16 @@ def aggregate_value(world: int, head_tokens: int, steps: int, total_ms_max: floa
 # loglinear.cuh for log-linear attention) at capture time; a changed source reports null.
 # Summaries with the commands are under profiles/.
 NCU_TRAFFIC = {
-    ("kda_bf16", "43f6f4db325460ec"): 673318912 + 119138816,
-    ("gdn_bf16", "43f6f4db325460ec"): 101819904 + 12947456,
+    ("kda_bf16", "c661a4b94a22c92c"): 673364992 + 119821312,
+    ("gdn_bf16", "c661a4b94a22c92c"): 101819904 + 12610304,
     # Gated DeltaNet-2: the pre-scaling kernel and the chunked kernel of one call
-    ("gdn2_bf16", "a9af0fde3cb9bcdf"): 201332992 + 44423168 + 101875712 + 9543424,
+    ("gdn2_bf16", "08557876d53c25c0"): 201332992 + 44987904 + 101819136 + 9339392,
     # the segmented scan: the segment launch, the hand-off check, the conditional launch
-    ("gdn_long_t4096", "a9af0fde3cb9bcdf"): 52016896 + 676096 + 3169024 + 67584,
-    ("gdn_long_t8192", "a9af0fde3cb9bcdf"): 109074432 + 14610432 + 3168768 + 67584,
-    ("gdn_long_t16384", "a9af0fde3cb9bcdf"): 210963968 + 47341568 + 3168768 + 67840,
-    ("gdn_long_t32768", "a9af0fde3cb9bcdf"): 414718464 + 115881472 + 3169280 + 67840,
+    ("gdn_long_t4096", "08557876d53c25c0"): 52017152 + 672768 + 3168768 + 68096,
+    ("gdn_long_t8192", "08557876d53c25c0"): 109080064 + 14750464 + 3169024 + 67584,
+    ("gdn_long_t16384", "08557876d53c25c0"): 210959360 + 47117312 + 3169024 + 68096,
+    ("gdn_long_t32768", "08557876d53c25c0"): 414369024 + 116253184 + 3169024 + 67840,
+    ("kda_long_t32768", "08557876d53c25c0"): 747988992 + 127770880 + 15751936 + 68096,
     ("gdn_decode_bf16", "6c9773f81f64a408"): 271627008 + 211260672,
     ("loglinear_bf16", "79c1bdb9297c23dc"): 107535616 + 22006784,
 }
