@@ -290,8 +290,9 @@ __global__ void __launch_bounds__(CHUNK_THREADS, 1) dr_chunked_kernel(
     if (seg.run_if && *seg.run_if == 0) return;
     if (seg.run_if && blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0)
         atomicAdd(&g_seg_reruns, 1ull);
-    static_assert(!SEG || (SPLIT && MODE == DR_GDN) || (!SPLIT && MODE == DR_KDA),
-                  "segments run on split Gated DeltaNet and on unsplit KDA");
+    static_assert(!SEG || (SPLIT && (MODE == DR_GDN || MODE == DR_DELTANET)) ||
+                      (!SPLIT && MODE == DR_KDA),
+                  "segments run on split DeltaNet / Gated DeltaNet and on unsplit KDA");
     const long Ts = seg.Ts;
     const int gseg = SEG ? (int)(blockIdx.x % seg.G) : 0;
     // tokens this CTA runs, and the chunks whose outputs it leaves to the segment before
@@ -1708,7 +1709,8 @@ inline SplitPlan pick_split(int variant, long BH, int dv) {
 template <int MODE, bool SEG = false>
 int launch_chunked_plan(const ChunkArgs& a, const SplitPlan& plan, const ChunkSeg& sg, int maps,
                         cudaStream_t stream) {
-    static_assert(!SEG || MODE == DR_GDN || MODE == DR_KDA, "segments: GDN and KDA");
+    static_assert(!SEG || MODE == DR_GDN || MODE == DR_KDA || MODE == DR_DELTANET,
+                  "segments: DeltaNet, GDN and KDA");
     if constexpr (MODE != DR_KDA) {
         if (plan.nprep > 0) {
             switch (plan.bv) {
@@ -1779,11 +1781,18 @@ int launch_chunked_mode(const ChunkArgs& a, cudaStream_t stream) {
 // ---------------------------------------------------------------------------------------
 constexpr int SEG_WINDOW = 8;        // chunks of overlap between consecutive segments
 constexpr int SEG_MIN_CHUNKS = 32;   // shortest segment (four windows)
+// DeltaNet has no gate: a state difference shrinks only along the keys written, by about
+// 0.85 per chunk for keys spread over all directions (fp64 on the workloads' inputs: 0.26,
+// 7e-2, 1.7e-2, 4.7e-3 of the row norm after 8, 16, 24, 32 chunks), so its window is 48
+// chunks (about 3e-4) and its segments at least twice that
+constexpr int SEG_WINDOW_DN = 48;
+constexpr int SEG_MIN_CHUNKS_DN = 96;
 constexpr float SEG_EPS = 1.0f / 128.f;
 
 struct SegPlan {
-    int nseg = 1;     // segments per head (1: the chained kernel alone)
-    SplitPlan split;  // plan of the segment launch (BH * nseg sequences)
+    int nseg = 1;               // segments per head (1: the chained kernel alone)
+    int window = SEG_WINDOW;    // chunks of overlap
+    SplitPlan split;            // plan of the segment launch (BH * nseg sequences)
 };
 
 // Segments pay where the chain is long: measured on B200 (Gated DeltaNet, dk = dv = 128), a
@@ -1821,19 +1830,22 @@ inline SegPlan pick_segments(int variant, long BH, int T, int dv) {
         }
         return sp;
     }
-    if (variant != DR_GDN || dv < 32 || T % CK != 0) return sp;
+    if ((variant != DR_GDN && variant != DR_DELTANET) || dv < 32 || T % CK != 0) return sp;
     const int nch = T / CK;
+    const int window = variant == DR_DELTANET ? SEG_WINDOW_DN : SEG_WINDOW;
+    const int min_chunks = variant == DR_DELTANET ? SEG_MIN_CHUNKS_DN : SEG_MIN_CHUNKS;
     double best = 0.9 * nch;
-    for (int G = 2; G <= nch / SEG_MIN_CHUNKS; ++G) {
+    for (int G = 2; G <= nch / min_chunks; ++G) {
         if (nch % G) continue;
         const long n = BH * G;
         if (n * 4 > 148 || n > max_active_clusters(4)) break;
         const SplitPlan p = pick_split(variant, n, dv);
         if (p.nprep < 2) continue;
-        const double est = 1.18 * (nch / G + SEG_WINDOW) + 5.0;
+        const double est = 1.18 * (nch / G + window) + 5.0;
         if (est < best) {
             best = est;
             sp.nseg = G;
+            sp.window = window;
             sp.split = p;
         }
     }

@@ -231,7 +231,7 @@ int launch_segmented(const ChunkArgs& a, const SegPlan& sp, cudaStream_t stream)
     p.S_final = X;
     if (rc == DR_OK)
         rc = launch_chunked_plan<MODE, true>(
-            p, sp.split, ChunkSeg{(long)p.T, Z, SEG_WINDOW, flag, nullptr, G, SEG_WINDOW * CK}, 1,
+            p, sp.split, ChunkSeg{(long)p.T, Z, sp.window, flag, nullptr, G, sp.window * CK}, 1,
             stream);
     // 2. the hand-off checks (and the final states)
     if (rc == DR_OK) {
@@ -248,14 +248,21 @@ int launch_segmented(const ChunkArgs& a, const SegPlan& sp, cudaStream_t stream)
     return rc;
 }
 
-// The chunked path: the segmented scan where its plan applies (Gated DeltaNet and KDA, few
-// heads, long sequences; not with DR_CHAINED), else one launch of the chained kernel.
+// The chunked path: the segmented scan where its plan applies (few heads, long sequences; not
+// with DR_CHAINED), else one launch of the chained kernel.
 int launch_chunked_auto(const ChunkArgs& a, int variant, bool chained, cudaStream_t stream) {
-    if (!chained && (variant == DR_GDN || variant == DR_KDA)) {
+    if (!chained) {
         const SegPlan sp = pick_segments(variant, a.BH, a.T, a.dv);
-        if (sp.nseg > 1)
-            return variant == DR_KDA ? launch_segmented<DR_KDA>(a, sp, stream)
-                                     : launch_segmented<DR_GDN>(a, sp, stream);
+        if (sp.nseg > 1) {
+            switch (variant) {
+                case DR_DELTANET:
+                    return launch_segmented<DR_DELTANET>(a, sp, stream);
+                case DR_GDN:
+                    return launch_segmented<DR_GDN>(a, sp, stream);
+                case DR_KDA:
+                    return launch_segmented<DR_KDA>(a, sp, stream);
+            }
+        }
     }
     return launch_chunked(a, variant, stream);
 }

@@ -55,7 +55,10 @@ def test_plan_segments_only_gated_deltanet_with_few_heads():
     assert plan("gdn", 16, 4096 + 64, 128, 128)[2] == 1
     assert plan("gdn", 2, 4095, 128, 128)[2] == 1
     assert plan("gdn", 2, 4096 - 64, 128, 128)[2] == 1
-    assert plan("deltanet", 2, 32768, 128, 128)[2] == 1
+    # DeltaNet: a 48-chunk window, segments of at least 96 chunks
+    assert plan("deltanet", 16, 32768, 128, 128) == (64, 2, 2)
+    assert plan("deltanet", 2, 32768, 128, 128)[2] == 4
+    assert plan("deltanet", 16, 8192, 128, 128)[2] == 1
     # KDA: one CTA per segment with every value channel
     assert plan("kda", 16, 32768, 128, 128) == (128, 0, 8)
     assert plan("kda", 2, 32768, 128, 128) == (128, 0, 16)
@@ -261,3 +264,20 @@ def test_kda_expanding_step_falls_back_to_the_chained_scan(oracle):
     inputs["k_raw"] = wl.bf16_bits(inputs["k"])
     inputs["beta"][0, 0, 6000] = 0.9
     _kda_fallback_equals_chained(oracle, inputs)
+
+
+# DeltaNet has no gate: the hand-off difference shrinks only along the keys written, over a
+# 48-chunk window
+@pytest.mark.parametrize("H,T", [(2, 16384), (2, 32768)])
+def test_segmented_deltanet_matches_oracle(oracle, H, T):
+    w = wl.DRWorkload("deltanet_seg", 1, H, T, 128, 128, wl.DELTANET, "bf16", s0_std=0.1)
+    assert drs.chunked_plan_ex("deltanet", H, T, 128, 128)[2] > 1
+    inputs = wl.generate_dr(w, seed=50 + H)
+    dev = to_device(inputs)
+    before = drs.segment_counters()
+    out, Sf, _ = _scan(dev, "deltanet")
+    after = drs.segment_counters()
+    assert (after[0] - before[0], after[1] - before[1]) == (1, 0)
+    ref_out, ref_S = oracle_dr(oracle, inputs)
+    e_out, e_S = rel_err(tensor_np(out), ref_out), rel_err(tensor_np(Sf), ref_S)
+    assert e_out <= TOL and e_S <= TOL, (e_out, e_S)
