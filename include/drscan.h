@@ -58,8 +58,8 @@ enum {
 /* Use the per-token kernel (fp32 state, CUDA cores) even where the chunked tensor-core
  * kernel applies. Same results up to rounding; slower. For testing and as a baseline. */
 #define DR_FORCE_SEQUENTIAL 0x200
-/* Keep Gated DeltaNet and KDA on the chained chunked kernel (one pass, one dependent chain of
- * chunks per head) where dr_scan_fwd would take the segmented scan (see dr_scan_fwd). */
+/* Keep DeltaNet, Gated DeltaNet and KDA on the chained chunked kernel (one pass, one dependent
+ * chain of chunks per head) where dr_scan_fwd would take the segmented scan (see dr_scan_fwd). */
 #define DR_CHAINED 0x400
 
 /* status codes */
@@ -106,16 +106,17 @@ enum {
  * below that latches DR_ERR_GATE_RANGE, which dr_poll_error() reports (the outputs of
  * that call are then invalid: rerun it with DR_FORCE_SEQUENTIAL, which has no such limit).
  *
- * Segmented scan (Gated DeltaNet and KDA, bf16, dk = 128, T a multiple of 64, heads too few
- * to fill the GPU; see dr_chunked_plan_ex). A sequence's state carries over from chunk to chunk,
+ * Segmented scan (DeltaNet, Gated DeltaNet and KDA, bf16, dk = 128, T a multiple of 64, heads
+ * too few to fill the GPU; see dr_chunked_plan_ex). A sequence's state carries over from chunk to chunk,
  * so the chained kernel runs T/64 dependent chunk steps per head ("Mechanisms, trade-offs and
  * cross-layer routing of linear-attention architectures", Technical details: the state is
  * decayed by alpha and corrected by the delta rule at every token). With few heads the call
  * instead cuts each head into G equal segments and runs them at once, in one launch: every
- * segment from a zero state (the first from S0); every segment but the last runs 8 chunks on
- * into the next one, carrying its state, and writes the outputs there, while the next one
- * writes none for those chunks. A check per boundary then compares the carried state at the
- * end of those 8 chunks with the next segment's zero-start state there: they must agree
+ * segment from a zero state (the first from S0); every segment but the last runs a window of
+ * 8 chunks (48 for DeltaNet, which has no gate) on into the next one, carrying its state, and
+ * writes the outputs there, while the next one writes none for those chunks. A check per
+ * boundary then compares the carried state at the end of the window with the next segment's
+ * zero-start state there: they must agree
  * within 2^-7 of the carried state's largest value-row norm (row-wise 2-norm). A step whose
  * transition diag(alpha)(I - beta k k^T) could grow a difference (any alpha > 1 or
  * beta |k|^2 > 2, both checked on every token) also fails the check. When every check
