@@ -147,16 +147,16 @@ def aggregate_value(world: int, head_tokens: int, steps: int, total_ms_max: floa
 # loglinear.cuh for log-linear attention) at capture time; a changed source reports null.
 # Summaries with the commands are under profiles/.
 NCU_TRAFFIC = {
-    ("kda_bf16", "c661a4b94a22c92c"): 673364992 + 119821312,
-    ("gdn_bf16", "c661a4b94a22c92c"): 101819904 + 12610304,
+    ("kda_bf16", "b213a8f2dcd89007"): 673309440 + 119424512,
+    ("gdn_bf16", "b213a8f2dcd89007"): 101836288 + 14326784,
     # Gated DeltaNet-2: the pre-scaling kernel and the chunked kernel of one call
-    ("gdn2_bf16", "08557876d53c25c0"): 201332992 + 44987904 + 101819136 + 9339392,
+    ("gdn2_bf16", "522518ff6411b1c8"): 201334272 + 45484544 + 101819136 + 9624832,
     # the segmented scan: the segment launch, the hand-off check, the conditional launch
-    ("gdn_long_t4096", "08557876d53c25c0"): 52017152 + 672768 + 3168768 + 68096,
-    ("gdn_long_t8192", "08557876d53c25c0"): 109080064 + 14750464 + 3169024 + 67584,
-    ("gdn_long_t16384", "08557876d53c25c0"): 210959360 + 47117312 + 3169024 + 68096,
-    ("gdn_long_t32768", "08557876d53c25c0"): 414369024 + 116253184 + 3169024 + 67840,
-    ("kda_long_t32768", "08557876d53c25c0"): 747988992 + 127770880 + 15751936 + 68096,
+    ("gdn_long_t4096", "522518ff6411b1c8"): 52038400 + 633600 + 3169024 + 67840,
+    ("gdn_long_t8192", "522518ff6411b1c8"): 109064192 + 14753024 + 3172608 + 67840,
+    ("gdn_long_t16384", "522518ff6411b1c8"): 210941440 + 47334400 + 3168512 + 67840,
+    ("gdn_long_t32768", "522518ff6411b1c8"): 414370048 + 116414464 + 3169024 + 68096,
+    ("kda_long_t32768", "522518ff6411b1c8"): 747991040 + 128194560 + 15752192 + 68352,
     ("gdn_decode_bf16", "6c9773f81f64a408"): 271627008 + 211260672,
     ("loglinear_bf16", "79c1bdb9297c23dc"): 107535616 + 22006784,
 }
