@@ -281,3 +281,24 @@ def test_segmented_deltanet_matches_oracle(oracle, H, T):
     ref_out, ref_S = oracle_dr(oracle, inputs)
     e_out, e_S = rel_err(tensor_np(out), ref_out), rel_err(tensor_np(Sf), ref_S)
     assert e_out <= TOL and e_S <= TOL, (e_out, e_S)
+
+
+# the write values through the segment launch of every variant, and DR_CHAINED leaving the
+# segment counters alone
+@pytest.mark.parametrize("mode,T", [(wl.KDA, 8192), (wl.DELTANET, 16384)])
+def test_segmented_write_values_kda_deltanet(oracle, mode, T):
+    name = "kda" if mode == wl.KDA else "deltanet"
+    w = wl.DRWorkload("seg_u", 1, 2, T, 128, 128, mode, "bf16", s0_std=0.1)
+    assert drs.chunked_plan_ex(name, 2, T, 128, 128)[2] > 1
+    inputs = wl.generate_dr(w, seed=60 + mode)
+    dev = to_device(inputs)
+    before = drs.segment_counters()
+    out, Sf, u = _scan(dev, name, want_u=True)
+    mid = drs.segment_counters()
+    assert (mid[0] - before[0], mid[1] - before[1]) == (1, 0)
+    ref_out, ref_S, ref_u = oracle_dr_ex(oracle, inputs)
+    errs = (rel_err(tensor_np(out), ref_out), rel_err(tensor_np(Sf), ref_S),
+            rel_err(tensor_np(u), ref_u))
+    assert max(errs) <= TOL, (name, errs)
+    _scan(dev, name, chained=True, want_u=True)
+    assert drs.segment_counters() == mid
